@@ -1,0 +1,356 @@
+"""CPU oracle for Laplacian-kernel Nystrom attention -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, float64 numpy restatement of what the attention block computes.
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference legs may import it. The CUDA library never calls it and shares no
+code, header, table or helper with it.
+
+Sources (cited below by these tags, page title + section):
+  [P1] papernotes.org ICLR 2026 note "LaplacianFormer：用拉普拉斯核重新思考线性注意力"
+       sections: 研究背景与动机 (核心 idea), 方法详解 / 整体框架 (flowchart),
+       关键设计 1 (injective whitened map), 关键设计 2 (Nystrom),
+       关键设计 3 (Newton-Schulz + CUDA).
+  [P2] shd-paper.top summary "LaplacianFormer:Rethinking Linear Attention with
+       Laplacian Kernel" (abstract; pipeline summary in §方法详解).
+
+Readings taken where the pages are silent or garbled (each one is listed in the
+design notes with its reason):
+  R1  keys are the queries: landmarks are pooled from Q and C is query-vs-landmark
+      ([P1] 关键设计 2), so one point set feeds both C and W.
+  R2  pooling: non-overlapping r x r windows, stride r, landmark order row-major.
+  R3  the same eps regularises W (关键设计 3) and the whitening root (关键设计 1).
+  R4  alpha = 2/||W||_2 is tested against ||I - alpha W W^T||_2 < 1 as printed; when
+      the test fails (it always does: W has unit diagonal so ||W||_2 > 1) the
+      oracle uses alpha = 1/||W||_2^2 and raises a flag.
+  R5  whitening statistics are per landmark column over the N rows of one
+      (batch, head) unit, population variance (divide by N).
+  R6  "Reading A": the whitened C~ = (C - mu)/sqrt(var + eps) + 1/N replaces C on
+      both sides of the Nystrom product, O_attn = C~ (X (C~^T V)).
+  R7  no row normalisation of Z V (the pages give none).
+  R8  DWC: 3x3 depthwise cross-correlation, zero padding 1, stride 1, no bias,
+      weights fixed (no weight gradient).
+  R9  the printed kernel gradient (+1/lam) sign(x - y) k has the wrong sign; the
+      oracle differentiates k = exp(-||x - y||_1 / lam) itself, giving
+      -(1/lam) sign(x - y) k, with sign(0) = 0.
+  R10 alpha is held constant in the backward pass (stop-gradient).
+  R11 exactly T Newton-Schulz steps, no early exit.
+
+Parity pins (tests/test_oracle_*.py): closed forms of the kernel, scipy cdist,
+torch avg_pool2d / conv2d in float64, the per-step eigen closed form of
+Newton-Schulz, a Cholesky inverse, the r = 1 Nystrom identity against a dense
+O(N^2) product, sklearn's StandardScaler, whitening moments, and central finite
+differences for the backward pass. The whitening placement (R6) itself is
+"parity unpinned": nothing on the pages fixes it beyond self-consistency.
+"""
+from __future__ import annotations
+
+import dataclasses
+from concurrent.futures import ThreadPoolExecutor
+from typing import List, Optional, Tuple
+
+import numpy as np
+
+_ROW_CHUNK = 512
+_THREADS = 8
+
+
+def set_threads(n: int) -> None:
+    """Threads used for the row-chunked distance loops (numpy releases the GIL)."""
+    global _THREADS
+    _THREADS = max(1, int(n))
+
+
+def _chunked(n_rows: int, fn, threads: Optional[int] = None):
+    starts = list(range(0, n_rows, _ROW_CHUNK))
+    t = _THREADS if threads is None else threads
+    if t <= 1 or len(starts) == 1:
+        return [fn(s, min(s + _ROW_CHUNK, n_rows)) for s in starts]
+    with ThreadPoolExecutor(max_workers=t) as ex:
+        return list(ex.map(lambda s: fn(s, min(s + _ROW_CHUNK, n_rows)), starts))
+
+
+# ---------------------------------------------------------------------------
+# Building blocks
+# ---------------------------------------------------------------------------
+
+def pool_landmarks(Qu: np.ndarray, H: int, W: int, r: int) -> np.ndarray:
+    """Landmarks L = r x r average pool of the query map ([P1] 关键设计 2, R2).
+
+    Qu: [N, d] tokens of one unit, token n = y*W + x. Returns L [m, d] with
+    landmark index l = Y*(W/r) + X for window (Y, X).
+    """
+    N, d = Qu.shape
+    assert N == H * W and H % r == 0 and W % r == 0
+    g = Qu.reshape(H // r, r, W // r, r, d)
+    L = np.zeros((H // r, W // r, d))
+    for dy in range(r):
+        for dx in range(r):
+            L += g[:, dy, :, dx, :]
+    return (L / (r * r)).reshape(-1, d)
+
+
+def l1_distances(X: np.ndarray, Y: np.ndarray) -> np.ndarray:
+    """D[i, j] = sum_k |x_ik - y_jk| ([P1] 研究背景与动机, 核心 idea: the l1 norm)."""
+    X = np.asarray(X, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+
+    def rows(a, b):
+        return np.abs(X[a:b, None, :] - Y[None, :, :]).sum(axis=2)
+
+    return np.concatenate(_chunked(X.shape[0], rows), axis=0)
+
+
+def laplacian_kernel(X: np.ndarray, Y: np.ndarray, lam: float) -> np.ndarray:
+    """k(x, y) = exp(-||x - y||_1 / lam) for every pair ([P1] 核心 idea; 关键设计 2)."""
+    return np.exp(-l1_distances(X, Y) / lam)
+
+
+def landmark_gram(L: np.ndarray, lam: float, eps: float) -> np.ndarray:
+    """W = [k(l_a, l_b)] + eps I ([P1] 关键设计 2 defines W; 关键设计 3 adds eps I)."""
+    return laplacian_kernel(L, L, lam) + eps * np.eye(L.shape[0])
+
+
+@dataclasses.dataclass
+class AlphaChoice:
+    alpha: float            # the alpha actually used for X_0 = alpha W^T
+    alpha_pages: float      # 2 / ||W||_2, as printed
+    cond_pages: float       # ||I - alpha_pages W W^T||_2
+    fallback: bool          # True when the printed condition fails (R4)
+    norm2: float            # ||W||_2
+
+
+def select_alpha(W: np.ndarray) -> AlphaChoice:
+    """alpha per [P1] 关键设计 3, with the R4 fallback alpha = 1/||W||_2^2."""
+    norm2 = float(np.linalg.norm(W, 2))
+    a = 2.0 / norm2
+    m = W.shape[0]
+    cond = float(np.linalg.norm(np.eye(m) - a * (W @ W.T), 2))
+    if cond < 1.0:
+        return AlphaChoice(a, a, cond, False, norm2)
+    return AlphaChoice(1.0 / norm2 ** 2, a, cond, True, norm2)
+
+
+def newton_schulz(W: np.ndarray, alpha: float, T: int, keep_iterates: bool = False):
+    """X_0 = alpha W^T; X_{k+1} = X_k (2I - W X_k), exactly T steps ([P1] 关键设计 3, R11).
+
+    Returns (X_T, residuals, iterates) where residuals[k] = (||I - W X_k||_F,
+    ||I - W X_k||_2) for k = 0..T and iterates = [X_0..X_T] when requested.
+    """
+    m = W.shape[0]
+    I = np.eye(m)
+    X = alpha * W.T
+    its = [X] if keep_iterates else None
+    res = []
+    for _ in range(T):
+        R = I - W @ X
+        res.append((float(np.linalg.norm(R, "fro")), float(np.linalg.norm(R, 2))))
+        X = X @ (2.0 * I - W @ X)
+        if keep_iterates:
+            its.append(X)
+    R = I - W @ X
+    res.append((float(np.linalg.norm(R, "fro")), float(np.linalg.norm(R, 2))))
+    return X, res, its
+
+
+def whiten_columns(C: np.ndarray, eps: float):
+    """Diagonal centring + whitening of [P1] 关键设计 1 (R5): per column mean mu and
+    population variance var over the N rows; C~ = (C - mu)/sqrt(var + eps) + 1/N.
+
+    Returns (C~, mu, var).
+    """
+    N = C.shape[0]
+    mu = C.mean(axis=0)
+    var = ((C - mu) ** 2).mean(axis=0)
+    return (C - mu) / np.sqrt(var + eps) + 1.0 / N, mu, var
+
+
+def dwc3x3(Vu: np.ndarray, w: np.ndarray, H: int, W: int) -> np.ndarray:
+    """DWC(V): per-channel 3x3 cross-correlation with zero padding 1 ([P1] 整体框架
+    flowchart node "DWC(V) 深度卷积"; 关键设计 1 output ZV + DWC(V); R8).
+
+    Vu: [N, d]; w: [d, 3, 3] with w[k, dy+1, dx+1] multiplying V[y+dy, x+dx, k].
+    """
+    N, d = Vu.shape
+    g = Vu.reshape(H, W, d)
+    pad = np.zeros((H + 2, W + 2, d))
+    pad[1:-1, 1:-1] = g
+    out = np.zeros((H, W, d))
+    for a in range(3):
+        for b in range(3):
+            out += w[:, a, b][None, None, :] * pad[a:a + H, b:b + W, :]
+    return out.reshape(N, d)
+
+
+def dwc3x3_transpose(G: np.ndarray, w: np.ndarray, H: int, W: int) -> np.ndarray:
+    """Adjoint of dwc3x3 in its input: dV[y', x'] = sum_{a,b} w[a,b] G[y'-a+1, x'-b+1]."""
+    N, d = G.shape
+    g = G.reshape(H, W, d)
+    pad = np.zeros((H + 2, W + 2, d))
+    pad[1:-1, 1:-1] = g
+    out = np.zeros((H, W, d))
+    for a in range(3):
+        for b in range(3):
+            out += w[:, a, b][None, None, :] * pad[2 - a:2 - a + H, 2 - b:2 - b + W, :]
+    return out.reshape(N, d)
+
+
+# ---------------------------------------------------------------------------
+# One (batch, head) unit
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class UnitForward:
+    L: np.ndarray           # [m, d] landmarks
+    C: np.ndarray           # [N, m] cross kernel
+    W: np.ndarray           # [m, m] landmark kernel + eps I
+    alpha: AlphaChoice
+    X: np.ndarray           # [m, m] X_T
+    ns_residuals: List[Tuple[float, float]]
+    Ct: np.ndarray          # [N, m] the matrix used in the product (whitened or raw C)
+    mu: Optional[np.ndarray]
+    var: Optional[np.ndarray]
+    A: np.ndarray           # Ct^T V   [m, d]
+    M: np.ndarray           # X A      [m, d]
+    O_attn: np.ndarray      # Ct M     [N, d]
+    O: np.ndarray           # O_attn + DWC(V)
+    iterates: Optional[List[np.ndarray]] = None
+
+
+def unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten=True, keep_iterates=False) -> UnitForward:
+    """Forward pass of one unit, in the pages' order ([P1] 整体框架 flowchart):
+    pool -> Laplacian kernels -> Newton-Schulz W^+ -> whitening -> C~ (X (C~^T V)) + DWC(V).
+    """
+    Qu = np.asarray(Qu, dtype=np.float64)
+    Vu = np.asarray(Vu, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    L = pool_landmarks(Qu, H, W, r)
+    C = laplacian_kernel(Qu, L, lam)
+    Wm = landmark_gram(L, lam, eps)
+    ac = select_alpha(Wm)
+    X, res, its = newton_schulz(Wm, ac.alpha, T, keep_iterates)
+    if whiten:
+        Ct, mu, var = whiten_columns(C, eps)
+    else:
+        Ct, mu, var = C, None, None
+    A = Ct.T @ Vu
+    M = X @ A
+    O_attn = Ct @ M
+    O = O_attn + dwc3x3(Vu, w, H, W)
+    return UnitForward(L, C, Wm, ac, X, res, Ct, mu, var, A, M, O_attn, O, its)
+
+
+def _sign_contractions(Qu, L, dD):
+    """dq[i,k] = sum_l dD[i,l] sign(q_ik - l_lk);  dl[l,k] = -sum_i dD[i,l] sign(q_ik - l_lk)."""
+    N, d = Qu.shape
+
+    def rows(a, b):
+        S = np.sign(Qu[a:b, None, :] - L[None, :, :])           # [rows, m, d]
+        dq = np.einsum("il,ilk->ik", dD[a:b], S)
+        dl = -np.einsum("il,ilk->lk", dD[a:b], S)
+        return dq, dl
+
+    parts = _chunked(N, rows)
+    dQ = np.concatenate([p[0] for p in parts], axis=0)
+    dL = np.sum([p[1] for p in parts], axis=0)
+    return dQ, dL
+
+
+def unit_backward(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten=True):
+    """Reverse mode through unit_forward (R9 kernel sign, R10 alpha constant).
+
+    Returns (dQ [N, d], dV [N, d], fwd). The loss is <dO, O>.
+    """
+    Qu = np.asarray(Qu, dtype=np.float64)
+    Vu = np.asarray(Vu, dtype=np.float64)
+    dO = np.asarray(dOu, dtype=np.float64)
+    f = unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten, keep_iterates=True)
+    N, d = Qu.shape
+    m = f.L.shape[0]
+    # O = Ct M + DWC(V),  M = X A,  A = Ct^T V
+    dV = dwc3x3_transpose(dO, np.asarray(w, dtype=np.float64), H, W)
+    dM = f.Ct.T @ dO
+    dX = dM @ f.A.T
+    dA = f.X.T @ dM
+    dCt = dO @ f.M.T + Vu @ dA.T
+    dV = dV + f.Ct @ dA
+    # whitening (population-variance batch-norm form), then C = exp(-D/lam)
+    if whiten:
+        s = 1.0 / np.sqrt(f.var + eps)
+        Chat = (f.C - f.mu) * s
+        dC = s * (dCt - dCt.mean(axis=0) - Chat * (dCt * Chat).mean(axis=0))
+    else:
+        dC = dCt
+    dD = -(f.C * dC) / lam
+    dQ, dL = _sign_contractions(Qu, f.L, dD)
+    # Newton-Schulz: X_{k+1} = 2 X_k - X_k W X_k, X_0 = alpha W^T (alpha held constant)
+    Wm = f.W
+    G = dX
+    dW = np.zeros((m, m))
+    for k in range(T - 1, -1, -1):
+        Xk = f.iterates[k]
+        dW -= Xk.T @ G @ Xk.T
+        G = 2.0 * G - G @ Xk.T @ Wm.T - Wm.T @ Xk.T @ G
+    dW += f.alpha.alpha * G.T
+    # W = exp(-E/lam) + eps I,  E_ab = sum_k |l_ak - l_bk|
+    dE = -(Wm - eps * np.eye(m)) * dW / lam
+    Sl = np.sign(f.L[:, None, :] - f.L[None, :, :])            # [m, m, d]
+    dL = dL + np.einsum("ab,abk->ak", dE, Sl) - np.einsum("ab,abk->bk", dE, Sl)
+    # L = pool(Q): every token of window l receives dL_l / r^2
+    Wr = W // r
+    g = dL.reshape(H // r, 1, Wr, 1, d) / (r * r)
+    dQ = dQ + np.broadcast_to(g, (H // r, r, Wr, r, d)).reshape(N, d)
+    return dQ, dV, f
+
+
+# ---------------------------------------------------------------------------
+# Whole calls ([B, heads, N, d] tensors)
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Forward:
+    O: np.ndarray           # [B, heads, N, d]
+    O_attn: np.ndarray
+    units: List[UnitForward]
+
+
+def forward(Q, V, dwc, wl, whiten=True, units=None, keep_units=True) -> Forward:
+    """Oracle forward over all (or the listed) units of a workload.
+
+    Q, V: [B, heads, N, d] array-likes (float values already in the storage
+    precision); dwc: [heads, d, 3, 3]. ``units`` restricts to a list of flat
+    unit indices u = b*heads + h (others are left zero).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    w = np.asarray(dwc, dtype=np.float64)
+    B, nh, N, d = Q.shape
+    O = np.zeros_like(Q)
+    Oa = np.zeros_like(Q)
+    us = []
+    todo = range(B * nh) if units is None else units
+    for u in todo:
+        b, h = divmod(u, nh)
+        f = unit_forward(Q[b, h], V[b, h], w[h], wl.H, wl.W, wl.r, wl.lam, wl.eps, wl.T, whiten)
+        O[b, h] = f.O
+        Oa[b, h] = f.O_attn
+        us.append(f if keep_units else None)
+    return Forward(O, Oa, us)
+
+
+def backward(Q, V, dwc, dO, wl, whiten=True, units=None):
+    """Oracle gradients (dQ, dV), [B, heads, N, d], for the loss <dO, O>."""
+    Q = np.asarray(Q, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    w = np.asarray(dwc, dtype=np.float64)
+    B, nh, N, d = Q.shape
+    dQ = np.zeros_like(Q)
+    dV = np.zeros_like(Q)
+    todo = range(B * nh) if units is None else units
+    for u in todo:
+        b, h = divmod(u, nh)
+        gq, gv, _ = unit_backward(Q[b, h], V[b, h], w[h], dO[b, h], wl.H, wl.W, wl.r,
+                                  wl.lam, wl.eps, wl.T, whiten)
+        dQ[b, h] = gq
+        dV[b, h] = gv
+    return dQ, dV
