@@ -1,0 +1,320 @@
+#!/usr/bin/env python
+"""Benchmark of one Laplacian-kernel Nystrom attention call (forward) on a B200.
+
+Workload: the PVT stage-1 shape (B=32, heads=1, 56x56 grid so N=3136, d=64, 8x8 pooled
+landmarks so m=49, lambda=4, eps=1e-6, T=20, bf16 Q/V/O with fp32 arithmetic), synthetic
+inputs from laplacian_nystr_attention_avg_b200.inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lfa|reference]
+
+Prints ONE JSON line (rank 0). Under torchrun each rank runs its own full batch on its
+own GPU (independent units, no data-path collective: weak scaling); the step time is the
+max over ranks. ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s per Laplacian-Nyström attention call (N=3136,d=64,m=49); % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["lfa", "reference"], default="lfa")
+    ap.add_argument("--workload", default="pvt1")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="approximate CPU work of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def workload_config(wl, extra=None):
+    cfg = {"workload": f"{wl.name}: B={wl.B} heads={wl.heads} grid={wl.H}x{wl.W} N={wl.N} d={wl.d} "
+                       f"r={wl.r} m={wl.m} lambda={wl.lam:g} eps={wl.eps:g} T={wl.T} {wl.dtype} "
+                       f"Q~{wl.qdist}",
+           "B": wl.B, "heads": wl.heads, "H": wl.H, "W": wl.W, "N": wl.N, "d": wl.d, "r": wl.r,
+           "m": wl.m, "lambda": wl.lam, "eps": wl.eps, "T": wl.T, "storage": wl.dtype,
+           "whiten": True}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if its source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None, None
+    for ln in lines:
+        if ln.startswith("#") or not ln.strip():
+            continue
+        kv = dict(tok.split("=", 1) for tok in ln.split() if "=" in tok)
+        if kv.get("kernel") != kernel or kv.get("workload") != workload:
+            continue
+        src = os.path.join(ROOT, kv.get("source", ""))
+        try:
+            sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        except OSError:
+            return None, None
+        if sha != kv.get("source_sha"):
+            return None, "stale"
+        return float(kv["dram_bytes_per_launch"]), kv.get("note")
+    return None, None
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(device_index)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for ln in open(self.path).read().splitlines():
+            f = [c.strip() for c in ln.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[5 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def run_reference(args):
+    """The CPU oracle, as it stands, on a bounded sample of units per step (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, make_inputs
+    from oracle import lfa_oracle as O
+
+    wl = WORKLOADS[args.workload]
+    x = make_inputs(wl)
+    Q, V, w = x.Q.numpy(), x.V.numpy(), x.dwc.numpy()
+    cores = os.cpu_count() or 1
+    O.set_threads(cores)
+    per_step = 1  # units per step: keeps --steps K --warmup W within a few minutes
+    units = [u % wl.units for u in range(per_step)]
+    for _ in range(args.warmup):
+        O.forward(Q, V, w, wl, units=units, keep_units=False)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        O.forward(Q, V, w, wl, units=[(k + u) % wl.units for u in range(per_step)], keep_units=False)
+    dt = time.perf_counter() - t0
+    tokens = per_step * wl.N * args.steps
+    value = tokens / dt
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": workload_config(wl, {"sample": f"{per_step} of {wl.units} units per step"}),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} (batch, head) unit of {wl.N} tokens per step, "
+                                       f"{args.steps} steps"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, x, seconds):
+    from oracle import lfa_oracle as O
+
+    cores = os.cpu_count() or 1
+    O.set_threads(cores)
+    Q, V, w = x.Q.numpy(), x.V.numpy(), x.dwc.numpy()
+    t0 = time.perf_counter()
+    O.forward(Q, V, w, wl, units=[0], keep_units=False)
+    one = time.perf_counter() - t0
+    n = max(1, min(wl.units, int(seconds / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    O.forward(Q, V, w, wl, units=list(range(n)), keep_units=False)
+    dt = time.perf_counter() - t0
+    return {"value": n * wl.N / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.units} (batch, head) units of the same workload ({n * wl.N} tokens), "
+                      f"float64 numpy, {dt:.1f} s"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    from laplacian_nystr_attention_avg_b200 import lfa
+    from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    wl = WORKLOADS[args.workload]
+    x = make_inputs(wl, seed=rank)
+    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl), x.dwc, str(dev))
+    set_bytes = 3 * wl.units * wl.N * wl.d * x.Q_store.element_size()
+    n_sets = max(2, math.ceil(1.8 * L2_BYTES / set_bytes))
+    Qs = [x.Q_store.to(dev) for _ in range(n_sets)]
+    Vs = [x.V_store.to(dev) for _ in range(n_sets)]
+    Os = [mod.new_output() for _ in range(n_sets)]
+    stream = torch.cuda.current_stream()
+
+    for k in range(args.warmup):
+        mod.forward(Qs[k % n_sets], Vs[k % n_sets], Os[k % n_sets])
+    st, info = mod.info()
+    if st != lfa.LFA_OK:
+        raise RuntimeError(f"device status after warm-up: {lfa.status_string(st)}")
+
+    K = args.steps
+    kb = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    t_begin.record(stream)
+    for k in range(K):
+        mod.set_profile_events(kb[k], ke[k])
+        mod.forward(Qs[k % n_sets], Vs[k % n_sets], Os[k % n_sets])
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    mod.set_profile_events(None, None)
+    total_ms = t_begin.elapsed_time(t_end)
+    kern_ms = statistics.fmean(kb[k].elapsed_time(ke[k]) for k in range(K))
+    if world > 1:
+        t = torch.tensor([total_ms, kern_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, kern_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / K
+    value = world * wl.units * wl.N * K / (total_ms * 1e-3)
+
+    # end to end through the host-buffer entry point: pinned host Q, V -> device -> O -> host
+    Qh = x.Q_store.pin_memory()
+    Vh = x.V_store.pin_memory()
+    Oh = torch.empty(Qh.shape, dtype=Qh.dtype).pin_memory()
+    E = args.e2e_steps
+    for _ in range(3):
+        mod.forward_host(Qh, Vh, Oh, Qs[0], Vs[0], Os[0])
+    e_b = torch.cuda.Event(enable_timing=True)
+    e_e = torch.cuda.Event(enable_timing=True)
+    barrier()
+    e_b.record(stream)
+    for _ in range(E):
+        mod.forward_host(Qh, Vh, Oh, Qs[0], Vs[0], Os[0])
+    e_e.record(stream)
+    barrier()
+    e2e_ms = e_b.elapsed_time(e_e)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * wl.units * wl.N * E / (e2e_ms * 1e-3)
+    nbytes = wl.units * wl.N * wl.d * x.Q_store.element_size()
+
+    if rank == 0:
+        peaks, peak_kind = read_peaks()
+        props = torch.cuda.get_device_properties(dev)
+        sms = props.multi_processor_count
+        f_max = float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+        alu_peak = sms * 128 * f_max                      # FP32-pipe lane-instructions / s
+        alg_instr = 2.0 * wl.units * wl.N * wl.m * wl.d   # one |q - l| sub + abs-add per element
+        achieved = alg_instr / (kern_ms * 1e-3)
+        traffic, tnote = kernel_traffic(mod.dominant_kernel, wl.name)
+        hbm = float(peaks["hbm_gbs"]) * 1e9
+        io_bytes = 3.0 * nbytes
+        t_roof = max(alg_instr / alu_peak, io_bytes / hbm)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(wl, {
+                "path": mod.path, "parallelism": f"replicas{world}" if world > 1 else "single",
+                "l2": f"{n_sets} rotating input/output sets of {set_bytes / 2**20:.1f} MiB "
+                      f"({n_sets * set_bytes / 2**20:.0f} MiB > 126 MiB L2), no flush",
+                "call_roofline_frac": t_roof / (ms_per_step * 1e-3),
+                "call_roofline_us": t_roof * 1e6}),
+            "roofline": {"bound": "alu", "kernel": mod.dominant_kernel, "achieved": achieved / 1e12,
+                         "peak": alu_peak / 1e12, "unit": "Tinstr/s", "frac": achieved / alu_peak,
+                         "traffic": traffic,
+                         "peak_note": f"{sms} SMs x 128 FP32 lanes x {f_max / 1e6:.0f} MHz "
+                                      f"(sm_max_mhz, {peak_kind}); algorithmic work = 2 B*heads*N*m*d "
+                                      f"FP32 instructions per launch",
+                         "kernel_us": kern_ms * 1e3},
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": 2 * nbytes,
+                    "d2h_bytes_per_step": nbytes},
+            "gpu_launches": K * mod.launches_per_forward,
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,163 @@
+/*
+ * lfa.h -- C ABI of the Laplacian-kernel Nystrom attention library (liblfa.so),
+ * built for NVIDIA B200 (sm_100a).
+ *
+ * What one call computes, per (batch b, head h) unit with tokens Q, V in
+ * R^{N x d} on an H x W grid (token n = y*W + x):
+ *   L   = r x r average pool of the query map, m = (H/r)(W/r) landmarks
+ *         [LaplacianFormer note (papernotes.org), §关键设计 2: landmarks from
+ *          average-pooling the reshaped query tensor, as in PVTv2];
+ *   C   = exp(-||q_i - l_l||_1 / lambda)       (N x m cross kernel)
+ *   W   = exp(-||l_a - l_b||_1 / lambda) + eps I   (m x m landmark kernel)
+ *         [same note, §研究背景与动机 (核心 idea) for the kernel, §关键设计 2 for C and W,
+ *          §关键设计 3 for the eps I shift];
+ *   X   = Newton-Schulz pseudo-inverse of W, X_0 = alpha W^T,
+ *         X_{k+1} = X_k (2I - W X_k), exactly T steps [§关键设计 3]. alpha = 2/||W||_2 as
+ *         printed is kept only if ||I - alpha W W^T||_2 < 1; otherwise (always, since W
+ *         has unit diagonal) alpha = 1/||W||_2^2 and the fallback is reported;
+ *   C~  = (C - mu) / sqrt(var + eps) + 1/N, per-landmark-column mean and population
+ *         variance over the unit's N rows [§关键设计 1, diagonal whitening];
+ *   O   = C~ (X (C~^T V)) + DWC(V), DWC = 3x3 depthwise cross-correlation, zero
+ *         padding 1, weights [heads][d][3][3] [§关键设计 1 output "ZV + DWC(V)";
+ *         §整体框架 flowchart]. With whiten = 0 the raw C is used on both sides.
+ *
+ * Conventions for every entry point:
+ *   - Tensors Q, V, O, dO, dQ, dV are contiguous [B][heads][N][d] in the config's
+ *     dtype (fp32 or bf16); arithmetic is fp32 throughout. Device pointers must be
+ *     16-byte aligned. The DWC weight is fp32 [heads][d][3][3] on the device.
+ *   - All device memory is owned by the caller. The handle owns host state only and
+ *     keeps the weight and workspace pointers it was created with; the weight is read
+ *     at every call, not copied.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Forward and
+ *     backward only enqueue work: they never synchronise the host.
+ *   - Errors are returned as lfa_status; nothing is thrown across the ABI and the
+ *     library never exits the process. Argument errors are detected on the host
+ *     before any launch. Device-side conditions (a bounded wait that expired, a
+ *     non-finite landmark kernel) set a status word in the workspace that
+ *     lfa_get_info returns.
+ *   - A handle must not be used by two host threads at once; calls on one handle
+ *     that overlap on the GPU (different streams without ordering) race on its
+ *     workspace.
+ */
+#ifndef LFA_H_
+#define LFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LFA_OK = 0,
+  LFA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, H%r or W%r != 0 ... */
+  LFA_ERR_UNSUPPORTED = 2,   /* d not in {32, 64}, m > 256, unknown dtype */
+  LFA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, copy, attribute) */
+  LFA_ERR_STATE = 4,         /* backward without a matching forward on this handle */
+  LFA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (reported by lfa_get_info) */
+  LFA_ERR_NONFINITE = 6      /* the landmark kernel or its norm was not finite */
+} lfa_status;
+
+typedef enum { LFA_F32 = 0, LFA_BF16 = 1 } lfa_dtype;
+
+typedef struct {
+  int B;          /* batch */
+  int heads;      /* heads; units = B * heads */
+  int H, W;       /* token grid, N = H * W */
+  int d;          /* channels per head: 32 or 64 */
+  int r;          /* pooling window; H % r == 0 and W % r == 0; m = (H/r)(W/r) <= 256 */
+  float lambda;   /* Laplacian kernel scale, > 0 */
+  float eps;      /* W regulariser and whitening epsilon, >= 0 */
+  int T;          /* Newton-Schulz steps, 0 <= T <= 64 */
+  int dtype;      /* lfa_dtype of Q, V, O, dO, dQ, dV */
+  int whiten;     /* 1: whitened C~ on both sides (default); 0: raw C */
+} lfa_config;
+
+/* Per-unit diagnostics of the most recent forward call. */
+typedef struct {
+  int alpha_fallback;    /* 1 when 2/||W||_2 failed ||I - alpha W W^T||_2 < 1 */
+  float alpha;           /* alpha used for X_0 */
+  float lambda_max;      /* estimate of ||W||_2 (power iteration; W is SPD) */
+  float ns_residual_fro; /* ||I - W X_T||_F after the last step */
+} lfa_unit_info;
+
+typedef struct lfa_ctx* lfa_handle;
+
+/* Bytes of device workspace a handle needs for `cfg` (0 if cfg is invalid). The
+ * workspace holds the per-unit landmarks, W, X, whitening statistics, reduction
+ * partials, the forward context that backward reuses, and the status word. */
+size_t lfa_workspace_size(const lfa_config* cfg);
+
+/* Validate cfg and build a handle. dwc_weight: device fp32 [heads][d][3][3].
+ * workspace: device, >= lfa_workspace_size(cfg) bytes, 256-byte aligned, caller
+ * owned for the handle's lifetime. No launch happens here. */
+lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* workspace,
+                      size_t workspace_bytes, lfa_handle* out);
+
+/* Forward pass (see the file comment). Q, V: device inputs; O: device output, all
+ * [B][heads][N][d] in cfg.dtype. Enqueued on `stream`. */
+lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void* stream);
+
+/* Forward pass from and to HOST buffers: copies Q, V (host, [B][heads][N][d] in
+ * cfg.dtype; pinned memory gives asynchronous copies) into the caller's device
+ * buffers Q_dev, V_dev, runs lfa_forward into O_dev and copies O back to O_host.
+ * Synchronises `stream` before returning, so O_host is ready on LFA_OK. */
+lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
+                            void* Q_dev, void* V_dev, void* O_dev, void* stream);
+
+/* Backward pass for the loss <dO, O>: writes dQ and dV ([B][heads][N][d], cfg.dtype).
+ * Reuses the context saved by the most recent lfa_forward on this handle, which
+ * must have been called with the same Q and V pointers (else LFA_ERR_STATE).
+ * The kernel gradient is -(1/lambda) sign(q - l) k with sign(0) = 0 [the note's
+ * §研究背景与动机 prints the opposite sign]; alpha is held constant; the DWC
+ * weight gets no gradient. */
+lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* dO,
+                        void* dQ, void* dV, void* stream);
+
+/* Copy per-unit diagnostics of the last forward into host_out[0..n_units-1]
+ * (n_units must equal B * heads) and return the device status word
+ * (LFA_OK, LFA_ERR_TIMEOUT or LFA_ERR_NONFINITE). Synchronises `stream`. */
+lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void* stream);
+
+/* Release the handle (host memory only; device memory stays the caller's). */
+lfa_status lfa_destroy(lfa_handle h);
+
+/* Static, human-readable name of a status code. */
+const char* lfa_status_string(lfa_status s);
+
+/* ---- inspection entry points used by the parity tests ---------------------- */
+
+/* Cross kernel C of one unit, written as fp32 [N][m] to the device buffer C_out,
+ * computed by the same device code the forward pass uses. */
+lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* C_out,
+                                  void* stream);
+
+/* Copy the forward context of one unit (device -> device, fp32): landmarks L [m][d],
+ * Newton-Schulz result X [m][m], whitening mean mu [m] and scale s [m]. Any output
+ * pointer may be NULL. Valid after lfa_forward on this handle. */
+lfa_status lfa_debug_context(lfa_handle h, int unit, float* L_out, float* X_out, float* mu_out,
+                             float* s_out, void* stream);
+
+/* Benchmark timing hook: with non-NULL ev_begin / ev_end (each a cudaEvent_t created by
+ * the caller), every later lfa_forward on this handle records ev_begin on its stream
+ * immediately before launching the forward's dominant kernel and ev_end immediately after
+ * it, so the caller can time that one kernel with cudaEventElapsedTime. NULL, NULL turns
+ * the hook off. Host-only; returns LFA_ERR_INVALID_ARG if exactly one event is NULL. */
+lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end);
+
+/* Name of the kernel the timing hook brackets for this handle's config (static string). */
+const char* lfa_dominant_kernel(lfa_handle h);
+
+/* Number of kernels one lfa_forward launches for this handle's config (0 if h is NULL). */
+int lfa_launches_per_forward(lfa_handle h);
+
+/* Name of the forward implementation chosen for this handle's config
+ * ("fused" or "generic"), static string. */
+const char* lfa_forward_path(lfa_handle h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LFA_H_ */

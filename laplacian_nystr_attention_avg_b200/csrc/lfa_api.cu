@@ -1,0 +1,316 @@
+// C-ABI entry points of liblfa (declared in include/lfa.h): validation, workspace
+// carve-up, launch sequencing and diagnostics read-back. No compute happens here.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <new>
+
+#include "lfa_internal.h"
+
+using lfa::Layout;
+using lfa::Params;
+
+struct lfa_ctx {
+  lfa_config cfg;
+  Params p;
+  Layout lay;
+  unsigned char* ws;
+  size_t ws_bytes;
+  const void* last_Q;
+  const void* last_V;
+  int have_forward;
+  int path;   // 0 = generic, 1 = fused
+};
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+lfa_status validate(const lfa_config* c) {
+  if (!c) return LFA_ERR_INVALID_ARG;
+  if (c->B < 1 || c->heads < 1 || c->H < 1 || c->W < 1 || c->r < 1) return LFA_ERR_INVALID_ARG;
+  if (c->H % c->r != 0 || c->W % c->r != 0) return LFA_ERR_INVALID_ARG;
+  if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return LFA_ERR_INVALID_ARG;
+  if (!(c->eps >= 0.f) || !isfinite(c->eps)) return LFA_ERR_INVALID_ARG;
+  if (c->T < 0 || c->T > lfa::kMaxT) return LFA_ERR_INVALID_ARG;
+  if (c->whiten != 0 && c->whiten != 1) return LFA_ERR_INVALID_ARG;
+  if (c->d != 32 && c->d != 64) return LFA_ERR_UNSUPPORTED;
+  if (c->dtype != LFA_F32 && c->dtype != LFA_BF16) return LFA_ERR_UNSUPPORTED;
+  const long long m = (long long)(c->H / c->r) * (c->W / c->r);
+  if (m > lfa::kMaxM) return LFA_ERR_UNSUPPORTED;
+  const long long rows = (long long)c->B * c->heads * c->H * c->W;
+  if (rows * c->d >= (1ll << 31)) return LFA_ERR_UNSUPPORTED;   // element index fits int32
+  return LFA_OK;
+}
+
+// Shape-derived parameters and workspace offsets (no pointers yet).
+void plan(const lfa_config* c, Params* p, Layout* L) {
+  memset(p, 0, sizeof(*p));
+  p->B = c->B;
+  p->heads = c->heads;
+  p->H = c->H;
+  p->W = c->W;
+  p->N = c->H * c->W;
+  p->d = c->d;
+  p->r = c->r;
+  p->m = (c->H / c->r) * (c->W / c->r);
+  p->T = c->T;
+  p->whiten = c->whiten;
+  p->dtype = c->dtype;
+  p->U = c->B * c->heads;
+  p->lam = c->lambda;
+  p->eps = c->eps;
+  p->neg_log2e_over_lam = (float)(-1.4426950408889634 / (double)c->lambda);
+  p->n_tiles = lfa::ceil_div(p->N, lfa::kRowTile);
+  // about two pass-1 CTAs per SM of a 148-SM part
+  const int want = lfa::ceil_div(296, p->U);
+  int P = want < p->n_tiles ? want : p->n_tiles;
+  if (P < 1) P = 1;
+  p->tiles_per_cta = lfa::ceil_div(p->n_tiles, P);
+  p->P = lfa::ceil_div(p->n_tiles, p->tiles_per_cta);
+  p->part_stride = 2 * p->m + p->m * p->d + p->d;
+  p->n_chunks = lfa::ceil_div(p->m, 16);
+
+  const size_t U = p->U, m = p->m, d = p->d;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L->status = take(64);
+  L->info = take(sizeof(float) * U * lfa::kInfoStride);
+  L->L = take(sizeof(float) * U * m * d);
+  L->Wm = take(sizeof(float) * U * m * m);
+  L->X = take(sizeof(float) * U * m * m);
+  L->Xb = take(sizeof(float) * U * m * m);
+  L->Y = take(sizeof(float) * U * m * m);
+  L->part = take(sizeof(float) * U * p->P * p->part_stride);
+  L->red = take(sizeof(double) * U * p->part_stride);
+  L->mu = take(sizeof(float) * U * m);
+  L->s = take(sizeof(float) * U * m);
+  L->A = take(sizeof(float) * U * m * d);
+  L->M = take(sizeof(float) * U * m * d);
+  L->Mp = take(sizeof(float) * U * m * d);
+  L->bpart = take(sizeof(float) * U * p->n_chunks * d);
+  L->fused = take(0);
+  L->bwd = take(0);
+  L->total = off;
+}
+
+void bind(Params* p, const Layout& L, unsigned char* ws) {
+  p->status = reinterpret_cast<int*>(ws + L.status);
+  p->info = reinterpret_cast<float*>(ws + L.info);
+  p->L = reinterpret_cast<float*>(ws + L.L);
+  p->Wm = reinterpret_cast<float*>(ws + L.Wm);
+  p->X = reinterpret_cast<float*>(ws + L.X);
+  p->Xb = reinterpret_cast<float*>(ws + L.Xb);
+  p->Y = reinterpret_cast<float*>(ws + L.Y);
+  p->part = reinterpret_cast<float*>(ws + L.part);
+  p->red = reinterpret_cast<double*>(ws + L.red);
+  p->mu = reinterpret_cast<float*>(ws + L.mu);
+  p->s = reinterpret_cast<float*>(ws + L.s);
+  p->A = reinterpret_cast<float*>(ws + L.A);
+  p->M = reinterpret_cast<float*>(ws + L.M);
+  p->Mp = reinterpret_cast<float*>(ws + L.Mp);
+  p->bpart = reinterpret_cast<float*>(ws + L.bpart);
+}
+
+// Kernel attributes (dynamic shared memory opt-in) are per device; set them once each.
+std::mutex g_attr_mu;
+unsigned long long g_attr_done = 0;
+
+lfa_status ensure_attributes() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LFA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (dev < 64 && (g_attr_done >> dev) & 1ull) return LFA_OK;
+  if (lfa::generic_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (dev < 64) g_attr_done |= 1ull << dev;
+  return LFA_OK;
+}
+
+size_t elem_bytes(const lfa_config& c) { return c.dtype == LFA_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+const char* lfa_status_string(lfa_status s) {
+  switch (s) {
+    case LFA_OK: return "ok";
+    case LFA_ERR_INVALID_ARG: return "invalid argument";
+    case LFA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LFA_ERR_CUDA: return "CUDA runtime error";
+    case LFA_ERR_STATE: return "backward without a matching forward";
+    case LFA_ERR_TIMEOUT: return "device wait timed out";
+    case LFA_ERR_NONFINITE: return "non-finite landmark kernel";
+  }
+  return "unknown status";
+}
+
+size_t lfa_workspace_size(const lfa_config* cfg) {
+  if (validate(cfg) != LFA_OK) return 0;
+  Params p;
+  Layout L;
+  plan(cfg, &p, &L);
+  return L.total;
+}
+
+lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* workspace,
+                      size_t workspace_bytes, lfa_handle* out) {
+  if (!out) return LFA_ERR_INVALID_ARG;
+  *out = nullptr;
+  lfa_status st = validate(cfg);
+  if (st != LFA_OK) return st;
+  if (!dwc_weight || !workspace) return LFA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || !aligned16(dwc_weight))
+    return LFA_ERR_INVALID_ARG;
+  lfa_ctx* h = new (std::nothrow) lfa_ctx;
+  if (!h) return LFA_ERR_INVALID_ARG;
+  memset(h, 0, sizeof(*h));
+  h->cfg = *cfg;
+  plan(cfg, &h->p, &h->lay);
+  if (workspace_bytes < h->lay.total) {
+    delete h;
+    return LFA_ERR_INVALID_ARG;
+  }
+  st = ensure_attributes();
+  if (st != LFA_OK) {
+    delete h;
+    return st;
+  }
+  h->ws = static_cast<unsigned char*>(workspace);
+  h->ws_bytes = workspace_bytes;
+  bind(&h->p, h->lay, h->ws);
+  h->p.dwc = dwc_weight;
+  h->path = 0;
+  *out = h;
+  return LFA_OK;
+}
+
+lfa_status lfa_destroy(lfa_handle h) {
+  if (!h) return LFA_ERR_INVALID_ARG;
+  delete h;
+  return LFA_OK;
+}
+
+lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void* stream) {
+  if (!h || !Q || !V || !O) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(V) || !aligned16(O)) return LFA_ERR_INVALID_ARG;
+  Params p = h->p;
+  p.Q = Q;
+  p.V = V;
+  p.O = O;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (lfa::launch_generic_forward(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  h->last_Q = Q;
+  h->last_V = V;
+  h->have_forward = 1;
+  return LFA_OK;
+}
+
+lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
+                            void* Q_dev, void* V_dev, void* O_dev, void* stream) {
+  if (!h || !Q_host || !V_host || !O_host || !Q_dev || !V_dev || !O_dev) return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)h->p.U * h->p.N * h->p.d * elem_bytes(h->cfg);
+  if (cudaMemcpyAsync(Q_dev, Q_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (cudaMemcpyAsync(V_dev, V_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return LFA_ERR_CUDA;
+  lfa_status s = lfa_forward(h, Q_dev, V_dev, O_dev, stream);
+  if (s != LFA_OK) return s;
+  if (cudaMemcpyAsync(O_host, O_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LFA_ERR_CUDA;
+  return LFA_OK;
+}
+
+lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* dO, void* dQ,
+                        void* dV, void* stream) {
+  if (!h || !Q || !V || !dO || !dQ || !dV) return LFA_ERR_INVALID_ARG;
+  if (!h->have_forward || h->last_Q != Q || h->last_V != V) return LFA_ERR_STATE;
+  (void)stream;
+  return LFA_ERR_UNSUPPORTED;
+}
+
+lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void* stream) {
+  if (!h || !host_out || n_units != h->p.U) return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = (size_t)h->p.U * lfa::kInfoStride;
+  float* tmp = static_cast<float*>(malloc(n * sizeof(float)));
+  if (!tmp) return LFA_ERR_INVALID_ARG;
+  int status = 0;
+  lfa_status ret = LFA_OK;
+  if (cudaMemcpyAsync(tmp, h->p.info, n * sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(&status, h->p.status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    ret = LFA_ERR_CUDA;
+  } else {
+    for (int u = 0; u < h->p.U; ++u) {
+      const float* f = tmp + (size_t)u * lfa::kInfoStride;
+      host_out[u].alpha = f[lfa::kInfoAlpha];
+      host_out[u].lambda_max = f[lfa::kInfoLambdaMax];
+      host_out[u].alpha_fallback = f[lfa::kInfoFallback] != 0.f;
+      host_out[u].ns_residual_fro = f[lfa::kInfoResidual];
+    }
+    if (status & lfa::kStatusTimeout) ret = LFA_ERR_TIMEOUT;
+    else if (status & lfa::kStatusNonFinite) ret = LFA_ERR_NONFINITE;
+  }
+  free(tmp);
+  return ret;
+}
+
+lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* C_out, void* stream) {
+  if (!h || !Q || !C_out || unit < 0 || unit >= h->p.U || !aligned16(Q)) return LFA_ERR_INVALID_ARG;
+  Params p = h->p;
+  p.Q = Q;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (lfa::launch_pool(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::launch_cross_kernel(p, unit, C_out, st) != cudaSuccess) return LFA_ERR_CUDA;
+  return LFA_OK;
+}
+
+lfa_status lfa_debug_context(lfa_handle h, int unit, float* L_out, float* X_out, float* mu_out,
+                             float* s_out, void* stream) {
+  if (!h || unit < 0 || unit >= h->p.U) return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t m = h->p.m, d = h->p.d;
+  struct { float* dst; const float* src; size_t n; } cp[4] = {
+      {L_out, h->p.L + unit * m * d, m * d},
+      {X_out, h->p.X + unit * m * m, m * m},
+      {mu_out, h->p.mu + unit * m, m},
+      {s_out, h->p.s + unit * m, m}};
+  for (auto& c : cp) {
+    if (!c.dst) continue;
+    if (cudaMemcpyAsync(c.dst, c.src, c.n * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return LFA_ERR_CUDA;
+  }
+  return LFA_OK;
+}
+
+lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end) {
+  if (!h || ((ev_begin == nullptr) != (ev_end == nullptr))) return LFA_ERR_INVALID_ARG;
+  h->p.ev_begin = ev_begin;
+  h->p.ev_end = ev_end;
+  return LFA_OK;
+}
+
+const char* lfa_dominant_kernel(lfa_handle h) {
+  if (!h) return "invalid";
+  return h->path == 1 ? "lfa_fused_forward" : "k_pass2";
+}
+
+int lfa_launches_per_forward(lfa_handle h) {
+  if (!h) return 0;
+  return lfa::generic_launch_count(h->p);
+}
+
+const char* lfa_forward_path(lfa_handle h) {
+  if (!h) return "invalid";
+  return h->path == 1 ? "fused" : "generic";
+}
+
+}  // extern "C"

@@ -1,0 +1,786 @@
+// Generic forward path of Laplacian-kernel Nystrom attention: every shape and dtype the
+// ABI accepts, CUDA cores only, two streaming passes over the tokens (C recomputed in
+// pass 2, never stored in HBM).
+//
+// Steps (LaplacianFormer note, papernotes.org: §整体框架 flowchart, §关键设计 1-3):
+//   k_pool          L = r x r average pool of Q                         (§关键设计 2)
+//   k_ns_small      W = exp(-E/lam) + eps I, ||W||_2, alpha, T Newton-Schulz steps, m <= 64
+//   k_gram / k_alpha / k_ns_gemm   the same for 64 < m <= 256, spread over CTAs (§关键设计 3)
+//   k_pass1         C tiles in registers/smem, column sums of C and C^2, raw C^T V, sum V
+//   k_combine_*     mu, var, s = 1/sqrt(var + eps); A = C~^T V by rank-1 folding; M = X A;
+//                   M' = diag(s) M; bias b = (1/N 1 - s o mu)^T M               (§关键设计 1)
+//   k_pass2         O = C M' + 1 b^T + DWC(V)                                  (§关键设计 1)
+#include <math.h>
+
+#include "lfa_internal.h"
+
+namespace lfa {
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// 4 consecutive elements -> float4 (16-byte / 8-byte aligned by the callers' layout)
+__device__ __forceinline__ float4 load4(const float* g) { return *reinterpret_cast<const float4*>(g); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* g) {
+  uint2 raw = *reinterpret_cast<const uint2*>(g);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&raw.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&raw.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+__device__ __forceinline__ void store4(float* g, float4 v) { *reinterpret_cast<float4*>(g) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* g, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 raw;
+  raw.x = *reinterpret_cast<uint32_t*>(&a);
+  raw.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(g) = raw;
+}
+
+__device__ __forceinline__ float l1_4(float4 a, float4 b, float acc) {
+  acc += fabsf(a.x - b.x);
+  acc += fabsf(a.y - b.y);
+  acc += fabsf(a.z - b.z);
+  acc += fabsf(a.w - b.w);
+  return acc;
+}
+
+// ---------------------------------------------------------------------------------------
+// Landmark pooling: one warp per landmark, lanes over channels (coalesced along d).
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pool(Params p) {
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.status = 0;
+  const int u = blockIdx.y;
+  const int l = blockIdx.x * (kThreads / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (l >= p.m) return;
+  const int Wr = p.W / p.r;
+  const int Y0 = (l / Wr) * p.r, X0 = (l % Wr) * p.r;
+  const T* q = static_cast<const T*>(p.Q) + (size_t)u * p.N * p.d;
+  const float inv = 1.0f / float(p.r * p.r);
+  for (int k = lane; k < p.d; k += 32) {
+    float acc = 0.f;
+    for (int dy = 0; dy < p.r; ++dy)
+      for (int dx = 0; dx < p.r; ++dx) acc += to_f(q[((size_t)(Y0 + dy) * p.W + X0 + dx) * p.d + k]);
+    p.L[((size_t)u * p.m + l) * p.d + k] = acc * inv;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Small-m landmark kernel + alpha + Newton-Schulz, one CTA per unit, all in shared memory.
+// ---------------------------------------------------------------------------------------
+constexpr int kNsS = 68;   // row stride (floats) of the 64 x 64 shared matrices
+
+// C = A * B for MP x MP matrices (MP <= 64, multiple of 16) in shared memory; 4x4 per thread.
+__device__ void smem_mm(const float* A, const float* B, float* C, int MP, float diag_scale,
+                        float add_diag) {
+  // C = diag_scale * (A B) + add_diag * I
+  const int nbj = MP / 4;
+  const int t = threadIdx.x;
+  if (t < nbj * nbj) {
+    const int bi = t / nbj, bj = t % nbj;
+    float acc[4][4] = {};
+    for (int l = 0; l < MP; ++l) {
+      float a[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) a[x] = A[(4 * bi + x) * kNsS + l];
+      float4 b = *reinterpret_cast<const float4*>(&B[l * kNsS + 4 * bj]);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
+        acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
+        acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
+        acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int i = 4 * bi + x, j = 4 * bj + y;
+        C[i * kNsS + j] = diag_scale * acc[x][y] + (i == j ? add_diag : 0.f);
+      }
+  }
+}
+
+__device__ float block_sum(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < (int)(blockDim.x / 32); ++i) s += red[i];
+  return s;
+}
+
+// Power iteration for lambda_max of the SPD matrix W (shared, MP x MP, zero padded).
+// Returns the Rayleigh quotient v^T W v of the final unit vector.
+__device__ float power_lambda_max(const float* Wsm, int m, float* v, float* w, float* red,
+                                  int iters) {
+  const int t = threadIdx.x;
+  if (t < kSmallM) v[t] = t < m ? rsqrtf(float(m)) : 0.f;
+  __syncthreads();
+  float rq = 0.f;
+  for (int it = 0; it <= iters; ++it) {
+    float wi = 0.f;
+    if (t < m) {
+      for (int j = 0; j < m; ++j) wi = fmaf(Wsm[t * kNsS + j], v[j], wi);
+    }
+    const float vw = block_sum(t < m ? wi * v[t] : 0.f, red);   // v^T W v
+    const float nn = block_sum(t < m ? wi * wi : 0.f, red);
+    rq = vw;
+    if (it == iters) break;
+    const float inv = rsqrtf(nn);
+    __syncthreads();
+    if (t < m) w[t] = wi * inv;
+    __syncthreads();
+    if (t < kSmallM) v[t] = t < m ? w[t] : 0.f;
+    __syncthreads();
+  }
+  return rq;
+}
+
+__global__ void __launch_bounds__(kThreads) k_ns_small(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  float* Wsm = sm;                         // [64][kNsS]
+  float* Xs = Wsm + 64 * kNsS;             // [64][kNsS]
+  float* Ys = Xs + 64 * kNsS;              // [64][kNsS]
+  float* Ls = Ys + 64 * kNsS;              // [64][d + 4]
+  float* vec = Ls + 64 * (64 + 4);         // 2 x 64
+  float* red = vec + 128;                  // 32
+  const int u = blockIdx.x, t = threadIdx.x;
+  const int m = p.m, d = p.d, MP = round_up(m, 16);
+  const int ds = d + 4;
+  for (int e = t; e < 64 * kNsS; e += blockDim.x) { Wsm[e] = 0.f; Xs[e] = 0.f; Ys[e] = 0.f; }
+  for (int e = t; e < m * d; e += blockDim.x) Ls[(e / d) * ds + e % d] = p.L[(size_t)u * m * d + e];
+  __syncthreads();
+  // W_ab = exp(-||l_a - l_b||_1 / lam) + eps delta_ab
+  for (int e = t; e < m * m; e += blockDim.x) {
+    const int a = e / m, b = e % m;
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc += fabsf(Ls[a * ds + k] - Ls[b * ds + k]);
+    Wsm[a * kNsS + b] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
+  }
+  __syncthreads();
+  const float lmax = power_lambda_max(Wsm, m, vec, vec + 64, red, 32);
+  // alpha = 2/||W||_2 as printed, kept only if ||I - alpha W W^T||_2 < 1; for SPD W that
+  // norm is max_j |1 - alpha w_j^2| = max(|1 - alpha lmax^2|, ...) which is < 1 iff
+  // alpha lmax^2 < 2.
+  const float alpha_p = 2.f / lmax;
+  const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
+  const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
+  // X_0 = alpha W^T
+  for (int e = t; e < m * m; e += blockDim.x) {
+    const int a = e / m, b = e % m;
+    Xs[a * kNsS + b] = alpha * Wsm[b * kNsS + a];
+  }
+  __syncthreads();
+  for (int k = 0; k < p.T; ++k) {
+    smem_mm(Wsm, Xs, Ys, MP, -1.f, 2.f);   // Y = 2I - W X
+    __syncthreads();
+    // X <- X Y: every thread reads its operands before anyone overwrites X
+    {
+      const int nbj = MP / 4;
+      float acc[4][4] = {};
+      int bi = 0, bj = 0;
+      const bool active = t < nbj * nbj;
+      if (active) {
+        bi = t / nbj;
+        bj = t % nbj;
+        for (int l = 0; l < MP; ++l) {
+          float a[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) a[x] = Xs[(4 * bi + x) * kNsS + l];
+          float4 b = *reinterpret_cast<const float4*>(&Ys[l * kNsS + 4 * bj]);
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
+            acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
+            acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
+            acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
+          }
+        }
+      }
+      __syncthreads();
+      if (active) {
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) Xs[(4 * bi + x) * kNsS + 4 * bj + y] = acc[x][y];
+      }
+      __syncthreads();
+    }
+  }
+  // residual ||I - W X_T||_F
+  smem_mm(Wsm, Xs, Ys, MP, -1.f, 1.f);
+  __syncthreads();
+  float sq = 0.f;
+  for (int e = t; e < m * m; e += blockDim.x) {
+    const float r = Ys[(e / m) * kNsS + e % m];
+    sq += r * r;
+  }
+  const float res = sqrtf(block_sum(sq, red));
+  for (int e = t; e < m * m; e += blockDim.x) {
+    const int a = e / m, b = e % m;
+    p.X[(size_t)u * m * m + e] = Xs[a * kNsS + b];
+    p.Wm[(size_t)u * m * m + e] = Wsm[a * kNsS + b];
+  }
+  if (t == 0) {
+    float* inf = p.info + (size_t)u * kInfoStride;
+    inf[kInfoAlpha] = alpha;
+    inf[kInfoLambdaMax] = lmax;
+    inf[kInfoFallback] = float(fallback);
+    inf[kInfoResidual] = res;
+    if (!isfinite(lmax) || !isfinite(res)) atomicOr(p.status, kStatusNonFinite);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Large-m Newton-Schulz (64 < m <= 256): W and X in global memory, one launch per product.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_gram(Params p) {
+  const int u = blockIdx.y, m = p.m, d = p.d;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= m * m) return;
+  const int a = e / m, b = e % m;
+  const float* La = p.L + ((size_t)u * m + a) * d;
+  const float* Lb = p.L + ((size_t)u * m + b) * d;
+  float acc = 0.f;
+  for (int k = 0; k < d; ++k) acc += fabsf(La[k] - Lb[k]);
+  p.Wm[(size_t)u * m * m + e] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
+}
+
+__global__ void __launch_bounds__(kThreads) k_alpha(Params p) {
+  __shared__ float v[kMaxM], w[kMaxM], red[32];
+  const int u = blockIdx.x, m = p.m, t = threadIdx.x;
+  const float* Wg = p.Wm + (size_t)u * m * m;
+  const int warp = t / 32, lane = t & 31, nw = blockDim.x / 32;
+  if (t < m) v[t] = rsqrtf(float(m));
+  __syncthreads();
+  float rq = 0.f;
+  const int iters = 24;
+  for (int it = 0; it <= iters; ++it) {
+    // w = W v, one warp per row (coalesced along the row)
+    for (int i = warp; i < m; i += nw) {
+      float acc = 0.f;
+      for (int j = lane; j < m; j += 32) acc = fmaf(Wg[(size_t)i * m + j], v[j], acc);
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) w[i] = acc;
+    }
+    __syncthreads();
+    const float vw = block_sum(t < m ? w[t] * v[t] : 0.f, red);
+    const float nn = block_sum(t < m ? w[t] * w[t] : 0.f, red);
+    rq = vw;
+    if (it == iters) break;
+    const float inv = rsqrtf(nn);
+    __syncthreads();
+    if (t < m) v[t] = w[t] * inv;
+    __syncthreads();
+  }
+  const float lmax = rq;
+  const float alpha_p = 2.f / lmax;
+  const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
+  const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
+  float* Xg = p.X + (size_t)u * m * m;
+  for (int e = t; e < m * m; e += blockDim.x) {
+    const int a = e / m, b = e % m;
+    Xg[e] = alpha * Wg[(size_t)b * m + a];
+  }
+  if (t == 0) {
+    float* inf = p.info + (size_t)u * kInfoStride;
+    inf[kInfoAlpha] = alpha;
+    inf[kInfoLambdaMax] = lmax;
+    inf[kInfoFallback] = float(fallback);
+    inf[kInfoResidual] = 0.f;
+    if (!isfinite(lmax)) atomicOr(p.status, kStatusNonFinite);
+  }
+}
+
+// out = scale * (A B) + add_diag * I for m x m row-major matrices of unit blockIdx.z.
+// 64 x 64 output tile per CTA, 16-wide K chunks staged in shared memory.
+// mode 2 additionally accumulates ||out||_F^2 into info[residual].
+__global__ void __launch_bounds__(kThreads) k_ns_gemm(Params p, const float* Ab, const float* Bb,
+                                                      float* Ob, float scale, float add_diag,
+                                                      int accumulate_norm) {
+  __shared__ float As[64][17];
+  __shared__ __align__(16) float Bs[16][64];
+  const int u = blockIdx.z, m = p.m;
+  const float* A = Ab + (size_t)u * m * m;
+  const float* B = Bb + (size_t)u * m * m;
+  float* Out = Ob + (size_t)u * m * m;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  const int t = threadIdx.x, bi = t / 16, bj = t % 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < m; k0 += 16) {
+    for (int e = t; e < 64 * 16; e += blockDim.x) {
+      const int r = e / 16, c = e % 16;
+      As[r][c] = (i0 + r < m && k0 + c < m) ? A[(size_t)(i0 + r) * m + k0 + c] : 0.f;
+      const int r2 = e / 64, c2 = e % 64;
+      Bs[r2][c2] = (k0 + r2 < m && j0 + c2 < m) ? B[(size_t)(k0 + r2) * m + j0 + c2] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int l = 0; l < 16; ++l) {
+      float a[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) a[x] = As[4 * bi + x][l];
+      float4 b = *reinterpret_cast<const float4*>(&Bs[l][4 * bj]);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
+        acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
+        acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
+        acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
+      }
+    }
+    __syncthreads();
+  }
+  float sq = 0.f;
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int i = i0 + 4 * bi + x, j = j0 + 4 * bj + y;
+      if (i < m && j < m) {
+        const float v = scale * acc[x][y] + (i == j ? add_diag : 0.f);
+        Out[(size_t)i * m + j] = v;
+        sq += v * v;
+      }
+    }
+  if (accumulate_norm) {
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if ((t & 31) == 0) atomicAdd(p.info + (size_t)u * kInfoStride + kInfoResidual, sq);
+  }
+}
+
+__global__ void k_residual_sqrt(Params p) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= p.U) return;
+  float* r = p.info + (size_t)u * kInfoStride + kInfoResidual;
+  *r = sqrtf(*r);
+  if (!isfinite(*r)) atomicOr(p.status, kStatusNonFinite);
+}
+
+// ---------------------------------------------------------------------------------------
+// Cross-kernel tile: rows [0, 64) of Qs against landmarks [j0, j0 + 64) of Ls.
+// 256 threads: thread (tr, tl) owns rows 4tr..4tr+3 and landmarks j0 + tl + 16 jj.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void cross_tile(const float* Qs, const float* Ls, float* Cs, int d,
+                                           int j0, int m, int cs_stride, float scale,
+                                           int valid_rows) {
+  const int t = threadIdx.x, tr = t >> 4, tl = t & 15;
+  const int ds = d + 4;
+  float acc[4][4] = {};
+  for (int k = 0; k < d; k += 4) {
+    float4 q[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = *reinterpret_cast<const float4*>(&Qs[(4 * tr + i) * ds + k]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      l[j] = *reinterpret_cast<const float4*>(&Ls[(j0 + tl + 16 * j) * ds + k]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = l1_4(q[i], l[j], acc[i][j]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int row = 4 * tr + i, col = j0 + tl + 16 * j;
+      Cs[row * cs_stride + col] = (col < m && row < valid_rows) ? exp2f(acc[i][j] * scale) : 0.f;
+    }
+}
+
+// Stage a 64-row tile of a [N][d] token tensor into shared memory (fp32, row stride d + 4),
+// zero-filling rows past `valid`.
+template <typename T>
+__device__ __forceinline__ void stage_rows(const T* g, float* s, int d, int valid) {
+  const int ds = d + 4, q4 = d / 4;
+  for (int e = threadIdx.x; e < kRowTile * q4; e += blockDim.x) {
+    const int r = e / q4, c = (e % q4) * 4;
+    float4 v = r < valid ? load4(g + (size_t)r * d + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(&s[r * ds + c]) = v;
+  }
+}
+
+__device__ __forceinline__ void stage_landmarks(const float* Lg, float* Ls, int m, int mpl, int d) {
+  const int ds = d + 4;
+  for (int e = threadIdx.x; e < mpl * d; e += blockDim.x) {
+    const int r = e / d, c = e % d;
+    Ls[r * ds + c] = r < m ? Lg[(size_t)r * d + c] : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Pass 1: per unit and CTA, sums over its rows of C, C^2, C^T V and V.
+// ---------------------------------------------------------------------------------------
+template <typename T, int BPT>
+__global__ void __launch_bounds__(kThreads) k_pass1(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, ds = d + 4;
+  const int mpl = round_up(m, 64), cs = mpl + 4;
+  float* Ls = sm;                    // [mpl][ds]
+  float* Qs = Ls + mpl * ds;         // [64][ds]
+  float* Vs = Qs + kRowTile * ds;    // [64][ds]
+  float* Cs = Vs + kRowTile * ds;    // [64][cs]
+  const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x;
+  const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
+  const T* Vg = static_cast<const T*>(p.V) + (size_t)u * p.N * d;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
+
+  const int nbk = d / 4, nbj = round_up(m, 4) / 4, nb = nbj * nbk;
+  float accP[BPT][4][4] = {};
+  float s1 = 0.f, s2 = 0.f, sv = 0.f;
+  const int tile0 = pc * p.tiles_per_cta;
+  const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
+  for (int tile = tile0; tile < tile1; ++tile) {
+    const int row0 = tile * kRowTile;
+    const int valid = min(kRowTile, p.N - row0);
+    __syncthreads();
+    stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+    stage_rows(Vg + (size_t)row0 * d, Vs, d, valid);
+    __syncthreads();
+    for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
+    __syncthreads();
+    if (t < m) {
+      for (int i = 0; i < kRowTile; ++i) {
+        const float c = Cs[i * cs + t];
+        s1 += c;
+        s2 = fmaf(c, c, s2);
+      }
+    }
+    if (t < d) {
+      for (int i = 0; i < kRowTile; ++i) sv += Vs[i * ds + t];
+    }
+#pragma unroll
+    for (int q = 0; q < BPT; ++q) {
+      const int b = t + q * kThreads;
+      if (b < nb) {
+        const int jb = b / nbk, kb = b % nbk;
+        for (int i = 0; i < kRowTile; ++i) {
+          const float4 c = *reinterpret_cast<const float4*>(&Cs[i * cs + 4 * jb]);
+          const float4 v = *reinterpret_cast<const float4*>(&Vs[i * ds + 4 * kb]);
+          const float cc[4] = {c.x, c.y, c.z, c.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) accP[q][x][y] = fmaf(cc[x], vv[y], accP[q][x][y]);
+        }
+      }
+    }
+  }
+  float* out = p.part + ((size_t)u * p.P + pc) * p.part_stride;
+  if (t < m) {
+    out[t] = s1;
+    out[m + t] = s2;
+  }
+  if (t < d) out[2 * m + m * d + t] = sv;
+#pragma unroll
+  for (int q = 0; q < BPT; ++q) {
+    const int b = t + q * kThreads;
+    if (b < nb) {
+      const int jb = b / nbk, kb = b % nbk;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int j = 4 * jb + x;
+        if (j < m)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) out[2 * m + j * d + 4 * kb + y] = accP[q][x][y];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Combine: reduce the pass-1 partials of a unit in fp64.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_combine_reduce(Params p) {
+  const int u = blockIdx.y;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= p.part_stride) return;
+  double acc = 0.0;
+  const float* src = p.part + (size_t)u * p.P * p.part_stride + e;
+  for (int pc = 0; pc < p.P; ++pc) acc += (double)src[(size_t)pc * p.part_stride];
+  p.red[(size_t)u * p.part_stride + e] = acc;
+}
+
+// mu, s, A (all landmarks), then M = X A, M' and bias partials for 16 landmark rows.
+__global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, u = blockIdx.y, c = blockIdx.x, t = threadIdx.x;
+  float* As = sm;               // [m][d]
+  float* mus = As + m * d;      // [m]
+  float* ss = mus + m;          // [m]
+  const double* red = p.red + (size_t)u * p.part_stride;
+  const double invN = 1.0 / double(p.N);
+  for (int j = t; j < m; j += blockDim.x) {
+    const double mu = red[j] * invN;
+    double var = red[m + j] * invN - mu * mu;
+    if (var < 0.0) var = 0.0;
+    const double s = 1.0 / sqrt(var + (double)p.eps);
+    mus[j] = (float)mu;
+    ss[j] = (float)s;
+    if (c == 0) {
+      p.mu[(size_t)u * m + j] = (float)mu;
+      p.s[(size_t)u * m + j] = (float)s;
+    }
+  }
+  const double* P = red + 2 * m;
+  const double* SV = red + 2 * m + m * d;
+  for (int e = t; e < m * d; e += blockDim.x) {
+    const int j = e / d, k = e % d;
+    double a;
+    if (p.whiten) {
+      const double mu = red[j] * invN;
+      double var = red[m + j] * invN - mu * mu;
+      if (var < 0.0) var = 0.0;
+      const double s = 1.0 / sqrt(var + (double)p.eps);
+      a = s * (P[e] - mu * SV[k]) + SV[k] * invN;
+    } else {
+      a = P[e];
+    }
+    As[e] = (float)a;
+    if (c == 0) p.A[(size_t)u * m * d + e] = (float)a;
+  }
+  __syncthreads();
+  // rows [16c, 16c + 16) of M = X A
+  const float* Xg = p.X + (size_t)u * m * m;
+  float* bp = p.bpart + ((size_t)u * p.n_chunks + c) * d;
+  const int j0 = c * 16;
+  for (int e = t; e < 16 * d; e += blockDim.x) {
+    const int jj = e / d, k = e % d, j = j0 + jj;
+    if (j < m) {
+      float acc = 0.f;
+      for (int l = 0; l < m; ++l) acc = fmaf(Xg[(size_t)j * m + l], As[l * d + k], acc);
+      p.M[((size_t)u * m + j) * d + k] = acc;
+      p.Mp[((size_t)u * m + j) * d + k] = p.whiten ? ss[j] * acc : acc;
+    }
+  }
+  __syncthreads();
+  // bias partial: b[k] = sum_j (1/N - s_j mu_j) M[j][k] over this chunk's rows
+  for (int k = t; k < d; k += blockDim.x) {
+    float acc = 0.f;
+    if (p.whiten) {
+      for (int jj = 0; jj < 16; ++jj) {
+        const int j = j0 + jj;
+        if (j < m) acc += (float)(invN - (double)ss[j] * (double)mus[j]) * p.M[((size_t)u * m + j) * d + k];
+      }
+    }
+    bp[k] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Pass 2: O = C M' + 1 b^T + DWC(V) for one 64-row tile.
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_pass2(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, ds = d + 4;
+  const int mpl = round_up(m, 64), cs = mpl + 4;
+  float* Ls = sm;                    // [mpl][ds], later M'
+  float* Qs = Ls + mpl * ds;         // [64][ds]
+  float* Cs = Qs + kRowTile * ds;    // [64][cs]
+  float* bs = Cs + kRowTile * cs;    // [d]
+  const int u = blockIdx.y, tile = blockIdx.x, t = threadIdx.x;
+  const int row0 = tile * kRowTile, valid = min(kRowTile, p.N - row0);
+  const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
+  const T* Vg = static_cast<const T*>(p.V) + (size_t)u * p.N * d;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
+  stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+  if (t < d) {
+    float b = 0.f;
+    for (int c = 0; c < p.n_chunks; ++c) b += p.bpart[((size_t)u * p.n_chunks + c) * d + t];
+    bs[t] = b;
+  }
+  __syncthreads();
+  for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
+  __syncthreads();
+  stage_landmarks(p.Mp + (size_t)u * m * d, Ls, m, round_up(m, 4), d);
+  __syncthreads();
+  const int nbk = d / 4;
+  if (t < 16 * nbk) {
+    const int ib = t / nbk, kb = t % nbk;
+    float acc[4][4] = {};
+    const int m4 = round_up(m, 4);
+    for (int j = 0; j < m4; j += 4) {
+      float4 c[4], mp[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) c[x] = *reinterpret_cast<const float4*>(&Cs[(4 * ib + x) * cs + j]);
+#pragma unroll
+      for (int y = 0; y < 4; ++y) mp[y] = *reinterpret_cast<const float4*>(&Ls[(j + y) * ds + 4 * kb]);
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float cc[4] = {c[x].x, c[x].y, c[x].z, c[x].w};
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          acc[x][0] = fmaf(cc[y], mp[y].x, acc[x][0]);
+          acc[x][1] = fmaf(cc[y], mp[y].y, acc[x][1]);
+          acc[x][2] = fmaf(cc[y], mp[y].z, acc[x][2]);
+          acc[x][3] = fmaf(cc[y], mp[y].w, acc[x][3]);
+        }
+      }
+    }
+    // DWC(V): w[h][k][a][b] multiplies V[y + a - 1][x + b - 1][k]
+    const int h = u % p.heads;
+    float wt[4][9];
+#pragma unroll
+    for (int y = 0; y < 4; ++y)
+#pragma unroll
+      for (int e = 0; e < 9; ++e) wt[y][e] = p.dwc[((size_t)h * d + 4 * kb + y) * 9 + e];
+    T* Og = static_cast<T*>(p.O) + (size_t)u * p.N * d;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int i = 4 * ib + x;
+      if (i >= valid) continue;
+      const int n = row0 + i, gy = n / p.W, gx = n % p.W;
+      float o[4] = {acc[x][0] + bs[4 * kb], acc[x][1] + bs[4 * kb + 1], acc[x][2] + bs[4 * kb + 2],
+                    acc[x][3] + bs[4 * kb + 3]};
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        const int yy = gy + a - 1;
+        if (yy < 0 || yy >= p.H) continue;
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+          const int xx = gx + b - 1;
+          if (xx < 0 || xx >= p.W) continue;
+          const float4 v = load4(Vg + ((size_t)yy * p.W + xx) * d + 4 * kb);
+          o[0] = fmaf(wt[0][a * 3 + b], v.x, o[0]);
+          o[1] = fmaf(wt[1][a * 3 + b], v.y, o[1]);
+          o[2] = fmaf(wt[2][a * 3 + b], v.z, o[2]);
+          o[3] = fmaf(wt[3][a * 3 + b], v.w, o[3]);
+        }
+      }
+      store4(Og + (size_t)n * d + 4 * kb, make_float4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
+// C of one unit, [N][m] fp32, from the same tile code as the passes.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_cross_out(Params p, int u, float* C_out) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, ds = d + 4;
+  const int mpl = round_up(m, 64), cs = mpl + 4;
+  float* Ls = sm;
+  float* Qs = Ls + mpl * ds;
+  float* Cs = Qs + kRowTile * ds;
+  const int row0 = blockIdx.x * kRowTile, valid = min(kRowTile, p.N - row0);
+  const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
+  stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+  __syncthreads();
+  for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
+  __syncthreads();
+  for (int e = threadIdx.x; e < valid * m; e += blockDim.x) {
+    const int i = e / m, j = e % m;
+    C_out[(size_t)(row0 + i) * m + j] = Cs[i * cs + j];
+  }
+}
+
+template <typename T>
+cudaError_t forward_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m, d = p.d;
+  k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
+  if (m <= kSmallM) {
+    const size_t smem = (3 * 64 * kNsS + 64 * 68 + 128 + 32) * sizeof(float);
+    k_ns_small<<<U, kThreads, smem, st>>>(p);
+  } else {
+    k_gram<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
+    k_alpha<<<U, kThreads, 0, st>>>(p);
+    const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
+    float* x = p.X;
+    float* xb = p.Xb;
+    for (int k = 0; k < p.T; ++k) {
+      k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, x, p.Y, -1.f, 2.f, 0);   // Y = 2I - W X
+      k_ns_gemm<<<g, kThreads, 0, st>>>(p, x, p.Y, xb, 1.f, 0.f, 0);      // X' = X Y
+      float* tmp = x; x = xb; xb = tmp;
+    }
+    if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
+    k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
+    k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
+  }
+  const int bpt = ceil_div((round_up(m, 4) / 4) * (d / 4), kThreads);
+  const dim3 g1(p.P, U);
+  const size_t s1 = generic_smem_pass1(m, d);
+  if (bpt <= 1) k_pass1<T, 1><<<g1, kThreads, s1, st>>>(p);
+  else if (bpt <= 2) k_pass1<T, 2><<<g1, kThreads, s1, st>>>(p);
+  else k_pass1<T, 4><<<g1, kThreads, s1, st>>>(p);
+  k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
+  k_combine_finish<<<dim3(p.n_chunks, U), kThreads, (size_t)(m * d + 2 * m) * sizeof(float), st>>>(p);
+  if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
+  k_pass2<T><<<dim3(p.n_tiles, U), kThreads, generic_smem_pass2(m, d), st>>>(p);
+  if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t generic_smem_pass1(int m, int d) {
+  const int mpl = round_up(m, 64), ds = d + 4;
+  return sizeof(float) * ((size_t)mpl * ds + 2 * kRowTile * ds + (size_t)kRowTile * (mpl + 4));
+}
+
+size_t generic_smem_pass2(int m, int d) {
+  const int mpl = round_up(m, 64), ds = d + 4;
+  return sizeof(float) * ((size_t)mpl * ds + kRowTile * ds + (size_t)kRowTile * (mpl + 4) + d);
+}
+
+cudaError_t generic_set_attributes() {
+  const int big = 227 * 1024;
+  cudaError_t e = cudaSuccess;
+#define LFA_ATTR(fn) \
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, big)
+  LFA_ATTR(k_ns_small);
+  LFA_ATTR((k_pass1<float, 1>));
+  LFA_ATTR((k_pass1<float, 2>));
+  LFA_ATTR((k_pass1<float, 4>));
+  LFA_ATTR((k_pass1<__nv_bfloat16, 1>));
+  LFA_ATTR((k_pass1<__nv_bfloat16, 2>));
+  LFA_ATTR((k_pass1<__nv_bfloat16, 4>));
+  LFA_ATTR(k_combine_finish);
+  LFA_ATTR(k_pass2<float>);
+  LFA_ATTR(k_pass2<__nv_bfloat16>);
+  LFA_ATTR(k_cross_out<float>);
+  LFA_ATTR(k_cross_out<__nv_bfloat16>);
+#undef LFA_ATTR
+  return e;
+}
+
+int generic_launch_count(const Params& p) {
+  // pool, Newton-Schulz chain, pass 1, two combine kernels, pass 2
+  const int ns = p.m <= kSmallM ? 1 : 2 + 2 * p.T + 2;
+  return 1 + ns + 1 + 2 + 1;
+}
+
+cudaError_t launch_generic_forward(const Params& p, cudaStream_t st) {
+  return p.dtype == LFA_BF16 ? forward_t<__nv_bfloat16>(p, st) : forward_t<float>(p, st);
+}
+
+cudaError_t launch_pool(const Params& p, cudaStream_t st) {
+  const dim3 g(ceil_div(p.m, kThreads / 32), p.U);
+  if (p.dtype == LFA_BF16) k_pool<__nv_bfloat16><<<g, kThreads, 0, st>>>(p);
+  else k_pool<float><<<g, kThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cross_kernel(const Params& p, int unit, float* C_out, cudaStream_t st) {
+  const size_t smem = generic_smem_pass2(p.m, p.d);
+  if (p.dtype == LFA_BF16)
+    k_cross_out<__nv_bfloat16><<<p.n_tiles, kThreads, smem, st>>>(p, unit, C_out);
+  else
+    k_cross_out<float><<<p.n_tiles, kThreads, smem, st>>>(p, unit, C_out);
+  return cudaGetLastError();
+}
+
+}  // namespace lfa

@@ -1,0 +1,84 @@
+// Internal declarations shared by the host entry points and the kernels of liblfa.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "lfa.h"
+
+namespace lfa {
+
+constexpr int kMaxM = 256;        // largest landmark count supported
+constexpr int kMaxT = 64;         // largest Newton-Schulz step count accepted
+constexpr int kRowTile = 64;      // token rows per tile in the generic kernels
+constexpr int kThreads = 256;     // threads per CTA in the generic kernels
+constexpr int kSmallM = 64;       // m <= kSmallM: one CTA solves a unit's Newton-Schulz chain
+
+// status-word bits (device side); lfa_get_info maps them to lfa_status
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusNonFinite = 2;
+
+// per-unit diagnostics slots (floats) in the workspace
+constexpr int kInfoAlpha = 0, kInfoLambdaMax = 1, kInfoFallback = 2, kInfoResidual = 3;
+constexpr int kInfoStride = 4;
+
+__host__ __device__ inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Byte offsets of every buffer carved from the caller's workspace.
+struct Layout {
+  size_t status, info, L, Wm, X, Xb, Y, part, red, mu, s, A, M, Mp, bpart;
+  size_t fused;    // scratch of the fused forward (per-CTA partials, barriers)
+  size_t bwd;      // backward-pass buffers
+  size_t total;
+};
+
+// Everything a kernel needs, passed by value.
+struct Params {
+  // shape
+  int B, heads, H, W, N, d, r, m, T, whiten, dtype, U;
+  float lam, eps;
+  float neg_log2e_over_lam;  // C = exp2(D * neg_log2e_over_lam)
+  // generic pass-1 decomposition
+  int P;             // pass-1 CTAs per unit
+  int tiles_per_cta; // 64-row tiles per pass-1 CTA
+  int n_tiles;       // 64-row tiles per unit
+  int part_stride;   // floats per partial record: S1[m], S2[m], P[m][d], SV[d]
+  int n_chunks;      // combine row chunks of 16 landmarks (bias partials)
+  // tensors
+  const void* Q;
+  const void* V;
+  void* O;
+  const float* dwc;
+  // workspace views
+  int* status;
+  float* info;
+  float* L;      // [U][m][d]
+  float* Wm;     // [U][m][m] (W + eps I)
+  float* X;      // [U][m][m]
+  float* Xb;     // [U][m][m] ping-pong buffer of the multi-CTA Newton-Schulz
+  float* Y;      // [U][m][m]
+  float* part;   // [U][P][part_stride]
+  double* red;   // [U][part_stride]
+  float* mu;     // [U][m]
+  float* s;      // [U][m]
+  float* A;      // [U][m][d]
+  float* M;      // [U][m][d]
+  float* Mp;     // [U][m][d]
+  float* bpart;  // [U][n_chunks][d]
+  // optional timing events bracketing the dominant kernel (cudaEvent_t or null)
+  void* ev_begin;
+  void* ev_end;
+};
+
+// host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu
+cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
+cudaError_t launch_pool(const Params& p, cudaStream_t st);
+cudaError_t launch_cross_kernel(const Params& p, int unit, float* C_out, cudaStream_t st);
+size_t generic_smem_pass1(int m, int d);
+size_t generic_smem_pass2(int m, int d);
+cudaError_t generic_set_attributes();
+int generic_launch_count(const Params& p);
+
+}  // namespace lfa

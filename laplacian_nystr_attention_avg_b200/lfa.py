@@ -1,0 +1,221 @@
+"""Thin ctypes binding of liblfa.so (include/lfa.h). Argument marshalling only.
+
+PyTorch supplies device memory and streams; every step of the attention path runs
+in the library's CUDA kernels. If the library is missing this module raises: there
+is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import List, Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblfa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "lfa.h")
+
+LFA_OK, LFA_ERR_INVALID_ARG, LFA_ERR_UNSUPPORTED, LFA_ERR_CUDA, LFA_ERR_STATE, \
+    LFA_ERR_TIMEOUT, LFA_ERR_NONFINITE = range(7)
+LFA_F32, LFA_BF16 = 0, 1
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("d", ctypes.c_int), ("r", ctypes.c_int), ("lambda_", ctypes.c_float),
+                ("eps", ctypes.c_float), ("T", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("whiten", ctypes.c_int)]
+
+
+class UnitInfo(ctypes.Structure):
+    _fields_ = [("alpha_fallback", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("lambda_max", ctypes.c_float), ("ns_residual_fro", ctypes.c_float)]
+
+
+class LfaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def _declare(lib: ctypes.CDLL) -> None:
+    vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    cfgp = ctypes.POINTER(Config)
+    sig = {
+        "lfa_workspace_size": (sz, [cfgp]),
+        "lfa_create": (ci, [cfgp, vp, vp, sz, ctypes.POINTER(vp)]),
+        "lfa_forward": (ci, [vp, vp, vp, vp, vp]),
+        "lfa_forward_host": (ci, [vp, vp, vp, vp, vp, vp, vp, vp]),
+        "lfa_backward": (ci, [vp, vp, vp, vp, vp, vp, vp]),
+        "lfa_get_info": (ci, [vp, ctypes.POINTER(UnitInfo), ci, vp]),
+        "lfa_destroy": (ci, [vp]),
+        "lfa_status_string": (ctypes.c_char_p, [ci]),
+        "lfa_debug_cross_kernel": (ci, [vp, vp, ci, vp, vp]),
+        "lfa_debug_context": (ci, [vp, ci, vp, vp, vp, vp, vp]),
+        "lfa_forward_path": (ctypes.c_char_p, [vp]),
+        "lfa_set_profile_events": (ci, [vp, vp, vp]),
+        "lfa_dominant_kernel": (ctypes.c_char_p, [vp]),
+        "lfa_launches_per_forward": (ci, [vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+
+
+def load() -> ctypes.CDLL:
+    """Open liblfa.so from the package directory (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"liblfa.so not found at {LIB_PATH}; build it with "
+                               "`python -m laplacian_nystr_attention_avg_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        _declare(lib)
+        _lib = lib
+    return _lib
+
+
+def header_symbols() -> List[str]:
+    """Names of the entry points declared in include/lfa.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lfa_[a-z_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load().lfa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != LFA_OK:
+        raise LfaError(status, what)
+
+
+def make_config(wl, whiten: bool = True) -> Config:
+    """lfa_config from a Workload (laplacian_nystr_attention_avg_b200.inputs)."""
+    return Config(wl.B, wl.heads, wl.H, wl.W, wl.d, wl.r, float(wl.lam), float(wl.eps), int(wl.T),
+                  LFA_BF16 if wl.dtype == "bf16" else LFA_F32, 1 if whiten else 0)
+
+
+def workspace_size(cfg: Config) -> int:
+    return int(load().lfa_workspace_size(ctypes.byref(cfg)))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+class LaplacianNystromAttention:
+    """One configured attention call: owns a torch-allocated workspace and an lfa handle.
+
+    dwc_weight: float32 [heads, d, 3, 3] (moved to the device). Q, V, O tensors are
+    [B, heads, N, d] contiguous in the config's dtype on the same device.
+    """
+
+    def __init__(self, cfg: Config, dwc_weight: torch.Tensor, device: str = "cuda"):
+        self.lib = load()
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.dtype = torch.bfloat16 if cfg.dtype == LFA_BF16 else torch.float32
+        self.units = cfg.B * cfg.heads
+        self.N = cfg.H * cfg.W
+        self.m = (cfg.H // cfg.r) * (cfg.W // cfg.r)
+        self.shape = (cfg.B, cfg.heads, self.N, cfg.d)
+        self.weight = dwc_weight.to(self.device, torch.float32).contiguous()
+        nbytes = workspace_size(cfg)
+        if nbytes == 0:
+            raise LfaError(LFA_ERR_INVALID_ARG, "lfa_workspace_size")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        _check(self.lib.lfa_create(ctypes.byref(cfg), self.weight.data_ptr(), self.workspace.data_ptr(),
+                                   nbytes, ctypes.byref(h)), "lfa_create")
+        self.handle = h
+
+    @property
+    def path(self) -> str:
+        return self.lib.lfa_forward_path(self.handle).decode()
+
+    @property
+    def launches_per_forward(self) -> int:
+        return int(self.lib.lfa_launches_per_forward(self.handle))
+
+    @property
+    def dominant_kernel(self) -> str:
+        return self.lib.lfa_dominant_kernel(self.handle).decode()
+
+    def set_profile_events(self, begin=None, end=None) -> None:
+        """Bracket the dominant kernel of later forwards with two torch.cuda.Event objects."""
+        b = None if begin is None else begin.cuda_event
+        e = None if end is None else end.cuda_event
+        _check(self.lib.lfa_set_profile_events(self.handle, b, e), "lfa_set_profile_events")
+
+    def new_output(self) -> torch.Tensor:
+        return torch.empty(self.shape, dtype=self.dtype, device=self.device)
+
+    def forward(self, Q: torch.Tensor, V: torch.Tensor, O: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+        if O is None:
+            O = self.new_output()
+        _check(self.lib.lfa_forward(self.handle, _ptr(Q), _ptr(V), _ptr(O), _stream(stream)), "lfa_forward")
+        return O
+
+    def forward_host(self, Q_host, V_host, O_host, Q_dev, V_dev, O_dev, stream=None) -> None:
+        _check(self.lib.lfa_forward_host(self.handle, _ptr(Q_host), _ptr(V_host), _ptr(O_host), _ptr(Q_dev),
+                                         _ptr(V_dev), _ptr(O_dev), _stream(stream)), "lfa_forward_host")
+
+    def backward(self, Q, V, dO, dQ=None, dV=None, stream=None):
+        if dQ is None:
+            dQ = self.new_output()
+        if dV is None:
+            dV = self.new_output()
+        _check(self.lib.lfa_backward(self.handle, _ptr(Q), _ptr(V), _ptr(dO), _ptr(dQ), _ptr(dV),
+                                     _stream(stream)), "lfa_backward")
+        return dQ, dV
+
+    def info(self, stream=None):
+        """(status, [UnitInfo]) of the most recent forward; synchronises the stream."""
+        arr = (UnitInfo * self.units)()
+        st = self.lib.lfa_get_info(self.handle, arr, self.units, _stream(stream))
+        if st not in (LFA_OK, LFA_ERR_TIMEOUT, LFA_ERR_NONFINITE):
+            raise LfaError(st, "lfa_get_info")
+        return st, list(arr)
+
+    def cross_kernel(self, Q: torch.Tensor, unit: int, stream=None) -> torch.Tensor:
+        C = torch.empty((self.N, self.m), dtype=torch.float32, device=self.device)
+        _check(self.lib.lfa_debug_cross_kernel(self.handle, _ptr(Q), int(unit), _ptr(C), _stream(stream)),
+               "lfa_debug_cross_kernel")
+        return C
+
+    def context(self, unit: int, stream=None):
+        d = self.cfg.d
+        L = torch.empty((self.m, d), dtype=torch.float32, device=self.device)
+        X = torch.empty((self.m, self.m), dtype=torch.float32, device=self.device)
+        mu = torch.empty((self.m,), dtype=torch.float32, device=self.device)
+        s = torch.empty((self.m,), dtype=torch.float32, device=self.device)
+        _check(self.lib.lfa_debug_context(self.handle, int(unit), _ptr(L), _ptr(X), _ptr(mu), _ptr(s),
+                                          _stream(stream)), "lfa_debug_context")
+        return L, X, mu, s
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            self.lib.lfa_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

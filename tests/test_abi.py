@@ -1,0 +1,97 @@
+"""The C-ABI library loads and exports what include/lfa.h declares; host-side validation.
+
+No compute call is made here (no GPU needed): only entry points that return before
+touching the device.
+"""
+import ctypes
+import os
+
+import pytest
+
+from laplacian_nystr_attention_avg_b200 import build as lfa_build
+from laplacian_nystr_attention_avg_b200 import lfa
+from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lfa_build.build()
+    return lfa.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = lfa.header_symbols()
+    assert "lfa_forward" in names and "lfa_backward" in names and "lfa_create" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/lfa.h but not exported"
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lfa.status_string(s) and lfa.status_string(s) != "unknown status"
+    assert lfa.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_workspace_size_valid_configs(lib, name):
+    cfg = lfa.make_config(WORKLOADS[name])
+    n = lfa.workspace_size(cfg)
+    assert n > 0 and n % 256 == 0
+
+
+def _cfg(**kw):
+    base = dict(B=1, heads=1, H=16, W=16, d=32, r=4, lambda_=4.0, eps=1e-6, T=20, dtype=lfa.LFA_F32, whiten=1)
+    base.update(kw)
+    return lfa.Config(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(H=15), lfa.LFA_ERR_INVALID_ARG),              # H % r != 0
+    (dict(W=18), lfa.LFA_ERR_INVALID_ARG),              # W % r != 0
+    (dict(lambda_=0.0), lfa.LFA_ERR_INVALID_ARG),
+    (dict(lambda_=-1.0), lfa.LFA_ERR_INVALID_ARG),
+    (dict(lambda_=float("nan")), lfa.LFA_ERR_INVALID_ARG),
+    (dict(eps=-1e-6), lfa.LFA_ERR_INVALID_ARG),
+    (dict(T=-1), lfa.LFA_ERR_INVALID_ARG),
+    (dict(T=65), lfa.LFA_ERR_INVALID_ARG),
+    (dict(B=0), lfa.LFA_ERR_INVALID_ARG),
+    (dict(r=0), lfa.LFA_ERR_INVALID_ARG),
+    (dict(whiten=2), lfa.LFA_ERR_INVALID_ARG),
+    (dict(d=48), lfa.LFA_ERR_UNSUPPORTED),
+    (dict(d=128), lfa.LFA_ERR_UNSUPPORTED),
+    (dict(dtype=7), lfa.LFA_ERR_UNSUPPORTED),
+    (dict(H=64, W=68, r=4), lfa.LFA_ERR_UNSUPPORTED),   # m = 272 > 256
+])
+def test_create_rejects_bad_configs(lib, kw, expect):
+    cfg = _cfg(**kw)
+    assert lfa.workspace_size(cfg) == 0
+    h = ctypes.c_void_p()
+    st = lib.lfa_create(ctypes.byref(cfg), 256, 256, 1 << 20, ctypes.byref(h))
+    assert st == expect
+    assert not h.value
+
+
+def test_create_rejects_null_and_misaligned(lib):
+    cfg = _cfg()
+    h = ctypes.c_void_p()
+    n = lfa.workspace_size(cfg)
+    assert lib.lfa_create(ctypes.byref(cfg), None, 256, n, ctypes.byref(h)) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_create(ctypes.byref(cfg), 256, None, n, ctypes.byref(h)) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_create(ctypes.byref(cfg), 256, 256 + 16, n, ctypes.byref(h)) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_create(ctypes.byref(cfg), 256 + 4, 256, n, ctypes.byref(h)) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_create(ctypes.byref(cfg), 256, 256, n - 1, ctypes.byref(h)) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_create(ctypes.byref(cfg), 256, 256, n, None) == lfa.LFA_ERR_INVALID_ARG
+
+
+def test_null_handle_calls(lib):
+    assert lib.lfa_forward(None, 16, 16, 16, None) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_backward(None, 16, 16, 16, 16, 16, None) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_destroy(None) == lfa.LFA_ERR_INVALID_ARG
+    assert lib.lfa_forward_path(None) == b"invalid"
+
+
+def test_workspace_is_linear_in_nothing_but_partials(lib):
+    # workspace does not hold an N x m matrix: doubling N at fixed m grows it far less than N*m*4 bytes
+    a = lfa.workspace_size(_cfg(H=64, W=64, r=16, d=64))
+    b = lfa.workspace_size(_cfg(H=128, W=128, r=32, d=64))
+    assert b - a < 4 * 128 * 128 * 16
