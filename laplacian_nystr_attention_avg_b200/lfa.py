@@ -158,6 +158,9 @@ class LaplacianNystromAttention:
 
     def set_profile_events(self, begin=None, end=None) -> None:
         """Bracket the dominant kernel of later forwards with two torch.cuda.Event objects."""
+        for ev in (begin, end):
+            if ev is not None and not ev.cuda_event:
+                ev.record()          # torch creates the CUDA event lazily, on first record
         b = None if begin is None else begin.cuda_event
         e = None if end is None else end.cuda_event
         _check(self.lib.lfa_set_profile_events(self.handle, b, e), "lfa_set_profile_events")

@@ -39,10 +39,19 @@ def c_error(Cg: np.ndarray, Co: np.ndarray) -> float:
 
 
 def o_error(Og: np.ndarray, Oo: np.ndarray, bf16: bool) -> float:
-    """Per-unit error, worst over units: Og, Oo are [U, N, d]."""
+    """Per-unit error, worst over units: Og, Oo are [U, N, d].
+
+    A unit whose exact output lies entirely below the fp32 normal range (possible
+    only when every C entry underflows, e.g. lambda = 0.25 without whitening) is
+    compared absolutely: the fp32 result must be below 2^-126 as well.
+    """
     worst = 0.0
     for u in range(Oo.shape[0]):
         a, b = Og[u].astype(np.float64), Oo[u]
+        if np.max(np.abs(b)) < TINY:
+            if np.max(np.abs(a)) > TINY:
+                return float("inf")
+            continue
         if bf16:
             e = np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
         else:
