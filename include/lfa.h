@@ -117,7 +117,9 @@ lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* 
 
 /* Copy per-unit diagnostics of the last forward into host_out[0..n_units-1]
  * (n_units must equal B * heads) and return the device status word
- * (LFA_OK, LFA_ERR_TIMEOUT or LFA_ERR_NONFINITE). Synchronises `stream`. */
+ * (LFA_OK, LFA_ERR_TIMEOUT or LFA_ERR_NONFINITE). Synchronises `stream`. After a
+ * timeout the outputs of that call are invalid; the handle resets its cross-CTA flags
+ * on the next forward. */
 lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void* stream);
 
 /* Release the handle (host memory only; device memory stays the caller's). */
@@ -139,6 +141,15 @@ lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* 
 lfa_status lfa_debug_context(lfa_handle h, int unit, float* L_out, float* X_out, float* mu_out,
                              float* s_out, void* stream);
 
+/* Self-test of the tensor-core and TMA building blocks of the fused forward pass (no
+ * handle needed). modes 0, 1, 3, 5, 7 run one tcgen05 product on fp32 inputs A, B (device, row-major;
+ * shapes documented beside each mode in the library source) and write the fp32 result to D
+ * (device, [128][64]); mode 4 loads 128 rows of the bf16 [tma_rows][64] device tensor
+ * tma_src starting at row `param` through TMA and writes them to D as fp32 (rows outside
+ * the tensor read as zero). status: device int, set non-zero if a bounded wait expired. */
+lfa_status lfa_debug_selftest(int mode, const float* A, const float* B, float* D, int param,
+                              const void* tma_src, int tma_rows, int* status, void* stream);
+
 /* Benchmark timing hook: with non-NULL ev_begin / ev_end (each a cudaEvent_t created by
  * the caller), every later lfa_forward on this handle records ev_begin on its stream
  * immediately before launching the forward's dominant kernel and ev_end immediately after
@@ -152,8 +163,10 @@ const char* lfa_dominant_kernel(lfa_handle h);
 /* Number of kernels one lfa_forward launches for this handle's config (0 if h is NULL). */
 int lfa_launches_per_forward(lfa_handle h);
 
-/* Name of the forward implementation chosen for this handle's config
- * ("fused" or "generic"), static string. */
+/* Name of the forward implementation chosen for this handle's config, static string:
+ * "fused" (one cooperative kernel: bf16, d = 64, m <= 63, B*heads <= SMs/2, rows per CTA
+ * within its on-chip C capacity) or "generic" (every other accepted shape). Setting the
+ * environment variable LFA_FORWARD_PATH=generic before lfa_create forces the generic path. */
 const char* lfa_forward_path(lfa_handle h);
 
 #ifdef __cplusplus

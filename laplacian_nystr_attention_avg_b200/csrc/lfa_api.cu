@@ -22,6 +22,8 @@ struct lfa_ctx {
   const void* last_V;
   int have_forward;
   int path;   // 0 = generic, 1 = fused
+  int grid;   // CTAs of the fused kernel
+  unsigned long long epoch;   // forward calls issued (the fused kernel's flag generation)
 };
 
 namespace {
@@ -97,7 +99,8 @@ void plan(const lfa_config* c, Params* p, Layout* L) {
   L->M = take(sizeof(float) * U * m * d);
   L->Mp = take(sizeof(float) * U * m * d);
   L->bpart = take(sizeof(float) * U * p->n_chunks * d);
-  L->fused = take(0);
+  const bool fusable = c->dtype == LFA_BF16 && c->d == 64 && p->m <= 63;
+  L->fused = take(fusable ? lfa::fused_workspace_bytes(p->U) : 0);
   L->bwd = take(0);
   L->total = off;
 }
@@ -189,6 +192,13 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
   bind(&h->p, h->lay, h->ws);
   h->p.dwc = dwc_weight;
   h->path = 0;
+  const char* force = getenv("LFA_FORWARD_PATH");
+  const bool want_generic = force && strcmp(force, "generic") == 0;
+  if (!want_generic && h->lay.fused != h->lay.bwd) {
+    h->grid = lfa::fused_grid(h->p);
+    if (h->grid > 0) h->path = 1;
+  }
+  cudaGetLastError();   // an ineligible probe must not leave a sticky error behind
   *out = h;
   return LFA_OK;
 }
@@ -207,7 +217,13 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
   p.V = V;
   p.O = O;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (lfa::launch_generic_forward(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (h->path == 1) {
+    const unsigned long long epoch = h->epoch + 1;
+    if (lfa::launch_fused_forward(p, h->grid, h->ws + h->lay.fused, epoch, st) != cudaSuccess) return LFA_ERR_CUDA;
+    h->epoch = epoch;
+  } else {
+    if (lfa::launch_generic_forward(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  }
   h->last_Q = Q;
   h->last_V = V;
   h->have_forward = 1;
@@ -256,7 +272,10 @@ lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void
       host_out[u].alpha_fallback = f[lfa::kInfoFallback] != 0.f;
       host_out[u].ns_residual_fro = f[lfa::kInfoResidual];
     }
-    if (status & lfa::kStatusTimeout) ret = LFA_ERR_TIMEOUT;
+    if (status & lfa::kStatusTimeout) {
+      ret = LFA_ERR_TIMEOUT;
+      h->epoch = 0;   // flags may be inconsistent: the next fused forward re-zeroes them
+    }
     else if (status & lfa::kStatusNonFinite) ret = LFA_ERR_NONFINITE;
   }
   free(tmp);
@@ -291,6 +310,19 @@ lfa_status lfa_debug_context(lfa_handle h, int unit, float* L_out, float* X_out,
   return LFA_OK;
 }
 
+lfa_status lfa_debug_selftest(int mode, const float* A, const float* B, float* D, int param,
+                              const void* tma_src, int tma_rows, int* status, void* stream) {
+  if (!(mode == 0 || mode == 1 || mode == 3 || mode == 4 || mode == 5 || mode == 7) || !D || !status)
+    return LFA_ERR_INVALID_ARG;
+  if (mode != 4 && (!A || !B)) return LFA_ERR_INVALID_ARG;
+  if (mode == 3 && (param < 0 || param > 64 || param % 8 != 0)) return LFA_ERR_INVALID_ARG;
+  if (mode == 4 && (!tma_src || tma_rows < 1 || !aligned16(tma_src))) return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return lfa::launch_selftest(mode, A, B, D, param, tma_src, tma_rows, status, st) == cudaSuccess
+             ? LFA_OK
+             : LFA_ERR_CUDA;
+}
+
 lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end) {
   if (!h || ((ev_begin == nullptr) != (ev_end == nullptr))) return LFA_ERR_INVALID_ARG;
   h->p.ev_begin = ev_begin;
@@ -300,12 +332,12 @@ lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end) {
 
 const char* lfa_dominant_kernel(lfa_handle h) {
   if (!h) return "invalid";
-  return h->path == 1 ? "lfa_fused_forward" : "k_pass2";
+  return h->path == 1 ? "k_fused_forward" : "k_pass2";
 }
 
 int lfa_launches_per_forward(lfa_handle h) {
   if (!h) return 0;
-  return lfa::generic_launch_count(h->p);
+  return h->path == 1 ? 1 : lfa::generic_launch_count(h->p);
 }
 
 const char* lfa_forward_path(lfa_handle h) {

@@ -80,5 +80,11 @@ size_t generic_smem_pass1(int m, int d);
 size_t generic_smem_pass2(int m, int d);
 cudaError_t generic_set_attributes();
 int generic_launch_count(const Params& p);
+size_t fused_workspace_bytes(int U);
+int fused_grid(const Params& p);
+cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws, unsigned long long epoch,
+                                 cudaStream_t st);
+cudaError_t launch_selftest(int mode, const float* A, const float* B, float* D, int param, const void* tma_src,
+                            int tma_rows, int* status, cudaStream_t st);
 
 }  // namespace lfa

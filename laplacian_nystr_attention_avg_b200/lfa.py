@@ -61,6 +61,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_set_profile_events": (ci, [vp, vp, vp]),
         "lfa_dominant_kernel": (ctypes.c_char_p, [vp]),
         "lfa_launches_per_forward": (ci, [vp]),
+        "lfa_debug_selftest": (ci, [ci, vp, vp, vp, ci, vp, ci, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -87,6 +88,21 @@ def header_symbols() -> List[str]:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(lfa_[a-z_]+)\s*\(", text)))
+
+
+def selftest(mode: int, A: Optional[torch.Tensor], B: Optional[torch.Tensor], param: int = 0,
+             tma_src: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Run one tensor-core / TMA building-block self-test; returns D [128, 64] fp32 (device)."""
+    dev = (A if A is not None else tma_src).device
+    D = torch.zeros((128, 64), dtype=torch.float32, device=dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    rows = 0 if tma_src is None else tma_src.shape[0]
+    _check(load().lfa_debug_selftest(int(mode), _ptr(A), _ptr(B), _ptr(D), int(param), _ptr(tma_src), int(rows),
+                                     _ptr(status), _stream(None)), "lfa_debug_selftest")
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise LfaError(LFA_ERR_TIMEOUT, "lfa_debug_selftest")
+    return D
 
 
 def status_string(status: int) -> str:

@@ -170,3 +170,21 @@ def test_forward_host_buffers():
     mod.forward_host(Qh, Vh, Oh, Qd, Vd, Od)
     ref = mod.forward(x.Q_store.cuda(), x.V_store.cuda()).cpu()
     assert torch.equal(Oh, ref)
+
+
+@pytest.mark.parametrize("name", ["pvt1", "pvt2", "hr49"])
+def test_fused_and_generic_paths_agree(name, monkeypatch):
+    wl = pu.workload(name)
+    x = pu.inputs_for(wl)
+    fused = pu.gpu_module(wl, True, False)
+    monkeypatch.setenv("LFA_FORWARD_PATH", "generic")
+    generic = pu.gpu_module(wl, True, False)
+    monkeypatch.delenv("LFA_FORWARD_PATH")
+    assert fused.path == "fused" and generic.path == "generic"
+    Q, V = x.Q_store.cuda(), x.V_store.cuda()
+    a = pu.unit_rows(fused.forward(Q, V), range(wl.units))
+    b = pu.unit_rows(generic.forward(Q, V), range(wl.units))
+    assert pu.o_error(a, b, True) <= 1e-2
+    # repeated calls reuse the cross-CTA flags (epochs) and give identical results
+    c = pu.unit_rows(fused.forward(Q, V), range(wl.units))
+    assert np.array_equal(a, c)
