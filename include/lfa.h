@@ -157,8 +157,17 @@ lfa_status lfa_debug_selftest(int mode, const float* A, const float* B, float* D
  * the hook off. Host-only; returns LFA_ERR_INVALID_ARG if exactly one event is NULL. */
 lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end);
 
+/* Diagnostic timeline of the fused kernel: with a non-NULL device buffer of
+ * grid * 16 uint64 entries, later forwards on this handle record %globaltimer (ns) stamps at
+ * phase boundaries of every CTA (slot 0 start, 1 pooled, 2 grid barrier passed, then per
+ * role; 15 end). NULL turns it off. Host-only. */
+lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf);
+
 /* Name of the kernel the timing hook brackets for this handle's config (static string). */
 const char* lfa_dominant_kernel(lfa_handle h);
+
+/* CTAs of the fused kernel for this handle (0 when the generic path serves it). */
+int lfa_fused_grid(lfa_handle h);
 
 /* Number of kernels one lfa_forward launches for this handle's config (0 if h is NULL). */
 int lfa_launches_per_forward(lfa_handle h);

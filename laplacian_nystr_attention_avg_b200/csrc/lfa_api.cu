@@ -330,10 +330,18 @@ lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end) {
   return LFA_OK;
 }
 
+lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf) {
+  if (!h) return LFA_ERR_INVALID_ARG;
+  h->p.trace = dev_buf;
+  return LFA_OK;
+}
+
 const char* lfa_dominant_kernel(lfa_handle h) {
   if (!h) return "invalid";
   return h->path == 1 ? "k_fused_forward" : "k_pass2";
 }
+
+int lfa_fused_grid(lfa_handle h) { return h ? h->grid : 0; }
 
 int lfa_launches_per_forward(lfa_handle h) {
   if (!h) return 0;

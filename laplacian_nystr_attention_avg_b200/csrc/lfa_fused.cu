@@ -37,7 +37,7 @@ constexpr int kMaxChunks = 8;             // resident C chunks per row CTA
 constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q and L tiles
 constexpr int kRec = 128 + 64 * 64;       // floats per partial record: S1[64], S2[64], P[64][64]
 constexpr int kMaxGrid = 256;             // records are sized for up to this many CTAs
-constexpr int kPowerIters = 16;
+constexpr int kPowerIters = 8;
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kOffC = 0;                                   // 8 x 16 KB C chunks (SW128 rows)
@@ -48,17 +48,21 @@ constexpr uint32_t kOffMp = kOffL + 64 * kQS * 4;               // M'^T bf16 [64
 constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [64]
 constexpr uint32_t kOffWd = kOffBv + 256;                       // DWC weights fp32 [9][64]
 constexpr uint32_t kOffBar = kOffWd + 9 * 64 * 4;               // mbarriers + TMEM address
-constexpr uint32_t kSmemBytes = kOffBar + 128;
+constexpr uint32_t kOffCt = kOffBar + 128;                       // int [32] record offsets
+constexpr uint32_t kSmemBytes = kOffCt + 128;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
-// combine scratch (aliases V/Q/L, free once pass 1 is done)
-constexpr uint32_t kOffAs = kOffV;                              // fp32 [64][65]
-constexpr uint32_t kOffXs = kOffAs + 64 * 65 * 4;               // fp32 [64][65]
-constexpr uint32_t kOffS1 = kOffXs + 64 * 65 * 4;               // double [64]
+// combine scratch (aliases V/Q/L, free once pass 1 is done); then the pass-2 V halo tile
+constexpr uint32_t kOffAs = kOffV;                              // fp32 [64][68]  A (row l, col k)
+constexpr uint32_t kOffXt = kOffAs + 64 * kQS * 4;              // fp32 [64][68]  X^T (row l, col j)
+constexpr uint32_t kOffS1 = kOffXt + 64 * kQS * 4;              // double [64]
 constexpr uint32_t kOffS2 = kOffS1 + 512;                       // double [64]
 constexpr uint32_t kOffMu = kOffS2 + 512;                       // float [64]
 constexpr uint32_t kOffSc = kOffMu + 256;                       // float [64]
 constexpr uint32_t kOffSv = kOffSc + 256;                       // float [64]
-constexpr uint32_t kOffBp = kOffSv + 256;                       // float [4][64]
+constexpr uint32_t kOffBp = kOffSv + 256;                       // float [16][64]
+constexpr uint32_t kOffHalo = kOffV;                            // V halo rows: fp32 [rows][68] or bf16 [rows][72]
+constexpr uint32_t kHaloBytes = kOffMp - kOffHalo;
+constexpr int kHaloItems = 12;                                  // 16-byte halo loads per thread
 // solver scratch (aliases the C region: solver CTAs hold no C)
 constexpr uint32_t kOffNsHi = 0;                                // tf32 hi [2 K-halves][128 rows][128 B]
 constexpr uint32_t kOffNsLo = 32768;                            // tf32 lo
@@ -68,7 +72,7 @@ constexpr uint32_t kOffNsL = kOffNsX + 64 * kQS * 4;            // fp32 [64][68]
 constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [64] x 2, red [64]
 
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
-static_assert(kOffBp + 1024 <= kOffMp, "combine scratch overlaps M'");
+static_assert(kOffBp + 16 * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -86,6 +90,14 @@ struct FusedArgs {
   unsigned long long* xready; // [U] X published (holds the epoch)
   float* rec;                 // [n1][2][kRec]
 };
+
+__device__ __forceinline__ void trace_mark(const Params& p, int slot) {
+  if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 16 + slot] = globaltimer();
+}
+
+__device__ __forceinline__ void trace_clock(const Params& p, int slot) {
+  if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 16 + slot] = (unsigned long long)clock64();
+}
 
 __device__ __forceinline__ int row_cta(long long R, int n1, long long T) {
   return (int)(((R + 1) * n1 + T - 1) / T) - 1;
@@ -112,6 +124,22 @@ __device__ __forceinline__ void block_reduce2(float& a, float& b, float* red) {
   for (int i = 0; i < kFT / 32; ++i) {
     a += red[i];
     b += red[8 + i];
+  }
+}
+
+// L [m][64] fp32 (global, written by other CTAs of this launch) -> [64][kQS] shared, zero rows >= m.
+// 1024 float4 per CTA, 4 per thread, all loads issued before the stores.
+__device__ __forceinline__ void load_landmarks(const float* Lg, float* Ls, int m) {
+  float4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e4 = threadIdx.x + kFT * i, r = e4 >> 4;
+    v[i] = r < m ? __ldcg(reinterpret_cast<const float4*>(Lg) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e4 = threadIdx.x + kFT * i;
+    *reinterpret_cast<float4*>(Ls + (e4 >> 4) * kQS + 4 * (e4 & 15)) = v[i];
   }
 }
 
@@ -142,16 +170,17 @@ __device__ void ns_store(unsigned char* base, int r, int h, const float* v) {
 __device__ void ns_issue(uint32_t sbase, uint32_t tmem, uint64_t* bar) {
   tc_fence_after();
   const uint32_t id = idesc(2, 128, 64, 0, 0);
-  const uint32_t hi = sbase + kOffNsHi, lo = sbase + kOffNsLo;
+  // descriptors of the 1024-aligned bases; a K step adds its byte offset / 16 to the address field
+  const uint64_t dhi = desc_sw128(sbase + kOffNsHi, 16, 1024), dlo = desc_sw128(sbase + kOffNsLo, 16, 1024);
+  const uint64_t bofs = 8192 >> 4;
 #pragma unroll
   for (int g = 0; g < 3; ++g) {
-    const uint32_t ab = (g == 2) ? lo : hi;
-    const uint32_t bb = (g == 1) ? lo : hi;
+    const uint64_t ab = (g == 2) ? dlo : dhi;
+    const uint64_t bb = ((g == 1) ? dlo : dhi) + bofs;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-      mma_tf32(tmem, desc_sw128(ab + koff, 16, 1024), desc_sw128(bb + 8192 + koff, 16, 1024), id,
-               (g > 0 || ks > 0) ? 1u : 0u);
+      const uint64_t koff = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+      mma_tf32(tmem, ab + koff, bb + koff, id, (g > 0 || ks > 0) ? 1u : 0u);
     }
   }
   mma_commit(bar);
@@ -166,10 +195,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   float* Xsm = reinterpret_cast<float*>(sm + kOffNsX);
   float* vec = reinterpret_cast<float*>(sm + kOffNsVec);
   float* red = vec + 128;
-  for (int e = t; e < 64 * 64; e += kFT) {
-    const int r = e >> 6, c = e & 63;
-    Ls[r * kQS + c] = r < m ? __ldcg(p.L + ((size_t)u * m + r) * 64 + c) : 0.f;
-  }
+  load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
   __syncthreads();
   for (int e = t; e < 64 * 64; e += kFT) {
     const int a = e >> 6, b = e & 63;
@@ -191,6 +217,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   }
   if (t < 64) vec[t] = t < m ? rsqrtf((float)m) : 0.f;
   __syncthreads();
+  trace_mark(p, 5);
   // ||W||_2 = lambda_max (W symmetric positive definite): power iteration, 4 threads per row
   float lmax = 0.f;
   {
@@ -219,6 +246,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   const float alpha_p = 2.f / lmax;
   const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
   const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
+  trace_mark(p, 3);
 
   const int q = w & 3, h = w >> 2;
   const int r = 32 * q + lane;         // stacked row 0..127
@@ -233,11 +261,17 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (round == 5) trace_mark(p, 8);
     if (t == 0) ns_issue(sbase, tmem, bar);
+    if (round == 5) trace_mark(p, 9);
     __syncwarp();
     mbar_wait(bar, round & 1, p.status, kStatusTimeout);
+    if (round == 5) trace_mark(p, 10);
     tc_fence_after();
     tmem_ld32(trow, d);
+    if (round == 5) trace_mark(p, 11);
+    if (round == 0) trace_mark(p, 6);
+    if (round == 10) trace_mark(p, 7);
     ++round;
   };
   auto clean = [&](float* v) {
@@ -332,6 +366,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     __threadfence();
     st_release_u64(fa.xready + u, fa.epoch);
   }
+  trace_mark(p, 4);
   // diagnostics: ||I - W X_T||_F
   stage_w_over_x();
   run_round();
@@ -459,6 +494,8 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   const int g = blockIdx.x;
   const int U = p.U, N = p.N, m = p.m;
 
+  trace_mark(p, 0);
+  trace_clock(p, 13);
   if (w == 0) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
@@ -470,35 +507,57 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   }
   if (t == 32) tma_prefetch_desc(&tmapV);
 
-  // ---- phase 0: landmark pooling, one warp per landmark, 2 channels per lane ----
+  // ---- phase 0: landmark pooling, one warp per landmark ----
+  // lane = (token group tg = lane / 8, 8 channels c8 = lane % 8); each load instruction of the
+  // warp covers 4 window tokens x 128 bytes, all loads of a window are issued before use.
   {
     const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(p.Q);
-    const int total = U * m, Wr = p.W / p.r;
-    const float inv = 1.f / (float)(p.r * p.r);
+    const int total = U * m, Wr = p.W / p.r, rr = p.r * p.r;
+    const float inv = 1.f / (float)rr;
+    const int tg = lane >> 3, c8 = lane & 7;
     for (int gl = g * (kFT / 32) + w; gl < total; gl += gridDim.x * (kFT / 32)) {
       const int u = gl / m, l = gl % m;
       const int y0 = (l / Wr) * p.r, x0 = (l % Wr) * p.r;
-      const __nv_bfloat16* base = Q + ((size_t)u * N) * 64 + 2 * lane;
-      float a0 = 0.f, a1 = 0.f;
-      for (int dy = 0; dy < p.r; ++dy) {
-        const __nv_bfloat16* rowp = base + ((size_t)(y0 + dy) * p.W + x0) * 64;
-#pragma unroll 4
-        for (int dx = 0; dx < p.r; ++dx) {
-          const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(rowp + (size_t)dx * 64));
-          a0 += bf_lo(v);
-          a1 += bf_hi(v);
+      const __nv_bfloat16* base = Q + ((size_t)u * N) * 64 + 8 * c8;
+      float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int k0 = 0; k0 < rr; k0 += 64) {
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int k = k0 + tg + 4 * i;
+          v[i] = make_uint4(0u, 0u, 0u, 0u);
+          if (k < rr) {
+            const int dy = k / p.r, dx = k % p.r;
+            v[i] = __ldg(reinterpret_cast<const uint4*>(base + ((size_t)(y0 + dy) * p.W + x0 + dx) * 64));
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          a[0] += bf_lo(v[i].x); a[1] += bf_hi(v[i].x); a[2] += bf_lo(v[i].y); a[3] += bf_hi(v[i].y);
+          a[4] += bf_lo(v[i].z); a[5] += bf_hi(v[i].z); a[6] += bf_lo(v[i].w); a[7] += bf_hi(v[i].w);
         }
       }
-      *reinterpret_cast<float2*>(p.L + ((size_t)u * m + l) * 64 + 2 * lane) = make_float2(a0 * inv, a1 * inv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        a[e] += __shfl_xor_sync(0xffffffffu, a[e], 8);
+        a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+      }
+      if (tg == 0) {
+        float* dst = p.L + ((size_t)u * m + l) * 64 + 8 * c8;
+        *reinterpret_cast<float4*>(dst) = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
+      }
     }
   }
   __syncthreads();
+  trace_mark(p, 1);
   if (t == 0) {
     __threadfence();
     red_release_add_u64(fa.gbar, 1ull);
     spin_until_geq(fa.gbar, fa.epoch * (unsigned long long)gridDim.x, p.status, kStatusTimeout);
   }
   __syncthreads();
+  trace_mark(p, 2);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -569,10 +628,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
       unsigned char* cslot = sm + kOffC + gc * 16384;
       __syncthreads();     // previous chunk's readers of Qs / Ls are done
       if (seg_first) {
-        for (int e = t; e < 64 * 64; e += kFT) {
-          const int r = e >> 6, c = e & 63;
-          Ls[r * kQS + c] = r < m ? __ldcg(p.L + ((size_t)u * m + r) * 64 + c) : 0.f;
-        }
+        load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
           s1[b] = 0.f;
@@ -597,10 +653,12 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
           issue_v(gc + 1);
         }
       }
+      if (gc == 0) trace_mark(p, 10);
       if (lt > 0) cross_dispatch(lt, Qs, Ls, cslot, j0, nrows, scale, s1, s2);
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
+      if (gc < 2) trace_mark(p, 11 + gc);
       if (t == 0) {
         mbar_wait(bars + kBarV + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
         tc_fence_after();
@@ -655,9 +713,10 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
       }
     }
 
+    trace_mark(p, 3);
     // ---- phases 2 + 3 per segment ----
     float* As = reinterpret_cast<float*>(sm + kOffAs);
-    float* Xs = reinterpret_cast<float*>(sm + kOffXs);
+    float* Xt = reinterpret_cast<float*>(sm + kOffXt);
     double* S1d = reinterpret_cast<double*>(sm + kOffS1);
     double* S2d = reinterpret_cast<double*>(sm + kOffS2);
     float* mus = reinterpret_cast<float*>(sm + kOffMu);
@@ -666,31 +725,101 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     float* bps = reinterpret_cast<float*>(sm + kOffBp);
     float* bvec = reinterpret_cast<float*>(sm + kOffBv);
     float* wd = reinterpret_cast<float*>(sm + kOffWd);
+    int* ctr = reinterpret_cast<int*>(sm + kOffCt);
+    const float invNf = 1.f / (float)N;
     const double invN = 1.0 / (double)N;
+    const bool halo_f32 = (kChunk + 2 * p.W + 2) * kQS * 4 <= (int)kHaloBytes;
     int pc = 0;    // pass-2 chunk counter (accumulator buffer parity)
     for (int s = 0; s < nseg; ++s) {
       const int u = seg[s].u;
+      const __nv_bfloat16* Vu = static_cast<const __nv_bfloat16*>(p.V) + (size_t)u * N * 64;
+      __nv_bfloat16* Ou = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * N * 64;
+      // V rows needed by chunk c's 3x3 stencil: [hlo, hhi) of unit u
+      auto halo_range = [&](int c, int& hlo, int& hhi) {
+        const int lo = seg[s].lo + c * kChunk, nr = min(kChunk, seg[s].hi - lo);
+        hlo = max(0, lo - p.W - 1);
+        hhi = min(N, lo + nr + p.W + 1);
+      };
+      uint4 hv[kHaloItems];
+      auto halo_fetch = [&](int c) {
+        int hlo, hhi;
+        halo_range(c, hlo, hhi);
+        const int n16 = (hhi - hlo) * 8;
+        const uint4* src = reinterpret_cast<const uint4*>(Vu + (size_t)hlo * 64);
+#pragma unroll
+        for (int i = 0; i < kHaloItems; ++i) {
+          const int e = t + kFT * i;
+          hv[i] = e < n16 ? __ldg(src + e) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      };
+      auto halo_store = [&](int c) {
+        int hlo, hhi;
+        halo_range(c, hlo, hhi);
+        const int n16 = (hhi - hlo) * 8;
+#pragma unroll
+        for (int i = 0; i < kHaloItems; ++i) {
+          const int e = t + kFT * i;
+          if (e < n16) {
+            const int row = e >> 3, c8 = e & 7;
+            if (halo_f32) {
+              float* dst = reinterpret_cast<float*>(sm + kOffHalo) + row * kQS + 8 * c8;
+              *reinterpret_cast<float4*>(dst) =
+                  make_float4(bf_lo(hv[i].x), bf_hi(hv[i].x), bf_lo(hv[i].y), bf_hi(hv[i].y));
+              *reinterpret_cast<float4*>(dst + 4) =
+                  make_float4(bf_lo(hv[i].z), bf_hi(hv[i].z), bf_lo(hv[i].w), bf_hi(hv[i].w));
+            } else {
+              *reinterpret_cast<uint4*>(sm + kOffHalo + row * 144 + 16 * c8) = hv[i];
+            }
+          }
+        }
+      };
+      halo_fetch(0);
+
       const int jf = row_cta((long long)u * N, n1, Trows);
       const int jl = row_cta((long long)(u + 1) * N - 1, n1, Trows);
+      const int nct = jl - jf + 1;
       __syncthreads();
       if (t == 0) {
-        spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)(jl - jf + 1), p.status, kStatusTimeout);
+        spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout);
         spin_until_geq(fa.xready + u, fa.epoch, p.status, kStatusTimeout);
       }
-      __syncthreads();
-      for (int e = t; e < kRec; e += kFT) {
-        double acc = 0.0;
-        for (int jj = jf; jj <= jl; ++jj) {
-          const int sj = (row_start(jj, n1, Trows) / N == u) ? 0 : 1;
-          acc += (double)__ldcg(fa.rec + ((size_t)jj * 2 + sj) * kRec + e);
-        }
-        if (e < 64) S1d[e] = acc;
-        else if (e < 128) S2d[e - 64] = acc;
-        else As[((e - 128) >> 6) * 65 + ((e - 128) & 63)] = (float)acc;
+      if (t < nct && t < 32) {
+        const int jj = jf + t;
+        const int sj = row_start(jj, n1, Trows) < (long long)u * N ? 1 : 0;
+        ctr[t] = (jj * 2 + sj) * kRec;
       }
-      for (int e = t; e < 64 * 64; e += kFT) {
-        const int a = e >> 6, b = e & 63;
-        Xs[a * 65 + b] = (a < m && b < m) ? __ldcg(p.X + ((size_t)u * m + a) * m + b) : 0.f;
+      __syncthreads();
+      trace_mark(p, 4 + 3 * s);
+      // sum the unit's records: S1, S2 in fp64, P in fp32 (float4)
+      if (t < 128) {
+        double acc = 0.0;
+        for (int c = 0; c < nct; ++c) acc += (double)__ldcg(fa.rec + ctr[c] + t);
+        if (t < 64) S1d[t] = acc;
+        else S2d[t - 64] = acc;
+      }
+      for (int e4 = t; e4 < 1024; e4 += kFT) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c = 0; c < nct; ++c) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(fa.rec + ctr[c] + 128) + e4);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(As + (e4 >> 4) * kQS + 4 * (e4 & 15)) = acc;
+      }
+      for (int e0 = t; e0 < 64 * 64; e0 += 4 * kFT) {
+        float xv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = e0 + kFT * i, jr = e >> 6, l = e & 63;
+          xv[i] = (jr < m && l < m) ? __ldcg(p.X + ((size_t)u * m + jr) * m + l) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = e0 + kFT * i;
+          Xt[(e & 63) * kQS + (e >> 6)] = xv[i];
+        }
       }
       const int head = u % p.heads;
       for (int e = t; e < 9 * 64; e += kFT) {
@@ -705,7 +834,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
         const double sc = 1.0 / sqrt(var + (double)p.eps);
         mus[t] = t < m ? (float)mu : 0.f;
         scs[t] = t < m ? (float)sc : 0.f;
-        svs[t] = As[63 * 65 + t];       // landmark column 63 holds sum_i v_i
+        svs[t] = As[63 * kQS + t];       // landmark column 63 holds sum_i v_i
         if (j == jf && t < m) {
           p.mu[(size_t)u * m + t] = (float)mu;
           p.s[(size_t)u * m + t] = (float)sc;
@@ -716,41 +845,55 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
         const int a = e >> 6, k = e & 63;
         float v = 0.f;
         if (a < m) {
-          const float P = As[a * 65 + k];
-          v = p.whiten ? scs[a] * (P - mus[a] * svs[k]) + svs[k] * (float)invN : P;
+          const float P = As[a * kQS + k];
+          v = p.whiten ? scs[a] * (P - mus[a] * svs[k]) + svs[k] * invNf : P;
         }
-        As[a * 65 + k] = v;
+        As[a * kQS + k] = v;
       }
       __syncthreads();
       {
-        const int k = t & 63, jq = t >> 6;
-        float acc[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) acc[ii] = 0.f;
+        // M = X A with a 4 x 4 register tile per thread; M' = diag(s) M (bf16, K-major B of pass 2)
+        const int jb = t >> 4, kb = t & 15;
+        float acc[4][4] = {};
         for (int l = 0; l < m; ++l) {
-          const float a = As[l * 65 + k];
+          const float4 x4 = *reinterpret_cast<const float4*>(Xt + l * kQS + 4 * jb);
+          const float4 a4 = *reinterpret_cast<const float4*>(As + l * kQS + 4 * kb);
+          const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-          for (int ii = 0; ii < 16; ++ii) acc[ii] = fmaf(Xs[(jq + 4 * ii) * 65 + l], a, acc[ii]);
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(xv[x], av[y], acc[x][y]);
         }
-        float bp = 0.f;
         unsigned char* mp = sm + kOffMp;
+        float bp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          const int jr = jq + 4 * ii;
-          float v = 0.f;
-          if (jr < m) {
-            v = p.whiten ? scs[jr] * acc[ii] : acc[ii];
-            if (p.whiten) bp += ((float)invN - scs[jr] * mus[jr]) * acc[ii];
+        for (int x = 0; x < 4; ++x) {
+          const int jr = 4 * jb + x;
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const int k = 4 * kb + y;
+            float v = 0.f;
+            if (jr < m) {
+              v = p.whiten ? scs[jr] * acc[x][y] : acc[x][y];
+              if (p.whiten) bp[y] += (invNf - scs[jr] * mus[jr]) * acc[x][y];
+            }
+            *reinterpret_cast<__nv_bfloat16*>(mp + sw128(k, jr >> 3) + ((jr & 7) << 1)) = __float2bfloat16_rn(v);
           }
-          *reinterpret_cast<__nv_bfloat16*>(mp + sw128(k, jr >> 3) + ((jr & 7) << 1)) = __float2bfloat16_rn(v);
         }
-        bps[jq * 64 + k] = bp;
+#pragma unroll
+        for (int y = 0; y < 4; ++y) bps[jb * 64 + 4 * kb + y] = bp[y];
       }
       __syncthreads();
-      if (t < 64) bvec[t] = bps[t] + bps[64 + t] + bps[128 + t] + bps[192 + t];
+      if (t < 64) {
+        float b = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) b += bps[q * 64 + t];
+        bvec[t] = b;
+      }
       fence_async_smem();
       tc_fence_before();
       __syncthreads();
+      trace_mark(p, 5 + 3 * s);
 
       // phase 3: O = C M' + b + DWC(V)
       auto issue_o = [&](int gcc, int pcc) {
@@ -763,12 +906,17 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
           mma_bf16(dt, desc_sw128(ca + kk * 32, 16, 1024), desc_sw128(mb + kk * 32, 16, 1024), id, kk > 0 ? 1u : 0u);
         mma_commit(bars + kBarP2 + (pcc & 1));
       };
-      const __nv_bfloat16* Vu = static_cast<const __nv_bfloat16*>(p.V) + (size_t)u * N * 64;
-      __nv_bfloat16* Ou = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * N * 64;
       if (t == 0) issue_o(seg[s].first_chunk, pc);
       for (int c = 0; c < seg[s].nch; ++c) {
         const int gc = seg[s].first_chunk + c;
-        if (t == 0 && c + 1 < seg[s].nch) issue_o(gc + 1, pc + 1);
+        int hlo, hhi;
+        halo_range(c, hlo, hhi);
+        halo_store(c);
+        __syncthreads();
+        if (c + 1 < seg[s].nch) {
+          halo_fetch(c + 1);
+          if (t == 0) issue_o(gc + 1, pc + 1);
+        }
         __syncwarp();
         mbar_wait(bars + kBarP2 + (pc & 1), (pc >> 1) & 1, p.status, kStatusTimeout);
         tc_fence_after();
@@ -781,7 +929,13 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
         if (row < nrows) {
           const int n = lo + row, y = n / p.W, x = n % p.W;
 #pragma unroll
-          for (int cc = 0; cc < 32; ++cc) v[cc] += bvec[32 * h + cc];
+          for (int cc = 0; cc < 32; cc += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(bvec + 32 * h + cc);
+            v[cc] += b4.x;
+            v[cc + 1] += b4.y;
+            v[cc + 2] += b4.z;
+            v[cc + 3] += b4.w;
+          }
 #pragma unroll
           for (int a = 0; a < 3; ++a) {
             const int yy = y + a - 1;
@@ -790,16 +944,30 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
             for (int b = 0; b < 3; ++b) {
               const int xx = x + b - 1;
               if (xx < 0 || xx >= p.W) continue;
-              const uint4* src = reinterpret_cast<const uint4*>(Vu + ((size_t)yy * p.W + xx) * 64 + 32 * h);
+              const int hr = yy * p.W + xx - hlo;
               const float* wt = wd + (a * 3 + b) * 64 + 32 * h;
+              if (halo_f32) {
+                const float* vr = reinterpret_cast<const float*>(sm + kOffHalo) + hr * kQS + 32 * h;
 #pragma unroll
-              for (int k4 = 0; k4 < 4; ++k4) {
-                const uint4 vv = __ldg(src + k4);
-                const uint32_t wv[4] = {vv.x, vv.y, vv.z, vv.w};
+                for (int c4 = 0; c4 < 32; c4 += 4) {
+                  const float4 vv = *reinterpret_cast<const float4*>(vr + c4);
+                  const float4 ww = *reinterpret_cast<const float4*>(wt + c4);
+                  v[c4] = fmaf(ww.x, vv.x, v[c4]);
+                  v[c4 + 1] = fmaf(ww.y, vv.y, v[c4 + 1]);
+                  v[c4 + 2] = fmaf(ww.z, vv.z, v[c4 + 2]);
+                  v[c4 + 3] = fmaf(ww.w, vv.w, v[c4 + 3]);
+                }
+              } else {
+                const uint4* vr = reinterpret_cast<const uint4*>(sm + kOffHalo + hr * 144 + 64 * h);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  v[8 * k4 + 2 * e] = fmaf(wt[8 * k4 + 2 * e], bf_lo(wv[e]), v[8 * k4 + 2 * e]);
-                  v[8 * k4 + 2 * e + 1] = fmaf(wt[8 * k4 + 2 * e + 1], bf_hi(wv[e]), v[8 * k4 + 2 * e + 1]);
+                for (int k4 = 0; k4 < 4; ++k4) {
+                  const uint4 vv = vr[k4];
+                  const uint32_t wv[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    v[8 * k4 + 2 * e] = fmaf(wt[8 * k4 + 2 * e], bf_lo(wv[e]), v[8 * k4 + 2 * e]);
+                    v[8 * k4 + 2 * e + 1] = fmaf(wt[8 * k4 + 2 * e + 1], bf_hi(wv[e]), v[8 * k4 + 2 * e + 1]);
+                  }
                 }
               }
             }
@@ -820,8 +988,11 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
         __syncthreads();
         ++pc;
       }
+      trace_mark(p, 6 + 3 * s);
     }
   }
+  trace_mark(p, 15);
+  trace_clock(p, 14);
   __syncthreads();
   if (w == 0) {
     tc_fence_after();
@@ -849,10 +1020,12 @@ int fused_grid(const Params& p) {
   if (major != 10) return 0;
   const int G = sms < kMaxGrid ? sms : kMaxGrid;
   if (2 * p.U > G) return 0;
+  if ((kChunk + 2 * p.W + 2) * 8 > kHaloItems * kFT) return 0;   // V halo of one chunk fits the prefetch
   const int n1 = G - p.U;
   const long long T = (long long)p.U * p.N;
   const long long rpc = (T + n1 - 1) / n1;
   if (rpc > (long long)(kMaxChunks - 1) * kChunk || rpc > p.N) return 0;
+  if (p.N / (T / n1) + 2 > 32) return 0;     // contributors of one unit fit the offset table
   if (cudaFuncSetAttribute(k_fused_forward, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) !=
       cudaSuccess)
     return 0;

@@ -70,6 +70,8 @@ struct Params {
   // optional timing events bracketing the dominant kernel (cudaEvent_t or null)
   void* ev_begin;
   void* ev_end;
+  // optional per-CTA phase timestamps (%globaltimer, ns) of the fused kernel: [grid][16]
+  unsigned long long* trace;
 };
 
 // host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu

@@ -61,6 +61,8 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_set_profile_events": (ci, [vp, vp, vp]),
         "lfa_dominant_kernel": (ctypes.c_char_p, [vp]),
         "lfa_launches_per_forward": (ci, [vp]),
+        "lfa_debug_trace": (ci, [vp, vp]),
+        "lfa_fused_grid": (ci, [vp]),
         "lfa_debug_selftest": (ci, [ci, vp, vp, vp, ci, vp, ci, vp, vp]),
     }
     for name, (res, args) in sig.items():
@@ -180,6 +182,14 @@ class LaplacianNystromAttention:
         b = None if begin is None else begin.cuda_event
         e = None if end is None else end.cuda_event
         _check(self.lib.lfa_set_profile_events(self.handle, b, e), "lfa_set_profile_events")
+
+    @property
+    def fused_grid(self) -> int:
+        return int(self.lib.lfa_fused_grid(self.handle))
+
+    def set_trace(self, buf: Optional[torch.Tensor]) -> None:
+        """Record fused-kernel phase timestamps into buf (int64 [grid, 16], device) or stop (None)."""
+        _check(self.lib.lfa_debug_trace(self.handle, _ptr(buf)), "lfa_debug_trace")
 
     def new_output(self) -> torch.Tensor:
         return torch.empty(self.shape, dtype=self.dtype, device=self.device)
