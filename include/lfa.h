@@ -158,9 +158,9 @@ lfa_status lfa_debug_selftest(int mode, const float* A, const float* B, float* D
 lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end);
 
 /* Diagnostic timeline of the fused kernel: with a non-NULL device buffer of
- * grid * 16 uint64 entries, later forwards on this handle record %globaltimer (ns) stamps at
+ * grid * 32 uint64 entries, later forwards on this handle record %globaltimer (ns) stamps at
  * phase boundaries of every CTA (slot 0 start, 1 pooled, 2 grid barrier passed, then per
- * role; 15 end). NULL turns it off. Host-only. */
+ * role; 15 end; 13 / 14 the SM clock64 at start / end). NULL turns it off. Host-only. */
 lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf);
 
 /* Name of the kernel the timing hook brackets for this handle's config (static string). */

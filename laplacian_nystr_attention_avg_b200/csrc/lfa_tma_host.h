@@ -25,9 +25,10 @@ inline EncodeTiledFn encode_tiled_fn() {
 }
 
 // bf16 tensor [outer][rows][64] (contiguous, 128-byte rows) viewed as 3-D {64, rows, outer};
-// box {64, box_rows, 1}, 128-byte swizzle, out-of-range elements read as zero.
+// box {64, box_rows, 1}, 128-byte swizzle (or none: plain 128-byte rows), out-of-range elements read
+// as zero.
 inline bool make_tmap_rows_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t outer,
-                                uint32_t box_rows) {
+                                uint32_t box_rows, bool swizzle128 = true) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {64, rows, outer};
@@ -35,7 +36,8 @@ inline bool make_tmap_rows_bf16(CUtensorMap* map, const void* base, uint64_t row
   const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

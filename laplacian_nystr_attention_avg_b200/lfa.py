@@ -188,7 +188,7 @@ class LaplacianNystromAttention:
         return int(self.lib.lfa_fused_grid(self.handle))
 
     def set_trace(self, buf: Optional[torch.Tensor]) -> None:
-        """Record fused-kernel phase timestamps into buf (int64 [grid, 16], device) or stop (None)."""
+        """Record fused-kernel phase timestamps into buf (int64 [grid, 32], device) or stop (None)."""
         _check(self.lib.lfa_debug_trace(self.handle, _ptr(buf)), "lfa_debug_trace")
 
     def new_output(self) -> torch.Tensor:
