@@ -95,3 +95,13 @@ def test_workspace_is_linear_in_nothing_but_partials(lib):
     a = lfa.workspace_size(_cfg(H=64, W=64, r=16, d=64))
     b = lfa.workspace_size(_cfg(H=128, W=128, r=32, d=64))
     assert b - a < 4 * 128 * 128 * 16
+
+
+def test_library_needs_no_python_or_torch(lib):
+    # the dynamic section of the built library lists its shared-library dependencies
+    import subprocess
+    out = subprocess.run(["readelf", "-d", lfa.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    needed = [line.split("[")[1].split("]")[0] for line in out.splitlines() if "(NEEDED)" in line]
+    assert needed, out
+    for n in needed:
+        assert "python" not in n and "torch" not in n and "c10" not in n, n
