@@ -56,7 +56,8 @@ typedef enum {
   LFA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, copy, attribute) */
   LFA_ERR_STATE = 4,         /* backward without a matching forward on this handle */
   LFA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (reported by lfa_get_info) */
-  LFA_ERR_NONFINITE = 6      /* the landmark kernel or its norm was not finite */
+  LFA_ERR_NONFINITE = 6,     /* the landmark kernel or its norm was not finite */
+  LFA_ERR_SCRATCH_LIMIT = 7  /* lfa_forward_noalloc: cfg needs more than LFA_NOALLOC_SCRATCH_BYTES */
 } lfa_status;
 
 typedef enum { LFA_F32 = 0, LFA_BF16 = 1 } lfa_dtype;
@@ -98,6 +99,37 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
 /* Forward pass (see the file comment). Q, V: device inputs; O: device output, all
  * [B][heads][N][d] in cfg.dtype. Enqueued on `stream`. */
 lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void* stream);
+
+/* Size of the static device scratch area behind lfa_forward_noalloc (16 MiB). */
+#define LFA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* Forward pass without a handle and without allocating anything: the same result as
+ * lfa_forward (computed by the per-stage kernels that lfa_forward_path reports as
+ * "generic"), with the intermediate data in one static device array of
+ * LFA_NOALLOC_SCRATCH_BYTES inside the library instead of a caller workspace. This
+ * entry point is a deployment convenience with no counterpart in the method's
+ * description. It is meant for callers that may not allocate device memory: an
+ * operator inside a host framework that owns the device memory pool and gives it no
+ * allocator, or a latency-critical caller that cannot take the device-wide
+ * synchronisation of cudaMalloc / cudaFree.
+ *   cfg, dwc_weight, Q, V, O, stream: as for lfa_create and lfa_forward.
+ *   Setup: the first call on each device (with that device current) resolves the
+ *   address of the scratch array for that device; make that first call before any
+ *   stream capture begins. Later calls only validate and enqueue.
+ *   Zeroing: nothing has to start at zero. Every scratch byte a call reads is written
+ *   earlier by the same call; its status word is cleared by the call's first kernel.
+ *   Limit: the scratch a config needs grows with B*heads and m (about
+ *   B*heads*(16 m^2 + 24 m d + 4 P (m d + 2 m + d)) bytes with
+ *   P <= min(ceil(296 / (B*heads)), ceil(N / 64)) row partitions); a config that needs more than LFA_NOALLOC_SCRATCH_BYTES is
+ *   rejected with LFA_ERR_SCRATCH_LIMIT before any device work. B*heads = 32 on a
+ *   56 x 56 grid with m = 49, d = 64 needs about 7.6 MiB; B*heads = 8 on a 112 x 112
+ *   grid with m = 196 needs about 20 MiB and is rejected.
+ *   Concurrency: there is one scratch array per device, shared by every call on that
+ *   device. Calls that overlap on the GPU (two streams without ordering, or two host
+ *   threads) race on it and give wrong results; order them on one stream.
+ *   Diagnostics (lfa_get_info) are not available for these calls. */
+lfa_status lfa_forward_noalloc(const lfa_config* cfg, const float* dwc_weight, const void* Q,
+                               const void* V, void* O, void* stream);
 
 /* Forward pass from and to HOST buffers: copies Q, V (host, [B][heads][N][d] in
  * cfg.dtype; pinned memory gives asynchronous copies) into the caller's device

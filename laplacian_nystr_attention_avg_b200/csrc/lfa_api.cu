@@ -152,6 +152,7 @@ const char* lfa_status_string(lfa_status s) {
     case LFA_ERR_STATE: return "backward without a matching forward";
     case LFA_ERR_TIMEOUT: return "device wait timed out";
     case LFA_ERR_NONFINITE: return "non-finite landmark kernel";
+    case LFA_ERR_SCRATCH_LIMIT: return "configuration needs more scratch than the static no-alloc area holds";
   }
   return "unknown status";
 }
@@ -228,6 +229,61 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
   h->last_V = V;
   h->have_forward = 1;
   return LFA_OK;
+}
+
+}  // extern "C"
+
+// Static scratch of lfa_forward_noalloc: one array per device, placed by module load.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LFA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+unsigned char* g_noalloc_ptr[kNoAllocMaxDevices];   // device address of the array, per device
+
+// Address of the scratch array on the current device, resolved once per device.
+lfa_status noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LFA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return LFA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LFA_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<unsigned char*>(ptr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return LFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+lfa_status lfa_forward_noalloc(const lfa_config* cfg, const float* dwc_weight, const void* Q,
+                               const void* V, void* O, void* stream) {
+  lfa_status st = validate(cfg);
+  if (st != LFA_OK) return st;
+  if (!dwc_weight || !Q || !V || !O) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(dwc_weight) || !aligned16(Q) || !aligned16(V) || !aligned16(O)) return LFA_ERR_INVALID_ARG;
+  Params p;
+  Layout lay;
+  plan(cfg, &p, &lay);
+  // the per-stage kernels use the layout up to the fused kernel's area
+  if (lay.fused > (size_t)LFA_NOALLOC_SCRATCH_BYTES) return LFA_ERR_SCRATCH_LIMIT;
+  st = ensure_attributes();
+  if (st != LFA_OK) return st;
+  unsigned char* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != LFA_OK) return st;
+  bind(&p, lay, ws);
+  p.dwc = dwc_weight;
+  p.Q = Q;
+  p.V = V;
+  p.O = O;
+  return lfa::launch_generic_forward(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LFA_OK
+                                                                                           : LFA_ERR_CUDA;
 }
 
 lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,

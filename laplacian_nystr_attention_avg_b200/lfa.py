@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(_PKG, "liblfa.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "lfa.h")
 
 LFA_OK, LFA_ERR_INVALID_ARG, LFA_ERR_UNSUPPORTED, LFA_ERR_CUDA, LFA_ERR_STATE, \
-    LFA_ERR_TIMEOUT, LFA_ERR_NONFINITE = range(7)
+    LFA_ERR_TIMEOUT, LFA_ERR_NONFINITE, LFA_ERR_SCRATCH_LIMIT = range(8)
+LFA_NOALLOC_SCRATCH_BYTES = 16 << 20
 LFA_F32, LFA_BF16 = 0, 1
 
 
@@ -51,6 +52,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_create": (ci, [cfgp, vp, vp, sz, ctypes.POINTER(vp)]),
         "lfa_forward": (ci, [vp, vp, vp, vp, vp]),
         "lfa_forward_host": (ci, [vp, vp, vp, vp, vp, vp, vp, vp]),
+        "lfa_forward_noalloc": (ci, [cfgp, vp, vp, vp, vp, vp]),
         "lfa_backward": (ci, [vp, vp, vp, vp, vp, vp, vp]),
         "lfa_get_info": (ci, [vp, ctypes.POINTER(UnitInfo), ci, vp]),
         "lfa_destroy": (ci, [vp]),
@@ -124,6 +126,18 @@ def make_config(wl, whiten: bool = True) -> Config:
 
 def workspace_size(cfg: Config) -> int:
     return int(load().lfa_workspace_size(ctypes.byref(cfg)))
+
+
+def forward_noalloc(cfg: Config, dwc_weight: torch.Tensor, Q: torch.Tensor, V: torch.Tensor,
+                    O: torch.Tensor, stream=None) -> torch.Tensor:
+    """lfa_forward_noalloc: handle-free forward over the library's static scratch area.
+
+    dwc_weight: device float32 [heads, d, 3, 3]; Q, V, O: device [B, heads, N, d] in the
+    config's dtype. Raises LfaError (LFA_ERR_SCRATCH_LIMIT) when the config does not fit.
+    """
+    _check(load().lfa_forward_noalloc(ctypes.byref(cfg), _ptr(dwc_weight), _ptr(Q), _ptr(V), _ptr(O),
+                                      _stream(stream)), "lfa_forward_noalloc")
+    return O
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
