@@ -101,7 +101,28 @@ void plan(const lfa_config* c, Params* p, Layout* L) {
   L->bpart = take(sizeof(float) * U * p->n_chunks * d);
   const bool fusable = c->dtype == LFA_BF16 && c->d == 64 && p->m <= 63;
   L->fused = take(fusable ? lfa::fused_workspace_bytes(p->U) : 0);
-  L->bwd = take(0);
+  // backward: Newton-Schulz iterates and reverse-step matrices, partials, dQ in fp32
+  const size_t mm = m * m, T = p->T > 0 ? p->T : 1;
+  L->bwd = off;
+  L->b_its = take(sizeof(float) * U * T * mm);
+  L->b_G = take(sizeof(float) * U * mm);
+  L->b_Gn = take(sizeof(float) * U * mm);
+  L->b_T1 = take(sizeof(float) * U * mm);
+  L->b_T2 = take(sizeof(float) * U * mm);
+  L->b_T3 = take(sizeof(float) * U * mm);
+  L->b_dW = take(sizeof(float) * U * mm);
+  L->b_part2 = take(sizeof(float) * U * p->P * p->part_stride);
+  L->b_red2 = take(sizeof(double) * U * p->part_stride);
+  L->b_dA = take(sizeof(float) * U * m * d);
+  L->b_Gm = take(sizeof(float) * U * m * d);
+  L->b_Gd = take(sizeof(float) * U * m * d);
+  L->b_beta = take(sizeof(float) * U * m);
+  L->b_gamma = take(sizeof(float) * U * m);
+  L->b_bpart2 = take(sizeof(float) * U * p->n_chunks * d);
+  L->b_dLpart = take(sizeof(float) * U * p->P * m * d);
+  L->b_dLns = take(sizeof(float) * U * m * d);
+  L->b_dLpool = take(sizeof(float) * U * m * d);
+  L->b_dQd = take(sizeof(float) * U * (size_t)p->N * d);
   L->total = off;
 }
 
@@ -123,6 +144,31 @@ void bind(Params* p, const Layout& L, unsigned char* ws) {
   p->bpart = reinterpret_cast<float*>(ws + L.bpart);
 }
 
+void bind_backward(lfa::BwdParams* b, const Params& p, const Layout& L, unsigned char* ws) {
+  memset(b, 0, sizeof(*b));
+  b->p = p;
+  auto f = [&](size_t off) { return reinterpret_cast<float*>(ws + off); };
+  b->its = f(L.b_its);
+  b->G = f(L.b_G);
+  b->Gn = f(L.b_Gn);
+  b->T1 = f(L.b_T1);
+  b->T2 = f(L.b_T2);
+  b->T3 = f(L.b_T3);
+  b->dW = f(L.b_dW);
+  b->part2 = f(L.b_part2);
+  b->red2 = reinterpret_cast<double*>(ws + L.b_red2);
+  b->dA = f(L.b_dA);
+  b->Gm = f(L.b_Gm);
+  b->Gd = f(L.b_Gd);
+  b->beta = f(L.b_beta);
+  b->gamma = f(L.b_gamma);
+  b->bpart2 = f(L.b_bpart2);
+  b->dLpart = f(L.b_dLpart);
+  b->dLns = f(L.b_dLns);
+  b->dLpool = f(L.b_dLpool);
+  b->dQd = f(L.b_dQd);
+}
+
 // Kernel attributes (dynamic shared memory opt-in) are per device; set them once each.
 std::mutex g_attr_mu;
 unsigned long long g_attr_done = 0;
@@ -133,6 +179,7 @@ lfa_status ensure_attributes() {
   std::lock_guard<std::mutex> lk(g_attr_mu);
   if (dev < 64 && (g_attr_done >> dev) & 1ull) return LFA_OK;
   if (lfa::generic_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::backward_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (dev < 64) g_attr_done |= 1ull << dev;
   return LFA_OK;
 }
@@ -303,9 +350,25 @@ lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host
 lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* dO, void* dQ,
                         void* dV, void* stream) {
   if (!h || !Q || !V || !dO || !dQ || !dV) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dV))
+    return LFA_ERR_INVALID_ARG;
   if (!h->have_forward || h->last_Q != Q || h->last_V != V) return LFA_ERR_STATE;
-  (void)stream;
-  return LFA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = h->p;
+  p.Q = Q;
+  p.V = V;
+  p.O = nullptr;
+  p.ev_begin = nullptr;
+  p.ev_end = nullptr;
+  p.trace = nullptr;
+  // the fused forward keeps its intermediates on chip: rebuild the per-stage context
+  if (h->path == 1 && lfa::launch_generic_context(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  lfa::BwdParams b;
+  bind_backward(&b, p, h->lay, h->ws);
+  b.dO = dO;
+  b.dQ = dQ;
+  b.dV = dV;
+  return lfa::launch_backward(b, st) == cudaSuccess ? LFA_OK : LFA_ERR_CUDA;
 }
 
 lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void* stream) {

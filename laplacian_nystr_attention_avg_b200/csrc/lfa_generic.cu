@@ -688,8 +688,23 @@ __global__ void __launch_bounds__(kThreads) k_cross_out(Params p, int u, float* 
   }
 }
 
+// Pass 1 over the tokens (sums of C, C^2, C^T V and V per CTA) and their fp64 reduction
+// into p.red. With p.V pointing at another [N][d] tensor (dO) the same code forms C^T dO.
 template <typename T>
-cudaError_t forward_t(const Params& p, cudaStream_t st) {
+void pass1_reduce_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m, d = p.d;
+  const int bpt = ceil_div((round_up(m, 4) / 4) * (d / 4), kThreads);
+  const dim3 g1(p.P, U);
+  const size_t s1 = generic_smem_pass1(m, d);
+  if (bpt <= 1) k_pass1<T, 1><<<g1, kThreads, s1, st>>>(p);
+  else if (bpt <= 2) k_pass1<T, 2><<<g1, kThreads, s1, st>>>(p);
+  else k_pass1<T, 4><<<g1, kThreads, s1, st>>>(p);
+  k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
+}
+
+// Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b.
+template <typename T>
+void context_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
   if (m <= kSmallM) {
@@ -710,14 +725,14 @@ cudaError_t forward_t(const Params& p, cudaStream_t st) {
     k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
     k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
   }
-  const int bpt = ceil_div((round_up(m, 4) / 4) * (d / 4), kThreads);
-  const dim3 g1(p.P, U);
-  const size_t s1 = generic_smem_pass1(m, d);
-  if (bpt <= 1) k_pass1<T, 1><<<g1, kThreads, s1, st>>>(p);
-  else if (bpt <= 2) k_pass1<T, 2><<<g1, kThreads, s1, st>>>(p);
-  else k_pass1<T, 4><<<g1, kThreads, s1, st>>>(p);
-  k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
+  pass1_reduce_t<T>(p, st);
   k_combine_finish<<<dim3(p.n_chunks, U), kThreads, (size_t)(m * d + 2 * m) * sizeof(float), st>>>(p);
+}
+
+template <typename T>
+cudaError_t forward_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m, d = p.d;
+  context_t<T>(p, st);
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
   k_pass2<T><<<dim3(p.n_tiles, U), kThreads, generic_smem_pass2(m, d), st>>>(p);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
@@ -765,6 +780,18 @@ int generic_launch_count(const Params& p) {
 
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st) {
   return p.dtype == LFA_BF16 ? forward_t<__nv_bfloat16>(p, st) : forward_t<float>(p, st);
+}
+
+cudaError_t launch_generic_context(const Params& p, cudaStream_t st) {
+  if (p.dtype == LFA_BF16) context_t<__nv_bfloat16>(p, st);
+  else context_t<float>(p, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st) {
+  if (p.dtype == LFA_BF16) pass1_reduce_t<__nv_bfloat16>(p, st);
+  else pass1_reduce_t<float>(p, st);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_pool(const Params& p, cudaStream_t st) {

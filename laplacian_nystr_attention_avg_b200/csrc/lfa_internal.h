@@ -30,7 +30,9 @@ __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; 
 struct Layout {
   size_t status, info, L, Wm, X, Xb, Y, part, red, mu, s, A, M, Mp, bpart;
   size_t fused;    // scratch of the fused forward (per-CTA partials, barriers)
-  size_t bwd;      // backward-pass buffers
+  size_t bwd;      // backward-pass buffers (start of the region)
+  size_t b_its, b_G, b_Gn, b_T1, b_T2, b_T3, b_dW, b_part2, b_red2, b_dA, b_Gm, b_Gd, b_beta, b_gamma,
+      b_bpart2, b_dLpart, b_dLns, b_dLpool, b_dQd;
   size_t total;
 };
 
@@ -74,8 +76,41 @@ struct Params {
   unsigned long long* trace;
 };
 
+// Backward-pass tensors and workspace views (with the forward's Params).
+struct BwdParams {
+  Params p;
+  const void* dO;
+  void* dQ;
+  void* dV;
+  float* its;      // [U][T][m][m] Newton-Schulz iterates X_0 .. X_{T-1}
+  float* G;        // [U][m][m] adjoint of the current iterate (starts as dX)
+  float* Gn;       // [U][m][m]
+  float* T1;       // [U][m][m] products of the reverse step
+  float* T2;
+  float* T3;
+  float* dW;       // [U][m][m]
+  float* part2;    // [U][P][part_stride] pass-1 partials with dO in the place of V
+  double* red2;    // [U][part_stride]
+  float* dA;       // [U][m][d]
+  float* Gm;       // [U][m][d] s o M
+  float* Gd;       // [U][m][d] s o dA
+  float* beta;     // [U][m] whitening-backward coefficients
+  float* gamma;    // [U][m]
+  float* bpart2;   // [U][n_chunks][d] bias partials of dV
+  float* dLpart;   // [U][P][m][d] main-pass partials of dL
+  float* dLns;     // [U][m][d] landmark-gram part of dL
+  float* dLpool;   // [U][m][d] dL / r^2
+  float* dQd;      // [U][N][d] fp32 direct part of dQ
+};
+
 // host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
+cudaError_t launch_generic_context(const Params& p, cudaStream_t st);
+cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st);
+cudaError_t launch_backward(const BwdParams& b, cudaStream_t st);
+size_t backward_smem_main(int d);
+cudaError_t backward_set_attributes();
+int backward_launch_count(const Params& p);
 cudaError_t launch_pool(const Params& p, cudaStream_t st);
 cudaError_t launch_cross_kernel(const Params& p, int unit, float* C_out, cudaStream_t st);
 size_t generic_smem_pass1(int m, int d);
