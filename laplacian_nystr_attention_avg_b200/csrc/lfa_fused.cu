@@ -2,30 +2,34 @@
 //
 // One cooperative persistent kernel, one CTA per SM. Token rows of all U = B*heads units are
 // split into contiguous per-CTA ranges (cut at unit boundaries into at most two segments,
-// processed in 128-row chunks).
+// processed in 128-row chunks); CTAs 0..U-1 are the units' solver CTAs and own no rows.
 //   phase 0  all CTAs: landmark pooling L = r x r average pool of Q (LaplacianFormer note,
 //            §关键设计 2); arrive on a grid-wide barrier.
-//   phase 1  while the barrier completes: DWC(V) of the CTA's own rows (3x3 depthwise, zero
-//            padding; §关键设计 1 "ZV + DWC(V)") written to O as bf16.
-//   phase 2  CTAs 0..U-1 first run one unit's solver each: W = exp(-E/lam) + eps I, ||W||_2 by
-//            power iteration, alpha (§关键设计 3 with the fallback), and the T Newton-Schulz
-//            steps on tcgen05 in 3xTF32 (fp32-accurate): X_{k+1} = X_k + X_k R_k,
-//            R_{k+1} = R_k R_k^T (R_k = I - W X_k; the same iterates in exact arithmetic, one
-//            stacked [X; R] product per step), then the printed product form X (2I - W X) for
-//            the last two steps, which re-anchors R to I - W X. X is published with a release
-//            flag. (These CTAs own a smaller row share and do their DWC afterwards.)
-//   phase 3  pass 1 per chunk: C = exp(-||q - l||_1 / lam) on CUDA cores in fp32 (the dominant
-//            cost), kept in shared memory as bf16 for the whole kernel (never in HBM);
+//   phase 1  solver CTA of unit u: W = exp(-E/lam) + eps I, ||W||_2 by power iteration, alpha
+//            (§关键设计 3 with the fallback), and the T Newton-Schulz steps on tcgen05 in 3xTF32
+//            (fp32-accurate): X_{k+1} = X_k + X_k R_k, R_{k+1} = R_k R_k^T (R_k = I - W X_k; the
+//            same iterates in exact arithmetic, one stacked [X; R] product per step), then the
+//            printed product form X (2I - W X) for the last two steps, which re-anchors R to
+//            I - W X.
+//   phase 2  row CTAs, pass 1 per chunk (Q rows by TMA): C = exp(-||q - l||_1 / lam) on CUDA cores
+//            in fp32 (the dominant cost), kept in shared memory as bf16 for the whole kernel (never
+//            in HBM);
 //            per-landmark sums of C and C^2 in registers; P += C^T V on tcgen05 (V chunk staged
 //            by TMA; a constant-1 landmark column 63 yields sum_i v_i in the same product).
 //            Each CTA publishes one partial record per segment.
-//   phase 4  per unit, every CTA of the unit sums the unit's records and forms mu, var,
-//            s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A,
-//            M' = diag(s) M, b = (1/N - s o mu)^T M.
-//   phase 5  per chunk: O = C M' (tcgen05, TMEM accumulator) + b + DWC(V) (read back), bf16.
+//   phase 3  solver CTA of unit u, once the unit's records are out: mu, var, s = 1/sqrt(var +
+//            eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A, M' = diag(s) M,
+//            b = (1/N - s o mu)^T M; M'^T (bf16, in the shared-memory image pass 2 consumes) and
+//            b are published with a release flag.
+//   phase 3b row CTAs, while M' is formed: DWC(V) (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise,
+//            zero padding) of every chunk from a TMA-staged V tile with a one-grid-row halo,
+//            written to O as bf16.
+//   phase 4  row CTAs, per chunk: O = C M' (tcgen05, TMEM accumulator) + b + the DWC values.
 // Every cross-CTA wait is bounded; an expired wait sets the timeout bit of the status word.
 #include <stdlib.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "lfa_internal.h"
 #include "lfa_sm100.cuh"
@@ -36,7 +40,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kFT = 256;                  // threads per CTA (8 warps)
+constexpr int kFT = 512;                  // threads per CTA (16 warps, at most 128 registers each)
+constexpr int kWarps = kFT / 32;
 constexpr int kChunk = 128;               // token rows per chunk
 constexpr int kMaxChunks = 8;             // resident C chunks per CTA
 constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q, L and halo tiles
@@ -54,12 +59,15 @@ constexpr uint32_t kOffMp = kOffL + 64 * kQS * 4;               // M'^T bf16 [64
 constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [64]
 constexpr uint32_t kOffBar = kOffBv + 256;                      // mbarriers + TMEM address
 constexpr uint32_t kOffCt = kOffBar + 128;                      // int [32] record offsets
-constexpr uint32_t kSmemBytes = kOffCt + 128;
+constexpr uint32_t kOffWd = kOffCt + 128;                       // DWC weights fp32 [9 taps][64 ch]
+constexpr uint32_t kOffSr = kOffWd + 9 * 64 * 4;                // pass-1 column sums [segment][row half][128]
+constexpr uint32_t kSmemBytes = kOffSr + 2 * 256 * 4;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
-// phase-1 scratch: the V rows (with a one-grid-row halo) of this CTA's segments, bf16 [rows][64]
-// (plain 128-byte rows, TMA without swizzle), in the region below M' that pass 1 fills later
-constexpr uint32_t kOffHalo = kOffC;
-constexpr int kHaloRows = (int)(kOffMp / 128);
+// pass-2 scratch: V rows of one chunk with a one-grid-row halo on each side, SW128 (TMA boxes of
+// 128 rows), one or two buffers in the region of the V stages, Q and L (free after pass 1)
+constexpr uint32_t kOffHb = kOffV;
+constexpr uint32_t kHaloSpace = kOffMp - kOffV;
+constexpr int kImgBytes = 8192 + 256;                           // published M' image + b per unit
 // combine scratch (aliases V/Q/L, free once pass 1 is done)
 constexpr uint32_t kOffAs = kOffV;                              // fp32 [64][68]  A (row l, col k)
 constexpr uint32_t kOffXt = kOffAs + 64 * kQS * 4;              // fp32 [64][68]  X^T (row l, col j)
@@ -78,7 +86,7 @@ constexpr uint32_t kOffNsL = kOffNsX + 64 * kQS * 4;            // fp32 [64][68]
 constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64] + reduction [16]
 
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
-static_assert(kOffBp + 16 * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
+static_assert(kOffBp + (kFT / 16) * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -86,7 +94,10 @@ constexpr int kBarV = 0;      // [2] V stage filled by TMA
 constexpr int kBarP1 = 2;     // [2] pass-1 product done (stage free)
 constexpr int kBarP2 = 4;     // [2] pass-2 product done (accumulator ready)
 constexpr int kBarNs = 6;     // solver product done
-constexpr int kBarDwc = 7;    // DWC halo rows landed (TMA)
+constexpr int kBarH = 8;      // [2] DWC V halo tile landed (TMA)
+constexpr int kBarQ = 10;     // pass-1 Q chunk landed (TMA, bf16 rows in the spare C slot)
+constexpr int kNumBars = 11;
+constexpr uint32_t kTmemSlot = 96;   // byte offset of the TMEM address within the barrier area
 
 struct FusedArgs {
   unsigned long long epoch;   // launch count of this handle (>= 1); flags compare against it
@@ -95,7 +106,9 @@ struct FusedArgs {
   unsigned long long* gbar;   // grid barrier counter
   unsigned long long* cnt;    // [U] partial records published per unit
   unsigned long long* xready; // [U] X published (holds the epoch)
+  unsigned long long* mready; // [U] M' image and b published (holds the epoch)
   float* rec;                 // [G][2][kRec]
+  unsigned char* mimg;        // [U][kImgBytes] M'^T bf16 (SW128 image of the pass-2 B operand), b fp32
 };
 
 __device__ __forceinline__ void trace_mark(const Params& p, int slot) {
@@ -105,17 +118,24 @@ __device__ __forceinline__ void trace_clock(const Params& p, int slot) {
   if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 32 + slot] = (unsigned long long)clock64();
 }
 
-// first global row of CTA g (rows weighted: solver CTAs ws16/16 of a plain CTA)
-__device__ __forceinline__ long long cta_start(int g, int U, const FusedArgs& fa, long long T) {
-  const long long cw = g <= U ? (long long)fa.ws16 * g : (long long)fa.ws16 * U + 16ll * (g - U);
-  return T * cw / fa.totw16;
+// First global row (u * N + row) of CTA g. Each unit's rows are cut into 128-row chunks (the
+// last one may be short) and whole chunks are dealt out in proportion to the CTA weights
+// (a solver CTA weighs ws16/16 of a plain CTA), so no CTA gets a partial chunk mid-unit.
+__host__ __device__ __forceinline__ long long part_start(int g, int U, int N, int ws16, long long totw16) {
+  const long long cw = g <= U ? (long long)ws16 * g : (long long)ws16 * U + 16ll * (g - U);
+  const long long nchu = (N + kChunk - 1) / kChunk;
+  const long long ci = (long long)U * nchu * cw / totw16;
+  return (ci / nchu) * N + (ci % nchu) * kChunk;
+}
+__device__ __forceinline__ long long cta_start(int g, const Params& p, const FusedArgs& fa) {
+  return part_start(g, p.U, p.N, fa.ws16, fa.totw16);
 }
 // CTA whose range holds global row R
-__device__ __forceinline__ int cta_of_row(long long R, int U, int G, const FusedArgs& fa, long long T) {
-  int lo = 0, hi = G - 1;
+__device__ __forceinline__ int cta_of_row(long long R, const Params& p, const FusedArgs& fa) {
+  int lo = 0, hi = gridDim.x - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (cta_start(mid, U, fa, T) <= R) lo = mid;
+    if (cta_start(mid, p, fa) <= R) lo = mid;
     else hi = mid - 1;
   }
   return lo;
@@ -137,27 +157,28 @@ __device__ __forceinline__ void block_reduce2(float& a, float& b, float* red) {
   __syncthreads();
   if (lane == 0) {
     red[w] = a;
-    red[8 + w] = b;
+    red[kWarps + w] = b;
   }
   __syncthreads();
   a = 0.f;
   b = 0.f;
-  for (int i = 0; i < kFT / 32; ++i) {
+  for (int i = 0; i < kWarps; ++i) {
     a += red[i];
-    b += red[8 + i];
+    b += red[kWarps + i];
   }
 }
 
 // L [m][64] fp32 (global, written by other CTAs of this launch) -> [64][kQS] shared, zero rows >= m.
 __device__ __forceinline__ void load_landmarks(const float* Lg, float* Ls, int m) {
-  float4 v[4];
+  constexpr int kN4 = 1024 / kFT;   // float4 of the [64][64] block per thread
+  float4 v[kN4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < kN4; ++i) {
     const int e4 = threadIdx.x + kFT * i, r = e4 >> 4;
     v[i] = r < m ? __ldcg(reinterpret_cast<const float4*>(Lg) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < kN4; ++i) {
     const int e4 = threadIdx.x + kFT * i;
     *reinterpret_cast<float4*>(Ls + (e4 >> 4) * kQS + 4 * (e4 & 15)) = v[i];
   }
@@ -183,8 +204,7 @@ struct Rows {
 
 __device__ Rows cta_rows(int g, const Params& p, const FusedArgs& fa) {
   Rows R;
-  const long long T = (long long)p.U * p.N;
-  const long long r0 = cta_start(g, p.U, fa, T), r1 = cta_start(g + 1, p.U, fa, T);
+  const long long r0 = cta_start(g, p, fa), r1 = cta_start(g + 1, p, fa);
   R.nseg = 0;
   long long a = r0;
   int fc = 0;
@@ -206,113 +226,14 @@ __device__ Rows cta_rows(int g, const Params& p, const FusedArgs& fa) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 1: DWC(V) of this CTA's rows -> O (bf16). The V rows of each segment, with a
-// one-grid-row halo, are brought in by TMA (plain rows) in one batch; each thread then owns
-// 4 consecutive tokens of a grid row x 4 channels (weights in registers) and slides a
-// 3 x 6 window over the tile.
+// Phase 1: solver of one unit. Thread (warp w, lane) owns row r = 32 (w % 4) + lane of the
+// stacked 128 x 64 operand [top; bottom] and the column quarter h = w / 4 (16 columns).
 // ---------------------------------------------------------------------------------------
-struct HaloPlan {
-  int hlo[2];    // first unit row of each segment's halo range
-  int hhi[2];
-  int base[2];   // tile row holding row hlo
-  int rows;      // tile rows in use
-};
-
-__device__ __forceinline__ HaloPlan halo_plan(const Params& p, const Rows& R) {
-  HaloPlan h;
-  int base = 0;
-  for (int s = 0; s < 2; ++s) {
-    h.hlo[s] = h.hhi[s] = h.base[s] = 0;
-    if (s >= R.nseg) continue;
-    h.hlo[s] = max(0, R.seg[s].lo - p.W - 1);
-    h.hhi[s] = min(p.N, R.seg[s].hi + p.W + 1);
-    h.base[s] = base;
-    base += (h.hhi[s] - h.hlo[s] + kChunk - 1) / kChunk * kChunk;
-  }
-  h.rows = base;
-  return h;
-}
-
-// one thread: TMA loads of every segment's halo rows into the tile, completing on kBarDwc
-__device__ void dwc_issue(const Params& p, const Rows& R, const HaloPlan& h, unsigned char* sm, uint64_t* bars,
-                          const CUtensorMap* tmapVp) {
-  if (h.rows == 0) return;
-  fence_async_smem();
-  mbar_expect_tx(bars + kBarDwc, (uint32_t)h.rows * 128u);
-  for (int s = 0; s < R.nseg; ++s) {
-    const int nb = (h.hhi[s] - h.hlo[s] + kChunk - 1) / kChunk;
-    for (int b = 0; b < nb; ++b)
-      tma_load_3d(sm + kOffHalo + (size_t)(h.base[s] + b * kChunk) * 128, tmapVp, 0, h.hlo[s] + b * kChunk, R.seg[s].u,
-                  bars + kBarDwc);
-  }
-}
-
-__device__ void dwc_compute(const Params& p, const Rows& R, const HaloPlan& h, const unsigned char* sm) {
-  const int t = threadIdx.x, cq = t & 15, slot = t >> 4;
-  const int W = p.W, H = p.H;
-  const int runs = (W + 3) >> 2;
-  __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
-  float wt[9][4];
-  int head = -1;
-  for (int s = 0; s < R.nseg; ++s) {
-    const int u = R.seg[s].u, lo = R.seg[s].lo, hi = R.seg[s].hi;
-    const int hlo = h.hlo[s], hhi = h.hhi[s], base = h.base[s];
-    if (u % p.heads != head) {
-      head = u % p.heads;
-#pragma unroll
-      for (int tap = 0; tap < 9; ++tap)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) wt[tap][e] = __ldg(p.dwc + ((size_t)head * 64 + 4 * cq + e) * 9 + tap);
-    }
-    const int ylo = lo / W, yhi = (hi - 1) / W;
-    const int nitems = (yhi - ylo + 1) * runs;
-    __nv_bfloat16* Ou = O + (size_t)u * p.N * 64 + 4 * cq;
-    for (int item = slot; item < nitems; item += kFT / 16) {
-      const int y = ylo + item / runs, x0 = (item % runs) * 4;
-      float v[3][6][4];
-#pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        const int yy = y + a - 1;
-        const bool rv = yy >= 0 && yy < H;
-#pragma unroll
-        for (int b = 0; b < 6; ++b) {
-          const int xx = x0 + b - 1;
-          const int n2 = yy * W + xx;
-          float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (rv && xx >= 0 && xx < W && n2 >= hlo && n2 < hhi) {
-            const uint2 raw = *reinterpret_cast<const uint2*>(sm + kOffHalo + (size_t)(n2 - hlo + base) * 128 + 8 * cq);
-            f = make_float4(bf_lo(raw.x), bf_hi(raw.x), bf_lo(raw.y), bf_hi(raw.y));
-          }
-          v[a][b][0] = f.x;
-          v[a][b][1] = f.y;
-          v[a][b][2] = f.z;
-          v[a][b][3] = f.w;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int x = x0 + j, n = y * W + x;
-        if (x >= W || n < lo || n >= hi) continue;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int a = 0; a < 3; ++a)
-#pragma unroll
-          for (int b = 0; b < 3; ++b)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[c] = fmaf(wt[a * 3 + b][c], v[a][j + b][c], acc[c]);
-        *reinterpret_cast<uint2*>(Ou + (size_t)n * 64) = make_uint2(pack_bf16(acc[0], acc[1]), pack_bf16(acc[2], acc[3]));
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------------------
-// Phase 2: solver of one unit. Thread (warp w, lane) owns row r = 32 (w % 4) + lane of the
-// stacked 128 x 64 operand [top; bottom] and the column half h = w / 4.
-// ---------------------------------------------------------------------------------------
+// The operand is stored as two K-halves of 32 fp32 columns (128-byte SW128 rows), split into
+// tf32 hi and lo parts.
 __device__ void ns_store(unsigned char* base, int r, int h, const float* v) {
 #pragma unroll
-  for (int c4 = 0; c4 < 8; ++c4) {
+  for (int c4 = 0; c4 < 4; ++c4) {
     float4 hi, lo;
     hi.x = tf32_round(v[4 * c4 + 0]);
     hi.y = tf32_round(v[4 * c4 + 1]);
@@ -322,7 +243,7 @@ __device__ void ns_store(unsigned char* base, int r, int h, const float* v) {
     lo.y = v[4 * c4 + 1] - hi.y;
     lo.z = v[4 * c4 + 2] - hi.z;
     lo.w = v[4 * c4 + 3] - hi.w;
-    const uint32_t off = h * 16384 + sw128(r, c4);
+    const uint32_t off = (h >> 1) * 16384 + sw128(r, (h & 1) * 4 + c4);
     *reinterpret_cast<float4*>(base + kOffNsHi + off) = hi;
     *reinterpret_cast<float4*>(base + kOffNsLo + off) = lo;
   }
@@ -401,7 +322,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   // scaled by 1/m per step (the Rayleigh quotient is scale free), one barrier per step
   float lmax;
   {
-    const int row = t >> 2, part = t & 3;
+    const int row = t >> 3, part = t & 7;
     const float sc = 1.f / (float)m;
     float wi = 0.f;
     for (int it = 0; it <= kPowerIters; ++it) {
@@ -409,10 +330,11 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
       wi = 0.f;
       if (row < m) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) wi = fmaf(Ws[row * kQS + 16 * part + j], vin[16 * part + j], wi);
+        for (int j = 0; j < 8; ++j) wi = fmaf(Ws[row * kQS + 8 * part + j], vin[8 * part + j], wi);
       }
       wi += __shfl_xor_sync(0xffffffffu, wi, 1);
       wi += __shfl_xor_sync(0xffffffffu, wi, 2);
+      wi += __shfl_xor_sync(0xffffffffu, wi, 4);
       if (it == kPowerIters) break;
       if (part == 0) vec[64 * ((it + 1) & 1) + row] = row < m ? wi * sc : 0.f;
       __syncthreads();
@@ -434,12 +356,12 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   const int i = r & 63;                // matrix row
   const bool top = r < 64;
   const int nks = (m + 7) >> 3;        // K steps of 8 covering the m landmarks
-  const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + 32 * h;
+  const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16) + 16 * h;
   uint64_t* bar = bars + kBarNs;
   int round = 0;
-  float st[32], d[32], wrow[32];
+  float st[16], d[16], wrow[16];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) wrow[c] = Ws[i * kQS + 32 * h + c];
+  for (int c = 0; c < 16; ++c) wrow[c] = Ws[i * kQS + 16 * h + c];
 
   auto run_round = [&]() {
     fence_async_smem();
@@ -452,7 +374,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     mbar_wait(bar, round & 1, p.status, kStatusTimeout);
     if (round == 5) trace_mark(p, 22);
     tc_fence_after();
-    tmem_ld32(trow, d);
+    tmem_ld16(trow, d);
     if (round == 5) trace_mark(p, 23);
     if (round == 0) trace_mark(p, 18);
     if (round == 10) trace_mark(p, 19);
@@ -460,38 +382,46 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   };
   auto clean = [&](float* v) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (i >= m || 32 * h + c >= m) v[c] = 0.f;
+    for (int c = 0; c < 16; ++c)
+      if (i >= m || 16 * h + c >= m) v[c] = 0.f;
   };
 
   // round 0: D_bottom = W W^T = W^2; X_0 = alpha W^T (= alpha W), R_0 = I - alpha W^2
   {
-    float v[32];
+    float v[16];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = top ? 0.f : wrow[c];
+    for (int c = 0; c < 16; ++c) v[c] = top ? 0.f : wrow[c];
     ns_store(sm, r, h, v);
   }
   run_round();
   if (top) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) st[c] = alpha * wrow[c];
+    for (int c = 0; c < 16; ++c) st[c] = alpha * wrow[c];
   } else {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) st[c] = (i == 32 * h + c ? 1.f : 0.f) - alpha * d[c];
+    for (int c = 0; c < 16; ++c) st[c] = (i == 16 * h + c ? 1.f : 0.f) - alpha * d[c];
   }
   clean(st);
   const int n_lit = p.T < 2 ? p.T : 2;
   const int n_res = p.T - n_lit;
   // residual steps: A = [X; R], D = [X R^T; R R^T]
   for (int k = 0; k < n_res; ++k) {
+    // R_k exactly zero: every remaining residual step is the identity in floating point
+    // (X + X 0 = X, 0 0^T = 0), so the chain continues with the printed steps below
+    bool rnz = false;
+    if (!top) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) rnz |= st[c] != 0.f;
+    }
+    if (!__syncthreads_or(rnz)) break;
     ns_store(sm, r, h, st);
     run_round();
     if (top) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) st[c] += d[c];
+      for (int c = 0; c < 16; ++c) st[c] += d[c];
     } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) st[c] = d[c];
+      for (int c = 0; c < 16; ++c) st[c] = d[c];
     }
     clean(st);
   }
@@ -500,21 +430,21 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     // A = [W; X]: top rows W, bottom rows X (from the top threads through shared memory)
     if (top) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) Xsm[i * kQS + 32 * h + c] = st[c];
+      for (int c = 0; c < 16; ++c) Xsm[i * kQS + 16 * h + c] = st[c];
     }
     __syncthreads();
-    float v[32];
+    float v[16];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) v[c] = top ? wrow[c] : Xsm[i * kQS + 32 * h + c];
+    for (int c = 0; c < 16; ++c) v[c] = top ? wrow[c] : Xsm[i * kQS + 16 * h + c];
     ns_store(sm, r, h, v);
   };
   for (int k = 0; k < n_lit; ++k) {
     stage_w_over_x();
     run_round();                       // D_top = W X
     if (top) {
-      float rb[32];
+      float rb[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) rb[c] = (i == 32 * h + c ? 1.f : 0.f) - d[c];
+      for (int c = 0; c < 16; ++c) rb[c] = (i == 16 * h + c ? 1.f : 0.f) - d[c];
       clean(rb);
       ns_store(sm, r, h, st);          // A = [X; I - W X]
       ns_store(sm, r + 64, h, rb);
@@ -522,15 +452,15 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     run_round();                       // D_top = X (I - W X)
     if (top) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) st[c] += d[c];
+      for (int c = 0; c < 16; ++c) st[c] += d[c];
       clean(st);
     }
   }
   // publish X_T
   if (top && i < m) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (32 * h + c < m) p.X[((size_t)u * m + i) * m + 32 * h + c] = st[c];
+    for (int c = 0; c < 16; ++c)
+      if (16 * h + c < m) p.X[((size_t)u * m + i) * m + 16 * h + c] = st[c];
   }
   __syncthreads();
   if (t == 0) {
@@ -544,9 +474,9 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   float sq = 0.f, dummy = 0.f;
   if (top && i < m) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (32 * h + c < m) {
-        const float e = (i == 32 * h + c ? 1.f : 0.f) - d[c];
+    for (int c = 0; c < 16; ++c)
+      if (16 * h + c < m) {
+        const float e = (i == 16 * h + c ? 1.f : 0.f) - d[c];
         sq += e * e;
       }
   }
@@ -568,22 +498,22 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
 // ---------------------------------------------------------------------------------------
 template <int LT>
 __device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, unsigned char* cslot, int j0,
-                                            int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
+                                            int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
   const int lane = threadIdx.x & 31;
-  float acc[4][LT];
+  float acc[2][LT];
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+  for (int a = 0; a < 2; ++a)
 #pragma unroll
     for (int b = 0; b < LT; ++b) acc[a][b] = 0.f;
 #pragma unroll 2
   for (int k = 0; k < 64; k += 4) {
-    float4 q[4], l[LT];
+    float4 q[2], l[LT];
 #pragma unroll
-    for (int a = 0; a < 4; ++a) q[a] = *reinterpret_cast<const float4*>(&Qs[(lane + 32 * a) * kQS + k]);
+    for (int a = 0; a < 2; ++a) q[a] = *reinterpret_cast<const float4*>(&Qs[(rb + lane + 32 * a) * kQS + k]);
 #pragma unroll
     for (int b = 0; b < LT; ++b) l[b] = *reinterpret_cast<const float4*>(&Ls[(j0 + b) * kQS + k]);
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
       for (int b = 0; b < LT; ++b) {
         float s = acc[a][b];
@@ -596,8 +526,8 @@ __device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, un
   }
   const bool even = (j0 & 1) == 0;
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int row = lane + 32 * a;
+  for (int a = 0; a < 2; ++a) {
+    const int row = rb + lane + 32 * a;
     const bool valid = row < nrows;
     float c[LT];
 #pragma unroll
@@ -626,37 +556,32 @@ __device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, un
 }
 
 __device__ __forceinline__ void cross_dispatch(int lt, const float* Qs, const float* Ls, unsigned char* cslot,
-                                               int j0, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
+                                               int j0, int rb, int nrows, float scale, float (&s1)[8],
+                                               float (&s2)[8]) {
   switch (lt) {
-    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
-    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, nrows, scale, s1, s2); break;
+    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
     default: break;
   }
 }
 
-// Q rows of a chunk: thread t loads row t/2, 32 channels (t % 2) as 4 x 16 bytes.
-__device__ __forceinline__ void q_fetch(const __nv_bfloat16* Qu, int lo, int nrows, uint4 (&qr)[4]) {
-  const int t = threadIdx.x, row = t >> 1, half = t & 1;
+// Q rows of a chunk, bf16 [128][64] plain rows (TMA) -> fp32 [128][kQS]: thread t converts row
+// t/4, 16 channels (t % 4); rows at or past nrows become zero.
+__device__ __forceinline__ void q_stage(float* Qs, const unsigned char* qsrc, int nrows) {
+  const int t = threadIdx.x, row = t >> 2, qt = t & 3;
+  float* dst = Qs + row * kQS + 16 * qt;
+  uint4 qr[2];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) qr[k] = make_uint4(0u, 0u, 0u, 0u);
-  if (row < nrows) {
-    const uint4* src = reinterpret_cast<const uint4*>(Qu + ((size_t)(lo + row)) * 64 + 32 * half);
+  for (int k = 0; k < 2; ++k)
+    qr[k] = row < nrows ? reinterpret_cast<const uint4*>(qsrc + row * 128 + 32 * qt)[k] : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) qr[k] = __ldg(src + k);
-  }
-}
-
-__device__ __forceinline__ void q_stage(float* Qs, const uint4 (&qr)[4]) {
-  const int t = threadIdx.x, row = t >> 1, half = t & 1;
-  float* dst = Qs + row * kQS + 32 * half;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < 2; ++k) {
     const uint4 v = qr[k];
     *reinterpret_cast<float4*>(dst + 8 * k) = make_float4(bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y));
     *reinterpret_cast<float4*>(dst + 8 * k + 4) = make_float4(bf_lo(v.z), bf_hi(v.z), bf_lo(v.w), bf_hi(v.w));
@@ -664,18 +589,38 @@ __device__ __forceinline__ void q_stage(float* Qs, const uint4 (&qr)[4]) {
 }
 
 __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
-                      uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapV) {
+                      uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapV, const CUtensorMap* tmapQ) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31, g = blockIdx.x;
-  const int m = p.m, N = p.N;
+  const int m = p.m, nch = R.nchunks;
+  unsigned char* qslot = sm + kOffC + nch * 16384;       // spare C slot (nch < kMaxChunks)
   float* Qs = reinterpret_cast<float*>(sm + kOffQ);
   float* Ls = reinterpret_cast<float*>(sm + kOffL);
-  const __nv_bfloat16* Qg = static_cast<const __nv_bfloat16*>(p.Q);
-  // landmark groups: 8 warps, the m % 8 larger groups last so that every group starts at an
-  // even landmark when m / 8 is even (paired C stores)
-  const int lbase = m / 8, lextra = m % 8;
-  const int big = 8 - lextra;           // warps >= big take lbase + 1 landmarks
-  const int lt = lbase + (w >= big ? 1 : 0);
-  const int j0 = w * lbase + (w > big ? w - big : 0);
+  float* sred = reinterpret_cast<float*>(sm + kOffSr);   // [segment][row half][S1 64 | S2 64]
+  // Landmark groups: warps w and w + 8 share group w % 8 (rows 0-63 and 64-127). The groups
+  // start from m = 8 lbase + lextra split as evenly as possible; where some groups are one
+  // larger, group 0 hands up to two landmarks to smaller groups without raising the largest
+  // size, because warp 0 also issues the chunk products.
+  const int wg = w & 7, rh = w >> 3;
+  int lt = 0, j0 = 0;
+  {
+    const int lbase = m / 8, lextra = m % 8;
+    int sz[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sz[i] = lbase + (i >= 8 - lextra ? 1 : 0);
+    int give = lextra > 0 ? min(2, min(sz[0], 8 - lextra)) : 0;
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+      if (give > 0 && sz[i] == lbase) {
+        ++sz[i];
+        --sz[0];
+        --give;
+      }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i < wg) j0 += sz[i];
+      if (i == wg) lt = sz[i];
+    }
+  }
   const float scale = p.neg_log2e_over_lam;
   auto issue_v = [&](int gc) {
     int s, lo, nrows;
@@ -684,25 +629,44 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     mbar_expect_tx(fb, 16384);
     tma_load_3d(sm + kOffV + (gc & 1) * 16384, tmapV, 0, lo, R.seg[s].u, fb);
   };
-  uint4 qr[4];
-  {
+  // P_s += C^T V for chunk gc (M = 64 landmarks, N = 64 channels, K = 128 rows)
+  auto issue_mma = [&](int gc) {
     int s, lo, nrows;
-    R.chunk(0, s, lo, nrows);
-    q_fetch(Qg + (size_t)R.seg[s].u * N * 64, lo, nrows, qr);
-    if (t == 0) {
-      fence_async_smem();     // the V stages were read by generic loads (DWC tile) before
-      issue_v(0);
-    }
+    R.chunk(gc, s, lo, nrows);
+    const bool first = gc == R.seg[s].first_chunk;
+    mbar_wait(bars + kBarV + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
+    tc_fence_after();
+    const uint32_t id = idesc(1, 64, 64, 1, 1);
+    const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 8192, 1024);
+    const uint64_t va = desc_sw128(sbase + kOffV + (gc & 1) * 16384, 8192, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tmem + 64 * s, ca + (uint64_t)(kk * 2048 >> 4), va + (uint64_t)(kk * 2048 >> 4), id,
+               (!first || kk > 0) ? 1u : 0u);
+    mma_commit(bars + kBarP1 + (gc & 1));
+  };
+  auto issue_q = [&](int gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    mbar_expect_tx(bars + kBarQ, 16384);
+    tma_load_3d(qslot, tmapQ, 0, lo, R.seg[s].u, bars + kBarQ);
+  };
+  if (t == 0) {
+    fence_async_smem();
+    issue_q(0);
+    issue_v(0);
+    if (nch > 1) issue_v(1);
   }
+  trace_mark(p, 28);
   float s1[8], s2[8];
-  for (int gc = 0; gc < R.nchunks; ++gc) {
+  for (int gc = 0; gc < nch; ++gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
     const int u = R.seg[s].u;
     const bool seg_first = gc == R.seg[s].first_chunk;
     const bool seg_last = gc == R.seg[s].first_chunk + R.seg[s].nch - 1;
     unsigned char* cslot = sm + kOffC + gc * 16384;
-    __syncthreads();     // previous chunk's readers of Qs / Ls are done
+    // Qs and Ls were last read before the previous chunk's closing barrier
     if (seg_first) {
       load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
 #pragma unroll
@@ -711,45 +675,30 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
         s2[b] = 0.f;
       }
     }
-    q_stage(Qs, qr);
+    mbar_wait(bars + kBarQ, gc & 1, p.status, kStatusTimeout);
+    if (gc < 2) trace_mark(p, 27 - 3 * gc);
+    q_stage(Qs, qslot, nrows);
     // padding landmark columns m..63: zero, except column 63 = 1 on valid rows (sum of V)
     for (int e = t; e < kChunk * (64 - m); e += kFT) {
       const int row = e / (64 - m), col = m + e % (64 - m);
       const float v = (col == 63 && row < nrows) ? 1.f : 0.f;
       *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = __float2bfloat16_rn(v);
     }
+    if (gc == 1) trace_mark(p, 26);
     __syncthreads();
-    if (gc + 1 < R.nchunks) {
-      int s2i, lo2, nr2;
-      R.chunk(gc + 1, s2i, lo2, nr2);
-      q_fetch(Qg + (size_t)R.seg[s2i].u * N * 64, lo2, nr2, qr);
+    // the spare slot has been converted: the next chunk's Q rows are fetched during this one
+    if (t == 0 && gc + 1 < nch) {
+      fence_async_smem();
+      issue_q(gc + 1);
     }
-    if (gc == 0) trace_mark(p, 10);
-    if (lt > 0) cross_dispatch(lt, Qs, Ls, cslot, j0, nrows, scale, s1, s2);
-    // the other V stage was last read by chunk gc-1's product, committed long before here
-    if (t == 0 && gc + 1 < R.nchunks) {
-      if (gc >= 1) mbar_wait(bars + kBarP1 + ((gc + 1) & 1), ((gc - 1) >> 1) & 1, p.status, kStatusTimeout);
-      issue_v(gc + 1);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (gc < 2) trace_mark(p, 11 + gc);
-    if (t == 0) {
-      mbar_wait(bars + kBarV + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
-      tc_fence_after();
-      const uint32_t id = idesc(1, 64, 64, 1, 1);
-      const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 8192, 1024);
-      const uint64_t va = desc_sw128(sbase + kOffV + (gc & 1) * 16384, 8192, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + 64 * s, ca + (uint64_t)(kk * 2048 >> 4), va + (uint64_t)(kk * 2048 >> 4), id,
-                 (!seg_first || kk > 0) ? 1u : 0u);
-      mma_commit(bars + kBarP1 + (gc & 1));
-    }
+    if (gc < 2) trace_mark(p, 10 + 11 * gc);
+    // the previous chunk's C tile is complete (closing barrier): its product goes out now,
+    // overlapping this chunk's distances
+    if (t == 0 && gc >= 1) issue_mma(gc - 1);
+    if (lt > 0) cross_dispatch(lt, Qs, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
+    if (gc == 1) trace_mark(p, 22);
     if (seg_last) {
-      // publish this CTA's record for unit u: S1, S2 (warp shuffles) and P (TMEM)
-      float* rec = fa.rec + ((size_t)g * 2 + s) * kRec;
+      // this segment's column sums of C and C^2, per row half
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         float a1 = s1[b], a2 = s2[b];
@@ -758,47 +707,62 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
           a2 += __shfl_xor_sync(0xffffffffu, a2, o);
         }
         if (lane == 0 && b < lt) {
-          rec[j0 + b] = a1;
-          rec[64 + j0 + b] = a2;
+          sred[256 * s + 128 * rh + j0 + b] = a1;
+          sred[256 * s + 128 * rh + 64 + j0 + b] = a2;
         }
-      }
-      if (t < 64 && t >= m) {
-        rec[t] = 0.f;
-        rec[64 + t] = 0.f;
-      }
-      mbar_wait(bars + kBarP1 + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
-      tc_fence_after();
-      if (w < 4) {
-        float v[32];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(tmem + 64 * s + ((uint32_t)(32 * w) << 16) + 32 * hh, v);
-          if (lane < 16) {
-            float* dst = rec + 128 + (16 * w + lane) * 64 + 32 * hh;
-#pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-          }
-        }
-      }
-      tc_fence_before();
-      __syncthreads();
-      if (t == 0) {
-        __threadfence();
-        red_release_add_u64(fa.cnt + u, 1ull);
       }
     }
+    // V stage (gc + 1) & 1 was read by the product of chunk gc - 1, issued at this chunk's start
+    if (t == 0 && gc >= 1 && gc + 1 < nch) {
+      mbar_wait(bars + kBarP1 + ((gc - 1) & 1), ((gc - 1) >> 1) & 1, p.status, kStatusTimeout);
+      issue_v(gc + 1);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (gc < 2) trace_mark(p, 11 + gc);
+  }
+  // last chunk's product, then the records: S1, S2 and P (TMEM columns 64 s) per segment
+  if (t == 0) {
+    issue_mma(nch - 1);
+    if (nch >= 2) mbar_wait(bars + kBarP1 + ((nch - 2) & 1), ((nch - 2) >> 1) & 1, p.status, kStatusTimeout);
+  }
+  mbar_wait(bars + kBarP1 + ((nch - 1) & 1), ((nch - 1) >> 1) & 1, p.status, kStatusTimeout);
+  tc_fence_after();
+  for (int s = 0; s < R.nseg; ++s) {
+    float* rec = fa.rec + ((size_t)g * 2 + s) * kRec;
+    if (w < 4) {
+      float v[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        tmem_ld32(tmem + 64 * s + ((uint32_t)(32 * w) << 16) + 32 * hh, v);
+        if (lane < 16) {
+          float* dst = rec + 128 + (16 * w + lane) * 64 + 32 * hh;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+        }
+      }
+    }
+    if (t < 128) rec[t] = (t & 63) < m ? sred[256 * s + t] + sred[256 * s + 128 + t] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0) {
+    __threadfence();
+    for (int s = 0; s < R.nseg; ++s) red_release_add_u64(fa.cnt + R.seg[s].u, 1ull);
   }
 }
 
 // ---------------------------------------------------------------------------------------
-// Phases 4 + 5 for one segment: combine the unit's records, then O = C M' + b + DWC.
+// Phase 4, on the unit's solver CTA once X is known: sum the unit's records and form mu, var,
+// s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A, M' = diag(s) M and
+// b = (1/N - s o mu)^T M. M'^T is written as the bf16 SW128 image of pass 2's B operand and
+// published with b under a release flag.
 // ---------------------------------------------------------------------------------------
-__device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Rows& R, int s, int& pc,
-                                  unsigned char* sm, uint32_t sbase, uint32_t tmem, uint64_t* bars) {
-  const int t = threadIdx.x, w = t >> 5, lane = t & 31, g = blockIdx.x;
-  const int m = p.m, N = p.N, U = p.U, G = gridDim.x;
-  const long long Trows = (long long)U * N;
+__device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, int u) {
+  const int t = threadIdx.x;
+  const int m = p.m, N = p.N;
   float* As = reinterpret_cast<float*>(sm + kOffAs);
   float* Xt = reinterpret_cast<float*>(sm + kOffXt);
   double* S1d = reinterpret_cast<double*>(sm + kOffS1);
@@ -807,68 +771,91 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
   float* scs = reinterpret_cast<float*>(sm + kOffSc);
   float* svs = reinterpret_cast<float*>(sm + kOffSv);
   float* bps = reinterpret_cast<float*>(sm + kOffBp);
-  float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   int* ctr = reinterpret_cast<int*>(sm + kOffCt);
   const float invNf = 1.f / (float)N;
   const double invN = 1.0 / (double)N;
-  const int u = R.seg[s].u;
-  const int gf = cta_of_row((long long)u * N, U, G, fa, Trows);
-  const int gl = cta_of_row((long long)(u + 1) * N - 1, U, G, fa, Trows);
-  const int nct = gl - gf + 1;
-  __syncthreads();
-  if (t == 0) {
-    spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout);
-    spin_until_geq(fa.xready + u, fa.epoch, p.status, kStatusTimeout);
-  }
-  if (t < nct && t < kMaxContrib) {
-    const int gg = gf + t;
-    const int sj = cta_start(gg, U, fa, Trows) < (long long)u * N ? 1 : 0;
-    ctr[t] = (gg * 2 + sj) * kRec;
-  }
-  __syncthreads();
-  trace_mark(p, 4 + 3 * s);
-  // sum the unit's records: S1, S2 in fp64, P in fp32 (float4), eight records in flight
-  if (t < 128) {
-    double acc = 0.0;
-    for (int c0 = 0; c0 < nct; c0 += 8) {
-      float v[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) v[c] = c0 + c < nct ? __ldcg(fa.rec + ctr[c0 + c] + t) : 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc += (double)v[c];
-    }
-    if (t < 64) S1d[t] = acc;
-    else S2d[t - 64] = acc;
-  }
-  for (int e4 = t; e4 < 1024; e4 += kFT) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < nct; c0 += 8) {
-      float4 v[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        v[c] = c0 + c < nct ? __ldcg(reinterpret_cast<const float4*>(fa.rec + ctr[c0 + c] + 128) + e4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        acc.x += v[c].x;
-        acc.y += v[c].y;
-        acc.z += v[c].z;
-        acc.w += v[c].w;
-      }
-    }
-    *reinterpret_cast<float4*>(As + (e4 >> 4) * kQS + 4 * (e4 & 15)) = acc;
-  }
+  // candidates gf..gl; CTAs with an empty range (possible when there are fewer chunks than
+  // CTAs) publish nothing and are dropped from the contributor table
+  const int gf = cta_of_row((long long)u * N, p, fa);
+  const int gl = cta_of_row((long long)(u + 1) * N - 1, p, fa);
+  const int ncand = gl - gf + 1;
+  // X^T of this unit (written by this CTA before its X flag)
   {
-    float xv[16];
+    constexpr int kNX = 4096 / kFT;
+    float xv[kNX];
 #pragma unroll
-    for (int i2 = 0; i2 < 16; ++i2) {
+    for (int i2 = 0; i2 < kNX; ++i2) {
       const int e = t + kFT * i2, jr = e >> 6, l = e & 63;
-      xv[i2] = (jr < m && l < m) ? __ldcg(p.X + ((size_t)u * m + jr) * m + l) : 0.f;
+      xv[i2] = (jr < m && l < m) ? p.X[((size_t)u * m + jr) * m + l] : 0.f;
     }
 #pragma unroll
-    for (int i2 = 0; i2 < 16; ++i2) {
+    for (int i2 = 0; i2 < kNX; ++i2) {
       const int e = t + kFT * i2;
       Xt[(e & 63) * kQS + (e >> 6)] = xv[i2];
+    }
+  }
+  int* wcount = reinterpret_cast<int*>(sm + kOffBp);
+  bool nonempty = false;
+  int rec_off = 0;
+  if (t < ncand) {
+    const int gg = gf + t;
+    const long long a = cta_start(gg, p, fa);
+    nonempty = cta_start(gg + 1, p, fa) > a;
+    rec_off = (gg * 2 + (a < (long long)u * N ? 1 : 0)) * kRec;
+  }
+  const unsigned bal = __ballot_sync(0xffffffffu, nonempty);
+  if ((t & 31) == 0) wcount[t >> 5] = __popc(bal);
+  __syncthreads();
+  int before = __popc(bal & ((1u << (t & 31)) - 1u)), nct = 0;
+  for (int i = 0; i < kWarps; ++i) {
+    if (i < (t >> 5)) before += wcount[i];
+    nct += wcount[i];
+  }
+  if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
+  nct = nct < kMaxContrib ? nct : kMaxContrib;
+  __syncthreads();
+  if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout);
+  __syncthreads();
+  trace_mark(p, 26);
+  // sum the unit's records: S1, S2 in fp64, P in fp32. Every load of a batch of 8 records
+  // (4 float4 of P per thread, plus one S value for threads < 128) is issued before any use.
+  {
+    constexpr int kNP = 1024 / kFT;   // float4 of P per thread
+    double sacc = 0.0;
+    float4 pacc[kNP];
+#pragma unroll
+    for (int i = 0; i < kNP; ++i) pacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < nct; c0 += 8) {
+      float sv[8];
+      float4 pv[8][kNP];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const bool ok = c0 + c < nct;
+        const float* r = fa.rec + (ok ? ctr[c0 + c] : 0);
+        sv[c] = (ok && t < 128) ? __ldcg(r + t) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kNP; ++i)
+          pv[c][i] = ok ? __ldcg(reinterpret_cast<const float4*>(r + 128) + t + kFT * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        sacc += (double)sv[c];
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) {
+          pacc[i].x += pv[c][i].x;
+          pacc[i].y += pv[c][i].y;
+          pacc[i].z += pv[c][i].z;
+          pacc[i].w += pv[c][i].w;
+        }
+      }
+    }
+    if (t < 64) S1d[t] = sacc;
+    else if (t < 128) S2d[t - 64] = sacc;
+    trace_mark(p, 28);
+#pragma unroll
+    for (int i = 0; i < kNP; ++i) {
+      const int e4 = t + kFT * i;
+      *reinterpret_cast<float4*>(As + (e4 >> 4) * kQS + 4 * (e4 & 15)) = pacc[i];
     }
   }
   __syncthreads();
@@ -880,7 +867,7 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
     mus[t] = t < m ? (float)mu : 0.f;
     scs[t] = t < m ? (float)sc : 0.f;
     svs[t] = As[63 * kQS + t];       // landmark column 63 holds sum_i v_i
-    if (g == gf && t < m) {
+    if (t < m) {
       p.mu[(size_t)u * m + t] = (float)mu;
       p.s[(size_t)u * m + t] = (float)sc;
     }
@@ -896,24 +883,25 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
     As[a * kQS + k] = v;
   }
   __syncthreads();
+  trace_mark(p, 29);
   {
-    // M = X A with a 4 x 4 register tile per thread; M' = diag(s) M (bf16, K-major B of pass 2)
+    // M = X A with a 2 x 4 register tile per thread; M' = diag(s) M as bf16 (K-major B of pass 2)
     const int jb = t >> 4, kb = t & 15;
-    float acc[4][4] = {};
+    float acc[2][4] = {};
     for (int l = 0; l < m; ++l) {
-      const float4 x4 = *reinterpret_cast<const float4*>(Xt + l * kQS + 4 * jb);
+      const float2 x2 = *reinterpret_cast<const float2*>(Xt + l * kQS + 2 * jb);
       const float4 a4 = *reinterpret_cast<const float4*>(As + l * kQS + 4 * kb);
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w}, av[4] = {a4.x, a4.y, a4.z, a4.w};
+      const float xv[2] = {x2.x, x2.y}, av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
+      for (int x = 0; x < 2; ++x)
 #pragma unroll
         for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(xv[x], av[y], acc[x][y]);
     }
     unsigned char* mp = sm + kOffMp;
     float bp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int jr = 4 * jb + x;
+    for (int x = 0; x < 2; ++x) {
+      const int jr = 2 * jb + x;
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
         const int k = 4 * kb + y;
@@ -929,19 +917,127 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
     for (int y = 0; y < 4; ++y) bps[jb * 64 + 4 * kb + y] = bp[y];
   }
   __syncthreads();
+  trace_mark(p, 30);
+  unsigned char* img = fa.mimg + (size_t)u * kImgBytes;
   if (t < 64) {
     float b = 0.f;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) b += bps[q * 64 + t];
-    bvec[t] = b;
+    for (int q = 0; q < kFT / 16; ++q) b += bps[q * 64 + t];
+    reinterpret_cast<float*>(img + 8192)[t] = b;
   }
-  fence_async_smem();
-  tc_fence_before();
+  for (int e = t; e < 512; e += kFT)
+    reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(sm + kOffMp)[e];
   __syncthreads();
-  trace_mark(p, 5 + 3 * s);
+  if (t == 0) {
+    __threadfence();
+    st_release_u64(fa.mready + u, fa.epoch);
+  }
+  trace_mark(p, 27);
+}
 
-  // phase 5: O = C M' + b + DWC(V); the DWC values are in O already (phase 1)
-  __nv_bfloat16* Ou = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * N * 64;
+// ---------------------------------------------------------------------------------------
+// Phase 3b (row CTAs, while the unit's M' is being formed): DWC(V) of every chunk -> O (bf16),
+// the 3 x 3 depthwise taps (§关键设计 1 "ZV + DWC(V)", zero padding 1). The chunk's V rows with a
+// one-grid-row halo on each side arrive by TMA (SW128, boxes of 128 rows, rows outside the unit
+// read as zero), two chunks in flight where both tiles fit. Thread t owns 4 consecutive tokens of
+// one grid row (W % 4 == 0, so a group never wraps) and 4 channels (t % 16), weights in registers,
+// and slides the 3 x 6 input window along the group.
+// ---------------------------------------------------------------------------------------
+__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV,
+                        int (&hc)[2]) {
+  const int t = threadIdx.x, W = p.W;
+  const int nbox = (kChunk + 2 * (W + 1) + kChunk - 1) / kChunk;
+  const uint32_t hbytes = (uint32_t)nbox * 16384u;
+  const int nbuf = 2 * hbytes <= kHaloSpace ? 2 : 1;
+  const int nch = R.nchunks;
+  auto issue = [&](int gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    const int bi = gc % nbuf;
+    uint64_t* hb = bars + kBarH + bi;
+    fence_async_smem();
+    mbar_expect_tx(hb, hbytes);
+    for (int b = 0; b < nbox; ++b)
+      tma_load_3d(sm + kOffHb + bi * hbytes + b * 16384, tmapV, 0, lo - (W + 1) + kChunk * b, R.seg[s].u, hb);
+  };
+  __syncthreads();   // pass 1 is done with the V stages, Q and L (the halo region)
+  if (t == 0) {
+    issue(0);
+    if (nbuf == 2 && nch > 1) issue(1);
+  }
+  const int grp = t >> 4, c4 = t & 15;   // tokens 4 grp .. 4 grp + 3 of the chunk, channels 4 c4 ..
+  float wt[9][4];
+  int head = -1;
+  for (int gc = 0; gc < nch; ++gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    const int u = R.seg[s].u;
+    if (u % p.heads != head) {
+      head = u % p.heads;
+#pragma unroll
+      for (int tap = 0; tap < 9; ++tap)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wt[tap][e] = __ldg(p.dwc + ((size_t)head * 64 + 4 * c4 + e) * 9 + tap);
+    }
+    const int bi = gc % nbuf;
+    mbar_wait(bars + kBarH + bi, hc[bi] & 1, p.status, kStatusTimeout);
+    const int r0 = 4 * grp;                // chunk row of the group's first token
+    if (r0 < nrows) {
+      const int n0 = lo + r0, x0 = n0 % W;
+      const unsigned char* hbuf = sm + kOffHb + bi * hbytes;
+      float acc[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        // tile rows of tokens x0 - 1 .. x0 + 4 on grid row y + a - 1: r0 + a W + j, j = 0..5
+        float v[6][4];
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+          const int tr = r0 + a * W + j;
+          const bool inside = (j > 0 || x0 > 0) && (j < 5 || x0 + 4 < W);
+          uint2 raw = make_uint2(0u, 0u);
+          if (inside)
+            raw = *reinterpret_cast<const uint2*>(hbuf + tr * 128 + ((((c4 >> 1) ^ (tr & 7))) << 4) + (c4 & 1) * 8);
+          v[j][0] = bf_lo(raw.x);
+          v[j][1] = bf_hi(raw.x);
+          v[j][2] = bf_lo(raw.y);
+          v[j][3] = bf_hi(raw.y);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int b = 0; b < 3; ++b)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(wt[a * 3 + b][e], v[i + b][e], acc[i][e]);
+      }
+      __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * p.N * 64 + 4 * c4;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (r0 + i < nrows)
+          *reinterpret_cast<uint2*>(O + (size_t)(n0 + i) * 64) =
+              make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
+    }
+    ++hc[bi];
+    __syncthreads();
+    if (t == 0 && gc + nbuf < nch) issue(gc + nbuf);
+  }
+  trace_mark(p, 25);
+}
+
+// ---------------------------------------------------------------------------------------
+// Phase 4 for one segment: O = C M' + b + DWC(V) per chunk. M'^T and b come from the unit's
+// solver CTA; the DWC values are already in O (phase 3b). The product of the next chunk is in
+// flight while the epilogue of this one runs (two TMEM accumulators).
+// ---------------------------------------------------------------------------------------
+__device__ void pass2_segment(const Params& p, const FusedArgs& fa, const Rows& R, int s, int& pc, unsigned char* sm,
+                              uint32_t sbase, uint32_t tmem, uint64_t* bars) {
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const Seg& sg = R.seg[s];
+  const int u = sg.u, nch = sg.nch;
+  float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   auto issue_o = [&](int gcc, int pcc) {
     tc_fence_after();
     const uint32_t id = idesc(1, 128, 64, 0, 0);
@@ -953,37 +1049,64 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
       mma_bf16(dt, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
     mma_commit(bars + kBarP2 + (pcc & 1));
   };
+  __syncthreads();   // the previous segment's products have read M'
+  if (t == 0) spin_until_geq(fa.mready + u, fa.epoch, p.status, kStatusTimeout);
+  __syncthreads();
+  trace_mark(p, 4 + 3 * s);
+  {
+    const unsigned char* img = fa.mimg + (size_t)u * kImgBytes;
+    for (int e = t; e < 512; e += kFT)
+      reinterpret_cast<uint4*>(sm + kOffMp)[e] = __ldcg(reinterpret_cast<const uint4*>(img) + e);
+    if (t < 64) bvec[t] = __ldcg(reinterpret_cast<const float*>(img + 8192) + t);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  trace_mark(p, 5 + 3 * s);
+  __nv_bfloat16* Ou = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * p.N * 64;
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
-  if (t == 0) issue_o(R.seg[s].first_chunk, pc);
-  for (int c = 0; c < R.seg[s].nch; ++c) {
-    const int gc = R.seg[s].first_chunk + c;
-    const int lo = R.seg[s].lo + c * kChunk;
-    const int nrows = min(kChunk, R.seg[s].hi - lo);
-    if (t == 0 && c + 1 < R.seg[s].nch) issue_o(gc + 1, pc + 1);
-    uint4 dw[4];
-    uint4* orow = reinterpret_cast<uint4*>(Ou + (size_t)(lo + row) * 64 + 32 * h);
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) dw[k4] = row < nrows ? orow[k4] : make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();
+  if (t == 0) issue_o(sg.first_chunk, pc);
+  // DWC values of a chunk's rows, loaded one chunk ahead of their use
+  auto fetch_dwc = [&](int c, uint4 (&dw)[2]) {
+    const int lo = sg.lo + c * kChunk;
+    dw[0] = dw[1] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < nch && row < min(kChunk, sg.hi - lo)) {
+      const uint4* src = reinterpret_cast<const uint4*>(Ou + (size_t)(lo + row) * 64 + 16 * h);
+      dw[0] = __ldcg(src);
+      dw[1] = __ldcg(src + 1);
+    }
+  };
+  uint4 dn[2];
+  fetch_dwc(0, dn);
+  for (int c = 0; c < nch; ++c) {
+    const int gc = sg.first_chunk + c;
+    const int lo = sg.lo + c * kChunk;
+    const int nrows = min(kChunk, sg.hi - lo);
+    if (t == 0 && c + 1 < nch) issue_o(gc + 1, pc + 1);
+    uint4* orow = reinterpret_cast<uint4*>(Ou + (size_t)(lo + row) * 64 + 16 * h);
+    const uint4 dw[2] = {dn[0], dn[1]};
+    fetch_dwc(c + 1, dn);
     mbar_wait(bars + kBarP2 + (pc & 1), (pc >> 1) & 1, p.status, kStatusTimeout);
+    if (s == 0 && c == 0) trace_mark(p, 29);
     tc_fence_after();
-    float v[32];
-    tmem_ld32(tmem + 128 + 64 * (pc & 1) + ((uint32_t)(32 * q) << 16) + 32 * h, v);
+    float v[16];
+    tmem_ld16(tmem + 128 + 64 * (pc & 1) + ((uint32_t)(32 * q) << 16) + 16 * h, v);
     if (row < nrows) {
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
+      for (int k4 = 0; k4 < 2; ++k4) {
         const uint32_t wv[4] = {dw[k4].x, dw[k4].y, dw[k4].z, dw[k4].w};
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int cc = 8 * k4 + 2 * e;
-          o[e] = pack_bf16(v[cc] + bvec[32 * h + cc] + bf_lo(wv[e]), v[cc + 1] + bvec[32 * h + cc + 1] + bf_hi(wv[e]));
+          o[e] = pack_bf16(v[cc] + bvec[16 * h + cc] + bf_lo(wv[e]), v[cc + 1] + bvec[16 * h + cc + 1] + bf_hi(wv[e]));
         }
         orow[k4] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
     tc_fence_before();
     __syncthreads();
+    if (s == 0 && c < 2) trace_mark(p, 30 + c);
     ++pc;
   }
   trace_mark(p, 6 + 3 * s);
@@ -991,13 +1114,13 @@ __device__ void combine_and_pass2(const Params& p, const FusedArgs& fa, const Ro
 
 __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const FusedArgs fa,
                                                            const __grid_constant__ CUtensorMap tmapV,
-                                                           const __grid_constant__ CUtensorMap tmapVp) {
+                                                           const __grid_constant__ CUtensorMap tmapQ) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + pad;
   const uint32_t sbase = smem_u32(sm);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 64);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + kTmemSlot);
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int g = blockIdx.x;
   const int U = p.U, N = p.N, m = p.m;
@@ -1010,17 +1133,14 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   }
   const Rows R = cta_rows(g, p, fa);
   const bool solver = g < U;
-  const HaloPlan hp = halo_plan(p, R);
   if (t == 0) {
-    for (int b = 0; b < 8; ++b) mbar_init(bars + b, 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, 1);
     mbar_init_fence();
     if (g == 0) *p.status = 0;
-    // V rows for this CTA's DWC: in flight while pooling runs (solver CTAs: after their solver)
-    if (!solver) dwc_issue(p, R, hp, sm, bars, &tmapVp);
   }
   if (t == 32) {
     tma_prefetch_desc(&tmapV);
-    tma_prefetch_desc(&tmapVp);
+    tma_prefetch_desc(&tmapQ);
   }
 
   // ---- phase 0: landmark pooling, one warp per landmark ----
@@ -1071,31 +1191,25 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     __threadfence();
     red_release_add_u64(fa.gbar, 1ull);
   }
-  // ---- phase 1: DWC of this CTA's rows while the barrier completes (solver CTAs: later) ----
-  if (!solver && hp.rows > 0) {
-    mbar_wait(bars + kBarDwc, 0, p.status, kStatusTimeout);
-    dwc_compute(p, R, hp, sm);
-  }
-  trace_mark(p, 25);
   if (t == 0) spin_until_geq(fa.gbar, fa.epoch * (unsigned long long)gridDim.x, p.status, kStatusTimeout);
   __syncthreads();
   trace_mark(p, 2);
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (solver) {
-    solver_cta(p, fa, sm, sbase, tmem, bars, g);
-    if (hp.rows > 0) {
-      if (t == 0) dwc_issue(p, R, hp, sm, bars, &tmapVp);
-      mbar_wait(bars + kBarDwc, 0, p.status, kStatusTimeout);
-      dwc_compute(p, R, hp, sm);
-    }
-  }
+  if (solver) solver_cta(p, fa, sm, sbase, tmem, bars, g);
   __syncthreads();
-  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
+  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV, &tmapQ);
   trace_mark(p, 3);
+  // the unit's combine runs on its solver CTA after this CTA's own records are out (no self-wait)
+  if (solver) {
+    __syncthreads();
+    solver_combine(p, fa, sm, g);
+  }
+  int hc[2] = {0, 0};
+  if (R.nchunks > 0) dwc_all(p, R, sm, bars, &tmapV, hc);
   int pc = 0;
-  for (int s = 0; s < R.nseg; ++s) combine_and_pass2(p, fa, R, s, pc, sm, sbase, tmem, bars);
+  for (int s = 0; s < R.nseg; ++s) pass2_segment(p, fa, R, s, pc, sm, sbase, tmem, bars);
   __syncthreads();
   trace_mark(p, 15);
   trace_clock(p, 14);
@@ -1107,9 +1221,13 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
 
 }  // namespace
 
+// Flag area: grid barrier (256 B), then three [U] flag arrays (cnt, xready, mready), each padded
+// to 256 B; then the per-CTA records and the per-unit M' images.
+static size_t flag_stride(int U) { return 256 * (size_t)((U * 8 + 255) / 256); }
+static size_t flag_bytes(int U) { return 256 + 3 * flag_stride(U); }
+
 size_t fused_workspace_bytes(int U) {
-  const size_t flags = 256 + 2 * 256 * (size_t)((U * 8 + 255) / 256);
-  return flags + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
+  return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * kImgBytes;
 }
 
 // Row share of a solver CTA (in 1/16 of a plain CTA's share): they start their rows only after
@@ -1138,32 +1256,28 @@ int fused_grid(const Params& p) {
   if (2 * p.U > G) return 0;
   const int ws16 = solver_share16();
   const long long totw16 = (long long)ws16 * p.U + 16ll * (G - p.U);
-  const long long T = (long long)p.U * p.N;
-  const long long rpc = (T * 16 + totw16 - 1) / totw16;           // rows of a plain CTA (rounded up)
-  if (rpc > (long long)(kMaxChunks - 1) * kChunk || rpc > p.N) return 0;
-  // replay the row partition: contributors of every unit must fit the offset table and every
-  // CTA's DWC rows (segments plus one-grid-row halos, rounded to TMA boxes) must fit the tile
+  // chunks of a plain CTA: resident C capacity, and at most two units (segments) per CTA
+  const long long nchu = (p.N + kChunk - 1) / kChunk;
+  const long long cpc = ((long long)p.U * nchu * 16 + totw16 - 1) / totw16;
+  if (cpc > kMaxChunks - 1 || cpc > nchu) return 0;   // one C slot stays free for the Q chunk
+  // the DWC phase's token groups of 4 stay on one grid row
+  if (p.W % 4 != 0) return 0;
+  // its V halo tile (a chunk plus one grid row on each side, in boxes of 128 rows) must fit
+  if ((long long)((kChunk + 2 * (p.W + 1) + kChunk - 1) / kChunk) * 16384 > (long long)kHaloSpace) return 0;
+  // replay the row partition: contributors of every unit must fit the offset table
   {
     int worst = 0, cur_u = -1, cur = 0;
     for (int g = 0; g < G; ++g) {
-      const long long cw0 = g <= p.U ? (long long)ws16 * g : (long long)ws16 * p.U + 16ll * (g - p.U);
-      const long long cw1 = g + 1 <= p.U ? (long long)ws16 * (g + 1) : (long long)ws16 * p.U + 16ll * (g + 1 - p.U);
-      const long long r0 = T * cw0 / totw16, r1 = T * cw1 / totw16;
+      const long long r0 = part_start(g, p.U, p.N, ws16, totw16);
+      const long long r1 = part_start(g + 1, p.U, p.N, ws16, totw16);
       if (r1 <= r0) continue;
-      long long halo_rows = 0;
       for (long long u = r0 / p.N; u <= (r1 - 1) / p.N; ++u) {
         if ((int)u != cur_u) {
           cur_u = (int)u;
           cur = 0;
         }
         if (++cur > worst) worst = cur;
-        const long long lo = (r0 > u * p.N ? r0 : u * p.N) - u * p.N;
-        const long long hi = (r1 < (u + 1) * p.N ? r1 : (u + 1) * p.N) - u * p.N;
-        const long long hlo = lo - p.W - 1 > 0 ? lo - p.W - 1 : 0;
-        const long long hhi = hi + p.W + 1 < p.N ? hi + p.W + 1 : p.N;
-        halo_rows += (hhi - hlo + kChunk - 1) / kChunk * kChunk;
       }
-      if (halo_rows > kHaloRows) return 0;
     }
     if (worst > kMaxContrib) return 0;
   }
@@ -1179,54 +1293,57 @@ int fused_grid(const Params& p) {
 
 // Tensor maps of recently used V pointers (host side; encoding costs a driver call).
 struct TmapCache {
-  const void* ptr[8];
-  int N[8], U[8];
-  CUtensorMap map[8], plain[8];
+  const void* ptr[16];
+  int N[16], U[16], sw[16];
+  CUtensorMap map[16];
   int next;
 };
 static TmapCache g_tmaps;
+static std::mutex g_tmaps_mu;
 
-static bool tmap_for(const void* V, int N, int U, CUtensorMap* out, CUtensorMap* out_plain) {
-  for (int i = 0; i < 8; ++i)
-    if (g_tmaps.ptr[i] == V && g_tmaps.N[i] == N && g_tmaps.U[i] == U) {
+// [U][N][64] bf16 viewed as {64, N, U}, boxes of 128 rows; 128-byte swizzle or plain rows
+static bool tmap_for(const void* X, int N, int U, bool swizzle, CUtensorMap* out) {
+  std::lock_guard<std::mutex> lk(g_tmaps_mu);
+  for (int i = 0; i < 16; ++i)
+    if (g_tmaps.ptr[i] == X && g_tmaps.N[i] == N && g_tmaps.U[i] == U && g_tmaps.sw[i] == (int)swizzle) {
       *out = g_tmaps.map[i];
-      *out_plain = g_tmaps.plain[i];
       return true;
     }
-  CUtensorMap m, mp;
-  if (!make_tmap_rows_bf16(&m, V, (uint64_t)N, (uint64_t)U, kChunk, true)) return false;
-  if (!make_tmap_rows_bf16(&mp, V, (uint64_t)N, (uint64_t)U, kChunk, false)) return false;
+  CUtensorMap m;
+  if (!make_tmap_rows_bf16(&m, X, (uint64_t)N, (uint64_t)U, kChunk, swizzle)) return false;
   const int i = g_tmaps.next;
-  g_tmaps.next = (i + 1) & 7;
-  g_tmaps.ptr[i] = V;
+  g_tmaps.next = (i + 1) & 15;
+  g_tmaps.ptr[i] = X;
   g_tmaps.N[i] = N;
   g_tmaps.U[i] = U;
+  g_tmaps.sw[i] = (int)swizzle;
   g_tmaps.map[i] = m;
-  g_tmaps.plain[i] = mp;
   *out = m;
-  *out_plain = mp;
   return true;
 }
 
 cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws, unsigned long long epoch,
                                  cudaStream_t st) {
   if (epoch == 1) {
-    const cudaError_t e = cudaMemsetAsync(fused_ws, 0, 256 + 2 * 256 * (size_t)((p.U * 8 + 255) / 256), st);
+    const cudaError_t e = cudaMemsetAsync(fused_ws, 0, flag_bytes(p.U), st);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tmap, tmapp;
-  if (!tmap_for(p.V, p.N, p.U, &tmap, &tmapp)) return cudaErrorInvalidValue;
+  CUtensorMap tmap, tmapq;
+  if (!tmap_for(p.V, p.N, p.U, true, &tmap)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.Q, p.N, p.U, false, &tmapq)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.epoch = epoch;
   fa.ws16 = solver_share16();
   fa.totw16 = fa.ws16 * p.U + 16 * (G - p.U);
   fa.gbar = reinterpret_cast<unsigned long long*>(fused_ws);
-  const size_t flag_stride = 256 * (size_t)((p.U * 8 + 255) / 256);
+  const size_t fs = flag_stride(p.U);
   fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + 256);
-  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + flag_stride);
-  fa.rec = reinterpret_cast<float*>(fused_ws + 256 + 2 * flag_stride);
+  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + fs);
+  fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + 2 * fs);
+  fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
+  fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
   Params pp = p;
-  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapp};
+  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq};
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
   cudaError_t e = cudaLaunchCooperativeKernel((const void*)k_fused_forward, dim3(G), dim3(kFT), args, kSmemAlloc, st);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
