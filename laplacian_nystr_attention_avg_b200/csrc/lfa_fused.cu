@@ -24,7 +24,8 @@
 //   phase 3b row CTAs, while M' is formed: DWC(V) (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise,
 //            zero padding) of every chunk from a TMA-staged V tile with a one-grid-row halo,
 //            written to O as bf16.
-//   phase 4  row CTAs, per chunk: O = C M' (tcgen05, TMEM accumulator) + b + the DWC values.
+//   phase 4  row CTAs: O = C M' (tcgen05; all chunks' products at once, one TMEM accumulator each)
+//            + b + the DWC values.
 // Every cross-CTA wait is bounded; an expired wait sets the timeout bit of the status word.
 #include <stdlib.h>
 #include <string.h>
@@ -52,16 +53,17 @@ constexpr int kPowerIters = 8;
 
 // shared-memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kOffC = 0;                                   // 8 x 16 KB C chunks (SW128 rows)
-constexpr uint32_t kOffV = kOffC + kMaxChunks * 16384;          // 2 x 16 KB V stages (TMA, SW128)
-constexpr uint32_t kOffQ = kOffV + 2 * 16384;                   // Q chunk, fp32 [128][68]
+constexpr uint32_t kOffV = kOffC + kMaxChunks * 16384;          // 3 x 16 KB V stages (TMA, SW128)
+constexpr uint32_t kOffQ = kOffV + 2 * 16384;                   // third V stage + 18 KB spare in pass 1
 constexpr uint32_t kOffL = kOffQ + kChunk * kQS * 4;            // landmarks, fp32 [64][68]
 constexpr uint32_t kOffMp = kOffL + 64 * kQS * 4;               // M'^T bf16 [64 ch][64 lm] (SW128)
-constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [64]
-constexpr uint32_t kOffBar = kOffBv + 256;                      // mbarriers + TMEM address
-constexpr uint32_t kOffCt = kOffBar + 128;                      // int [32] record offsets
+constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [segment][64]
+constexpr uint32_t kOffBar = kOffBv + 512;                      // mbarriers + TMEM address
+constexpr uint32_t kOffCt = kOffBar + 256;                      // int [32] record offsets
 constexpr uint32_t kOffWd = kOffCt + 128;                       // DWC weights fp32 [9 taps][64 ch]
 constexpr uint32_t kOffSr = kOffWd + 9 * 64 * 4;                // pass-1 column sums [segment][row half][128]
-constexpr uint32_t kSmemBytes = kOffSr + 2 * 256 * 4;
+constexpr uint32_t kOffRows = kOffSr + 2 * 256 * 4;            // this CTA's row plan (struct Rows)
+constexpr uint32_t kSmemBytes = kOffRows + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
 // pass-2 scratch: V rows of one chunk with a one-grid-row halo on each side, SW128 (TMA boxes of
 // 128 rows), one or two buffers in the region of the V stages, Q and L (free after pass 1)
@@ -90,14 +92,16 @@ static_assert(kOffBp + (kFT / 16) * 64 * 4 <= kOffMp, "combine scratch overlaps 
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
-constexpr int kBarV = 0;      // [2] V stage filled by TMA
-constexpr int kBarP1 = 2;     // [2] pass-1 product done (stage free)
-constexpr int kBarP2 = 4;     // [2] pass-2 product done (accumulator ready)
-constexpr int kBarNs = 6;     // solver product done
-constexpr int kBarH = 8;      // [2] DWC V halo tile landed (TMA)
-constexpr int kBarQ = 10;     // pass-1 Q chunk landed (TMA, bf16 rows in the spare C slot)
-constexpr int kNumBars = 11;
-constexpr uint32_t kTmemSlot = 96;   // byte offset of the TMEM address within the barrier area
+constexpr int kBarV = 0;      // [3] V stage filled by TMA
+constexpr int kBarP1 = 3;     // [2] pass-1 product done
+constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (one use per launch)
+constexpr int kBarNs = 13;    // solver product done
+constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
+constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
+constexpr int kNumBars = 17;
+constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
+constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
+static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
 
 struct FusedArgs {
   unsigned long long epoch;   // launch count of this handle (>= 1); flags compare against it
@@ -496,8 +500,10 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
 // ---------------------------------------------------------------------------------------
 // Phase 3: C for a 128-row chunk: this warp's landmarks [j0, j0 + LT), lane rows lane + 32 a.
 // ---------------------------------------------------------------------------------------
+// Q rows come from a bf16 SW128 tile (TMA): one 16-byte read gives 8 channels of a row, and the
+// lanes' rows spread the reads over all banks.
 template <int LT>
-__device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, unsigned char* cslot, int j0,
+__device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float* Ls, unsigned char* cslot, int j0,
                                             int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
   const int lane = threadIdx.x & 31;
   float acc[2][LT];
@@ -506,23 +512,32 @@ __device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, un
 #pragma unroll
     for (int b = 0; b < LT; ++b) acc[a][b] = 0.f;
 #pragma unroll 2
-  for (int k = 0; k < 64; k += 4) {
-    float4 q[2], l[LT];
+  for (int k8 = 0; k8 < 8; ++k8) {
+    float q[2][8];
 #pragma unroll
-    for (int a = 0; a < 2; ++a) q[a] = *reinterpret_cast<const float4*>(&Qs[(rb + lane + 32 * a) * kQS + k]);
+    for (int a = 0; a < 2; ++a) {
+      const int r = rb + lane + 32 * a;
+      const uint4 raw = *reinterpret_cast<const uint4*>(qb + sw128(r, k8));
+      q[a][0] = bf_lo(raw.x); q[a][1] = bf_hi(raw.x); q[a][2] = bf_lo(raw.y); q[a][3] = bf_hi(raw.y);
+      q[a][4] = bf_lo(raw.z); q[a][5] = bf_hi(raw.z); q[a][6] = bf_lo(raw.w); q[a][7] = bf_hi(raw.w);
+    }
 #pragma unroll
-    for (int b = 0; b < LT; ++b) l[b] = *reinterpret_cast<const float4*>(&Ls[(j0 + b) * kQS + k]);
+    for (int h4 = 0; h4 < 2; ++h4) {
+      float4 l[LT];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+      for (int b = 0; b < LT; ++b) l[b] = *reinterpret_cast<const float4*>(&Ls[(j0 + b) * kQS + 8 * k8 + 4 * h4]);
 #pragma unroll
-      for (int b = 0; b < LT; ++b) {
-        float s = acc[a][b];
-        s += fabsf(q[a].x - l[b].x);
-        s += fabsf(q[a].y - l[b].y);
-        s += fabsf(q[a].z - l[b].z);
-        s += fabsf(q[a].w - l[b].w);
-        acc[a][b] = s;
-      }
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < LT; ++b) {
+          float s = acc[a][b];
+          s += fabsf(q[a][4 * h4 + 0] - l[b].x);
+          s += fabsf(q[a][4 * h4 + 1] - l[b].y);
+          s += fabsf(q[a][4 * h4 + 2] - l[b].z);
+          s += fabsf(q[a][4 * h4 + 3] - l[b].w);
+          acc[a][b] = s;
+        }
+    }
   }
   const bool even = (j0 & 1) == 0;
 #pragma unroll
@@ -555,7 +570,7 @@ __device__ __forceinline__ void cross_chunk(const float* Qs, const float* Ls, un
   }
 }
 
-__device__ __forceinline__ void cross_dispatch(int lt, const float* Qs, const float* Ls, unsigned char* cslot,
+__device__ __forceinline__ void cross_dispatch(int lt, const unsigned char* Qs, const float* Ls, unsigned char* cslot,
                                                int j0, int rb, int nrows, float scale, float (&s1)[8],
                                                float (&s2)[8]) {
   switch (lt) {
@@ -571,29 +586,31 @@ __device__ __forceinline__ void cross_dispatch(int lt, const float* Qs, const fl
   }
 }
 
-// Q rows of a chunk, bf16 [128][64] plain rows (TMA) -> fp32 [128][kQS]: thread t converts row
-// t/4, 16 channels (t % 4); rows at or past nrows become zero.
-__device__ __forceinline__ void q_stage(float* Qs, const unsigned char* qsrc, int nrows) {
-  const int t = threadIdx.x, row = t >> 2, qt = t & 3;
-  float* dst = Qs + row * kQS + 16 * qt;
-  uint4 qr[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-    qr[k] = row < nrows ? reinterpret_cast<const uint4*>(qsrc + row * 128 + 32 * qt)[k] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const uint4 v = qr[k];
-    *reinterpret_cast<float4*>(dst + 8 * k) = make_float4(bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y));
-    *reinterpret_cast<float4*>(dst + 8 * k + 4) = make_float4(bf_lo(v.z), bf_hi(v.z), bf_lo(v.w), bf_hi(v.w));
+// Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
+// (bf16, SW128) goes to C slot gc + 1 (chunk gc writes its C tile into slot gc, which held the
+// previous chunk's rows), one barrier for all of them; the first two V chunks go to stages 0, 1.
+__device__ void pass1_prefetch(const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV,
+                               const CUtensorMap* tmapQ) {
+  const int nch = R.nchunks;
+  if (nch == 0) return;
+  mbar_expect_tx(bars + kBarQ, (uint32_t)nch * 16384u);
+  for (int gc = 0; gc < nch; ++gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    tma_load_3d(sm + kOffC + (gc + 1) * 16384, tmapQ, 0, lo, R.seg[s].u, bars + kBarQ);
+  }
+  for (int gc = 0; gc < nch && gc < 2; ++gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    mbar_expect_tx(bars + kBarV + gc, 16384);
+    tma_load_3d(sm + kOffV + gc * 16384, tmapV, 0, lo, R.seg[s].u, bars + kBarV + gc);
   }
 }
 
 __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
-                      uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapV, const CUtensorMap* tmapQ) {
+                      uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapV) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31, g = blockIdx.x;
   const int m = p.m, nch = R.nchunks;
-  unsigned char* qslot = sm + kOffC + nch * 16384;       // spare C slot (nch < kMaxChunks)
-  float* Qs = reinterpret_cast<float*>(sm + kOffQ);
   float* Ls = reinterpret_cast<float*>(sm + kOffL);
   float* sred = reinterpret_cast<float*>(sm + kOffSr);   // [segment][row half][S1 64 | S2 64]
   // Landmark groups: warps w and w + 8 share group w % 8 (rows 0-63 and 64-127). The groups
@@ -622,51 +639,48 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     }
   }
   const float scale = p.neg_log2e_over_lam;
+  // V chunk gc -> stage gc % 3 (its (gc / 3)-th fill)
   auto issue_v = [&](int gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    uint64_t* fb = bars + kBarV + (gc & 1);
+    uint64_t* fb = bars + kBarV + gc % 3;
     mbar_expect_tx(fb, 16384);
-    tma_load_3d(sm + kOffV + (gc & 1) * 16384, tmapV, 0, lo, R.seg[s].u, fb);
+    tma_load_3d(sm + kOffV + (gc % 3) * 16384, tmapV, 0, lo, R.seg[s].u, fb);
   };
   // P_s += C^T V for chunk gc (M = 64 landmarks, N = 64 channels, K = 128 rows)
   auto issue_mma = [&](int gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
     const bool first = gc == R.seg[s].first_chunk;
-    mbar_wait(bars + kBarV + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
+    mbar_wait(bars + kBarV + gc % 3, (gc / 3) & 1, p.status, kStatusTimeout);
     tc_fence_after();
     const uint32_t id = idesc(1, 64, 64, 1, 1);
     const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 8192, 1024);
-    const uint64_t va = desc_sw128(sbase + kOffV + (gc & 1) * 16384, 8192, 1024);
+    const uint64_t va = desc_sw128(sbase + kOffV + (gc % 3) * 16384, 8192, 1024);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
       mma_bf16(tmem + 64 * s, ca + (uint64_t)(kk * 2048 >> 4), va + (uint64_t)(kk * 2048 >> 4), id,
                (!first || kk > 0) ? 1u : 0u);
     mma_commit(bars + kBarP1 + (gc & 1));
   };
-  auto issue_q = [&](int gc) {
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    mbar_expect_tx(bars + kBarQ, 16384);
-    tma_load_3d(qslot, tmapQ, 0, lo, R.seg[s].u, bars + kBarQ);
+  // product gc done (commit gc on slot gc & 1 is that slot's (gc >> 1)-th completion)
+  auto wait_mma = [&](int gc) {
+    mbar_wait(bars + kBarP1 + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
   };
-  if (t == 0) {
-    fence_async_smem();
-    issue_q(0);
-    issue_v(0);
-    if (nch > 1) issue_v(1);
-  }
   trace_mark(p, 28);
   float s1[8], s2[8];
   for (int gc = 0; gc < nch; ++gc) {
+    if (gc == 1) trace_mark(p, 24);
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
     const int u = R.seg[s].u;
     const bool seg_first = gc == R.seg[s].first_chunk;
     const bool seg_last = gc == R.seg[s].first_chunk + R.seg[s].nch - 1;
     unsigned char* cslot = sm + kOffC + gc * 16384;
-    // Qs and Ls were last read before the previous chunk's closing barrier
+    if (gc == 1) trace_mark(p, 27);
+    // products run two chunks behind: tile gc - 2 is complete and its V stage has had a chunk
+    if (t == 0 && gc >= 2) issue_mma(gc - 2);
+    // Ls was last read before the previous chunk's closing barrier
     if (seg_first) {
       load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
 #pragma unroll
@@ -674,10 +688,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
         s1[b] = 0.f;
         s2[b] = 0.f;
       }
+      __syncthreads();
     }
-    mbar_wait(bars + kBarQ, gc & 1, p.status, kStatusTimeout);
-    if (gc < 2) trace_mark(p, 27 - 3 * gc);
-    q_stage(Qs, qslot, nrows);
     // padding landmark columns m..63: zero, except column 63 = 1 on valid rows (sum of V)
     for (int e = t; e < kChunk * (64 - m); e += kFT) {
       const int row = e / (64 - m), col = m + e % (64 - m);
@@ -685,17 +697,9 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
       *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = __float2bfloat16_rn(v);
     }
     if (gc == 1) trace_mark(p, 26);
-    __syncthreads();
-    // the spare slot has been converted: the next chunk's Q rows are fetched during this one
-    if (t == 0 && gc + 1 < nch) {
-      fence_async_smem();
-      issue_q(gc + 1);
-    }
+    if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
-    // the previous chunk's C tile is complete (closing barrier): its product goes out now,
-    // overlapping this chunk's distances
-    if (t == 0 && gc >= 1) issue_mma(gc - 1);
-    if (lt > 0) cross_dispatch(lt, Qs, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
+    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
     if (gc == 1) trace_mark(p, 22);
     if (seg_last) {
       // this segment's column sums of C and C^2, per row half
@@ -712,23 +716,29 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
         }
       }
     }
-    // V stage (gc + 1) & 1 was read by the product of chunk gc - 1, issued at this chunk's start
+    // the next V chunk, while the SM idles at the barrier: stage (gc + 1) % 3 last held chunk
+    // gc - 2, whose product was issued at this chunk's start
     if (t == 0 && gc >= 1 && gc + 1 < nch) {
-      mbar_wait(bars + kBarP1 + ((gc - 1) & 1), ((gc - 1) >> 1) & 1, p.status, kStatusTimeout);
+      if (gc >= 2) wait_mma(gc - 2);
       issue_v(gc + 1);
     }
+    if (gc == 1) trace_mark(p, 20);
     fence_async_smem();
+    if (gc == 1) trace_mark(p, 23);
     tc_fence_before();
     __syncthreads();
     if (gc < 2) trace_mark(p, 11 + gc);
   }
-  // last chunk's product, then the records: S1, S2 and P (TMEM columns 64 s) per segment
+  // the last two products, each waited before the next one on its commit slot goes out
   if (t == 0) {
+    if (nch >= 2) issue_mma(nch - 2);
+    if (nch >= 3) wait_mma(nch - 3);
     issue_mma(nch - 1);
-    if (nch >= 2) mbar_wait(bars + kBarP1 + ((nch - 2) & 1), ((nch - 2) >> 1) & 1, p.status, kStatusTimeout);
+    if (nch >= 2) wait_mma(nch - 2);
   }
-  mbar_wait(bars + kBarP1 + ((nch - 1) & 1), ((nch - 1) >> 1) & 1, p.status, kStatusTimeout);
+  wait_mma(nch - 1);
   tc_fence_after();
+  // records: S1, S2 and P (TMEM columns 64 s) per segment
   for (int s = 0; s < R.nseg; ++s) {
     float* rec = fa.rec + ((size_t)g * 2 + s) * kRec;
     if (w < 4) {
@@ -943,8 +953,7 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
 // one grid row (W % 4 == 0, so a group never wraps) and 4 channels (t % 16), weights in registers,
 // and slides the 3 x 6 input window along the group.
 // ---------------------------------------------------------------------------------------
-__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV,
-                        int (&hc)[2]) {
+__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV) {
   const int t = threadIdx.x, W = p.W;
   const int nbox = (kChunk + 2 * (W + 1) + kChunk - 1) / kChunk;
   const uint32_t hbytes = (uint32_t)nbox * 16384u;
@@ -955,7 +964,6 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
     R.chunk(gc, s, lo, nrows);
     const int bi = gc % nbuf;
     uint64_t* hb = bars + kBarH + bi;
-    fence_async_smem();
     mbar_expect_tx(hb, hbytes);
     for (int b = 0; b < nbox; ++b)
       tma_load_3d(sm + kOffHb + bi * hbytes + b * 16384, tmapV, 0, lo - (W + 1) + kChunk * b, R.seg[s].u, hb);
@@ -980,7 +988,7 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
         for (int e = 0; e < 4; ++e) wt[tap][e] = __ldg(p.dwc + ((size_t)head * 64 + 4 * c4 + e) * 9 + tap);
     }
     const int bi = gc % nbuf;
-    mbar_wait(bars + kBarH + bi, hc[bi] & 1, p.status, kStatusTimeout);
+    mbar_wait(bars + kBarH + bi, (gc / nbuf) & 1, p.status, kStatusTimeout);   // fill gc / nbuf of buffer bi
     const int r0 = 4 * grp;                // chunk row of the group's first token
     if (r0 < nrows) {
       const int n0 = lo + r0, x0 = n0 % W;
@@ -1020,7 +1028,6 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
           *reinterpret_cast<uint2*>(O + (size_t)(n0 + i) * 64) =
               make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
     }
-    ++hc[bi];
     __syncthreads();
     if (t == 0 && gc + nbuf < nch) issue(gc + nbuf);
   }
@@ -1028,70 +1035,77 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 4 for one segment: O = C M' + b + DWC(V) per chunk. M'^T and b come from the unit's
-// solver CTA; the DWC values are already in O (phase 3b). The product of the next chunk is in
-// flight while the epilogue of this one runs (two TMEM accumulators).
+// Phase 4: O = C M' + b + DWC(V) for every chunk. M'^T and b of each segment's unit come from
+// its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region); the DWC
+// values are already in O (phase 3b). All products are issued at once, each chunk into its own
+// 64-column TMEM accumulator with its own barrier, and the epilogues follow chunk by chunk.
 // ---------------------------------------------------------------------------------------
-__device__ void pass2_segment(const Params& p, const FusedArgs& fa, const Rows& R, int s, int& pc, unsigned char* sm,
-                              uint32_t sbase, uint32_t tmem, uint64_t* bars) {
+__device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
+                          uint32_t tmem, uint64_t* bars) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-  const Seg& sg = R.seg[s];
-  const int u = sg.u, nch = sg.nch;
+  const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
-  auto issue_o = [&](int gcc, int pcc) {
-    tc_fence_after();
-    const uint32_t id = idesc(1, 128, 64, 0, 0);
-    const uint64_t ca = desc_sw128(sbase + kOffC + gcc * 16384, 16, 1024);
-    const uint64_t mb = desc_sw128(sbase + kOffMp, 16, 1024);
-    const uint32_t dt = tmem + 128 + 64 * (pcc & 1);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(dt, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
-    mma_commit(bars + kBarP2 + (pcc & 1));
-  };
-  __syncthreads();   // the previous segment's products have read M'
-  if (t == 0) spin_until_geq(fa.mready + u, fa.epoch, p.status, kStatusTimeout);
+  auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffV; };
+  __syncthreads();   // the DWC phase is done with the halo region
+  if (t == 0)
+    for (int s = 0; s < R.nseg; ++s) spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout);
   __syncthreads();
-  trace_mark(p, 4 + 3 * s);
-  {
-    const unsigned char* img = fa.mimg + (size_t)u * kImgBytes;
+  trace_mark(p, 4);
+  for (int s = 0; s < R.nseg; ++s) {
+    const unsigned char* img = fa.mimg + (size_t)R.seg[s].u * kImgBytes;
     for (int e = t; e < 512; e += kFT)
-      reinterpret_cast<uint4*>(sm + kOffMp)[e] = __ldcg(reinterpret_cast<const uint4*>(img) + e);
-    if (t < 64) bvec[t] = __ldcg(reinterpret_cast<const float*>(img + 8192) + t);
+      reinterpret_cast<uint4*>(sm + img_off(s))[e] = __ldcg(reinterpret_cast<const uint4*>(img) + e);
+    if (t < 64) bvec[64 * s + t] = __ldcg(reinterpret_cast<const float*>(img + 8192) + t);
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  trace_mark(p, 5 + 3 * s);
-  __nv_bfloat16* Ou = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * p.N * 64;
+  trace_mark(p, 5);
+  if (t == 0) {
+    tc_fence_after();
+    const uint32_t id = idesc(1, 128, 64, 0, 0);
+    for (int gc = 0; gc < nch; ++gc) {
+      int s, lo, nrows;
+      R.chunk(gc, s, lo, nrows);
+      const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
+      const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
+      mma_commit(bars + kBarP2 + gc);
+    }
+  }
+  __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
-  if (t == 0) issue_o(sg.first_chunk, pc);
   // DWC values of a chunk's rows, loaded one chunk ahead of their use
-  auto fetch_dwc = [&](int c, uint4 (&dw)[2]) {
-    const int lo = sg.lo + c * kChunk;
+  auto fetch_dwc = [&](int gc, uint4 (&dw)[2]) {
     dw[0] = dw[1] = make_uint4(0u, 0u, 0u, 0u);
-    if (c < nch && row < min(kChunk, sg.hi - lo)) {
-      const uint4* src = reinterpret_cast<const uint4*>(Ou + (size_t)(lo + row) * 64 + 16 * h);
-      dw[0] = __ldcg(src);
-      dw[1] = __ldcg(src + 1);
+    if (gc < nch) {
+      int s, lo, nrows;
+      R.chunk(gc, s, lo, nrows);
+      if (row < nrows) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(O + ((size_t)R.seg[s].u * p.N + lo + row) * 64 + 16 * h);
+        dw[0] = __ldcg(src);
+        dw[1] = __ldcg(src + 1);
+      }
     }
   };
   uint4 dn[2];
   fetch_dwc(0, dn);
-  for (int c = 0; c < nch; ++c) {
-    const int gc = sg.first_chunk + c;
-    const int lo = sg.lo + c * kChunk;
-    const int nrows = min(kChunk, sg.hi - lo);
-    if (t == 0 && c + 1 < nch) issue_o(gc + 1, pc + 1);
-    uint4* orow = reinterpret_cast<uint4*>(Ou + (size_t)(lo + row) * 64 + 16 * h);
+  for (int gc = 0; gc < nch; ++gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
     const uint4 dw[2] = {dn[0], dn[1]};
-    fetch_dwc(c + 1, dn);
-    mbar_wait(bars + kBarP2 + (pc & 1), (pc >> 1) & 1, p.status, kStatusTimeout);
-    if (s == 0 && c == 0) trace_mark(p, 29);
+    fetch_dwc(gc + 1, dn);
+    mbar_wait(bars + kBarP2 + gc, 0, p.status, kStatusTimeout);
+    if (gc == 0) trace_mark(p, 29);
     tc_fence_after();
     float v[16];
-    tmem_ld16(tmem + 128 + 64 * (pc & 1) + ((uint32_t)(32 * q) << 16) + 16 * h, v);
+    tmem_ld16(tmem + 64 * gc + ((uint32_t)(32 * q) << 16) + 16 * h, v);
     if (row < nrows) {
+      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)R.seg[s].u * p.N + lo + row) * 64 + 16 * h);
+      const float* bs = bvec + 64 * s + 16 * h;
 #pragma unroll
       for (int k4 = 0; k4 < 2; ++k4) {
         const uint32_t wv[4] = {dw[k4].x, dw[k4].y, dw[k4].z, dw[k4].w};
@@ -1099,17 +1113,16 @@ __device__ void pass2_segment(const Params& p, const FusedArgs& fa, const Rows& 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int cc = 8 * k4 + 2 * e;
-          o[e] = pack_bf16(v[cc] + bvec[16 * h + cc] + bf_lo(wv[e]), v[cc + 1] + bvec[16 * h + cc + 1] + bf_hi(wv[e]));
+          o[e] = pack_bf16(v[cc] + bs[cc] + bf_lo(wv[e]), v[cc + 1] + bs[cc + 1] + bf_hi(wv[e]));
         }
         orow[k4] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (s == 0 && c < 2) trace_mark(p, 30 + c);
-    ++pc;
+    if (gc < 2) trace_mark(p, 30 + gc);
   }
-  trace_mark(p, 6 + 3 * s);
+  tc_fence_before();
+  __syncthreads();
+  trace_mark(p, 6);
 }
 
 __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const FusedArgs fa,
@@ -1128,15 +1141,19 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   trace_mark(p, 0);
   trace_clock(p, 13);
   if (w == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  const Rows R = cta_rows(g, p, fa);
+  // the row plan lives in shared memory: it is read at every chunk boundary by every thread
+  Rows* Rsm = reinterpret_cast<Rows*>(sm + kOffRows);
+  if (t == 0) *Rsm = cta_rows(g, p, fa);
+  const Rows& R = *Rsm;
   const bool solver = g < U;
   if (t == 0) {
     for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, 1);
     mbar_init_fence();
     if (g == 0) *p.status = 0;
+    if (!solver) pass1_prefetch(R, sm, bars, &tmapV, &tmapQ);
   }
   if (t == 32) {
     tma_prefetch_desc(&tmapV);
@@ -1197,25 +1214,27 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (solver) solver_cta(p, fa, sm, sbase, tmem, bars, g);
+  if (solver) {
+    solver_cta(p, fa, sm, sbase, tmem, bars, g);
+    __syncthreads();   // the solver's scratch in the C region is free
+    if (t == 0) pass1_prefetch(R, sm, bars, &tmapV, &tmapQ);
+  }
   __syncthreads();
-  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV, &tmapQ);
+  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
   trace_mark(p, 3);
   // the unit's combine runs on its solver CTA after this CTA's own records are out (no self-wait)
   if (solver) {
     __syncthreads();
     solver_combine(p, fa, sm, g);
   }
-  int hc[2] = {0, 0};
-  if (R.nchunks > 0) dwc_all(p, R, sm, bars, &tmapV, hc);
-  int pc = 0;
-  for (int s = 0; s < R.nseg; ++s) pass2_segment(p, fa, R, s, pc, sm, sbase, tmem, bars);
+  if (R.nchunks > 0) dwc_all(p, R, sm, bars, &tmapV);
+  if (R.nchunks > 0) pass2_all(p, fa, R, sm, sbase, tmem, bars);
   __syncthreads();
   trace_mark(p, 15);
   trace_clock(p, 14);
   if (w == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -1330,7 +1349,7 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   }
   CUtensorMap tmap, tmapq;
   if (!tmap_for(p.V, p.N, p.U, true, &tmap)) return cudaErrorInvalidValue;
-  if (!tmap_for(p.Q, p.N, p.U, false, &tmapq)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.Q, p.N, p.U, true, &tmapq)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.epoch = epoch;
   fa.ws16 = solver_share16();
