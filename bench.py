@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="approximate CPU work of the oracle baseline sample")
+    ap.add_argument("--backward", action="store_true",
+                    help="time forward + backward steps instead (1 GPU; e.g. --workload long)")
     return ap.parse_args()
 
 
@@ -185,10 +187,55 @@ def cpu_baseline(wl, x, seconds):
                       f"float64 numpy, {dt:.1f} s"}
 
 
+def run_backward(args):
+    """Secondary measurement: one step = lfa_forward + lfa_backward (dQ, dV) on resident inputs."""
+    import torch
+
+    from laplacian_nystr_attention_avg_b200 import lfa
+    from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, make_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = WORKLOADS[args.workload]
+    x = make_inputs(wl, with_dO=True)
+    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl), x.dwc, str(dev))
+    Q, V, dO = x.Q_store.to(dev), x.V_store.to(dev), x.dO_store.to(dev)
+    O, dQ, dV = mod.new_output(), mod.new_output(), mod.new_output()
+    for _ in range(args.warmup):
+        mod.forward(Q, V, O)
+        mod.backward(Q, V, dO, dQ, dV)
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    fwd_ms = bwd_ms = 0.0
+    for _ in range(K):
+        ev[0].record()
+        mod.forward(Q, V, O)
+        ev[1].record()
+        mod.backward(Q, V, dO, dQ, dV)
+        ev[2].record()
+        torch.cuda.synchronize()
+        fwd_ms += ev[0].elapsed_time(ev[1])
+        bwd_ms += ev[1].elapsed_time(ev[2])
+    st, _ = mod.info()
+    if st != lfa.LFA_OK:
+        raise RuntimeError(f"device status: {lfa.status_string(st)}")
+    step_ms = (fwd_ms + bwd_ms) / K
+    print(json.dumps({
+        "metric": "tokens/s per forward + backward call", "value": wl.units * wl.N / (step_ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
+        "forward_ms": fwd_ms / K, "backward_ms": bwd_ms / K, "higher_is_better": True, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(wl, {"path": mod.path, "inputs": "resident, no L2 flush"}),
+    }), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.backward:
+        run_backward(args)
         return
     import torch
     import torch.distributed as dist
@@ -287,7 +334,9 @@ def main():
         io_bytes = 3.0 * nbytes
         t_roof = max(alg_instr / alu_peak, io_bytes / hbm)
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "metric": METRIC if wl.name == "pvt1" else
+            f"tokens/s per Laplacian-Nyström attention call (N={wl.N},d={wl.d},m={wl.m}); % of roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(wl, {
