@@ -47,70 +47,6 @@ __device__ __forceinline__ void store4(__nv_bfloat16* g, float4 v) {
 // sign(t) * x with sign(0) = 0
 __device__ __forceinline__ float sgn_mul(float t, float x) { return t > 0.f ? x : (t < 0.f ? -x : 0.f); }
 
-// ---------------------------------------------------------------------------------------
-// Batched m x m products: Out = scale * op(A) op(B) + beta * Cin + add_diag * I, unit =
-// blockIdx.z, op = transpose when the template flag is set. Cin may alias Out (each
-// element is read and written by one thread); A and B must not.
-// ---------------------------------------------------------------------------------------
-struct Mat {
-  const float* base;
-  size_t unit_stride;   // floats between consecutive units' matrices
-};
-
-template <bool TA, bool TB>
-__global__ void __launch_bounds__(kThreads) k_bgemm(int m, Mat Am, Mat Bm, Mat Cm, float* Ob, size_t o_stride,
-                                                    float scale, float beta, float add_diag) {
-  __shared__ float As[64][17];
-  __shared__ __align__(16) float Bs[16][64];
-  const int u = blockIdx.z;
-  const float* A = Am.base + u * Am.unit_stride;
-  const float* B = Bm.base + u * Bm.unit_stride;
-  float* Out = Ob + u * o_stride;
-  const float* Cin = Cm.base ? Cm.base + u * Cm.unit_stride : nullptr;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
-  const int t = threadIdx.x, bi = t / 16, bj = t % 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < m; k0 += 16) {
-    for (int e = t; e < 64 * 16; e += blockDim.x) {
-      // A tile: rows i0..i0+63, cols k0..k0+15 of op(A)
-      const int r = TA ? e % 64 : e / 16, c = TA ? e / 64 : e % 16;
-      const int gi = i0 + r, gk = k0 + c;
-      As[r][c] = (gi < m && gk < m) ? (TA ? A[(size_t)gk * m + gi] : A[(size_t)gi * m + gk]) : 0.f;
-      // B tile: rows k0..k0+15, cols j0..j0+63 of op(B)
-      const int r2 = TB ? e % 16 : e / 64, c2 = TB ? e / 16 : e % 64;
-      const int gk2 = k0 + r2, gj = j0 + c2;
-      Bs[r2][c2] = (gk2 < m && gj < m) ? (TB ? B[(size_t)gj * m + gk2] : B[(size_t)gk2 * m + gj]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int l = 0; l < 16; ++l) {
-      float a[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) a[x] = As[4 * bi + x][l];
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[l][4 * bj]);
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
-        acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
-        acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
-        acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int x = 0; x < 4; ++x)
-#pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      const int i = i0 + 4 * bi + x, j = j0 + 4 * bj + y;
-      if (i < m && j < m) {
-        float v = scale * acc[x][y] + (i == j ? add_diag : 0.f);
-        if (Cin) v = fmaf(beta, Cin[(size_t)i * m + j], v);
-        Out[(size_t)i * m + j] = v;
-      }
-    }
-}
-
 // X_0 = alpha W^T with the alpha the forward chose (per-unit info slot).
 __global__ void k_init_iterate(BwdParams b) {
   const Params& p = b.p;
@@ -496,13 +432,6 @@ __global__ void __launch_bounds__(kThreads) k_dq_final(BwdParams b) {
   store4(static_cast<T*>(b.dQ) + o, make_float4(a.x + g.x, a.y + g.y, a.z + g.z, a.w + g.w));
 }
 
-template <bool TA, bool TB>
-void bgemm(const Params& p, Mat A, Mat B, Mat C, float* O, size_t o_stride, float scale, float beta, float add_diag,
-           cudaStream_t st) {
-  const dim3 g(ceil_div(p.m, 64), ceil_div(p.m, 64), p.U);
-  k_bgemm<TA, TB><<<g, kThreads, 0, st>>>(p.m, A, B, C, O, o_stride, scale, beta, add_diag);
-}
-
 template <typename T, int NC>
 void launch_main(const BwdParams& b, cudaStream_t st) {
   k_bwd_main<T, NC><<<dim3(b.p.P, b.p.U), kThreads, backward_smem_main(b.p.d), st>>>(b);
@@ -523,14 +452,15 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
   k_bwd_combine<<<dim3(p.n_chunks, U), kThreads, (size_t)m * d * sizeof(float), st>>>(b);
   // Newton-Schulz iterates X_0 .. X_{T-1} ([U][T][m][m])
   const size_t its_stride = (size_t)T_ * mm;
-  const Mat W{p.Wm, mm}, none{nullptr, 0};
   if (T_ > 0) {
     k_init_iterate<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(b);
     for (int k = 0; k + 1 < T_; ++k) {
-      const Mat Xk{b.its + k * mm, its_stride};
-      bgemm<false, false>(p, W, Xk, none, p.Y, mm, -1.f, 0.f, 2.f, st);                 // Y = 2I - W X_k
-      bgemm<false, false>(p, Xk, Mat{p.Y, mm}, none, b.its + (k + 1) * mm, its_stride,  // X_{k+1} = X_k Y
-                          1.f, 0.f, 0.f, st);
+      const float* Xk = b.its + k * mm;
+      const MmJob y{p.Wm, mm, Xk, its_stride, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};  // Y = 2I - W X_k
+      launch_mm(&y, 1, m, U, st);
+      const MmJob xn{Xk, its_stride, p.Y, mm, nullptr, 0, b.its + (k + 1) * mm, its_stride,  // X_{k+1} = X_k Y
+                     1.f, 0.f, 0.f, 0, 0};
+      launch_mm(&xn, 1, m, U, st);
     }
   }
   // reverse steps; G starts as dX
@@ -538,13 +468,18 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
   float* G = b.G;
   float* Gn = b.Gn;
   for (int k = T_ - 1; k >= 0; --k) {
-    const Mat Xk{b.its + k * mm, its_stride}, Gm{G, mm};
-    bgemm<true, false>(p, Xk, Gm, none, b.T1, mm, 1.f, 0.f, 0.f, st);                    // T1 = X_k^T G
-    bgemm<false, true>(p, Mat{b.T1, mm}, Xk, Mat{b.dW, mm}, b.dW, mm, -1.f, 1.f, 0.f, st);  // dW -= T1 X_k^T
-    bgemm<false, true>(p, Gm, Xk, none, b.T2, mm, 1.f, 0.f, 0.f, st);                    // T2 = G X_k^T
-    bgemm<true, true>(p, W, Xk, none, b.T3, mm, 1.f, 0.f, 0.f, st);                      // T3 = W^T X_k^T
-    bgemm<false, true>(p, Mat{b.T2, mm}, W, Gm, Gn, mm, -1.f, 2.f, 0.f, st);             // Gn = 2G - T2 W^T
-    bgemm<false, false>(p, Mat{b.T3, mm}, Gm, Mat{Gn, mm}, Gn, mm, -1.f, 1.f, 0.f, st);  // Gn -= T3 G
+    const float* Xk = b.its + k * mm;
+    const MmJob s1[3] = {
+        {Xk, its_stride, G, mm, nullptr, 0, b.T1, mm, 1.f, 0.f, 0.f, 1, 0},      // T1 = X_k^T G
+        {G, mm, Xk, its_stride, nullptr, 0, b.T2, mm, 1.f, 0.f, 0.f, 0, 1},      // T2 = G X_k^T
+        {p.Wm, mm, Xk, its_stride, nullptr, 0, b.T3, mm, 1.f, 0.f, 0.f, 1, 1}};  // T3 = W^T X_k^T
+    launch_mm(s1, 3, m, U, st);
+    const MmJob s2[2] = {
+        {b.T1, mm, Xk, its_stride, b.dW, mm, b.dW, mm, -1.f, 1.f, 0.f, 0, 1},    // dW -= T1 X_k^T
+        {b.T2, mm, p.Wm, mm, G, mm, Gn, mm, -1.f, 2.f, 0.f, 0, 1}};              // Gn = 2G - T2 W^T
+    launch_mm(s2, 2, m, U, st);
+    const MmJob s3{b.T3, mm, G, mm, Gn, mm, Gn, mm, -1.f, 1.f, 0.f, 0, 0};      // Gn -= T3 G
+    launch_mm(&s3, 1, m, U, st);
     float* tmp = G;
     G = Gn;
     Gn = tmp;
@@ -589,10 +524,10 @@ cudaError_t backward_set_attributes() {
 }
 
 int backward_launch_count(const Params& p) {
-  // pass 1 + reduce, combine, iterates (1 + 2 (T - 1)), 6 T reverse products, gram part of dL,
+  // pass 1 + reduce, combine, iterates (1 + 2 (T - 1)), 3 T reverse launches (6 products per step, batched), gram part of dL,
   // main pass, dL reduction, dQ
   const int its = p.T > 0 ? 1 + 2 * (p.T - 1) : 0;
-  return 2 + 1 + its + 6 * p.T + 1 + 1 + 1 + 1;
+  return 2 + 1 + its + 3 * p.T + 1 + 1 + 1 + 1;
 }
 
 cudaError_t launch_backward(const BwdParams& b, cudaStream_t st) {

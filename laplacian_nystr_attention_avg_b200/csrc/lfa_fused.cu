@@ -844,8 +844,14 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
         const float* r = fa.rec + (ok ? ctr[c0 + c] : 0);
         sv[c] = (ok && t < 128) ? __ldcg(r + t) : 0.f;
 #pragma unroll
-        for (int i = 0; i < kNP; ++i)
-          pv[c][i] = ok ? __ldcg(reinterpret_cast<const float4*>(r + 128) + t + kFT * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < kNP; ++i) {
+          pv[c][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ok) {
+            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * i);
+            pv[c][i] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
+                                   __uint_as_float(raw.w));
+          }
+        }
       }
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -1086,8 +1092,8 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
       if (row < nrows) {
         const uint4* src =
             reinterpret_cast<const uint4*>(O + ((size_t)R.seg[s].u * p.N + lo + row) * 64 + 16 * h);
-        dw[0] = __ldcg(src);
-        dw[1] = __ldcg(src + 1);
+        dw[0] = ld_cg_v4_ordered(src);
+        dw[1] = ld_cg_v4_ordered(src + 1);
       }
     }
   };

@@ -5,7 +5,8 @@
 // Steps (LaplacianFormer note, papernotes.org: §整体框架 flowchart, §关键设计 1-3):
 //   k_pool          L = r x r average pool of Q                         (§关键设计 2)
 //   k_ns_small      W = exp(-E/lam) + eps I, ||W||_2, alpha, T Newton-Schulz steps, m <= 64
-//   k_gram / k_alpha / k_ns_gemm   the same for 64 < m <= 256, spread over CTAs (§关键设计 3)
+//   k_gram / k_alpha / k_mm (lfa_gemm.cu) / k_ns_gemm   the same for 64 < m <= 256, spread over
+//                   CTAs (§关键设计 3); k_ns_gemm forms the closing residual I - W X_T and its norm
 //   k_pass1         C tiles in registers/smem, column sums of C and C^2, raw C^T V, sum V
 //   k_combine_*     mu, var, s = 1/sqrt(var + eps); A = C~^T V by rank-1 folding; M = X A;
 //                   M' = diag(s) M; bias b = (1/N 1 - s o mu)^T M               (§关键设计 1)
@@ -716,9 +717,12 @@ void context_t(const Params& p, cudaStream_t st) {
     const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
     float* x = p.X;
     float* xb = p.Xb;
+    const size_t mm = (size_t)m * m;
     for (int k = 0; k < p.T; ++k) {
-      k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, x, p.Y, -1.f, 2.f, 0);   // Y = 2I - W X
-      k_ns_gemm<<<g, kThreads, 0, st>>>(p, x, p.Y, xb, 1.f, 0.f, 0);      // X' = X Y
+      const MmJob y{p.Wm, mm, x, mm, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X
+      launch_mm(&y, 1, m, U, st);
+      const MmJob xn{x, mm, p.Y, mm, nullptr, 0, xb, mm, 1.f, 0.f, 0.f, 0, 0};     // X' = X Y
+      launch_mm(&xn, 1, m, U, st);
       float* tmp = x; x = xb; xb = tmp;
     }
     if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);

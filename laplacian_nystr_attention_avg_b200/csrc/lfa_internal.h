@@ -103,7 +103,28 @@ struct BwdParams {
   float* dQd;      // [U][N][d] fp32 direct part of dQ
 };
 
-// host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu
+// One batched m x m product: Out[u] = scale * op(A[u]) op(B[u]) + beta * C[u] + add_diag * I
+// (op = transpose when ta / tb is set; C may be null and may alias Out; A and B must not).
+struct MmJob {
+  const float* A;
+  size_t a_stride;   // floats between consecutive units' matrices
+  const float* B;
+  size_t b_stride;
+  const float* C;
+  size_t c_stride;
+  float* O;
+  size_t o_stride;
+  float scale, beta, add_diag;
+  int ta, tb;
+};
+struct MmJobs {
+  MmJob job[3];
+  int n;
+};
+
+// host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu / lfa_gemm.cu
+// Up to three independent jobs (none reads another's output) in one launch.
+cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st);
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_context(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st);
