@@ -580,88 +580,94 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Pass 2: O = C M' + 1 b^T + DWC(V) for one 64-row tile.
+// Pass 2: O = C M' + 1 b^T + DWC(V) over the CTA's 64-row tiles (the same row partition as
+// pass 1); L and M' are staged once per CTA.
 // ---------------------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pass2(Params p) {
   extern __shared__ float4 smem_f4[];
   float* sm = reinterpret_cast<float*>(smem_f4);
   const int m = p.m, d = p.d, ds = d + 4;
-  const int mpl = round_up(m, 64), cs = mpl + 4;
-  float* Ls = sm;                    // [mpl][ds], later M'
-  float* Qs = Ls + mpl * ds;         // [64][ds]
+  const int mpl = round_up(m, 64), cs = mpl + 4, m4 = round_up(m, 4);
+  float* Ls = sm;                    // [mpl][ds]
+  float* Ms = Ls + mpl * ds;         // [m4][ds] M'
+  float* Qs = Ms + m4 * ds;          // [64][ds]
   float* Cs = Qs + kRowTile * ds;    // [64][cs]
   float* bs = Cs + kRowTile * cs;    // [d]
-  const int u = blockIdx.y, tile = blockIdx.x, t = threadIdx.x;
-  const int row0 = tile * kRowTile, valid = min(kRowTile, p.N - row0);
+  const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x;
   const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
   const T* Vg = static_cast<const T*>(p.V) + (size_t)u * p.N * d;
   stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
-  stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+  stage_landmarks(p.Mp + (size_t)u * m * d, Ms, m, m4, d);
   if (t < d) {
     float b = 0.f;
     for (int c = 0; c < p.n_chunks; ++c) b += p.bpart[((size_t)u * p.n_chunks + c) * d + t];
     bs[t] = b;
   }
-  __syncthreads();
-  for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
-  __syncthreads();
-  stage_landmarks(p.Mp + (size_t)u * m * d, Ls, m, round_up(m, 4), d);
-  __syncthreads();
   const int nbk = d / 4;
-  if (t < 16 * nbk) {
-    const int ib = t / nbk, kb = t % nbk;
-    float acc[4][4] = {};
-    const int m4 = round_up(m, 4);
-    for (int j = 0; j < m4; j += 4) {
-      float4 c[4], mp[4];
+  const int ib = t / nbk, kb = t % nbk;
+  const bool mapped = t < 16 * nbk;
+  // DWC weights of this thread's 4 channels: w[h][k][a][b] multiplies V[y + a - 1][x + b - 1][k]
+  const int h = u % p.heads;
+  float wt[4][9];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) c[x] = *reinterpret_cast<const float4*>(&Cs[(4 * ib + x) * cs + j]);
+  for (int y = 0; y < 4; ++y)
 #pragma unroll
-      for (int y = 0; y < 4; ++y) mp[y] = *reinterpret_cast<const float4*>(&Ls[(j + y) * ds + 4 * kb]);
+    for (int e = 0; e < 9; ++e) wt[y][e] = mapped ? p.dwc[((size_t)h * d + 4 * kb + y) * 9 + e] : 0.f;
+  T* Og = static_cast<T*>(p.O) + (size_t)u * p.N * d;
+  const int tile0 = pc * p.tiles_per_cta;
+  const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
+  for (int tile = tile0; tile < tile1; ++tile) {
+    const int row0 = tile * kRowTile, valid = min(kRowTile, p.N - row0);
+    __syncthreads();   // the previous tile's readers of Qs and Cs are done
+    stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+    __syncthreads();
+    for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
+    __syncthreads();
+    if (mapped) {
+      float acc[4][4] = {};
+      for (int j = 0; j < m4; j += 4) {
+        float4 c[4], mp[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) c[x] = *reinterpret_cast<const float4*>(&Cs[(4 * ib + x) * cs + j]);
+#pragma unroll
+        for (int y = 0; y < 4; ++y) mp[y] = *reinterpret_cast<const float4*>(&Ms[(j + y) * ds + 4 * kb]);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float cc[4] = {c[x].x, c[x].y, c[x].z, c[x].w};
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            acc[x][0] = fmaf(cc[y], mp[y].x, acc[x][0]);
+            acc[x][1] = fmaf(cc[y], mp[y].y, acc[x][1]);
+            acc[x][2] = fmaf(cc[y], mp[y].z, acc[x][2]);
+            acc[x][3] = fmaf(cc[y], mp[y].w, acc[x][3]);
+          }
+        }
+      }
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
-        const float cc[4] = {c[x].x, c[x].y, c[x].z, c[x].w};
+        const int i = 4 * ib + x;
+        if (i >= valid) continue;
+        const int n = row0 + i, gy = n / p.W, gx = n % p.W;
+        float o[4] = {acc[x][0] + bs[4 * kb], acc[x][1] + bs[4 * kb + 1], acc[x][2] + bs[4 * kb + 2],
+                      acc[x][3] + bs[4 * kb + 3]};
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          acc[x][0] = fmaf(cc[y], mp[y].x, acc[x][0]);
-          acc[x][1] = fmaf(cc[y], mp[y].y, acc[x][1]);
-          acc[x][2] = fmaf(cc[y], mp[y].z, acc[x][2]);
-          acc[x][3] = fmaf(cc[y], mp[y].w, acc[x][3]);
+        for (int a = 0; a < 3; ++a) {
+          const int yy = gy + a - 1;
+          if (yy < 0 || yy >= p.H) continue;
+#pragma unroll
+          for (int b = 0; b < 3; ++b) {
+            const int xx = gx + b - 1;
+            if (xx < 0 || xx >= p.W) continue;
+            const float4 v = load4(Vg + ((size_t)yy * p.W + xx) * d + 4 * kb);
+            o[0] = fmaf(wt[0][a * 3 + b], v.x, o[0]);
+            o[1] = fmaf(wt[1][a * 3 + b], v.y, o[1]);
+            o[2] = fmaf(wt[2][a * 3 + b], v.z, o[2]);
+            o[3] = fmaf(wt[3][a * 3 + b], v.w, o[3]);
+          }
         }
+        store4(Og + (size_t)n * d + 4 * kb, make_float4(o[0], o[1], o[2], o[3]));
       }
-    }
-    // DWC(V): w[h][k][a][b] multiplies V[y + a - 1][x + b - 1][k]
-    const int h = u % p.heads;
-    float wt[4][9];
-#pragma unroll
-    for (int y = 0; y < 4; ++y)
-#pragma unroll
-      for (int e = 0; e < 9; ++e) wt[y][e] = p.dwc[((size_t)h * d + 4 * kb + y) * 9 + e];
-    T* Og = static_cast<T*>(p.O) + (size_t)u * p.N * d;
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int i = 4 * ib + x;
-      if (i >= valid) continue;
-      const int n = row0 + i, gy = n / p.W, gx = n % p.W;
-      float o[4] = {acc[x][0] + bs[4 * kb], acc[x][1] + bs[4 * kb + 1], acc[x][2] + bs[4 * kb + 2],
-                    acc[x][3] + bs[4 * kb + 3]};
-#pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        const int yy = gy + a - 1;
-        if (yy < 0 || yy >= p.H) continue;
-#pragma unroll
-        for (int b = 0; b < 3; ++b) {
-          const int xx = gx + b - 1;
-          if (xx < 0 || xx >= p.W) continue;
-          const float4 v = load4(Vg + ((size_t)yy * p.W + xx) * d + 4 * kb);
-          o[0] = fmaf(wt[0][a * 3 + b], v.x, o[0]);
-          o[1] = fmaf(wt[1][a * 3 + b], v.y, o[1]);
-          o[2] = fmaf(wt[2][a * 3 + b], v.z, o[2]);
-          o[3] = fmaf(wt[3][a * 3 + b], v.w, o[3]);
-        }
-      }
-      store4(Og + (size_t)n * d + 4 * kb, make_float4(o[0], o[1], o[2], o[3]));
     }
   }
 }
@@ -738,7 +744,7 @@ cudaError_t forward_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   context_t<T>(p, st);
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
-  k_pass2<T><<<dim3(p.n_tiles, U), kThreads, generic_smem_pass2(m, d), st>>>(p);
+  k_pass2<T><<<dim3(p.P, U), kThreads, generic_smem_pass2(m, d), st>>>(p);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
   return cudaGetLastError();
 }
@@ -751,8 +757,8 @@ size_t generic_smem_pass1(int m, int d) {
 }
 
 size_t generic_smem_pass2(int m, int d) {
-  const int mpl = round_up(m, 64), ds = d + 4;
-  return sizeof(float) * ((size_t)mpl * ds + kRowTile * ds + (size_t)kRowTile * (mpl + 4) + d);
+  const int mpl = round_up(m, 64), ds = d + 4, m4 = round_up(m, 4);
+  return sizeof(float) * ((size_t)mpl * ds + (size_t)m4 * ds + kRowTile * ds + (size_t)kRowTile * (mpl + 4) + d);
 }
 
 cudaError_t generic_set_attributes() {
