@@ -98,7 +98,8 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kNumBars = 17;
+constexpr int kBarD = 17;     // [3] pass-2 DWC values of a chunk landed (TMA from O)
+constexpr int kNumBars = 20;
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
@@ -1034,6 +1035,7 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
           *reinterpret_cast<uint2*>(O + (size_t)(n0 + i) * 64) =
               make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
     }
+    if (gc + 1 == nch) fence_async_global();   // pass 2 reads these O rows back by TMA
     __syncthreads();
     if (t == 0 && gc + nbuf < nch) issue(gc + nbuf);
   }
@@ -1043,18 +1045,29 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
 // ---------------------------------------------------------------------------------------
 // Phase 4: O = C M' + b + DWC(V) for every chunk. M'^T and b of each segment's unit come from
 // its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region); the DWC
-// values are already in O (phase 3b). All products are issued at once, each chunk into its own
+// values are already in O (phase 3b) and come back by TMA three chunks ahead. All products are issued at once, each chunk into its own
 // 64-column TMEM accumulator with its own barrier, and the epilogues follow chunk by chunk.
 // ---------------------------------------------------------------------------------------
 __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
-                          uint32_t tmem, uint64_t* bars) {
+                          uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapO) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffV; };
-  __syncthreads();   // the DWC phase is done with the halo region
-  if (t == 0)
+  // DWC values of chunk gc (O rows, SW128) in ring buffer gc % 3 after segment 1's M' image
+  auto dwc_buf = [&](int gc) { return sm + kOffV + 8192 + (gc % 3) * 16384; };
+  auto issue_dwc = [&](int gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    uint64_t* db = bars + kBarD + gc % 3;
+    mbar_expect_tx(db, 16384);
+    tma_load_3d(dwc_buf(gc), tmapO, 0, lo, R.seg[s].u, db);
+  };
+  __syncthreads();   // the DWC phase is done with the halo region; its O rows are fenced
+  if (t == 0) {
+    for (int gc = 0; gc < nch && gc < 3; ++gc) issue_dwc(gc);
     for (int s = 0; s < R.nseg; ++s) spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout);
+  }
   __syncthreads();
   trace_mark(p, 4);
   for (int s = 0; s < R.nseg; ++s) {
@@ -1083,27 +1096,13 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   }
   __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
-  // DWC values of a chunk's rows, loaded one chunk ahead of their use
-  auto fetch_dwc = [&](int gc, uint4 (&dw)[2]) {
-    dw[0] = dw[1] = make_uint4(0u, 0u, 0u, 0u);
-    if (gc < nch) {
-      int s, lo, nrows;
-      R.chunk(gc, s, lo, nrows);
-      if (row < nrows) {
-        const uint4* src =
-            reinterpret_cast<const uint4*>(O + ((size_t)R.seg[s].u * p.N + lo + row) * 64 + 16 * h);
-        dw[0] = ld_cg_v4_ordered(src);
-        dw[1] = ld_cg_v4_ordered(src + 1);
-      }
-    }
-  };
-  uint4 dn[2];
-  fetch_dwc(0, dn);
   for (int gc = 0; gc < nch; ++gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    const uint4 dw[2] = {dn[0], dn[1]};
-    fetch_dwc(gc + 1, dn);
+    mbar_wait(bars + kBarD + gc % 3, (gc / 3) & 1, p.status, kStatusTimeout);
+    uint4 dw[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) dw[j] = *reinterpret_cast<const uint4*>(dwc_buf(gc) + sw128(row, 2 * h + j));
     mbar_wait(bars + kBarP2 + gc, 0, p.status, kStatusTimeout);
     if (gc == 0) trace_mark(p, 29);
     tc_fence_after();
@@ -1124,6 +1123,10 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
         orow[k4] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
+    if (gc + 3 < nch) {
+      __syncthreads();   // ring buffer gc % 3 has been read
+      if (t == 0) issue_dwc(gc + 3);
+    }
     if (gc < 2) trace_mark(p, 30 + gc);
   }
   tc_fence_before();
@@ -1133,7 +1136,8 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
 
 __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const FusedArgs fa,
                                                            const __grid_constant__ CUtensorMap tmapV,
-                                                           const __grid_constant__ CUtensorMap tmapQ) {
+                                                           const __grid_constant__ CUtensorMap tmapQ,
+                                                           const __grid_constant__ CUtensorMap tmapO) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + pad;
@@ -1164,6 +1168,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   if (t == 32) {
     tma_prefetch_desc(&tmapV);
     tma_prefetch_desc(&tmapQ);
+    tma_prefetch_desc(&tmapO);
   }
 
   // ---- phase 0: landmark pooling, one warp per landmark ----
@@ -1234,7 +1239,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     solver_combine(p, fa, sm, g);
   }
   if (R.nchunks > 0) dwc_all(p, R, sm, bars, &tmapV);
-  if (R.nchunks > 0) pass2_all(p, fa, R, sm, sbase, tmem, bars);
+  if (R.nchunks > 0) pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
   __syncthreads();
   trace_mark(p, 15);
   trace_clock(p, 14);
@@ -1317,10 +1322,11 @@ int fused_grid(const Params& p) {
 }
 
 // Tensor maps of recently used V pointers (host side; encoding costs a driver call).
+constexpr int kTmapCache = 32;   // Q, V and O maps of a few rotating buffer sets
 struct TmapCache {
-  const void* ptr[16];
-  int N[16], U[16], sw[16];
-  CUtensorMap map[16];
+  const void* ptr[kTmapCache];
+  int N[kTmapCache], U[kTmapCache], sw[kTmapCache];
+  CUtensorMap map[kTmapCache];
   int next;
 };
 static TmapCache g_tmaps;
@@ -1329,7 +1335,7 @@ static std::mutex g_tmaps_mu;
 // [U][N][64] bf16 viewed as {64, N, U}, boxes of 128 rows; 128-byte swizzle or plain rows
 static bool tmap_for(const void* X, int N, int U, bool swizzle, CUtensorMap* out) {
   std::lock_guard<std::mutex> lk(g_tmaps_mu);
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < kTmapCache; ++i)
     if (g_tmaps.ptr[i] == X && g_tmaps.N[i] == N && g_tmaps.U[i] == U && g_tmaps.sw[i] == (int)swizzle) {
       *out = g_tmaps.map[i];
       return true;
@@ -1337,7 +1343,7 @@ static bool tmap_for(const void* X, int N, int U, bool swizzle, CUtensorMap* out
   CUtensorMap m;
   if (!make_tmap_rows_bf16(&m, X, (uint64_t)N, (uint64_t)U, kChunk, swizzle)) return false;
   const int i = g_tmaps.next;
-  g_tmaps.next = (i + 1) & 15;
+  g_tmaps.next = (i + 1) % kTmapCache;
   g_tmaps.ptr[i] = X;
   g_tmaps.N[i] = N;
   g_tmaps.U[i] = U;
@@ -1353,9 +1359,10 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
     const cudaError_t e = cudaMemsetAsync(fused_ws, 0, flag_bytes(p.U), st);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tmap, tmapq;
+  CUtensorMap tmap, tmapq, tmapo;
   if (!tmap_for(p.V, p.N, p.U, true, &tmap)) return cudaErrorInvalidValue;
   if (!tmap_for(p.Q, p.N, p.U, true, &tmapq)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.O, p.N, p.U, true, &tmapo)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.epoch = epoch;
   fa.ws16 = solver_share16();
@@ -1368,7 +1375,7 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
   fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
   Params pp = p;
-  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq};
+  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo};
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
   cudaError_t e = cudaLaunchCooperativeKernel((const void*)k_fused_forward, dim3(G), dim3(kFT), args, kSmemAlloc, st);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
