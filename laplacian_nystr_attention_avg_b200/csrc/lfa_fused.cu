@@ -90,6 +90,7 @@ constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64]
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(kOffBp + (kFT / 16) * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
+static_assert(kMaxChunks <= kFT / 32, "pass 2 issues one chunk's product per warp");
 
 // mbarrier slots
 constexpr int kBarV = 0;      // [3] V stage filled by TMA
@@ -1080,19 +1081,20 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   tc_fence_before();
   __syncthreads();
   trace_mark(p, 5);
-  if (t == 0) {
+  // chunk gc's product is issued by lane 0 of warp gc (separate accumulators and barriers, so the
+  // issues proceed in parallel and the results do not depend on their order)
+  if (lane == 0 && w < nch) {
+    const int gc = w;
     tc_fence_after();
     const uint32_t id = idesc(1, 128, 64, 0, 0);
-    for (int gc = 0; gc < nch; ++gc) {
-      int s, lo, nrows;
-      R.chunk(gc, s, lo, nrows);
-      const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
-      const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
+    const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
-      mma_commit(bars + kBarP2 + gc);
-    }
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
+    mma_commit(bars + kBarP2 + gc);
   }
   __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
