@@ -506,7 +506,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
 // lanes' rows spread the reads over all banks.
 template <int LT>
 __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float* Ls, unsigned char* cslot, int j0,
-                                            int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
+                                            int m, int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
   const int lane = threadIdx.x & 31;
   float acc[2][LT];
 #pragma unroll
@@ -569,21 +569,28 @@ __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float
         *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = __float2bfloat16_rn(c[b]);
       }
     }
+    // the last landmark group also writes the padding columns m..63 of its rows: zero, except
+    // column 63 = 1 on valid rows (it yields sum_i v_i in the C^T V product)
+    if (j0 + LT == m) {
+      const __nv_bfloat16 one = __float2bfloat16_rn(valid ? 1.f : 0.f), zero = __float2bfloat16_rn(0.f);
+      for (int col = m; col < 64; ++col)
+        *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = col == 63 ? one : zero;
+    }
   }
 }
 
 __device__ __forceinline__ void cross_dispatch(int lt, const unsigned char* Qs, const float* Ls, unsigned char* cslot,
-                                               int j0, int rb, int nrows, float scale, float (&s1)[8],
+                                               int j0, int m, int rb, int nrows, float scale, float (&s1)[8],
                                                float (&s2)[8]) {
   switch (lt) {
-    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
     default: break;
   }
 }
@@ -692,16 +699,10 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
       }
       __syncthreads();
     }
-    // padding landmark columns m..63: zero, except column 63 = 1 on valid rows (sum of V)
-    for (int e = t; e < kChunk * (64 - m); e += kFT) {
-      const int row = e / (64 - m), col = m + e % (64 - m);
-      const float v = (col == 63 && row < nrows) ? 1.f : 0.f;
-      *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = __float2bfloat16_rn(v);
-    }
     if (gc == 1) trace_mark(p, 26);
     if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
-    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
+    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, m, 64 * rh, nrows, scale, s1, s2);
     if (gc == 1) trace_mark(p, 22);
     if (seg_last) {
       // this segment's column sums of C and C^2, per row half
@@ -718,18 +719,17 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
         }
       }
     }
-    // the next V chunk, while the SM idles at the barrier: stage (gc + 1) % 3 last held chunk
-    // gc - 2, whose product was issued at this chunk's start
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (gc < 2) trace_mark(p, 11 + gc);
+    // the next V chunk, issued after the barrier so that this thread's proxy fence above does not
+    // wait for it: stage (gc + 1) % 3 last held chunk gc - 2, whose product went out at this
+    // chunk's start
     if (t == 0 && gc >= 1 && gc + 1 < nch) {
       if (gc >= 2) wait_mma(gc - 2);
       issue_v(gc + 1);
     }
-    if (gc == 1) trace_mark(p, 20);
-    fence_async_smem();
-    if (gc == 1) trace_mark(p, 23);
-    tc_fence_before();
-    __syncthreads();
-    if (gc < 2) trace_mark(p, 11 + gc);
   }
   // the last two products, each waited before the next one on its commit slot goes out
   if (t == 0) {
