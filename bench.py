@@ -49,6 +49,25 @@ def parse_args():
     return ap.parse_args()
 
 
+def max_over_ranks(values, world, device=None):
+    """Element-wise maximum of per-rank timings over all ranks (identity on one rank).
+
+    Every rank calls it at the same point; with NCCL the tensor lives on the rank's GPU.
+    """
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(world, units, N, steps, total_ms):
+    """Whole-job throughput: every rank processes its own units x N tokens per step."""
+    return world * units * N * steps / (total_ms * 1e-3)
+
+
 def workload_config(wl, extra=None):
     cfg = {"workload": f"{wl.name}: B={wl.B} heads={wl.heads} grid={wl.H}x{wl.W} N={wl.N} d={wl.d} "
                        f"r={wl.r} m={wl.m} lambda={wl.lam:g} eps={wl.eps:g} T={wl.T} {wl.dtype} "
@@ -291,12 +310,9 @@ def main():
     mod.set_profile_events(None, None)
     total_ms = t_begin.elapsed_time(t_end)
     kern_ms = statistics.fmean(kb[k].elapsed_time(ke[k]) for k in range(K))
-    if world > 1:
-        t = torch.tensor([total_ms, kern_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, kern_ms = float(t[0]), float(t[1])
+    total_ms, kern_ms = max_over_ranks([total_ms, kern_ms], world, dev)
     ms_per_step = total_ms / K
-    value = world * wl.units * wl.N * K / (total_ms * 1e-3)
+    value = job_tokens_per_s(world, wl.units, wl.N, K, total_ms)
 
     # end to end through the host-buffer entry point: pinned host Q, V -> device -> O -> host
     Qh = x.Q_store.pin_memory()
@@ -313,12 +329,8 @@ def main():
         mod.forward_host(Qh, Vh, Oh, Qs[0], Vs[0], Os[0])
     e_e.record(stream)
     barrier()
-    e2e_ms = e_b.elapsed_time(e_e)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * wl.units * wl.N * E / (e2e_ms * 1e-3)
+    e2e_ms = max_over_ranks([e_b.elapsed_time(e_e)], world, dev)[0]
+    e2e_value = job_tokens_per_s(world, wl.units, wl.N, E, e2e_ms)
     nbytes = wl.units * wl.N * wl.d * x.Q_store.element_size()
 
     if rank == 0:
