@@ -99,8 +99,10 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarD = 17;     // [3] pass-2 DWC values of a chunk landed (TMA from O)
-constexpr int kNumBars = 20;
+constexpr int kBarD = 17;     // [kDwcRing] pass-2 DWC values of a chunk landed (TMA from O)
+constexpr int kDwcRing = 4;
+constexpr int kNumBars = kBarD + kDwcRing;
+static_assert(8192 + kDwcRing * 16384 <= kHaloSpace, "pass-2 DWC ring overlaps M'");
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
@@ -906,6 +908,7 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
     // M = X A with a 2 x 4 register tile per thread; M' = diag(s) M as bf16 (K-major B of pass 2)
     const int jb = t >> 4, kb = t & 15;
     float acc[2][4] = {};
+#pragma unroll 4
     for (int l = 0; l < m; ++l) {
       const float2 x2 = *reinterpret_cast<const float2*>(Xt + l * kQS + 2 * jb);
       const float4 a4 = *reinterpret_cast<const float4*>(As + l * kQS + 4 * kb);
@@ -1046,7 +1049,7 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
 // ---------------------------------------------------------------------------------------
 // Phase 4: O = C M' + b + DWC(V) for every chunk. M'^T and b of each segment's unit come from
 // its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region); the DWC
-// values are already in O (phase 3b) and come back by TMA three chunks ahead. All products are issued at once, each chunk into its own
+// values are already in O (phase 3b) and come back by TMA four chunks ahead. All products are issued at once, each chunk into its own
 // 64-column TMEM accumulator with its own barrier, and the epilogues follow chunk by chunk.
 // ---------------------------------------------------------------------------------------
 __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
@@ -1055,18 +1058,18 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffV; };
-  // DWC values of chunk gc (O rows, SW128) in ring buffer gc % 3 after segment 1's M' image
-  auto dwc_buf = [&](int gc) { return sm + kOffV + 8192 + (gc % 3) * 16384; };
+  // DWC values of chunk gc (O rows, SW128) in ring buffer gc % kDwcRing after segment 1's M' image
+  auto dwc_buf = [&](int gc) { return sm + kOffV + 8192 + (gc % kDwcRing) * 16384; };
   auto issue_dwc = [&](int gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    uint64_t* db = bars + kBarD + gc % 3;
+    uint64_t* db = bars + kBarD + gc % kDwcRing;
     mbar_expect_tx(db, 16384);
     tma_load_3d(dwc_buf(gc), tmapO, 0, lo, R.seg[s].u, db);
   };
   __syncthreads();   // the DWC phase is done with the halo region; its O rows are fenced
   if (t == 0) {
-    for (int gc = 0; gc < nch && gc < 3; ++gc) issue_dwc(gc);
+    for (int gc = 0; gc < nch && gc < kDwcRing; ++gc) issue_dwc(gc);
     for (int s = 0; s < R.nseg; ++s) spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout);
   }
   __syncthreads();
@@ -1101,7 +1104,7 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   for (int gc = 0; gc < nch; ++gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    mbar_wait(bars + kBarD + gc % 3, (gc / 3) & 1, p.status, kStatusTimeout);
+    mbar_wait(bars + kBarD + gc % kDwcRing, (gc / kDwcRing) & 1, p.status, kStatusTimeout);
     uint4 dw[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) dw[j] = *reinterpret_cast<const uint4*>(dwc_buf(gc) + sw128(row, 2 * h + j));
@@ -1125,9 +1128,9 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
         orow[k4] = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    if (gc + 3 < nch) {
-      __syncthreads();   // ring buffer gc % 3 has been read
-      if (t == 0) issue_dwc(gc + 3);
+    if (gc + kDwcRing < nch) {
+      __syncthreads();   // ring buffer gc % kDwcRing has been read
+      if (t == 0) issue_dwc(gc + kDwcRing);
     }
     if (gc < 2) trace_mark(p, 30 + gc);
   }

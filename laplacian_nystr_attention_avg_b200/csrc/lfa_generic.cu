@@ -256,11 +256,23 @@ __global__ void __launch_bounds__(kThreads) k_gram(Params p) {
   p.Wm[(size_t)u * m * m + e] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
 }
 
-__global__ void __launch_bounds__(kThreads) k_alpha(Params p) {
+// Power iteration for ||W||_2 with 1024 threads; the first alpha_rows(m) rows of W are staged in
+// shared memory once (the rest are read from L2 at every step).
+constexpr int kAlphaThreads = 1024;
+__host__ __device__ inline int alpha_rows(int m) {
+  const int cap = (200 * 1024) / (4 * (m > 0 ? m : 1));
+  return m < cap ? m : cap;
+}
+
+__global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
   __shared__ float v[kMaxM], w[kMaxM], red[32];
+  extern __shared__ float4 smem_f4[];
+  float* Ws = reinterpret_cast<float*>(smem_f4);   // [alpha_rows(m)][m]
   const int u = blockIdx.x, m = p.m, t = threadIdx.x;
   const float* Wg = p.Wm + (size_t)u * m * m;
   const int warp = t / 32, lane = t & 31, nw = blockDim.x / 32;
+  const int rs = alpha_rows(m);
+  for (int e = t; e < rs * m; e += blockDim.x) Ws[e] = Wg[e];
   if (t < m) v[t] = rsqrtf(float(m));
   __syncthreads();
   float rq = 0.f;
@@ -268,8 +280,9 @@ __global__ void __launch_bounds__(kThreads) k_alpha(Params p) {
   for (int it = 0; it <= iters; ++it) {
     // w = W v, one warp per row (coalesced along the row)
     for (int i = warp; i < m; i += nw) {
+      const float* row = i < rs ? Ws + (size_t)i * m : Wg + (size_t)i * m;
       float acc = 0.f;
-      for (int j = lane; j < m; j += 32) acc = fmaf(Wg[(size_t)i * m + j], v[j], acc);
+      for (int j = lane; j < m; j += 32) acc = fmaf(row[j], v[j], acc);
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) w[i] = acc;
     }
@@ -719,7 +732,7 @@ void context_t(const Params& p, cudaStream_t st) {
     k_ns_small<<<U, kThreads, smem, st>>>(p);
   } else {
     k_gram<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
-    k_alpha<<<U, kThreads, 0, st>>>(p);
+    k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
     const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
     float* x = p.X;
     float* xb = p.Xb;
@@ -779,6 +792,10 @@ cudaError_t generic_set_attributes() {
   LFA_ATTR(k_cross_out<float>);
   LFA_ATTR(k_cross_out<__nv_bfloat16>);
 #undef LFA_ATTR
+  // k_alpha also has static shared memory: its dynamic part stays below the per-block limit
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_alpha, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(sizeof(float) * (size_t)alpha_rows(kMaxM) * kMaxM));
   return e;
 }
 
