@@ -681,14 +681,12 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
   trace_mark(p, 28);
   float s1[8], s2[8];
   for (int gc = 0; gc < nch; ++gc) {
-    if (gc == 1) trace_mark(p, 24);
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
     const int u = R.seg[s].u;
     const bool seg_first = gc == R.seg[s].first_chunk;
     const bool seg_last = gc == R.seg[s].first_chunk + R.seg[s].nch - 1;
     unsigned char* cslot = sm + kOffC + gc * 16384;
-    if (gc == 1) trace_mark(p, 27);
     // products run two chunks behind: tile gc - 2 is complete and its V stage has had a chunk
     if (t == 0 && gc >= 2) issue_mma(gc - 2);
     // Ls was last read before the previous chunk's closing barrier
@@ -701,7 +699,6 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
       }
       __syncthreads();
     }
-    if (gc == 1) trace_mark(p, 26);
     if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
     if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, m, 64 * rh, nrows, scale, s1, s2);
