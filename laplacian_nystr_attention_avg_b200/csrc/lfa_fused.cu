@@ -20,12 +20,13 @@
 //   phase 3  solver CTA of unit u, once the unit's records are out: mu, var, s = 1/sqrt(var +
 //            eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A, M' = diag(s) M,
 //            b = (1/N - s o mu)^T M; M'^T (bf16, in the shared-memory image pass 2 consumes) and
-//            b are published with a release flag.
+//            b are published with a release flag; then the solve's diagnostics, off the
+//            critical path.
 //   phase 3b row CTAs, while M' is formed: DWC(V) (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise,
 //            zero padding) of every chunk from a TMA-staged V tile with a one-grid-row halo,
-//            written to O as bf16.
-//   phase 4  row CTAs: O = C M' (tcgen05; all chunks' products at once, one TMEM accumulator each)
-//            + b + the DWC values.
+//            rounded to bf16 and written into the chunk's TMEM accumulator.
+//   phase 4  row CTAs: O = DWC + C M' (tcgen05 accumulating onto the DWC values; all chunks'
+//            products at once, one TMEM accumulator each) + b, stored once as bf16.
 // Every cross-CTA wait is bounded; an expired wait sets the timeout bit of the status word.
 #include <stdlib.h>
 #include <string.h>
@@ -60,8 +61,7 @@ constexpr uint32_t kOffMp = kOffL + 64 * kQS * 4;               // M'^T bf16 [64
 constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [segment][64]
 constexpr uint32_t kOffBar = kOffBv + 512;                      // mbarriers + TMEM address
 constexpr uint32_t kOffCt = kOffBar + 256;                      // int [32] record offsets
-constexpr uint32_t kOffWd = kOffCt + 128;                       // DWC weights fp32 [9 taps][64 ch]
-constexpr uint32_t kOffSr = kOffWd + 9 * 64 * 4;                // pass-1 column sums [segment][row half][128]
+constexpr uint32_t kOffSr = kOffCt + 128;                       // pass-1 column sums [segment][row half][128]
 constexpr uint32_t kOffRows = kOffSr + 2 * 256 * 4;            // this CTA's row plan (struct Rows)
 constexpr uint32_t kSmemBytes = kOffRows + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
@@ -99,24 +99,24 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarD = 17;     // [kDwcRing] pass-2 DWC values of a chunk landed (TMA from O)
-constexpr int kDwcRing = 4;
-constexpr int kNumBars = kBarD + kDwcRing;
-static_assert(8192 + kDwcRing * 16384 <= kHaloSpace, "pass-2 DWC ring overlaps M'");
+constexpr int kBarDiag = kBarP2;   // solver CTAs (which run no pass 2): the diagnostics product
+constexpr int kBarDw = 17;    // [2] DWC transfer product of staging buffer b done
+constexpr int kNumBars = kBarDw + 2;
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
 
 struct FusedArgs {
   unsigned long long epoch;   // launch count of this handle (>= 1); flags compare against it
-  int ws16;                   // row share of a solver CTA in 1/16 of a plain CTA's share
-  int totw16;                 // ws16 * U + 16 * (G - U)
   unsigned long long* gbar;   // grid barrier counter
   unsigned long long* cnt;    // [U] partial records published per unit
   unsigned long long* xready; // [U] X published (holds the epoch)
   unsigned long long* mready; // [U] M' image and b published (holds the epoch)
   float* rec;                 // [G][2][kRec]
   unsigned char* mimg;        // [U][kImgBytes] M'^T bf16 (SW128 image of the pass-2 B operand), b fp32
+  // pass-1 warp plan: warp w computes landmarks [wj0[w], wj0[w] + wlt[w]) of row half w / 8;
+  // warp padw[h] writes the padding columns of row half h
+  unsigned char wj0[kWarps], wlt[kWarps], padw[2];
 };
 
 __device__ __forceinline__ void trace_mark(const Params& p, int slot) {
@@ -126,27 +126,26 @@ __device__ __forceinline__ void trace_clock(const Params& p, int slot) {
   if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 32 + slot] = (unsigned long long)clock64();
 }
 
-// First global row (u * N + row) of CTA g. Each unit's rows are cut into 128-row chunks (the
-// last one may be short) and whole chunks are dealt out in proportion to the CTA weights
-// (a solver CTA weighs ws16/16 of a plain CTA), so no CTA gets a partial chunk mid-unit.
-__host__ __device__ __forceinline__ long long part_start(int g, int U, int N, int ws16, long long totw16) {
-  const long long cw = g <= U ? (long long)ws16 * g : (long long)ws16 * U + 16ll * (g - U);
-  const long long nchu = (N + kChunk - 1) / kChunk;
-  const long long ci = (long long)U * nchu * cw / totw16;
+// Row partition. Each unit's rows are cut into nchu 128-row chunks (the last one may be short);
+// the T = U nchu chunks of all units, in unit order, are dealt out evenly to the P = G - U row
+// CTAs: row CTA k = g - U starts at chunk floor(T k / P). Solver CTAs (g < U) take no rows: they
+// run the Newton-Schulz chain while the others compute C. No CTA gets a partial chunk mid-unit.
+// 32-bit arithmetic: on the shapes the fused kernel accepts (at most kMaxChunks - 1 chunks per row
+// CTA, at most kMaxGrid CTAs) T P stays below 7 kMaxGrid^2 and every row index below
+// 7 kMaxGrid kChunk. (64-bit division is a long software sequence on the GPU.)
+static_assert((long long)(kMaxChunks - 1) * kMaxGrid * kMaxGrid * 2 < (1ll << 31),
+              "partition arithmetic overflows 32 bits");
+// first global row (u N + row) of CTA g
+__host__ __device__ __forceinline__ int part_start(int g, int U, int N, int G) {
+  const int nchu = (N + kChunk - 1) / kChunk, T = U * nchu, P = G - U;
+  const int ci = g <= U ? 0 : T * (g - U) / P;
   return (ci / nchu) * N + (ci % nchu) * kChunk;
 }
-__device__ __forceinline__ long long cta_start(int g, const Params& p, const FusedArgs& fa) {
-  return part_start(g, p.U, p.N, fa.ws16, fa.totw16);
-}
-// CTA whose range holds global row R
-__device__ __forceinline__ int cta_of_row(long long R, const Params& p, const FusedArgs& fa) {
-  int lo = 0, hi = gridDim.x - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (cta_start(mid, p, fa) <= R) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
+__device__ __forceinline__ int cta_start(int g, const Params& p) { return part_start(g, p.U, p.N, gridDim.x); }
+// CTA whose range holds global chunk C: the largest k with floor(T k / P) <= C, i.e. T k < (C + 1) P
+__device__ __forceinline__ int chunk_owner(int C, const Params& p) {
+  const int nchu = (p.N + kChunk - 1) / kChunk, T = p.U * nchu, P = (int)gridDim.x - p.U;
+  return p.U + ((C + 1) * P - 1) / T;
 }
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -210,19 +209,19 @@ struct Rows {
   }
 };
 
-__device__ Rows cta_rows(int g, const Params& p, const FusedArgs& fa) {
+__device__ Rows cta_rows(int g, const Params& p) {
   Rows R;
-  const long long r0 = cta_start(g, p, fa), r1 = cta_start(g + 1, p, fa);
+  const int r0 = cta_start(g, p), r1 = cta_start(g + 1, p);
   R.nseg = 0;
-  long long a = r0;
+  int a = r0;
   int fc = 0;
   while (a < r1 && R.nseg < 2) {
-    const int u = (int)(a / p.N);
-    const long long e = ((long long)(u + 1) * p.N < r1) ? (long long)(u + 1) * p.N : r1;
+    const int u = a / p.N;
+    const int e = (u + 1) * p.N < r1 ? (u + 1) * p.N : r1;
     Seg& s = R.seg[R.nseg];
     s.u = u;
-    s.lo = (int)(a - (long long)u * p.N);
-    s.hi = (int)(e - (long long)u * p.N);
+    s.lo = a - u * p.N;
+    s.hi = e - u * p.N;
     s.first_chunk = fc;
     s.nch = (s.hi - s.lo + kChunk - 1) / kChunk;
     fc += s.nch;
@@ -291,8 +290,14 @@ __device__ void ns_issue(uint32_t sbase, uint32_t tmem, uint64_t* bar, int nks) 
   }
 }
 
-__device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* sm, uint32_t sbase,
-                           uint32_t tmem, uint64_t* bars, int u) {
+// Scalars of the solver that its diagnostics report after the combine.
+struct SolverInfo {
+  float alpha, lmax;
+  int fallback;
+};
+
+__device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned char* sm, uint32_t sbase,
+                                 uint32_t tmem, uint64_t* bars, int u) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int m = p.m;
   float* Ls = reinterpret_cast<float*>(sm + kOffNsL);
@@ -464,11 +469,15 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
       clean(st);
     }
   }
-  // publish X_T
-  if (top && i < m) {
+  // publish X_T; its transpose, zero outside m x m, stays in shared memory for the combine
+  {
+    float* Xt = reinterpret_cast<float*>(sm + kOffXt);
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      if (16 * h + c < m) p.X[((size_t)u * m + i) * m + 16 * h + c] = st[c];
+    for (int c = 0; c < 16; ++c) {
+      const bool in = top && i < m && 16 * h + c < m;
+      if (in) p.X[((size_t)u * m + i) * m + 16 * h + c] = st[c];
+      if (top) Xt[(16 * h + c) * kQS + i] = in ? st[c] : 0.f;
+    }
   }
   __syncthreads();
   if (t == 0) {
@@ -476,9 +485,38 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
     st_release_u64(fa.xready + u, fa.epoch);
   }
   trace_mark(p, 24);
-  // diagnostics: ||I - W X_T||_F
-  stage_w_over_x();
-  run_round();
+  tc_fence_before();
+  __syncthreads();
+  return SolverInfo{alpha, lmax, fallback};
+}
+
+// Diagnostics of the unit's solve, ||I - W X_T||_F, by one more product of the same kind as the
+// Newton-Schulz steps ([W; X_T] times X_T^T, 3xTF32). It runs after M' is published, off the
+// critical path: W is still in the solver's scratch, X_T^T in the combine's (the combine leaves
+// both unchanged).
+__device__ void solver_diagnostics(const Params& p, unsigned char* sm, uint32_t sbase, uint32_t tmem,
+                                   uint64_t* bars, int u, const SolverInfo& si) {
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int m = p.m;
+  const float* Ws = reinterpret_cast<const float*>(sm + kOffNsW);
+  const float* Xt = reinterpret_cast<const float*>(sm + kOffXt);
+  float* red = reinterpret_cast<float*>(sm + kOffNsVec) + 128;
+  const int q = w & 3, h = w >> 2;
+  const int r = 32 * q + lane, i = r & 63;
+  const bool top = r < 64;
+  float v[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) v[c] = top ? Ws[i * kQS + 16 * h + c] : Xt[(16 * h + c) * kQS + i];
+  ns_store(sm, r, h, v);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (t == 0) ns_issue(sbase, tmem, bars + kBarDiag, (m + 7) >> 3);
+  __syncwarp();
+  mbar_wait(bars + kBarDiag, 0, p.status, kStatusTimeout);
+  tc_fence_after();
+  float d[16];
+  tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 16 * h, d);
   float sq = 0.f, dummy = 0.f;
   if (top && i < m) {
 #pragma unroll
@@ -491,11 +529,11 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
   block_reduce2(sq, dummy, red);
   if (t == 0) {
     float* inf = p.info + (size_t)u * kInfoStride;
-    inf[kInfoAlpha] = alpha;
-    inf[kInfoLambdaMax] = lmax;
-    inf[kInfoFallback] = (float)fallback;
+    inf[kInfoAlpha] = si.alpha;
+    inf[kInfoLambdaMax] = si.lmax;
+    inf[kInfoFallback] = (float)si.fallback;
     inf[kInfoResidual] = sqrtf(sq);
-    if (!isfinite(lmax) || !isfinite(sq)) atomicOr(p.status, kStatusNonFinite);
+    if (!isfinite(si.lmax) || !isfinite(sq)) atomicOr(p.status, kStatusNonFinite);
   }
   tc_fence_before();
   __syncthreads();
@@ -508,7 +546,7 @@ __device__ void solver_cta(const Params& p, const FusedArgs& fa, unsigned char* 
 // lanes' rows spread the reads over all banks.
 template <int LT>
 __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float* Ls, unsigned char* cslot, int j0,
-                                            int m, int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
+                                            int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
   const int lane = threadIdx.x & 31;
   float acc[2][LT];
 #pragma unroll
@@ -571,28 +609,40 @@ __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float
         *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = __float2bfloat16_rn(c[b]);
       }
     }
-    // the last landmark group also writes the padding columns m..63 of its rows: zero, except
-    // column 63 = 1 on valid rows (it yields sum_i v_i in the C^T V product)
-    if (j0 + LT == m) {
-      const __nv_bfloat16 one = __float2bfloat16_rn(valid ? 1.f : 0.f), zero = __float2bfloat16_rn(0.f);
-      for (int col = m; col < 64; ++col)
-        *reinterpret_cast<__nv_bfloat16*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) = col == 63 ? one : zero;
-    }
+  }
+}
+
+// Padding columns m..63 of the rows rb + lane, rb + lane + 32: zero, except column 63 = 1 on valid
+// rows (it yields sum_i v_i in the C^T V product). Whole 16-byte column groups are written at once;
+// only the group that holds landmark m - 1 is written column by column.
+__device__ __forceinline__ void write_padding(unsigned char* cslot, int rb, int nrows, int m) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t one = 0x3f80u;   // bf16 1.0
+#pragma unroll
+  for (int a = 0; a < 2; ++a) {
+    const int row = rb + lane + 32 * a;
+    const bool valid = row < nrows;
+    int col = m;
+    for (; col < 64 && (col & 7) != 0; ++col)
+      *reinterpret_cast<uint16_t*>(cslot + sw128(row, col >> 3) + ((col & 7) << 1)) =
+          (col == 63 && valid) ? (uint16_t)one : (uint16_t)0;
+    for (int c8 = col >> 3; c8 < 8; ++c8)
+      *reinterpret_cast<uint4*>(cslot + sw128(row, c8)) = make_uint4(0u, 0u, 0u, (c8 == 7 && valid) ? (one << 16) : 0u);
   }
 }
 
 __device__ __forceinline__ void cross_dispatch(int lt, const unsigned char* Qs, const float* Ls, unsigned char* cslot,
-                                               int j0, int m, int rb, int nrows, float scale, float (&s1)[8],
+                                               int j0, int rb, int nrows, float scale, float (&s1)[8],
                                                float (&s2)[8]) {
   switch (lt) {
-    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
-    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, m, rb, nrows, scale, s1, s2); break;
+    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
     default: break;
   }
 }
@@ -624,31 +674,16 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
   const int m = p.m, nch = R.nchunks;
   float* Ls = reinterpret_cast<float*>(sm + kOffL);
   float* sred = reinterpret_cast<float*>(sm + kOffSr);   // [segment][row half][S1 64 | S2 64]
-  // Landmark groups: warps w and w + 8 share group w % 8 (rows 0-63 and 64-127). The groups
-  // start from m = 8 lbase + lextra split as evenly as possible; where some groups are one
-  // larger, group 0 hands up to two landmarks to smaller groups without raising the largest
-  // size, because warp 0 also issues the chunk products.
-  const int wg = w & 7, rh = w >> 3;
+  // (constant indices only: a variable index into the parameter arrays would copy them to the stack)
+  const int rh = w >> 3;
   int lt = 0, j0 = 0;
-  {
-    const int lbase = m / 8, lextra = m % 8;
-    int sz[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sz[i] = lbase + (i >= 8 - lextra ? 1 : 0);
-    int give = lextra > 0 ? min(2, min(sz[0], 8 - lextra)) : 0;
-#pragma unroll
-    for (int i = 1; i < 8; ++i)
-      if (give > 0 && sz[i] == lbase) {
-        ++sz[i];
-        --sz[0];
-        --give;
-      }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i < wg) j0 += sz[i];
-      if (i == wg) lt = sz[i];
+  for (int k = 0; k < kWarps; ++k)
+    if (k == w) {
+      lt = fa.wlt[k];
+      j0 = fa.wj0[k];
     }
-  }
+  const bool padder = w == (rh ? fa.padw[1] : fa.padw[0]);
   const float scale = p.neg_log2e_over_lam;
   // V chunk gc -> stage gc % 3 (its (gc / 3)-th fill)
   auto issue_v = [&](int gc) {
@@ -701,7 +736,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     }
     if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
-    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, m, 64 * rh, nrows, scale, s1, s2);
+    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
+    if (padder) write_padding(cslot, 64 * rh, nrows, m);
     if (gc == 1) trace_mark(p, 22);
     if (seg_last) {
       // this segment's column sums of C and C^2, per row half
@@ -787,32 +823,19 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   const double invN = 1.0 / (double)N;
   // candidates gf..gl; CTAs with an empty range (possible when there are fewer chunks than
   // CTAs) publish nothing and are dropped from the contributor table
-  const int gf = cta_of_row((long long)u * N, p, fa);
-  const int gl = cta_of_row((long long)(u + 1) * N - 1, p, fa);
+  const int nchu = (N + kChunk - 1) / kChunk;
+  const int gf = chunk_owner(u * nchu, p);
+  const int gl = chunk_owner(u * nchu + nchu - 1, p);
   const int ncand = gl - gf + 1;
-  // X^T of this unit (written by this CTA before its X flag)
-  {
-    constexpr int kNX = 4096 / kFT;
-    float xv[kNX];
-#pragma unroll
-    for (int i2 = 0; i2 < kNX; ++i2) {
-      const int e = t + kFT * i2, jr = e >> 6, l = e & 63;
-      xv[i2] = (jr < m && l < m) ? p.X[((size_t)u * m + jr) * m + l] : 0.f;
-    }
-#pragma unroll
-    for (int i2 = 0; i2 < kNX; ++i2) {
-      const int e = t + kFT * i2;
-      Xt[(e & 63) * kQS + (e >> 6)] = xv[i2];
-    }
-  }
+  // X^T of this unit is in shared memory (written by solver_cta at publication)
   int* wcount = reinterpret_cast<int*>(sm + kOffBp);
   bool nonempty = false;
   int rec_off = 0;
   if (t < ncand) {
     const int gg = gf + t;
-    const long long a = cta_start(gg, p, fa);
-    nonempty = cta_start(gg + 1, p, fa) > a;
-    rec_off = (gg * 2 + (a < (long long)u * N ? 1 : 0)) * kRec;
+    const int a = cta_start(gg, p);
+    nonempty = cta_start(gg + 1, p) > a;
+    rec_off = (gg * 2 + (a < u * N ? 1 : 0)) * kRec;
   }
   const unsigned bal = __ballot_sync(0xffffffffu, nonempty);
   if ((t & 31) == 0) wcount[t >> 5] = __popc(bal);
@@ -954,19 +977,27 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3b (row CTAs, while the unit's M' is being formed): DWC(V) of every chunk -> O (bf16),
-// the 3 x 3 depthwise taps (§关键设计 1 "ZV + DWC(V)", zero padding 1). The chunk's V rows with a
-// one-grid-row halo on each side arrive by TMA (SW128, boxes of 128 rows, rows outside the unit
-// read as zero), two chunks in flight where both tiles fit. Thread t owns 4 consecutive tokens of
-// one grid row (W % 4 == 0, so a group never wraps) and 4 channels (t % 16), weights in registers,
-// and slides the 3 x 6 input window along the group.
+// Phase 3b (row CTAs, while the unit's M' is being formed): DWC(V) of every chunk, the 3 x 3
+// depthwise taps (§关键设计 1 "ZV + DWC(V)", zero padding 1), rounded to bf16 and placed in the
+// chunk's pass-2 TMEM accumulator (columns 64 gc), on which pass 2's product then accumulates.
+// The chunk's V rows with a one-grid-row halo on each side arrive by TMA (SW128, boxes of 128
+// rows, rows outside the unit read as zero), two chunks in flight where both tiles fit. Thread t
+// owns 4 consecutive tokens of one grid row (W % 4 == 0, so a group never wraps) and 4 channels
+// (t % 16), weights in registers, and slides the 3 x 6 input window along the group. The results
+// go to a bf16 staging tile (SW128 rows, two alternating buffers), which one tcgen05 product with a
+// 64 x 64 identity (exact: every product is by 1 or 0, summed in fp32) copies into the chunk's TMEM
+// accumulator.
 // ---------------------------------------------------------------------------------------
-__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV) {
+__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint32_t sbase, uint32_t tmem,
+                        uint64_t* bars, const CUtensorMap* tmapV) {
   const int t = threadIdx.x, W = p.W;
   const int nbox = (kChunk + 2 * (W + 1) + kChunk - 1) / kChunk;
   const uint32_t hbytes = (uint32_t)nbox * 16384u;
-  const int nbuf = 2 * hbytes <= kHaloSpace ? 2 : 1;
+  const int nbuf = 2 * hbytes + 16384 <= kHaloSpace ? 2 : 1;
   const int nch = R.nchunks;
+  // staging buffers: C slot kMaxChunks - 1 (free: a CTA has at most kMaxChunks - 1 chunks, and the
+  // Q tile that slot held is consumed) and the halo region after the halo buffers
+  unsigned char* stg[2] = {sm + kOffC + (kMaxChunks - 1) * 16384, sm + kOffHb + nbuf * hbytes};
   auto issue = [&](int gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
@@ -976,10 +1007,39 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
     for (int b = 0; b < nbox; ++b)
       tma_load_3d(sm + kOffHb + bi * hbytes + b * 16384, tmapV, 0, lo - (W + 1) + kChunk * b, R.seg[s].u, hb);
   };
-  __syncthreads();   // pass 1 is done with the V stages, Q and L (the halo region)
+  // staged chunk gc -> its TMEM accumulator (columns 64 gc): D = S I over K = 64 channels, the
+  // identity (K-major B) in the M' area, which pass 2 fills only later
+  auto transfer = [&](int gc) {
+    tc_fence_after();
+    const uint32_t id = idesc(1, 128, 64, 0, 0);
+    const uint64_t sa = desc_sw128(sbase + (uint32_t)(stg[gc & 1] - sm), 16, 1024);
+    const uint64_t ib = desc_sw128(sbase + kOffMp, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + 64 * gc, sa + (uint64_t)(kk * 2), ib + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
+    mma_commit(bars + kBarDw + (gc & 1));
+  };
+  // transfer gc (the (gc >> 1)-th completion of its buffer's barrier) done
+  auto wait_transfer = [&](int gc) {
+    mbar_wait(bars + kBarDw + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
+  };
+  __syncthreads();   // pass 1 is done with the V stages, Q and L (the halo region), and with TMEM
   if (t == 0) {
     issue(0);
     if (nbuf == 2 && nch > 1) issue(1);
+  }
+  // the 64 x 64 bf16 identity, SW128 rows (row n, column k): 512 16-byte groups
+  for (int e = t; e < 512; e += kFT) {
+    const int n = e >> 3, c8 = e & 7;
+    const uint32_t one = 0x3f80u << (16 * (n & 1));
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if ((n >> 3) == c8) {
+      const int word = (n & 7) >> 1;
+      if (word == 0) v.x = one;
+      else if (word == 1) v.y = one;
+      else if (word == 2) v.z = one;
+      else v.w = one;
+    }
+    *reinterpret_cast<uint4*>(sm + kOffMp + sw128(n, c8)) = v;
   }
   const int grp = t >> 4, c4 = t & 15;   // tokens 4 grp .. 4 grp + 3 of the chunk, channels 4 c4 ..
   float wt[9][4];
@@ -998,14 +1058,14 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
     const int bi = gc % nbuf;
     mbar_wait(bars + kBarH + bi, (gc / nbuf) & 1, p.status, kStatusTimeout);   // fill gc / nbuf of buffer bi
     const int r0 = 4 * grp;                // chunk row of the group's first token
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
     if (r0 < nrows) {
       const int n0 = lo + r0, x0 = n0 % W;
       const unsigned char* hbuf = sm + kOffHb + bi * hbytes;
-      float acc[4][4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
 #pragma unroll
       for (int a = 0; a < 3; ++a) {
         // tile rows of tokens x0 - 1 .. x0 + 4 on grid row y + a - 1: r0 + a W + j, j = 0..5
@@ -1029,25 +1089,39 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint6
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(wt[a * 3 + b][e], v[i + b][e], acc[i][e]);
       }
-      __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * p.N * 64 + 4 * c4;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (r0 + i < nrows)
-          *reinterpret_cast<uint2*>(O + (size_t)(n0 + i) * 64) =
-              make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
     }
-    if (gc + 1 == nch) fence_async_global();   // pass 2 reads these O rows back by TMA
-    __syncthreads();
-    if (t == 0 && gc + nbuf < nch) issue(gc + nbuf);
+    // rows past the chunk's end stage zeros (their accumulator rows are never stored); staging
+    // buffer gc & 1 was last read by transfer gc - 2
+    if (gc >= 2) wait_transfer(gc - 2);
+    unsigned char* st = stg[gc & 1];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<uint2*>(st + sw128(r0 + i, c4 >> 1) + (c4 & 1) * 8) =
+          make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
+    fence_async_smem();
+    __syncthreads();   // staging gc written (and, at gc = 0, the identity), halo buffer bi read
+    if (t == 0) {
+      transfer(gc);
+      if (gc + nbuf < nch) issue(gc + nbuf);
+    }
   }
+  // the last transfers (earlier ones were waited before their buffer was reused)
+  if (nch >= 2) wait_transfer(nch - 2);
+  if (nch >= 1) wait_transfer(nch - 1);
+  tc_fence_before();
+  __syncthreads();
   trace_mark(p, 25);
 }
 
 // ---------------------------------------------------------------------------------------
 // Phase 4: O = C M' + b + DWC(V) for every chunk. M'^T and b of each segment's unit come from
-// its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region); the DWC
-// values are already in O (phase 3b) and come back by TMA four chunks ahead. All products are issued at once, each chunk into its own
-// 64-column TMEM accumulator with its own barrier, and the epilogues follow chunk by chunk.
+// its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region). Each
+// chunk's product accumulates onto the DWC values already in its TMEM accumulator (phase 3b); all
+// products are issued at once, each with its own barrier, and the epilogues (+ b, bf16) follow
+// chunk by chunk. The bf16 rows are staged in the chunk's C slot (free once its product is done)
+// and leave by TMA stores of 32-row quarters: warps w, w + 4, w + 8, w + 12 hold the same 32 rows
+// (16 channels each) and meet on named barrier 1 + w % 4 before warp w % 4 issues the quarter's
+// store.
 // ---------------------------------------------------------------------------------------
 __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
                           uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapO) {
@@ -1055,20 +1129,8 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffV; };
-  // DWC values of chunk gc (O rows, SW128) in ring buffer gc % kDwcRing after segment 1's M' image
-  auto dwc_buf = [&](int gc) { return sm + kOffV + 8192 + (gc % kDwcRing) * 16384; };
-  auto issue_dwc = [&](int gc) {
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    uint64_t* db = bars + kBarD + gc % kDwcRing;
-    mbar_expect_tx(db, 16384);
-    tma_load_3d(dwc_buf(gc), tmapO, 0, lo, R.seg[s].u, db);
-  };
-  __syncthreads();   // the DWC phase is done with the halo region; its O rows are fenced
-  if (t == 0) {
-    for (int gc = 0; gc < nch && gc < kDwcRing; ++gc) issue_dwc(gc);
+  if (t == 0)
     for (int s = 0; s < R.nseg; ++s) spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout);
-  }
   __syncthreads();
   trace_mark(p, 4);
   for (int s = 0; s < R.nseg; ++s) {
@@ -1092,45 +1154,40 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
     const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
     const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, 1u);
     mma_commit(bars + kBarP2 + gc);
   }
-  __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O);
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
   for (int gc = 0; gc < nch; ++gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    mbar_wait(bars + kBarD + gc % kDwcRing, (gc / kDwcRing) & 1, p.status, kStatusTimeout);
-    uint4 dw[2];
-#pragma unroll
-    for (int j = 0; j < 2; ++j) dw[j] = *reinterpret_cast<const uint4*>(dwc_buf(gc) + sw128(row, 2 * h + j));
     mbar_wait(bars + kBarP2 + gc, 0, p.status, kStatusTimeout);
     if (gc == 0) trace_mark(p, 29);
     tc_fence_after();
     float v[16];
     tmem_ld16(tmem + 64 * gc + ((uint32_t)(32 * q) << 16) + 16 * h, v);
-    if (row < nrows) {
-      uint4* orow = reinterpret_cast<uint4*>(O + ((size_t)R.seg[s].u * p.N + lo + row) * 64 + 16 * h);
-      const float* bs = bvec + 64 * s + 16 * h;
+    unsigned char* ob = sm + kOffC + gc * 16384;
+    const float* bs = bvec + 64 * s + 16 * h;
 #pragma unroll
-      for (int k4 = 0; k4 < 2; ++k4) {
-        const uint32_t wv[4] = {dw[k4].x, dw[k4].y, dw[k4].z, dw[k4].w};
-        uint32_t o[4];
+    for (int k4 = 0; k4 < 2; ++k4) {
+      uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int cc = 8 * k4 + 2 * e;
-          o[e] = pack_bf16(v[cc] + bs[cc] + bf_lo(wv[e]), v[cc + 1] + bs[cc + 1] + bf_hi(wv[e]));
-        }
-        orow[k4] = make_uint4(o[0], o[1], o[2], o[3]);
+      for (int e = 0; e < 4; ++e) {
+        const int cc = 8 * k4 + 2 * e;
+        o[e] = pack_bf16(v[cc] + bs[cc], v[cc + 1] + bs[cc + 1]);
       }
+      *reinterpret_cast<uint4*>(ob + sw128(row, 2 * h + k4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    if (gc + kDwcRing < nch) {
-      __syncthreads();   // ring buffer gc % kDwcRing has been read
-      if (t == 0) issue_dwc(gc + kDwcRing);
+    fence_async_smem();
+    named_bar_sync(1 + q, 128);
+    // rows past the unit's end (a short last chunk) fall outside the tensor and are not written
+    if (h == 0 && lane == 0 && 32 * q < nrows) {
+      tma_store_3d(tmapO, 0, lo + 32 * q, R.seg[s].u, ob + 4096 * q);
+      bulk_commit_group();
     }
     if (gc < 2) trace_mark(p, 30 + gc);
   }
+  if (h == 0 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   trace_mark(p, 6);
@@ -1158,7 +1215,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   }
   // the row plan lives in shared memory: it is read at every chunk boundary by every thread
   Rows* Rsm = reinterpret_cast<Rows*>(sm + kOffRows);
-  if (t == 0) *Rsm = cta_rows(g, p, fa);
+  if (t == 0) *Rsm = cta_rows(g, p);
   const Rows& R = *Rsm;
   const bool solver = g < U;
   if (t == 0) {
@@ -1227,20 +1284,16 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // solver CTAs take no rows (R.nchunks == 0): solve, combine, then the diagnostics
   if (solver) {
-    solver_cta(p, fa, sm, sbase, tmem, bars, g);
-    __syncthreads();   // the solver's scratch in the C region is free
-    if (t == 0) pass1_prefetch(R, sm, bars, &tmapV, &tmapQ);
-  }
-  __syncthreads();
-  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
-  trace_mark(p, 3);
-  // the unit's combine runs on its solver CTA after this CTA's own records are out (no self-wait)
-  if (solver) {
-    __syncthreads();
+    const SolverInfo si = solver_cta(p, fa, sm, sbase, tmem, bars, g);
+    trace_mark(p, 3);
     solver_combine(p, fa, sm, g);
+    solver_diagnostics(p, sm, sbase, tmem, bars, g, si);
   }
-  if (R.nchunks > 0) dwc_all(p, R, sm, bars, &tmapV);
+  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
+  if (!solver) trace_mark(p, 3);
+  if (R.nchunks > 0) dwc_all(p, R, sm, sbase, tmem, bars, &tmapV);
   if (R.nchunks > 0) pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
   __syncthreads();
   trace_mark(p, 15);
@@ -1262,17 +1315,6 @@ size_t fused_workspace_bytes(int U) {
   return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * kImgBytes;
 }
 
-// Row share of a solver CTA (in 1/16 of a plain CTA's share): they start their rows only after
-// the Newton-Schulz chain. LFA_SOLVER_ROW_SHARE (0..16) overrides the default.
-static int solver_share16() {
-  const char* e = getenv("LFA_SOLVER_ROW_SHARE");
-  if (e) {
-    const int v = atoi(e);
-    if (v >= 0 && v <= 16) return v;
-  }
-  return 0;
-}
-
 // Decide whether the fused kernel serves this shape on the current device; returns the grid size
 // (0 if not eligible).
 int fused_grid(const Params& p) {
@@ -1286,24 +1328,23 @@ int fused_grid(const Params& p) {
   if (major != 10) return 0;
   const int G = sms < kMaxGrid ? sms : kMaxGrid;
   if (2 * p.U > G) return 0;
-  const int ws16 = solver_share16();
-  const long long totw16 = (long long)ws16 * p.U + 16ll * (G - p.U);
-  // chunks of a plain CTA: resident C capacity, and at most two units (segments) per CTA
+  // chunks of a row CTA: resident C capacity, and at most two units (segments) per CTA
   const long long nchu = (p.N + kChunk - 1) / kChunk;
-  const long long cpc = ((long long)p.U * nchu * 16 + totw16 - 1) / totw16;
+  const long long cpc = ((long long)p.U * nchu + (G - p.U) - 1) / (G - p.U);
   if (cpc > kMaxChunks - 1 || cpc > nchu) return 0;   // one C slot stays free for the Q chunk
   // the DWC phase's token groups of 4 stay on one grid row
   if (p.W % 4 != 0) return 0;
-  // its V halo tile (a chunk plus one grid row on each side, in boxes of 128 rows) must fit
-  if ((long long)((kChunk + 2 * (p.W + 1) + kChunk - 1) / kChunk) * 16384 > (long long)kHaloSpace) return 0;
+  // its V halo tile (a chunk plus one grid row on each side, in boxes of 128 rows) and one DWC
+  // staging tile must fit the halo region
+  if ((long long)((kChunk + 2 * (p.W + 1) + kChunk - 1) / kChunk) * 16384 + 16384 > (long long)kHaloSpace) return 0;
   // replay the row partition: contributors of every unit must fit the offset table
   {
     int worst = 0, cur_u = -1, cur = 0;
     for (int g = 0; g < G; ++g) {
-      const long long r0 = part_start(g, p.U, p.N, ws16, totw16);
-      const long long r1 = part_start(g + 1, p.U, p.N, ws16, totw16);
+      const int r0 = part_start(g, p.U, p.N, G);
+      const int r1 = part_start(g + 1, p.U, p.N, G);
       if (r1 <= r0) continue;
-      for (long long u = r0 / p.N; u <= (r1 - 1) / p.N; ++u) {
+      for (int u = r0 / p.N; u <= (r1 - 1) / p.N; ++u) {
         if ((int)u != cur_u) {
           cur_u = (int)u;
           cur = 0;
@@ -1327,32 +1368,73 @@ int fused_grid(const Params& p) {
 constexpr int kTmapCache = 32;   // Q, V and O maps of a few rotating buffer sets
 struct TmapCache {
   const void* ptr[kTmapCache];
-  int N[kTmapCache], U[kTmapCache], sw[kTmapCache];
+  int N[kTmapCache], U[kTmapCache], sw[kTmapCache], box[kTmapCache];
   CUtensorMap map[kTmapCache];
   int next;
 };
 static TmapCache g_tmaps;
 static std::mutex g_tmaps_mu;
 
-// [U][N][64] bf16 viewed as {64, N, U}, boxes of 128 rows; 128-byte swizzle or plain rows
-static bool tmap_for(const void* X, int N, int U, bool swizzle, CUtensorMap* out) {
+// [U][N][64] bf16 viewed as {64, N, U}, boxes of box_rows rows; 128-byte swizzle or plain rows
+static bool tmap_for(const void* X, int N, int U, int box_rows, bool swizzle, CUtensorMap* out) {
   std::lock_guard<std::mutex> lk(g_tmaps_mu);
   for (int i = 0; i < kTmapCache; ++i)
-    if (g_tmaps.ptr[i] == X && g_tmaps.N[i] == N && g_tmaps.U[i] == U && g_tmaps.sw[i] == (int)swizzle) {
+    if (g_tmaps.ptr[i] == X && g_tmaps.N[i] == N && g_tmaps.U[i] == U && g_tmaps.sw[i] == (int)swizzle &&
+        g_tmaps.box[i] == box_rows) {
       *out = g_tmaps.map[i];
       return true;
     }
   CUtensorMap m;
-  if (!make_tmap_rows_bf16(&m, X, (uint64_t)N, (uint64_t)U, kChunk, swizzle)) return false;
+  if (!make_tmap_rows_bf16(&m, X, (uint64_t)N, (uint64_t)U, (uint32_t)box_rows, swizzle)) return false;
   const int i = g_tmaps.next;
   g_tmaps.next = (i + 1) % kTmapCache;
   g_tmaps.ptr[i] = X;
   g_tmaps.N[i] = N;
   g_tmaps.U[i] = U;
   g_tmaps.sw[i] = (int)swizzle;
+  g_tmaps.box[i] = box_rows;
   g_tmaps.map[i] = m;
   *out = m;
   return true;
+}
+
+// Pass-1 warp plan. Each row half's m landmarks are cut into 8 contiguous ranges, one per warp of
+// that half (warps 0-7 take rows 0-63, warps 8-15 rows 64-127); warp w issues on scheduler w % 4,
+// which therefore serves four ranges. Every range gets b = m / 8 landmarks; the e = m % 8 ranges of
+// each half that take one more go to the least-loaded scheduler, scheduler 0 counted one landmark
+// heavier because its warp 0 also issues the chunk products. Each half's padding columns go to a
+// warp on the least-loaded scheduler, warp 0 avoided.
+static void plan_pass1_warps(int m, FusedArgs& fa) {
+  const int b = m / 8, e = m % 8;
+  int sz[kWarps], load[4] = {1, 0, 0, 0};
+  for (int w = 0; w < kWarps; ++w) {
+    sz[w] = b;
+    load[w % 4] += b;
+  }
+  for (int i = 0; i < 2 * e; ++i) {
+    const int half = i % 2;
+    int best = -1;
+    for (int k = 0; k < 8; ++k) {
+      const int w = 8 * half + k;
+      if (sz[w] != b || w == 0) continue;
+      if (best < 0 || load[w % 4] < load[best % 4]) best = w;
+    }
+    if (best < 0) best = 0;   // only when every other warp of half 0 already has b + 1
+    ++sz[best];
+    ++load[best % 4];
+  }
+  for (int half = 0; half < 2; ++half) {
+    int j = 0, best = -1;
+    for (int k = 0; k < 8; ++k) {
+      const int w = 8 * half + k;
+      fa.wj0[w] = (unsigned char)j;
+      fa.wlt[w] = (unsigned char)sz[w];
+      j += sz[w];
+      if (w == 0) continue;
+      if (best < 0 || load[w % 4] < load[best % 4] || (load[w % 4] == load[best % 4] && sz[w] < sz[best])) best = w;
+    }
+    fa.padw[half] = (unsigned char)best;
+  }
 }
 
 cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws, unsigned long long epoch,
@@ -1362,13 +1444,11 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
     if (e != cudaSuccess) return e;
   }
   CUtensorMap tmap, tmapq, tmapo;
-  if (!tmap_for(p.V, p.N, p.U, true, &tmap)) return cudaErrorInvalidValue;
-  if (!tmap_for(p.Q, p.N, p.U, true, &tmapq)) return cudaErrorInvalidValue;
-  if (!tmap_for(p.O, p.N, p.U, true, &tmapo)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.V, p.N, p.U, kChunk, true, &tmap)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.Q, p.N, p.U, kChunk, true, &tmapq)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.O, p.N, p.U, 32, true, &tmapo)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.epoch = epoch;
-  fa.ws16 = solver_share16();
-  fa.totw16 = fa.ws16 * p.U + 16 * (G - p.U);
   fa.gbar = reinterpret_cast<unsigned long long*>(fused_ws);
   const size_t fs = flag_stride(p.U);
   fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + 256);
@@ -1376,6 +1456,7 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + 2 * fs);
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
   fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
+  plan_pass1_warps(p.m, fa);
   Params pp = p;
   void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo};
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
