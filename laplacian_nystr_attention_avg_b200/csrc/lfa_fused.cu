@@ -90,7 +90,6 @@ constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64]
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(kOffBp + (kFT / 16) * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
-static_assert(kMaxChunks <= kFT / 32, "pass 2 issues one chunk's product per warp");
 
 // mbarrier slots
 constexpr int kBarV = 0;      // [3] V stage filled by TMA
@@ -99,7 +98,8 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarDiag = kBarP2;   // solver CTAs (which run no pass 2): the diagnostics product
+constexpr int kBarDiag = kBarP2;       // solver CTAs (which run no pass 2): the diagnostics product
+constexpr int kBarComb = kBarP2 + 1;   // solver CTAs: the combine's M = X A product
 constexpr int kBarDw = 17;    // [2] DWC transfer product of staging buffer b done
 constexpr int kNumBars = kBarDw + 2;
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
@@ -807,7 +807,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
 // b = (1/N - s o mu)^T M. M'^T is written as the bf16 SW128 image of pass 2's B operand and
 // published with b under a release flag.
 // ---------------------------------------------------------------------------------------
-__device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, int u) {
+__device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, uint32_t sbase,
+                               uint32_t tmem, uint64_t* bars, int u) {
   const int t = threadIdx.x;
   const int m = p.m, N = p.N;
   float* As = reinterpret_cast<float*>(sm + kOffAs);
@@ -913,57 +914,70 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
     }
   }
   __syncthreads();
-  for (int e = t; e < 64 * 64; e += kFT) {
-    const int a = e >> 6, k = e & 63;
-    float v = 0.f;
-    if (a < m) {
-      const float P = As[a * kQS + k];
-      v = p.whiten ? scs[a] * (P - mus[a] * svs[k]) + svs[k] * invNf : P;
-    }
-    As[a * kQS + k] = v;
-  }
-  __syncthreads();
   trace_mark(p, 29);
   {
-    // M = X A with a 2 x 4 register tile per thread; M' = diag(s) M as bf16 (K-major B of pass 2)
-    const int jb = t >> 4, kb = t & 15;
-    float acc[2][4] = {};
-#pragma unroll 4
-    for (int l = 0; l < m; ++l) {
-      const float2 x2 = *reinterpret_cast<const float2*>(Xt + l * kQS + 2 * jb);
-      const float4 a4 = *reinterpret_cast<const float4*>(As + l * kQS + 4 * kb);
-      const float xv[2] = {x2.x, x2.y}, av[4] = {a4.x, a4.y, a4.z, a4.w};
+    // M = X A on tcgen05 in 3xTF32, as one product of the Newton-Schulz kind: stacked rows
+    // [X; A^T] times A (its bottom half, transposed), so D_top = X A. A is folded on the fly:
+    // A[l][k] = s_l (P[l][k] - mu_l sum_i v_ik) + sum_i v_ik / N. Thread (w, lane) stages row
+    // r = 32 (w % 4) + lane, columns 16 (w / 4) ..
+    const int w = t >> 5, lane = t & 31, q = w & 3, h = w >> 2, r = 32 * q + lane, i = r & 63;
+    const bool top = r < 64;
+    float v[16];
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(xv[x], av[y], acc[x][y]);
-    }
-    unsigned char* mp = sm + kOffMp;
-    float bp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const int jr = 2 * jb + x;
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int k = 4 * kb + y;
-        float v = 0.f;
-        if (jr < m) {
-          v = p.whiten ? scs[jr] * acc[x][y] : acc[x][y];
-          if (p.whiten) bp[y] += (invNf - scs[jr] * mus[jr]) * acc[x][y];
+    for (int c = 0; c < 16; ++c) {
+      const int l = 16 * h + c;
+      if (top) {
+        v[c] = Xt[l * kQS + i];
+      } else {
+        float a = 0.f;
+        if (l < m) {
+          const float P = As[l * kQS + i];
+          a = p.whiten ? scs[l] * (P - mus[l] * svs[i]) + svs[i] * invNf : P;
         }
-        *reinterpret_cast<__nv_bfloat16*>(mp + sw128(k, jr >> 3) + ((jr & 7) << 1)) = __float2bfloat16_rn(v);
+        v[c] = a;
       }
     }
+    ns_store(sm, r, h, v);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (t == 0) ns_issue(sbase, tmem, bars + kBarComb, (m + 7) >> 3);
+    __syncwarp();
+    mbar_wait(bars + kBarComb, 0, p.status, kStatusTimeout);
+    tc_fence_after();
+    float d[16];
+    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 16 * h, d);
+    if (top) {
+      // M' = diag(s) M as bf16 (K-major B of pass 2: image row k = channel, column i = landmark,
+      // zero for i >= m); b = (1/N - s o mu)^T M, reduced over the 64 rows
+      const bool in = i < m;
+      const float sc = in ? (p.whiten ? scs[i] : 1.f) : 0.f;
+      const float wb = (in && p.whiten) ? invNf - scs[i] * mus[i] : 0.f;
+      unsigned char* mp = sm + kOffMp;
+      float bp[16];
 #pragma unroll
-    for (int y = 0; y < 4; ++y) bps[jb * 64 + 4 * kb + y] = bp[y];
+      for (int c = 0; c < 16; ++c) {
+        *reinterpret_cast<__nv_bfloat16*>(mp + sw128(16 * h + c, i >> 3) + ((i & 7) << 1)) =
+            __float2bfloat16_rn(sc * d[c]);
+        bp[c] = wb * d[c];
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        for (int o = 16; o > 0; o >>= 1) bp[c] += __shfl_xor_sync(0xffffffffu, bp[c], o);
+      if (lane == 0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) bps[q * 64 + 16 * h + c] = bp[c];
+      }
+    }
   }
+  tc_fence_before();
   __syncthreads();
   trace_mark(p, 30);
   unsigned char* img = fa.mimg + (size_t)u * kImgBytes;
   if (t < 64) {
     float b = 0.f;
 #pragma unroll
-    for (int q = 0; q < kFT / 16; ++q) b += bps[q * 64 + t];
+    for (int q = 0; q < 2; ++q) b += bps[q * 64 + t];
     reinterpret_cast<float*>(img + 8192)[t] = b;
   }
   for (int e = t; e < 512; e += kFT)
@@ -1100,10 +1114,9 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint3
           make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
     fence_async_smem();
     __syncthreads();   // staging gc written (and, at gc = 0, the identity), halo buffer bi read
-    if (t == 0) {
-      transfer(gc);
-      if (gc + nbuf < nch) issue(gc + nbuf);
-    }
+    // two issuing threads in different warps, so that neither warp's chunk is late by both
+    if (t == 0) transfer(gc);
+    if (t == 32 && gc + nbuf < nch) issue(gc + nbuf);
   }
   // the last transfers (earlier ones were waited before their buffer was reused)
   if (nch >= 2) wait_transfer(nch - 2);
@@ -1143,19 +1156,21 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   tc_fence_before();
   __syncthreads();
   trace_mark(p, 5);
-  // chunk gc's product is issued by lane 0 of warp gc (separate accumulators and barriers, so the
-  // issues proceed in parallel and the results do not depend on their order)
-  if (lane == 0 && w < nch) {
-    const int gc = w;
+  // one thread (in warp 15, which issues no stores) issues the products in chunk order, each
+  // chunk's four followed by its commit, so the epilogues can start while later chunks are issued
+  if (t == kFT - 32) {
     tc_fence_after();
     const uint32_t id = idesc(1, 128, 64, 0, 0);
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
-    const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
+    for (int gc = 0; gc < nch; ++gc) {
+      int s, lo, nrows;
+      R.chunk(gc, s, lo, nrows);
+      const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
+      const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, 1u);
-    mma_commit(bars + kBarP2 + gc);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, 1u);
+      mma_commit(bars + kBarP2 + gc);
+    }
   }
   const int q = w & 3, h = w >> 2, row = 32 * q + lane;
   for (int gc = 0; gc < nch; ++gc) {
@@ -1288,7 +1303,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   if (solver) {
     const SolverInfo si = solver_cta(p, fa, sm, sbase, tmem, bars, g);
     trace_mark(p, 3);
-    solver_combine(p, fa, sm, g);
+    solver_combine(p, fa, sm, sbase, tmem, bars, g);
     solver_diagnostics(p, sm, sbase, tmem, bars, g, si);
   }
   if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
