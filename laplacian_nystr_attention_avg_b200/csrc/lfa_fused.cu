@@ -44,6 +44,7 @@ using namespace sm100;
 
 constexpr int kFT = 512;                  // threads per CTA (16 warps, at most 128 registers each)
 constexpr int kWarps = kFT / 32;
+constexpr int kV1Thread = 12 * 32;        // pass 1: issues the V chunk loads (warp 12, scheduler 0)
 constexpr int kChunk = 128;               // token rows per chunk
 constexpr int kMaxChunks = 8;             // resident C chunks per CTA
 constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q, L and halo tiles
@@ -760,8 +761,9 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     if (gc < 2) trace_mark(p, 11 + gc);
     // the next V chunk, issued after the barrier so that this thread's proxy fence above does not
     // wait for it: stage (gc + 1) % 3 last held chunk gc - 2, whose product went out at this
-    // chunk's start
-    if (t == 0 && gc >= 1 && gc + 1 < nch) {
+    // chunk's start. Warp 12 issues it (warp 0, which issues the products, starts its distances
+    // late; the other warps of its scheduler finish early).
+    if (t == kV1Thread && gc >= 1 && gc + 1 < nch) {
       if (gc >= 2) wait_mma(gc - 2);
       issue_v(gc + 1);
     }
@@ -1417,8 +1419,9 @@ static bool tmap_for(const void* X, int N, int U, int box_rows, bool swizzle, CU
 // that half (warps 0-7 take rows 0-63, warps 8-15 rows 64-127); warp w issues on scheduler w % 4,
 // which therefore serves four ranges. Every range gets b = m / 8 landmarks; the e = m % 8 ranges of
 // each half that take one more go to the least-loaded scheduler, scheduler 0 counted one landmark
-// heavier because its warp 0 also issues the chunk products. Each half's padding columns go to a
-// warp on the least-loaded scheduler, warp 0 avoided.
+// heavier because its warp 0 also issues the chunk products. Each half's padding columns go to
+// scheduler 0's other warp of that half (warps 4 and 8): warp 0 starts its distances late while it
+// issues the products, so the other warps of its scheduler finish first.
 static void plan_pass1_warps(int m, FusedArgs& fa) {
   const int b = m / 8, e = m % 8;
   int sz[kWarps], load[4] = {1, 0, 0, 0};
@@ -1439,16 +1442,14 @@ static void plan_pass1_warps(int m, FusedArgs& fa) {
     ++load[best % 4];
   }
   for (int half = 0; half < 2; ++half) {
-    int j = 0, best = -1;
+    int j = 0;
     for (int k = 0; k < 8; ++k) {
       const int w = 8 * half + k;
       fa.wj0[w] = (unsigned char)j;
       fa.wlt[w] = (unsigned char)sz[w];
       j += sz[w];
-      if (w == 0) continue;
-      if (best < 0 || load[w % 4] < load[best % 4] || (load[w % 4] == load[best % 4] && sz[w] < sz[best])) best = w;
     }
-    fa.padw[half] = (unsigned char)best;
+    fa.padw[half] = (unsigned char)(half == 0 ? 4 : 8);
   }
 }
 
