@@ -192,10 +192,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
-// Orders this thread's earlier generic-proxy global writes before later async-proxy (TMA) reads.
-__device__ __forceinline__ void fence_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // 16-byte global load through L2, kept in program order with the other asm statements (the
 // compiler may not sink it to its use, which would expose its latency there)
