@@ -34,6 +34,11 @@ design notes with its reason):
       -(1/lam) sign(x - y) k, with sign(0) = 0.
   R10 alpha is held constant in the backward pass (stop-gradient).
   R11 exactly T Newton-Schulz steps, no early exit.
+  R12 (alternative reading of R5, selected by batch_stats=True) the note's whitening
+      statistics "over a batch" of similarity vectors: mu and var of landmark column l
+      are taken over the B*N rows of every unit that shares the head h (all batch
+      elements), population variance; C~ of each unit is then formed as in R6 with
+      that unit's own N in the 1/N offset. Forward only.
 
 Parity pins (tests/test_oracle_*.py): closed forms of the kernel, scipy cdist,
 torch avg_pool2d / conv2d in float64, the per-step eigen closed form of
@@ -164,6 +169,20 @@ def whiten_columns(C: np.ndarray, eps: float):
     return (C - mu) / np.sqrt(var + eps) + 1.0 / N, mu, var
 
 
+def pooled_column_stats(Cs: List[np.ndarray]):
+    """R12: per-column mean and population variance over the stacked rows of several
+    units' cross kernels ([P1] 关键设计 1, statistics over a batch). Returns (mu, var)."""
+    S = np.concatenate([np.asarray(C, dtype=np.float64) for C in Cs], axis=0)
+    mu = S.mean(axis=0)
+    var = ((S - mu) ** 2).mean(axis=0)
+    return mu, var
+
+
+def batch_groups(B: int, heads: int) -> List[List[int]]:
+    """R12: the units u = b*heads + h that pool their statistics: one group per head."""
+    return [[b * heads + h for b in range(B)] for h in range(heads)]
+
+
 def dwc3x3(Vu: np.ndarray, w: np.ndarray, H: int, W: int) -> np.ndarray:
     """DWC(V): per-channel 3x3 cross-correlation with zero padding 1 ([P1] 整体框架
     flowchart node "DWC(V) 深度卷积"; 关键设计 1 output ZV + DWC(V); R8).
@@ -216,9 +235,12 @@ class UnitForward:
     iterates: Optional[List[np.ndarray]] = None
 
 
-def unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten=True, keep_iterates=False) -> UnitForward:
+def unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten=True, keep_iterates=False,
+                 stats=None) -> UnitForward:
     """Forward pass of one unit, in the pages' order ([P1] 整体框架 flowchart):
     pool -> Laplacian kernels -> Newton-Schulz W^+ -> whitening -> C~ (X (C~^T V)) + DWC(V).
+
+    ``stats`` = (mu, var) replaces the unit's own column statistics (R12).
     """
     Qu = np.asarray(Qu, dtype=np.float64)
     Vu = np.asarray(Vu, dtype=np.float64)
@@ -228,7 +250,10 @@ def unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten=True, keep_iterates=Fal
     Wm = landmark_gram(L, lam, eps)
     ac = select_alpha(Wm)
     X, res, its = newton_schulz(Wm, ac.alpha, T, keep_iterates)
-    if whiten:
+    if whiten and stats is not None:
+        mu, var = stats
+        Ct = (C - mu) / np.sqrt(var + eps) + 1.0 / C.shape[0]
+    elif whiten:
         Ct, mu, var = whiten_columns(C, eps)
     else:
         Ct, mu, var = C, None, None
@@ -313,12 +338,14 @@ class Forward:
     units: List[UnitForward]
 
 
-def forward(Q, V, dwc, wl, whiten=True, units=None, keep_units=True) -> Forward:
+def forward(Q, V, dwc, wl, whiten=True, units=None, keep_units=True, batch_stats=False) -> Forward:
     """Oracle forward over all (or the listed) units of a workload.
 
     Q, V: [B, heads, N, d] array-likes (float values already in the storage
     precision); dwc: [heads, d, 3, 3]. ``units`` restricts to a list of flat
-    unit indices u = b*heads + h (others are left zero).
+    unit indices u = b*heads + h (others are left zero). ``batch_stats`` selects
+    the R12 reading: whitening statistics pooled over the batch, per head (the
+    pooled statistics always use every batch element, also when ``units`` is set).
     """
     Q = np.asarray(Q, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
@@ -328,9 +355,21 @@ def forward(Q, V, dwc, wl, whiten=True, units=None, keep_units=True) -> Forward:
     Oa = np.zeros_like(Q)
     us = []
     todo = range(B * nh) if units is None else units
+    pooled = {}
+    if whiten and batch_stats:
+        for grp in batch_groups(B, nh):
+            Cs = []
+            for u in grp:
+                b, h = divmod(u, nh)
+                L = pool_landmarks(Q[b, h], wl.H, wl.W, wl.r)
+                Cs.append(laplacian_kernel(Q[b, h], L, wl.lam))
+            st = pooled_column_stats(Cs)
+            for u in grp:
+                pooled[u] = st
     for u in todo:
         b, h = divmod(u, nh)
-        f = unit_forward(Q[b, h], V[b, h], w[h], wl.H, wl.W, wl.r, wl.lam, wl.eps, wl.T, whiten)
+        f = unit_forward(Q[b, h], V[b, h], w[h], wl.H, wl.W, wl.r, wl.lam, wl.eps, wl.T, whiten,
+                         stats=pooled.get(u))
         O[b, h] = f.O
         Oa[b, h] = f.O_attn
         us.append(f if keep_units else None)

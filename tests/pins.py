@@ -221,6 +221,60 @@ def check_whitened_assembly_vs_solve():
     assert np.allclose(g.O_attn, ref, rtol=0, atol=1e-9 * np.abs(ref).max())
 
 
+# --- batch-pooled whitening statistics (reading R12) ----------------------------
+
+class _BatchWl:
+    """Minimal workload record for the oracle's whole-call forward."""
+
+    def __init__(self, H, W, r, lam, eps, T):
+        self.H, self.W, self.r, self.lam, self.eps, self.T = H, W, r, lam, eps, T
+
+
+def _batch_case(B, heads, seed, H=8, W=8, d=8, r=2, replicate=False):
+    rng = _rng(seed)
+    N = H * W
+    shape = (1 if replicate else B, heads, N, d)
+    q = rng.standard_normal(shape)
+    v = rng.standard_normal(shape)
+    if replicate:
+        q = np.repeat(q, B, axis=0)
+        v = np.repeat(v, B, axis=0)
+    w = rng.standard_normal((heads, d, 3, 3)) * 0.1
+    return q, v, w, _BatchWl(H, W, r, 2.0, 1e-6, 16)
+
+
+def check_batch_stats_single_batch():
+    # B = 1: the pooled statistics are the unit's own, so the two readings coincide
+    q, v, w, wl = _batch_case(1, 3, 51)
+    a = O.forward(q, v, w, wl)
+    b = O.forward(q, v, w, wl, batch_stats=True)
+    assert np.allclose(a.O, b.O, rtol=0, atol=1e-12 * np.abs(a.O).max())
+
+
+def check_batch_stats_replicated():
+    # identical batch elements: pooling copies of the same rows leaves mean and variance unchanged
+    q, v, w, wl = _batch_case(4, 2, 52, replicate=True)
+    a = O.forward(q, v, w, wl)
+    b = O.forward(q, v, w, wl, batch_stats=True)
+    assert np.allclose(a.O, b.O, rtol=0, atol=1e-10 * np.abs(a.O).max())
+
+
+def check_batch_stats_vs_sklearn():
+    # per head: standard scaling of the vertically stacked C of all batch elements
+    from sklearn.preprocessing import StandardScaler
+    B, heads = 3, 2
+    q, v, w, wl = _batch_case(B, heads, 53)
+    wl.eps = 0.0
+    f = O.forward(q, v, w, wl, batch_stats=True)
+    N = q.shape[2]
+    for h in range(heads):
+        units = [b * heads + h for b in range(B)]
+        Cs = [f.units[u].C for u in units]
+        ref = StandardScaler().fit_transform(np.concatenate(Cs, axis=0)) + 1.0 / N
+        got = np.concatenate([f.units[u].Ct for u in units], axis=0)
+        assert np.allclose(got, ref, rtol=1e-10, atol=1e-12), f"head {h}"
+
+
 # --- DWC ------------------------------------------------------------------------
 
 def check_dwc_vs_conv2d():
@@ -365,4 +419,5 @@ ALL_PINS = [
     check_ns_kappa50_and_quadratic, check_nystrom_r1_dense, check_whitening_moments,
     check_whitening_vs_sklearn, check_whitened_assembly_vs_solve, check_dwc_vs_conv2d,
     check_dwc_taps, check_backward_fd, check_injectivity_generic,
+    check_batch_stats_single_batch, check_batch_stats_replicated, check_batch_stats_vs_sklearn,
 ]

@@ -11,7 +11,8 @@ from tests import pins
 
 _orig = {name: getattr(O, name) for name in (
     "laplacian_kernel", "l1_distances", "pool_landmarks", "landmark_gram", "newton_schulz",
-    "whiten_columns", "dwc3x3", "_sign_contractions", "select_alpha")}
+    "whiten_columns", "dwc3x3", "_sign_contractions", "select_alpha", "pooled_column_stats",
+    "batch_groups")}
 
 
 def _kernel_no_lambda(X, Y, lam):
@@ -83,6 +84,20 @@ def _whiten_sample_var(C, eps):
     return (C - mu) / np.sqrt(var + eps) + 1.0 / N, mu, var
 
 
+def _pooled_sample_var(Cs):
+    S = np.concatenate(Cs, axis=0)
+    mu = S.mean(axis=0)
+    return mu, ((S - mu) ** 2).sum(axis=0) / (S.shape[0] - 1)
+
+
+def _pooled_first_unit_only(Cs):
+    return _orig["pooled_column_stats"](Cs[:1])
+
+
+def _groups_across_heads(B, heads):
+    return [list(range(B * heads))]
+
+
 def _dwc_convolution(Vu, w, H, W):
     return _orig["dwc3x3"](Vu, w[:, ::-1, ::-1].copy(), H, W)
 
@@ -104,6 +119,10 @@ MUTATIONS = [
     ("whiten_no_offset", "whiten_columns", _whiten_no_offset, [pins.check_whitening_moments]),
     ("whiten_sample_variance", "whiten_columns", _whiten_sample_var, [pins.check_whitening_vs_sklearn]),
     ("dwc_convolution_not_correlation", "dwc3x3", _dwc_convolution, [pins.check_dwc_vs_conv2d]),
+    ("batch_stats_sample_variance", "pooled_column_stats", _pooled_sample_var, [pins.check_batch_stats_vs_sklearn]),
+    ("batch_stats_first_unit_only", "pooled_column_stats", _pooled_first_unit_only,
+     [pins.check_batch_stats_vs_sklearn]),
+    ("batch_stats_pooled_across_heads", "batch_groups", _groups_across_heads, [pins.check_batch_stats_vs_sklearn]),
     ("kernel_gradient_sign_as_printed", "_sign_contractions", _sign_as_printed,
      [lambda: pins.check_backward_fd([(8, 8, 8, 2, 2.0, 1e-3, 24, 44, True)])]),
 ]
