@@ -40,6 +40,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["lfa", "reference"], default="lfa")
     ap.add_argument("--workload", default="pvt1")
+    ap.add_argument("--whiten", choices=["unit", "batch"], default="unit",
+                    help="column statistics per (batch, head) unit, or pooled per head over the batch "
+                         "(per-stage kernels; no CPU baseline)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -278,7 +281,8 @@ def main():
 
     wl = WORKLOADS[args.workload]
     x = make_inputs(wl, seed=rank)
-    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl), x.dwc, str(dev))
+    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, True if args.whiten == "unit" else "batch"),
+                                        x.dwc, str(dev))
     set_bytes = 3 * wl.units * wl.N * wl.d * x.Q_store.element_size()
     n_sets = max(2, math.ceil(1.8 * L2_BYTES / set_bytes))
     Qs = [x.Q_store.to(dev) for _ in range(n_sets)]
@@ -352,7 +356,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": workload_config(wl, {
-                "path": mod.path, "parallelism": f"replicas{world}" if world > 1 else "single",
+                "path": mod.path, "whiten": args.whiten,
+                "parallelism": f"replicas{world}" if world > 1 else "single",
                 "l2": f"{n_sets} rotating input/output sets of {set_bytes / 2**20:.1f} MiB "
                       f"({n_sets * set_bytes / 2**20:.0f} MiB > 126 MiB L2), no flush",
                 "call_roofline_frac": t_roof / (ms_per_step * 1e-3),
@@ -369,7 +374,7 @@ def main():
             "gpu_launches": K * mod.launches_per_forward,
             "clocks": clk,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.whiten == "unit":
             line["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_seconds)
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   LFA_OK = 0,
   LFA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, H%r or W%r != 0 ... */
-  LFA_ERR_UNSUPPORTED = 2,   /* d not in {32, 64}, m > 256, unknown dtype */
+  LFA_ERR_UNSUPPORTED = 2,   /* d not in {32, 64}, m > 256, unknown dtype; backward with whiten = 2 */
   LFA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, copy, attribute) */
   LFA_ERR_STATE = 4,         /* backward without a matching forward on this handle */
   LFA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (reported by lfa_get_info) */
@@ -72,7 +72,10 @@ typedef struct {
   float eps;      /* W regulariser and whitening epsilon, >= 0 */
   int T;          /* Newton-Schulz steps, 0 <= T <= 64 */
   int dtype;      /* lfa_dtype of Q, V, O, dO, dQ, dV */
-  int whiten;     /* 1: whitened C~ on both sides (default); 0: raw C */
+  int whiten;     /* 1: whitened C~ on both sides (default); 0: raw C; 2: whitened, with mu and
+                     var of each landmark column pooled per head over the B*N rows of all batch
+                     elements (the note's statistics "over a batch", §关键设计 1; C~ keeps the
+                     1/N of one unit). whiten = 2 runs the per-stage kernels, forward only. */
 } lfa_config;
 
 /* Per-unit diagnostics of the most recent forward call. */
@@ -141,6 +144,7 @@ lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host
 /* Backward pass for the loss <dO, O>: writes dQ and dV ([B][heads][N][d], cfg.dtype).
  * Reuses the context saved by the most recent lfa_forward on this handle, which
  * must have been called with the same Q and V pointers (else LFA_ERR_STATE).
+ * Batch-pooled statistics (whiten = 2) have no backward: LFA_ERR_UNSUPPORTED.
  * The kernel gradient is -(1/lambda) sign(q - l) k with sign(0) = 0 [the note's
  * §研究背景与动机 prints the opposite sign]; alpha is held constant; the DWC
  * weight gets no gradient. */

@@ -39,7 +39,7 @@ lfa_status validate(const lfa_config* c) {
   if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return LFA_ERR_INVALID_ARG;
   if (!(c->eps >= 0.f) || !isfinite(c->eps)) return LFA_ERR_INVALID_ARG;
   if (c->T < 0 || c->T > lfa::kMaxT) return LFA_ERR_INVALID_ARG;
-  if (c->whiten != 0 && c->whiten != 1) return LFA_ERR_INVALID_ARG;
+  if (c->whiten < 0 || c->whiten > 2) return LFA_ERR_INVALID_ARG;
   if (c->d != 32 && c->d != 64) return LFA_ERR_UNSUPPORTED;
   if (c->dtype != LFA_F32 && c->dtype != LFA_BF16) return LFA_ERR_UNSUPPORTED;
   const long long m = (long long)(c->H / c->r) * (c->W / c->r);
@@ -242,7 +242,8 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
   h->path = 0;
   const char* force = getenv("LFA_FORWARD_PATH");
   const bool want_generic = force && strcmp(force, "generic") == 0;
-  if (!want_generic && h->lay.fused != h->lay.bwd) {
+  // batch-pooled statistics need every unit's column sums before any unit's combine: per-stage
+  if (!want_generic && h->p.whiten != 2 && h->lay.fused != h->lay.bwd) {
     h->grid = lfa::fused_grid(h->p);
     if (h->grid > 0) h->path = 1;
   }
@@ -352,6 +353,7 @@ lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* 
   if (!h || !Q || !V || !dO || !dQ || !dV) return LFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dV))
     return LFA_ERR_INVALID_ARG;
+  if (h->p.whiten == 2) return LFA_ERR_UNSUPPORTED;
   if (!h->have_forward || h->last_Q != Q || h->last_V != V) return LFA_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Params p = h->p;

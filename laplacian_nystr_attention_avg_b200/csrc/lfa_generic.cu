@@ -525,6 +525,20 @@ __global__ void __launch_bounds__(kThreads) k_combine_reduce(Params p) {
   p.red[(size_t)u * p.part_stride + e] = acc;
 }
 
+// Batch-pooled statistics (whiten = 2; the note's whitening statistics over a batch of
+// similarity vectors, §关键设计 1): for each head and landmark column, the fp64 sums of C and
+// C^2 of the B units u = b * heads + h are replaced in every one of them by their mean over b,
+// so that the per-unit combine's sum / N becomes the pooled sum / (B N). One thread per (head,
+// entry): it reads all B sums before writing any.
+__global__ void __launch_bounds__(kThreads) k_pool_batch_stats(Params p) {
+  const int h = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= 2 * p.m) return;
+  double acc = 0.0;
+  for (int b = 0; b < p.B; ++b) acc += p.red[(size_t)(b * p.heads + h) * p.part_stride + e];
+  acc /= (double)p.B;
+  for (int b = 0; b < p.B; ++b) p.red[(size_t)(b * p.heads + h) * p.part_stride + e] = acc;
+}
+
 // mu, s, A (all landmarks), then M = X A, M' and bias partials for 16 landmark rows.
 __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   extern __shared__ float4 smem_f4[];
@@ -749,6 +763,7 @@ void context_t(const Params& p, cudaStream_t st) {
     k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
   }
   pass1_reduce_t<T>(p, st);
+  if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, st>>>(p);
   k_combine_finish<<<dim3(p.n_chunks, U), kThreads, (size_t)(m * d + 2 * m) * sizeof(float), st>>>(p);
 }
 
@@ -800,9 +815,10 @@ cudaError_t generic_set_attributes() {
 }
 
 int generic_launch_count(const Params& p) {
-  // pool, Newton-Schulz chain, pass 1, two combine kernels, pass 2
+  // pool, Newton-Schulz chain, pass 1, two combine kernels (three with batch-pooled statistics),
+  // pass 2
   const int ns = p.m <= kSmallM ? 1 : 2 + 2 * p.T + 2;
-  return 1 + ns + 1 + 2 + 1;
+  return 1 + ns + 1 + 2 + (p.whiten == 2 ? 1 : 0) + 1;
 }
 
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st) {

@@ -21,6 +21,7 @@ LFA_OK, LFA_ERR_INVALID_ARG, LFA_ERR_UNSUPPORTED, LFA_ERR_CUDA, LFA_ERR_STATE, \
     LFA_ERR_TIMEOUT, LFA_ERR_NONFINITE, LFA_ERR_SCRATCH_LIMIT = range(8)
 LFA_NOALLOC_SCRATCH_BYTES = 16 << 20
 LFA_F32, LFA_BF16 = 0, 1
+LFA_WHITEN_BATCH = 2   # cfg.whiten: column statistics pooled per head over the batch
 
 
 class Config(ctypes.Structure):
@@ -118,10 +119,15 @@ def _check(status: int, what: str) -> None:
         raise LfaError(status, what)
 
 
-def make_config(wl, whiten: bool = True) -> Config:
-    """lfa_config from a Workload (laplacian_nystr_attention_avg_b200.inputs)."""
+def make_config(wl, whiten=True) -> Config:
+    """lfa_config from a Workload (laplacian_nystr_attention_avg_b200.inputs).
+
+    whiten: True (per-unit column statistics), False (raw C) or "batch" (statistics
+    pooled per head over the batch; cfg.whiten = LFA_WHITEN_BATCH).
+    """
+    wv = LFA_WHITEN_BATCH if whiten == "batch" else (1 if whiten else 0)
     return Config(wl.B, wl.heads, wl.H, wl.W, wl.d, wl.r, float(wl.lam), float(wl.eps), int(wl.T),
-                  LFA_BF16 if wl.dtype == "bf16" else LFA_F32, 1 if whiten else 0)
+                  LFA_BF16 if wl.dtype == "bf16" else LFA_F32, wv)
 
 
 def workspace_size(cfg: Config) -> int:
