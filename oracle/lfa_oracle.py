@@ -39,6 +39,13 @@ design notes with its reason):
       are taken over the B*N rows of every unit that shares the head h (all batch
       elements), population variance; C~ of each unit is then formed as in R6 with
       that unit's own N in the 1/N offset. Forward only.
+  R13 (alternative reading of R6, "Reading B", unit_forward_reading_b) the whitening acts
+      on the columns of the whole Nystrom similarity matrix G^ = C X C^T (N x N, one
+      column per key token j): g~_j = (g_j - mean_i g_ij) / sqrt(var_i g_ij + eps) + 1/N,
+      population variance, and O_attn = G~ V. In factored form, with c_j the j-th row
+      of C, c- the column mean of C, Cc = C - 1 c-^T and S = Cc^T Cc / N:
+      mean_i g_ij = c-^T X c_j, var_i g_ij = c_j^T X^T S X c_j, and
+      O_attn = Cc X C^T D^-1/2 V + (1/N) 1 (1^T V), D = diag(var_j + eps). Forward only.
 
 Parity pins (tests/test_oracle_*.py): closed forms of the kernel, scipy cdist,
 torch avg_pool2d / conv2d in float64, the per-step eigen closed form of
@@ -325,6 +332,61 @@ def unit_backward(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten=True):
     g = dL.reshape(H // r, 1, Wr, 1, d) / (r * r)
     dQ = dQ + np.broadcast_to(g, (H // r, r, Wr, r, d)).reshape(N, d)
     return dQ, dV, f
+
+
+@dataclasses.dataclass
+class UnitForwardB:
+    C: np.ndarray           # [N, m] cross kernel
+    X: np.ndarray           # [m, m] X_T
+    cbar: np.ndarray        # [m] column mean of C
+    S: np.ndarray           # [m, m] covariance of the columns of C
+    col_mean: np.ndarray    # [N] mean over i of column j of G^ = C X C^T
+    col_var: np.ndarray     # [N] its population variance
+    O_attn: np.ndarray      # G~ V
+    O: np.ndarray           # O_attn + DWC(V)
+
+
+def unit_forward_reading_b(Qu, Vu, w, H, W, r, lam, eps, T) -> UnitForwardB:
+    """R13: column whitening of the full Nystrom similarity matrix ([P1] 关键设计 1 applied to
+    关键设计 2's G^), in the O(N m^2) factored form; the steps before X as in unit_forward."""
+    Qu = np.asarray(Qu, dtype=np.float64)
+    Vu = np.asarray(Vu, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    L = pool_landmarks(Qu, H, W, r)
+    C = laplacian_kernel(Qu, L, lam)
+    Wm = landmark_gram(L, lam, eps)
+    ac = select_alpha(Wm)
+    X, _, _ = newton_schulz(Wm, ac.alpha, T)
+    N = C.shape[0]
+    cbar = C.mean(axis=0)
+    Cc = C - cbar
+    S = Cc.T @ Cc / N
+    K = X.T @ S @ X
+    col_mean = C @ (X.T @ cbar)                       # c-^T X c_j for every j
+    col_var = np.einsum("jl,lk,jk->j", C, K, C)       # c_j^T K c_j
+    dinv = 1.0 / np.sqrt(col_var + eps)
+    M = X @ (C.T @ (dinv[:, None] * Vu))              # X C^T D^-1/2 V
+    O_attn = Cc @ M + Vu.sum(axis=0)[None, :] / N
+    O = O_attn + dwc3x3(Vu, w, H, W)
+    return UnitForwardB(C, X, cbar, S, col_mean, col_var, O_attn, O)
+
+
+def forward_reading_b(Q, V, dwc, wl, units=None):
+    """R13 over all (or the listed) units of a workload: returns (O, O_attn, [UnitForwardB])."""
+    Q = np.asarray(Q, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    w = np.asarray(dwc, dtype=np.float64)
+    B, nh, N, d = Q.shape
+    O = np.zeros_like(Q)
+    Oa = np.zeros_like(Q)
+    us = []
+    for u in (range(B * nh) if units is None else units):
+        b, h = divmod(u, nh)
+        f = unit_forward_reading_b(Q[b, h], V[b, h], w[h], wl.H, wl.W, wl.r, wl.lam, wl.eps, wl.T)
+        O[b, h] = f.O
+        Oa[b, h] = f.O_attn
+        us.append(f)
+    return O, Oa, us
 
 
 # ---------------------------------------------------------------------------

@@ -275,6 +275,40 @@ def check_batch_stats_vs_sklearn():
         assert np.allclose(got, ref, rtol=1e-10, atol=1e-12), f"head {h}"
 
 
+# --- Reading B: column whitening of the full Nystrom matrix (reading R13) --------
+
+def check_reading_b_vs_dense():
+    # materialise G^ = C X C^T (N x N), standard-scale its columns, add 1/N, multiply by V
+    from sklearn.preprocessing import StandardScaler
+    rng = _rng(61)
+    H = W = 8
+    d, r, lam, T = 8, 2, 2.0, 30
+    q = rng.standard_normal((H * W, d))
+    v = rng.standard_normal((H * W, d))
+    w = rng.standard_normal((d, 3, 3)) * 0.1
+    f = O.unit_forward_reading_b(q, v, w, H, W, r, lam, 0.0, T)
+    G = f.C @ f.X @ f.C.T
+    ref = (StandardScaler().fit_transform(G) + 1.0 / G.shape[0]) @ v
+    assert np.allclose(f.O_attn, ref, rtol=0, atol=1e-10 * np.abs(ref).max())
+    assert np.allclose(f.col_var, G.var(axis=0), rtol=1e-10)
+
+
+def check_reading_b_r1_is_whitened_kernel():
+    # r = 1 and eps = 0: the landmarks are the tokens, W = G, X -> G^-1 and G^ = G G^-1 G = G, so
+    # Reading B is the column-whitened Laplacian kernel matrix itself applied to V
+    rng = _rng(62)
+    H = W = 4
+    d, lam = 8, 2.0
+    q = rng.standard_normal((H * W, d))
+    v = rng.standard_normal((H * W, d))
+    w = np.zeros((d, 3, 3))
+    f = O.unit_forward_reading_b(q, v, w, H, W, 1, lam, 0.0, 40)
+    G = np.exp(-np.abs(q[:, None, :] - q[None, :, :]).sum(-1) / lam)
+    Z = (G - G.mean(axis=0)) / G.std(axis=0) + 1.0 / G.shape[0]
+    ref = Z @ v
+    assert np.allclose(f.O_attn, ref, rtol=0, atol=1e-9 * np.abs(ref).max())
+
+
 # --- DWC ------------------------------------------------------------------------
 
 def check_dwc_vs_conv2d():
@@ -420,4 +454,5 @@ ALL_PINS = [
     check_whitening_vs_sklearn, check_whitened_assembly_vs_solve, check_dwc_vs_conv2d,
     check_dwc_taps, check_backward_fd, check_injectivity_generic,
     check_batch_stats_single_batch, check_batch_stats_replicated, check_batch_stats_vs_sklearn,
+    check_reading_b_vs_dense, check_reading_b_r1_is_whitened_kernel,
 ]

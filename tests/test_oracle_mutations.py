@@ -12,7 +12,7 @@ from tests import pins
 _orig = {name: getattr(O, name) for name in (
     "laplacian_kernel", "l1_distances", "pool_landmarks", "landmark_gram", "newton_schulz",
     "whiten_columns", "dwc3x3", "_sign_contractions", "select_alpha", "pooled_column_stats",
-    "batch_groups")}
+    "batch_groups", "unit_forward_reading_b")}
 
 
 def _kernel_no_lambda(X, Y, lam):
@@ -98,6 +98,25 @@ def _groups_across_heads(B, heads):
     return [list(range(B * heads))]
 
 
+def _reading_b_variant(uncentred_cov=False, no_offset=False, sample_var=False):
+    def f(Qu, Vu, w, H, W, r, lam, eps, T):
+        Qu = np.asarray(Qu, float)
+        Vu = np.asarray(Vu, float)
+        L = O.pool_landmarks(Qu, H, W, r)
+        C = O.laplacian_kernel(Qu, L, lam)
+        Wm = O.landmark_gram(L, lam, eps)
+        X, _, _ = O.newton_schulz(Wm, O.select_alpha(Wm).alpha, T)
+        N = C.shape[0]
+        cbar = C.mean(axis=0)
+        Cc = C - cbar
+        S = (C.T @ C if uncentred_cov else Cc.T @ Cc) / (N - 1 if sample_var else N)
+        var = np.einsum("jl,lk,jk->j", C, X.T @ S @ X, C)
+        M = X @ (C.T @ (Vu / np.sqrt(var + eps)[:, None]))
+        Oa = Cc @ M + (0.0 if no_offset else Vu.sum(axis=0)[None, :] / N)
+        return O.UnitForwardB(C, X, cbar, S, C @ (X.T @ cbar), var, Oa, Oa)
+    return f
+
+
 def _dwc_convolution(Vu, w, H, W):
     return _orig["dwc3x3"](Vu, w[:, ::-1, ::-1].copy(), H, W)
 
@@ -123,6 +142,12 @@ MUTATIONS = [
     ("batch_stats_first_unit_only", "pooled_column_stats", _pooled_first_unit_only,
      [pins.check_batch_stats_vs_sklearn]),
     ("batch_stats_pooled_across_heads", "batch_groups", _groups_across_heads, [pins.check_batch_stats_vs_sklearn]),
+    ("reading_b_uncentred_covariance", "unit_forward_reading_b", _reading_b_variant(uncentred_cov=True),
+     [pins.check_reading_b_vs_dense]),
+    ("reading_b_no_offset", "unit_forward_reading_b", _reading_b_variant(no_offset=True),
+     [pins.check_reading_b_vs_dense]),
+    ("reading_b_sample_variance", "unit_forward_reading_b", _reading_b_variant(sample_var=True),
+     [pins.check_reading_b_vs_dense, pins.check_reading_b_r1_is_whitened_kernel]),
     ("kernel_gradient_sign_as_printed", "_sign_contractions", _sign_as_printed,
      [lambda: pins.check_backward_fd([(8, 8, 8, 2, 2.0, 1e-3, 24, 44, True)])]),
 ]
