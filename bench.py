@@ -40,9 +40,10 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["lfa", "reference"], default="lfa")
     ap.add_argument("--workload", default="pvt1")
-    ap.add_argument("--whiten", choices=["unit", "batch"], default="unit",
-                    help="column statistics per (batch, head) unit, or pooled per head over the batch "
-                         "(per-stage kernels; no CPU baseline)")
+    ap.add_argument("--whiten", choices=["unit", "batch", "full"], default="unit",
+                    help="column statistics per (batch, head) unit; 'batch': pooled per head over the "
+                         "batch; 'full': Reading B, the columns of the whole Nystrom matrix (both on the "
+                         "per-stage kernels, no CPU baseline)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -281,7 +282,7 @@ def main():
 
     wl = WORKLOADS[args.workload]
     x = make_inputs(wl, seed=rank)
-    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, True if args.whiten == "unit" else "batch"),
+    mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, True if args.whiten == "unit" else args.whiten),
                                         x.dwc, str(dev))
     set_bytes = 3 * wl.units * wl.N * wl.d * x.Q_store.element_size()
     n_sets = max(2, math.ceil(1.8 * L2_BYTES / set_bytes))

@@ -39,11 +39,12 @@ lfa_status validate(const lfa_config* c) {
   if (!(c->lambda > 0.f) || !isfinite(c->lambda)) return LFA_ERR_INVALID_ARG;
   if (!(c->eps >= 0.f) || !isfinite(c->eps)) return LFA_ERR_INVALID_ARG;
   if (c->T < 0 || c->T > lfa::kMaxT) return LFA_ERR_INVALID_ARG;
-  if (c->whiten < 0 || c->whiten > 2) return LFA_ERR_INVALID_ARG;
+  if (c->whiten < 0 || c->whiten > 3) return LFA_ERR_INVALID_ARG;
   if (c->d != 32 && c->d != 64) return LFA_ERR_UNSUPPORTED;
   if (c->dtype != LFA_F32 && c->dtype != LFA_BF16) return LFA_ERR_UNSUPPORTED;
   const long long m = (long long)(c->H / c->r) * (c->W / c->r);
   if (m > lfa::kMaxM) return LFA_ERR_UNSUPPORTED;
+  if (c->whiten == 3 && m > lfa::kSmallM) return LFA_ERR_UNSUPPORTED;   // Reading B: K tiles of 64
   const long long rows = (long long)c->B * c->heads * c->H * c->W;
   if (rows * c->d >= (1ll << 31)) return LFA_ERR_UNSUPPORTED;   // element index fits int32
   return LFA_OK;
@@ -74,7 +75,8 @@ void plan(const lfa_config* c, Params* p, Layout* L) {
   if (P < 1) P = 1;
   p->tiles_per_cta = lfa::ceil_div(p->n_tiles, P);
   p->P = lfa::ceil_div(p->n_tiles, p->tiles_per_cta);
-  p->part_stride = 2 * p->m + p->m * p->d + p->d;
+  // pass-1 partial record: S1 [m], S2 [m], C^T V [m][d], sum V [d]; Reading B adds C^T C [m][m]
+  p->part_stride = 2 * p->m + p->m * p->d + p->d + (c->whiten == 3 ? p->m * p->m : 0);
   p->n_chunks = lfa::ceil_div(p->m, 16);
 
   const size_t U = p->U, m = p->m, d = p->d;
@@ -242,8 +244,9 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
   h->path = 0;
   const char* force = getenv("LFA_FORWARD_PATH");
   const bool want_generic = force && strcmp(force, "generic") == 0;
-  // batch-pooled statistics need every unit's column sums before any unit's combine: per-stage
-  if (!want_generic && h->p.whiten != 2 && h->lay.fused != h->lay.bwd) {
+  // batch-pooled statistics need every unit's column sums before any unit's combine, and
+  // Reading B needs two more token passes: both run on the per-stage kernels
+  if (!want_generic && h->p.whiten <= 1 && h->lay.fused != h->lay.bwd) {
     h->grid = lfa::fused_grid(h->p);
     if (h->grid > 0) h->path = 1;
   }
@@ -353,7 +356,7 @@ lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* 
   if (!h || !Q || !V || !dO || !dQ || !dV) return LFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dV))
     return LFA_ERR_INVALID_ARG;
-  if (h->p.whiten == 2) return LFA_ERR_UNSUPPORTED;
+  if (h->p.whiten >= 2) return LFA_ERR_UNSUPPORTED;
   if (!h->have_forward || h->last_Q != Q || h->last_V != V) return LFA_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Params p = h->p;

@@ -607,6 +607,206 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Reading B (whiten = 3, m <= 64): whitening of the columns of the whole Nystrom matrix
+// G^ = C X C^T (LaplacianFormer note, §关键设计 1 applied to §关键设计 2's G^), one column per
+// key token j, in factored form. With c- the column mean of C and S = cov(C) (population):
+//   mean_i G^_ij = c-^T X c_j,  var_j = c_j^T K c_j with K = X^T S X,
+//   O_attn = (C - 1 c-^T) X C^T D^-1/2 V + (1/N) 1 (1^T V),  D = diag(var_j + eps),
+// so pass 2 runs unchanged with M' = X C^T D^-1/2 V and b = (1/N) sum_i v_i - M'^T c-.
+// Steps: k_rb_gram (C^T C partials, into the tail of the pass-1 partial record), the pass-1
+// reduction, k_rb_cov (S in fp64), K = X^T (S X) by two batched products, k_rb_pass (var_j per
+// token, partials of C^T D^-1/2 V), k_rb_reduce, k_rb_finish (M', b).
+// ---------------------------------------------------------------------------------------
+constexpr int kRbCs = 64 + 4;   // row stride (floats) of the 64-landmark C and K tiles
+
+// C^T C over the CTA's rows (the same row partition as pass 1); thread t owns the 4 x 4 block
+// rows 4 (t / 16) .., columns 4 (t % 16) .. of the 64 x 64 product.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_rb_gram(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, ds = d + 4;
+  float* Ls = sm;                    // [64][ds]
+  float* Qs = Ls + 64 * ds;          // [64][ds]
+  float* Cs = Qs + kRowTile * ds;    // [64][kRbCs]
+  const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x, jb = t >> 4, kb = t & 15;
+  const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, 64, d);
+  float acc[4][4] = {};
+  const int tile0 = pc * p.tiles_per_cta;
+  const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
+  for (int tile = tile0; tile < tile1; ++tile) {
+    const int row0 = tile * kRowTile;
+    const int valid = min(kRowTile, p.N - row0);
+    __syncthreads();
+    stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+    __syncthreads();
+    cross_tile(Qs, Ls, Cs, d, 0, m, kRbCs, p.neg_log2e_over_lam, valid);
+    __syncthreads();
+    for (int i = 0; i < kRowTile; ++i) {
+      const float4 a = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * jb]);
+      const float4 b = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * kb]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+    }
+  }
+  float* out = p.part + ((size_t)u * p.P + pc) * p.part_stride + (2 * m + m * d + d);
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int j = 4 * jb + x, k = 4 * kb + y;
+      if (j < m && k < m) out[j * m + k] = acc[x][y];
+    }
+}
+
+// S = C^T C / N - c- c-^T (fp64 from the reduced sums) into Y; mu = c-, s = 1 for inspection.
+__global__ void __launch_bounds__(kThreads) k_rb_cov(Params p) {
+  const int u = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x, m = p.m;
+  if (e >= m * m) return;
+  const double* red = p.red + (size_t)u * p.part_stride;
+  const double invN = 1.0 / double(p.N);
+  const int j = e / m, k = e % m;
+  const double cj = red[j] * invN, ck = red[k] * invN;
+  p.Y[(size_t)u * m * m + e] = (float)(red[2 * m + m * p.d + p.d + e] * invN - cj * ck);
+  if (e < m) {
+    p.mu[(size_t)u * m + e] = (float)(red[e] * invN);
+    p.s[(size_t)u * m + e] = 1.f;
+  }
+}
+
+// Per 64-row tile: C, var_i = c_i^T K c_i (thread (i = t / 4, t % 4) sums over landmarks
+// j = t % 4 + 4 n), w_i = 1 / sqrt(var_i + eps) (0 past the end), and C^T (w o V) into the
+// P slot of the CTA's partial record (pass 1's records are already reduced).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_rb_pass(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* sm = reinterpret_cast<float*>(smem_f4);
+  const int m = p.m, d = p.d, ds = d + 4;
+  float* Ls = sm;                    // [64][ds]
+  float* Qs = Ls + 64 * ds;          // [64][ds]
+  float* Vs = Qs + kRowTile * ds;    // [64][ds]
+  float* Cs = Vs + kRowTile * ds;    // [64][kRbCs]
+  float* Ks = Cs + kRowTile * kRbCs; // [64][kRbCs]
+  float* wr = Ks + 64 * kRbCs;       // [64]
+  const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x;
+  const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
+  const T* Vg = static_cast<const T*>(p.V) + (size_t)u * p.N * d;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, 64, d);
+  for (int e = t; e < 64 * 64; e += blockDim.x) {
+    const int j = e >> 6, k = e & 63;
+    Ks[j * kRbCs + k] = (j < m && k < m) ? p.Y[(size_t)u * m * m + j * m + k] : 0.f;
+  }
+  const int nbk = d / 4, nb = 16 * nbk;   // 4 x 4 blocks of the 64 x d product
+  const int jb = t / nbk, kb = t % nbk;
+  float acc[4][4] = {};
+  const int tile0 = pc * p.tiles_per_cta;
+  const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
+  for (int tile = tile0; tile < tile1; ++tile) {
+    const int row0 = tile * kRowTile;
+    const int valid = min(kRowTile, p.N - row0);
+    __syncthreads();
+    stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
+    stage_rows(Vg + (size_t)row0 * d, Vs, d, valid);
+    __syncthreads();
+    cross_tile(Qs, Ls, Cs, d, 0, m, kRbCs, p.neg_log2e_over_lam, valid);
+    __syncthreads();
+    {
+      const int i = t >> 2, j0 = t & 3;
+      float v = 0.f;
+      for (int j = j0; j < 64; j += 4) {
+        float y = 0.f;
+        for (int k = 0; k < 64; k += 4) {
+          const float4 kk = *reinterpret_cast<const float4*>(&Ks[j * kRbCs + k]);
+          const float4 cc = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + k]);
+          y = fmaf(kk.x, cc.x, y);
+          y = fmaf(kk.y, cc.y, y);
+          y = fmaf(kk.z, cc.z, y);
+          y = fmaf(kk.w, cc.w, y);
+        }
+        v = fmaf(Cs[i * kRbCs + j], y, v);
+      }
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      if (j0 == 0) wr[i] = i < valid ? 1.f / sqrtf(v + p.eps) : 0.f;
+    }
+    __syncthreads();
+    for (int e = t; e < kRowTile * d; e += blockDim.x) {
+      const int i = e / d, c = e % d;
+      Vs[i * ds + c] *= wr[i];
+    }
+    __syncthreads();
+    if (t < nb) {
+      for (int i = 0; i < kRowTile; ++i) {
+        const float4 c = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * jb]);
+        const float4 v = *reinterpret_cast<const float4*>(&Vs[i * ds + 4 * kb]);
+        const float cc[4] = {c.x, c.y, c.z, c.w}, vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(cc[x], vv[y], acc[x][y]);
+      }
+    }
+  }
+  if (t < nb) {
+    float* out = p.part + ((size_t)u * p.P + pc) * p.part_stride + 2 * m;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = 4 * jb + x;
+      if (j < m)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) out[j * d + 4 * kb + y] = acc[x][y];
+    }
+  }
+}
+
+// A = C^T D^-1/2 V: the partials' P slots summed in fp64.
+__global__ void __launch_bounds__(kThreads) k_rb_reduce(Params p) {
+  const int u = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= p.m * p.d) return;
+  double acc = 0.0;
+  const float* src = p.part + (size_t)u * p.P * p.part_stride + 2 * p.m + e;
+  for (int pc = 0; pc < p.P; ++pc) acc += (double)src[(size_t)pc * p.part_stride];
+  p.A[(size_t)u * p.m * p.d + e] = (float)acc;
+}
+
+// Rows [16c, 16c + 16) of M' = X A, and the bias partial -sum_j c-_j M'[j][k] over them; chunk 0
+// adds (1/N) sum_i v_ik.
+__global__ void __launch_bounds__(kThreads) k_rb_finish(Params p) {
+  extern __shared__ float4 smem_f4[];
+  float* As = reinterpret_cast<float*>(smem_f4);   // [m][d]
+  const int m = p.m, d = p.d, u = blockIdx.y, c = blockIdx.x, t = threadIdx.x;
+  for (int e = t; e < m * d; e += blockDim.x) As[e] = p.A[(size_t)u * m * d + e];
+  __syncthreads();
+  const double* red = p.red + (size_t)u * p.part_stride;
+  const double invN = 1.0 / double(p.N);
+  const float* Xg = p.X + (size_t)u * m * m;
+  const int j0 = c * 16;
+  for (int e = t; e < 16 * d; e += blockDim.x) {
+    const int j = j0 + e / d, k = e % d;
+    if (j < m) {
+      float acc = 0.f;
+      for (int l = 0; l < m; ++l) acc = fmaf(Xg[(size_t)j * m + l], As[l * d + k], acc);
+      p.M[((size_t)u * m + j) * d + k] = acc;
+      p.Mp[((size_t)u * m + j) * d + k] = acc;
+    }
+  }
+  __syncthreads();
+  float* bp = p.bpart + ((size_t)u * p.n_chunks + c) * d;
+  for (int k = t; k < d; k += blockDim.x) {
+    double acc = c == 0 ? red[2 * m + m * d + k] * invN : 0.0;
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = j0 + jj;
+      if (j < m) acc -= red[j] * invN * (double)p.M[((size_t)u * m + j) * d + k];
+    }
+    bp[k] = (float)acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 // Pass 2: O = C M' + 1 b^T + DWC(V) over the CTA's 64-row tiles (the same row partition as
 // pass 1); L and M' are staged once per CTA.
 // ---------------------------------------------------------------------------------------
@@ -725,7 +925,7 @@ __global__ void __launch_bounds__(kThreads) k_cross_out(Params p, int u, float* 
 // Pass 1 over the tokens (sums of C, C^2, C^T V and V per CTA) and their fp64 reduction
 // into p.red. With p.V pointing at another [N][d] tensor (dO) the same code forms C^T dO.
 template <typename T>
-void pass1_reduce_t(const Params& p, cudaStream_t st) {
+void pass1_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   const int bpt = ceil_div((round_up(m, 4) / 4) * (d / 4), kThreads);
   const dim3 g1(p.P, U);
@@ -733,7 +933,34 @@ void pass1_reduce_t(const Params& p, cudaStream_t st) {
   if (bpt <= 1) k_pass1<T, 1><<<g1, kThreads, s1, st>>>(p);
   else if (bpt <= 2) k_pass1<T, 2><<<g1, kThreads, s1, st>>>(p);
   else k_pass1<T, 4><<<g1, kThreads, s1, st>>>(p);
+}
+
+template <typename T>
+void pass1_reduce_t(const Params& p, cudaStream_t st) {
+  pass1_t<T>(p, st);
+  k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), p.U), kThreads, 0, st>>>(p);
+}
+
+size_t rb_gram_smem(int d) { return sizeof(float) * (size_t)(2 * 64 * (d + 4) + 64 * kRbCs); }
+size_t rb_pass_smem(int d) { return sizeof(float) * (size_t)(3 * 64 * (d + 4) + 2 * 64 * kRbCs + 64); }
+
+// Reading B after the Newton-Schulz chain (m <= 64, so X came from k_ns_small and the Y / Xb
+// buffers are free): every stage up to M' and b.
+template <typename T>
+void reading_b_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m, d = p.d;
+  const size_t mm = (size_t)m * m;
+  pass1_t<T>(p, st);
+  k_rb_gram<T><<<dim3(p.P, U), kThreads, rb_gram_smem(d), st>>>(p);
   k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
+  k_rb_cov<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
+  const MmJob sx{p.Y, mm, p.X, mm, nullptr, 0, p.Xb, mm, 1.f, 0.f, 0.f, 0, 0};   // Xb = S X
+  launch_mm(&sx, 1, m, U, st);
+  const MmJob k{p.X, mm, p.Xb, mm, nullptr, 0, p.Y, mm, 1.f, 0.f, 0.f, 1, 0};     // Y = X^T (S X)
+  launch_mm(&k, 1, m, U, st);
+  k_rb_pass<T><<<dim3(p.P, U), kThreads, rb_pass_smem(d), st>>>(p);
+  k_rb_reduce<<<dim3(ceil_div(m * d, kThreads), U), kThreads, 0, st>>>(p);
+  k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
 
 // Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b.
@@ -761,6 +988,10 @@ void context_t(const Params& p, cudaStream_t st) {
     if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
     k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
     k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
+  }
+  if (p.whiten == 3) {
+    reading_b_t<T>(p, st);
+    return;
   }
   pass1_reduce_t<T>(p, st);
   if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, st>>>(p);
@@ -802,6 +1033,10 @@ cudaError_t generic_set_attributes() {
   LFA_ATTR((k_pass1<__nv_bfloat16, 2>));
   LFA_ATTR((k_pass1<__nv_bfloat16, 4>));
   LFA_ATTR(k_combine_finish);
+  LFA_ATTR(k_rb_gram<float>);
+  LFA_ATTR(k_rb_gram<__nv_bfloat16>);
+  LFA_ATTR(k_rb_pass<float>);
+  LFA_ATTR(k_rb_pass<__nv_bfloat16>);
   LFA_ATTR(k_pass2<float>);
   LFA_ATTR(k_pass2<__nv_bfloat16>);
   LFA_ATTR(k_cross_out<float>);
@@ -818,6 +1053,8 @@ int generic_launch_count(const Params& p) {
   // pool, Newton-Schulz chain, pass 1, two combine kernels (three with batch-pooled statistics),
   // pass 2
   const int ns = p.m <= kSmallM ? 1 : 2 + 2 * p.T + 2;
+  // Reading B: pass 1, C^T C, reduction, covariance, two products, token pass, reduction, finish
+  if (p.whiten == 3) return 1 + ns + 9 + 1;
   return 1 + ns + 1 + 2 + (p.whiten == 2 ? 1 : 0) + 1;
 }
 

@@ -22,6 +22,7 @@ LFA_OK, LFA_ERR_INVALID_ARG, LFA_ERR_UNSUPPORTED, LFA_ERR_CUDA, LFA_ERR_STATE, \
 LFA_NOALLOC_SCRATCH_BYTES = 16 << 20
 LFA_F32, LFA_BF16 = 0, 1
 LFA_WHITEN_BATCH = 2   # cfg.whiten: column statistics pooled per head over the batch
+LFA_WHITEN_FULL = 3    # cfg.whiten: Reading B, whitening of the columns of the whole Nystrom matrix
 
 
 class Config(ctypes.Structure):
@@ -122,10 +123,14 @@ def _check(status: int, what: str) -> None:
 def make_config(wl, whiten=True) -> Config:
     """lfa_config from a Workload (laplacian_nystr_attention_avg_b200.inputs).
 
-    whiten: True (per-unit column statistics), False (raw C) or "batch" (statistics
-    pooled per head over the batch; cfg.whiten = LFA_WHITEN_BATCH).
+    whiten: True (per-unit column statistics), False (raw C), "batch" (statistics
+    pooled per head over the batch; cfg.whiten = LFA_WHITEN_BATCH) or "full" (Reading B:
+    the columns of the whole Nystrom matrix; cfg.whiten = LFA_WHITEN_FULL).
     """
-    wv = LFA_WHITEN_BATCH if whiten == "batch" else (1 if whiten else 0)
+    wv = {"batch": LFA_WHITEN_BATCH, "full": LFA_WHITEN_FULL}.get(whiten, None) if isinstance(whiten, str) \
+        else (1 if whiten else 0)
+    if wv is None:
+        raise ValueError(f"whiten: {whiten!r}")
     return Config(wl.B, wl.heads, wl.H, wl.W, wl.d, wl.r, float(wl.lam), float(wl.eps), int(wl.T),
                   LFA_BF16 if wl.dtype == "bf16" else LFA_F32, wv)
 

@@ -56,7 +56,8 @@ def _cfg(**kw):
     (dict(T=65), lfa.LFA_ERR_INVALID_ARG),
     (dict(B=0), lfa.LFA_ERR_INVALID_ARG),
     (dict(r=0), lfa.LFA_ERR_INVALID_ARG),
-    (dict(whiten=3), lfa.LFA_ERR_INVALID_ARG),          # 0 raw, 1 per unit, 2 batch-pooled
+    (dict(whiten=4), lfa.LFA_ERR_INVALID_ARG),          # 0 raw, 1 per unit, 2 batch-pooled, 3 reading B
+    (dict(whiten=3, H=64, W=64, r=4), lfa.LFA_ERR_UNSUPPORTED),   # reading B needs m <= 64
     (dict(whiten=-1), lfa.LFA_ERR_INVALID_ARG),
     (dict(d=48), lfa.LFA_ERR_UNSUPPORTED),
     (dict(d=128), lfa.LFA_ERR_UNSUPPORTED),
