@@ -164,6 +164,42 @@ def newton_schulz(W: np.ndarray, alpha: float, T: int, keep_iterates: bool = Fal
     return X, res, its
 
 
+def cg_solve(W: np.ndarray, B: np.ndarray, iters: int, dtype=np.float64) -> np.ndarray:
+    """Conjugate gradients for the SPD system W Y = B: the solver the note ablates against
+    Newton-Schulz ([P1] 关键设计 3 and its ablation). One independent Hestenes-Stiefel recursion
+    per right-hand-side column, Y_0 = 0, exactly ``iters`` iterations, every operation in
+    ``dtype`` (float64, or float32 to see the single-precision behaviour).
+    """
+    W = np.asarray(W, dtype=dtype)
+    B = np.asarray(B, dtype=dtype)
+    Y = np.zeros_like(B)
+    R = B.copy()
+    P = R.copy()
+    rr = (R * R).sum(axis=0)
+    for _ in range(iters):
+        WP = W @ P
+        pwp = (P * WP).sum(axis=0)
+        a = np.divide(rr, pwp, out=np.zeros_like(rr), where=pwp > 0)
+        Y = Y + a * P
+        R = R - a * WP
+        rr_new = (R * R).sum(axis=0)
+        beta = np.divide(rr_new, rr, out=np.zeros_like(rr), where=rr > 0)
+        P = R + beta * P
+        rr = rr_new
+    return Y
+
+
+def newton_schulz_dtype(W: np.ndarray, alpha: float, T: int, dtype=np.float32) -> np.ndarray:
+    """newton_schulz's X_T with every product in ``dtype`` (the single-precision counterpart
+    used to compare the two solvers' robustness)."""
+    W = np.asarray(W, dtype=dtype)
+    I2 = 2.0 * np.eye(W.shape[0], dtype=dtype)
+    X = dtype(alpha) * W.T
+    for _ in range(T):
+        X = X @ (I2 - W @ X)
+    return X
+
+
 def whiten_columns(C: np.ndarray, eps: float):
     """Diagonal centring + whitening of [P1] 关键设计 1 (R5): per column mean mu and
     population variance var over the N rows; C~ = (C - mu)/sqrt(var + eps) + 1/N.

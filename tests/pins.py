@@ -163,6 +163,30 @@ def check_ns_kappa50_and_quadratic():
             assert abs(r2n - r2 ** 2) <= 1e-9 + 1e-7 * r2 ** 2, f"||R_k+1|| != ||R_k||^2 at {k}"
 
 
+def check_cg_vs_solve():
+    # in exact arithmetic CG terminates in m steps; with a small condition number fp64 gets there
+    rng = _rng(71)
+    Wm = _spd(16, 5.0, 14)
+    Bm = rng.standard_normal((16, 6))
+    Y = O.cg_solve(Wm, Bm, 24)
+    ref = np.linalg.solve(Wm, Bm)
+    assert np.allclose(Y, ref, rtol=0, atol=1e-10 * np.abs(ref).max())
+
+
+def check_cg_error_bound():
+    # the classical bound ||e_k||_W <= 2 ((sqrt k - 1) / (sqrt k + 1))^k ||e_0||_W at kappa = 50
+    kappa = 50.0
+    Wm = _spd(49, kappa, 15)
+    b = _rng(72).standard_normal((49, 1))
+    y = np.linalg.solve(Wm, b)
+    e0 = float(np.sqrt((y.T @ Wm @ y).item()))
+    rho = (np.sqrt(kappa) - 1.0) / (np.sqrt(kappa) + 1.0)
+    for k in range(1, 25):
+        e = O.cg_solve(Wm, b, k) - y
+        ek = float(np.sqrt((e.T @ Wm @ e).item()))
+        assert ek <= 2.0 * rho ** k * e0 * (1 + 1e-9) + 1e-13 * e0, f"CG bound at step {k}"
+
+
 # --- Nystrom assembly -----------------------------------------------------------
 
 def check_nystrom_r1_dense():
@@ -454,5 +478,6 @@ ALL_PINS = [
     check_whitening_vs_sklearn, check_whitened_assembly_vs_solve, check_dwc_vs_conv2d,
     check_dwc_taps, check_backward_fd, check_injectivity_generic,
     check_batch_stats_single_batch, check_batch_stats_replicated, check_batch_stats_vs_sklearn,
-    check_reading_b_vs_dense, check_reading_b_r1_is_whitened_kernel,
+    check_reading_b_vs_dense, check_reading_b_r1_is_whitened_kernel, check_cg_vs_solve,
+    check_cg_error_bound,
 ]

@@ -12,7 +12,7 @@ from tests import pins
 _orig = {name: getattr(O, name) for name in (
     "laplacian_kernel", "l1_distances", "pool_landmarks", "landmark_gram", "newton_schulz",
     "whiten_columns", "dwc3x3", "_sign_contractions", "select_alpha", "pooled_column_stats",
-    "batch_groups", "unit_forward_reading_b")}
+    "batch_groups", "unit_forward_reading_b", "cg_solve")}
 
 
 def _kernel_no_lambda(X, Y, lam):
@@ -117,6 +117,19 @@ def _reading_b_variant(uncentred_cov=False, no_offset=False, sample_var=False):
     return f
 
 
+def _cg_steepest_descent(W, B, iters, dtype=np.float64):
+    # beta = 0: every direction is the residual (steepest descent), no conjugacy
+    W = np.asarray(W, dtype=dtype)
+    Y = np.zeros_like(np.asarray(B, dtype=dtype))
+    R = np.asarray(B, dtype=dtype).copy()
+    for _ in range(iters):
+        WR = W @ R
+        a = (R * R).sum(axis=0) / (R * WR).sum(axis=0)
+        Y = Y + a * R
+        R = R - a * WR
+    return Y
+
+
 def _dwc_convolution(Vu, w, H, W):
     return _orig["dwc3x3"](Vu, w[:, ::-1, ::-1].copy(), H, W)
 
@@ -142,6 +155,7 @@ MUTATIONS = [
     ("batch_stats_first_unit_only", "pooled_column_stats", _pooled_first_unit_only,
      [pins.check_batch_stats_vs_sklearn]),
     ("batch_stats_pooled_across_heads", "batch_groups", _groups_across_heads, [pins.check_batch_stats_vs_sklearn]),
+    ("cg_without_conjugacy", "cg_solve", _cg_steepest_descent, [pins.check_cg_vs_solve, pins.check_cg_error_bound]),
     ("reading_b_uncentred_covariance", "unit_forward_reading_b", _reading_b_variant(uncentred_cov=True),
      [pins.check_reading_b_vs_dense]),
     ("reading_b_no_offset", "unit_forward_reading_b", _reading_b_variant(no_offset=True),
