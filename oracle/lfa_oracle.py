@@ -38,7 +38,8 @@ design notes with its reason):
       statistics "over a batch" of similarity vectors: mu and var of landmark column l
       are taken over the B*N rows of every unit that shares the head h (all batch
       elements), population variance; C~ of each unit is then formed as in R6 with
-      that unit's own N in the 1/N offset. Forward only.
+      that unit's own N in the 1/N offset. Its reverse mode shares the whitening's
+      batch-norm backward across those units (backward(..., batch_stats=True)).
   R13 (alternative reading of R6, "Reading B", unit_forward_reading_b) the whitening acts
       on the columns of the whole Nystrom similarity matrix G^ = C X C^T (N x N, one
       column per key token j): g~_j = (g_j - mean_i g_ij) / sqrt(var_i g_ij + eps) + 1/N,
@@ -323,31 +324,28 @@ def _sign_contractions(Qu, L, dD):
     return dQ, dL
 
 
-def unit_backward(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten=True):
-    """Reverse mode through unit_forward (R9 kernel sign, R10 alpha constant).
-
-    Returns (dQ [N, d], dV [N, d], fwd). The loss is <dO, O>.
-    """
+def _backward_to_ct(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten, stats=None):
+    """First half of the reverse mode: through O = Ct M + DWC(V), M = X A, A = Ct^T V.
+    Returns (fwd, dCt, dX, dV)."""
     Qu = np.asarray(Qu, dtype=np.float64)
     Vu = np.asarray(Vu, dtype=np.float64)
     dO = np.asarray(dOu, dtype=np.float64)
-    f = unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten, keep_iterates=True)
-    N, d = Qu.shape
-    m = f.L.shape[0]
-    # O = Ct M + DWC(V),  M = X A,  A = Ct^T V
+    f = unit_forward(Qu, Vu, w, H, W, r, lam, eps, T, whiten, keep_iterates=True, stats=stats)
     dV = dwc3x3_transpose(dO, np.asarray(w, dtype=np.float64), H, W)
     dM = f.Ct.T @ dO
     dX = dM @ f.A.T
     dA = f.X.T @ dM
     dCt = dO @ f.M.T + Vu @ dA.T
     dV = dV + f.Ct @ dA
-    # whitening (population-variance batch-norm form), then C = exp(-D/lam)
-    if whiten:
-        s = 1.0 / np.sqrt(f.var + eps)
-        Chat = (f.C - f.mu) * s
-        dC = s * (dCt - dCt.mean(axis=0) - Chat * (dCt * Chat).mean(axis=0))
-    else:
-        dC = dCt
+    return f, dCt, dX, dV
+
+
+def _backward_from_c(Qu, f, dC, dX, H, W, r, lam, eps, T):
+    """Second half: through C = exp(-D/lam), the Newton-Schulz chain, W and the pooling.
+    Returns dQ."""
+    Qu = np.asarray(Qu, dtype=np.float64)
+    N, d = Qu.shape
+    m = f.L.shape[0]
     dD = -(f.C * dC) / lam
     dQ, dL = _sign_contractions(Qu, f.L, dD)
     # Newton-Schulz: X_{k+1} = 2 X_k - X_k W X_k, X_0 = alpha W^T (alpha held constant)
@@ -366,7 +364,28 @@ def unit_backward(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten=True):
     # L = pool(Q): every token of window l receives dL_l / r^2
     Wr = W // r
     g = dL.reshape(H // r, 1, Wr, 1, d) / (r * r)
-    dQ = dQ + np.broadcast_to(g, (H // r, r, Wr, r, d)).reshape(N, d)
+    return dQ + np.broadcast_to(g, (H // r, r, Wr, r, d)).reshape(N, d)
+
+
+def _whitening_backward(dCts, Cs, mu, var, eps):
+    """Batch-norm form of the whitening's reverse mode (population variance) over the stacked
+    rows of the listed units, whose statistics (mu, var) are shared: returns one dC per unit."""
+    s = 1.0 / np.sqrt(var + eps)
+    Chat = np.concatenate([(C - mu) * s for C in Cs])
+    dCt = np.concatenate(dCts)
+    dC = s * (dCt - dCt.mean(axis=0) - Chat * (dCt * Chat).mean(axis=0))
+    return np.split(dC, np.cumsum([len(C) for C in Cs])[:-1])
+
+
+def unit_backward(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten=True):
+    """Reverse mode through unit_forward (R9 kernel sign, R10 alpha constant).
+
+    Returns (dQ [N, d], dV [N, d], fwd). The loss is <dO, O>.
+    """
+    f, dCt, dX, dV = _backward_to_ct(Qu, Vu, w, dOu, H, W, r, lam, eps, T, whiten)
+    # whitening (population-variance batch-norm form), then C = exp(-D/lam)
+    dC = _whitening_backward([dCt], [f.C], f.mu, f.var, eps)[0] if whiten else dCt
+    dQ = _backward_from_c(Qu, f, dC, dX, H, W, r, lam, eps, T)
     return dQ, dV, f
 
 
@@ -474,8 +493,14 @@ def forward(Q, V, dwc, wl, whiten=True, units=None, keep_units=True, batch_stats
     return Forward(O, Oa, us)
 
 
-def backward(Q, V, dwc, dO, wl, whiten=True, units=None):
-    """Oracle gradients (dQ, dV), [B, heads, N, d], for the loss <dO, O>."""
+def backward(Q, V, dwc, dO, wl, whiten=True, units=None, batch_stats=False):
+    """Oracle gradients (dQ, dV), [B, heads, N, d], for the loss <dO, O>.
+
+    ``batch_stats`` (R12): the statistics, and so the whitening's reverse mode, are shared by
+    the units of a head; every unit is then computed (``units`` is ignored).
+    """
+    if whiten and batch_stats:
+        return _backward_batch_stats(Q, V, dwc, dO, wl)
     Q = np.asarray(Q, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
     dO = np.asarray(dO, dtype=np.float64)
@@ -490,4 +515,34 @@ def backward(Q, V, dwc, dO, wl, whiten=True, units=None):
                                   wl.lam, wl.eps, wl.T, whiten)
         dQ[b, h] = gq
         dV[b, h] = gv
+    return dQ, dV
+
+
+def _backward_batch_stats(Q, V, dwc, dO, wl):
+    """R12 reverse mode: per head, the whitening backward runs over the stacked rows of all
+    batch elements (their shared mean and variance), the rest per unit."""
+    Q = np.asarray(Q, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    w = np.asarray(dwc, dtype=np.float64)
+    B, nh, N, d = Q.shape
+    dQ = np.zeros_like(Q)
+    dV = np.zeros_like(Q)
+    for grp in batch_groups(B, nh):
+        Cs = []
+        for u in grp:
+            b, h = divmod(u, nh)
+            L = pool_landmarks(Q[b, h], wl.H, wl.W, wl.r)
+            Cs.append(laplacian_kernel(Q[b, h], L, wl.lam))
+        mu, var = pooled_column_stats(Cs)
+        halves = []
+        for u in grp:
+            b, h = divmod(u, nh)
+            halves.append(_backward_to_ct(Q[b, h], V[b, h], w[h], dO[b, h], wl.H, wl.W, wl.r, wl.lam,
+                                          wl.eps, wl.T, True, stats=(mu, var)))
+        dCs = _whitening_backward([hv[1] for hv in halves], [hv[0].C for hv in halves], mu, var, wl.eps)
+        for u, (f, _, dX, dVu), dC in zip(grp, halves, dCs):
+            b, h = divmod(u, nh)
+            dQ[b, h] = _backward_from_c(Q[b, h], f, dC, dX, wl.H, wl.W, wl.r, wl.lam, wl.eps, wl.T)
+            dV[b, h] = dVu
     return dQ, dV

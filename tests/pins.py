@@ -433,6 +433,53 @@ def check_backward_fd(cases=None):
         assert wv < 1e-6, f"dV vs finite differences: {wv} for {c}"
 
 
+def check_backward_batch_stats_fd(n_samples=24, h=1e-6):
+    # reading R12: two batch elements share the head's whitening statistics, so a token of one
+    # unit moves the other unit's output too; the gradient is checked through the whole call
+    B, heads = 2, 1
+    q, v, w, wl = _batch_case(B, heads, 81)
+    wl.eps = 1e-3
+    rng = _rng(82)
+    dO = rng.standard_normal(q.shape)
+    dQ, dV = O.backward(q, v, w, dO, wl, batch_stats=True)
+
+    def loss(qq, vv, attn_only=False):
+        f = O.forward(qq, vv, w, wl, batch_stats=True)
+        return float(np.sum(dO * (f.O_attn if attn_only else f.O)))
+
+    N, d = q.shape[2], q.shape[3]
+    Ls = [O.pool_landmarks(q[b, 0], wl.H, wl.W, wl.r) for b in range(B)]
+    worst_q, checked = 0.0, 0
+    scale_q = np.abs(dQ).max()
+    for idx in rng.permutation(B * N * d):
+        b, rest = divmod(int(idx), N * d)
+        i, k = divmod(rest, d)
+        L = Ls[b]
+        if np.min(np.abs(q[b, 0, i, k] - L[:, k])) < 20 * h:
+            continue
+        pd = np.abs(L[:, None, k] - L[None, :, k])[~np.eye(len(L), dtype=bool)]
+        if np.min(pd, initial=np.inf) < 20 * h / (wl.r * wl.r):
+            continue
+        qp = q.copy(); qp[b, 0, i, k] += h
+        qm = q.copy(); qm[b, 0, i, k] -= h
+        fd = (loss(qp, v, True) - loss(qm, v, True)) / (2 * h)
+        worst_q = max(worst_q, abs(fd - dQ[b, 0, i, k]) / scale_q)
+        checked += 1
+        if checked >= n_samples:
+            break
+    assert checked >= n_samples // 2, "too few kink-free coordinates"
+    assert worst_q < 1e-6, f"dQ vs finite differences: {worst_q}"
+    worst_v, scale_v = 0.0, np.abs(dV).max()
+    for idx in rng.choice(B * N * d, size=n_samples // 2, replace=False):
+        b, rest = divmod(int(idx), N * d)
+        i, k = divmod(rest, d)
+        vp = v.copy(); vp[b, 0, i, k] += h
+        vm = v.copy(); vm[b, 0, i, k] -= h
+        fd = (loss(q, vp) - loss(q, vm)) / (2 * h)
+        worst_v = max(worst_v, abs(fd - dV[b, 0, i, k]) / scale_v)
+    assert worst_v < 1e-6, f"dV vs finite differences: {worst_v}"
+
+
 # --- injectivity (the pages' claim for the exact map; see the counterexample) --------
 
 def check_injectivity_generic():
@@ -479,5 +526,5 @@ ALL_PINS = [
     check_dwc_taps, check_backward_fd, check_injectivity_generic,
     check_batch_stats_single_batch, check_batch_stats_replicated, check_batch_stats_vs_sklearn,
     check_reading_b_vs_dense, check_reading_b_r1_is_whitened_kernel, check_cg_vs_solve,
-    check_cg_error_bound,
+    check_cg_error_bound, check_backward_batch_stats_fd,
 ]

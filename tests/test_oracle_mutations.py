@@ -12,7 +12,7 @@ from tests import pins
 _orig = {name: getattr(O, name) for name in (
     "laplacian_kernel", "l1_distances", "pool_landmarks", "landmark_gram", "newton_schulz",
     "whiten_columns", "dwc3x3", "_sign_contractions", "select_alpha", "pooled_column_stats",
-    "batch_groups", "unit_forward_reading_b", "cg_solve")}
+    "batch_groups", "unit_forward_reading_b", "cg_solve", "_whitening_backward")}
 
 
 def _kernel_no_lambda(X, Y, lam):
@@ -130,6 +130,11 @@ def _cg_steepest_descent(W, B, iters, dtype=np.float64):
     return Y
 
 
+def _whitening_backward_per_unit(dCts, Cs, mu, var, eps):
+    # each unit's reverse mode on its own rows although the statistics are shared
+    return [_orig["_whitening_backward"]([g], [C], mu, var, eps)[0] for g, C in zip(dCts, Cs)]
+
+
 def _dwc_convolution(Vu, w, H, W):
     return _orig["dwc3x3"](Vu, w[:, ::-1, ::-1].copy(), H, W)
 
@@ -155,6 +160,8 @@ MUTATIONS = [
     ("batch_stats_first_unit_only", "pooled_column_stats", _pooled_first_unit_only,
      [pins.check_batch_stats_vs_sklearn]),
     ("batch_stats_pooled_across_heads", "batch_groups", _groups_across_heads, [pins.check_batch_stats_vs_sklearn]),
+    ("batch_stats_backward_per_unit", "_whitening_backward", _whitening_backward_per_unit,
+     [pins.check_backward_batch_stats_fd]),
     ("cg_without_conjugacy", "cg_solve", _cg_steepest_descent, [pins.check_cg_vs_solve, pins.check_cg_error_bound]),
     ("reading_b_uncentred_covariance", "unit_forward_reading_b", _reading_b_variant(uncentred_cov=True),
      [pins.check_reading_b_vs_dense]),
