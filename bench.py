@@ -21,6 +21,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -120,9 +121,9 @@ def kernel_traffic(kernel: str, workload: str):
 class ClockSampler:
     def __init__(self, device_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        fd, self.path = tempfile.mkstemp(prefix=f"lfa_clocks_rank{device_index}_", suffix=".csv")
+        os.close(fd)
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader,nounits",
@@ -140,7 +141,12 @@ class ClockSampler:
             self.proc.kill()
         self.fh.close()
         rows = []
-        for ln in open(self.path).read().splitlines():
+        text = open(self.path).read()
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
+        for ln in text.splitlines():
             f = [c.strip() for c in ln.split(",")]
             if len(f) >= 9:
                 rows.append(f)

@@ -23,8 +23,15 @@
  *
  * Conventions for every entry point:
  *   - Tensors Q, V, O, dO, dQ, dV are contiguous [B][heads][N][d] in the config's
- *     dtype (fp32 or bf16); arithmetic is fp32 throughout. Device pointers must be
- *     16-byte aligned. The DWC weight is fp32 [heads][d][3][3] on the device.
+ *     dtype (fp32 or bf16). Device pointers must be 16-byte aligned.
+ *     Arithmetic: distances, exponentials, sums and the whitening statistics are fp32 (the
+ *     statistics' cross-CTA reductions fp64). The per-stage kernels (every fp32 shape, and
+ *     the bf16 shapes the fused kernel does not take) do every product in fp32 on CUDA
+ *     cores. The fused bf16 kernel (lfa_forward_path "fused") instead keeps C as bf16 on
+ *     chip and runs C^T V and C M' as bf16-operand tensor-core products with fp32
+ *     accumulation, and the m x m Newton-Schulz and M = X A products as split-TF32
+ *     tensor-core products (hi*hi + hi*lo + lo*hi, fp32 accumulation).
+ *   - The DWC weight is fp32 [heads][d][3][3] on the device.
  *   - All device memory is owned by the caller. The handle owns host state only and
  *     keeps the weight and workspace pointers it was created with; the weight is read
  *     at every call, not copied.
@@ -89,6 +96,9 @@ typedef struct {
   float alpha;           /* alpha used for X_0 */
   float lambda_max;      /* estimate of ||W||_2 (power iteration; W is SPD) */
   float ns_residual_fro; /* ||I - W X_T||_F after the last step */
+  float kappa;           /* estimate of the condition number of W + eps I: lambda_max times
+                            ||X_T||_2 (power iteration; X_T approximates (W + eps I)^-1 once the
+                            chain has converged), computed by lfa_get_info itself */
 } lfa_unit_info;
 
 typedef struct lfa_ctx* lfa_handle;
@@ -121,9 +131,10 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
  * allocator, or a latency-critical caller that cannot take the device-wide
  * synchronisation of cudaMalloc / cudaFree.
  *   cfg, dwc_weight, Q, V, O, stream: as for lfa_create and lfa_forward.
- *   Setup: the first call on each device (with that device current) resolves the
- *   address of the scratch array for that device; make that first call before any
- *   stream capture begins. Later calls only validate and enqueue.
+ *   Setup: every call looks up the device address of the scratch array on the current device
+ *   (cudaGetSymbolAddress, a host-side query; nothing is cached across calls). The first call on a
+ *   device may also load the library's device code there, so make that first call before any
+ *   stream capture begins.
  *   Zeroing: nothing has to start at zero. Every scratch byte a call reads is written
  *   earlier by the same call; its status word is cleared by the call's first kernel.
  *   Limit: the scratch a config needs grows with B*heads and m (about
@@ -157,7 +168,8 @@ lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* 
                         void* dQ, void* dV, void* stream);
 
 /* Copy per-unit diagnostics of the last forward into host_out[0..n_units-1]
- * (n_units must equal B * heads) and return the device status word
+ * (n_units must equal B * heads; the kappa estimate comes from one small kernel this call
+ * launches on `stream`) and return the device status word
  * (LFA_OK, LFA_ERR_TIMEOUT or LFA_ERR_NONFINITE). Synchronises `stream`. After a
  * timeout the outputs of that call are invalid; the handle resets its cross-CTA flags
  * on the next forward. */
@@ -171,10 +183,35 @@ const char* lfa_status_string(lfa_status s);
 
 /* ---- inspection entry points used by the parity tests ---------------------- */
 
-/* Cross kernel C of one unit, written as fp32 [N][m] to the device buffer C_out,
- * computed by the same device code the forward pass uses. */
+/* Cross kernel C = exp(-||q_i - l_l||_1 / lambda) of one unit [the note's §关键设计 2],
+ * written as fp32 [N][m] to the device buffer C_out by the per-stage kernels' tile code
+ * (fp32 distance and exp2f), after pooling Q's landmarks into the handle's workspace. That
+ * pooling replaces the saved forward context: lfa_backward then needs a new lfa_forward
+ * (LFA_ERR_STATE until then). For the C that a fused forward itself computes, see
+ * lfa_debug_capture_cross. */
 lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* C_out,
                                   void* stream);
+
+/* Test of the bounded waits (no device fault, no hang): the NEXT lfa_forward on this handle waits
+ * for one pooled landmark more than any unit has (a flag value that nothing sets), and every wait of
+ * that call for a flag that other thread blocks set is bounded by budget_cycles SM clock cycles
+ * instead of about one second. Those waits run out, the call sets the timeout bit of the status
+ * word and still completes (its outputs are invalid); lfa_get_info then returns LFA_ERR_TIMEOUT and
+ * re-arms the flags, so the forward after it is a normal one. Waits on the thread block's own
+ * tensor-core and TMA operations keep their usual bound. Fused path only (LFA_ERR_UNSUPPORTED on the
+ * per-stage path, which has no cross-block waits); LFA_ERR_INVALID_ARG for a negative budget. */
+lfa_status lfa_debug_spin_test(lfa_handle h, long long budget_cycles);
+
+/* Arm a one-shot copy of the cross kernel C of `unit` as the NEXT lfa_forward on this handle
+ * computes it, written as fp32 [N][m] to the device buffer C_out (at least N*m floats, owned by the
+ * caller, untouched until that forward runs). On the fused path the forward keeps bf16(C - c) on chip
+ * and multiplies it in pass 2, with c a per-column shift that each thread block takes from the mean
+ * of C over the first 16 tokens of its rows of the unit (the bias of pass 2 adds c back exactly); C
+ * is computed by ex2.approx from the fp32 distance sum. The copy is that bf16 value widened to fp32
+ * plus c, and shift_out (NULL, or a device buffer of N*m floats) receives c for every entry. On the
+ * per-stage path the forward's tile code computes C again for the copy, in fp32, and shift_out is
+ * zeroed. Host-only; LFA_ERR_INVALID_ARG for a bad unit or a NULL C_out. */
+lfa_status lfa_debug_capture_cross(lfa_handle h, int unit, float* C_out, float* shift_out);
 
 /* Copy the forward context of one unit (device -> device, fp32): landmarks L [m][d],
  * Newton-Schulz result X [m][m], whitening mean mu [m] and scale s [m]. Any output

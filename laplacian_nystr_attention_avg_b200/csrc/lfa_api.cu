@@ -24,6 +24,10 @@ struct lfa_ctx {
   int path;   // 0 = generic, 1 = fused
   int grid;   // CTAs of the fused kernel
   unsigned long long epoch;   // forward calls issued (the fused kernel's flag generation)
+  float* cap_C;   // armed by lfa_debug_capture_cross: the next forward copies C of cap_unit here
+  float* cap_S;   // and, if set, the column shift of each entry
+  int cap_unit;
+  long long spin_test_budget;   // armed by lfa_debug_spin_test (>= 0): the next forward's flag waits
 };
 
 namespace {
@@ -68,6 +72,7 @@ void plan(const lfa_config* c, Params* p, Layout* L) {
   p->lam = c->lambda;
   p->eps = c->eps;
   p->neg_log2e_over_lam = (float)(-1.4426950408889634 / (double)c->lambda);
+  p->spin_budget = lfa::kFlagSpinBudget;
   p->n_tiles = lfa::ceil_div(p->N, lfa::kRowTile);
   // about two pass-1 CTAs per SM of a 148-SM part
   const int want = lfa::ceil_div(296, p->U);
@@ -239,6 +244,7 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
   }
   h->ws = static_cast<unsigned char*>(workspace);
   h->ws_bytes = workspace_bytes;
+  h->spin_test_budget = -1;
   bind(&h->p, h->lay, h->ws);
   h->p.dwc = dwc_weight;
   h->path = 0;
@@ -269,12 +275,29 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
   p.V = V;
   p.O = O;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* cap = h->cap_C;
+  float* cap_s = h->cap_S;
+  h->cap_C = nullptr;   // one-shot
+  h->cap_S = nullptr;
   if (h->path == 1) {
     const unsigned long long epoch = h->epoch + 1;
+    p.dbgC = cap;
+    p.dbgS = cap ? cap_s : nullptr;
+    p.dbg_unit = h->cap_unit;
+    if (h->spin_test_budget >= 0) {
+      p.spin_test = 1;
+      p.spin_budget = h->spin_test_budget;
+      h->spin_test_budget = -1;   // one-shot
+    }
     if (lfa::launch_fused_forward(p, h->grid, h->ws + h->lay.fused, epoch, st) != cudaSuccess) return LFA_ERR_CUDA;
     h->epoch = epoch;
   } else {
     if (lfa::launch_generic_forward(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+    // the per-stage passes keep C in registers: the same tile code, run once more for the copy
+    if (cap && lfa::launch_cross_kernel(p, h->cap_unit, cap, st) != cudaSuccess) return LFA_ERR_CUDA;
+    if (cap && cap_s &&
+        cudaMemsetAsync(cap_s, 0, sizeof(float) * (size_t)h->p.N * h->p.m, st) != cudaSuccess)
+      return LFA_ERR_CUDA;
   }
   h->last_Q = Q;
   h->last_V = V;
@@ -289,22 +312,13 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[LFA_NOALLOC_SCR
 
 namespace {
 
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-unsigned char* g_noalloc_ptr[kNoAllocMaxDevices];   // device address of the array, per device
-
-// Address of the scratch array on the current device, resolved once per device.
+// Address of the scratch array on the current device. Resolved at every call (a host-side query):
+// a cached address would go stale if the device's context were torn down and re-created, since the
+// module, and with it the array, is then loaded again at a new address.
 lfa_status noalloc_scratch(unsigned char** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LFA_ERR_CUDA;
-  if (dev < 0 || dev >= kNoAllocMaxDevices) return LFA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LFA_ERR_CUDA;
-    g_noalloc_ptr[dev] = static_cast<unsigned char*>(ptr);
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return LFA_ERR_CUDA;
+  *out = static_cast<unsigned char*>(ptr);
   return LFA_OK;
 }
 
@@ -384,6 +398,11 @@ lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void
   if (!tmp) return LFA_ERR_INVALID_ARG;
   int status = 0;
   lfa_status ret = LFA_OK;
+  // the condition-number estimate is computed here, outside the forward
+  if (h->have_forward && lfa::launch_kappa(h->p, st) != cudaSuccess) {
+    free(tmp);
+    return LFA_ERR_CUDA;
+  }
   if (cudaMemcpyAsync(tmp, h->p.info, n * sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaMemcpyAsync(&status, h->p.status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess) {
@@ -395,6 +414,7 @@ lfa_status lfa_get_info(lfa_handle h, lfa_unit_info* host_out, int n_units, void
       host_out[u].lambda_max = f[lfa::kInfoLambdaMax];
       host_out[u].alpha_fallback = f[lfa::kInfoFallback] != 0.f;
       host_out[u].ns_residual_fro = f[lfa::kInfoResidual];
+      host_out[u].kappa = h->have_forward ? f[lfa::kInfoKappa] : 0.f;
     }
     if (status & lfa::kStatusTimeout) {
       ret = LFA_ERR_TIMEOUT;
@@ -411,8 +431,25 @@ lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* 
   Params p = h->p;
   p.Q = Q;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the landmarks are pooled into the handle's workspace, replacing the forward context there
+  h->have_forward = 0;
   if (lfa::launch_pool(p, st) != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::launch_cross_kernel(p, unit, C_out, st) != cudaSuccess) return LFA_ERR_CUDA;
+  return LFA_OK;
+}
+
+lfa_status lfa_debug_spin_test(lfa_handle h, long long budget_cycles) {
+  if (!h || budget_cycles < 0) return LFA_ERR_INVALID_ARG;
+  if (h->path != 1) return LFA_ERR_UNSUPPORTED;
+  h->spin_test_budget = budget_cycles;
+  return LFA_OK;
+}
+
+lfa_status lfa_debug_capture_cross(lfa_handle h, int unit, float* C_out, float* shift_out) {
+  if (!h || unit < 0 || unit >= h->p.U || !C_out) return LFA_ERR_INVALID_ARG;
+  h->cap_C = C_out;
+  h->cap_S = shift_out;
+  h->cap_unit = unit;
   return LFA_OK;
 }
 

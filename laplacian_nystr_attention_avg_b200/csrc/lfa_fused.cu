@@ -48,7 +48,11 @@ constexpr int kV1Thread = 12 * 32;        // pass 1: issues the V chunk loads (w
 constexpr int kChunk = 128;               // token rows per chunk
 constexpr int kMaxChunks = 8;             // resident C chunks per CTA
 constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q, L and halo tiles
-constexpr int kRec = 128 + 64 * 64;       // floats per partial record: S1[64], S2[64], P[64][64]
+// floats per partial record: S1'[64], S2'[64], P'[64][64] (sums of the shifted C - c), c[64], the
+// segment's row count n, padding to a multiple of 64
+constexpr int kRec = 128 + 64 * 64 + 128;
+constexpr int kRecC = 128 + 64 * 64;      // offset of c
+constexpr int kRecN = kRecC + 64;         // offset of n
 constexpr int kMaxGrid = 256;             // records are sized for up to this many CTAs
 constexpr int kMaxContrib = 32;           // CTAs contributing to one unit
 constexpr int kPowerIters = 8;
@@ -64,22 +68,28 @@ constexpr uint32_t kOffBar = kOffBv + 512;                      // mbarriers + T
 constexpr uint32_t kOffCt = kOffBar + 256;                      // int [32] record offsets
 constexpr uint32_t kOffSr = kOffCt + 128;                       // pass-1 column sums [segment][row half][128]
 constexpr uint32_t kOffRows = kOffSr + 2 * 256 * 4;            // this CTA's row plan (struct Rows)
-constexpr uint32_t kSmemBytes = kOffRows + 64;
+constexpr uint32_t kOffSh = kOffRows + 64;                      // per-segment column shift of C, fp32 [2][64]
+constexpr uint32_t kSmemBytes = kOffSh + 2 * 64 * 4;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
-// pass-2 scratch: V rows of one chunk with a one-grid-row halo on each side, SW128 (TMA boxes of
-// 128 rows), one or two buffers in the region of the V stages, Q and L (free after pass 1)
-constexpr uint32_t kOffHb = kOffV;
-constexpr uint32_t kHaloSpace = kOffMp - kOffV;
-constexpr int kImgBytes = 8192 + 256;                           // published M' image + b per unit
-// combine scratch (aliases V/Q/L, free once pass 1 is done)
-constexpr uint32_t kOffAs = kOffV;                              // fp32 [64][68]  A (row l, col k)
-constexpr uint32_t kOffXt = kOffAs + 64 * kQS * 4;              // fp32 [64][68]  X^T (row l, col j)
+// After pass 1 the region of the V stages, Q and L (kOffV .. kOffMp) is free. It holds, in order:
+//   DWC: the second bf16 staging tile (the first is C slot kMaxChunks - 1) and the 3 x 3 weights of
+//        up to two heads, fp32 [2][9][64];
+//   combine scratch: A [64][68] and X^T [64][68] fp32, the column statistics, the contributor
+//        table and the partial sums of b;
+//   the second segment's M'^T image (the first segment's is at kOffMp).
+constexpr uint32_t kOffStg1 = kOffV;                            // bf16 SW128 [128][64]
+constexpr uint32_t kOffDw = kOffStg1 + 16384;                   // fp32 [2][9][64]
+constexpr uint32_t kOffAs = kOffDw + 2 * 9 * 64 * 4;            // fp32 [64][68]  A (row l, col k)
+constexpr uint32_t kOffXt = kOffAs + 64 * kQS * 4;              // fp32 [64][68]  X^T (row j, col l)
 constexpr uint32_t kOffS1 = kOffXt + 64 * kQS * 4;              // double [64]
 constexpr uint32_t kOffS2 = kOffS1 + 512;                       // double [64]
 constexpr uint32_t kOffMu = kOffS2 + 512;                       // float [64]
 constexpr uint32_t kOffSc = kOffMu + 256;                       // float [64]
 constexpr uint32_t kOffSv = kOffSc + 256;                       // float [64]
-constexpr uint32_t kOffBp = kOffSv + 256;                       // float [16][64]
+constexpr uint32_t kOffMt = kOffSv + 256;                       // float [64] unshifted column mean
+constexpr uint32_t kOffBp = kOffMt + 256;                       // float [kWarps][8] partial b
+constexpr uint32_t kOffWc = kOffBp + kWarps * 8 * 4;            // int [kWarps] contributor counts
+constexpr uint32_t kOffImg1 = (kOffWc + kWarps * 4 + 1023) / 1024 * 1024;   // M'^T of segment 1
 // solver scratch (aliases the C region: the solver runs before this CTA's pass 1)
 constexpr uint32_t kOffNsHi = 0;                                // tf32 hi [2 K-halves][128 rows][128 B]
 constexpr uint32_t kOffNsLo = 32768;                            // tf32 lo
@@ -89,7 +99,7 @@ constexpr uint32_t kOffNsL = kOffNsX + 64 * kQS * 4;            // fp32 [64][68]
 constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64] + reduction [16]
 
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
-static_assert(kOffBp + (kFT / 16) * 64 * 4 <= kOffMp, "combine scratch overlaps M'");
+static_assert(kOffImg1 + 8192 <= kOffMp, "post-pass-1 scratch overlaps M'");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -97,24 +107,21 @@ constexpr int kBarV = 0;      // [3] V stage filled by TMA
 constexpr int kBarP1 = 3;     // [2] pass-1 product done
 constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (one use per launch)
 constexpr int kBarNs = 13;    // solver product done
-constexpr int kBarH = 14;     // [2] DWC V halo tile landed (TMA)
+constexpr int kBarDiag = 14;  // the solver's diagnostics product done
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarDiag = kBarP2;       // solver CTAs (which run no pass 2): the diagnostics product
-constexpr int kBarComb = kBarP2 + 1;   // solver CTAs: the combine's M = X A product
 constexpr int kBarDw = 17;    // [2] DWC transfer product of staging buffer b done
-constexpr int kNumBars = kBarDw + 2;
+constexpr int kBarDrain = 19; // every tcgen05 operation of both issuing threads done (count 2)
+constexpr int kNumBars = kBarDrain + 1;
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
 
 struct FusedArgs {
   unsigned long long epoch;   // launch count of this handle (>= 1); flags compare against it
-  unsigned long long* gbar;   // grid barrier counter
+  unsigned long long* lready; // [U] landmarks of the unit pooled (counts landmarks, m per launch)
   unsigned long long* cnt;    // [U] partial records published per unit
   unsigned long long* xready; // [U] X published (holds the epoch)
-  unsigned long long* mready; // [U] M' image and b published (holds the epoch)
   float* rec;                 // [G][2][kRec]
-  unsigned char* mimg;        // [U][kImgBytes] M'^T bf16 (SW128 image of the pass-2 B operand), b fp32
   // pass-1 warp plan: warp w computes landmarks [wj0[w], wj0[w] + wlt[w]) of row half w / 8;
   // warp padw[h] writes the padding columns of row half h
   unsigned char wj0[kWarps], wlt[kWarps], padw[2];
@@ -307,63 +314,43 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
   float* vec = reinterpret_cast<float*>(sm + kOffNsVec);
   float* red = vec + 128;
   load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
-  if (t < 128) vec[t] = (t & 63) < m ? 1.f : 0.f;
   __syncthreads();
-  // W (symmetric): upper triangle, mirrored
-  for (int e = t; e < 64 * 64; e += kFT) {
-    const int a = e >> 6, b = e & 63;
-    if (a > b) continue;
-    float v = 0.f;
-    if (b < m) {
-      float acc = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < 64; k += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(&Ls[a * kQS + k]);
-        const float4 y = *reinterpret_cast<const float4*>(&Ls[b * kQS + k]);
-        acc += fabsf(x.x - y.x);
-        acc += fabsf(x.y - y.y);
-        acc += fabsf(x.z - y.z);
-        acc += fabsf(x.w - y.w);
+  // W (symmetric): entries a <= b < m of the upper triangle, dealt out evenly (entry e -> (a, b)
+  // in row-major triangle order), mirrored; padding rows and columns are zero
+  {
+    const int ntri = m * (m + 1) / 2;
+    for (int e = t; e < 64 * 64; e += kFT) Ws[(e >> 6) * kQS + (e & 63)] = 0.f;
+    __syncthreads();
+    for (int e = t; e < ntri; e += kFT) {
+      // row a holds entries [a m - a (a - 1) / 2, ...): invert with a float estimate, then fix up
+      int a = (int)((2.f * m + 1.f - sqrtf((2.f * m + 1.f) * (2.f * m + 1.f) - 8.f * (float)e)) * 0.5f);
+      a = a < 0 ? 0 : (a >= m ? m - 1 : a);
+      while (a > 0 && a * m - a * (a - 1) / 2 > e) --a;
+      while ((a + 1) * m - (a + 1) * a / 2 <= e) ++a;
+      const int b = a + (e - (a * m - a * (a - 1) / 2));
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < 64; k += 8) {
+        const float4 x0 = *reinterpret_cast<const float4*>(&Ls[a * kQS + k]);
+        const float4 y0 = *reinterpret_cast<const float4*>(&Ls[b * kQS + k]);
+        const float4 x1 = *reinterpret_cast<const float4*>(&Ls[a * kQS + k + 4]);
+        const float4 y1 = *reinterpret_cast<const float4*>(&Ls[b * kQS + k + 4]);
+        acc0 += fabsf(x0.x - y0.x);
+        acc1 += fabsf(x1.x - y1.x);
+        acc0 += fabsf(x0.y - y0.y);
+        acc1 += fabsf(x1.y - y1.y);
+        acc0 += fabsf(x0.z - y0.z);
+        acc1 += fabsf(x1.z - y1.z);
+        acc0 += fabsf(x0.w - y0.w);
+        acc1 += fabsf(x1.w - y1.w);
       }
-      v = exp2f(acc * p.neg_log2e_over_lam);
+      const float v = exp2f((acc0 + acc1) * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
+      Ws[a * kQS + b] = v;
+      Ws[b * kQS + a] = v;
     }
-    Ws[a * kQS + b] = v + (a == b && a < m ? p.eps : 0.f);
-    Ws[b * kQS + a] = v + (a == b && a < m ? p.eps : 0.f);
   }
   __syncthreads();
   trace_mark(p, 16);
-  // lambda_max = ||W||_2 (W symmetric positive definite): power iteration from the ones vector,
-  // scaled by 1/m per step (the Rayleigh quotient is scale free), one barrier per step
-  float lmax;
-  {
-    const int row = t >> 3, part = t & 7;
-    const float sc = 1.f / (float)m;
-    float wi = 0.f;
-    for (int it = 0; it <= kPowerIters; ++it) {
-      const float* vin = vec + 64 * (it & 1);
-      wi = 0.f;
-      if (row < m) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) wi = fmaf(Ws[row * kQS + 8 * part + j], vin[8 * part + j], wi);
-      }
-      wi += __shfl_xor_sync(0xffffffffu, wi, 1);
-      wi += __shfl_xor_sync(0xffffffffu, wi, 2);
-      wi += __shfl_xor_sync(0xffffffffu, wi, 4);
-      if (it == kPowerIters) break;
-      if (part == 0) vec[64 * ((it + 1) & 1) + row] = row < m ? wi * sc : 0.f;
-      __syncthreads();
-    }
-    const float* vl = vec + 64 * (kPowerIters & 1);
-    float vw = (part == 0 && row < m) ? wi * vl[row] : 0.f;
-    float vv = (part == 0 && row < m) ? vl[row] * vl[row] : 0.f;
-    block_reduce2(vw, vv, red);
-    lmax = vw / vv;
-  }
-  // alpha = 2/||W||_2 as printed is kept only if ||I - alpha W W^T||_2 < 1, i.e. alpha lmax^2 < 2
-  const float alpha_p = 2.f / lmax;
-  const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
-  const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
-  trace_mark(p, 17);
 
   const int q = w & 3, h = w >> 2;
   const int r = 32 * q + lane;         // stacked row 0..127
@@ -377,22 +364,22 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
 #pragma unroll
   for (int c = 0; c < 16; ++c) wrow[c] = Ws[i * kQS + 16 * h + c];
 
+  auto issue_round = [&]() {
+    if (t == 0) ns_issue(sbase, tmem, bar, nks);
+    __syncwarp();
+  };
+  auto finish_round = [&]() {
+    mbar_wait(bar, round & 1, p.status, kStatusTimeout);
+    tc_fence_after();
+    tmem_ld16(trow, d);
+    ++round;
+  };
   auto run_round = [&]() {
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (round == 5) trace_mark(p, 20);
-    if (t == 0) ns_issue(sbase, tmem, bar, nks);
-    if (round == 5) trace_mark(p, 21);
-    __syncwarp();
-    mbar_wait(bar, round & 1, p.status, kStatusTimeout);
-    if (round == 5) trace_mark(p, 22);
-    tc_fence_after();
-    tmem_ld16(trow, d);
-    if (round == 5) trace_mark(p, 23);
-    if (round == 0) trace_mark(p, 18);
-    if (round == 10) trace_mark(p, 19);
-    ++round;
+    issue_round();
+    finish_round();
   };
   auto clean = [&](float* v) {
 #pragma unroll
@@ -400,14 +387,64 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
       if (i >= m || 16 * h + c >= m) v[c] = 0.f;
   };
 
-  // round 0: D_bottom = W W^T = W^2; X_0 = alpha W^T (= alpha W), R_0 = I - alpha W^2
+  // round 0: D_bottom = W W^T = W^2, which does not depend on alpha; while the tensor cores run it,
+  // warps 2-3 (one W row per thread; warp 0 is busy issuing the product) find lambda_max = ||W||_2
+  // (W symmetric positive definite) by power iteration from the ones vector, scaled by 1/m per
+  // step (the Rayleigh quotient is scale free), synchronising on named barrier 1 only
   {
     float v[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) v[c] = top ? 0.f : wrow[c];
     ns_store(sm, r, h, v);
   }
-  run_round();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  issue_round();
+  if (w == 2 || w == 3) {
+    const int row = t - 64;
+    const float sc = 1.f / (float)m;
+    float* v0 = vec;          // [2][64] ping-pong
+    v0[row] = row < m ? 1.f : 0.f;
+    named_bar_sync(1, 64);
+    float wi = 0.f;
+    for (int it = 0; it <= kPowerIters; ++it) {
+      const float* vin = v0 + 64 * (it & 1);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 64; j += 4) {
+        const float4 wv = *reinterpret_cast<const float4*>(&Ws[row * kQS + j]);
+        const float4 xv = *reinterpret_cast<const float4*>(&vin[j]);
+        a0 = fmaf(wv.x, xv.x, a0);
+        a1 = fmaf(wv.y, xv.y, a1);
+        a2 = fmaf(wv.z, xv.z, a2);
+        a3 = fmaf(wv.w, xv.w, a3);
+      }
+      wi = (a0 + a1) + (a2 + a3);
+      if (it == kPowerIters) break;
+      v0[64 * ((it + 1) & 1) + row] = wi * sc;
+      named_bar_sync(1, 64);
+    }
+    const float vl = v0[64 * (kPowerIters & 1) + row];
+    float vw = wi * vl, vv = vl * vl;
+    for (int o = 16; o > 0; o >>= 1) {
+      vw += __shfl_xor_sync(0xffffffffu, vw, o);
+      vv += __shfl_xor_sync(0xffffffffu, vv, o);
+    }
+    if (lane == 0) {
+      red[2 * (w - 2)] = vw;
+      red[2 * (w - 2) + 1] = vv;
+    }
+  }
+  __syncthreads();
+  const float lmax = (red[0] + red[2]) / (red[1] + red[3]);
+  // alpha = 2/||W||_2 as printed is kept only if ||I - alpha W W^T||_2 < 1, i.e. alpha lmax^2 < 2
+  const float alpha_p = 2.f / lmax;
+  const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
+  const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
+  trace_mark(p, 17);
+  finish_round();
+  // X_0 = alpha W^T (= alpha W), R_0 = I - alpha W^2
   if (top) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) st[c] = alpha * wrow[c];
@@ -416,20 +453,25 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
     for (int c = 0; c < 16; ++c) st[c] = (i == 16 * h + c ? 1.f : 0.f) - alpha * d[c];
   }
   clean(st);
-  const int n_lit = p.T < 2 ? p.T : 2;
+  trace_mark(p, 18);
+  const int n_lit = p.T < 1 ? p.T : 1;
   const int n_res = p.T - n_lit;
-  // residual steps: A = [X; R], D = [X R^T; R R^T]
+  // residual steps: A = [X; R], D = [X R^T; R R^T]. Once every |R_k| entry is at most 2^-30, X R_k
+  // and all later corrections (R squares at each step) are below 64 * 2^-30 = 2^-24 of max |X|, under
+  // one fp32 rounding of X's largest entries: the chain moves on to the printed step, which
+  // re-anchors R to I - W X. The test shares the barrier before the product's issue.
   for (int k = 0; k < n_res; ++k) {
-    // R_k exactly zero: every remaining residual step is the identity in floating point
-    // (X + X 0 = X, 0 0^T = 0), so the chain continues with the printed steps below
-    bool rnz = false;
+    bool big = false;
     if (!top) {
 #pragma unroll
-      for (int c = 0; c < 16; ++c) rnz |= st[c] != 0.f;
+      for (int c = 0; c < 16; ++c) big |= fabsf(st[c]) > 0x1p-30f;
     }
-    if (!__syncthreads_or(rnz)) break;
     ns_store(sm, r, h, st);
-    run_round();
+    fence_async_smem();
+    tc_fence_before();
+    if (!__syncthreads_or(big)) break;
+    issue_round();
+    finish_round();
     if (top) {
 #pragma unroll
       for (int c = 0; c < 16; ++c) st[c] += d[c];
@@ -439,6 +481,7 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
     }
     clean(st);
   }
+  trace_mark(p, 19);
   // printed product steps X <- X (2I - W X) = X + X (I - W X), two products each
   auto stage_w_over_x = [&]() {
     // A = [W; X]: top rows W, bottom rows X (from the top threads through shared memory)
@@ -547,7 +590,8 @@ __device__ void solver_diagnostics(const Params& p, unsigned char* sm, uint32_t 
 // lanes' rows spread the reads over all banks.
 template <int LT>
 __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float* Ls, unsigned char* cslot, int j0,
-                                            int rb, int nrows, float scale, float (&s1)[8], float (&s2)[8]) {
+                                            int rb, int nrows, float scale, const float (&sh)[8], float (&s1)[8],
+                                            float (&s2)[8]) {
   const int lane = threadIdx.x & 31;
   float acc[2][LT];
 #pragma unroll
@@ -590,7 +634,7 @@ __device__ __forceinline__ void cross_chunk(const unsigned char* qb, const float
     float c[LT];
 #pragma unroll
     for (int b = 0; b < LT; ++b) {
-      c[b] = valid ? ex2_approx(acc[a][b] * scale) : 0.f;
+      c[b] = valid ? ex2_approx(acc[a][b] * scale) - sh[b] : 0.f;
       s1[b] += c[b];
       s2[b] = fmaf(c[b], c[b], s2[b]);
     }
@@ -633,19 +677,58 @@ __device__ __forceinline__ void write_padding(unsigned char* cslot, int rb, int 
 }
 
 __device__ __forceinline__ void cross_dispatch(int lt, const unsigned char* Qs, const float* Ls, unsigned char* cslot,
-                                               int j0, int rb, int nrows, float scale, float (&s1)[8],
-                                               float (&s2)[8]) {
+                                               int j0, int rb, int nrows, float scale, const float (&sh)[8],
+                                               float (&s1)[8], float (&s2)[8]) {
   switch (lt) {
-    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
-    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, rb, nrows, scale, s1, s2); break;
+    case 1: cross_chunk<1>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 2: cross_chunk<2>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 3: cross_chunk<3>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 4: cross_chunk<4>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 5: cross_chunk<5>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 6: cross_chunk<6>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 7: cross_chunk<7>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
+    case 8: cross_chunk<8>(Qs, Ls, cslot, j0, rb, nrows, scale, sh, s1, s2); break;
     default: break;
   }
+}
+
+// Column shift of C for one segment of this CTA: c_l = the mean of C over the first min(16, rows)
+// tokens of the segment's first chunk, from its resident Q tile (bf16 SW128), in the pass-1
+// arithmetic. Pass 1 keeps bf16(C - c) on chip instead of bf16(C), so the rounding error of a
+// resident entry is relative to |C - c|, of the order of the column's spread, not to C: once
+// whitening divides by that spread, the error stays at the bf16 level whatever mu / sigma is (large
+// lambda). The segment's record carries c and its row count; the combine rebases every record of the
+// unit to this CTA's own c, and pass 2's bias adds c back. Warp w takes token w, lane the landmarks
+// lane and lane + 32; red is [16][64] fp32 scratch.
+__device__ void segment_shift(const Params& p, const unsigned char* qtile, int nrows, const float* Ls, float* red,
+                              float* shift) {
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31, m = p.m;
+  const int nr = nrows < 16 ? nrows : 16;
+  if (w < nr) {
+    float acc0 = 0.f, acc1 = 0.f;
+    const int l0 = lane, l1 = lane + 32 < m ? lane + 32 : lane;
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {
+      const uint4 qv = *reinterpret_cast<const uint4*>(qtile + sw128(w, k8));
+      const float q[8] = {bf_lo(qv.x), bf_hi(qv.x), bf_lo(qv.y), bf_hi(qv.y),
+                          bf_lo(qv.z), bf_hi(qv.z), bf_lo(qv.w), bf_hi(qv.w)};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        acc0 += fabsf(q[e] - Ls[l0 * kQS + 8 * k8 + e]);
+        acc1 += fabsf(q[e] - Ls[l1 * kQS + 8 * k8 + e]);
+      }
+    }
+    const float scale = p.neg_log2e_over_lam;
+    red[w * 64 + lane] = lane < m ? ex2_approx(acc0 * scale) : 0.f;
+    red[w * 64 + lane + 32] = lane + 32 < m ? ex2_approx(acc1 * scale) : 0.f;
+  }
+  __syncthreads();
+  if (t < 64) {
+    float c = 0.f;
+    for (int r = 0; r < nr; ++r) c += red[r * 64 + t];
+    shift[t] = t < m ? c / (float)nr : 0.f;
+  }
+  __syncthreads();
 }
 
 // Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
@@ -686,6 +769,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     }
   const bool padder = w == (rh ? fa.padw[1] : fa.padw[0]);
   const float scale = p.neg_log2e_over_lam;
+  float* shift = reinterpret_cast<float*>(sm + kOffSh);   // [segment][landmark]
+  float sh[8];
   // V chunk gc -> stage gc % 3 (its (gc / 3)-th fill)
   auto issue_v = [&](int gc) {
     int s, lo, nrows;
@@ -726,7 +811,12 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     // products run two chunks behind: tile gc - 2 is complete and its V stage has had a chunk
     if (t == 0 && gc >= 2) issue_mma(gc - 2);
     // Ls was last read before the previous chunk's closing barrier
+    if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (seg_first) {
+      if (t == 0) spin_until_geq(fa.lready + u, fa.epoch * (unsigned long long)m + (p.spin_test ? 1 : 0), p.status,
+                                     kStatusTimeout, p.spin_budget);
+      __syncthreads();
+      if (gc == 0) trace_mark(p, 2);
       load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
@@ -734,10 +824,13 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
         s2[b] = 0.f;
       }
       __syncthreads();
+      segment_shift(p, sm + kOffC + (gc + 1) * 16384, nrows, Ls, reinterpret_cast<float*>(sm + kOffQ + 16384),
+                    shift + 64 * s);
+#pragma unroll
+      for (int b = 0; b < 8; ++b) sh[b] = b < lt ? shift[64 * s + j0 + b] : 0.f;
     }
-    if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
-    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, s1, s2);
+    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, sh, s1, s2);
     if (padder) write_padding(cslot, 64 * rh, nrows, m);
     if (gc == 1) trace_mark(p, 22);
     if (seg_last) {
@@ -777,6 +870,22 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
   }
   wait_mma(nch - 1);
   tc_fence_after();
+  // inspection copy (lfa_debug_capture_cross): the resident bf16 tiles of C minus the column shift of
+  // one unit, widened to fp32 [N][m] with the shift added back: the C that pass 2 effectively uses
+  if (p.dbgC != nullptr) {
+    for (int gc = 0; gc < nch; ++gc) {
+      int s, lo, nrows;
+      R.chunk(gc, s, lo, nrows);
+      if (R.seg[s].u != p.dbg_unit) continue;
+      const unsigned char* cs = sm + kOffC + gc * 16384;
+      for (int e = t; e < nrows * m; e += kFT) {
+        const int row = e / m, col = e % m;
+        const uint32_t raw = *reinterpret_cast<const uint16_t*>(cs + sw128(row, col >> 3) + ((col & 7) << 1));
+        p.dbgC[(size_t)(lo + row) * m + col] = __uint_as_float(raw << 16) + shift[64 * s + col];
+        if (p.dbgS != nullptr) p.dbgS[(size_t)(lo + row) * m + col] = shift[64 * s + col];
+      }
+    }
+  }
   // records: S1, S2 and P (TMEM columns 64 s) per segment
   for (int s = 0; s < R.nseg; ++s) {
     float* rec = fa.rec + ((size_t)g * 2 + s) * kRec;
@@ -794,6 +903,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
       }
     }
     if (t < 128) rec[t] = (t & 63) < m ? sred[256 * s + t] + sred[256 * s + 128 + t] : 0.f;
+    if (t < 64) rec[kRecC + t] = shift[64 * s + t];
+    if (t == 64) rec[kRecN] = (float)(R.seg[s].hi - R.seg[s].lo);
   }
   tc_fence_before();
   __syncthreads();
@@ -804,14 +915,17 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 4, on the unit's solver CTA once X is known: sum the unit's records and form mu, var,
-// s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A, M' = diag(s) M and
-// b = (1/N - s o mu)^T M. M'^T is written as the bf16 SW128 image of pass 2's B operand and
-// published with b under a release flag.
+// Phase 3c, on every CTA holding rows of unit u, once X (from the unit's solver CTA) and every
+// contributor's pass-1 record are out: sum the unit's records and form mu, var, s = 1/sqrt(var +
+// eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A (fp32 FMA), M' = diag(s) M and
+// b = (1/N - s o mu)^T M. M'^T goes to `img` as the bf16 SW128 image of pass 2's B operand (row k =
+// channel, column l = landmark, zero for l >= m) and b to `bvec`. Every such CTA repeats this small
+// computation for itself (the same sums in the same order, so the same bits), which spares the
+// round trip through a single combining CTA before pass 2.
 // ---------------------------------------------------------------------------------------
-__device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, uint32_t sbase,
-                               uint32_t tmem, uint64_t* bars, int u) {
-  const int t = threadIdx.x;
+__device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, int u, const float* shift,
+                            unsigned char* img, float* bvec, bool write_stats) {
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int m = p.m, N = p.N;
   float* As = reinterpret_cast<float*>(sm + kOffAs);
   float* Xt = reinterpret_cast<float*>(sm + kOffXt);
@@ -821,17 +935,16 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   float* scs = reinterpret_cast<float*>(sm + kOffSc);
   float* svs = reinterpret_cast<float*>(sm + kOffSv);
   float* bps = reinterpret_cast<float*>(sm + kOffBp);
+  int* wcount = reinterpret_cast<int*>(sm + kOffWc);
   int* ctr = reinterpret_cast<int*>(sm + kOffCt);
   const float invNf = 1.f / (float)N;
   const double invN = 1.0 / (double)N;
-  // candidates gf..gl; CTAs with an empty range (possible when there are fewer chunks than
-  // CTAs) publish nothing and are dropped from the contributor table
+  // contributors: candidates gf..gl (the owners of the unit's first and last chunks); CTAs with an
+  // empty range (possible when there are fewer chunks than CTAs) publish nothing and are dropped
   const int nchu = (N + kChunk - 1) / kChunk;
   const int gf = chunk_owner(u * nchu, p);
   const int gl = chunk_owner(u * nchu + nchu - 1, p);
   const int ncand = gl - gf + 1;
-  // X^T of this unit is in shared memory (written by solver_cta at publication)
-  int* wcount = reinterpret_cast<int*>(sm + kOffBp);
   bool nonempty = false;
   int rec_off = 0;
   if (t < ncand) {
@@ -841,190 +954,234 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
     rec_off = (gg * 2 + (a < u * N ? 1 : 0)) * kRec;
   }
   const unsigned bal = __ballot_sync(0xffffffffu, nonempty);
-  if ((t & 31) == 0) wcount[t >> 5] = __popc(bal);
+  if (lane == 0) wcount[w] = __popc(bal);
   __syncthreads();
-  int before = __popc(bal & ((1u << (t & 31)) - 1u)), nct = 0;
-  for (int i = 0; i < kWarps; ++i) {
-    if (i < (t >> 5)) before += wcount[i];
-    nct += wcount[i];
+  int before = __popc(bal & ((1u << lane) - 1u)), nct = 0;
+  for (int k = 0; k < kWarps; ++k) {
+    if (k < w) before += wcount[k];
+    nct += wcount[k];
   }
   if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
   nct = nct < kMaxContrib ? nct : kMaxContrib;
+  if (t == 0) {
+    spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
+    spin_until_geq(fa.xready + u, fa.epoch, p.status, kStatusTimeout, p.spin_budget);
+  }
   __syncthreads();
-  if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout);
-  __syncthreads();
-  trace_mark(p, 26);
-  // sum the unit's records: S1, S2 in fp64, P in fp32. Every load of a batch of 8 records
-  // (4 float4 of P per thread, plus one S value for threads < 128) is issued before any use.
+  if (write_stats || true) trace_mark(p, 7);
+  // X^T (row j, column l), zero outside m x m: the product below reads it along l
   {
-    constexpr int kNP = 1024 / kFT;   // float4 of P per thread
-    double sacc = 0.0;
+    constexpr int kNX = 64 * 64 / kFT;   // X entries per thread, all loads issued first
+    float xv[kNX];
+#pragma unroll
+    for (int k = 0; k < kNX; ++k) {
+      const int e = t + kFT * k, l = e >> 6, j = e & 63;
+      xv[k] = 0.f;
+      if (l < m && j < m) xv[k] = ld_cg_f32_ordered(p.X + ((size_t)u * m + l) * m + j);
+    }
+#pragma unroll
+    for (int k = 0; k < kNX; ++k) {
+      const int e = t + kFT * k, l = e >> 6, j = e & 63;
+      Xt[j * kQS + l] = xv[k];
+    }
+  }
+  // sum the unit's records, each rebased from its own column shift c_k to this CTA's shift c* (the
+  // `shift` argument, with which this CTA's resident C was stored): for d_k = c_k - c*,
+  //   S1 += S1'_k + n_k d_k,  S2 += S2'_k + 2 d_k S1'_k + n_k d_k^2   (fp64),
+  //   P  += P'_k + d_k (sum_i v_i)_k^T                                 (fp32; row 63 holds sum_i v_i)
+  // so that the totals are the sums of C - c* over the unit. All loads of a batch of 4 records are
+  // issued before any use.
+  {
+    constexpr int kNP = 1024 / kFT;   // float4 of P per thread: rows (t / 16) + 32 i, columns 4 (t % 16)
+    constexpr int kB = 4;
+    double a1 = 0.0, a2 = 0.0;
     float4 pacc[kNP];
 #pragma unroll
-    for (int i = 0; i < kNP; ++i) pacc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < nct; c0 += 8) {
-      float sv[8];
-      float4 pv[8][kNP];
+    for (int k = 0; k < kNP; ++k) pacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int col4 = t & 15;
+    float cst[kNP];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+    for (int k = 0; k < kNP; ++k) cst[k] = shift[(t >> 4) + 32 * k];
+    const double cs = t < 64 ? (double)shift[t] : 0.0;
+    for (int c0 = 0; c0 < nct; c0 += kB) {
+      float s1v[kB], s2v[kB], ckv[kB], nkv[kB], ck[kB][kNP];
+      float4 pv[kB][kNP], sv[kB];
+#pragma unroll
+      for (int c = 0; c < kB; ++c) {
         const bool ok = c0 + c < nct;
         const float* r = fa.rec + (ok ? ctr[c0 + c] : 0);
-        sv[c] = (ok && t < 128) ? __ldcg(r + t) : 0.f;
+        s1v[c] = s2v[c] = ckv[c] = nkv[c] = 0.f;
+        if (ok && t < 64) {
+          s1v[c] = ld_cg_f32_ordered(r + t);
+          s2v[c] = ld_cg_f32_ordered(r + 64 + t);
+          ckv[c] = ld_cg_f32_ordered(r + kRecC + t);
+          nkv[c] = ld_cg_f32_ordered(r + kRecN);
+        }
+        sv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ok) {
+          const uint4 raw = ld_cg_v4_ordered(r + 128 + 63 * 64 + 4 * col4);
+          sv[c] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
+                              __uint_as_float(raw.w));
+        }
 #pragma unroll
-        for (int i = 0; i < kNP; ++i) {
-          pv[c][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < kNP; ++k) {
+          pv[c][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          ck[c][k] = 0.f;
           if (ok) {
-            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * i);
-            pv[c][i] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
+            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * k);
+            pv[c][k] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
                                    __uint_as_float(raw.w));
+            ck[c][k] = ld_cg_f32_ordered(r + kRecC + (t >> 4) + 32 * k);
           }
         }
       }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        sacc += (double)sv[c];
+      for (int c = 0; c < kB; ++c) {
+        const double dk = (double)ckv[c] - cs, nk = (double)nkv[c];
+        a1 += (double)s1v[c] + nk * dk;
+        a2 += (double)s2v[c] + 2.0 * dk * (double)s1v[c] + nk * dk * dk;
 #pragma unroll
-        for (int i = 0; i < kNP; ++i) {
-          pacc[i].x += pv[c][i].x;
-          pacc[i].y += pv[c][i].y;
-          pacc[i].z += pv[c][i].z;
-          pacc[i].w += pv[c][i].w;
+        for (int k = 0; k < kNP; ++k) {
+          const float d = ck[c][k] - cst[k];
+          pacc[k].x += fmaf(d, sv[c].x, pv[c][k].x);
+          pacc[k].y += fmaf(d, sv[c].y, pv[c][k].y);
+          pacc[k].z += fmaf(d, sv[c].z, pv[c][k].z);
+          pacc[k].w += fmaf(d, sv[c].w, pv[c][k].w);
         }
       }
     }
-    if (t < 64) S1d[t] = sacc;
-    else if (t < 128) S2d[t - 64] = sacc;
-    trace_mark(p, 28);
+    if (t < 64) {
+      S1d[t] = a1;
+      S2d[t] = a2;
+    }
 #pragma unroll
-    for (int i = 0; i < kNP; ++i) {
-      const int e4 = t + kFT * i;
-      *reinterpret_cast<float4*>(As + (e4 >> 4) * kQS + 4 * (e4 & 15)) = pacc[i];
+    for (int k = 0; k < kNP; ++k) {
+      const int e4 = t + kFT * k;
+      *reinterpret_cast<float4*>(As + (e4 >> 4) * kQS + 4 * (e4 & 15)) = pacc[k];
     }
   }
   __syncthreads();
+  trace_mark(p, 8);
+  // the totals are sums of C - c*: mu* = mean(C - c*) = mu - c*, and the variance does not see the shift
   if (t < 64) {
-    const double mu = S1d[t] * invN;
-    double var = S2d[t] * invN - mu * mu;
+    const double c = (double)shift[t];
+    const double mup = S1d[t] * invN;
+    double var = S2d[t] * invN - mup * mup;
     if (var < 0.0) var = 0.0;
     const double sc = 1.0 / sqrt(var + (double)p.eps);
-    mus[t] = t < m ? (float)mu : 0.f;
+    mus[t] = t < m ? (float)mup : 0.f;
     scs[t] = t < m ? (float)sc : 0.f;
     svs[t] = As[63 * kQS + t];       // landmark column 63 holds sum_i v_i
-    if (t < m) {
-      p.mu[(size_t)u * m + t] = (float)mu;
+    if (write_stats && t < m) {
+      p.mu[(size_t)u * m + t] = (float)(mup + c);
       p.s[(size_t)u * m + t] = (float)sc;
     }
   }
   __syncthreads();
-  trace_mark(p, 29);
+  // A = C~^T V from P* = (C - c*)^T V by the rank-1 fold, in place. Whitened: C~ = (C - mu) s + 1/N
+  // with C - mu = (C - c*) - mu*, so A[l][k] = s_l (P*[l][k] - mu*_l sum_i v_ik) + sum_i v_ik / N;
+  // raw: A = C^T V = P* + c* sum_i v_i^T. Zero for l >= m.
+  for (int e = t; e < 64 * 64; e += kFT) {
+    const int l = e >> 6, k = e & 63;
+    float a = 0.f;
+    if (l < m) {
+      const float P = As[l * kQS + k];
+      a = p.whiten ? scs[l] * (P - mus[l] * svs[k]) + svs[k] * invNf : P + shift[l] * svs[k];
+    }
+    As[l * kQS + k] = a;
+  }
+  __syncthreads();
+  trace_mark(p, 9);
+  // M = X A: thread (k0 = 8 (t / 64), l = t % 64) forms M[l][k0 .. k0 + 7]; the lanes of a warp share
+  // k0 (A reads are broadcasts) and take consecutive l (X^T reads and image stores are conflict free)
   {
-    // M = X A on tcgen05 in 3xTF32, as one product of the Newton-Schulz kind: stacked rows
-    // [X; A^T] times A (its bottom half, transposed), so D_top = X A. A is folded on the fly:
-    // A[l][k] = s_l (P[l][k] - mu_l sum_i v_ik) + sum_i v_ik / N. Thread (w, lane) stages row
-    // r = 32 (w % 4) + lane, columns 16 (w / 4) ..
-    const int w = t >> 5, lane = t & 31, q = w & 3, h = w >> 2, r = 32 * q + lane, i = r & 63;
-    const bool top = r < 64;
-    float v[16];
+    const int l = t & 63, k0 = 8 * (t >> 6);
+    float acc[8];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const int l = 16 * h + c;
-      if (top) {
-        v[c] = Xt[l * kQS + i];
-      } else {
-        float a = 0.f;
-        if (l < m) {
-          const float P = As[l * kQS + i];
-          a = p.whiten ? scs[l] * (P - mus[l] * svs[i]) + svs[i] * invNf : P;
-        }
-        v[c] = a;
-      }
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int j = 0; j < m; ++j) {
+      const float x = Xt[j * kQS + l];
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[j * kQS + k0]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[j * kQS + k0 + 4]);
+      acc[0] = fmaf(x, a0.x, acc[0]);
+      acc[1] = fmaf(x, a0.y, acc[1]);
+      acc[2] = fmaf(x, a0.z, acc[2]);
+      acc[3] = fmaf(x, a0.w, acc[3]);
+      acc[4] = fmaf(x, a1.x, acc[4]);
+      acc[5] = fmaf(x, a1.y, acc[5]);
+      acc[6] = fmaf(x, a1.z, acc[6]);
+      acc[7] = fmaf(x, a1.w, acc[7]);
     }
-    ns_store(sm, r, h, v);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (t == 0) ns_issue(sbase, tmem, bars + kBarComb, (m + 7) >> 3);
-    __syncwarp();
-    mbar_wait(bars + kBarComb, 0, p.status, kStatusTimeout);
-    tc_fence_after();
-    float d[16];
-    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 16 * h, d);
-    if (top) {
-      // M' = diag(s) M as bf16 (K-major B of pass 2: image row k = channel, column i = landmark,
-      // zero for i >= m); b = (1/N - s o mu)^T M, reduced over the 64 rows
-      const bool in = i < m;
-      const float sc = in ? (p.whiten ? scs[i] : 1.f) : 0.f;
-      const float wb = (in && p.whiten) ? invNf - scs[i] * mus[i] : 0.f;
-      unsigned char* mp = sm + kOffMp;
-      float bp[16];
+    // pass 2 multiplies the resident C - c*: C~ M = (C - c*) M' + 1 b^T with M' = diag(s) M and
+    // b = sum_l (1/N - s_l mu*_l) M[l] (whitened), or b = sum_l c*_l M[l] (raw, M' = M); b takes the
+    // unrounded M, so the bf16 rounding of M' enters only through the small factor C - c*
+    const bool in = l < m;
+    const float sc = in ? (p.whiten ? scs[l] : 1.f) : 0.f;
+    const float coef = in ? (p.whiten ? invNf - scs[l] * mus[l] : shift[l]) : 0.f;
+    float bp[8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        *reinterpret_cast<__nv_bfloat16*>(mp + sw128(16 * h + c, i >> 3) + ((i & 7) << 1)) =
-            __float2bfloat16_rn(sc * d[c]);
-        bp[c] = wb * d[c];
-      }
+    for (int c = 0; c < 8; ++c) {
+      *reinterpret_cast<__nv_bfloat16*>(img + sw128(k0 + c, l >> 3) + ((l & 7) << 1)) =
+          __float2bfloat16_rn(sc * acc[c]);
+      bp[c] = coef * acc[c];
+    }
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        for (int o = 16; o > 0; o >>= 1) bp[c] += __shfl_xor_sync(0xffffffffu, bp[c], o);
-      if (lane == 0) {
+    for (int c = 0; c < 8; ++c)
+      for (int o = 16; o > 0; o >>= 1) bp[c] += __shfl_xor_sync(0xffffffffu, bp[c], o);
+    if (lane == 0) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) bps[q * 64 + 16 * h + c] = bp[c];
-      }
+      for (int c = 0; c < 8; ++c) bps[w * 8 + c] = bp[c];
     }
   }
-  tc_fence_before();
   __syncthreads();
-  trace_mark(p, 30);
-  unsigned char* img = fa.mimg + (size_t)u * kImgBytes;
-  if (t < 64) {
-    float b = 0.f;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) b += bps[q * 64 + t];
-    reinterpret_cast<float*>(img + 8192)[t] = b;
-  }
-  for (int e = t; e < 512; e += kFT)
-    reinterpret_cast<uint4*>(img)[e] = reinterpret_cast<const uint4*>(sm + kOffMp)[e];
+  trace_mark(p, 20);
+  // b[k]: warps 2 (k / 8) and 2 (k / 8) + 1 hold the two halves of the landmark sum of column k
+  if (t < 64) bvec[t] = bps[(2 * (t >> 3)) * 8 + (t & 7)] + bps[(2 * (t >> 3) + 1) * 8 + (t & 7)];
   __syncthreads();
-  if (t == 0) {
-    __threadfence();
-    st_release_u64(fa.mready + u, fa.epoch);
-  }
-  trace_mark(p, 27);
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3b (row CTAs, while the unit's M' is being formed): DWC(V) of every chunk, the 3 x 3
-// depthwise taps (§关键设计 1 "ZV + DWC(V)", zero padding 1), rounded to bf16 and placed in the
-// chunk's pass-2 TMEM accumulator (columns 64 gc), on which pass 2's product then accumulates.
-// The chunk's V rows with a one-grid-row halo on each side arrive by TMA (SW128, boxes of 128
-// rows, rows outside the unit read as zero), two chunks in flight where both tiles fit. Thread t
-// owns 4 consecutive tokens of one grid row (W % 4 == 0, so a group never wraps) and 4 channels
-// (t % 16), weights in registers, and slides the 3 x 6 input window along the group. The results
-// go to a bf16 staging tile (SW128 rows, two alternating buffers), which one tcgen05 product with a
-// 64 x 64 identity (exact: every product is by 1 or 0, summed in fp32) copies into the chunk's TMEM
-// accumulator.
+// Phase 3b (row CTAs, after pass 1): DWC(V) of every chunk, the 3 x 3 depthwise taps (§关键设计 1
+// "ZV + DWC(V)", zero padding 1), rounded to bf16 and placed in the chunk's pass-2 TMEM accumulator
+// (columns 64 gc), on which pass 2's product then accumulates. Thread t owns 4 consecutive tokens of
+// one grid row (W % 4 == 0, so a group never wraps) and 4 channels (t % 16). Its 3 x 6 window of V
+// (8-byte loads through L2: pass 1 has just read these rows) is loaded one chunk ahead into a second
+// register set, so the load latency overlaps the previous chunk's arithmetic; the weights of the
+// segments' heads are staged in shared memory. The results go to a bf16 staging tile (SW128 rows,
+// two alternating buffers), which one tcgen05 product with a 64 x 64 identity (exact: every product
+// is by 1 or 0, summed in fp32) copies into the chunk's TMEM accumulator.
 // ---------------------------------------------------------------------------------------
-__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint32_t sbase, uint32_t tmem,
-                        uint64_t* bars, const CUtensorMap* tmapV) {
+__device__ __forceinline__ void dwc_load(const Params& p, const Rows& R, int gc, uint2 (&v)[3][6]) {
   const int t = threadIdx.x, W = p.W;
-  const int nbox = (kChunk + 2 * (W + 1) + kChunk - 1) / kChunk;
-  const uint32_t hbytes = (uint32_t)nbox * 16384u;
-  const int nbuf = 2 * hbytes + 16384 <= kHaloSpace ? 2 : 1;
+  const int r0 = 4 * (t >> 4), c4 = t & 15;
+  int s, lo, nrows;
+  R.chunk(gc, s, lo, nrows);
+  const int n0 = lo + r0, y = n0 / W, x0 = n0 - y * W;
+  const uint2* base = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.V) +
+                                                     (size_t)R.seg[s].u * p.N * 64) + c4;
+#pragma unroll
+  for (int a = 0; a < 3; ++a) {
+    const int yy = y + a - 1;
+    const bool rowok = r0 < nrows && yy >= 0 && yy < p.H;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) {
+      const int xx = x0 + j - 1;
+      v[a][j] = make_uint2(0u, 0u);
+      if (rowok && xx >= 0 && xx < W) v[a][j] = ld_cg_v2_ordered(base + (size_t)(yy * W + xx) * 16);
+    }
+  }
+}
+
+__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint32_t sbase, uint32_t tmem,
+                        uint64_t* bars) {
+  const int t = threadIdx.x;
   const int nch = R.nchunks;
   // staging buffers: C slot kMaxChunks - 1 (free: a CTA has at most kMaxChunks - 1 chunks, and the
-  // Q tile that slot held is consumed) and the halo region after the halo buffers
-  unsigned char* stg[2] = {sm + kOffC + (kMaxChunks - 1) * 16384, sm + kOffHb + nbuf * hbytes};
-  auto issue = [&](int gc) {
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    const int bi = gc % nbuf;
-    uint64_t* hb = bars + kBarH + bi;
-    mbar_expect_tx(hb, hbytes);
-    for (int b = 0; b < nbox; ++b)
-      tma_load_3d(sm + kOffHb + bi * hbytes + b * 16384, tmapV, 0, lo - (W + 1) + kChunk * b, R.seg[s].u, hb);
-  };
+  // Q tile that slot held is consumed) and kOffStg1
+  unsigned char* stg[2] = {sm + kOffC + (kMaxChunks - 1) * 16384, sm + kOffStg1};
+  float* wsm = reinterpret_cast<float*>(sm + kOffDw);   // [segment][tap][channel]
   // staged chunk gc -> its TMEM accumulator (columns 64 gc): D = S I over K = 64 channels, the
-  // identity (K-major B) in the M' area, which pass 2 fills only later
+  // identity (K-major B) in the M' area, which the combine fills only later
   auto transfer = [&](int gc) {
     tc_fence_after();
     const uint32_t id = idesc(1, 128, 64, 0, 0);
@@ -1038,10 +1195,23 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint3
   auto wait_transfer = [&](int gc) {
     mbar_wait(bars + kBarDw + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
   };
-  __syncthreads();   // pass 1 is done with the V stages, Q and L (the halo region), and with TMEM
-  if (t == 0) {
-    issue(0);
-    if (nbuf == 2 && nch > 1) issue(1);
+  __syncthreads();   // pass 1 is done with the V stages, Q and L, and with TMEM columns 0..127
+  // the weights of each segment's head, fp32 [tap][channel]
+  {
+    constexpr int kNW = (2 * 9 * 64 + kFT - 1) / kFT;   // weights per thread, all loads issued first
+    float wv[kNW];
+#pragma unroll
+    for (int k = 0; k < kNW; ++k) {
+      const int e = t + kFT * k;
+      wv[k] = 0.f;
+      if (e < R.nseg * 9 * 64) {
+        const int sg = e / (9 * 64), rem = e - sg * 9 * 64, tap = rem >> 6, ch = rem & 63;
+        wv[k] = ld_cg_f32_ordered(p.dwc + ((size_t)(R.seg[sg].u % p.heads) * 64 + ch) * 9 + tap);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kNW; ++k)
+      if (t + kFT * k < 2 * 9 * 64) wsm[t + kFT * k] = wv[k];
   }
   // the 64 x 64 bf16 identity, SW128 rows (row n, column k): 512 16-byte groups
   for (int e = t; e < 512; e += kFT) {
@@ -1057,53 +1227,38 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint3
     }
     *reinterpret_cast<uint4*>(sm + kOffMp + sw128(n, c8)) = v;
   }
-  const int grp = t >> 4, c4 = t & 15;   // tokens 4 grp .. 4 grp + 3 of the chunk, channels 4 c4 ..
-  float wt[9][4];
-  int head = -1;
-  for (int gc = 0; gc < nch; ++gc) {
+  __syncthreads();
+  trace_mark(p, 23);
+  const int r0 = 4 * (t >> 4), c4 = t & 15;
+  auto compute = [&](int gc, const uint2 (&v)[3][6]) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    const int u = R.seg[s].u;
-    if (u % p.heads != head) {
-      head = u % p.heads;
-#pragma unroll
-      for (int tap = 0; tap < 9; ++tap)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) wt[tap][e] = __ldg(p.dwc + ((size_t)head * 64 + 4 * c4 + e) * 9 + tap);
-    }
-    const int bi = gc % nbuf;
-    mbar_wait(bars + kBarH + bi, (gc / nbuf) & 1, p.status, kStatusTimeout);   // fill gc / nbuf of buffer bi
-    const int r0 = 4 * grp;                // chunk row of the group's first token
+    const float* wv = wsm + s * 9 * 64 + 4 * c4;
     float acc[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
-    if (r0 < nrows) {
-      const int n0 = lo + r0, x0 = n0 % W;
-      const unsigned char* hbuf = sm + kOffHb + bi * hbytes;
 #pragma unroll
-      for (int a = 0; a < 3; ++a) {
-        // tile rows of tokens x0 - 1 .. x0 + 4 on grid row y + a - 1: r0 + a W + j, j = 0..5
-        float v[6][4];
+    for (int a = 0; a < 3; ++a) {
+      float x[6][4];
 #pragma unroll
-        for (int j = 0; j < 6; ++j) {
-          const int tr = r0 + a * W + j;
-          const bool inside = (j > 0 || x0 > 0) && (j < 5 || x0 + 4 < W);
-          uint2 raw = make_uint2(0u, 0u);
-          if (inside)
-            raw = *reinterpret_cast<const uint2*>(hbuf + tr * 128 + ((((c4 >> 1) ^ (tr & 7))) << 4) + (c4 & 1) * 8);
-          v[j][0] = bf_lo(raw.x);
-          v[j][1] = bf_hi(raw.x);
-          v[j][2] = bf_lo(raw.y);
-          v[j][3] = bf_hi(raw.y);
+      for (int j = 0; j < 6; ++j) {
+        x[j][0] = bf_lo(v[a][j].x);
+        x[j][1] = bf_hi(v[a][j].x);
+        x[j][2] = bf_lo(v[a][j].y);
+        x[j][3] = bf_hi(v[a][j].y);
+      }
+#pragma unroll
+      for (int b = 0; b < 3; ++b) {
+        const float4 wt = *reinterpret_cast<const float4*>(wv + (a * 3 + b) * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i][0] = fmaf(wt.x, x[i + b][0], acc[i][0]);
+          acc[i][1] = fmaf(wt.y, x[i + b][1], acc[i][1]);
+          acc[i][2] = fmaf(wt.z, x[i + b][2], acc[i][2]);
+          acc[i][3] = fmaf(wt.w, x[i + b][3], acc[i][3]);
         }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int b = 0; b < 3; ++b)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(wt[a * 3 + b][e], v[i + b][e], acc[i][e]);
       }
     }
     // rows past the chunk's end stage zeros (their accumulator rows are never stored); staging
@@ -1115,11 +1270,21 @@ __device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint3
       *reinterpret_cast<uint2*>(st + sw128(r0 + i, c4 >> 1) + (c4 & 1) * 8) =
           make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
     fence_async_smem();
-    __syncthreads();   // staging gc written (and, at gc = 0, the identity), halo buffer bi read
-    // two issuing threads in different warps, so that neither warp's chunk is late by both
+    __syncthreads();   // staging gc written
     if (t == 0) transfer(gc);
-    if (t == 32 && gc + nbuf < nch) issue(gc + nbuf);
+    if (gc == 0) trace_mark(p, 26);
+  };
+  uint2 va[3][6], vb[3][6];
+  if (nch > 0) dwc_load(p, R, 0, va);
+  for (int gc = 0; gc < nch; gc += 2) {
+    if (gc + 1 < nch) dwc_load(p, R, gc + 1, vb);
+    compute(gc, va);
+    if (gc + 1 < nch) {
+      if (gc + 2 < nch) dwc_load(p, R, gc + 2, va);
+      compute(gc + 1, vb);
+    }
   }
+  trace_mark(p, 27);
   // the last transfers (earlier ones were waited before their buffer was reused)
   if (nch >= 2) wait_transfer(nch - 2);
   if (nch >= 1) wait_transfer(nch - 1);
@@ -1143,17 +1308,12 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
-  auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffV; };
-  if (t == 0)
-    for (int s = 0; s < R.nseg; ++s) spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout);
-  __syncthreads();
+  auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffImg1; };
+  // each segment's M'^T image and b, formed by this CTA's own combine
+  for (int s = 0; s < R.nseg; ++s)
+    row_combine(p, fa, sm, R.seg[s].u, reinterpret_cast<const float*>(sm + kOffSh) + 64 * s, sm + img_off(s),
+                bvec + 64 * s, R.seg[s].lo == 0);
   trace_mark(p, 4);
-  for (int s = 0; s < R.nseg; ++s) {
-    const unsigned char* img = fa.mimg + (size_t)R.seg[s].u * kImgBytes;
-    for (int e = t; e < 512; e += kFT)
-      reinterpret_cast<uint4*>(sm + img_off(s))[e] = __ldcg(reinterpret_cast<const uint4*>(img) + e);
-    if (t < 64) bvec[64 * s + t] = __ldcg(reinterpret_cast<const float*>(img + 8192) + t);
-  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -1236,7 +1396,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   const Rows& R = *Rsm;
   const bool solver = g < U;
   if (t == 0) {
-    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, b == kBarDrain ? 2 : 1);
     mbar_init_fence();
     if (g == 0) *p.status = 0;
     if (!solver) pass1_prefetch(R, sm, bars, &tmapV, &tmapQ);
@@ -1287,31 +1447,41 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
         *reinterpret_cast<float4*>(dst) = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
         *reinterpret_cast<float4*>(dst + 4) = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
       }
+      // one landmark of unit u is out: the unit's consumers wait for m of them (no grid barrier)
+      __syncwarp();
+      if (lane == 0) {
+        __threadfence();
+        red_release_add_u64(fa.lready + u, 1ull);
+      }
     }
   }
-  __syncthreads();
   trace_mark(p, 1);
-  if (t == 0) {
-    __threadfence();
-    red_release_add_u64(fa.gbar, 1ull);
-  }
-  if (t == 0) spin_until_geq(fa.gbar, fa.epoch * (unsigned long long)gridDim.x, p.status, kStatusTimeout);
-  __syncthreads();
-  trace_mark(p, 2);
+  __syncthreads();   // the TMEM address, the mbarrier initialisation and the row plan are visible
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // solver CTAs take no rows (R.nchunks == 0): solve, combine, then the diagnostics
+  // solver CTAs take no rows (R.nchunks == 0): the unit's chain, then its diagnostics; the row
+  // CTAs of the unit pick up X for their own combine
   if (solver) {
+    if (t == 0) spin_until_geq(fa.lready + g, fa.epoch * (unsigned long long)m + (p.spin_test ? 1 : 0), p.status,
+                               kStatusTimeout, p.spin_budget);
+    __syncthreads();
+    trace_mark(p, 2);
     const SolverInfo si = solver_cta(p, fa, sm, sbase, tmem, bars, g);
     trace_mark(p, 3);
-    solver_combine(p, fa, sm, sbase, tmem, bars, g);
     solver_diagnostics(p, sm, sbase, tmem, bars, g, si);
   }
-  if (R.nchunks > 0) pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
-  if (!solver) trace_mark(p, 3);
-  if (R.nchunks > 0) dwc_all(p, R, sm, sbase, tmem, bars, &tmapV);
-  if (R.nchunks > 0) pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
+  if (R.nchunks > 0) {
+    pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
+    trace_mark(p, 3);
+    dwc_all(p, R, sm, sbase, tmem, bars);
+    pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
+  }
+  // drain: the tcgen05 operations of both issuing threads (thread 0: solver, pass-1 and DWC products;
+  // the first thread of the last warp: pass-2 products) have completed before TMEM is released. In a
+  // normal run each was waited already; after an expired wait this bounds the wait for any still running.
+  if (t == 0 || t == kFT - 32) mma_commit(bars + kBarDrain);
+  if (t == 0) mbar_wait(bars + kBarDrain, 0, p.status, kStatusTimeout);
   __syncthreads();
   trace_mark(p, 15);
   trace_clock(p, 14);
@@ -1323,13 +1493,13 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
 
 }  // namespace
 
-// Flag area: grid barrier (256 B), then three [U] flag arrays (cnt, xready, mready), each padded
-// to 256 B; then the per-CTA records and the per-unit M' images.
+// Flag area: three [U] flag arrays (lready, cnt, xready), each padded to 256 B; then the per-CTA
+// pass-1 records.
 static size_t flag_stride(int U) { return 256 * (size_t)((U * 8 + 255) / 256); }
-static size_t flag_bytes(int U) { return 256 + 3 * flag_stride(U); }
+static size_t flag_bytes(int U) { return 3 * flag_stride(U); }
 
 size_t fused_workspace_bytes(int U) {
-  return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * kImgBytes;
+  return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
 }
 
 // Decide whether the fused kernel serves this shape on the current device; returns the grid size
@@ -1351,9 +1521,6 @@ int fused_grid(const Params& p) {
   if (cpc > kMaxChunks - 1 || cpc > nchu) return 0;   // one C slot stays free for the Q chunk
   // the DWC phase's token groups of 4 stay on one grid row
   if (p.W % 4 != 0) return 0;
-  // its V halo tile (a chunk plus one grid row on each side, in boxes of 128 rows) and one DWC
-  // staging tile must fit the halo region
-  if ((long long)((kChunk + 2 * (p.W + 1) + kChunk - 1) / kChunk) * 16384 + 16384 > (long long)kHaloSpace) return 0;
   // replay the row partition: contributors of every unit must fit the offset table
   {
     int worst = 0, cur_u = -1, cur = 0;
@@ -1465,13 +1632,11 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   if (!tmap_for(p.O, p.N, p.U, 32, true, &tmapo)) return cudaErrorInvalidValue;
   FusedArgs fa;
   fa.epoch = epoch;
-  fa.gbar = reinterpret_cast<unsigned long long*>(fused_ws);
   const size_t fs = flag_stride(p.U);
-  fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + 256);
-  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + fs);
-  fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 256 + 2 * fs);
+  fa.lready = reinterpret_cast<unsigned long long*>(fused_ws);
+  fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + fs);
+  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 2 * fs);
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
-  fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
   plan_pass1_warps(p.m, fa);
   Params pp = p;
   void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo};

@@ -1081,6 +1081,59 @@ cudaError_t launch_pool(const Params& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Condition number estimate of W + eps I for lfa_get_info (not part of the forward): ||X_T||_2 by
+// power iteration on X_T, which approximates (W + eps I)^-1 (symmetric positive definite) once the
+// Newton-Schulz chain has converged, times the forward's lambda_max = ||W||_2, i.e. lambda_max /
+// lambda_min. One CTA of 256 threads per unit, a warp per matrix row, kKappaIters normalised steps
+// from the ones vector and a final Rayleigh quotient.
+constexpr int kKappaIters = 48;
+__global__ void __launch_bounds__(kThreads) k_kappa(Params p) {
+  __shared__ float v[2][kMaxM];
+  __shared__ float red[2 * (kThreads / 32)];
+  const int u = blockIdx.x, t = threadIdx.x, w = t >> 5, lane = t & 31, m = p.m;
+  const float* X = p.X + (size_t)u * m * m;
+  for (int i = t; i < kMaxM; i += kThreads) v[0][i] = i < m ? rsqrtf((float)m) : 0.f;
+  __syncthreads();
+  float rq = 0.f;
+  for (int it = 0; it <= kKappaIters; ++it) {
+    const float* vin = v[it & 1];
+    float* vout = v[(it + 1) & 1];
+    float num = 0.f, den = 0.f;
+    for (int i = w; i < m; i += kThreads / 32) {
+      float s = 0.f;
+      for (int j = lane; j < m; j += 32) s = fmaf(X[(size_t)i * m + j], vin[j], s);
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) vout[i] = s;
+      num = fmaf(s, vin[i], num);   // lane-uniform: every lane adds the same terms
+      den = fmaf(s, s, den);
+    }
+    if (lane == 0) {
+      red[w] = num;
+      red[kThreads / 32 + w] = den;
+    }
+    __syncthreads();
+    float nsum = 0.f, dsum = 0.f;
+    for (int k = 0; k < kThreads / 32; ++k) {
+      nsum += red[k];
+      dsum += red[kThreads / 32 + k];
+    }
+    rq = nsum;   // v^T X v with ||v|| = 1
+    const float sc = dsum > 0.f ? rsqrtf(dsum) : 0.f;
+    __syncthreads();
+    for (int i = t; i < m; i += kThreads) vout[i] *= sc;
+    __syncthreads();
+  }
+  if (t == 0) {
+    float* inf = p.info + (size_t)u * kInfoStride;
+    inf[kInfoKappa] = inf[kInfoLambdaMax] * rq;
+  }
+}
+
+cudaError_t launch_kappa(const Params& p, cudaStream_t st) {
+  k_kappa<<<p.U, kThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_cross_kernel(const Params& p, int unit, float* C_out, cudaStream_t st) {
   const size_t smem = generic_smem_pass2(p.m, p.d);
   if (p.dtype == LFA_BF16)

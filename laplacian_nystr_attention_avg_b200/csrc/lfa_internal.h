@@ -15,13 +15,16 @@ constexpr int kRowTile = 64;      // token rows per tile in the generic kernels
 constexpr int kThreads = 256;     // threads per CTA in the generic kernels
 constexpr int kSmallM = 64;       // m <= kSmallM: one CTA solves a unit's Newton-Schulz chain
 
+// default bound (SM clock cycles, about 1 s) on the fused kernel's waits for flags of other CTAs
+constexpr long long kFlagSpinBudget = 1ll << 31;
+
 // status-word bits (device side); lfa_get_info maps them to lfa_status
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusNonFinite = 2;
 
 // per-unit diagnostics slots (floats) in the workspace
-constexpr int kInfoAlpha = 0, kInfoLambdaMax = 1, kInfoFallback = 2, kInfoResidual = 3;
-constexpr int kInfoStride = 4;
+constexpr int kInfoAlpha = 0, kInfoLambdaMax = 1, kInfoFallback = 2, kInfoResidual = 3, kInfoKappa = 4;
+constexpr int kInfoStride = 5;
 
 __host__ __device__ inline int round_up(int a, int b) { return (a + b - 1) / b * b; }
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -74,6 +77,14 @@ struct Params {
   void* ev_end;
   // optional per-CTA phase timestamps (%globaltimer, ns) of the fused kernel: [grid][16]
   unsigned long long* trace;
+  // optional copy of the cross kernel C of unit dbg_unit as computed by this forward, fp32 [N][m]
+  float* dbgC;
+  float* dbgS;   // optional: the column shift subtracted before bf16 rounding, per entry, fp32 [N][m]
+  int dbg_unit;
+  // fused kernel: bound (SM cycles) on its waits for flags that other CTAs set; with spin_test the
+  // landmark waits look for one landmark more than exist, so every one of them runs out (tests)
+  long long spin_budget;
+  int spin_test;
 };
 
 // Backward-pass tensors and workspace views (with the forward's Params).
@@ -134,6 +145,7 @@ cudaError_t backward_set_attributes();
 int backward_launch_count(const Params& p);
 cudaError_t launch_pool(const Params& p, cudaStream_t st);
 cudaError_t launch_cross_kernel(const Params& p, int unit, float* C_out, cudaStream_t st);
+cudaError_t launch_kappa(const Params& p, cudaStream_t st);
 size_t generic_smem_pass1(int m, int d);
 size_t generic_smem_pass2(int m, int d);
 cudaError_t generic_set_attributes();

@@ -203,6 +203,19 @@ __device__ __forceinline__ uint4 ld_cg_v4_ordered(const void* p) {
   return v;
 }
 
+// 8-byte global load through L2, kept in program order with the other asm statements (issued where
+// it stands, so a prefetch one step ahead really overlaps that step)
+__device__ __forceinline__ uint2 ld_cg_v2_ordered(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float ld_cg_f32_ordered(const void* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
+}
+
 // ---- global-memory flags (acquire/release at gpu scope) ------------------------------------
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
   unsigned long long v;
@@ -215,14 +228,15 @@ __device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsig
 __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
-// Bounded spin until *p >= target; returns false (and sets the status bit) on expiry.
+// Bounded spin until *p >= target; returns false (and sets the status bit) on expiry, after `budget`
+// SM clock cycles (kSpinBudget unless a test asks for less).
 __device__ __forceinline__ bool spin_until_geq(const unsigned long long* p, unsigned long long target,
-                                               int* status, int status_bit) {
+                                               int* status, int status_bit, long long budget = kSpinBudget) {
   if (ld_acquire_u64(p) >= target) return true;
   const long long t0 = clock64();
   while (ld_acquire_u64(p) < target) {
     __nanosleep(64);
-    if (clock64() - t0 > kSpinBudget) {
+    if (clock64() - t0 > budget) {
       atomicOr(status, status_bit);
       return false;
     }

@@ -154,3 +154,21 @@ def crop_grid(x: torch.Tensor, H: int, W: int, h: int, w: int) -> torch.Tensor:
     B, nh, N, d = x.shape
     assert N == H * W
     return x.reshape(B, nh, H, W, d)[:, :, :h, :w, :].reshape(B, nh, h * w, d).contiguous()
+
+
+def make_crop_inputs(wl: Workload, h: int, w: int, r: int, seed: int = 0, name: Optional[str] = None):
+    """A workload's own inputs cut down to the top-left h x w tokens of every (batch, head) grid.
+
+    Draws the full workload's tensors with ``make_inputs`` (so the values are the workload's own,
+    not a fresh draw), crops Q, V and dO with ``crop_grid`` and keeps the DWC weight. Returns the
+    crop's Workload (same B, heads, d, lambda, eps, T, dtype; grid h x w; pooling window r) and
+    its Inputs.
+    """
+    full = make_inputs(wl, seed=seed, with_dO=True)
+    cw = wl.replace(name=name or f"{wl.name}_crop{h}x{w}_r{r}", H=h, W=w, r=r, backward=True)
+
+    def crop(t):
+        return crop_grid(t, wl.H, wl.W, h, w)
+
+    return cw, Inputs(wl=cw, Q=crop(full.Q), V=crop(full.V), dwc=full.dwc, dO=crop(full.dO),
+                      Q_store=crop(full.Q_store), V_store=crop(full.V_store), dO_store=crop(full.dO_store))

@@ -34,7 +34,8 @@ class Config(ctypes.Structure):
 
 class UnitInfo(ctypes.Structure):
     _fields_ = [("alpha_fallback", ctypes.c_int), ("alpha", ctypes.c_float),
-                ("lambda_max", ctypes.c_float), ("ns_residual_fro", ctypes.c_float)]
+                ("lambda_max", ctypes.c_float), ("ns_residual_fro", ctypes.c_float),
+                ("kappa", ctypes.c_float)]
 
 
 class LfaError(RuntimeError):
@@ -60,6 +61,8 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_destroy": (ci, [vp]),
         "lfa_status_string": (ctypes.c_char_p, [ci]),
         "lfa_debug_cross_kernel": (ci, [vp, vp, ci, vp, vp]),
+        "lfa_debug_capture_cross": (ci, [vp, ci, vp, vp]),
+        "lfa_debug_spin_test": (ci, [vp, ctypes.c_longlong]),
         "lfa_debug_context": (ci, [vp, ci, vp, vp, vp, vp, vp]),
         "lfa_forward_path": (ctypes.c_char_p, [vp]),
         "lfa_set_profile_events": (ci, [vp, vp, vp]),
@@ -146,9 +149,40 @@ def forward_noalloc(cfg: Config, dwc_weight: torch.Tensor, Q: torch.Tensor, V: t
     dwc_weight: device float32 [heads, d, 3, 3]; Q, V, O: device [B, heads, N, d] in the
     config's dtype. Raises LfaError (LFA_ERR_SCRATCH_LIMIT) when the config does not fit.
     """
+    shape, dt = _cfg_shape(cfg), _cfg_dtype(cfg)
+    _require(Q, "Q", shape, dt)
+    _require(V, "V", shape, dt, Q.device)
+    _require(O, "O", shape, dt, Q.device)
+    _require(dwc_weight, "dwc_weight", (cfg.heads, cfg.d, 3, 3), torch.float32, Q.device)
     _check(load().lfa_forward_noalloc(ctypes.byref(cfg), _ptr(dwc_weight), _ptr(Q), _ptr(V), _ptr(O),
                                       _stream(stream)), "lfa_forward_noalloc")
     return O
+
+
+def _require(t: torch.Tensor, name: str, shape, dtype, device=None, host: bool = False) -> None:
+    """Reject a tensor the library would read or write out of bounds: wrong dtype, shape, layout or
+    device. (The library sees only a pointer, so these checks live in the binding.)"""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if host:
+        if t.device.type != "cpu":
+            raise ValueError(f"{name}: expected a host tensor")
+    elif t.device.type != "cuda" or (device is not None and t.device != device):
+        raise ValueError(f"{name}: on {t.device}, expected {device if device is not None else 'a CUDA device'}")
+
+
+def _cfg_shape(cfg: Config):
+    return (cfg.B, cfg.heads, cfg.H * cfg.W, cfg.d)
+
+
+def _cfg_dtype(cfg: Config):
+    return torch.bfloat16 if cfg.dtype == LFA_BF16 else torch.float32
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -172,12 +206,15 @@ class LaplacianNystromAttention:
         self.lib = load()
         self.cfg = cfg
         self.device = torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
         self.dtype = torch.bfloat16 if cfg.dtype == LFA_BF16 else torch.float32
         self.units = cfg.B * cfg.heads
         self.N = cfg.H * cfg.W
         self.m = (cfg.H // cfg.r) * (cfg.W // cfg.r)
         self.shape = (cfg.B, cfg.heads, self.N, cfg.d)
         self.weight = dwc_weight.to(self.device, torch.float32).contiguous()
+        _require(self.weight, "dwc_weight", (cfg.heads, cfg.d, 3, 3), torch.float32, self.device)
         nbytes = workspace_size(cfg)
         if nbytes == 0:
             raise LfaError(LFA_ERR_INVALID_ARG, "lfa_workspace_size")
@@ -223,10 +260,16 @@ class LaplacianNystromAttention:
                 stream=None) -> torch.Tensor:
         if O is None:
             O = self.new_output()
+        for name, t in (("Q", Q), ("V", V), ("O", O)):
+            _require(t, name, self.shape, self.dtype, self.device)
         _check(self.lib.lfa_forward(self.handle, _ptr(Q), _ptr(V), _ptr(O), _stream(stream)), "lfa_forward")
         return O
 
     def forward_host(self, Q_host, V_host, O_host, Q_dev, V_dev, O_dev, stream=None) -> None:
+        for name, t in (("Q_host", Q_host), ("V_host", V_host), ("O_host", O_host)):
+            _require(t, name, self.shape, self.dtype, host=True)
+        for name, t in (("Q_dev", Q_dev), ("V_dev", V_dev), ("O_dev", O_dev)):
+            _require(t, name, self.shape, self.dtype, self.device)
         _check(self.lib.lfa_forward_host(self.handle, _ptr(Q_host), _ptr(V_host), _ptr(O_host), _ptr(Q_dev),
                                          _ptr(V_dev), _ptr(O_dev), _stream(stream)), "lfa_forward_host")
 
@@ -235,6 +278,8 @@ class LaplacianNystromAttention:
             dQ = self.new_output()
         if dV is None:
             dV = self.new_output()
+        for name, t in (("Q", Q), ("V", V), ("dO", dO), ("dQ", dQ), ("dV", dV)):
+            _require(t, name, self.shape, self.dtype, self.device)
         _check(self.lib.lfa_backward(self.handle, _ptr(Q), _ptr(V), _ptr(dO), _ptr(dQ), _ptr(dV),
                                      _stream(stream)), "lfa_backward")
         return dQ, dV
@@ -252,6 +297,21 @@ class LaplacianNystromAttention:
         _check(self.lib.lfa_debug_cross_kernel(self.handle, _ptr(Q), int(unit), _ptr(C), _stream(stream)),
                "lfa_debug_cross_kernel")
         return C
+
+    def capture_cross(self, Q: torch.Tensor, V: torch.Tensor, unit: int, O: Optional[torch.Tensor] = None,
+                      stream=None):
+        """(C, shift) of `unit` as one forward computes it (lfa_debug_capture_cross + lfa_forward), each
+        fp32 [N, m]: the C that pass 2 uses and the column shift subtracted before its bf16 rounding."""
+        C = torch.empty((self.N, self.m), dtype=torch.float32, device=self.device)
+        S = torch.empty((self.N, self.m), dtype=torch.float32, device=self.device)
+        _check(self.lib.lfa_debug_capture_cross(self.handle, int(unit), _ptr(C), _ptr(S)),
+               "lfa_debug_capture_cross")
+        self.forward(Q, V, O, stream)
+        return C, S
+
+    def arm_spin_test(self, budget_cycles: int) -> None:
+        """lfa_debug_spin_test: the next forward's cross-block waits run out after budget_cycles."""
+        _check(self.lib.lfa_debug_spin_test(self.handle, int(budget_cycles)), "lfa_debug_spin_test")
 
     def context(self, unit: int, stream=None):
         d = self.cfg.d

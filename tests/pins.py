@@ -377,6 +377,11 @@ def _fd_case(H, W, d, r, lam, eps, T, seed, whiten, n_samples=40, h=1e-6):
     v = rng.standard_normal((H * W, d))
     w = rng.standard_normal((d, 3, 3)) * 0.1
     dO = rng.standard_normal((H * W, d))
+    return _fd_check(q, v, w, dO, H, W, r, lam, eps, T, whiten, rng, n_samples, n_samples // 2, h)
+
+
+def _fd_check(q, v, w, dO, H, W, r, lam, eps, T, whiten, rng, n_q, n_v, h=1e-6):
+    """Worst |central difference - analytic| / max|analytic| over sampled Q and V coordinates."""
     dQ, dV, f = O.unit_backward(q, v, w, dO, H, W, r, lam, eps, T, whiten)
 
     def loss(qq, vv):
@@ -387,6 +392,7 @@ def _fd_case(H, W, d, r, lam, eps, T, seed, whiten, n_samples=40, h=1e-6):
         # above the rounding floor of the loss when the attention part is small
         return float(np.sum(dO * O.unit_forward(qq, v, w, H, W, r, lam, eps, T, whiten).O_attn))
 
+    d = q.shape[1]
     L = f.L
     pooled_dist = np.abs(L[:, None, :] - L[None, :, :])
     off = ~np.eye(len(L), dtype=bool)
@@ -405,18 +411,40 @@ def _fd_case(H, W, d, r, lam, eps, T, seed, whiten, n_samples=40, h=1e-6):
         fd = (loss_attn(qp) - loss_attn(qm)) / (2 * h)
         worst_q = max(worst_q, abs(fd - dQ[i, k]) / scale_q)
         checked += 1
-        if checked >= n_samples:
+        if checked >= n_q:
             break
-    assert checked >= n_samples // 2, "too few kink-free coordinates"
+    assert checked >= n_q // 2, "too few kink-free coordinates"
     worst_v = 0.0
     scale_v = np.abs(dV).max()
-    for idx in rng.choice(H * W * d, size=n_samples // 2, replace=False):
+    for idx in rng.choice(H * W * d, size=n_v, replace=False):
         i, k = divmod(int(idx), d)
         vp = v.copy(); vp[i, k] += h
         vm = v.copy(); vm[i, k] -= h
         fd = (loss(q, vp) - loss(q, vm)) / (2 * h)
         worst_v = max(worst_v, abs(fd - dV[i, k]) / scale_v)
     return worst_q, worst_v
+
+
+def check_backward_fd_long_crop(n_per_head=64, heads=None):
+    """The long-sequence workload's own Q, V, dO and DWC weight, cropped to the top-left 16 x 16
+    tokens of every head's 256 x 256 grid (bf16-rounded values, as the library consumes them), at
+    the literal pooling window r = 16 (one landmark) and at r = 4 (16 landmarks, so that the
+    Newton-Schulz chain is not trivial). Central differences in float64 against the analytic
+    gradient, 64 Q and 64 V coordinates per head."""
+    from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, make_crop_inputs
+
+    wl = WORKLOADS["long"]
+    for r in (16, 4):
+        cw, x = make_crop_inputs(wl, 16, 16, r)
+        for hh in (range(cw.heads) if heads is None else heads):
+            q = x.Q[0, hh].double().numpy()
+            v = x.V[0, hh].double().numpy()
+            w = x.dwc[hh].double().numpy()
+            dO = x.dO[0, hh].double().numpy()
+            wq, wv = _fd_check(q, v, w, dO, cw.H, cw.W, r, cw.lam, cw.eps, cw.T, True,
+                               _rng(1000 + 16 * r + hh), n_per_head, n_per_head)
+            assert wq < 1e-6, f"dQ vs finite differences: {wq} (long crop, r={r}, head {hh})"
+            assert wv < 1e-6, f"dV vs finite differences: {wv} (long crop, r={r}, head {hh})"
 
 
 def check_backward_fd(cases=None):
@@ -526,5 +554,5 @@ ALL_PINS = [
     check_dwc_taps, check_backward_fd, check_injectivity_generic,
     check_batch_stats_single_batch, check_batch_stats_replicated, check_batch_stats_vs_sklearn,
     check_reading_b_vs_dense, check_reading_b_r1_is_whitened_kernel, check_cg_vs_solve,
-    check_cg_error_bound, check_backward_batch_stats_fd,
+    check_cg_error_bound, check_backward_batch_stats_fd, check_backward_fd_long_crop,
 ]

@@ -11,15 +11,16 @@ import pytest
 import torch
 
 from laplacian_nystr_attention_avg_b200 import lfa
-from laplacian_nystr_attention_avg_b200.inputs import Workload, make_inputs
+from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, Workload, make_crop_inputs, make_inputs
 from oracle import lfa_oracle as O
 from tests import parity_util as pu
 
 pytestmark = pytest.mark.gpu
 
 
-def _check_backward(wl: Workload, whiten: bool, units, zero_dwc: bool = False, seed: int = 0):
-    x = make_inputs(wl, seed=seed, with_dO=True)
+def _check_backward(wl: Workload, whiten: bool, units, zero_dwc: bool = False, seed: int = 0, x=None):
+    if x is None:
+        x = make_inputs(wl, seed=seed, with_dO=True)
     w = torch.zeros_like(x.dwc) if zero_dwc else x.dwc
     mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, whiten), w, "cuda")
     Q, V, dO = x.Q_store.cuda(), x.V_store.cuda(), x.dO_store.cuda()
@@ -57,6 +58,16 @@ CROPS = [
 @pytest.mark.parametrize("whiten", [True, False], ids=["whiten", "raw"])
 def test_backward_small(wl, whiten):
     _check_backward(wl, whiten, tuple(range(wl.units)))
+
+
+@pytest.mark.parametrize("r", [16, 4])
+@pytest.mark.parametrize("whiten", [True, False], ids=["whiten", "raw"])
+def test_backward_long_crop(r, whiten):
+    # the long-sequence workload's own Q, V, dO (bf16) and DWC weight, cropped to the top-left
+    # 16 x 16 tokens of all 8 heads' grids: r = 16 (one landmark) and r = 4 (16 landmarks); the
+    # oracle's gradient on these same values is pinned by finite differences
+    cw, x = make_crop_inputs(WORKLOADS["long"], 16, 16, r)
+    _check_backward(cw, whiten, tuple(range(cw.units)), x=x)
 
 
 @pytest.mark.parametrize("whiten", [True, False], ids=["whiten", "raw"])

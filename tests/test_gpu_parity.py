@@ -82,7 +82,13 @@ def test_newton_schulz_context(name):
         assert errX <= 33 * u_eff * kappa + 1e-5, f"{name} unit {u}: X error {errX:.2e} (kappa {kappa:.0f})"
         assert abs(info[u].lambda_max - f.alpha.norm2) <= 1e-4 * f.alpha.norm2
         assert info[u].alpha_fallback == int(f.alpha.fallback) == 1
-        assert info[u].ns_residual_fro < 5e-2   # fp32 floor of the computed residual itself
+        # ||I - W X_gpu||_F, computed on the device, against a bound from its parts: the oracle's own
+        # residual after T steps, the distance of X_gpu from the oracle's X (times ||W||_F), and the
+        # rounding of the device product W X_gpu (at most m u_eff ||W||_F ||X_gpu||_F per side)
+        Wn, Xn = np.linalg.norm(f.W), np.linalg.norm(X)
+        res_o = np.linalg.norm(np.eye(wl.m) - f.W @ f.X)
+        bound = res_o + Wn * np.linalg.norm(X - f.X) + 2 * wl.m * u_eff * Wn * Xn
+        assert info[u].ns_residual_fro <= bound, f"{name} unit {u}: residual {info[u].ns_residual_fro:.2e} > {bound:.2e}"
         np.testing.assert_allclose(mu, f.mu, rtol=1e-4)
         np.testing.assert_allclose(s, 1.0 / np.sqrt(f.var + wl.eps), rtol=1e-4)
 
