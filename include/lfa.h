@@ -251,7 +251,7 @@ int lfa_fused_grid(lfa_handle h);
 int lfa_launches_per_forward(lfa_handle h);
 
 /* Name of the forward implementation chosen for this handle's config, static string:
- * "fused" (one cooperative kernel: bf16, d = 64, m <= 63, W % 4 == 0, B*heads <= SMs/2, rows
+ * "fused" (one cooperative kernel: bf16, d = 64, m <= 56, W % 4 == 0, B*heads <= SMs/2, rows
  * per CTA within its on-chip C capacity) or "generic" (every other accepted shape). Setting the
  * environment variable LFA_FORWARD_PATH=generic before lfa_create forces the generic path. */
 const char* lfa_forward_path(lfa_handle h);

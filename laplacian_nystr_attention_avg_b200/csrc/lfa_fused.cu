@@ -49,10 +49,12 @@ constexpr int kChunk = 128;               // token rows per chunk
 constexpr int kMaxChunks = 8;             // resident C chunks per CTA
 constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q, L and halo tiles
 // floats per partial record: S1'[64], S2'[64], P'[64][64] (sums of the shifted C - c), c[64], the
-// segment's row count n, padding to a multiple of 64
-constexpr int kRec = 128 + 64 * 64 + 128;
+// segment's row count n (padded to 64 floats), and the pass-2 bias b[64] for this record's shift,
+// which the unit's solver CTA fills in
+constexpr int kRec = 128 + 64 * 64 + 128 + 64;
 constexpr int kRecC = 128 + 64 * 64;      // offset of c
 constexpr int kRecN = kRecC + 64;         // offset of n
+constexpr int kRecB = kRecN + 64;         // offset of b
 constexpr int kMaxGrid = 256;             // records are sized for up to this many CTAs
 constexpr int kMaxContrib = 32;           // CTAs contributing to one unit
 constexpr int kPowerIters = 8;
@@ -71,15 +73,10 @@ constexpr uint32_t kOffRows = kOffSr + 2 * 256 * 4;            // this CTA's row
 constexpr uint32_t kOffSh = kOffRows + 64;                      // per-segment column shift of C, fp32 [2][64]
 constexpr uint32_t kSmemBytes = kOffSh + 2 * 64 * 4;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;              // slack for 1024-byte alignment
-// After pass 1 the region of the V stages, Q and L (kOffV .. kOffMp) is free. It holds, in order:
-//   DWC: the second bf16 staging tile (the first is C slot kMaxChunks - 1) and the 3 x 3 weights of
-//        up to two heads, fp32 [2][9][64];
-//   combine scratch: A [64][68] and X^T [64][68] fp32, the column statistics, the contributor
-//        table and the partial sums of b;
-//   the second segment's M'^T image (the first segment's is at kOffMp).
-constexpr uint32_t kOffStg1 = kOffV;                            // bf16 SW128 [128][64]
-constexpr uint32_t kOffDw = kOffStg1 + 16384;                   // fp32 [2][9][64]
-constexpr uint32_t kOffAs = kOffDw + 2 * 9 * 64 * 4;            // fp32 [64][68]  A (row l, col k)
+// After pass 1 the region of the V stages, Q and L (kOffV .. kOffMp) is free. It holds the combine
+// scratch: A [64][68] and X^T [64][68] fp32, the column statistics, the contributor table and the
+// partial sums of b; then the second segment's M'^T image (the first segment's is at kOffMp).
+constexpr uint32_t kOffAs = kOffV;                              // fp32 [64][68]  A (row l, col k)
 constexpr uint32_t kOffXt = kOffAs + 64 * kQS * 4;              // fp32 [64][68]  X^T (row j, col l)
 constexpr uint32_t kOffS1 = kOffXt + 64 * kQS * 4;              // double [64]
 constexpr uint32_t kOffS2 = kOffS1 + 512;                       // double [64]
@@ -90,6 +87,11 @@ constexpr uint32_t kOffMt = kOffSv + 256;                       // float [64] un
 constexpr uint32_t kOffBp = kOffMt + 256;                       // float [kWarps][8] partial b
 constexpr uint32_t kOffWc = kOffBp + kWarps * 8 * 4;            // int [kWarps] contributor counts
 constexpr uint32_t kOffImg1 = (kOffWc + kWarps * 4 + 1023) / 1024 * 1024;   // M'^T of segment 1
+// row CTAs' DWC tiles after pass 1: C slot kMaxChunks - 1 and the V / Q / L region, contiguous
+constexpr uint32_t kOffDwcTiles = kOffC + (kMaxChunks - 1) * 16384;
+// solver combine only (no pass 2 there): M' fp32 [64][68] and a zero shift vector, after the image
+constexpr uint32_t kOffMpf = kOffImg1 + 8192;
+constexpr uint32_t kOffZero = kOffMpf + 64 * kQS * 4;
 // solver scratch (aliases the C region: the solver runs before this CTA's pass 1)
 constexpr uint32_t kOffNsHi = 0;                                // tf32 hi [2 K-halves][128 rows][128 B]
 constexpr uint32_t kOffNsLo = 32768;                            // tf32 lo
@@ -100,6 +102,9 @@ constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64]
 
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(kOffImg1 + 8192 <= kOffMp, "post-pass-1 scratch overlaps M'");
+static_assert(kOffDwcTiles + 6 * 16384 <= kOffMp, "DWC tiles overlap M'");
+static_assert(kOffV == kOffDwcTiles + 16384, "the DWC tile region is not contiguous");
+static_assert(kOffZero + 256 <= kOffBar, "solver combine scratch overlaps the barriers");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -109,9 +114,10 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarDiag = 14;  // the solver's diagnostics product done
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarDw = 17;    // [2] DWC transfer product of staging buffer b done
-constexpr int kBarDrain = 19; // every tcgen05 operation of both issuing threads done (count 2)
-constexpr int kNumBars = kBarDrain + 1;
+constexpr int kBarDrain = 17; // every tcgen05 operation of the two issuing threads done (count 2)
+constexpr int kBarH = 18;     // [4] DWC halo tile landed (TMA)
+constexpr int kNumBars = kBarH + 4;
+constexpr int kIssueP2 = kFT - 32;          // pass 2: issues the C M' products
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
@@ -121,6 +127,10 @@ struct FusedArgs {
   unsigned long long* lready; // [U] landmarks of the unit pooled (counts landmarks, m per launch)
   unsigned long long* cnt;    // [U] partial records published per unit
   unsigned long long* xready; // [U] X published (holds the epoch)
+  unsigned long long* mready; // [U] M' image, the contributors' biases and the solver's DWC chunks
+                              // published (holds the epoch)
+  int dwc_k;                  // DWC of each unit's first dwc_k chunks: by the unit's solver CTA
+  unsigned char* mimg;        // [U][8192] M'^T bf16, the SW128 image of the pass-2 B operand
   float* rec;                 // [G][2][kRec]
   // pass-1 warp plan: warp w computes landmarks [wj0[w], wj0[w] + wlt[w]) of row half w / 8;
   // warp padw[h] writes the padding columns of row half h
@@ -285,7 +295,9 @@ __device__ __forceinline__ void ns_issue_k(uint32_t sbase, uint32_t tmem, uint64
   mma_commit(bar);
 }
 
-__device__ void ns_issue(uint32_t sbase, uint32_t tmem, uint64_t* bar, int nks) {
+// One thread issues; out of line, so that the unrolled bodies exist once in the kernel's code
+// (it is called from several places).
+__device__ __noinline__ void ns_issue(uint32_t sbase, uint32_t tmem, uint64_t* bar, int nks) {
   switch (nks) {
     case 1: ns_issue_k<1>(sbase, tmem, bar); break;
     case 2: ns_issue_k<2>(sbase, tmem, bar); break;
@@ -734,6 +746,9 @@ __device__ void segment_shift(const Params& p, const unsigned char* qtile, int n
 // Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
 // (bf16, SW128) goes to C slot gc + 1 (chunk gc writes its C tile into slot gc, which held the
 // previous chunk's rows), one barrier for all of them; the first two V chunks go to stages 0, 1.
+// Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
+// (bf16, SW128) goes to C slot gc + 1 (chunk gc writes its C tile into slot gc, which held the
+// previous chunk's rows), one barrier for all of them; the first two V chunks go to stages 0, 1.
 __device__ void pass1_prefetch(const Rows& R, unsigned char* sm, uint64_t* bars, const CUtensorMap* tmapV,
                                const CUtensorMap* tmapQ) {
   const int nch = R.nchunks;
@@ -915,16 +930,159 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3c, on every CTA holding rows of unit u, once X (from the unit's solver CTA) and every
-// contributor's pass-1 record are out: sum the unit's records and form mu, var, s = 1/sqrt(var +
-// eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A (fp32 FMA), M' = diag(s) M and
-// b = (1/N - s o mu)^T M. M'^T goes to `img` as the bf16 SW128 image of pass 2's B operand (row k =
-// channel, column l = landmark, zero for l >= m) and b to `bvec`. Every such CTA repeats this small
-// computation for itself (the same sums in the same order, so the same bits), which spares the
-// round trip through a single combining CTA before pass 2.
+// Row CTAs, after pass 1: DWC(V) of every chunk (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise taps, zero
+// padding 1), written to O as bf16; pass 2 then adds C M' + b onto it with TMA reduces. Chunk gc (rows
+// [lo, lo + 128) of its unit) comes in as a V tile with a halo, in plain 128-byte rows (no swizzle):
+// rows [lo - top, lo - top + 128 nbox) with top = 64, nbox = 2 when one grid row (W + 1 tokens) fits in
+// 64 rows, else top = 128, nbox = 3; rows outside the unit read as zero. Three (two) tiles are in
+// flight. Thread
+// t owns 4 consecutive tokens of one grid row (4 (t / 16) .. of the chunk; W % 4 == 0, so a group never
+// wraps) and 4 channels (t % 16), with the head's weights in registers as channel pairs; the products
+// run as paired fp32 FMAs (two channels per instruction, each rounded as fmaf).
 // ---------------------------------------------------------------------------------------
-__device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, int u, const float* shift,
-                            unsigned char* img, float* bvec, bool write_stats) {
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+// two bf16 (low half: even channel) -> the fp32 pair
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t v) {
+  return (uint64_t)(v << 16) | ((uint64_t)(v & 0xffff0000u) << 32);
+}
+__device__ __forceinline__ void ffma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint32_t pack_f32x2_bf16(uint64_t v) {
+  return pack_bf16(__uint_as_float((uint32_t)v), __uint_as_float((uint32_t)(v >> 32)));
+}
+
+// DWC of `count` chunks, chunk i = (unit, first row) from get(i) (a callable), from V tiles with a
+// halo in `nbuf` contiguous buffers at `tiles` (barriers kBarH ..), results to O as bf16.
+template <typename Get>
+__device__ void dwc_chunks(const Params& p, unsigned char* tiles, int nbuf, uint64_t* bars,
+                           const CUtensorMap* tmapVp, int count, Get get) {
+  const int t = threadIdx.x, W = p.W, H = p.H, N = p.N;
+  const int nbox = (W + 1 <= 64) ? 2 : 3, top = (nbox == 2) ? 64 : 128;
+  const uint32_t tbytes = (uint32_t)nbox * 16384u;
+  auto issue = [&](int i) {
+    int u, lo;
+    get(i, u, lo);
+    const int b = i % nbuf;
+    mbar_expect_tx(bars + kBarH + b, tbytes);
+    for (int k = 0; k < nbox; ++k)
+      tma_load_3d(tiles + b * tbytes + k * 16384, tmapVp, 0, lo - top + kChunk * k, u, bars + kBarH + b);
+  };
+  if (t == 0)
+    for (int i = 0; i < count && i < nbuf; ++i) issue(i);
+  const int grp = t >> 4, c4 = t & 15, r0 = 4 * grp;
+  uint64_t wt[9][2];   // tap, channel pair (4 c4, 4 c4 + 1), (4 c4 + 2, 4 c4 + 3)
+  int head = -1;
+#pragma unroll 1
+  for (int i = 0; i < count; ++i) {
+    int u, lo;
+    get(i, u, lo);
+    const int nrows = min(kChunk, N - lo);
+    if (u % p.heads != head) {
+      head = u % p.heads;
+      const float* wp = p.dwc + (size_t)head * 64 * 9;
+#pragma unroll
+      for (int tap = 0; tap < 9; ++tap)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          wt[tap][e] = f32x2(__ldg(wp + (4 * c4 + 2 * e) * 9 + tap), __ldg(wp + (4 * c4 + 2 * e + 1) * 9 + tap));
+    }
+    const int b = i % nbuf;
+    mbar_wait(bars + kBarH + b, (i / nbuf) & 1, p.status, kStatusTimeout);
+    if (r0 < nrows) {
+      __nv_bfloat16* O = static_cast<__nv_bfloat16*>(p.O) + (size_t)u * N * 64;
+      const int n0 = lo + r0, y = n0 / W, x0 = n0 - y * W;
+      const bool xl = x0 > 0, xr = x0 + 4 < W;
+      // tile row of token (y - 1, x0 - 1): (n0 - W - 1) - (lo - top); grid row y + a - 1 is W rows on
+      const unsigned char* base = tiles + b * tbytes + (size_t)(r0 - W - 1 + top) * 128 + 8 * c4;
+      uint64_t acc[4][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k][0] = acc[k][1] = 0ull;
+#pragma unroll
+      for (int a = 0; a < 3; ++a) {
+        const int yy = y + a - 1;
+        if (yy < 0 || yy >= H) continue;
+        const unsigned char* rowp = base + (size_t)a * W * 128;
+        uint64_t x[6][2];
+#pragma unroll
+        for (int j = 0; j < 6; ++j) {
+          uint2 raw = make_uint2(0u, 0u);
+          if ((j > 0 || xl) && (j < 5 || xr)) raw = *reinterpret_cast<const uint2*>(rowp + j * 128);
+          x[j][0] = bf16x2_to_f32x2(raw.x);
+          x[j][1] = bf16x2_to_f32x2(raw.y);
+        }
+#pragma unroll
+        for (int bb = 0; bb < 3; ++bb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            ffma2(acc[k][0], wt[a * 3 + bb][0], x[k + bb][0]);
+            ffma2(acc[k][1], wt[a * 3 + bb][1], x[k + bb][1]);
+          }
+      }
+      uint2* op = reinterpret_cast<uint2*>(O + (size_t)n0 * 64 + 4 * c4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (r0 + k < nrows) op[16 * k] = make_uint2(pack_f32x2_bf16(acc[k][0]), pack_f32x2_bf16(acc[k][1]));
+    }
+    __syncthreads();   // tile b read by every thread
+    if (t == 0 && i + nbuf < count) issue(i + nbuf);
+  }
+  // the DWC values in O (generic-proxy stores) come before any TMA reduce onto them
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Row CTAs, after pass 1: DWC of this CTA's chunks, except each unit's first dwc_k chunks, which the
+// unit's solver CTA computes while it waits for the pass-1 records. The tile buffers are contiguous
+// from C slot kMaxChunks - 1 (free: a CTA has at most kMaxChunks - 1 chunks, and the Q tile that slot
+// held is consumed) through the V stages, Q and L (free after pass 1): three of two boxes or two of three.
+__device__ void row_dwc(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint64_t* bars,
+                        const CUtensorMap* tmapVp) {
+  const int nbuf = (p.W + 1 <= 64) ? 3 : 2;
+  // this CTA's chunks outside the solvers' shares (each unit's rows below 128 dwc_k)
+  int list[kMaxChunks];
+  int n = 0;
+  for (int gc = 0; gc < R.nchunks; ++gc) {
+    int s, lo, nrows;
+    R.chunk(gc, s, lo, nrows);
+    if (lo >= kChunk * fa.dwc_k) list[n++] = gc;
+  }
+  __syncthreads();   // pass 1 is done with the V stages, Q and L
+  dwc_chunks(p, sm + kOffDwcTiles, nbuf, bars, tmapVp, n, [&](int i, int& u, int& lo) {
+    int s, nrows;
+    R.chunk(list[i], s, lo, nrows);
+    u = R.seg[s].u;
+  });
+  __syncthreads();
+  trace_mark(p, 25);
+}
+
+// Solver CTA of unit u, after its chain and diagnostics: DWC of the unit's first dwc_k chunks, tiles in
+// its free scratch from offset 0 (four buffers of two boxes or two of three).
+__device__ void solver_dwc(const Params& p, const FusedArgs& fa, unsigned char* sm, uint64_t* bars, int u,
+                           const CUtensorMap* tmapVp) {
+  const int nchu = (p.N + kChunk - 1) / kChunk;
+  const int count = fa.dwc_k < nchu ? fa.dwc_k : nchu;
+  __syncthreads();   // the chain's scratch is no longer read
+  dwc_chunks(p, sm, (p.W + 1 <= 64) ? 4 : 2, bars, tmapVp, count, [&](int i, int& uu, int& lo) {
+    uu = u;
+    lo = kChunk * i;
+  });
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------------------
+// Phase 3, on the unit's solver CTA once every contributor's pass-1 record is out (X is its own):
+// sum the records (each rebased from its column shift c_k to none: S1 += S1'_k + n_k c_k, S2 += S2'_k +
+// 2 c_k S1'_k + n_k c_k^2 in fp64, P += P'_k + c_k (sum_i v_i)_k^T in fp32), form mu, var,
+// s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A (fp32 FMA), M' = diag(s) M
+// and b0 = (1/N - s o mu)^T M. M'^T goes out as the bf16 SW128 image of pass 2's B operand (row k =
+// channel, column l = landmark, zero for l >= m), and each contributor's record gets its pass-2 bias
+// b_k = b0 + c_k^T M' (its resident tiles hold C - c_k, so C M' = (C - c_k) M' + 1 c_k^T M'), in fp32
+// from the unrounded M'. Then a release flag.
+// ---------------------------------------------------------------------------------------
+__device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned char* sm, int u) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int m = p.m, N = p.N;
   float* As = reinterpret_cast<float*>(sm + kOffAs);
@@ -934,7 +1092,6 @@ __device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char*
   float* mus = reinterpret_cast<float*>(sm + kOffMu);
   float* scs = reinterpret_cast<float*>(sm + kOffSc);
   float* svs = reinterpret_cast<float*>(sm + kOffSv);
-  float* bps = reinterpret_cast<float*>(sm + kOffBp);
   int* wcount = reinterpret_cast<int*>(sm + kOffWc);
   int* ctr = reinterpret_cast<int*>(sm + kOffCt);
   const float invNf = 1.f / (float)N;
@@ -963,12 +1120,13 @@ __device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char*
   }
   if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
   nct = nct < kMaxContrib ? nct : kMaxContrib;
-  if (t == 0) {
-    spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
-    spin_until_geq(fa.xready + u, fa.epoch, p.status, kStatusTimeout, p.spin_budget);
-  }
+  if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
   __syncthreads();
-  if (write_stats || true) trace_mark(p, 7);
+  trace_mark(p, 7);
+  float* Mp = reinterpret_cast<float*>(sm + kOffMpf);   // M' fp32 [64][68] (row l)
+  unsigned char* img = sm + kOffMp;
+  const float* shift = reinterpret_cast<const float*>(sm + kOffZero);   // the zero reference
+  if (t < 64) reinterpret_cast<float*>(sm + kOffZero)[t] = 0.f;
   // X^T (row j, column l), zero outside m x m: the product below reads it along l
   {
     constexpr int kNX = 64 * 64 / kFT;   // X entries per thread, all loads issued first
@@ -1072,7 +1230,7 @@ __device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char*
     mus[t] = t < m ? (float)mup : 0.f;
     scs[t] = t < m ? (float)sc : 0.f;
     svs[t] = As[63 * kQS + t];       // landmark column 63 holds sum_i v_i
-    if (write_stats && t < m) {
+    if (t < m) {
       p.mu[(size_t)u * m + t] = (float)(mup + c);
       p.s[(size_t)u * m + t] = (float)sc;
     }
@@ -1092,216 +1250,93 @@ __device__ void row_combine(const Params& p, const FusedArgs& fa, unsigned char*
   }
   __syncthreads();
   trace_mark(p, 9);
-  // M = X A: thread (k0 = 8 (t / 64), l = t % 64) forms M[l][k0 .. k0 + 7]; the lanes of a warp share
-  // k0 (A reads are broadcasts) and take consecutive l (X^T reads and image stores are conflict free)
-  {
-    const int l = t & 63, k0 = 8 * (t >> 6);
-    float acc[8];
+  // M = X A on 256 threads: thread (k0 = 8 (t / 32), l0 = 2 (t % 32)) forms M[l0 .. l0 + 1][k0 .. k0 + 7].
+  // A warp shares k0 (the A reads are broadcasts) and takes the 64 landmarks in pairs (conflict-free
+  // X^T reads and image stores); each step's operands are loaded one step ahead
+  float* bvec = reinterpret_cast<float*>(sm + kOffBv);
+  if (t < 256) {
+    const int l0 = 2 * (t & 31), k0 = 8 * (t >> 5);
+    float acc[2][8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+    float2 xn = *reinterpret_cast<const float2*>(&Xt[l0]);
+    float4 a0n = *reinterpret_cast<const float4*>(&As[k0]);
+    float4 a1n = *reinterpret_cast<const float4*>(&As[k0 + 4]);
+#pragma unroll 1
     for (int j = 0; j < m; ++j) {
-      const float x = Xt[j * kQS + l];
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[j * kQS + k0]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[j * kQS + k0 + 4]);
-      acc[0] = fmaf(x, a0.x, acc[0]);
-      acc[1] = fmaf(x, a0.y, acc[1]);
-      acc[2] = fmaf(x, a0.z, acc[2]);
-      acc[3] = fmaf(x, a0.w, acc[3]);
-      acc[4] = fmaf(x, a1.x, acc[4]);
-      acc[5] = fmaf(x, a1.y, acc[5]);
-      acc[6] = fmaf(x, a1.z, acc[6]);
-      acc[7] = fmaf(x, a1.w, acc[7]);
+      const float2 x = xn;
+      const float4 a0 = a0n, a1 = a1n;
+      const int jn = j + 1 < m ? j + 1 : j;
+      xn = *reinterpret_cast<const float2*>(&Xt[jn * kQS + l0]);
+      a0n = *reinterpret_cast<const float4*>(&As[jn * kQS + k0]);
+      a1n = *reinterpret_cast<const float4*>(&As[jn * kQS + k0 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        acc[0][c] = fmaf(x.x, av[c], acc[0][c]);
+        acc[1][c] = fmaf(x.y, av[c], acc[1][c]);
+      }
     }
-    // pass 2 multiplies the resident C - c*: C~ M = (C - c*) M' + 1 b^T with M' = diag(s) M and
-    // b = sum_l (1/N - s_l mu*_l) M[l] (whitened), or b = sum_l c*_l M[l] (raw, M' = M); b takes the
-    // unrounded M, so the bf16 rounding of M' enters only through the small factor C - c*
-    const bool in = l < m;
-    const float sc = in ? (p.whiten ? scs[l] : 1.f) : 0.f;
-    const float coef = in ? (p.whiten ? invNf - scs[l] * mus[l] : shift[l]) : 0.f;
+    // M' = diag(s) M (raw: M), as fp32 rows for the bias and as the bf16 image; b0 = sum_l
+    // (1/N - s_l mu_l) M[l] (raw: 0)
+    float sc[2], coef[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int l = l0 + r;
+      const bool in = l < m;
+      sc[r] = in ? (p.whiten ? scs[l] : 1.f) : 0.f;
+      coef[r] = (in && p.whiten) ? invNf - scs[l] * mus[l] : 0.f;
+    }
     float bp[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-      *reinterpret_cast<__nv_bfloat16*>(img + sw128(k0 + c, l >> 3) + ((l & 7) << 1)) =
-          __float2bfloat16_rn(sc * acc[c]);
-      bp[c] = coef * acc[c];
+      const float m0 = sc[0] * acc[0][c], m1 = sc[1] * acc[1][c];
+      Mp[l0 * kQS + k0 + c] = m0;
+      Mp[(l0 + 1) * kQS + k0 + c] = m1;
+      *reinterpret_cast<uint32_t*>(img + sw128(k0 + c, l0 >> 3) + ((l0 & 7) << 1)) = pack_bf16(m0, m1);
+      bp[c] = coef[0] * acc[0][c] + coef[1] * acc[1][c];
     }
 #pragma unroll
     for (int c = 0; c < 8; ++c)
       for (int o = 16; o > 0; o >>= 1) bp[c] += __shfl_xor_sync(0xffffffffu, bp[c], o);
     if (lane == 0) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) bps[w * 8 + c] = bp[c];
+      for (int c = 0; c < 8; ++c) bvec[k0 + c] = bp[c];
     }
   }
+  __syncthreads();   // the product above is done reading X^T
+  // every contributor's column shift, [record][landmark], in the place of X^T
+  float* cks = Xt;
+  for (int e = t; e < nct * 64; e += kFT) cks[e] = __ldcg(fa.rec + ctr[e >> 6] + kRecC + (e & 63));
   __syncthreads();
   trace_mark(p, 20);
-  // b[k]: warps 2 (k / 8) and 2 (k / 8) + 1 hold the two halves of the landmark sum of column k
-  if (t < 64) bvec[t] = bps[(2 * (t >> 3)) * 8 + (t & 7)] + bps[(2 * (t >> 3) + 1) * 8 + (t & 7)];
+  // the contributors' biases b_k = b0 + c_k^T M', and the image, out before the flag
+  for (int e = t; e < nct * 64; e += kFT) {
+    const int k = e >> 6, jc = e & 63;
+    float b = bvec[jc];
+    for (int l = 0; l < m; ++l) b = fmaf(cks[k * 64 + l], Mp[l * kQS + jc], b);
+    fa.rec[ctr[k] + kRecB + jc] = b;
+  }
+  for (int e = t; e < 512; e += kFT)
+    reinterpret_cast<uint4*>(fa.mimg + (size_t)u * 8192)[e] = reinterpret_cast<const uint4*>(img)[e];
   __syncthreads();
+  if (t == 0) {
+    __threadfence();
+    st_release_u64(fa.mready + u, fa.epoch);
+  }
+  trace_mark(p, 21);
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3b (row CTAs, after pass 1): DWC(V) of every chunk, the 3 x 3 depthwise taps (§关键设计 1
-// "ZV + DWC(V)", zero padding 1), rounded to bf16 and placed in the chunk's pass-2 TMEM accumulator
-// (columns 64 gc), on which pass 2's product then accumulates. Thread t owns 4 consecutive tokens of
-// one grid row (W % 4 == 0, so a group never wraps) and 4 channels (t % 16). Its 3 x 6 window of V
-// (8-byte loads through L2: pass 1 has just read these rows) is loaded one chunk ahead into a second
-// register set, so the load latency overlaps the previous chunk's arithmetic; the weights of the
-// segments' heads are staged in shared memory. The results go to a bf16 staging tile (SW128 rows,
-// two alternating buffers), which one tcgen05 product with a 64 x 64 identity (exact: every product
-// is by 1 or 0, summed in fp32) copies into the chunk's TMEM accumulator.
-// ---------------------------------------------------------------------------------------
-__device__ __forceinline__ void dwc_load(const Params& p, const Rows& R, int gc, uint2 (&v)[3][6]) {
-  const int t = threadIdx.x, W = p.W;
-  const int r0 = 4 * (t >> 4), c4 = t & 15;
-  int s, lo, nrows;
-  R.chunk(gc, s, lo, nrows);
-  const int n0 = lo + r0, y = n0 / W, x0 = n0 - y * W;
-  const uint2* base = reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(p.V) +
-                                                     (size_t)R.seg[s].u * p.N * 64) + c4;
-#pragma unroll
-  for (int a = 0; a < 3; ++a) {
-    const int yy = y + a - 1;
-    const bool rowok = r0 < nrows && yy >= 0 && yy < p.H;
-#pragma unroll
-    for (int j = 0; j < 6; ++j) {
-      const int xx = x0 + j - 1;
-      v[a][j] = make_uint2(0u, 0u);
-      if (rowok && xx >= 0 && xx < W) v[a][j] = ld_cg_v2_ordered(base + (size_t)(yy * W + xx) * 16);
-    }
-  }
-}
-
-__device__ void dwc_all(const Params& p, const Rows& R, unsigned char* sm, uint32_t sbase, uint32_t tmem,
-                        uint64_t* bars) {
-  const int t = threadIdx.x;
-  const int nch = R.nchunks;
-  // staging buffers: C slot kMaxChunks - 1 (free: a CTA has at most kMaxChunks - 1 chunks, and the
-  // Q tile that slot held is consumed) and kOffStg1
-  unsigned char* stg[2] = {sm + kOffC + (kMaxChunks - 1) * 16384, sm + kOffStg1};
-  float* wsm = reinterpret_cast<float*>(sm + kOffDw);   // [segment][tap][channel]
-  // staged chunk gc -> its TMEM accumulator (columns 64 gc): D = S I over K = 64 channels, the
-  // identity (K-major B) in the M' area, which the combine fills only later
-  auto transfer = [&](int gc) {
-    tc_fence_after();
-    const uint32_t id = idesc(1, 128, 64, 0, 0);
-    const uint64_t sa = desc_sw128(sbase + (uint32_t)(stg[gc & 1] - sm), 16, 1024);
-    const uint64_t ib = desc_sw128(sbase + kOffMp, 16, 1024);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) mma_bf16(tmem + 64 * gc, sa + (uint64_t)(kk * 2), ib + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
-    mma_commit(bars + kBarDw + (gc & 1));
-  };
-  // transfer gc (the (gc >> 1)-th completion of its buffer's barrier) done
-  auto wait_transfer = [&](int gc) {
-    mbar_wait(bars + kBarDw + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
-  };
-  __syncthreads();   // pass 1 is done with the V stages, Q and L, and with TMEM columns 0..127
-  // the weights of each segment's head, fp32 [tap][channel]
-  {
-    constexpr int kNW = (2 * 9 * 64 + kFT - 1) / kFT;   // weights per thread, all loads issued first
-    float wv[kNW];
-#pragma unroll
-    for (int k = 0; k < kNW; ++k) {
-      const int e = t + kFT * k;
-      wv[k] = 0.f;
-      if (e < R.nseg * 9 * 64) {
-        const int sg = e / (9 * 64), rem = e - sg * 9 * 64, tap = rem >> 6, ch = rem & 63;
-        wv[k] = ld_cg_f32_ordered(p.dwc + ((size_t)(R.seg[sg].u % p.heads) * 64 + ch) * 9 + tap);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kNW; ++k)
-      if (t + kFT * k < 2 * 9 * 64) wsm[t + kFT * k] = wv[k];
-  }
-  // the 64 x 64 bf16 identity, SW128 rows (row n, column k): 512 16-byte groups
-  for (int e = t; e < 512; e += kFT) {
-    const int n = e >> 3, c8 = e & 7;
-    const uint32_t one = 0x3f80u << (16 * (n & 1));
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if ((n >> 3) == c8) {
-      const int word = (n & 7) >> 1;
-      if (word == 0) v.x = one;
-      else if (word == 1) v.y = one;
-      else if (word == 2) v.z = one;
-      else v.w = one;
-    }
-    *reinterpret_cast<uint4*>(sm + kOffMp + sw128(n, c8)) = v;
-  }
-  __syncthreads();
-  trace_mark(p, 23);
-  const int r0 = 4 * (t >> 4), c4 = t & 15;
-  auto compute = [&](int gc, const uint2 (&v)[3][6]) {
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    const float* wv = wsm + s * 9 * 64 + 4 * c4;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
-#pragma unroll
-    for (int a = 0; a < 3; ++a) {
-      float x[6][4];
-#pragma unroll
-      for (int j = 0; j < 6; ++j) {
-        x[j][0] = bf_lo(v[a][j].x);
-        x[j][1] = bf_hi(v[a][j].x);
-        x[j][2] = bf_lo(v[a][j].y);
-        x[j][3] = bf_hi(v[a][j].y);
-      }
-#pragma unroll
-      for (int b = 0; b < 3; ++b) {
-        const float4 wt = *reinterpret_cast<const float4*>(wv + (a * 3 + b) * 64);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[i][0] = fmaf(wt.x, x[i + b][0], acc[i][0]);
-          acc[i][1] = fmaf(wt.y, x[i + b][1], acc[i][1]);
-          acc[i][2] = fmaf(wt.z, x[i + b][2], acc[i][2]);
-          acc[i][3] = fmaf(wt.w, x[i + b][3], acc[i][3]);
-        }
-      }
-    }
-    // rows past the chunk's end stage zeros (their accumulator rows are never stored); staging
-    // buffer gc & 1 was last read by transfer gc - 2
-    if (gc >= 2) wait_transfer(gc - 2);
-    unsigned char* st = stg[gc & 1];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint2*>(st + sw128(r0 + i, c4 >> 1) + (c4 & 1) * 8) =
-          make_uint2(pack_bf16(acc[i][0], acc[i][1]), pack_bf16(acc[i][2], acc[i][3]));
-    fence_async_smem();
-    __syncthreads();   // staging gc written
-    if (t == 0) transfer(gc);
-    if (gc == 0) trace_mark(p, 26);
-  };
-  uint2 va[3][6], vb[3][6];
-  if (nch > 0) dwc_load(p, R, 0, va);
-  for (int gc = 0; gc < nch; gc += 2) {
-    if (gc + 1 < nch) dwc_load(p, R, gc + 1, vb);
-    compute(gc, va);
-    if (gc + 1 < nch) {
-      if (gc + 2 < nch) dwc_load(p, R, gc + 2, va);
-      compute(gc + 1, vb);
-    }
-  }
-  trace_mark(p, 27);
-  // the last transfers (earlier ones were waited before their buffer was reused)
-  if (nch >= 2) wait_transfer(nch - 2);
-  if (nch >= 1) wait_transfer(nch - 1);
-  tc_fence_before();
-  __syncthreads();
-  trace_mark(p, 25);
-}
-
-// ---------------------------------------------------------------------------------------
-// Phase 4: O = C M' + b + DWC(V) for every chunk. M'^T and b of each segment's unit come from
-// its solver CTA (segment 0's image in the M' area, segment 1's in the free halo region). Each
-// chunk's product accumulates onto the DWC values already in its TMEM accumulator (phase 3b); all
-// products are issued at once, each with its own barrier, and the epilogues (+ b, bf16) follow
-// chunk by chunk. The bf16 rows are staged in the chunk's C slot (free once its product is done)
-// and leave by TMA stores of 32-row quarters: warps w, w + 4, w + 8, w + 12 hold the same 32 rows
-// (16 channels each) and meet on named barrier 1 + w % 4 before warp w % 4 issues the quarter's
-// store.
+// Phase 4: O += C M' + b for every chunk, onto the DWC values pass 1 wrote to O. M'^T and b of each
+// segment's unit come from this CTA's own combine (segment 0's image in the M' area, segment 1's at
+// kOffImg1). All products are issued at once, each with its own barrier, and the epilogues (+ b,
+// bf16) follow chunk by chunk. The bf16 rows are staged in the chunk's C slot (free once its product
+// is done) and leave by TMA reduce-adds of 32-row quarters onto O: warps w, w + 4, w + 8, w + 12 hold
+// the same 32 rows (16 channels each) and meet on named barrier 1 + w % 4 before warp w % 4 issues
+// the quarter's reduce.
 // ---------------------------------------------------------------------------------------
 __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
                           uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapO) {
@@ -1309,18 +1344,29 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   const int nch = R.nchunks;
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
   auto img_off = [](int s) -> uint32_t { return s == 0 ? kOffMp : kOffImg1; };
-  // each segment's M'^T image and b, formed by this CTA's own combine
-  for (int s = 0; s < R.nseg; ++s)
-    row_combine(p, fa, sm, R.seg[s].u, reinterpret_cast<const float*>(sm + kOffSh) + 64 * s, sm + img_off(s),
-                bvec + 64 * s, R.seg[s].lo == 0);
+  // each segment's M'^T image from its unit's solver CTA, and the pass-2 bias that CTA computed for
+  // this CTA's record (its column shift)
+  if (t == 0)
+    for (int s = 0; s < R.nseg; ++s)
+      spin_until_geq(fa.mready + R.seg[s].u, fa.epoch, p.status, kStatusTimeout, p.spin_budget);
+  __syncthreads();
+  // the solver CTAs' DWC values in O (generic-proxy stores, released with mready) come before this
+  // CTA's TMA reduces onto them
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   trace_mark(p, 4);
+  for (int s = 0; s < R.nseg; ++s) {
+    const unsigned char* img = fa.mimg + (size_t)R.seg[s].u * 8192;
+    for (int e = t; e < 512; e += kFT)
+      reinterpret_cast<uint4*>(sm + img_off(s))[e] = __ldcg(reinterpret_cast<const uint4*>(img) + e);
+    if (t < 64) bvec[64 * s + t] = __ldcg(fa.rec + ((size_t)blockIdx.x * 2 + s) * kRec + kRecB + t);
+  }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   trace_mark(p, 5);
-  // one thread (in warp 15, which issues no stores) issues the products in chunk order, each
+  // one thread (in warp 15, which issues no reduces) issues the products in chunk order, each
   // chunk's four followed by its commit, so the epilogues can start while later chunks are issued
-  if (t == kFT - 32) {
+  if (t == kIssueP2) {
     tc_fence_after();
     const uint32_t id = idesc(1, 128, 64, 0, 0);
     for (int gc = 0; gc < nch; ++gc) {
@@ -1330,7 +1376,7 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
       const uint64_t mb = desc_sw128(sbase + img_off(s), 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, 1u);
+        mma_bf16(tmem + 64 * gc, ca + (uint64_t)(kk * 2), mb + (uint64_t)(kk * 2), id, kk > 0 ? 1u : 0u);
       mma_commit(bars + kBarP2 + gc);
     }
   }
@@ -1357,9 +1403,9 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
     }
     fence_async_smem();
     named_bar_sync(1 + q, 128);
-    // rows past the unit's end (a short last chunk) fall outside the tensor and are not written
+    // rows past the unit's end (a short last chunk) fall outside the tensor and are skipped
     if (h == 0 && lane == 0 && 32 * q < nrows) {
-      tma_store_3d(tmapO, 0, lo + 32 * q, R.seg[s].u, ob + 4096 * q);
+      tma_reduce_add_3d(tmapO, 0, lo + 32 * q, R.seg[s].u, ob + 4096 * q);
       bulk_commit_group();
     }
     if (gc < 2) trace_mark(p, 30 + gc);
@@ -1373,7 +1419,8 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
 __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const FusedArgs fa,
                                                            const __grid_constant__ CUtensorMap tmapV,
                                                            const __grid_constant__ CUtensorMap tmapQ,
-                                                           const __grid_constant__ CUtensorMap tmapO) {
+                                                           const __grid_constant__ CUtensorMap tmapO,
+                                                           const __grid_constant__ CUtensorMap tmapVp) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + pad;
@@ -1405,6 +1452,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     tma_prefetch_desc(&tmapV);
     tma_prefetch_desc(&tmapQ);
     tma_prefetch_desc(&tmapO);
+    tma_prefetch_desc(&tmapVp);
   }
 
   // ---- phase 0: landmark pooling, one warp per landmark ----
@@ -1470,17 +1518,19 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     const SolverInfo si = solver_cta(p, fa, sm, sbase, tmem, bars, g);
     trace_mark(p, 3);
     solver_diagnostics(p, sm, sbase, tmem, bars, g, si);
+    solver_dwc(p, fa, sm, bars, g, &tmapVp);
+    solver_combine(p, fa, sm, g);
   }
   if (R.nchunks > 0) {
     pass1(p, fa, R, sm, sbase, tmem, bars, &tmapV);
     trace_mark(p, 3);
-    dwc_all(p, R, sm, sbase, tmem, bars);
+    row_dwc(p, fa, R, sm, bars, &tmapVp);
     pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
   }
-  // drain: the tcgen05 operations of both issuing threads (thread 0: solver, pass-1 and DWC products;
-  // the first thread of the last warp: pass-2 products) have completed before TMEM is released. In a
-  // normal run each was waited already; after an expired wait this bounds the wait for any still running.
-  if (t == 0 || t == kFT - 32) mma_commit(bars + kBarDrain);
+  // drain: the tcgen05 operations of the two issuing threads (thread 0: solver and pass-1 products;
+  // kIssueP2: pass-2 products) have completed before TMEM is released. In a normal run each was
+  // waited already; after an expired wait this bounds the wait for any still running.
+  if (t == 0 || t == kIssueP2) mma_commit(bars + kBarDrain);
   if (t == 0) mbar_wait(bars + kBarDrain, 0, p.status, kStatusTimeout);
   __syncthreads();
   trace_mark(p, 15);
@@ -1493,13 +1543,13 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
 
 }  // namespace
 
-// Flag area: three [U] flag arrays (lready, cnt, xready), each padded to 256 B; then the per-CTA
-// pass-1 records.
+// Flag area: four [U] flag arrays (lready, cnt, xready, mready), each padded to 256 B; then the
+// per-CTA pass-1 records and the per-unit M' images.
 static size_t flag_stride(int U) { return 256 * (size_t)((U * 8 + 255) / 256); }
-static size_t flag_bytes(int U) { return 3 * flag_stride(U); }
+static size_t flag_bytes(int U) { return 4 * flag_stride(U); }
 
 size_t fused_workspace_bytes(int U) {
-  return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
+  return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * 8192;
 }
 
 // Decide whether the fused kernel serves this shape on the current device; returns the grid size
@@ -1519,8 +1569,9 @@ int fused_grid(const Params& p) {
   const long long nchu = (p.N + kChunk - 1) / kChunk;
   const long long cpc = ((long long)p.U * nchu + (G - p.U) - 1) / (G - p.U);
   if (cpc > kMaxChunks - 1 || cpc > nchu) return 0;   // one C slot stays free for the Q chunk
-  // the DWC phase's token groups of 4 stay on one grid row
-  if (p.W % 4 != 0) return 0;
+  // the DWC phase's token groups of 4 stay on one grid row, and one grid row plus a token fits in the
+  // 128-row halo above and below a chunk
+  if (p.W % 4 != 0 || p.W > 127) return 0;
   // replay the row partition: contributors of every unit must fit the offset table
   {
     int worst = 0, cur_u = -1, cur = 0;
@@ -1549,7 +1600,7 @@ int fused_grid(const Params& p) {
 }
 
 // Tensor maps of recently used V pointers (host side; encoding costs a driver call).
-constexpr int kTmapCache = 32;   // Q, V and O maps of a few rotating buffer sets
+constexpr int kTmapCache = 48;   // Q, V (two layouts) and O maps of a few rotating buffer sets
 struct TmapCache {
   const void* ptr[kTmapCache];
   int N[kTmapCache], U[kTmapCache], sw[kTmapCache], box[kTmapCache];
@@ -1626,8 +1677,9 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
     const cudaError_t e = cudaMemsetAsync(fused_ws, 0, flag_bytes(p.U), st);
     if (e != cudaSuccess) return e;
   }
-  CUtensorMap tmap, tmapq, tmapo;
+  CUtensorMap tmap, tmapq, tmapo, tmapvp;
   if (!tmap_for(p.V, p.N, p.U, kChunk, true, &tmap)) return cudaErrorInvalidValue;
+  if (!tmap_for(p.V, p.N, p.U, kChunk, false, &tmapvp)) return cudaErrorInvalidValue;
   if (!tmap_for(p.Q, p.N, p.U, kChunk, true, &tmapq)) return cudaErrorInvalidValue;
   if (!tmap_for(p.O, p.N, p.U, 32, true, &tmapo)) return cudaErrorInvalidValue;
   FusedArgs fa;
@@ -1636,10 +1688,23 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   fa.lready = reinterpret_cast<unsigned long long*>(fused_ws);
   fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + fs);
   fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 2 * fs);
+  fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 3 * fs);
+  fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
   plan_pass1_warps(p.m, fa);
+  // The solver CTAs wait, after their chain, for the pass-1 records; they spend that time on the DWC
+  // of their unit's first chunks. Rough model: a chunk of pass 1 takes about 6.8 us, the chain about
+  // 33 us, a chunk of DWC about 1.5 us, so a solver has room for (6.8 cpc - 33) / 1.5 chunks, cpc the
+  // chunks of a row CTA.
+  {
+    const int nchu = (p.N + kChunk - 1) / kChunk;
+    const int cpc = (p.U * nchu + (G - p.U) - 1) / (G - p.U);
+    int k = (68 * cpc - 330) / 15;
+    k = k < 0 ? 0 : (k > nchu ? nchu : k);
+    fa.dwc_k = k;
+  }
   Params pp = p;
-  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo};
+  void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo, (void*)&tmapvp};
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
   cudaError_t e = cudaLaunchCooperativeKernel((const void*)k_fused_forward, dim3(G), dim3(kFT), args, kSmemAlloc, st);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);

@@ -181,6 +181,15 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int
                "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
                : "memory");
 }
+// Tiled reduce-add shared -> global of one box at {x, y, z} in the tensor map's element type (here
+// bf16: global = bf16(global + smem)); elements outside the tensor are skipped. Tracked by this
+// thread's bulk async-group like a store.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, int x, int y, int z, const void* src) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                   tmap),
+               "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // every bulk store this thread committed has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
