@@ -187,6 +187,8 @@ lfa_status ensure_attributes() {
   if (dev < 64 && (g_attr_done >> dev) & 1ull) return LFA_OK;
   if (lfa::generic_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::backward_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::gemm_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::ns_tc_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (dev < 64) g_attr_done |= 1ull << dev;
   return LFA_OK;
 }

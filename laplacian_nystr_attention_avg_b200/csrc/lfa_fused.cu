@@ -193,14 +193,16 @@ __device__ __forceinline__ void block_reduce2(float& a, float& b, float* red) {
   }
 }
 
-// L [m][64] fp32 (global, written by other CTAs of this launch) -> [64][kQS] shared, zero rows >= m.
-__device__ __forceinline__ void load_landmarks(const float* Lg, float* Ls, int m) {
+// L [m][d] fp32 (global, written by other CTAs of this launch) -> [64][kQS] shared, zero outside m x d
+// (zero columns add nothing to an L1 distance, so d = 32 landmarks work in the same 64-wide layout).
+__device__ __forceinline__ void load_landmarks(const float* Lg, float* Ls, int m, int d = 64) {
   constexpr int kN4 = 1024 / kFT;   // float4 of the [64][64] block per thread
   float4 v[kN4];
 #pragma unroll
   for (int i = 0; i < kN4; ++i) {
-    const int e4 = threadIdx.x + kFT * i, r = e4 >> 4;
-    v[i] = r < m ? __ldcg(reinterpret_cast<const float4*>(Lg) + e4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const int e4 = threadIdx.x + kFT * i, r = e4 >> 4, c = 4 * (e4 & 15);
+    v[i] = (r < m && c < d) ? __ldcg(reinterpret_cast<const float4*>(Lg + (size_t)r * d + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int i = 0; i < kN4; ++i) {
@@ -325,7 +327,7 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
   float* Xsm = reinterpret_cast<float*>(sm + kOffNsX);
   float* vec = reinterpret_cast<float*>(sm + kOffNsVec);
   float* red = vec + 128;
-  load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
+  load_landmarks(p.L + (size_t)u * m * p.d, Ls, m, p.d);
   __syncthreads();
   // W (symmetric): entries a <= b < m of the upper triangle, dealt out evenly (entry e -> (a, b)
   // in row-major triangle order), mirrored; padding rows and columns are zero
@@ -363,6 +365,8 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
   }
   __syncthreads();
   trace_mark(p, 16);
+  // W + eps I for the backward pass, which reads the forward's context from the workspace
+  for (int e = t; e < m * m; e += kFT) p.Wm[(size_t)u * m * m + e] = Ws[(e / m) * kQS + e % m];
 
   const int q = w & 3, h = w >> 2;
   const int r = 32 * q + lane;         // stacked row 0..127
@@ -536,7 +540,7 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
     }
   }
   __syncthreads();
-  if (t == 0) {
+  if (t == 0 && fa.xready != nullptr) {
     __threadfence();
     st_release_u64(fa.xready + u, fa.epoch);
   }
@@ -1543,6 +1547,43 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
 
 }  // namespace
 
+// The Newton-Schulz chain of the fused kernel as a kernel of its own, one CTA per (batch, head) unit,
+// for the per-stage path (any dtype, d = 32 or 64, m <= 64): W, alpha, the T steps on tcgen05 in
+// 3xTF32 and the diagnostics, from landmarks already pooled into the workspace; X and W go to the
+// workspace (the per-stage passes and the backward read them there).
+__global__ void __launch_bounds__(kFT, 1) k_ns_tc(const Params p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sm = smem_raw + pad;
+  const uint32_t sbase = smem_u32(sm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + kTmemSlot);
+  const int t = threadIdx.x, w = t >> 5;
+  if (w == 0) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  if (t == 0) {
+    mbar_init(bars + kBarNs, 1);
+    mbar_init(bars + kBarDiag, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  FusedArgs fa;
+  memset(&fa, 0, sizeof(fa));
+  fa.epoch = 1;
+  const SolverInfo si = solver_cta(p, fa, sm, sbase, tmem, bars, blockIdx.x);
+  solver_diagnostics(p, sm, sbase, tmem, bars, blockIdx.x, si);
+  tc_fence_before();
+  __syncthreads();
+  if (w == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
+  }
+}
+
 // Flag area: four [U] flag arrays (lready, cnt, xready, mready), each padded to 256 B; then the
 // per-CTA pass-1 records and the per-unit M' images.
 static size_t flag_stride(int U) { return 256 * (size_t)((U * 8 + 255) / 256); }
@@ -1550,6 +1591,15 @@ static size_t flag_bytes(int U) { return 4 * flag_stride(U); }
 
 size_t fused_workspace_bytes(int U) {
   return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * 8192;
+}
+
+cudaError_t ns_tc_set_attributes() {
+  return cudaFuncSetAttribute(k_ns_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
+}
+
+cudaError_t launch_ns_tc(const Params& p, cudaStream_t st) {
+  k_ns_tc<<<p.U, kFT, kSmemAlloc, st>>>(p);
+  return cudaGetLastError();
 }
 
 // Decide whether the fused kernel serves this shape on the current device; returns the grid size

@@ -4,7 +4,7 @@
 //
 // Steps (LaplacianFormer note, papernotes.org: §整体框架 flowchart, §关键设计 1-3):
 //   k_pool          L = r x r average pool of Q                         (§关键设计 2)
-//   k_ns_small      W = exp(-E/lam) + eps I, ||W||_2, alpha, T Newton-Schulz steps, m <= 64
+//   (m <= 64: k_ns_tc in lfa_fused.cu: W, ||W||_2, alpha and the T steps on tcgen05, one CTA per unit)
 //   k_gram / k_alpha / k_mm (lfa_gemm.cu) / k_ns_gemm   the same for 64 < m <= 256, spread over
 //                   CTAs (§关键设计 3); k_ns_gemm forms the closing residual I - W X_T and its norm
 //   k_pass1         C tiles in registers/smem, column sums of C and C^2, raw C^T V, sum V
@@ -73,40 +73,7 @@ __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
 // ---------------------------------------------------------------------------------------
 // Small-m landmark kernel + alpha + Newton-Schulz, one CTA per unit, all in shared memory.
 // ---------------------------------------------------------------------------------------
-constexpr int kNsS = 68;   // row stride (floats) of the 64 x 64 shared matrices
-
-// C = A * B for MP x MP matrices (MP <= 64, multiple of 16) in shared memory; 4x4 per thread.
-__device__ void smem_mm(const float* A, const float* B, float* C, int MP, float diag_scale,
-                        float add_diag) {
-  // C = diag_scale * (A B) + add_diag * I
-  const int nbj = MP / 4;
-  const int t = threadIdx.x;
-  if (t < nbj * nbj) {
-    const int bi = t / nbj, bj = t % nbj;
-    float acc[4][4] = {};
-    for (int l = 0; l < MP; ++l) {
-      float a[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) a[x] = A[(4 * bi + x) * kNsS + l];
-      float4 b = *reinterpret_cast<const float4*>(&B[l * kNsS + 4 * bj]);
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
-        acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
-        acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
-        acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
-      }
-    }
-#pragma unroll
-    for (int x = 0; x < 4; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int i = 4 * bi + x, j = 4 * bj + y;
-        C[i * kNsS + j] = diag_scale * acc[x][y] + (i == j ? add_diag : 0.f);
-      }
-  }
-}
-
+// Sum of v over the block (every thread gets the total; all threads must call it).
 __device__ float block_sum(float v, float* red) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -116,129 +83,6 @@ __device__ float block_sum(float v, float* red) {
   float s = 0.f;
   for (int i = 0; i < (int)(blockDim.x / 32); ++i) s += red[i];
   return s;
-}
-
-// Power iteration for lambda_max of the SPD matrix W (shared, MP x MP, zero padded).
-// Returns the Rayleigh quotient v^T W v of the final unit vector.
-__device__ float power_lambda_max(const float* Wsm, int m, float* v, float* w, float* red,
-                                  int iters) {
-  const int t = threadIdx.x;
-  if (t < kSmallM) v[t] = t < m ? rsqrtf(float(m)) : 0.f;
-  __syncthreads();
-  float rq = 0.f;
-  for (int it = 0; it <= iters; ++it) {
-    float wi = 0.f;
-    if (t < m) {
-      for (int j = 0; j < m; ++j) wi = fmaf(Wsm[t * kNsS + j], v[j], wi);
-    }
-    const float vw = block_sum(t < m ? wi * v[t] : 0.f, red);   // v^T W v
-    const float nn = block_sum(t < m ? wi * wi : 0.f, red);
-    rq = vw;
-    if (it == iters) break;
-    const float inv = rsqrtf(nn);
-    __syncthreads();
-    if (t < m) w[t] = wi * inv;
-    __syncthreads();
-    if (t < kSmallM) v[t] = t < m ? w[t] : 0.f;
-    __syncthreads();
-  }
-  return rq;
-}
-
-__global__ void __launch_bounds__(kThreads) k_ns_small(Params p) {
-  extern __shared__ float4 smem_f4[];
-  float* sm = reinterpret_cast<float*>(smem_f4);
-  float* Wsm = sm;                         // [64][kNsS]
-  float* Xs = Wsm + 64 * kNsS;             // [64][kNsS]
-  float* Ys = Xs + 64 * kNsS;              // [64][kNsS]
-  float* Ls = Ys + 64 * kNsS;              // [64][d + 4]
-  float* vec = Ls + 64 * (64 + 4);         // 2 x 64
-  float* red = vec + 128;                  // 32
-  const int u = blockIdx.x, t = threadIdx.x;
-  const int m = p.m, d = p.d, MP = round_up(m, 16);
-  const int ds = d + 4;
-  for (int e = t; e < 64 * kNsS; e += blockDim.x) { Wsm[e] = 0.f; Xs[e] = 0.f; Ys[e] = 0.f; }
-  for (int e = t; e < m * d; e += blockDim.x) Ls[(e / d) * ds + e % d] = p.L[(size_t)u * m * d + e];
-  __syncthreads();
-  // W_ab = exp(-||l_a - l_b||_1 / lam) + eps delta_ab
-  for (int e = t; e < m * m; e += blockDim.x) {
-    const int a = e / m, b = e % m;
-    float acc = 0.f;
-    for (int k = 0; k < d; ++k) acc += fabsf(Ls[a * ds + k] - Ls[b * ds + k]);
-    Wsm[a * kNsS + b] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
-  }
-  __syncthreads();
-  const float lmax = power_lambda_max(Wsm, m, vec, vec + 64, red, 32);
-  // alpha = 2/||W||_2 as printed, kept only if ||I - alpha W W^T||_2 < 1; for SPD W that
-  // norm is max_j |1 - alpha w_j^2| = max(|1 - alpha lmax^2|, ...) which is < 1 iff
-  // alpha lmax^2 < 2.
-  const float alpha_p = 2.f / lmax;
-  const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
-  const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
-  // X_0 = alpha W^T
-  for (int e = t; e < m * m; e += blockDim.x) {
-    const int a = e / m, b = e % m;
-    Xs[a * kNsS + b] = alpha * Wsm[b * kNsS + a];
-  }
-  __syncthreads();
-  for (int k = 0; k < p.T; ++k) {
-    smem_mm(Wsm, Xs, Ys, MP, -1.f, 2.f);   // Y = 2I - W X
-    __syncthreads();
-    // X <- X Y: every thread reads its operands before anyone overwrites X
-    {
-      const int nbj = MP / 4;
-      float acc[4][4] = {};
-      int bi = 0, bj = 0;
-      const bool active = t < nbj * nbj;
-      if (active) {
-        bi = t / nbj;
-        bj = t % nbj;
-        for (int l = 0; l < MP; ++l) {
-          float a[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) a[x] = Xs[(4 * bi + x) * kNsS + l];
-          float4 b = *reinterpret_cast<const float4*>(&Ys[l * kNsS + 4 * bj]);
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            acc[x][0] = fmaf(a[x], b.x, acc[x][0]);
-            acc[x][1] = fmaf(a[x], b.y, acc[x][1]);
-            acc[x][2] = fmaf(a[x], b.z, acc[x][2]);
-            acc[x][3] = fmaf(a[x], b.w, acc[x][3]);
-          }
-        }
-      }
-      __syncthreads();
-      if (active) {
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) Xs[(4 * bi + x) * kNsS + 4 * bj + y] = acc[x][y];
-      }
-      __syncthreads();
-    }
-  }
-  // residual ||I - W X_T||_F
-  smem_mm(Wsm, Xs, Ys, MP, -1.f, 1.f);
-  __syncthreads();
-  float sq = 0.f;
-  for (int e = t; e < m * m; e += blockDim.x) {
-    const float r = Ys[(e / m) * kNsS + e % m];
-    sq += r * r;
-  }
-  const float res = sqrtf(block_sum(sq, red));
-  for (int e = t; e < m * m; e += blockDim.x) {
-    const int a = e / m, b = e % m;
-    p.X[(size_t)u * m * m + e] = Xs[a * kNsS + b];
-    p.Wm[(size_t)u * m * m + e] = Wsm[a * kNsS + b];
-  }
-  if (t == 0) {
-    float* inf = p.info + (size_t)u * kInfoStride;
-    inf[kInfoAlpha] = alpha;
-    inf[kInfoLambdaMax] = lmax;
-    inf[kInfoFallback] = float(fallback);
-    inf[kInfoResidual] = res;
-    if (!isfinite(lmax) || !isfinite(res)) atomicOr(p.status, kStatusNonFinite);
-  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -969,8 +813,7 @@ void context_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
   if (m <= kSmallM) {
-    const size_t smem = (3 * 64 * kNsS + 64 * 68 + 128 + 32) * sizeof(float);
-    k_ns_small<<<U, kThreads, smem, st>>>(p);
+    launch_ns_tc(p, st);
   } else {
     k_gram<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
     k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
@@ -1025,7 +868,6 @@ cudaError_t generic_set_attributes() {
   cudaError_t e = cudaSuccess;
 #define LFA_ATTR(fn) \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, big)
-  LFA_ATTR(k_ns_small);
   LFA_ATTR((k_pass1<float, 1>));
   LFA_ATTR((k_pass1<float, 2>));
   LFA_ATTR((k_pass1<float, 4>));

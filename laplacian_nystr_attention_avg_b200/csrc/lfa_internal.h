@@ -136,6 +136,9 @@ struct MmJobs {
 // host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu / lfa_gemm.cu
 // Up to three independent jobs (none reads another's output) in one launch.
 cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st);
+cudaError_t gemm_set_attributes();
+cudaError_t ns_tc_set_attributes();
+cudaError_t launch_ns_tc(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_context(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st);

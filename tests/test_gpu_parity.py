@@ -76,9 +76,9 @@ def test_newton_schulz_context(name):
         kappa = np.linalg.cond(f.W)
         errX = np.max(np.abs(X - f.X)) / np.max(np.abs(f.X))
         # First-order error of the last printed Newton-Schulz step is ~ c * kappa * u for unit
-        # roundoff u of the products: c = 33 covers fp32 FMA (u = 2^-24); the fused bf16 path
-        # runs the products as split TF32 (hi + lo, the lo part truncated to 11 bits), u = 2^-21.
-        u_eff = 2.0 ** -21 if mod.path == "fused" else 2.0 ** -24
+        # roundoff u of the products (c = 33). Every path runs the m x m products on the tensor cores
+        # as split TF32 (hi + lo, the lo part truncated to 11 bits): u = 2^-21.
+        u_eff = 2.0 ** -21
         assert errX <= 33 * u_eff * kappa + 1e-5, f"{name} unit {u}: X error {errX:.2e} (kappa {kappa:.0f})"
         assert abs(info[u].lambda_max - f.alpha.norm2) <= 1e-4 * f.alpha.norm2
         assert info[u].alpha_fallback == int(f.alpha.fallback) == 1
