@@ -51,6 +51,9 @@ def parse_args():
                     help="approximate CPU work of the oracle baseline sample")
     ap.add_argument("--backward", action="store_true",
                     help="time forward + backward steps instead (1 GPU; e.g. --workload long)")
+    ap.add_argument("--seqsplit", action="store_true",
+                    help="split every unit's grid rows over the ranks (bands; NCCL all-reduces and "
+                         "neighbour exchanges); default workload long")
     return ap.parse_args()
 
 
@@ -258,6 +261,90 @@ def run_backward(args):
     }), flush=True)
 
 
+def run_seqsplit(args):
+    """One step = one forward of the whole workload with every unit's grid rows split over the ranks
+    (laplacian_nystr_attention_avg_b200.seqsplit: band calls of the library, NCCL exchanges).
+    Total work is fixed as ranks are added (strong scaling); value = all tokens / max-over-ranks time."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from laplacian_nystr_attention_avg_b200 import lfa, seqsplit
+    from laplacian_nystr_attention_avg_b200.inputs import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = WORKLOADS[args.workload if args.workload != "pvt1" else "long"]
+    x = make_inputs(wl)
+    y0, ny = seqsplit.band_rows(wl.H, world, rank)
+    band = lfa.SeqSplitBand(lfa.make_config(wl), y0, ny, x.dwc, str(dev))
+    sl = slice(y0 * wl.W, (y0 + ny) * wl.W)
+    Qh = x.Q_store[:, :, sl].contiguous().pin_memory()
+    Vh = x.V_store[:, :, sl].contiguous().pin_memory()
+    Q, V = Qh.to(dev), Vh.to(dev)
+    O = torch.empty_like(Q)
+    comm = seqsplit.TorchComm(rank, world)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        seqsplit.forward_rank(band, Q, V, O, comm, wl.W)
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    t0.record(stream)
+    for _ in range(K):
+        seqsplit.forward_rank(band, Q, V, O, comm, wl.W)
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks([t0.elapsed_time(t1)], world, dev)[0]
+    # end to end: this band's Q, V from pinned host memory and O back, every step
+    Oh = torch.empty(Qh.shape, dtype=Qh.dtype).pin_memory()
+    E = max(1, args.e2e_steps // 10)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        Q.copy_(Qh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        seqsplit.forward_rank(band, Q, V, O, comm, wl.W)
+        Oh.copy_(O, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0]
+    tokens = wl.units * wl.N
+    if rank == 0:
+        nbytes = Qh.numel() * Qh.element_size()
+        print(json.dumps({
+            "metric": f"tokens/s per Laplacian-Nyström attention call (N={wl.N},d={wl.d},m={wl.m}), "
+                      f"grid rows split over ranks", "value": tokens * K / (ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16 storage, fp32 arithmetic",
+            "data": "synthetic",
+            "config": workload_config(wl, {"path": "generic (band calls)", "parallelism": f"seqsplit{world}",
+                                           "bands": [seqsplit.band_rows(wl.H, world, k) for k in range(world)],
+                                           "l2": "inputs resident; no flush"}),
+            "e2e": {"value": tokens * E / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * nbytes * world, "d2h_bytes_per_step": nbytes * world},
+            "gpu_launches": K * int(band.lib.lfa_launches_per_forward(band.handle)), "clocks": clk}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -265,6 +352,9 @@ def main():
         return
     if args.backward:
         run_backward(args)
+        return
+    if args.seqsplit:
+        run_seqsplit(args)
         return
     import torch
     import torch.distributed as dist

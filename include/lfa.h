@@ -181,6 +181,34 @@ lfa_status lfa_destroy(lfa_handle h);
 /* Static, human-readable name of a status code. */
 const char* lfa_status_string(lfa_status s);
 
+/* ---- sequence split over several devices ---------------------------------- *
+ * One unit's N tokens can be split over devices in bands of whole grid rows (the note's 实验关键数据
+ * and 局限 sections: memory grows linearly with the sequence, long sequences are the target). A
+ * band handle holds grid rows [y0, y0 + ny) of every unit (its Q, V and O tensors are
+ * [B][heads][ny * W][d] in cfg.dtype, token n = (y - y0) W + x). One forward is three exchanges of the
+ * caller's choosing (all-reduce, neighbour send/receive), between four calls:
+ *   1. lfa_sp_pool: this band's share of every landmark, L_partial [B*heads][m][d] fp32 (the sum over
+ *      the window's tokens inside the band, divided by r^2); the SUM over all bands is L.
+ *   2. lfa_sp_pass1(L): W, alpha and the Newton-Schulz chain from the full L (the same on every band),
+ *      and this band's pass-1 sums, partial [B*heads][S] fp64 with S = lfa_sp_partial_size: column
+ *      sums of C and C^2 [m] each, C^T V [m][d] and sum V [d]; the SUM over all bands is the unit's.
+ *   3. lfa_sp_pass2(totals, halo): the combine from the summed partials (statistics over all H W
+ *      tokens), then pass 2 and DWC for this band's rows. V_halo [B*heads][2][W][d] in cfg.dtype holds
+ *      the V rows y0 - 1 and y0 + ny (from the neighbouring bands; any values where the row is outside
+ *      the grid); it may be NULL when the band is the whole grid.
+ * The result equals lfa_forward's on the whole grid up to the order of the sums. whiten = 0 or 1 only
+ * (LFA_ERR_UNSUPPORTED otherwise); per-stage kernels; no backward. Band handles are rejected by
+ * lfa_forward and lfa_backward (LFA_ERR_INVALID_ARG). Argument conventions as for lfa_create. */
+size_t lfa_sp_workspace_size(const lfa_config* cfg, int y0, int ny);
+lfa_status lfa_sp_create(const lfa_config* cfg, int y0, int ny, const float* dwc_weight, void* workspace,
+                         size_t workspace_bytes, lfa_handle* out);
+int lfa_sp_partial_size(lfa_handle h);
+lfa_status lfa_sp_pool(lfa_handle h, const void* Q_local, float* L_partial, void* stream);
+lfa_status lfa_sp_pass1(lfa_handle h, const void* Q_local, const void* V_local, const float* L_full,
+                        double* partial_out, void* stream);
+lfa_status lfa_sp_pass2(lfa_handle h, const void* Q_local, const void* V_local, const void* V_halo,
+                        const double* partial_total, void* O_local, void* stream);
+
 /* ---- inspection entry points used by the parity tests ---------------------- */
 
 /* Cross kernel C = exp(-||q_i - l_l||_1 / lambda) of one unit [the note's §关键设计 2],

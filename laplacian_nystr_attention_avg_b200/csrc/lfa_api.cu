@@ -27,6 +27,7 @@ struct lfa_ctx {
   float* cap_C;   // armed by lfa_debug_capture_cross: the next forward copies C of cap_unit here
   float* cap_S;   // and, if set, the column shift of each entry
   int cap_unit;
+  int sp;   // sequence-split handle (lfa_sp_create): per-stage kernels over a band of grid rows
   long long spin_test_budget;   // armed by lfa_debug_spin_test (>= 0): the next forward's flag waits
 };
 
@@ -73,6 +74,10 @@ void plan(const lfa_config* c, Params* p, Layout* L) {
   p->eps = c->eps;
   p->neg_log2e_over_lam = (float)(-1.4426950408889634 / (double)c->lambda);
   p->spin_budget = lfa::kFlagSpinBudget;
+  p->y0 = 0;
+  p->Hg = c->H;
+  p->Ng = c->H * c->W;
+  p->Vh = nullptr;
   p->n_tiles = lfa::ceil_div(p->N, lfa::kRowTile);
   // about two pass-1 CTAs per SM of a 148-SM part
   const int want = lfa::ceil_div(296, p->U);
@@ -270,7 +275,7 @@ lfa_status lfa_destroy(lfa_handle h) {
 }
 
 lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void* stream) {
-  if (!h || !Q || !V || !O) return LFA_ERR_INVALID_ARG;
+  if (!h || !Q || !V || !O || h->sp) return LFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(V) || !aligned16(O)) return LFA_ERR_INVALID_ARG;
   Params p = h->p;
   p.Q = Q;
@@ -369,7 +374,7 @@ lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host
 
 lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* dO, void* dQ,
                         void* dV, void* stream) {
-  if (!h || !Q || !V || !dO || !dQ || !dV) return LFA_ERR_INVALID_ARG;
+  if (!h || !Q || !V || !dO || !dQ || !dV || h->sp) return LFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dV))
     return LFA_ERR_INVALID_ARG;
   if (h->p.whiten >= 2) return LFA_ERR_UNSUPPORTED;
@@ -514,6 +519,125 @@ int lfa_launches_per_forward(lfa_handle h) {
 const char* lfa_forward_path(lfa_handle h) {
   if (!h) return "invalid";
   return h->path == 1 ? "fused" : "generic";
+}
+
+// ---- sequence split -------------------------------------------------------------------------
+
+}  // extern "C"
+
+namespace {
+
+// The global plan (workspace sized for the whole grid, so any band fits), then the band's shape
+// for the passes: grid rows [y0, y0 + ny), the pass-1 decomposition over the band's tokens.
+lfa_status sp_plan(const lfa_config* c, int y0, int ny, Params* p, Layout* L) {
+  lfa_status st = validate(c);
+  if (st != LFA_OK) return st;
+  if (c->whiten != 0 && c->whiten != 1) return LFA_ERR_UNSUPPORTED;
+  if (y0 < 0 || ny < 1 || y0 + ny > c->H) return LFA_ERR_INVALID_ARG;
+  plan(c, p, L);
+  p->y0 = y0;
+  p->H = ny;
+  p->N = ny * c->W;
+  p->n_tiles = lfa::ceil_div(p->N, lfa::kRowTile);
+  const int want = lfa::ceil_div(296, p->U);
+  int P = want < p->n_tiles ? want : p->n_tiles;
+  if (P < 1) P = 1;
+  p->tiles_per_cta = lfa::ceil_div(p->n_tiles, P);
+  p->P = lfa::ceil_div(p->n_tiles, p->tiles_per_cta);
+  return LFA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t lfa_sp_workspace_size(const lfa_config* cfg, int y0, int ny) {
+  Params p;
+  Layout L;
+  if (sp_plan(cfg, y0, ny, &p, &L) != LFA_OK) return 0;
+  return L.total;
+}
+
+lfa_status lfa_sp_create(const lfa_config* cfg, int y0, int ny, const float* dwc_weight, void* workspace,
+                         size_t workspace_bytes, lfa_handle* out) {
+  if (!out) return LFA_ERR_INVALID_ARG;
+  *out = nullptr;
+  Params p;
+  Layout lay;
+  lfa_status st = sp_plan(cfg, y0, ny, &p, &lay);
+  if (st != LFA_OK) return st;
+  if (!dwc_weight || !workspace || workspace_bytes < lay.total) return LFA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || !aligned16(dwc_weight)) return LFA_ERR_INVALID_ARG;
+  st = ensure_attributes();
+  if (st != LFA_OK) return st;
+  lfa_ctx* h = new (std::nothrow) lfa_ctx;
+  if (!h) return LFA_ERR_INVALID_ARG;
+  memset(h, 0, sizeof(*h));
+  h->cfg = *cfg;
+  h->p = p;
+  h->lay = lay;
+  h->ws = static_cast<unsigned char*>(workspace);
+  h->ws_bytes = workspace_bytes;
+  h->spin_test_budget = -1;
+  bind(&h->p, h->lay, h->ws);
+  h->p.dwc = dwc_weight;
+  h->path = 0;
+  h->sp = 1;
+  *out = h;
+  return LFA_OK;
+}
+
+int lfa_sp_partial_size(lfa_handle h) { return (h && h->sp) ? h->p.part_stride : 0; }
+
+lfa_status lfa_sp_pool(lfa_handle h, const void* Q_local, float* L_partial, void* stream) {
+  if (!h || !h->sp || !Q_local || !L_partial || !aligned16(Q_local) || !aligned16(L_partial))
+    return LFA_ERR_INVALID_ARG;
+  Params p = h->p;
+  p.Q = Q_local;
+  p.L = L_partial;
+  return lfa::launch_pool(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? LFA_OK : LFA_ERR_CUDA;
+}
+
+lfa_status lfa_sp_pass1(lfa_handle h, const void* Q_local, const void* V_local, const float* L_full,
+                        double* partial_out, void* stream) {
+  if (!h || !h->sp || !Q_local || !V_local || !L_full || !partial_out) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(Q_local) || !aligned16(V_local) || !aligned16(L_full) || !aligned16(partial_out))
+    return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = h->p;
+  p.Q = Q_local;
+  p.V = V_local;
+  const size_t nL = (size_t)p.U * p.m * p.d;
+  if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (cudaMemcpyAsync(p.L, L_full, nL * sizeof(float), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return LFA_ERR_CUDA;
+  if (lfa::launch_generic_ns(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::launch_generic_pass1_reduce(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (cudaMemcpyAsync(partial_out, p.red, sizeof(double) * (size_t)p.U * p.part_stride, cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return LFA_ERR_CUDA;
+  h->have_forward = 0;   // the band's context is not a whole forward: no backward from it
+  return LFA_OK;
+}
+
+lfa_status lfa_sp_pass2(lfa_handle h, const void* Q_local, const void* V_local, const void* V_halo,
+                        const double* partial_total, void* O_local, void* stream) {
+  if (!h || !h->sp || !Q_local || !V_local || !partial_total || !O_local) return LFA_ERR_INVALID_ARG;
+  const bool need_halo = h->p.y0 > 0 || h->p.y0 + h->p.H < h->p.Hg;
+  if (need_halo && !V_halo) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(Q_local) || !aligned16(V_local) || !aligned16(O_local) || !aligned16(partial_total) ||
+      (V_halo && !aligned16(V_halo)))
+    return LFA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Params p = h->p;
+  p.Q = Q_local;
+  p.V = V_local;
+  p.O = O_local;
+  p.Vh = V_halo;
+  if (cudaMemcpyAsync(p.red, partial_total, sizeof(double) * (size_t)p.U * p.part_stride, cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return LFA_ERR_CUDA;
+  return lfa::launch_generic_finish(p, st) == cudaSuccess ? LFA_OK : LFA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -62,10 +62,14 @@ __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
   const int Y0 = (l / Wr) * p.r, X0 = (l % Wr) * p.r;
   const T* q = static_cast<const T*>(p.Q) + (size_t)u * p.N * p.d;
   const float inv = 1.0f / float(p.r * p.r);
+  // window rows outside this call's band of grid rows (sequence split) contribute nothing here
   for (int k = lane; k < p.d; k += 32) {
     float acc = 0.f;
-    for (int dy = 0; dy < p.r; ++dy)
-      for (int dx = 0; dx < p.r; ++dx) acc += to_f(q[((size_t)(Y0 + dy) * p.W + X0 + dx) * p.d + k]);
+    for (int dy = 0; dy < p.r; ++dy) {
+      const int yl = Y0 + dy - p.y0;
+      if (yl < 0 || yl >= p.H) continue;
+      for (int dx = 0; dx < p.r; ++dx) acc += to_f(q[((size_t)yl * p.W + X0 + dx) * p.d + k]);
+    }
     p.L[((size_t)u * p.m + l) * p.d + k] = acc * inv;
   }
 }
@@ -392,7 +396,7 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   float* mus = As + m * d;      // [m]
   float* ss = mus + m;          // [m]
   const double* red = p.red + (size_t)u * p.part_stride;
-  const double invN = 1.0 / double(p.N);
+  const double invN = 1.0 / double(p.Ng);
   for (int j = t; j < m; j += blockDim.x) {
     const double mu = red[j] * invN;
     double var = red[m + j] * invN - mu * mu;
@@ -512,7 +516,7 @@ __global__ void __launch_bounds__(kThreads) k_rb_cov(Params p) {
   const int u = blockIdx.y, e = blockIdx.x * blockDim.x + threadIdx.x, m = p.m;
   if (e >= m * m) return;
   const double* red = p.red + (size_t)u * p.part_stride;
-  const double invN = 1.0 / double(p.N);
+  const double invN = 1.0 / double(p.Ng);
   const int j = e / m, k = e % m;
   const double cj = red[j] * invN, ck = red[k] * invN;
   p.Y[(size_t)u * m * m + e] = (float)(red[2 * m + m * p.d + p.d + e] * invN - cj * ck);
@@ -626,7 +630,7 @@ __global__ void __launch_bounds__(kThreads) k_rb_finish(Params p) {
   for (int e = t; e < m * d; e += blockDim.x) As[e] = p.A[(size_t)u * m * d + e];
   __syncthreads();
   const double* red = p.red + (size_t)u * p.part_stride;
-  const double invN = 1.0 / double(p.N);
+  const double invN = 1.0 / double(p.Ng);
   const float* Xg = p.X + (size_t)u * m * m;
   const int j0 = c * 16;
   for (int e = t; e < 16 * d; e += blockDim.x) {
@@ -724,13 +728,17 @@ __global__ void __launch_bounds__(kThreads) k_pass2(Params p) {
                       acc[x][3] + bs[4 * kb + 3]};
 #pragma unroll
         for (int a = 0; a < 3; ++a) {
-          const int yy = gy + a - 1;
-          if (yy < 0 || yy >= p.H) continue;
+          // local row yy, global row p.y0 + yy; the rows just outside a band come from the halo
+          const int yy = gy + a - 1, yg = p.y0 + yy;
+          if (yg < 0 || yg >= p.Hg) continue;
+          const T* vrow = (yy >= 0 && yy < p.H)
+                              ? Vg + (size_t)yy * p.W * d
+                              : static_cast<const T*>(p.Vh) + ((size_t)u * 2 + (yy < 0 ? 0 : 1)) * p.W * d;
 #pragma unroll
           for (int b = 0; b < 3; ++b) {
             const int xx = gx + b - 1;
             if (xx < 0 || xx >= p.W) continue;
-            const float4 v = load4(Vg + ((size_t)yy * p.W + xx) * d + 4 * kb);
+            const float4 v = load4(vrow + (size_t)xx * d + 4 * kb);
             o[0] = fmaf(wt[0][a * 3 + b], v.x, o[0]);
             o[1] = fmaf(wt[1][a * 3 + b], v.y, o[1]);
             o[2] = fmaf(wt[2][a * 3 + b], v.z, o[2]);
@@ -807,11 +815,9 @@ void reading_b_t(const Params& p, cudaStream_t st) {
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
 
-// Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b.
-template <typename T>
-void context_t(const Params& p, cudaStream_t st) {
-  const int U = p.U, m = p.m, d = p.d;
-  k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
+// W, alpha and the Newton-Schulz chain from the landmarks in the workspace.
+void ns_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m;
   if (m <= kSmallM) {
     launch_ns_tc(p, st);
   } else {
@@ -832,6 +838,14 @@ void context_t(const Params& p, cudaStream_t st) {
     k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
     k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
   }
+}
+
+// Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b.
+template <typename T>
+void context_t(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m, d = p.d;
+  k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
+  ns_t(p, st);
   if (p.whiten == 3) {
     reading_b_t<T>(p, st);
     return;
@@ -913,6 +927,21 @@ cudaError_t launch_generic_context(const Params& p, cudaStream_t st) {
 cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st) {
   if (p.dtype == LFA_BF16) pass1_reduce_t<__nv_bfloat16>(p, st);
   else pass1_reduce_t<float>(p, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_generic_ns(const Params& p, cudaStream_t st) {
+  ns_t(p, st);
+  return cudaGetLastError();
+}
+
+// The combine from the fp64 totals in the workspace (mu, s, A, M, M', b), then pass 2.
+cudaError_t launch_generic_finish(const Params& p, cudaStream_t st) {
+  k_combine_finish<<<dim3(p.n_chunks, p.U), kThreads, (size_t)(p.m * p.d + 2 * p.m) * sizeof(float), st>>>(p);
+  if (p.dtype == LFA_BF16)
+    k_pass2<__nv_bfloat16><<<dim3(p.P, p.U), kThreads, generic_smem_pass2(p.m, p.d), st>>>(p);
+  else
+    k_pass2<float><<<dim3(p.P, p.U), kThreads, generic_smem_pass2(p.m, p.d), st>>>(p);
   return cudaGetLastError();
 }
 

@@ -81,6 +81,11 @@ struct Params {
   float* dbgC;
   float* dbgS;   // optional: the column shift subtracted before bf16 rounding, per entry, fp32 [N][m]
   int dbg_unit;
+  // sequence split (per-stage kernels only): this call holds grid rows [y0, y0 + H) of every unit's
+  // Hg x W grid (Ng = Hg W tokens enter the column statistics); Vh, when not null, holds the V rows
+  // y0 - 1 and y0 + H of every unit ([U][2][W][d], zero rows outside the grid) for DWC
+  int y0, Hg, Ng;
+  const void* Vh;
   // fused kernel: bound (SM cycles) on its waits for flags that other CTAs set; with spin_test the
   // landmark waits look for one landmark more than exist, so every one of them runs out (tests)
   long long spin_budget;
@@ -142,6 +147,8 @@ cudaError_t launch_ns_tc(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_context(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st);
+cudaError_t launch_generic_ns(const Params& p, cudaStream_t st);
+cudaError_t launch_generic_finish(const Params& p, cudaStream_t st);
 cudaError_t launch_backward(const BwdParams& b, cudaStream_t st);
 size_t backward_smem_main(int d);
 cudaError_t backward_set_attributes();

@@ -71,6 +71,12 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_debug_trace": (ci, [vp, vp]),
         "lfa_fused_grid": (ci, [vp]),
         "lfa_debug_selftest": (ci, [ci, vp, vp, vp, ci, vp, ci, vp, vp]),
+        "lfa_sp_workspace_size": (sz, [cfgp, ci, ci]),
+        "lfa_sp_create": (ci, [cfgp, ci, ci, vp, vp, sz, ctypes.POINTER(vp)]),
+        "lfa_sp_partial_size": (ci, [vp]),
+        "lfa_sp_pool": (ci, [vp, vp, vp, vp]),
+        "lfa_sp_pass1": (ci, [vp, vp, vp, vp, vp, vp]),
+        "lfa_sp_pass2": (ci, [vp, vp, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -322,6 +328,68 @@ class LaplacianNystromAttention:
         _check(self.lib.lfa_debug_context(self.handle, int(unit), _ptr(L), _ptr(X), _ptr(mu), _ptr(s),
                                           _stream(stream)), "lfa_debug_context")
         return L, X, mu, s
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            self.lib.lfa_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class SeqSplitBand:
+    """A band of grid rows [y0, y0 + ny) of every unit (lfa_sp_create): the library's three band
+    calls. Q, V, O of the band are [B, heads, ny * W, d] in the config's dtype on one device."""
+
+    def __init__(self, cfg: Config, y0: int, ny: int, dwc_weight: torch.Tensor, device: str = "cuda"):
+        self.lib = load()
+        self.cfg = cfg
+        self.y0, self.ny = int(y0), int(ny)
+        self.device = torch.device(device)
+        if self.device.type == "cuda" and self.device.index is None:
+            self.device = torch.device("cuda", torch.cuda.current_device())
+        self.dtype = torch.bfloat16 if cfg.dtype == LFA_BF16 else torch.float32
+        self.m = (cfg.H // cfg.r) * (cfg.W // cfg.r)
+        self.shape = (cfg.B, cfg.heads, self.ny * cfg.W, cfg.d)
+        self.weight = dwc_weight.to(self.device, torch.float32).contiguous()
+        _require(self.weight, "dwc_weight", (cfg.heads, cfg.d, 3, 3), torch.float32, self.device)
+        nbytes = int(self.lib.lfa_sp_workspace_size(ctypes.byref(cfg), self.y0, self.ny))
+        if nbytes == 0:
+            raise LfaError(LFA_ERR_INVALID_ARG, "lfa_sp_workspace_size")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        _check(self.lib.lfa_sp_create(ctypes.byref(cfg), self.y0, self.ny, self.weight.data_ptr(),
+                                      self.workspace.data_ptr(), nbytes, ctypes.byref(h)), "lfa_sp_create")
+        self.handle = h
+        self.S = int(self.lib.lfa_sp_partial_size(h))
+
+    def pool(self, Q: torch.Tensor, stream=None) -> torch.Tensor:
+        _require(Q, "Q", self.shape, self.dtype, self.device)
+        L = torch.empty((self.cfg.B, self.cfg.heads, self.m, self.cfg.d), dtype=torch.float32, device=self.device)
+        _check(self.lib.lfa_sp_pool(self.handle, _ptr(Q), _ptr(L), _stream(stream)), "lfa_sp_pool")
+        return L
+
+    def pass1(self, Q: torch.Tensor, V: torch.Tensor, L: torch.Tensor, stream=None) -> torch.Tensor:
+        for name, t in (("Q", Q), ("V", V)):
+            _require(t, name, self.shape, self.dtype, self.device)
+        _require(L, "L", (self.cfg.B, self.cfg.heads, self.m, self.cfg.d), torch.float32, self.device)
+        part = torch.empty((self.cfg.B, self.cfg.heads, self.S), dtype=torch.float64, device=self.device)
+        _check(self.lib.lfa_sp_pass1(self.handle, _ptr(Q), _ptr(V), _ptr(L), _ptr(part), _stream(stream)),
+               "lfa_sp_pass1")
+        return part
+
+    def pass2(self, Q, V, halo, part, O, stream=None):
+        for name, t in (("Q", Q), ("V", V), ("O", O)):
+            _require(t, name, self.shape, self.dtype, self.device)
+        _require(halo, "halo", (self.cfg.B, self.cfg.heads, 2, self.cfg.W, self.cfg.d), self.dtype, self.device)
+        _require(part, "partials", (self.cfg.B, self.cfg.heads, self.S), torch.float64, self.device)
+        _check(self.lib.lfa_sp_pass2(self.handle, _ptr(Q), _ptr(V), _ptr(halo), _ptr(part), _ptr(O),
+                                     _stream(stream)), "lfa_sp_pass2")
+        return O
 
     def close(self) -> None:
         if getattr(self, "handle", None):
