@@ -86,7 +86,7 @@ typedef struct {
                      1/N of one unit). 3 ("Reading B"): the columns of the whole Nystrom matrix
                      G^ = C X C^T are whitened instead of those of C, O_attn = G~ V, in the
                      factored form (C - 1 c-^T) X C^T D^-1/2 V + (1/N) 1 1^T V with
-                     D = diag(c_j^T X^T cov(C) X c_j + eps) over key tokens j; needs m <= 64.
+                     D = diag(c_j^T X^T cov(C) X c_j + eps) over key tokens j; any m.
                      whiten = 2 and 3 run the per-stage kernels, forward only. */
 } lfa_config;
 
@@ -263,10 +263,12 @@ lfa_status lfa_debug_selftest(int mode, const float* A, const float* B, float* D
  * the hook off. Host-only; returns LFA_ERR_INVALID_ARG if exactly one event is NULL. */
 lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end);
 
-/* Diagnostic timeline of the fused kernel: with a non-NULL device buffer of
- * grid * 32 uint64 entries, later forwards on this handle record %globaltimer (ns) stamps at
- * phase boundaries of every CTA (slot 0 start, 1 pooled, 2 grid barrier passed, then per
- * role; 15 end; 13 / 14 the SM clock64 at start / end). NULL turns it off. Host-only. */
+/* Diagnostic timeline of the fused kernel, present only in a library built with
+ * -DLFA_PHASE_TRACE (python -m laplacian_nystr_attention_avg_b200.build --phase-trace); the
+ * default build returns LFA_ERR_UNSUPPORTED and its kernels carry no stamp code. With a non-NULL
+ * device buffer of grid * 32 uint64 entries, later forwards on this handle record %globaltimer
+ * (ns) stamps at phase boundaries of every CTA (slot 0 start, 1 landmarks pooled, then per role;
+ * 15 end; 13 / 14 the SM clock64 at start / end). NULL turns it off. Host-only. */
 lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf);
 
 /* Name of the kernel the timing hook brackets for this handle's config (static string). */

@@ -1,6 +1,10 @@
 """Builds liblfa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-Usage: python -m laplacian_nystr_attention_avg_b200.build [--verbose]
+Usage: python -m laplacian_nystr_attention_avg_b200.build [--verbose] [--force] [--phase-trace]
+
+--phase-trace compiles the fused kernel's phase timeline stamps in (-DLFA_PHASE_TRACE; see
+lfa_debug_trace). The flags of the last build are kept beside the library, so a build with other
+flags is never taken as up to date.
 """
 from __future__ import annotations
 
@@ -15,6 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblfa.so")
+STAMP = LIB + ".flags"
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr"]
@@ -31,8 +36,18 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def up_to_date() -> bool:
+def _flag_line(extra) -> str:
+    return " ".join([*ARCH, *FLAGS, *extra])
+
+
+def up_to_date(extra=()) -> bool:
     if not os.path.exists(LIB):
+        return False
+    if os.path.exists(STAMP):
+        with open(STAMP) as f:
+            if f.read().strip() != _flag_line(extra):
+                return False
+    elif extra:
         return False
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) \
@@ -41,7 +56,7 @@ def up_to_date() -> bool:
 
 
 def build(verbose: bool = False, force: bool = False, extra=()) -> str:
-    if not force and up_to_date():
+    if not force and up_to_date(extra):
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
@@ -60,8 +75,11 @@ def build(verbose: bool = False, force: bool = False, extra=()) -> str:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(_flag_line(extra) + "\n")
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv))
+    extra = ("-DLFA_PHASE_TRACE",) if "--phase-trace" in sys.argv else ()
+    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv, extra=extra))

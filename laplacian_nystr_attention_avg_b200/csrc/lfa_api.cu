@@ -49,7 +49,6 @@ lfa_status validate(const lfa_config* c) {
   if (c->dtype != LFA_F32 && c->dtype != LFA_BF16) return LFA_ERR_UNSUPPORTED;
   const long long m = (long long)(c->H / c->r) * (c->W / c->r);
   if (m > lfa::kMaxM) return LFA_ERR_UNSUPPORTED;
-  if (c->whiten == 3 && m > lfa::kSmallM) return LFA_ERR_UNSUPPORTED;   // Reading B: K tiles of 64
   const long long rows = (long long)c->B * c->heads * c->H * c->W;
   if (rows * c->d >= (1ll << 31)) return LFA_ERR_UNSUPPORTED;   // element index fits int32
   return LFA_OK;
@@ -500,8 +499,13 @@ lfa_status lfa_set_profile_events(lfa_handle h, void* ev_begin, void* ev_end) {
 
 lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf) {
   if (!h) return LFA_ERR_INVALID_ARG;
+#ifdef LFA_PHASE_TRACE
   h->p.trace = dev_buf;
   return LFA_OK;
+#else
+  (void)dev_buf;
+  return LFA_ERR_UNSUPPORTED;
+#endif
 }
 
 const char* lfa_dominant_kernel(lfa_handle h) {

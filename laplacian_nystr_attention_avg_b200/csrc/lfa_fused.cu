@@ -137,12 +137,18 @@ struct FusedArgs {
   unsigned char wj0[kWarps], wlt[kWarps], padw[2];
 };
 
+// Phase timeline stamps (compiled in only with -DLFA_PHASE_TRACE; lfa_debug_trace arms them).
+#ifdef LFA_PHASE_TRACE
 __device__ __forceinline__ void trace_mark(const Params& p, int slot) {
   if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 32 + slot] = globaltimer();
 }
 __device__ __forceinline__ void trace_clock(const Params& p, int slot) {
   if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 32 + slot] = (unsigned long long)clock64();
 }
+#else
+__device__ __forceinline__ void trace_mark(const Params&, int) {}
+__device__ __forceinline__ void trace_clock(const Params&, int) {}
+#endif
 
 // Row partition. Each unit's rows are cut into nchu 128-row chunks (the last one may be short);
 // the T = U nchu chunks of all units, in unit order, are dealt out evenly to the P = G - U row
@@ -551,9 +557,9 @@ __device__ SolverInfo solver_cta(const Params& p, const FusedArgs& fa, unsigned 
 }
 
 // Diagnostics of the unit's solve, ||I - W X_T||_F, by one more product of the same kind as the
-// Newton-Schulz steps ([W; X_T] times X_T^T, 3xTF32). It runs after M' is published, off the
-// critical path: W is still in the solver's scratch, X_T^T in the combine's (the combine leaves
-// both unchanged).
+// Newton-Schulz steps ([W; X_T] times X_T^T, 3xTF32). It runs right after the chain, while the row
+// CTAs are still in pass 1 (the solver waits for their records anyway): W is still in the solver's
+// scratch and X_T^T where the chain left it.
 __device__ void solver_diagnostics(const Params& p, unsigned char* sm, uint32_t sbase, uint32_t tmem,
                                    uint64_t* bars, int u, const SolverInfo& si) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
@@ -747,9 +753,6 @@ __device__ void segment_shift(const Params& p, const unsigned char* qtile, int n
   __syncthreads();
 }
 
-// Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
-// (bf16, SW128) goes to C slot gc + 1 (chunk gc writes its C tile into slot gc, which held the
-// previous chunk's rows), one barrier for all of them; the first two V chunks go to stages 0, 1.
 // Pass-1 inputs, issued by one thread while the SM is otherwise idle: every Q chunk of this CTA
 // (bf16, SW128) goes to C slot gc + 1 (chunk gc writes its C tile into slot gc, which held the
 // previous chunk's rows), one barrier for all of them; the first two V chunks go to stages 0, 1.
@@ -1124,13 +1127,14 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   }
   if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
   nct = nct < kMaxContrib ? nct : kMaxContrib;
+  // the zero reference shift, read by every thread below: written before the barrier
+  if (t < 64) reinterpret_cast<float*>(sm + kOffZero)[t] = 0.f;
   if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
   __syncthreads();
   trace_mark(p, 7);
   float* Mp = reinterpret_cast<float*>(sm + kOffMpf);   // M' fp32 [64][68] (row l)
   unsigned char* img = sm + kOffMp;
   const float* shift = reinterpret_cast<const float*>(sm + kOffZero);   // the zero reference
-  if (t < 64) reinterpret_cast<float*>(sm + kOffZero)[t] = 0.f;
   // X^T (row j, column l), zero outside m x m: the product below reads it along l
   {
     constexpr int kNX = 64 * 64 / kFT;   // X entries per thread, all loads issued first

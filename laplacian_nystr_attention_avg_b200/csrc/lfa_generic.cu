@@ -455,31 +455,46 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Reading B (whiten = 3, m <= 64): whitening of the columns of the whole Nystrom matrix
+// Reading B (whiten = 3): whitening of the columns of the whole Nystrom matrix
 // G^ = C X C^T (LaplacianFormer note, §关键设计 1 applied to §关键设计 2's G^), one column per
 // key token j, in factored form. With c- the column mean of C and S = cov(C) (population):
 //   mean_i G^_ij = c-^T X c_j,  var_j = c_j^T K c_j with K = X^T S X,
 //   O_attn = (C - 1 c-^T) X C^T D^-1/2 V + (1/N) 1 (1^T V),  D = diag(var_j + eps),
 // so pass 2 runs unchanged with M' = X C^T D^-1/2 V and b = (1/N) sum_i v_i - M'^T c-.
-// Steps: k_rb_gram (C^T C partials, into the tail of the pass-1 partial record), the pass-1
-// reduction, k_rb_cov (S in fp64), K = X^T (S X) by two batched products, k_rb_pass (var_j per
-// token, partials of C^T D^-1/2 V), k_rb_reduce, k_rb_finish (M', b).
+// Steps: k_rb_gram (C^T C partials, into the tail of the pass-1 partial record, one 64 x 64 block
+// pair of landmarks per CTA), the pass-1 reduction, k_rb_cov (S in fp64), K = X^T (S X) by two
+// batched products, k_rb_pass (var_j per token with K streamed in 64 x 64 blocks, partials of
+// C^T D^-1/2 V), k_rb_reduce, k_rb_finish (M', b). Any m up to the library's maximum.
 // ---------------------------------------------------------------------------------------
-constexpr int kRbCs = 64 + 4;   // row stride (floats) of the 64-landmark C and K tiles
+constexpr int kRbKs = 64 + 4;   // row stride (floats) of a staged 64 x 64 block of K
 
-// C^T C over the CTA's rows (the same row partition as pass 1); thread t owns the 4 x 4 block
-// rows 4 (t / 16) .., columns 4 (t % 16) .. of the 64 x 64 product.
+// Upper-triangle block pair (bj <= bk) number `idx` of an nb x nb grid of 64 x 64 blocks.
+__device__ __forceinline__ void block_pair(int idx, int nb, int& bj, int& bk) {
+  bj = 0;
+  while (idx >= nb - bj) {
+    idx -= nb - bj;
+    ++bj;
+  }
+  bk = bj + idx;
+}
+
+// C^T C over the CTA's rows (the same row partition as pass 1), one 64 x 64 block pair (bj, bk) per
+// blockIdx.z: C is formed for those two landmark blocks only, and thread t owns the 4 x 4 block rows
+// 64 bj + 4 (t / 16) .., columns 64 bk + 4 (t % 16) ..; the mirror block is written too.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_rb_gram(Params p) {
   extern __shared__ float4 smem_f4[];
   float* sm = reinterpret_cast<float*>(smem_f4);
   const int m = p.m, d = p.d, ds = d + 4;
-  float* Ls = sm;                    // [64][ds]
-  float* Qs = Ls + 64 * ds;          // [64][ds]
-  float* Cs = Qs + kRowTile * ds;    // [64][kRbCs]
+  const int mpl = round_up(m, 64), cs = mpl + 4, nb = mpl / 64;
+  float* Ls = sm;                    // [mpl][ds]
+  float* Qs = Ls + mpl * ds;         // [64][ds]
+  float* Cs = Qs + kRowTile * ds;    // [64][cs]
   const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x, jb = t >> 4, kb = t & 15;
+  int bj, bk;
+  block_pair(blockIdx.z, nb, bj, bk);
   const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
-  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, 64, d);
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
   float acc[4][4] = {};
   const int tile0 = pc * p.tiles_per_cta;
   const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
@@ -489,11 +504,12 @@ __global__ void __launch_bounds__(kThreads) k_rb_gram(Params p) {
     __syncthreads();
     stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
     __syncthreads();
-    cross_tile(Qs, Ls, Cs, d, 0, m, kRbCs, p.neg_log2e_over_lam, valid);
+    cross_tile(Qs, Ls, Cs, d, 64 * bj, m, cs, p.neg_log2e_over_lam, valid);
+    if (bk != bj) cross_tile(Qs, Ls, Cs, d, 64 * bk, m, cs, p.neg_log2e_over_lam, valid);
     __syncthreads();
     for (int i = 0; i < kRowTile; ++i) {
-      const float4 a = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * jb]);
-      const float4 b = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * kb]);
+      const float4 a = *reinterpret_cast<const float4*>(&Cs[i * cs + 64 * bj + 4 * jb]);
+      const float4 b = *reinterpret_cast<const float4*>(&Cs[i * cs + 64 * bk + 4 * kb]);
       const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int x = 0; x < 4; ++x)
@@ -506,8 +522,11 @@ __global__ void __launch_bounds__(kThreads) k_rb_gram(Params p) {
   for (int x = 0; x < 4; ++x)
 #pragma unroll
     for (int y = 0; y < 4; ++y) {
-      const int j = 4 * jb + x, k = 4 * kb + y;
-      if (j < m && k < m) out[j * m + k] = acc[x][y];
+      const int j = 64 * bj + 4 * jb + x, k = 64 * bk + 4 * kb + y;
+      if (j < m && k < m) {
+        out[j * m + k] = acc[x][y];
+        if (bk != bj) out[k * m + j] = acc[x][y];
+      }
     }
 }
 
@@ -526,31 +545,38 @@ __global__ void __launch_bounds__(kThreads) k_rb_cov(Params p) {
   }
 }
 
-// Per 64-row tile: C, var_i = c_i^T K c_i (thread (i = t / 4, t % 4) sums over landmarks
-// j = t % 4 + 4 n), w_i = 1 / sqrt(var_i + eps) (0 past the end), and C^T (w o V) into the
-// P slot of the CTA's partial record (pass 1's records are already reduced).
+// Per 64-row tile: C (all landmarks), var_i = c_i^T K c_i by a blocked product C K (K streamed in
+// 64 x 64 blocks through shared memory; thread (t / 16, t % 16) owns a 4 x 4 block of each output
+// block and keeps its share of sum_k C_ik (C K)_ik), w_i = 1 / sqrt(var_i + eps) (0 past the end), and
+// C^T (w o V) into the P slot of the CTA's partial record (pass 1's records are already reduced):
+// thread (t / (d / 4), t % (d / 4)) owns a 4 x 4 block of every 64-landmark block of the m x d sum.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_rb_pass(Params p) {
   extern __shared__ float4 smem_f4[];
   float* sm = reinterpret_cast<float*>(smem_f4);
   const int m = p.m, d = p.d, ds = d + 4;
-  float* Ls = sm;                    // [64][ds]
-  float* Qs = Ls + 64 * ds;          // [64][ds]
+  const int mpl = round_up(m, 64), cs = mpl + 4, nb = mpl / 64;
+  float* Ls = sm;                    // [mpl][ds]
+  float* Qs = Ls + mpl * ds;         // [64][ds]
   float* Vs = Qs + kRowTile * ds;    // [64][ds]
-  float* Cs = Vs + kRowTile * ds;    // [64][kRbCs]
-  float* Ks = Cs + kRowTile * kRbCs; // [64][kRbCs]
-  float* wr = Ks + 64 * kRbCs;       // [64]
+  float* Cs = Vs + kRowTile * ds;    // [64][cs]
+  float* Ks = Cs + kRowTile * cs;    // [64][kRbKs] one block of K
+  float* wr = Ks + 64 * kRbKs;       // [64]
   const int u = blockIdx.y, pc = blockIdx.x, t = threadIdx.x;
   const T* Qg = static_cast<const T*>(p.Q) + (size_t)u * p.N * d;
   const T* Vg = static_cast<const T*>(p.V) + (size_t)u * p.N * d;
-  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, 64, d);
-  for (int e = t; e < 64 * 64; e += blockDim.x) {
-    const int j = e >> 6, k = e & 63;
-    Ks[j * kRbCs + k] = (j < m && k < m) ? p.Y[(size_t)u * m * m + j * m + k] : 0.f;
-  }
-  const int nbk = d / 4, nb = 16 * nbk;   // 4 x 4 blocks of the 64 x d product
-  const int jb = t / nbk, kb = t % nbk;
-  float acc[4][4] = {};
+  const float* Kg = p.Y + (size_t)u * m * m;
+  stage_landmarks(p.L + (size_t)u * m * d, Ls, m, mpl, d);
+  const int ib = t >> 4, kk = t & 15;                     // C K blocks
+  const int nbk = d / 4, nt = 16 * nbk;                   // C^T (w o V) blocks
+  const int jb2 = t / nbk, kb2 = t % nbk;
+  float acc2[4][4][4];
+#pragma unroll
+  for (int b = 0; b < 4; ++b)
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc2[b][x][y] = 0.f;
   const int tile0 = pc * p.tiles_per_cta;
   const int tile1 = min(tile0 + p.tiles_per_cta, p.n_tiles);
   for (int tile = tile0; tile < tile1; ++tile) {
@@ -560,26 +586,43 @@ __global__ void __launch_bounds__(kThreads) k_rb_pass(Params p) {
     stage_rows(Qg + (size_t)row0 * d, Qs, d, valid);
     stage_rows(Vg + (size_t)row0 * d, Vs, d, valid);
     __syncthreads();
-    cross_tile(Qs, Ls, Cs, d, 0, m, kRbCs, p.neg_log2e_over_lam, valid);
-    __syncthreads();
-    {
-      const int i = t >> 2, j0 = t & 3;
-      float v = 0.f;
-      for (int j = j0; j < 64; j += 4) {
-        float y = 0.f;
-        for (int k = 0; k < 64; k += 4) {
-          const float4 kk = *reinterpret_cast<const float4*>(&Ks[j * kRbCs + k]);
-          const float4 cc = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + k]);
-          y = fmaf(kk.x, cc.x, y);
-          y = fmaf(kk.y, cc.y, y);
-          y = fmaf(kk.z, cc.z, y);
-          y = fmaf(kk.w, cc.w, y);
+    for (int j0 = 0; j0 < mpl; j0 += 64) cross_tile(Qs, Ls, Cs, d, j0, m, cs, p.neg_log2e_over_lam, valid);
+    float vp[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int kbk = 0; kbk < nb; ++kbk) {
+      float acc[4][4] = {};
+      for (int jbk = 0; jbk < nb; ++jbk) {
+        __syncthreads();   // C is complete; the previous K block is no longer read
+        for (int e = t; e < 64 * 64; e += blockDim.x) {
+          const int j = e >> 6, k = e & 63, gj = 64 * jbk + j, gk = 64 * kbk + k;
+          Ks[j * kRbKs + k] = (gj < m && gk < m) ? Kg[(size_t)gj * m + gk] : 0.f;
         }
-        v = fmaf(Cs[i * kRbCs + j], y, v);
+        __syncthreads();
+        for (int j = 0; j < 64; ++j) {
+          const float4 b = *reinterpret_cast<const float4*>(&Ks[j * kRbKs + 4 * kk]);
+          const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const float a = Cs[(4 * ib + x) * cs + 64 * jbk + j];
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(a, bv[y], acc[x][y]);
+          }
+        }
       }
-      v += __shfl_xor_sync(0xffffffffu, v, 1);
-      v += __shfl_xor_sync(0xffffffffu, v, 2);
-      if (j0 == 0) wr[i] = i < valid ? 1.f / sqrtf(v + p.eps) : 0.f;
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) vp[x] = fmaf(Cs[(4 * ib + x) * cs + 64 * kbk + 4 * kk + y], acc[x][y], vp[x]);
+    }
+    // rows 4 ib .. are shared by the 16 threads with the same ib (consecutive lanes)
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+      for (int o = 8; o > 0; o >>= 1) vp[x] += __shfl_xor_sync(0xffffffffu, vp[x], o);
+    if (kk == 0) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int i = 4 * ib + x;
+        wr[i] = i < valid ? 1.f / sqrtf(vp[x] + p.eps) : 0.f;
+      }
     }
     __syncthreads();
     for (int e = t; e < kRowTile * d; e += blockDim.x) {
@@ -587,26 +630,35 @@ __global__ void __launch_bounds__(kThreads) k_rb_pass(Params p) {
       Vs[i * ds + c] *= wr[i];
     }
     __syncthreads();
-    if (t < nb) {
+    if (t < nt) {
       for (int i = 0; i < kRowTile; ++i) {
-        const float4 c = *reinterpret_cast<const float4*>(&Cs[i * kRbCs + 4 * jb]);
-        const float4 v = *reinterpret_cast<const float4*>(&Vs[i * ds + 4 * kb]);
-        const float cc[4] = {c.x, c.y, c.z, c.w}, vv[4] = {v.x, v.y, v.z, v.w};
+        const float4 v = *reinterpret_cast<const float4*>(&Vs[i * ds + 4 * kb2]);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
+        for (int b = 0; b < 4; ++b) {
+          if (b >= nb) break;
+          const float4 c = *reinterpret_cast<const float4*>(&Cs[i * cs + 64 * b + 4 * jb2]);
+          const float cc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(cc[x], vv[y], acc[x][y]);
+          for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) acc2[b][x][y] = fmaf(cc[x], vv[y], acc2[b][x][y]);
+        }
       }
     }
   }
-  if (t < nb) {
+  if (t < nt) {
     float* out = p.part + ((size_t)u * p.P + pc) * p.part_stride + 2 * m;
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int j = 4 * jb + x;
-      if (j < m)
+    for (int b = 0; b < 4; ++b) {
+      if (b >= nb) break;
 #pragma unroll
-        for (int y = 0; y < 4; ++y) out[j * d + 4 * kb + y] = acc[x][y];
+      for (int x = 0; x < 4; ++x) {
+        const int j = 64 * b + 4 * jb2 + x;
+        if (j < m)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) out[j * d + 4 * kb2 + y] = acc2[b][x][y];
+      }
     }
   }
 }
@@ -793,24 +845,31 @@ void pass1_reduce_t(const Params& p, cudaStream_t st) {
   k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), p.U), kThreads, 0, st>>>(p);
 }
 
-size_t rb_gram_smem(int d) { return sizeof(float) * (size_t)(2 * 64 * (d + 4) + 64 * kRbCs); }
-size_t rb_pass_smem(int d) { return sizeof(float) * (size_t)(3 * 64 * (d + 4) + 2 * 64 * kRbCs + 64); }
+size_t rb_gram_smem(int m, int d) {
+  const int mpl = round_up(m, 64);
+  return sizeof(float) * ((size_t)mpl * (d + 4) + 64 * (d + 4) + 64 * (size_t)(mpl + 4));
+}
+size_t rb_pass_smem(int m, int d) {
+  const int mpl = round_up(m, 64);
+  return sizeof(float) * ((size_t)mpl * (d + 4) + 2 * 64 * (d + 4) + 64 * (size_t)(mpl + 4) + 64 * kRbKs + 64);
+}
 
-// Reading B after the Newton-Schulz chain (m <= 64, so X came from k_ns_small and the Y / Xb
-// buffers are free): every stage up to M' and b.
+// Reading B after the Newton-Schulz chain (the Y / Xb buffers are free once X is in p.X): every stage
+// up to M' and b.
 template <typename T>
 void reading_b_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   const size_t mm = (size_t)m * m;
   pass1_t<T>(p, st);
-  k_rb_gram<T><<<dim3(p.P, U), kThreads, rb_gram_smem(d), st>>>(p);
+  const int nb = round_up(m, 64) / 64;
+  k_rb_gram<T><<<dim3(p.P, U, nb * (nb + 1) / 2), kThreads, rb_gram_smem(m, d), st>>>(p);
   k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
   k_rb_cov<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
   const MmJob sx{p.Y, mm, p.X, mm, nullptr, 0, p.Xb, mm, 1.f, 0.f, 0.f, 0, 0};   // Xb = S X
   launch_mm(&sx, 1, m, U, st);
   const MmJob k{p.X, mm, p.Xb, mm, nullptr, 0, p.Y, mm, 1.f, 0.f, 0.f, 1, 0};     // Y = X^T (S X)
   launch_mm(&k, 1, m, U, st);
-  k_rb_pass<T><<<dim3(p.P, U), kThreads, rb_pass_smem(d), st>>>(p);
+  k_rb_pass<T><<<dim3(p.P, U), kThreads, rb_pass_smem(m, d), st>>>(p);
   k_rb_reduce<<<dim3(ceil_div(m * d, kThreads), U), kThreads, 0, st>>>(p);
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
@@ -889,6 +948,7 @@ cudaError_t generic_set_attributes() {
   LFA_ATTR((k_pass1<__nv_bfloat16, 2>));
   LFA_ATTR((k_pass1<__nv_bfloat16, 4>));
   LFA_ATTR(k_combine_finish);
+  LFA_ATTR(k_rb_finish);
   LFA_ATTR(k_rb_gram<float>);
   LFA_ATTR(k_rb_gram<__nv_bfloat16>);
   LFA_ATTR(k_rb_pass<float>);

@@ -38,7 +38,8 @@ class Workload:
     d: channels per head. r: landmark pooling window (m = (H/r)*(W/r)).
     lam: Laplacian kernel scale lambda. eps: the regulariser added to W and
     inside the whitening square root. T: Newton-Schulz steps. dtype: 'f32' or
-    'bf16' (storage type of Q, V, O; arithmetic is fp32). qdist: 'normal' or
+    'bf16' (storage type of Q, V, O; the library's arithmetic is set by the path, not by
+    this field). qdist: 'normal' or
     'student_t3'. backward: whether the workload includes lfa_backward.
     """
 

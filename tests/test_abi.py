@@ -57,7 +57,7 @@ def _cfg(**kw):
     (dict(B=0), lfa.LFA_ERR_INVALID_ARG),
     (dict(r=0), lfa.LFA_ERR_INVALID_ARG),
     (dict(whiten=4), lfa.LFA_ERR_INVALID_ARG),          # 0 raw, 1 per unit, 2 batch-pooled, 3 reading B
-    (dict(whiten=3, H=64, W=64, r=4), lfa.LFA_ERR_UNSUPPORTED),   # reading B needs m <= 64
+    (dict(whiten=3, H=64, W=68, r=4), lfa.LFA_ERR_UNSUPPORTED),   # reading B: m = 272 > 256 too
     (dict(whiten=-1), lfa.LFA_ERR_INVALID_ARG),
     (dict(d=48), lfa.LFA_ERR_UNSUPPORTED),
     (dict(d=128), lfa.LFA_ERR_UNSUPPORTED),
@@ -71,6 +71,12 @@ def test_create_rejects_bad_configs(lib, kw, expect):
     st = lib.lfa_create(ctypes.byref(cfg), 256, 256, 1 << 20, ctypes.byref(h))
     assert st == expect
     assert not h.value
+
+
+def test_reading_b_accepts_the_largest_m(lib):
+    # whiten = 3 streams the landmark covariance in 64 x 64 blocks: m = 256 (and a ragged m) plan
+    for kw in (dict(H=64, W=64, r=4), dict(H=52, W=76, r=4)):
+        assert lfa.workspace_size(_cfg(whiten=3, **kw)) > 0
 
 
 def test_create_rejects_null_and_misaligned(lib):
