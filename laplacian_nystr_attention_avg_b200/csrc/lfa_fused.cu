@@ -64,9 +64,15 @@ constexpr uint32_t kOffC = 0;                                   // 8 x 16 KB C c
 constexpr uint32_t kOffV = kOffC + kMaxChunks * 16384;          // 3 x 16 KB V stages (TMA, SW128)
 constexpr uint32_t kOffQ = kOffV + 2 * 16384;                   // third V stage + 18 KB spare in pass 1
 constexpr uint32_t kOffL = kOffQ + kChunk * kQS * 4;            // landmarks, fp32 [64][68]
+constexpr uint32_t kOffL2 = kOffQ + 16384;                      // pass 1: segment 1's landmarks [64][68]
 constexpr uint32_t kOffMp = kOffL + 64 * kQS * 4;               // M'^T bf16 [64 ch][64 lm] (SW128)
 constexpr uint32_t kOffBv = kOffMp + 8192;                      // b, fp32 [segment][64]
 constexpr uint32_t kOffBar = kOffBv + 512;                      // mbarriers + TMEM address
+// the solver's DWC chunk list lives in the b area: a count and at most 127 chunks, enough for the
+// first 3 chunks of each of kMaxContrib row CTAs (the host caps dwc_take at 3)
+constexpr int kDwcListCap = 127;
+constexpr int kMaxDwcTake = 3;
+static_assert(kMaxDwcTake * kMaxContrib <= kDwcListCap && (1 + kDwcListCap) * 4 <= 512, "DWC list overflows");
 constexpr uint32_t kOffCt = kOffBar + 256;                      // int [32] record offsets
 constexpr uint32_t kOffSr = kOffCt + 128;                       // pass-1 column sums [segment][row half][128]
 constexpr uint32_t kOffRows = kOffSr + 2 * 256 * 4;            // this CTA's row plan (struct Rows)
@@ -89,9 +95,13 @@ constexpr uint32_t kOffWc = kOffBp + kWarps * 8 * 4;            // int [kWarps] 
 constexpr uint32_t kOffImg1 = (kOffWc + kWarps * 4 + 1023) / 1024 * 1024;   // M'^T of segment 1
 // row CTAs' DWC tiles after pass 1: C slot kMaxChunks - 1 and the V / Q / L region, contiguous
 constexpr uint32_t kOffDwcTiles = kOffC + (kMaxChunks - 1) * 16384;
-// solver combine only (no pass 2 there): M' fp32 [64][68] and a zero shift vector, after the image
+// solver combine only (no pass 2 there): M' fp32 [64][68], after the image
 constexpr uint32_t kOffMpf = kOffImg1 + 8192;
-constexpr uint32_t kOffZero = kOffMpf + 64 * kQS * 4;
+// solver combine: the contributors' column shifts and a batch of their sum_i v_i rows, in the DWC tile
+// area (free once the solver's DWC is done)
+constexpr int kRecBatch = 6;                                    // records summed per round trip
+constexpr uint32_t kOffCks = 0;                                 // float [kMaxContrib][64]
+constexpr uint32_t kOffSvk = kOffCks + kMaxContrib * 64 * 4;   // float [kRecBatch][64]
 // solver scratch (aliases the C region: the solver runs before this CTA's pass 1)
 constexpr uint32_t kOffNsHi = 0;                                // tf32 hi [2 K-halves][128 rows][128 B]
 constexpr uint32_t kOffNsLo = 32768;                            // tf32 lo
@@ -103,8 +113,9 @@ constexpr uint32_t kOffNsVec = kOffNsL + 64 * kQS * 4;          // float [2][64]
 static_assert(kSmemAlloc <= 232448, "shared memory over the sm_100 per-block limit");
 static_assert(kOffImg1 + 8192 <= kOffMp, "post-pass-1 scratch overlaps M'");
 static_assert(kOffDwcTiles + 6 * 16384 <= kOffMp, "DWC tiles overlap M'");
+static_assert(kOffL2 + 64 * kQS * 4 <= kOffL, "segment 1's landmarks overlap the L area");
 static_assert(kOffV == kOffDwcTiles + 16384, "the DWC tile region is not contiguous");
-static_assert(kOffZero + 256 <= kOffBar, "solver combine scratch overlaps the barriers");
+static_assert(kOffMpf + 64 * kQS * 4 <= kOffBar, "solver combine scratch overlaps the barriers");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -129,7 +140,8 @@ struct FusedArgs {
   unsigned long long* xready; // [U] X published (holds the epoch)
   unsigned long long* mready; // [U] M' image, the contributors' biases and the solver's DWC chunks
                               // published (holds the epoch)
-  int dwc_k;                  // DWC of each unit's first dwc_k chunks: by the unit's solver CTA
+  int dwc_take;               // DWC of the first dwc_take chunks of every row CTA's part of a unit: by
+                              // the unit's solver CTA
   unsigned char* mimg;        // [U][8192] M'^T bf16, the SW128 image of the pass-2 B operand
   float* rec;                 // [G][2][kRec]
   // pass-1 warp plan: warp w computes landmarks [wj0[w], wj0[w] + wlt[w]) of row half w / 8;
@@ -145,9 +157,13 @@ __device__ __forceinline__ void trace_mark(const Params& p, int slot) {
 __device__ __forceinline__ void trace_clock(const Params& p, int slot) {
   if (p.trace != nullptr && threadIdx.x == 0) p.trace[(size_t)blockIdx.x * 32 + slot] = (unsigned long long)clock64();
 }
+__device__ __forceinline__ void trace_mark_by(const Params& p, int slot, int thread) {
+  if (p.trace != nullptr && (int)threadIdx.x == thread) p.trace[(size_t)blockIdx.x * 32 + slot] = globaltimer();
+}
 #else
 __device__ __forceinline__ void trace_mark(const Params&, int) {}
 __device__ __forceinline__ void trace_clock(const Params&, int) {}
+__device__ __forceinline__ void trace_mark_by(const Params&, int, int) {}
 #endif
 
 // Row partition. Each unit's rows are cut into nchu 128-row chunks (the last one may be short);
@@ -166,6 +182,11 @@ __host__ __device__ __forceinline__ int part_start(int g, int U, int N, int G) {
   return (ci / nchu) * N + (ci % nchu) * kChunk;
 }
 __device__ __forceinline__ int cta_start(int g, const Params& p) { return part_start(g, p.U, p.N, gridDim.x); }
+// first global chunk of CTA g (the row CTAs' ranges; G for the end of the last one)
+__device__ __forceinline__ int cta_chunk0(int g, const Params& p) {
+  const int nchu = (p.N + kChunk - 1) / kChunk, T = p.U * nchu, P = (int)gridDim.x - p.U;
+  return g <= p.U ? 0 : T * (g - p.U) / P;
+}
 // CTA whose range holds global chunk C: the largest k with floor(T k / P) <= C, i.e. T k < (C + 1) P
 __device__ __forceinline__ int chunk_owner(int C, const Params& p) {
   const int nchu = (p.N + kChunk - 1) / kChunk, T = p.U * nchu, P = (int)gridDim.x - p.U;
@@ -778,7 +799,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
                       uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapV) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31, g = blockIdx.x;
   const int m = p.m, nch = R.nchunks;
-  float* Ls = reinterpret_cast<float*>(sm + kOffL);
+  float* Ls = reinterpret_cast<float*>(sm + kOffL);     // segment 0's landmarks
+  float* Ls2 = reinterpret_cast<float*>(sm + kOffL2);   // segment 1's landmarks
   float* sred = reinterpret_cast<float*>(sm + kOffSr);   // [segment][row half][S1 64 | S2 64]
   // (constant indices only: a variable index into the parameter arrays would copy them to the stack)
   const int rh = w >> 3;
@@ -822,39 +844,52 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     mbar_wait(bars + kBarP1 + (gc & 1), (gc >> 1) & 1, p.status, kStatusTimeout);
   };
   trace_mark(p, 28);
+  // Both segments' landmarks and column shifts before the first chunk: segment 0's landmarks go to
+  // the L area, segment 1's to the spare area after the third V stage; the shifts need each segment's
+  // first Q chunk (all of them have landed once kBarQ completes) and scratch in C slot 0 (free until
+  // chunk 0's C tile).
+  mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
+  for (int s = 0; s < R.nseg; ++s) {
+    if (t == 0)
+      spin_until_geq(fa.lready + R.seg[s].u, fa.epoch * (unsigned long long)m + (p.spin_test ? 1 : 0), p.status,
+                     kStatusTimeout, p.spin_budget);
+    __syncthreads();
+    float* L = s ? Ls2 : Ls;
+    load_landmarks(p.L + (size_t)R.seg[s].u * m * 64, L, m);
+    __syncthreads();
+    int s_, lo, nrows;
+    R.chunk(R.seg[s].first_chunk, s_, lo, nrows);
+    segment_shift(p, sm + kOffC + (R.seg[s].first_chunk + 1) * 16384, nrows, L, reinterpret_cast<float*>(sm + kOffC),
+                  shift + 64 * s);
+  }
+  trace_mark(p, 2);
   float s1[8], s2[8];
   for (int gc = 0; gc < nch; ++gc) {
     int s, lo, nrows;
     R.chunk(gc, s, lo, nrows);
-    const int u = R.seg[s].u;
     const bool seg_first = gc == R.seg[s].first_chunk;
     const bool seg_last = gc == R.seg[s].first_chunk + R.seg[s].nch - 1;
     unsigned char* cslot = sm + kOffC + gc * 16384;
     // products run two chunks behind: tile gc - 2 is complete and its V stage has had a chunk
     if (t == 0 && gc >= 2) issue_mma(gc - 2);
-    // Ls was last read before the previous chunk's closing barrier
-    if (gc == 0) mbar_wait(bars + kBarQ, 0, p.status, kStatusTimeout);
     if (seg_first) {
-      if (t == 0) spin_until_geq(fa.lready + u, fa.epoch * (unsigned long long)m + (p.spin_test ? 1 : 0), p.status,
-                                     kStatusTimeout, p.spin_budget);
-      __syncthreads();
-      if (gc == 0) trace_mark(p, 2);
-      load_landmarks(p.L + (size_t)u * m * 64, Ls, m);
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         s1[b] = 0.f;
         s2[b] = 0.f;
+        sh[b] = b < lt ? shift[64 * s + j0 + b] : 0.f;
       }
-      __syncthreads();
-      segment_shift(p, sm + kOffC + (gc + 1) * 16384, nrows, Ls, reinterpret_cast<float*>(sm + kOffQ + 16384),
-                    shift + 64 * s);
-#pragma unroll
-      for (int b = 0; b < 8; ++b) sh[b] = b < lt ? shift[64 * s + j0 + b] : 0.f;
     }
     if (gc < 2) trace_mark(p, 10 + 11 * gc);
-    if (lt > 0) cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, Ls, cslot, j0, 64 * rh, nrows, scale, sh, s1, s2);
+    if (lt > 0)
+      cross_dispatch(lt, sm + kOffC + (gc + 1) * 16384, s ? Ls2 : Ls, cslot, j0, 64 * rh, nrows, scale, sh, s1, s2);
     if (padder) write_padding(cslot, 64 * rh, nrows, m);
     if (gc == 1) trace_mark(p, 22);
+    if (gc == 3) {
+      trace_mark_by(p, 23, 5 * 32);
+      trace_mark_by(p, 26, 10 * 32);
+      trace_mark_by(p, 27, 15 * 32);
+    }
     if (seg_last) {
       // this segment's column sums of C and C^2, per row half
 #pragma unroll
@@ -874,6 +909,7 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
     tc_fence_before();
     __syncthreads();
     if (gc < 2) trace_mark(p, 11 + gc);
+    if (gc >= 2 && gc < 7) trace_mark(p, gc == 6 ? 24 : 14 + gc);
     // the next V chunk, issued after the barrier so that this thread's proxy fence above does not
     // wait for it: stage (gc + 1) % 3 last held chunk gc - 2, whose product went out at this
     // chunk's start. Warp 12 issues it (warp 0, which issues the products, starts its distances
@@ -1040,20 +1076,19 @@ __device__ void dwc_chunks(const Params& p, unsigned char* tiles, int nbuf, uint
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Row CTAs, after pass 1: DWC of this CTA's chunks, except each unit's first dwc_k chunks, which the
-// unit's solver CTA computes while it waits for the pass-1 records. The tile buffers are contiguous
-// from C slot kMaxChunks - 1 (free: a CTA has at most kMaxChunks - 1 chunks, and the Q tile that slot
-// held is consumed) through the V stages, Q and L (free after pass 1): three of two boxes or two of three.
+// Row CTAs, after pass 1: DWC of this CTA's chunks, except the first dwc_take chunks of each segment,
+// which the segment's unit's solver CTA computes while it waits for the pass-1 records (so every row
+// CTA hands over the same share). The tile buffers are contiguous from C slot kMaxChunks - 1 (free: a
+// CTA has at most kMaxChunks - 1 chunks, and the Q tile that slot held is consumed) through the V
+// stages, Q and L (free after pass 1): three of two boxes or two of three.
 __device__ void row_dwc(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint64_t* bars,
                         const CUtensorMap* tmapVp) {
   const int nbuf = (p.W + 1 <= 64) ? 3 : 2;
-  // this CTA's chunks outside the solvers' shares (each unit's rows below 128 dwc_k)
   int list[kMaxChunks];
   int n = 0;
   for (int gc = 0; gc < R.nchunks; ++gc) {
-    int s, lo, nrows;
-    R.chunk(gc, s, lo, nrows);
-    if (lo >= kChunk * fa.dwc_k) list[n++] = gc;
+    const int s = (R.nseg > 1 && gc >= R.seg[1].first_chunk) ? 1 : 0;
+    if (gc - R.seg[s].first_chunk >= fa.dwc_take) list[n++] = gc;
   }
   __syncthreads();   // pass 1 is done with the V stages, Q and L
   dwc_chunks(p, sm + kOffDwcTiles, nbuf, bars, tmapVp, n, [&](int i, int& u, int& lo) {
@@ -1065,16 +1100,26 @@ __device__ void row_dwc(const Params& p, const FusedArgs& fa, const Rows& R, uns
   trace_mark(p, 25);
 }
 
-// Solver CTA of unit u, after its chain and diagnostics: DWC of the unit's first dwc_k chunks, tiles in
-// its free scratch from offset 0 (four buffers of two boxes or two of three).
+// Solver CTA of unit u, after its chain and diagnostics: its share of the unit's DWC, the first
+// dwc_take chunks of each row CTA's part of the unit. Thread 0 lists them (chunk indices in the unit, in
+// row order) in the b area, free until the combine; the tiles go to the free scratch from offset 0
+// (four buffers of two boxes or two of three).
 __device__ void solver_dwc(const Params& p, const FusedArgs& fa, unsigned char* sm, uint64_t* bars, int u,
                            const CUtensorMap* tmapVp) {
-  const int nchu = (p.N + kChunk - 1) / kChunk;
-  const int count = fa.dwc_k < nchu ? fa.dwc_k : nchu;
-  __syncthreads();   // the chain's scratch is no longer read
-  dwc_chunks(p, sm, (p.W + 1 <= 64) ? 4 : 2, bars, tmapVp, count, [&](int i, int& uu, int& lo) {
+  int* list = reinterpret_cast<int*>(sm + kOffBv);   // [0] count, then the chunks
+  if (threadIdx.x == 0) {
+    const int nchu = (p.N + kChunk - 1) / kChunk, lo = u * nchu, hi = lo + nchu;
+    int n = 0;
+    for (int gg = chunk_owner(lo, p); gg <= chunk_owner(hi - 1, p); ++gg) {
+      const int a = max(cta_chunk0(gg, p), lo), b = min(cta_chunk0(gg + 1, p), hi);
+      for (int c = a; c < b && c < a + fa.dwc_take && n < kDwcListCap; ++c) list[1 + n++] = c - lo;
+    }
+    list[0] = n;
+  }
+  __syncthreads();   // the list is out; the chain's scratch is no longer read
+  dwc_chunks(p, sm, (p.W + 1 <= 64) ? 4 : 2, bars, tmapVp, list[0], [&](int i, int& uu, int& lo) {
     uu = u;
-    lo = kChunk * i;
+    lo = kChunk * list[1 + i];
   });
   __syncthreads();
 }
@@ -1127,14 +1172,11 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   }
   if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
   nct = nct < kMaxContrib ? nct : kMaxContrib;
-  // the zero reference shift, read by every thread below: written before the barrier
-  if (t < 64) reinterpret_cast<float*>(sm + kOffZero)[t] = 0.f;
   if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
   __syncthreads();
   trace_mark(p, 7);
   float* Mp = reinterpret_cast<float*>(sm + kOffMpf);   // M' fp32 [64][68] (row l)
   unsigned char* img = sm + kOffMp;
-  const float* shift = reinterpret_cast<const float*>(sm + kOffZero);   // the zero reference
   // X^T (row j, column l), zero outside m x m: the product below reads it along l
   {
     constexpr int kNX = 64 * 64 / kFT;   // X entries per thread, all loads issued first
@@ -1151,31 +1193,38 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
       Xt[j * kQS + l] = xv[k];
     }
   }
-  // sum the unit's records, each rebased from its own column shift c_k to this CTA's shift c* (the
-  // `shift` argument, with which this CTA's resident C was stored): for d_k = c_k - c*,
-  //   S1 += S1'_k + n_k d_k,  S2 += S2'_k + 2 d_k S1'_k + n_k d_k^2   (fp64),
-  //   P  += P'_k + d_k (sum_i v_i)_k^T                                 (fp32; row 63 holds sum_i v_i)
-  // so that the totals are the sums of C - c* over the unit. All loads of a batch of 4 records are
-  // issued before any use.
+  // sum the unit's records in contributor order, each rebased from its own column shift c_k to none:
+  //   S1 += S1'_k + n_k c_k,  S2 += S2'_k + 2 c_k S1'_k + n_k c_k^2   (fp64),
+  //   P  += P'_k + c_k (sum_i v_i)_k^T                                 (fp32; row 63 of P'_k holds sum_i v_i)
+  // The loads of a batch of up to kB records go out together (one round trip to L2): P'_k by every
+  // thread, S1'_k, S2'_k, c_k and n_k by threads 0..63. The rank-1 terms are added from shared memory
+  // after the batch: each record's c_k goes to cks (kept for the biases at the end), its sum_i v_i to
+  // svk.
+  float* cks = reinterpret_cast<float*>(sm + kOffCks);   // [kMaxContrib][64] the contributors' shifts
+  float* svk = reinterpret_cast<float*>(sm + kOffSvk);   // [kRecBatch][64] sum_i v_i of a batch
   {
-    constexpr int kNP = 1024 / kFT;   // float4 of P per thread: rows (t / 16) + 32 i, columns 4 (t % 16)
-    constexpr int kB = 4;
+    constexpr int kNP = 1024 / kFT;   // float4 of P per thread: rows (t >> 4) + 32 k, columns 4 (t & 15)
+    constexpr int kB = kRecBatch;
     double a1 = 0.0, a2 = 0.0;
     float4 pacc[kNP];
 #pragma unroll
     for (int k = 0; k < kNP; ++k) pacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int col4 = t & 15;
-    float cst[kNP];
-#pragma unroll
-    for (int k = 0; k < kNP; ++k) cst[k] = shift[(t >> 4) + 32 * k];
-    const double cs = t < 64 ? (double)shift[t] : 0.0;
     for (int c0 = 0; c0 < nct; c0 += kB) {
-      float s1v[kB], s2v[kB], ckv[kB], nkv[kB], ck[kB][kNP];
-      float4 pv[kB][kNP], sv[kB];
+      float4 pv[kB][kNP];
+      float s1v[kB], s2v[kB], ckv[kB], nkv[kB];
 #pragma unroll
       for (int c = 0; c < kB; ++c) {
         const bool ok = c0 + c < nct;
         const float* r = fa.rec + (ok ? ctr[c0 + c] : 0);
+#pragma unroll
+        for (int k = 0; k < kNP; ++k) {
+          pv[c][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ok) {
+            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * k);
+            pv[c][k] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
+                                   __uint_as_float(raw.w));
+          }
+        }
         s1v[c] = s2v[c] = ckv[c] = nkv[c] = 0.f;
         if (ok && t < 64) {
           s1v[c] = ld_cg_f32_ordered(r + t);
@@ -1183,38 +1232,42 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
           ckv[c] = ld_cg_f32_ordered(r + kRecC + t);
           nkv[c] = ld_cg_f32_ordered(r + kRecN);
         }
-        sv[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (ok) {
-          const uint4 raw = ld_cg_v4_ordered(r + 128 + 63 * 64 + 4 * col4);
-          sv[c] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
-                              __uint_as_float(raw.w));
-        }
-#pragma unroll
-        for (int k = 0; k < kNP; ++k) {
-          pv[c][k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          ck[c][k] = 0.f;
-          if (ok) {
-            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * k);
-            pv[c][k] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
-                                   __uint_as_float(raw.w));
-            ck[c][k] = ld_cg_f32_ordered(r + kRecC + (t >> 4) + 32 * k);
-          }
-        }
       }
 #pragma unroll
       for (int c = 0; c < kB; ++c) {
-        const double dk = (double)ckv[c] - cs, nk = (double)nkv[c];
-        a1 += (double)s1v[c] + nk * dk;
-        a2 += (double)s2v[c] + 2.0 * dk * (double)s1v[c] + nk * dk * dk;
+        if (c0 + c >= nct) break;
 #pragma unroll
         for (int k = 0; k < kNP; ++k) {
-          const float d = ck[c][k] - cst[k];
-          pacc[k].x += fmaf(d, sv[c].x, pv[c][k].x);
-          pacc[k].y += fmaf(d, sv[c].y, pv[c][k].y);
-          pacc[k].z += fmaf(d, sv[c].z, pv[c][k].z);
-          pacc[k].w += fmaf(d, sv[c].w, pv[c][k].w);
+          pacc[k].x += pv[c][k].x;
+          pacc[k].y += pv[c][k].y;
+          pacc[k].z += pv[c][k].z;
+          pacc[k].w += pv[c][k].w;
+        }
+        if (t < 64) {
+          const double ck = (double)ckv[c], nk = (double)nkv[c];
+          a1 += (double)s1v[c] + nk * ck;
+          a2 += (double)s2v[c] + 2.0 * ck * (double)s1v[c] + nk * ck * ck;
+          cks[(c0 + c) * 64 + t] = ckv[c];
+        }
+        // row 63 (sum_i v_i) is the last float4 of threads 16 * 31 .. 16 * 31 + 15
+        if ((t >> 4) + 32 * (kNP - 1) == 63)
+          *reinterpret_cast<float4*>(svk + c * 64 + 4 * (t & 15)) = pv[c][kNP - 1];
+      }
+      __syncthreads();
+      const int nb = nct - c0 < kB ? nct - c0 : kB;
+#pragma unroll
+      for (int k = 0; k < kNP; ++k) {
+        const int l = (t >> 4) + 32 * k;
+        for (int c = 0; c < nb; ++c) {
+          const float ck = cks[(c0 + c) * 64 + l];
+          const float4 sv = *reinterpret_cast<const float4*>(svk + c * 64 + 4 * (t & 15));
+          pacc[k].x = fmaf(ck, sv.x, pacc[k].x);
+          pacc[k].y = fmaf(ck, sv.y, pacc[k].y);
+          pacc[k].z = fmaf(ck, sv.z, pacc[k].z);
+          pacc[k].w = fmaf(ck, sv.w, pacc[k].w);
         }
       }
+      __syncthreads();   // svk is refilled by the next batch
     }
     if (t < 64) {
       S1d[t] = a1;
@@ -1228,9 +1281,8 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   }
   __syncthreads();
   trace_mark(p, 8);
-  // the totals are sums of C - c*: mu* = mean(C - c*) = mu - c*, and the variance does not see the shift
+  // mu, var and s from the totals (fp64)
   if (t < 64) {
-    const double c = (double)shift[t];
     const double mup = S1d[t] * invN;
     double var = S2d[t] * invN - mup * mup;
     if (var < 0.0) var = 0.0;
@@ -1239,54 +1291,61 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
     scs[t] = t < m ? (float)sc : 0.f;
     svs[t] = As[63 * kQS + t];       // landmark column 63 holds sum_i v_i
     if (t < m) {
-      p.mu[(size_t)u * m + t] = (float)(mup + c);
+      p.mu[(size_t)u * m + t] = (float)mup;
       p.s[(size_t)u * m + t] = (float)sc;
     }
   }
   __syncthreads();
-  // A = C~^T V from P* = (C - c*)^T V by the rank-1 fold, in place. Whitened: C~ = (C - mu) s + 1/N
-  // with C - mu = (C - c*) - mu*, so A[l][k] = s_l (P*[l][k] - mu*_l sum_i v_ik) + sum_i v_ik / N;
-  // raw: A = C^T V = P* + c* sum_i v_i^T. Zero for l >= m.
+  // A = C~^T V from P = C^T V by the rank-1 fold, in place (whitened: C~ = (C - mu) s + 1/N, so
+  // A[l][k] = s_l (P[l][k] - mu_l sum_i v_ik) + sum_i v_ik / N; raw: A = P). Zero for l >= m.
   for (int e = t; e < 64 * 64; e += kFT) {
     const int l = e >> 6, k = e & 63;
     float a = 0.f;
     if (l < m) {
       const float P = As[l * kQS + k];
-      a = p.whiten ? scs[l] * (P - mus[l] * svs[k]) + svs[k] * invNf : P + shift[l] * svs[k];
+      a = p.whiten ? scs[l] * (P - mus[l] * svs[k]) + svs[k] * invNf : P;
     }
     As[l * kQS + k] = a;
   }
   __syncthreads();
   trace_mark(p, 9);
-  // M = X A on 256 threads: thread (k0 = 8 (t / 32), l0 = 2 (t % 32)) forms M[l0 .. l0 + 1][k0 .. k0 + 7].
+  // M = X A on all threads: thread (k0 = 4 (t / 32), l0 = 2 (t % 32)) forms M[l0 .. l0 + 1][k0 .. k0 + 3].
   // A warp shares k0 (the A reads are broadcasts) and takes the 64 landmarks in pairs (conflict-free
-  // X^T reads and image stores); each step's operands are loaded one step ahead
+  // X^T reads and image stores). Four steps j per iteration, alternating between two accumulator sets
+  // (rows j >= m of X^T and A are zero, so the steps run to a multiple of 4).
   float* bvec = reinterpret_cast<float*>(sm + kOffBv);
-  if (t < 256) {
-    const int l0 = 2 * (t & 31), k0 = 8 * (t >> 5);
-    float acc[2][8];
+  {
+    const int l0 = 2 * (t & 31), k0 = 4 * (t >> 5);
+    float acc[2][4], acc2[2][4];
 #pragma unroll
     for (int r = 0; r < 2; ++r)
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-    float2 xn = *reinterpret_cast<const float2*>(&Xt[l0]);
-    float4 a0n = *reinterpret_cast<const float4*>(&As[k0]);
-    float4 a1n = *reinterpret_cast<const float4*>(&As[k0 + 4]);
+      for (int c = 0; c < 4; ++c) acc[r][c] = acc2[r][c] = 0.f;
+    const int m4 = (m + 3) & ~3;
 #pragma unroll 1
-    for (int j = 0; j < m; ++j) {
-      const float2 x = xn;
-      const float4 a0 = a0n, a1 = a1n;
-      const int jn = j + 1 < m ? j + 1 : j;
-      xn = *reinterpret_cast<const float2*>(&Xt[jn * kQS + l0]);
-      a0n = *reinterpret_cast<const float4*>(&As[jn * kQS + k0]);
-      a1n = *reinterpret_cast<const float4*>(&As[jn * kQS + k0 + 4]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    for (int j0 = 0; j0 < m4; j0 += 4) {
+      float2 x[4];
+      float4 a[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        acc[0][c] = fmaf(x.x, av[c], acc[0][c]);
-        acc[1][c] = fmaf(x.y, av[c], acc[1][c]);
+      for (int q = 0; q < 4; ++q) {
+        x[q] = *reinterpret_cast<const float2*>(&Xt[(j0 + q) * kQS + l0]);
+        a[q] = *reinterpret_cast<const float4*>(&As[(j0 + q) * kQS + k0]);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float(&ac)[2][4] = (q & 1) ? acc2 : acc;
+        const float av[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          ac[0][c] = fmaf(x[q].x, av[c], ac[0][c]);
+          ac[1][c] = fmaf(x[q].y, av[c], ac[1][c]);
+        }
       }
     }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[r][c] += acc2[r][c];
     // M' = diag(s) M (raw: M), as fp32 rows for the bias and as the bf16 image; b0 = sum_l
     // (1/N - s_l mu_l) M[l] (raw: 0)
     float sc[2], coef[2];
@@ -1297,9 +1356,9 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
       sc[r] = in ? (p.whiten ? scs[l] : 1.f) : 0.f;
       coef[r] = (in && p.whiten) ? invNf - scs[l] * mus[l] : 0.f;
     }
-    float bp[8];
+    float bp[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       const float m0 = sc[0] * acc[0][c], m1 = sc[1] * acc[1][c];
       Mp[l0 * kQS + k0 + c] = m0;
       Mp[(l0 + 1) * kQS + k0 + c] = m1;
@@ -1307,25 +1366,26 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
       bp[c] = coef[0] * acc[0][c] + coef[1] * acc[1][c];
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
+    for (int c = 0; c < 4; ++c)
       for (int o = 16; o > 0; o >>= 1) bp[c] += __shfl_xor_sync(0xffffffffu, bp[c], o);
     if (lane == 0) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) bvec[k0 + c] = bp[c];
+      for (int c = 0; c < 4; ++c) bvec[k0 + c] = bp[c];
     }
   }
-  __syncthreads();   // the product above is done reading X^T
-  // every contributor's column shift, [record][landmark], in the place of X^T
-  float* cks = Xt;
-  for (int e = t; e < nct * 64; e += kFT) cks[e] = __ldcg(fa.rec + ctr[e >> 6] + kRecC + (e & 63));
   __syncthreads();
   trace_mark(p, 20);
   // the contributors' biases b_k = b0 + c_k^T M', and the image, out before the flag
   for (int e = t; e < nct * 64; e += kFT) {
     const int k = e >> 6, jc = e & 63;
-    float b = bvec[jc];
-    for (int l = 0; l < m; ++l) b = fmaf(cks[k * 64 + l], Mp[l * kQS + jc], b);
-    fa.rec[ctr[k] + kRecB + jc] = b;
+    float b0 = 0.f, b1 = 0.f;   // two chains over the landmarks
+    int l = 0;
+    for (; l + 1 < m; l += 2) {
+      b0 = fmaf(cks[k * 64 + l], Mp[l * kQS + jc], b0);
+      b1 = fmaf(cks[k * 64 + l + 1], Mp[(l + 1) * kQS + jc], b1);
+    }
+    if (l < m) b0 = fmaf(cks[k * 64 + l], Mp[l * kQS + jc], b0);
+    fa.rec[ctr[k] + kRecB + jc] = bvec[jc] + (b0 + b1);
   }
   for (int e = t; e < 512; e += kFT)
     reinterpret_cast<uint4*>(fa.mimg + (size_t)u * 8192)[e] = reinterpret_cast<const uint4*>(img)[e];
@@ -1747,15 +1807,19 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
   plan_pass1_warps(p.m, fa);
   // The solver CTAs wait, after their chain, for the pass-1 records; they spend that time on the DWC
-  // of their unit's first chunks. Rough model: a chunk of pass 1 takes about 6.8 us, the chain about
-  // 33 us, a chunk of DWC about 1.5 us, so a solver has room for (6.8 cpc - 33) / 1.5 chunks, cpc the
-  // chunks of a row CTA.
+  // of the first chunks of each row CTA's part of their unit. Rough model: a chunk of pass 1 takes
+  // about 6.8 us, the chain with its diagnostics about 34 us, a chunk of DWC about 1.5 us, so a
+  // solver has room for k = (6.8 cpc - 34) / 1.5 chunks (cpc the chunks of a row CTA), shared by the
+  // about nchu / cpc + 1 row CTAs of a unit: take = k cpc / (nchu + cpc), rounded.
   {
     const int nchu = (p.N + kChunk - 1) / kChunk;
     const int cpc = (p.U * nchu + (G - p.U) - 1) / (G - p.U);
-    int k = (68 * cpc - 330) / 15;
-    k = k < 0 ? 0 : (k > nchu ? nchu : k);
-    fa.dwc_k = k;
+    int k = (68 * cpc - 340) / 15;
+    k = k < 0 ? 0 : k;
+    int take = (2 * k * cpc + (nchu + cpc)) / (2 * (nchu + cpc));
+    take = take > cpc ? cpc : take;
+    take = take > kMaxDwcTake ? kMaxDwcTake : take;
+    fa.dwc_take = take;
   }
   Params pp = p;
   void* args[] = {(void*)&pp, (void*)&fa, (void*)&tmap, (void*)&tmapq, (void*)&tmapo, (void*)&tmapvp};
