@@ -113,6 +113,34 @@ def workspace_report(lfa, wl):
     return rows
 
 
+def solver_report(lfa, dev):
+    """Newton-Schulz (the forward's solver) against conjugate gradients on the device, both fp32, on
+    synthetic SPD landmark systems with condition number 50 (m = 49, 64 right-hand sides, 3 systems):
+    median relative error ||Y - W^-1 B||_F / ||W^-1 B||_F after the given steps."""
+    import numpy as np
+    import torch
+
+    from laplacian_nystr_attention_avg_b200.inputs import make_spd_systems
+
+    W, B = make_spd_systems(49, 50.0, 3, 64, seed=0)
+    Wd = torch.from_numpy(W.astype(np.float32)).to(dev)
+    Bd = torch.from_numpy(B.astype(np.float32)).to(dev)
+    W32, B32 = W.astype(np.float32).astype(np.float64), B.astype(np.float32).astype(np.float64)
+    Y = np.stack([np.linalg.solve(W32[u], B32[u]) for u in range(3)])
+
+    def rel(Z):
+        return float(np.median([np.linalg.norm(Z[u] - Y[u]) / np.linalg.norm(Y[u]) for u in range(3)]))
+
+    out = {}
+    for T in (10, 20):
+        X, _ = lfa.ns_solve(Wd, T)
+        out[f"ns_T{T}"] = rel(X.double().cpu().numpy() @ B32)
+    for k in (10, 20, 30, 49):
+        out[f"cg_{k}"] = rel(lfa.cg_solve(Wd, Bd, k).double().cpu().numpy())
+    out["note"] = "median relative error of Y over 3 systems; one NS step ~ 2 m^3 multiply-adds, one CG step m^2 x 64"
+    return out
+
+
 def read_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -518,6 +546,7 @@ def main():
                                 "note": "kappa_2(W + eps I) per unit after the forward: ||W||_2 (power "
                                         "iteration) x ||X_T||_2 with X_T ~ (W + eps I)^-1"},
                 "workspace_bytes": workspace_report(lfa, wl),
+                "solvers_kappa50": solver_report(lfa, dev),
             },
         }
         if world == 1 and not args.no_cpu_baseline and args.whiten == "unit":

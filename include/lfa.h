@@ -209,6 +209,36 @@ lfa_status lfa_sp_pass1(lfa_handle h, const void* Q_local, const void* V_local, 
 lfa_status lfa_sp_pass2(lfa_handle h, const void* Q_local, const void* V_local, const void* V_halo,
                         const double* partial_total, void* O_local, void* stream);
 
+/* ---- solvers for the landmark system W Y = B -------------------------------------------------
+ * The note solves with W by Newton-Schulz and ablates conjugate gradients against it, reporting
+ * that CG degrades on ill-conditioned systems (condition number 50) while Newton-Schulz stays
+ * stable (LaplacianFormer note, §关键设计 3 and the solver ablation). These two calls run both
+ * solvers on caller-supplied matrices so the claim can be measured on the device; the forward
+ * pass itself always uses Newton-Schulz. W: U symmetric positive-definite m x m matrices, fp32
+ * row-major [U][m][m], 1 <= m <= 256; device pointers, 16-byte aligned, owned by the caller. */
+
+/* Bytes of device workspace lfa_ns_solve needs for U systems of size m (0 for invalid sizes). */
+size_t lfa_solver_workspace_size(int U, int m);
+
+/* X [U][m][m] = the T-step Newton-Schulz approximation of W^-1 the forward pass computes:
+ * alpha = 2 / ||W||_2 (power iteration), or 1 / ||W||_2^2 when the printed condition
+ * ||I - alpha W W^T||_2 < 1 fails; X_0 = alpha W^T; X <- X (2I - W X), each product on tcgen05 in
+ * split TF32 (hi*hi + hi*lo + lo*hi, about 2^-21 relative). workspace: lfa_solver_workspace_size
+ * bytes, 256-byte aligned, overwritten. host_out (optional, U entries): alpha, lambda_max,
+ * the fallback flag and ||I - W X_T||_F per system (kappa = 0); with it the call synchronizes the
+ * stream and returns LFA_ERR_NONFINITE if a value is not finite. LFA_ERR_INVALID_ARG for NULL or
+ * misaligned pointers, sizes outside the bounds or T outside [0, 64]. */
+lfa_status lfa_ns_solve(const float* W, float* X, int U, int m, int T, void* workspace, size_t workspace_bytes,
+                        lfa_unit_info* host_out, void* stream);
+
+/* Y [U][m][nrhs] = conjugate gradients for W Y = B (B [U][m][nrhs], fp32 row-major): for every
+ * column an independent Hestenes-Stiefel recursion from Y_0 = 0, exactly `iters` iterations,
+ * a = r^T r / p^T W p (0 when p^T W p <= 0), beta = r'^T r' / r^T r (0 when r^T r = 0), all in
+ * fp32 with column sums in a fixed order (deterministic). W must be symmetric: the kernel reads
+ * W[j][i] for W[i][j]. 1 <= nrhs <= 4096, 0 <= iters <= 4096; LFA_ERR_INVALID_ARG otherwise or
+ * for NULL / misaligned pointers. Asynchronous on `stream`. */
+lfa_status lfa_cg_solve(const float* W, const float* B, float* Y, int U, int m, int nrhs, int iters, void* stream);
+
 /* ---- inspection entry points used by the parity tests ---------------------- */
 
 /* Cross kernel C = exp(-||q_i - l_l||_1 / lambda) of one unit [the note's §关键设计 2],

@@ -6,6 +6,7 @@
 
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "lfa_internal.h"
 
@@ -193,6 +194,7 @@ lfa_status ensure_attributes() {
   if (lfa::backward_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::gemm_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::ns_tc_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::cg_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (dev < 64) g_attr_done |= 1ull << dev;
   return LFA_OK;
 }
@@ -441,6 +443,85 @@ lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* 
   h->have_forward = 0;
   if (lfa::launch_pool(p, st) != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::launch_cross_kernel(p, unit, C_out, st) != cudaSuccess) return LFA_ERR_CUDA;
+  return LFA_OK;
+}
+
+// ---- solvers for W Y = B outside the forward pass -------------------------------------------
+
+namespace {
+// Newton-Schulz scratch: X_b and Y (U m^2 fp32 each), the per-unit info and the status word
+struct SolverLayout {
+  size_t xb, y, info, status, total;
+};
+SolverLayout solver_layout(int U, int m) {
+  SolverLayout l;
+  const size_t mm = (size_t)U * m * m * sizeof(float);
+  l.xb = 0;
+  l.y = align256(mm);
+  l.info = l.y + align256(mm);
+  l.status = l.info + align256((size_t)U * lfa::kInfoStride * sizeof(float));
+  l.total = l.status + 256;
+  return l;
+}
+bool solver_sizes_ok(int U, int m) { return U >= 1 && m >= 1 && m <= lfa::kMaxM && (size_t)U * m * m < (1ull << 31); }
+}  // namespace
+
+size_t lfa_solver_workspace_size(int U, int m) {
+  if (!solver_sizes_ok(U, m)) return 0;
+  return solver_layout(U, m).total;
+}
+
+lfa_status lfa_ns_solve(const float* W, float* X, int U, int m, int T, void* workspace, size_t workspace_bytes,
+                        lfa_unit_info* host_out, void* stream) {
+  if (!W || !X || !workspace || !solver_sizes_ok(U, m) || T < 0 || T > 64) return LFA_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(X) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return LFA_ERR_INVALID_ARG;
+  const SolverLayout l = solver_layout(U, m);
+  if (workspace_bytes < l.total) return LFA_ERR_INVALID_ARG;
+  const lfa_status st_attr = ensure_attributes();
+  if (st_attr != LFA_OK) return st_attr;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  lfa::Params p;
+  memset(&p, 0, sizeof(p));
+  p.U = U;
+  p.m = m;
+  p.T = T;
+  p.Wm = const_cast<float*>(W);   // read only on this path
+  p.X = X;
+  p.Xb = reinterpret_cast<float*>(ws + l.xb);
+  p.Y = reinterpret_cast<float*>(ws + l.y);
+  p.info = reinterpret_cast<float*>(ws + l.info);
+  p.status = reinterpret_cast<int*>(ws + l.status);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(p.status, 0, sizeof(int), st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::launch_ns_from_w(p, st) != cudaSuccess) return LFA_ERR_CUDA;
+  if (!host_out) return LFA_OK;
+  std::vector<float> tmp((size_t)U * lfa::kInfoStride);
+  int status = 0;
+  if (cudaMemcpyAsync(tmp.data(), p.info, tmp.size() * sizeof(float), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(&status, p.status, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return LFA_ERR_CUDA;
+  for (int u = 0; u < U; ++u) {
+    const float* f = tmp.data() + (size_t)u * lfa::kInfoStride;
+    host_out[u].alpha = f[lfa::kInfoAlpha];
+    host_out[u].lambda_max = f[lfa::kInfoLambdaMax];
+    host_out[u].alpha_fallback = f[lfa::kInfoFallback] != 0.f;
+    host_out[u].ns_residual_fro = f[lfa::kInfoResidual];
+    host_out[u].kappa = 0.f;
+  }
+  return (status & lfa::kStatusNonFinite) ? LFA_ERR_NONFINITE : LFA_OK;
+}
+
+lfa_status lfa_cg_solve(const float* W, const float* B, float* Y, int U, int m, int nrhs, int iters, void* stream) {
+  if (!W || !B || !Y || !solver_sizes_ok(U, m) || nrhs < 1 || nrhs > 4096 || iters < 0 || iters > 4096)
+    return LFA_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(B) || !aligned16(Y)) return LFA_ERR_INVALID_ARG;
+  if ((size_t)U * m * nrhs >= (1ull << 31)) return LFA_ERR_INVALID_ARG;
+  const lfa_status st_attr = ensure_attributes();
+  if (st_attr != LFA_OK) return st_attr;
+  if (lfa::launch_cg(W, B, Y, U, m, nrhs, iters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return LFA_ERR_CUDA;
   return LFA_OK;
 }
 

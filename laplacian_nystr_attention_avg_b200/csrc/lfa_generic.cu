@@ -874,6 +874,27 @@ void reading_b_t(const Params& p, cudaStream_t st) {
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
 
+// alpha (power iteration and the fallback rule), the T Newton-Schulz steps X <- X (2I - W X) as
+// tcgen05 products, and the closing residual ||I - W X_T||_F, from W in p.Wm (p.Y and p.Xb are scratch).
+void ns_from_w(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m;
+  k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
+  const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
+  float* x = p.X;
+  float* xb = p.Xb;
+  const size_t mm = (size_t)m * m;
+  for (int k = 0; k < p.T; ++k) {
+    const MmJob y{p.Wm, mm, x, mm, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X
+    launch_mm(&y, 1, m, U, st);
+    const MmJob xn{x, mm, p.Y, mm, nullptr, 0, xb, mm, 1.f, 0.f, 0.f, 0, 0};     // X' = X Y
+    launch_mm(&xn, 1, m, U, st);
+    float* tmp = x; x = xb; xb = tmp;
+  }
+  if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
+  k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
+  k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
+}
+
 // W, alpha and the Newton-Schulz chain from the landmarks in the workspace.
 void ns_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m;
@@ -881,21 +902,7 @@ void ns_t(const Params& p, cudaStream_t st) {
     launch_ns_tc(p, st);
   } else {
     k_gram<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
-    k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
-    const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
-    float* x = p.X;
-    float* xb = p.Xb;
-    const size_t mm = (size_t)m * m;
-    for (int k = 0; k < p.T; ++k) {
-      const MmJob y{p.Wm, mm, x, mm, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X
-      launch_mm(&y, 1, m, U, st);
-      const MmJob xn{x, mm, p.Y, mm, nullptr, 0, xb, mm, 1.f, 0.f, 0.f, 0, 0};     // X' = X Y
-      launch_mm(&xn, 1, m, U, st);
-      float* tmp = x; x = xb; xb = tmp;
-    }
-    if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
-    k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
-    k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
+    ns_from_w(p, st);
   }
 }
 
@@ -992,6 +999,11 @@ cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st) {
 
 cudaError_t launch_generic_ns(const Params& p, cudaStream_t st) {
   ns_t(p, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ns_from_w(const Params& p, cudaStream_t st) {
+  ns_from_w(p, st);
   return cudaGetLastError();
 }
 

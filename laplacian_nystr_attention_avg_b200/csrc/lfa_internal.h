@@ -148,6 +148,13 @@ cudaError_t launch_generic_forward(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_context(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_pass1_reduce(const Params& p, cudaStream_t st);
 cudaError_t launch_generic_ns(const Params& p, cudaStream_t st);
+// alpha, the Newton-Schulz steps and the closing residual from W in p.Wm (p.X out, p.Xb / p.Y scratch;
+// uses p.U, p.m, p.T, p.info, p.status)
+cudaError_t launch_ns_from_w(const Params& p, cudaStream_t st);
+// conjugate gradients for U systems W Y = B (lfa_solvers.cu)
+cudaError_t cg_set_attributes();
+cudaError_t launch_cg(const float* W, const float* B, float* Y, int U, int m, int nrhs, int iters,
+                      cudaStream_t st);
 cudaError_t launch_generic_finish(const Params& p, cudaStream_t st);
 cudaError_t launch_backward(const BwdParams& b, cudaStream_t st);
 size_t backward_smem_main(int d);

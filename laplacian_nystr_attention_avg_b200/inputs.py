@@ -27,6 +27,8 @@ import dataclasses
 import math
 from typing import Dict, Optional
 
+import numpy as np
+
 import torch
 
 
@@ -173,3 +175,17 @@ def make_crop_inputs(wl: Workload, h: int, w: int, r: int, seed: int = 0, name: 
 
     return cw, Inputs(wl=cw, Q=crop(full.Q), V=crop(full.V), dwc=full.dwc, dO=crop(full.dO),
                       Q_store=crop(full.Q_store), V_store=crop(full.V_store), dO_store=crop(full.dO_store))
+
+
+def make_spd_systems(m: int, kappa: float, U: int, nrhs: int, seed: int = 0):
+    """U symmetric positive-definite m x m matrices with eigenvalues spaced geometrically from 1 to
+    kappa (random orthogonal eigenvectors) and standard normal right-hand sides [U, m, nrhs]:
+    float64 numpy arrays (the solver comparison's synthetic systems)."""
+    rng = np.random.default_rng(seed)
+    W = np.empty((U, m, m))
+    for u in range(U):
+        Qm, _ = np.linalg.qr(rng.standard_normal((m, m)))
+        W[u] = (Qm * np.geomspace(1.0, kappa, m)) @ Qm.T
+    B = rng.standard_normal((U, m, nrhs))
+    return W, B
+

@@ -77,6 +77,9 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_sp_pool": (ci, [vp, vp, vp, vp]),
         "lfa_sp_pass1": (ci, [vp, vp, vp, vp, vp, vp]),
         "lfa_sp_pass2": (ci, [vp, vp, vp, vp, vp, vp, vp]),
+        "lfa_solver_workspace_size": (sz, [ci, ci]),
+        "lfa_ns_solve": (ci, [vp, vp, ci, ci, ci, vp, sz, ctypes.POINTER(UnitInfo), vp]),
+        "lfa_cg_solve": (ci, [vp, vp, vp, ci, ci, ci, ci, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -146,6 +149,42 @@ def make_config(wl, whiten=True) -> Config:
 
 def workspace_size(cfg: Config) -> int:
     return int(load().lfa_workspace_size(ctypes.byref(cfg)))
+
+
+def solver_workspace_size(U: int, m: int) -> int:
+    return int(load().lfa_solver_workspace_size(int(U), int(m)))
+
+
+def ns_solve(W: torch.Tensor, T: int, stream=None):
+    """lfa_ns_solve: the forward pass's T-step Newton-Schulz approximation of W^-1 for each of the
+    U symmetric positive-definite matrices W [U, m, m] (device float32). Returns (X, [UnitInfo])."""
+    if W.dim() != 3 or W.shape[1] != W.shape[2]:
+        raise ValueError(f"W: expected [U, m, m], got {tuple(W.shape)}")
+    U, m = int(W.shape[0]), int(W.shape[1])
+    _require(W, "W", (U, m, m), torch.float32, W.device)
+    X = torch.empty_like(W)
+    nbytes = solver_workspace_size(U, m)
+    if nbytes == 0:
+        raise LfaError(LFA_ERR_INVALID_ARG, "lfa_solver_workspace_size")
+    ws = torch.empty((nbytes + 256,), dtype=torch.uint8, device=W.device)
+    off = (-ws.data_ptr()) % 256
+    info = (UnitInfo * U)()
+    _check(load().lfa_ns_solve(_ptr(W), _ptr(X), U, m, int(T), ctypes.c_void_p(ws.data_ptr() + off), nbytes,
+                               info, _stream(stream)), "lfa_ns_solve")
+    return X, list(info)
+
+
+def cg_solve(W: torch.Tensor, B: torch.Tensor, iters: int, stream=None) -> torch.Tensor:
+    """lfa_cg_solve: conjugate gradients for W Y = B, W [U, m, m] symmetric positive definite,
+    B [U, m, nrhs] (device float32), exactly `iters` iterations from Y = 0. Returns Y."""
+    if W.dim() != 3 or W.shape[1] != W.shape[2] or B.dim() != 3:
+        raise ValueError(f"W [U, m, m] and B [U, m, nrhs] expected, got {tuple(W.shape)}, {tuple(B.shape)}")
+    U, m, nrhs = int(W.shape[0]), int(W.shape[1]), int(B.shape[2])
+    _require(W, "W", (U, m, m), torch.float32, W.device)
+    _require(B, "B", (U, m, nrhs), torch.float32, W.device)
+    Y = torch.empty_like(B)
+    _check(load().lfa_cg_solve(_ptr(W), _ptr(B), _ptr(Y), U, m, nrhs, int(iters), _stream(stream)), "lfa_cg_solve")
+    return Y
 
 
 def forward_noalloc(cfg: Config, dwc_weight: torch.Tensor, Q: torch.Tensor, V: torch.Tensor,

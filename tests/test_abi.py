@@ -79,6 +79,32 @@ def test_reading_b_accepts_the_largest_m(lib):
         assert lfa.workspace_size(_cfg(whiten=3, **kw)) > 0
 
 
+def test_solver_calls_validate_before_any_device_work(lib):
+    assert lfa.solver_workspace_size(0, 49) == 0
+    assert lfa.solver_workspace_size(1, 0) == 0
+    assert lfa.solver_workspace_size(1, 257) == 0
+    n = lfa.solver_workspace_size(3, 49)
+    assert n >= 2 * 3 * 49 * 49 * 4
+    bad = lfa.LFA_ERR_INVALID_ARG
+    p = 256   # an aligned non-null address; every call below must fail its checks before using it
+    cg = lib.lfa_cg_solve
+    assert cg(None, p, p, 1, 49, 8, 5, None) == bad
+    assert cg(p, None, p, 1, 49, 8, 5, None) == bad
+    assert cg(p, p, None, 1, 49, 8, 5, None) == bad
+    assert cg(p + 4, p, p, 1, 49, 8, 5, None) == bad          # misaligned
+    assert cg(p, p, p, 0, 49, 8, 5, None) == bad              # U
+    assert cg(p, p, p, 1, 257, 8, 5, None) == bad             # m > 256
+    assert cg(p, p, p, 1, 49, 0, 5, None) == bad              # nrhs
+    assert cg(p, p, p, 1, 49, 8, -1, None) == bad             # iters
+    ns = lib.lfa_ns_solve
+    assert ns(None, p, 1, 49, 20, p, n, None, None) == bad
+    assert ns(p, p, 1, 49, 65, p, n, None, None) == bad       # T > 64
+    assert ns(p, p, 1, 49, -1, p, n, None, None) == bad
+    assert ns(p, p, 3, 49, 20, p, n - 1, None, None) == bad   # workspace too small
+    assert ns(p, p, 3, 49, 20, p + 16, n, None, None) == bad  # workspace not 256-byte aligned
+    assert ns(p, p, 1, 0, 20, p, n, None, None) == bad
+
+
 def test_create_rejects_null_and_misaligned(lib):
     cfg = _cfg()
     h = ctypes.c_void_p()
