@@ -59,8 +59,8 @@ extern "C" {
 typedef enum {
   LFA_OK = 0,
   LFA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, H%r or W%r != 0 ... */
-  LFA_ERR_UNSUPPORTED = 2,   /* d not in {32, 64}, m > 256, unknown dtype; whiten = 3 with m > 64;
-                                backward with whiten = 2 or 3 */
+  LFA_ERR_UNSUPPORTED = 2,   /* d not in {32, 64}, m > 256, unknown dtype; backward with
+                                whiten = 3 */
   LFA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, copy, attribute) */
   LFA_ERR_STATE = 4,         /* backward without a matching forward on this handle */
   LFA_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired (reported by lfa_get_info) */
@@ -87,7 +87,7 @@ typedef struct {
                      G^ = C X C^T are whitened instead of those of C, O_attn = G~ V, in the
                      factored form (C - 1 c-^T) X C^T D^-1/2 V + (1/N) 1 1^T V with
                      D = diag(c_j^T X^T cov(C) X c_j + eps) over key tokens j; any m.
-                     whiten = 2 and 3 run the per-stage kernels, forward only. */
+                     whiten = 2 and 3 run the per-stage kernels; whiten = 3 is forward only. */
 } lfa_config;
 
 /* Per-unit diagnostics of the most recent forward call. */
@@ -160,7 +160,9 @@ lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host
 /* Backward pass for the loss <dO, O>: writes dQ and dV ([B][heads][N][d], cfg.dtype).
  * Reuses the context saved by the most recent lfa_forward on this handle, which
  * must have been called with the same Q and V pointers (else LFA_ERR_STATE).
- * Batch-pooled statistics and Reading B (whiten = 2, 3) have no backward: LFA_ERR_UNSUPPORTED.
+ * With batch-pooled statistics (whiten = 2) the whitening's reverse mode pools its two column
+ * means over the B N rows of each head, as the forward pools mu and var. Reading B (whiten = 3)
+ * has no backward: LFA_ERR_UNSUPPORTED.
  * The kernel gradient is -(1/lambda) sign(q - l) k with sign(0) = 0 [the note's
  * §研究背景与动机 prints the opposite sign]; alpha is held constant; the DWC
  * weight gets no gradient. */

@@ -378,7 +378,7 @@ lfa_status lfa_backward(lfa_handle h, const void* Q, const void* V, const void* 
   if (!h || !Q || !V || !dO || !dQ || !dV || h->sp) return LFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ) || !aligned16(dV))
     return LFA_ERR_INVALID_ARG;
-  if (h->p.whiten >= 2) return LFA_ERR_UNSUPPORTED;
+  if (h->p.whiten == 3) return LFA_ERR_UNSUPPORTED;   // Reading B: forward only
   if (!h->have_forward || h->last_Q != Q || h->last_V != V) return LFA_ERR_STATE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Params p = h->p;

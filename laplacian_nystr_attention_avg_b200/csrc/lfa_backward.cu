@@ -60,8 +60,8 @@ __global__ void k_init_iterate(BwdParams b) {
 
 // ---------------------------------------------------------------------------------------
 // Combine of the backward statistics: dM, then rows [16c, 16c + 16) of dX = dM A^T and
-// dA = X^T dM, the whitening-backward coefficients, Gm = s o M, Gd = s o dA and the
-// bias partial of dV.
+// dA = X^T dM, the whitening-backward coefficients (for batch-pooled statistics their per-unit sums,
+// pooled by k_bwd_pool_coef), Gm = s o M, Gd = s o dA and the bias partial of dV.
 //   dC_il = s_l dC~_il + beta_l + gamma_l C_il with
 //   a_l = mean_i dC~_il, e_l = sum_i dC~_il C_il, c_l = (s_l / N)(e_l - mu_l N a_l),
 //   gamma_l = -s_l^2 c_l, beta_l = -s_l a_l - gamma_l mu_l.
@@ -124,15 +124,23 @@ __global__ void __launch_bounds__(kThreads) k_bwd_combine(BwdParams b) {
       se += __shfl_xor_sync(0xffffffffu, se, o);
     }
     if (lane == 0) {
-      double beta = 0.0, gamma = 0.0;
-      if (p.whiten) {
-        const double a = sa * invN, sd = sj, mj = mu[j];
-        const double cc = sd * invN * (se - mj * double(p.N) * a);
-        gamma = -sd * sd * cc;
-        beta = -sd * a - gamma * mj;
+      if (p.whiten == 2) {
+        // batch-pooled statistics: the sums go to the unused column-sum slots of this unit's dO
+        // record; k_bwd_pool_coef adds them over the head's units and forms beta and gamma
+        double* rbw = b.red2 + (size_t)u * p.part_stride;
+        rbw[j] = sa;
+        rbw[m + j] = se;
+      } else {
+        double beta = 0.0, gamma = 0.0;
+        if (p.whiten) {
+          const double a = sa * invN, sd = sj, mj = mu[j];
+          const double cc = sd * invN * (se - mj * double(p.N) * a);
+          gamma = -sd * sd * cc;
+          beta = -sd * a - gamma * mj;
+        }
+        b.beta[(size_t)u * m + j] = (float)beta;
+        b.gamma[(size_t)u * m + j] = (float)gamma;
       }
-      b.beta[(size_t)u * m + j] = (float)beta;
-      b.gamma[(size_t)u * m + j] = (float)gamma;
     }
   }
   // bias partial of dV: sum over this chunk's rows of (1/N - s_j mu_j) dA[j][k]
@@ -145,6 +153,37 @@ __global__ void __launch_bounds__(kThreads) k_bwd_combine(BwdParams b) {
       }
     }
     b.bpart2[((size_t)u * p.n_chunks + c) * d + k] = (float)acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Whitening-backward coefficients for statistics pooled per head over the batch (whiten = 2): the
+// means over the B N stacked rows of the head's units (batch b = 0 .. B-1 in order), with the
+// shared mu and s: a_l = (sum_b sum_i dC~_il) / (B N), e_l = sum_b sum_i dC~_il C_il,
+// c_l = (s_l / (B N)) (e_l - mu_l B N a_l), gamma_l = -s_l^2 c_l, beta_l = -s_l a_l - gamma_l mu_l,
+// written to every unit of the head.
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) k_bwd_pool_coef(BwdParams b) {
+  const Params& p = b.p;
+  const int m = p.m, h = blockIdx.y, j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= m) return;
+  double sa = 0.0, se = 0.0;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const double* rb = b.red2 + (size_t)(bb * p.heads + h) * p.part_stride;
+    sa += rb[j];
+    se += rb[m + j];
+  }
+  // the per-unit formula's operation order with N -> B N (identical results at B = 1)
+  const double BN = double(p.B) * double(p.N), invBN = 1.0 / BN;
+  const double sj = p.s[(size_t)h * m + j], mj = p.mu[(size_t)h * m + j];
+  const double a = sa * invBN;
+  const double cc = sj * invBN * (se - mj * BN * a);
+  const double gamma = -sj * sj * cc;
+  const double beta = -sj * a - gamma * mj;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const size_t o = (size_t)(bb * p.heads + h) * m + j;
+    b.beta[o] = (float)beta;
+    b.gamma[o] = (float)gamma;
   }
 }
 
@@ -450,6 +489,7 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
   cudaError_t e = launch_generic_pass1_reduce(p1, st);
   if (e != cudaSuccess) return e;
   k_bwd_combine<<<dim3(p.n_chunks, U), kThreads, (size_t)m * d * sizeof(float), st>>>(b);
+  if (p.whiten == 2) k_bwd_pool_coef<<<dim3(ceil_div(m, kThreads), p.heads), kThreads, 0, st>>>(b);
   // Newton-Schulz iterates X_0 .. X_{T-1} ([U][T][m][m])
   const size_t its_stride = (size_t)T_ * mm;
   if (T_ > 0) {
@@ -527,7 +567,7 @@ int backward_launch_count(const Params& p) {
   // pass 1 + reduce, combine, iterates (1 + 2 (T - 1)), 3 T reverse launches (6 products per step, batched), gram part of dL,
   // main pass, dL reduction, dQ
   const int its = p.T > 0 ? 1 + 2 * (p.T - 1) : 0;
-  return 2 + 1 + its + 3 * p.T + 1 + 1 + 1 + 1;
+  return 2 + 1 + (p.whiten == 2 ? 1 : 0) + its + 3 * p.T + 1 + 1 + 1 + 1;
 }
 
 cudaError_t launch_backward(const BwdParams& b, cudaStream_t st) {

@@ -4,15 +4,15 @@ batch elements (LaplacianFormer note, 关键设计 1, statistics over a batch of
 
 Covers the heavy-tailed PVT stage-2 shape at full size (32 batch elements per head), a small fp32
 shape with a ragged tile and d = 32, the pooled statistics themselves, the reduction to the
-per-unit statistics at B = 1 (bit for bit on the GPU), the per-stage path choice and the
-unsupported backward.
+per-unit statistics at B = 1 (bit for bit on the GPU), the per-stage path choice, and the backward
+(pooled whitening reverse mode) at three shapes and its reduction to the per-unit one at B = 1.
 """
 import numpy as np
 import pytest
 import torch
 
 from laplacian_nystr_attention_avg_b200 import lfa
-from laplacian_nystr_attention_avg_b200.inputs import Workload
+from laplacian_nystr_attention_avg_b200.inputs import Workload, make_inputs
 from oracle import lfa_oracle as O
 from tests import parity_util as pu
 
@@ -73,12 +73,40 @@ def test_batch_stats_single_batch_is_per_unit():
     assert torch.equal(outs[0], outs[1])
 
 
-def test_batch_stats_backward_unsupported():
-    wl = SMALL
-    x = pu.inputs_for(wl)
+BWD = [SMALL.replace(backward=True),
+       Workload("batch_bwd_bf16", B=4, heads=2, H=16, W=16, d=64, r=4, T=24, dtype="bf16", backward=True)]
+
+
+@pytest.mark.parametrize("wl", BWD + [pu.workload("pvt2").replace(backward=True)],
+                         ids=[w.name for w in BWD] + ["pvt2"])
+def test_batch_stats_backward(wl):
+    # the reverse mode of the pooled whitening (the oracle's R12 gradient, pinned by finite
+    # differences): the column means of dC~ and dC~ o C^ over each head's B N rows
+    x = make_inputs(wl, with_dO=True)
     mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, "batch"), x.dwc, "cuda")
-    Q, V = x.Q_store.cuda(), x.V_store.cuda()
+    Q, V, dO = x.Q_store.cuda(), x.V_store.cuda(), x.dO_store.cuda()
     mod.forward(Q, V)
-    with pytest.raises(lfa.LfaError) as e:
-        mod.backward(Q, V, torch.ones_like(Q))
-    assert e.value.status == lfa.LFA_ERR_UNSUPPORTED
+    dQ, dV = mod.backward(Q, V, dO)
+    torch.cuda.synchronize()
+    gq, gv = O.backward(x.Q.numpy(), x.V.numpy(), x.dwc.numpy(), x.dO.numpy(), wl, True, batch_stats=True)
+    bf16 = wl.dtype == "bf16"
+    units = tuple(range(wl.units))
+    for name, g, ref in (("dQ", dQ, gq), ("dV", dV, gv)):
+        got = pu.unit_rows(g, units)
+        want = ref.reshape(wl.units, wl.N, wl.d)
+        assert np.isfinite(got).all()
+        err = pu.o_error(got, want, bf16)
+        assert err <= pu.o_tolerance(bf16), f"{wl.name} {name}: error {err:.3e}"
+
+
+def test_batch_stats_backward_single_batch_is_per_unit():
+    wl = pu.workload("pr1").replace(backward=True)   # B = 1: the pooled coefficients are the unit's own
+    x = make_inputs(wl, with_dO=True)
+    Q, V, dO = x.Q_store.cuda(), x.V_store.cuda(), x.dO_store.cuda()
+    grads = []
+    for whiten in (True, "batch"):
+        mod = lfa.LaplacianNystromAttention(lfa.make_config(wl, whiten), x.dwc, "cuda")
+        mod.forward(Q, V)
+        grads.append([t.clone() for t in mod.backward(Q, V, dO)])
+    torch.cuda.synchronize()
+    assert torch.equal(grads[0][0], grads[1][0]) and torch.equal(grads[0][1], grads[1][1])
