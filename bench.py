@@ -320,7 +320,8 @@ def run_backward(args):
     print(json.dumps({
         "metric": "tokens/s per forward + backward call", "value": wl.units * wl.N / (step_ms * 1e-3),
         "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
-        "forward_ms": fwd_ms / K, "backward_ms": bwd_ms / K, "higher_is_better": True, "dtype": "f32",
+        "forward_ms": fwd_ms / K, "backward_ms": bwd_ms / K, "higher_is_better": True,
+        "dtype": dtype_label(mod.path) + "; backward: fp32 SIMT main pass, split-TF32 tcgen05 reverse products",
         "data": "synthetic", "config": workload_config(wl, {"path": mod.path, "inputs": "resident, no L2 flush"}),
     }), flush=True)
 

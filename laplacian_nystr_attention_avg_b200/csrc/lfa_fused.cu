@@ -1,32 +1,30 @@
 // Fused single-launch forward pass for bf16 inputs, d = 64 and m <= 63 landmarks.
 //
-// One cooperative persistent kernel, one CTA per SM. Token rows of all U = B*heads units are
-// split into contiguous per-CTA ranges (cut at unit boundaries into at most two segments,
-// processed in 128-row chunks); CTAs 0..U-1 are the units' solver CTAs and own no rows.
+// One cooperative persistent kernel, one CTA per SM. Token rows of all U = B*heads units are cut into
+// 128-row chunks dealt out to the row CTAs (at most two units, "segments", per CTA); CTAs 0..U-1 are
+// the units' solver CTAs and own no rows. CTAs meet only through per-unit flags in global memory
+// (epoch-stamped counters, bounded waits); there is no grid-wide barrier.
 //   phase 0  all CTAs: landmark pooling L = r x r average pool of Q (LaplacianFormer note,
-//            §关键设计 2); arrive on a grid-wide barrier.
+//            §关键设计 2); each landmark raises its unit's landmark counter.
 //   phase 1  solver CTA of unit u: W = exp(-E/lam) + eps I, ||W||_2 by power iteration, alpha
 //            (§关键设计 3 with the fallback), and the T Newton-Schulz steps on tcgen05 in 3xTF32
 //            (fp32-accurate): X_{k+1} = X_k + X_k R_k, R_{k+1} = R_k R_k^T (R_k = I - W X_k; the
 //            same iterates in exact arithmetic, one stacked [X; R] product per step), then the
-//            printed product form X (2I - W X) for the last two steps, which re-anchors R to
-//            I - W X.
+//            printed product form X (2I - W X) for the last step, which re-anchors R to I - W X;
+//            the diagnostic ||I - W X_T||_F; then its share of the unit's DWC.
 //   phase 2  row CTAs, pass 1 per chunk (Q rows by TMA): C = exp(-||q - l||_1 / lam) on CUDA cores
-//            in fp32 (the dominant cost), kept in shared memory as bf16 for the whole kernel (never
-//            in HBM);
-//            per-landmark sums of C and C^2 in registers; P += C^T V on tcgen05 (V chunk staged
-//            by TMA; a constant-1 landmark column 63 yields sum_i v_i in the same product).
-//            Each CTA publishes one partial record per segment.
-//   phase 3  solver CTA of unit u, once the unit's records are out: mu, var, s = 1/sqrt(var +
-//            eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A, M' = diag(s) M,
-//            b = (1/N - s o mu)^T M; M'^T (bf16, in the shared-memory image pass 2 consumes) and
-//            b are published with a release flag; then the solve's diagnostics, off the
-//            critical path.
-//   phase 3b row CTAs, while M' is formed: DWC(V) (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise,
-//            zero padding) of every chunk from a TMA-staged V tile with a one-grid-row halo,
-//            rounded to bf16 and written into the chunk's TMEM accumulator.
-//   phase 4  row CTAs: O = DWC + C M' (tcgen05 accumulating onto the DWC values; all chunks'
-//            products at once, one TMEM accumulator each) + b, stored once as bf16.
+//            in fp32 (the dominant cost), kept in shared memory as bf16(C - c), c a per-column shift
+//            of the segment, for the whole kernel (never in HBM); per-landmark sums of C - c and
+//            (C - c)^2 in registers; P += (C - c)^T V on tcgen05 (V chunk staged by TMA; a constant-1
+//            landmark column 63 yields sum_i v_i in the same product). One record per segment.
+//   phase 3  solver CTA of unit u, once the unit's records are out: sums them rebased to no shift,
+//            mu, var, s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A,
+//            M' = diag(s) M, b0 = (1/N - s o mu)^T M; publishes M'^T (bf16, the shared-memory image
+//            pass 2 consumes) and each contributor's bias b0 + c_k^T M' with a release flag.
+//   phase 3b row CTAs, meanwhile: DWC(V) (§关键设计 1 "ZV + DWC(V)", 3 x 3 depthwise, zero padding)
+//            of their other chunks from TMA-staged V tiles with a one-grid-row halo, bf16 into O.
+//   phase 4  row CTAs: O += (C - c) M' + bias by tcgen05 products (one TMEM accumulator per chunk) and
+//            TMA bf16 reduce-adds of the epilogue rows onto the DWC values in O.
 // Every cross-CTA wait is bounded; an expired wait sets the timeout bit of the status word.
 #include <stdlib.h>
 #include <string.h>
