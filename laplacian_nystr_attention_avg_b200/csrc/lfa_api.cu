@@ -227,6 +227,30 @@ size_t lfa_workspace_size(const lfa_config* cfg) {
   return L.total;
 }
 
+// the handle's auxiliary stream and fork / join events (the per-stage kernels overlap the Newton-Schulz
+// chain with pass 1 on it); released by lfa_destroy
+void free_aux(lfa_ctx* h) {
+  if (h->p.ev_fork) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_fork));
+  if (h->p.ev_join) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_join));
+  if (h->p.aux_stream) cudaStreamDestroy(static_cast<cudaStream_t>(h->p.aux_stream));
+  h->p.ev_fork = h->p.ev_join = h->p.aux_stream = nullptr;
+}
+bool make_aux(lfa_ctx* h) {
+  cudaStream_t s = nullptr;
+  cudaEvent_t a = nullptr, b = nullptr;
+  const bool ok = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&a, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&b, cudaEventDisableTiming) == cudaSuccess;
+  h->p.aux_stream = s;
+  h->p.ev_fork = a;
+  h->p.ev_join = b;
+  if (!ok) {
+    free_aux(h);
+    cudaGetLastError();
+  }
+  return ok;
+}
+
 lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* workspace,
                       size_t workspace_bytes, lfa_handle* out) {
   if (!out) return LFA_ERR_INVALID_ARG;
@@ -255,6 +279,10 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
   h->spin_test_budget = -1;
   bind(&h->p, h->lay, h->ws);
   h->p.dwc = dwc_weight;
+  if (!make_aux(h)) {
+    delete h;
+    return LFA_ERR_CUDA;
+  }
   h->path = 0;
   const char* force = getenv("LFA_FORWARD_PATH");
   const bool want_generic = force && strcmp(force, "generic") == 0;
@@ -271,6 +299,7 @@ lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* work
 
 lfa_status lfa_destroy(lfa_handle h) {
   if (!h) return LFA_ERR_INVALID_ARG;
+  free_aux(h);
   delete h;
   return LFA_OK;
 }
@@ -666,6 +695,10 @@ lfa_status lfa_sp_create(const lfa_config* cfg, int y0, int ny, const float* dwc
   h->spin_test_budget = -1;
   bind(&h->p, h->lay, h->ws);
   h->p.dwc = dwc_weight;
+  if (!make_aux(h)) {
+    delete h;
+    return LFA_ERR_CUDA;
+  }
   h->path = 0;
   h->sp = 1;
   *out = h;

@@ -486,23 +486,29 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
   p1.V = b.dO;
   p1.part = b.part2;
   p1.red = b.red2;
-  cudaError_t e = launch_generic_pass1_reduce(p1, st);
-  if (e != cudaSuccess) return e;
-  k_bwd_combine<<<dim3(p.n_chunks, U), kThreads, (size_t)m * d * sizeof(float), st>>>(b);
-  if (p.whiten == 2) k_bwd_pool_coef<<<dim3(ceil_div(m, kThreads), p.heads), kThreads, 0, st>>>(b);
-  // Newton-Schulz iterates X_0 .. X_{T-1} ([U][T][m][m])
+  // C^T dO, the combine and the Newton-Schulz iterates X_0 .. X_{T-1} ([U][T][m][m]) share no data:
+  // with an auxiliary stream the iterates run concurrently with the other two
   const size_t its_stride = (size_t)T_ * mm;
-  if (T_ > 0) {
-    k_init_iterate<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(b);
-    for (int k = 0; k + 1 < T_; ++k) {
-      const float* Xk = b.its + k * mm;
-      const MmJob y{p.Wm, mm, Xk, its_stride, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};  // Y = 2I - W X_k
-      launch_mm(&y, 1, m, U, st);
-      const MmJob xn{Xk, its_stride, p.Y, mm, nullptr, 0, b.its + (k + 1) * mm, its_stride,  // X_{k+1} = X_k Y
-                     1.f, 0.f, 0.f, 0, 0};
-      launch_mm(&xn, 1, m, U, st);
-    }
-  }
+  cudaError_t e = cudaSuccess;
+  fork_join(p, st,
+            [&](cudaStream_t s) {
+              e = launch_generic_pass1_reduce(p1, s);
+              k_bwd_combine<<<dim3(p.n_chunks, U), kThreads, (size_t)m * d * sizeof(float), s>>>(b);
+              if (p.whiten == 2) k_bwd_pool_coef<<<dim3(ceil_div(m, kThreads), p.heads), kThreads, 0, s>>>(b);
+            },
+            [&](cudaStream_t s) {
+              if (T_ == 0) return;
+              k_init_iterate<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, s>>>(b);
+              for (int k = 0; k + 1 < T_; ++k) {
+                const float* Xk = b.its + k * mm;
+                const MmJob y{p.Wm, mm, Xk, its_stride, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};  // Y = 2I - W X_k
+                launch_mm(&y, 1, m, U, s);
+                const MmJob xn{Xk, its_stride, p.Y, mm, nullptr, 0, b.its + (k + 1) * mm, its_stride,  // X_{k+1} = X_k Y
+                               1.f, 0.f, 0.f, 0, 0};
+                launch_mm(&xn, 1, m, U, s);
+              }
+            });
+  if (e != cudaSuccess) return e;
   // reverse steps; G starts as dX
   if (cudaMemsetAsync(b.dW, 0, sizeof(float) * U * mm, st) != cudaSuccess) return cudaErrorUnknown;
   float* G = b.G;

@@ -906,18 +906,24 @@ void ns_t(const Params& p, cudaStream_t st) {
   }
 }
 
-// Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b.
+// Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b. The
+// Newton-Schulz chain (W, alpha, X) and pass 1 (the column sums, C^T V) share no data: with an
+// auxiliary stream they run concurrently, joined before the combine.
 template <typename T>
 void context_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
   k_pool<T><<<dim3(ceil_div(m, kThreads / 32), U), kThreads, 0, st>>>(p);
-  ns_t(p, st);
   if (p.whiten == 3) {
+    ns_t(p, st);
     reading_b_t<T>(p, st);
     return;
   }
-  pass1_reduce_t<T>(p, st);
-  if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, st>>>(p);
+  fork_join(p, st,
+            [&](cudaStream_t s) {
+              pass1_reduce_t<T>(p, s);
+              if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, s>>>(p);
+            },
+            [&](cudaStream_t s) { ns_t(p, s); });
   k_combine_finish<<<dim3(p.n_chunks, U), kThreads, (size_t)(m * d + 2 * m) * sizeof(float), st>>>(p);
 }
 

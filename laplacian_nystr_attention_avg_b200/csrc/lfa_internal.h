@@ -75,6 +75,11 @@ struct Params {
   // optional timing events bracketing the dominant kernel (cudaEvent_t or null)
   void* ev_begin;
   void* ev_end;
+  // optional second stream and fork / join events (cudaStream_t, cudaEvent_t, or null): the
+  // per-stage kernels run the Newton-Schulz chain there, concurrently with pass 1 (they share no data)
+  void* aux_stream;
+  void* ev_fork;
+  void* ev_join;
   // optional per-CTA phase timestamps (%globaltimer, ns) of the fused kernel: [grid][16]
   unsigned long long* trace;
   // optional copy of the cross kernel C of unit dbg_unit as computed by this forward, fp32 [N][m]
@@ -157,6 +162,24 @@ cudaError_t launch_cg(const float* W, const float* B, float* Y, int U, int m, in
                       cudaStream_t st);
 cudaError_t launch_generic_finish(const Params& p, cudaStream_t st);
 cudaError_t launch_backward(const BwdParams& b, cudaStream_t st);
+
+// on_main(st) and on_aux(s) with s = p.aux_stream, concurrently: s waits for st's work so far, and
+// st waits for s's before it continues. Without an auxiliary stream both run on st, on_aux first.
+template <typename FMain, typename FAux>
+void fork_join(const Params& p, cudaStream_t st, FMain on_main, FAux on_aux) {
+  if (p.aux_stream && p.ev_fork && p.ev_join) {
+    cudaStream_t aux = static_cast<cudaStream_t>(p.aux_stream);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), st);
+    cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_fork), 0);
+    on_aux(aux);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_join), aux);
+    on_main(st);
+    cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_join), 0);
+  } else {
+    on_aux(st);
+    on_main(st);
+  }
+}
 size_t backward_smem_main(int d);
 cudaError_t backward_set_attributes();
 int backward_launch_count(const Params& p);
