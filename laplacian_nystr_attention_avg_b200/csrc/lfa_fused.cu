@@ -52,6 +52,7 @@ constexpr int kQS = 68;                   // fp32 row stride (floats) of the Q, 
 constexpr int kRec = 128 + 64 * 64 + 128 + 64;
 constexpr int kRecC = 128 + 64 * 64;      // offset of c
 constexpr int kRecN = kRecC + 64;         // offset of n
+constexpr int kRecF = kRecN + 2;          // offset of the record's 64-bit published flag (holds the epoch)
 constexpr int kRecB = kRecN + 64;         // offset of b
 constexpr int kMaxGrid = 256;             // records are sized for up to this many CTAs
 constexpr int kMaxContrib = 32;           // CTAs contributing to one unit
@@ -95,11 +96,13 @@ constexpr uint32_t kOffImg1 = (kOffWc + kWarps * 4 + 1023) / 1024 * 1024;   // M
 constexpr uint32_t kOffDwcTiles = kOffC + (kMaxChunks - 1) * 16384;
 // solver combine only (no pass 2 there): M' fp32 [64][68], after the image
 constexpr uint32_t kOffMpf = kOffImg1 + 8192;
-// solver combine: the contributors' column shifts and a batch of their sum_i v_i rows, in the DWC tile
-// area (free once the solver's DWC is done)
-constexpr int kRecBatch = 6;                                    // records summed per round trip
+// solver combine: the contributors' column shifts and the size of the current batch of records, in the
+// DWC tile area (free once the solver's DWC is done)
 constexpr uint32_t kOffCks = 0;                                 // float [kMaxContrib][64]
-constexpr uint32_t kOffSvk = kOffCks + kMaxContrib * 64 * 4;   // float [kRecBatch][64]
+constexpr uint32_t kOffBatch = kOffCks + kMaxContrib * 64 * 4;  // int
+constexpr int kRecBatch = 6;                                    // records per bulk-copy batch
+constexpr uint32_t kRecBytes = kRec * 4;
+constexpr uint32_t kOffRecBuf = 16384;                          // kRecBatch records, copied whole
 // solver scratch (aliases the C region: the solver runs before this CTA's pass 1)
 constexpr uint32_t kOffNsHi = 0;                                // tf32 hi [2 K-halves][128 rows][128 B]
 constexpr uint32_t kOffNsLo = 32768;                            // tf32 lo
@@ -114,6 +117,8 @@ static_assert(kOffDwcTiles + 6 * 16384 <= kOffMp, "DWC tiles overlap M'");
 static_assert(kOffL2 + 64 * kQS * 4 <= kOffL, "segment 1's landmarks overlap the L area");
 static_assert(kOffV == kOffDwcTiles + 16384, "the DWC tile region is not contiguous");
 static_assert(kOffMpf + 64 * kQS * 4 <= kOffBar, "solver combine scratch overlaps the barriers");
+static_assert(kOffRecBuf + kRecBatch * kRecBytes <= kOffAs && kRecBytes % 16 == 0 && kOffBatch + 4 <= kOffRecBuf,
+              "combine record buffers overlap the combine scratch");
 static_assert(kOffNsVec + 1024 <= kOffV, "solver scratch overlaps V stages");
 
 // mbarrier slots
@@ -123,10 +128,15 @@ constexpr int kBarP2 = 5;     // [kMaxChunks] pass-2 product of chunk gc done (o
 constexpr int kBarNs = 13;    // solver product done
 constexpr int kBarDiag = 14;  // the solver's diagnostics product done
 constexpr int kBarQ = 16;     // all of the CTA's pass-1 Q chunks landed (TMA)
-constexpr int kBarDrain = 17; // every tcgen05 operation of the two issuing threads done (count 2)
+constexpr int kBarDrain = 17; // every tcgen05 operation of the issuing threads done (count kDrainCount)
 constexpr int kBarH = 18;     // [4] DWC halo tile landed (TMA)
+constexpr int kBarRec = kBarV;  // solver CTAs (which have no V stages): a batch of records copied in
 constexpr int kNumBars = kBarH + 4;
-constexpr int kIssueP2 = kFT - 32;          // pass 2: issues the C M' products
+// pass 2: lane 0 of warp kP2Warp0 + gc issues chunk gc's products (each chunk has its own accumulator,
+// so the issuers need no order among themselves); with thread 0 they make up the drain count
+constexpr int kP2Warp0 = 8;
+constexpr int kDrainCount = 1 + (kMaxChunks - 1);
+static_assert(kP2Warp0 + kMaxChunks - 1 <= kWarps, "pass-2 issuers beyond the last warp");
 constexpr uint32_t kTmemSlot = 248;  // byte offset of the TMEM address within the barrier area
 constexpr uint32_t kTmemCols = 512;  // whole TMEM: pass 2 gives every chunk its own accumulator
 static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers overlap the TMEM address slot");
@@ -134,7 +144,6 @@ static_assert(kNumBars * 8 <= (int)kTmemSlot && kTmemSlot + 4 <= 256, "mbarriers
 struct FusedArgs {
   unsigned long long epoch;   // launch count of this handle (>= 1); flags compare against it
   unsigned long long* lready; // [U] landmarks of the unit pooled (counts landmarks, m per launch)
-  unsigned long long* cnt;    // [U] partial records published per unit
   unsigned long long* xready; // [U] X published (holds the epoch)
   unsigned long long* mready; // [U] M' image, the contributors' biases and the solver's DWC chunks
                               // published (holds the epoch)
@@ -966,7 +975,8 @@ __device__ void pass1(const Params& p, const FusedArgs& fa, const Rows& R, unsig
   __syncthreads();
   if (t == 0) {
     __threadfence();
-    for (int s = 0; s < R.nseg; ++s) red_release_add_u64(fa.cnt + R.seg[s].u, 1ull);
+    for (int s = 0; s < R.nseg; ++s)
+      st_release_u64(reinterpret_cast<unsigned long long*>(fa.rec + ((size_t)g * 2 + s) * kRec + kRecF), fa.epoch);
   }
 }
 
@@ -1170,12 +1180,10 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
   }
   if (nonempty && before < kMaxContrib) ctr[before] = rec_off;
   nct = nct < kMaxContrib ? nct : kMaxContrib;
-  if (t == 0) spin_until_geq(fa.cnt + u, fa.epoch * (unsigned long long)nct, p.status, kStatusTimeout, p.spin_budget);
-  __syncthreads();
-  trace_mark(p, 7);
+  __syncthreads();   // the contributor table
   float* Mp = reinterpret_cast<float*>(sm + kOffMpf);   // M' fp32 [64][68] (row l)
   unsigned char* img = sm + kOffMp;
-  // X^T (row j, column l), zero outside m x m: the product below reads it along l
+  // X^T (row j, column l), zero outside m x m (X is this CTA's own): the product below reads it along l
   {
     constexpr int kNX = 64 * 64 / kFT;   // X entries per thread, all loads issued first
     float xv[kNX];
@@ -1191,81 +1199,69 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
       Xt[j * kQS + l] = xv[k];
     }
   }
-  // sum the unit's records in contributor order, each rebased from its own column shift c_k to none:
+  // Sum the unit's records in contributor order as they are published, each rebased from its own
+  // column shift c_k to none:
   //   S1 += S1'_k + n_k c_k,  S2 += S2'_k + 2 c_k S1'_k + n_k c_k^2   (fp64),
-  //   P  += P'_k + c_k (sum_i v_i)_k^T                                 (fp32; row 63 of P'_k holds sum_i v_i)
-  // The loads of a batch of up to kB records go out together (one round trip to L2): P'_k by every
-  // thread, S1'_k, S2'_k, c_k and n_k by threads 0..63. The rank-1 terms are added from shared memory
-  // after the batch: each record's c_k goes to cks (kept for the biases at the end), its sum_i v_i to
-  // svk.
+  //   P  += P'_k, then P += c_k (sum_i v_i)_k^T                       (fp32; row 63 of P'_k holds sum_i v_i)
+  // Thread 0 waits for the next record's flag, takes every consecutive record already out (at most
+  // kRecBatch) as one batch and copies them whole into shared memory by bulk copies on one mbarrier;
+  // then all threads add them in order. The additions follow the contributor order whatever the batches
+  // are, so the result does not depend on timing. Each record's c_k also goes to cks for the biases.
   float* cks = reinterpret_cast<float*>(sm + kOffCks);   // [kMaxContrib][64] the contributors' shifts
-  float* svk = reinterpret_cast<float*>(sm + kOffSvk);   // [kRecBatch][64] sum_i v_i of a batch
+  int* batch = reinterpret_cast<int*>(sm + kOffBatch);  // records in the current batch
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
   {
     constexpr int kNP = 1024 / kFT;   // float4 of P per thread: rows (t >> 4) + 32 k, columns 4 (t & 15)
-    constexpr int kB = kRecBatch;
+    const int col4 = t & 15;
     double a1 = 0.0, a2 = 0.0;
     float4 pacc[kNP];
 #pragma unroll
     for (int k = 0; k < kNP; ++k) pacc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < nct; c0 += kB) {
-      float4 pv[kB][kNP];
-      float s1v[kB], s2v[kB], ckv[kB], nkv[kB];
-#pragma unroll
-      for (int c = 0; c < kB; ++c) {
-        const bool ok = c0 + c < nct;
-        const float* r = fa.rec + (ok ? ctr[c0 + c] : 0);
-#pragma unroll
-        for (int k = 0; k < kNP; ++k) {
-          pv[c][k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (ok) {
-            const uint4 raw = ld_cg_v4_ordered(reinterpret_cast<const float4*>(r + 128) + t + kFT * k);
-            pv[c][k] = make_float4(__uint_as_float(raw.x), __uint_as_float(raw.y), __uint_as_float(raw.z),
-                                   __uint_as_float(raw.w));
-          }
-        }
-        s1v[c] = s2v[c] = ckv[c] = nkv[c] = 0.f;
-        if (ok && t < 64) {
-          s1v[c] = ld_cg_f32_ordered(r + t);
-          s2v[c] = ld_cg_f32_ordered(r + 64 + t);
-          ckv[c] = ld_cg_f32_ordered(r + kRecC + t);
-          nkv[c] = ld_cg_f32_ordered(r + kRecN);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < kB; ++c) {
-        if (c0 + c >= nct) break;
-#pragma unroll
-        for (int k = 0; k < kNP; ++k) {
-          pacc[k].x += pv[c][k].x;
-          pacc[k].y += pv[c][k].y;
-          pacc[k].z += pv[c][k].z;
-          pacc[k].w += pv[c][k].w;
-        }
-        if (t < 64) {
-          const double ck = (double)ckv[c], nk = (double)nkv[c];
-          a1 += (double)s1v[c] + nk * ck;
-          a2 += (double)s2v[c] + 2.0 * ck * (double)s1v[c] + nk * ck * ck;
-          cks[(c0 + c) * 64 + t] = ckv[c];
-        }
-        // row 63 (sum_i v_i) is the last float4 of threads 16 * 31 .. 16 * 31 + 15
-        if ((t >> 4) + 32 * (kNP - 1) == 63)
-          *reinterpret_cast<float4*>(svk + c * 64 + 4 * (t & 15)) = pv[c][kNP - 1];
+    auto flag = [&](int c) {
+      return reinterpret_cast<const unsigned long long*>(fa.rec + ctr[c] + kRecF);
+    };
+    int nbatch = 0;
+    for (int c0 = 0; c0 < nct;) {
+      if (t == 0) {
+        spin_until_geq(flag(c0), fa.epoch, p.status, kStatusTimeout, p.spin_budget);
+        int nb = 1;
+        while (c0 + nb < nct && nb < kRecBatch && ld_acquire_u64(flag(c0 + nb)) >= fa.epoch) ++nb;
+        *batch = nb;
+        // the records are generic-proxy stores of other CTAs, released with their flags; the buffers
+        // were last read (and the DWC tiles before them written) through the generic proxy
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        fence_async_smem();
+        mbar_expect_tx(bars + kBarRec, (uint32_t)nb * kRecBytes);
+        for (int c = 0; c < nb; ++c)
+          bulk_load(sm + kOffRecBuf + c * kRecBytes, fa.rec + ctr[c0 + c], kRecBytes, bars + kBarRec);
       }
       __syncthreads();
-      const int nb = nct - c0 < kB ? nct - c0 : kB;
+      if (nbatch == 0) trace_mark(p, 7);
+      const int nb = *batch;
+      mbar_wait(bars + kBarRec, nbatch & 1, p.status, kStatusTimeout);
+      for (int c = 0; c < nb; ++c) {
+        const float* r = reinterpret_cast<const float*>(sm + kOffRecBuf + c * kRecBytes);
+        if (t < 64) {
+          const double cc = (double)r[kRecC + t], nk = (double)r[kRecN];
+          const double s1 = (double)r[t];
+          a1 += s1 + nk * cc;
+          a2 += (double)r[64 + t] + 2.0 * cc * s1 + nk * cc * cc;
+          cks[(c0 + c) * 64 + t] = r[kRecC + t];
+        }
+        const float4 sv = *reinterpret_cast<const float4*>(r + 128 + 63 * 64 + 4 * col4);
 #pragma unroll
-      for (int k = 0; k < kNP; ++k) {
-        const int l = (t >> 4) + 32 * k;
-        for (int c = 0; c < nb; ++c) {
-          const float ck = cks[(c0 + c) * 64 + l];
-          const float4 sv = *reinterpret_cast<const float4*>(svk + c * 64 + 4 * (t & 15));
-          pacc[k].x = fmaf(ck, sv.x, pacc[k].x);
-          pacc[k].y = fmaf(ck, sv.y, pacc[k].y);
-          pacc[k].z = fmaf(ck, sv.z, pacc[k].z);
-          pacc[k].w = fmaf(ck, sv.w, pacc[k].w);
+        for (int k = 0; k < kNP; ++k) {
+          const float4 pv = reinterpret_cast<const float4*>(r + 128)[t + kFT * k];
+          const float ck = r[kRecC + (t >> 4) + 32 * k];
+          pacc[k].x = fmaf(ck, sv.x, pacc[k].x + pv.x);
+          pacc[k].y = fmaf(ck, sv.y, pacc[k].y + pv.y);
+          pacc[k].z = fmaf(ck, sv.z, pacc[k].z + pv.z);
+          pacc[k].w = fmaf(ck, sv.w, pacc[k].w + pv.w);
         }
       }
-      __syncthreads();   // svk is refilled by the next batch
+      c0 += nb;
+      ++nbatch;
+      __syncthreads();   // the buffers and the batch size are rewritten by the next batch
     }
     if (t < 64) {
       S1d[t] = a1;
@@ -1430,12 +1426,13 @@ __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, u
   tc_fence_before();
   __syncthreads();
   trace_mark(p, 5);
-  // one thread (in warp 15, which issues no reduces) issues the products in chunk order, each
-  // chunk's four followed by its commit, so the epilogues can start while later chunks are issued
-  if (t == kIssueP2) {
-    tc_fence_after();
-    const uint32_t id = idesc(1, 128, 64, 0, 0);
-    for (int gc = 0; gc < nch; ++gc) {
+  // each chunk's four products and its commit come from its own thread (lane 0 of warp kP2Warp0 + gc,
+  // warps that issue no reduces), so the issues of different chunks overlap
+  {
+    const int gc = w - kP2Warp0;
+    if (lane == 0 && gc >= 0 && gc < nch) {
+      tc_fence_after();
+      const uint32_t id = idesc(1, 128, 64, 0, 0);
       int s, lo, nrows;
       R.chunk(gc, s, lo, nrows);
       const uint64_t ca = desc_sw128(sbase + kOffC + gc * 16384, 16, 1024);
@@ -1509,7 +1506,7 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
   const Rows& R = *Rsm;
   const bool solver = g < U;
   if (t == 0) {
-    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, b == kBarDrain ? 2 : 1);
+    for (int b = 0; b < kNumBars; ++b) mbar_init(bars + b, b == kBarDrain ? kDrainCount : 1);
     mbar_init_fence();
     if (g == 0) *p.status = 0;
     if (!solver) pass1_prefetch(R, sm, bars, &tmapV, &tmapQ);
@@ -1521,51 +1518,78 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     tma_prefetch_desc(&tmapVp);
   }
 
-  // ---- phase 0: landmark pooling, one warp per landmark ----
-  // lane = (token group tg = lane / 8, 8 channels c8 = lane % 8); each load instruction of the
-  // warp covers 4 window tokens x 128 bytes, all loads of a window are issued before use.
+  // ---- phase 0: landmark pooling ----
+  // A landmark's r x r window is pooled by `span` warps of one CTA (1 for windows of at most 64 tokens,
+  // up to 4 for larger ones), each summing its share of the window's tokens in steps of 64; the partial
+  // sums meet in shared memory (C slot 0, free until the first chunk) and the group's first warp adds
+  // them in warp order. lane = (token group tg = lane / 8, 8 channels c8 = lane % 8); each load
+  // instruction of a warp covers 4 window tokens x 128 bytes, all loads of a step are issued before use.
   {
     const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(p.Q);
     const int total = U * m, Wr = p.W / p.r, rr = p.r * p.r;
+    const int span = rr >= 256 ? 4 : (rr >= 128 ? 2 : 1);
+    const int groups = kWarps / span, grp = w / span, part = w % span;
     const float inv = 1.f / (float)rr;
     const int tg = lane >> 3, c8 = lane & 7;
-    for (int gl = g * (kFT / 32) + w; gl < total; gl += gridDim.x * (kFT / 32)) {
-      const int u = gl / m, l = gl % m;
-      const int y0 = (l / Wr) * p.r, x0 = (l % Wr) * p.r;
-      const __nv_bfloat16* base = Q + ((size_t)u * N) * 64 + 8 * c8;
+    float* psum = reinterpret_cast<float*>(sm + kOffC);   // [kWarps][64] partial sums
+    for (int gl0 = g * groups; gl0 < total; gl0 += gridDim.x * groups) {
+      const int gl = gl0 + grp;   // the group's landmark (the whole CTA takes the same loop trips)
       float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int k0 = 0; k0 < rr; k0 += 64) {
-        uint4 v[16];
+      const int u = gl < total ? gl / m : 0, l = gl % m;
+      if (gl < total) {
+        const int y0 = (l / Wr) * p.r, x0 = (l % Wr) * p.r;
+        const __nv_bfloat16* base = Q + ((size_t)u * N) * 64 + 8 * c8;
+        for (int k0 = 64 * part; k0 < rr; k0 += 64 * span) {
+          uint4 v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int k = k0 + tg + 4 * i;
-          v[i] = make_uint4(0u, 0u, 0u, 0u);
-          if (k < rr) {
-            const int dy = k / p.r, dx = k % p.r;
-            v[i] = __ldg(reinterpret_cast<const uint4*>(base + ((size_t)(y0 + dy) * p.W + x0 + dx) * 64));
+          for (int i = 0; i < 16; ++i) {
+            const int k = k0 + tg + 4 * i;
+            v[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (k < rr) {
+              const int dy = k / p.r, dx = k % p.r;
+              v[i] = __ldg(reinterpret_cast<const uint4*>(base + ((size_t)(y0 + dy) * p.W + x0 + dx) * 64));
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            a[0] += bf_lo(v[i].x); a[1] += bf_hi(v[i].x); a[2] += bf_lo(v[i].y); a[3] += bf_hi(v[i].y);
+            a[4] += bf_lo(v[i].z); a[5] += bf_hi(v[i].z); a[6] += bf_lo(v[i].w); a[7] += bf_hi(v[i].w);
           }
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          a[0] += bf_lo(v[i].x); a[1] += bf_hi(v[i].x); a[2] += bf_lo(v[i].y); a[3] += bf_hi(v[i].y);
-          a[4] += bf_lo(v[i].z); a[5] += bf_hi(v[i].z); a[6] += bf_lo(v[i].w); a[7] += bf_hi(v[i].w);
+        for (int e = 0; e < 8; ++e) {
+          a[e] += __shfl_xor_sync(0xffffffffu, a[e], 8);
+          a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
         }
       }
+      if (span > 1) {
+        if (tg == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        a[e] += __shfl_xor_sync(0xffffffffu, a[e], 8);
-        a[e] += __shfl_xor_sync(0xffffffffu, a[e], 16);
+          for (int e = 0; e < 8; ++e) psum[w * 64 + 8 * c8 + e] = a[e];
+        }
+        named_bar_sync(1 + grp, 32 * span);
+        if (part == 0 && tg == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float acc = a[e];
+            for (int q = 1; q < span; ++q) acc += psum[(w + q) * 64 + 8 * c8 + e];
+            a[e] = acc;
+          }
+        }
+        named_bar_sync(1 + grp, 32 * span);   // psum is rewritten by the next trip
       }
-      if (tg == 0) {
-        float* dst = p.L + ((size_t)u * m + l) * 64 + 8 * c8;
-        *reinterpret_cast<float4*>(dst) = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
-      }
-      // one landmark of unit u is out: the unit's consumers wait for m of them (no grid barrier)
-      __syncwarp();
-      if (lane == 0) {
-        __threadfence();
-        red_release_add_u64(fa.lready + u, 1ull);
+      if (gl < total && part == 0) {
+        if (tg == 0) {
+          float* dst = p.L + ((size_t)u * m + l) * 64 + 8 * c8;
+          *reinterpret_cast<float4*>(dst) = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
+          *reinterpret_cast<float4*>(dst + 4) = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
+        }
+        // one landmark of unit u is out: the unit's consumers wait for m of them (no grid barrier)
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          red_release_add_u64(fa.lready + u, 1ull);
+        }
       }
     }
   }
@@ -1593,10 +1617,11 @@ __global__ void __launch_bounds__(kFT, 1) k_fused_forward(const Params p, const 
     row_dwc(p, fa, R, sm, bars, &tmapVp);
     pass2_all(p, fa, R, sm, sbase, tmem, bars, &tmapO);
   }
-  // drain: the tcgen05 operations of the two issuing threads (thread 0: solver and pass-1 products;
-  // kIssueP2: pass-2 products) have completed before TMEM is released. In a normal run each was
-  // waited already; after an expired wait this bounds the wait for any still running.
-  if (t == 0 || t == kIssueP2) mma_commit(bars + kBarDrain);
+  // drain: the tcgen05 operations of every issuing thread (thread 0: solver and pass-1 products;
+  // lane 0 of warps kP2Warp0 .. kP2Warp0 + 6: pass-2 products) have completed before TMEM is released.
+  // In a normal run each was waited already; after an expired wait this bounds the wait for any still
+  // running. (A commit with nothing outstanding arrives at once.)
+  if (t == 0 || (lane == 0 && w >= kP2Warp0 && w < kP2Warp0 + kMaxChunks - 1)) mma_commit(bars + kBarDrain);
   if (t == 0) mbar_wait(bars + kBarDrain, 0, p.status, kStatusTimeout);
   __syncthreads();
   trace_mark(p, 15);
@@ -1646,10 +1671,10 @@ __global__ void __launch_bounds__(kFT, 1) k_ns_tc(const Params p) {
   }
 }
 
-// Flag area: four [U] flag arrays (lready, cnt, xready, mready), each padded to 256 B; then the
+// Flag area: three [U] flag arrays (lready, xready, mready), each padded to 256 B; then the
 // per-CTA pass-1 records and the per-unit M' images.
 static size_t flag_stride(int U) { return 256 * (size_t)((U * 8 + 255) / 256); }
-static size_t flag_bytes(int U) { return 4 * flag_stride(U); }
+static size_t flag_bytes(int U) { return 3 * flag_stride(U); }
 
 size_t fused_workspace_bytes(int U) {
   return flag_bytes(U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec + (size_t)U * 8192;
@@ -1786,7 +1811,8 @@ static void plan_pass1_warps(int m, FusedArgs& fa) {
 cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws, unsigned long long epoch,
                                  cudaStream_t st) {
   if (epoch == 1) {
-    const cudaError_t e = cudaMemsetAsync(fused_ws, 0, flag_bytes(p.U), st);
+    // the flags and the records (whose published flags hold epochs of earlier launches)
+    const cudaError_t e = cudaMemsetAsync(fused_ws, 0, flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec, st);
     if (e != cudaSuccess) return e;
   }
   CUtensorMap tmap, tmapq, tmapo, tmapvp;
@@ -1798,9 +1824,8 @@ cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws
   fa.epoch = epoch;
   const size_t fs = flag_stride(p.U);
   fa.lready = reinterpret_cast<unsigned long long*>(fused_ws);
-  fa.cnt = reinterpret_cast<unsigned long long*>(fused_ws + fs);
-  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + 2 * fs);
-  fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 3 * fs);
+  fa.xready = reinterpret_cast<unsigned long long*>(fused_ws + fs);
+  fa.mready = reinterpret_cast<unsigned long long*>(fused_ws + 2 * fs);
   fa.mimg = fused_ws + flag_bytes(p.U) + sizeof(float) * (size_t)kMaxGrid * 2 * kRec;
   fa.rec = reinterpret_cast<float*>(fused_ws + flag_bytes(p.U));
   plan_pass1_warps(p.m, fa);

@@ -190,6 +190,14 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, int x, int y
                "r"(x), "r"(y), "r"(z), "r"(smem_u32(src))
                : "memory");
 }
+// untiled bulk copy global -> this CTA's shared memory, completing (complete_tx) on `bar`; both addresses
+// 16-byte aligned, `bytes` a multiple of 16 (no multicast)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // every bulk store this thread committed has completed
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
