@@ -634,7 +634,7 @@ __device__ void solver_diagnostics(const Params& p, unsigned char* sm, uint32_t 
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3: C for a 128-row chunk: this warp's landmarks [j0, j0 + LT), lane rows lane + 32 a.
+// Phase 2 (pass 1): C for a 128-row chunk: this warp's landmarks [j0, j0 + LT), lane rows lane + 32 a.
 // ---------------------------------------------------------------------------------------
 // Q rows come from a bf16 SW128 tile (TMA): one 16-byte read gives 8 channels of a row, and the
 // lanes' rows spread the reads over all banks.
@@ -1133,7 +1133,7 @@ __device__ void solver_dwc(const Params& p, const FusedArgs& fa, unsigned char* 
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 3, on the unit's solver CTA once every contributor's pass-1 record is out (X is its own):
+// Phase 3, on the unit's solver CTA as the contributors' pass-1 records come out (X is its own):
 // sum the records (each rebased from its column shift c_k to none: S1 += S1'_k + n_k c_k, S2 += S2'_k +
 // 2 c_k S1'_k + n_k c_k^2 in fp64, P += P'_k + c_k (sum_i v_i)_k^T in fp32), form mu, var,
 // s = 1/sqrt(var + eps), A = C~^T V by rank-1 folding (§关键设计 1), M = X A (fp32 FMA), M' = diag(s) M
@@ -1392,13 +1392,14 @@ __device__ void solver_combine(const Params& p, const FusedArgs& fa, unsigned ch
 }
 
 // ---------------------------------------------------------------------------------------
-// Phase 4: O += C M' + b for every chunk, onto the DWC values pass 1 wrote to O. M'^T and b of each
-// segment's unit come from this CTA's own combine (segment 0's image in the M' area, segment 1's at
-// kOffImg1). All products are issued at once, each with its own barrier, and the epilogues (+ b,
-// bf16) follow chunk by chunk. The bf16 rows are staged in the chunk's C slot (free once its product
-// is done) and leave by TMA reduce-adds of 32-row quarters onto O: warps w, w + 4, w + 8, w + 12 hold
-// the same 32 rows (16 channels each) and meet on named barrier 1 + w % 4 before warp w % 4 issues
-// the quarter's reduce.
+// Phase 4: O += (C - c) M' + b_k for every chunk, onto the DWC values already in O (from this CTA's
+// row_dwc or from the unit's solver). M'^T of each segment's unit is the image its solver CTA published
+// (copied to the M' area for segment 0, to kOffImg1 for segment 1); b_k is the bias that solver wrote
+// into this CTA's record for its column shift. Each chunk's products are issued by their own thread
+// with their own barrier, and the epilogues (+ b_k, bf16) follow chunk by chunk. The bf16 rows are
+// staged in the chunk's C slot (free once its product is done) and leave by TMA reduce-adds of 32-row
+// quarters onto O: warps w, w + 4, w + 8, w + 12 hold the same 32 rows (16 channels each) and meet on
+// named barrier 1 + w % 4 before warp w % 4 issues the quarter's reduce.
 // ---------------------------------------------------------------------------------------
 __device__ void pass2_all(const Params& p, const FusedArgs& fa, const Rows& R, unsigned char* sm, uint32_t sbase,
                           uint32_t tmem, uint64_t* bars, const CUtensorMap* tmapO) {

@@ -191,7 +191,7 @@ __device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, int x, int y
                : "memory");
 }
 // untiled bulk copy global -> this CTA's shared memory, completing (complete_tx) on `bar`; both addresses
-// 16-byte aligned, `bytes` a multiple of 16 (no multicast)
+// 16-byte aligned, `bytes` a multiple of 16; one destination CTA
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
