@@ -90,11 +90,14 @@ def workload_config(wl, extra=None):
     return cfg
 
 
-def dtype_label(path: str) -> str:
-    """The arithmetic of the call (storage type aside), by the path that serves it."""
+def dtype_label(path: str, kernel: str = "") -> str:
+    """The arithmetic of the call (storage type aside), by the path and pass-2 kernel that serve it."""
     if path == "fused":
         return ("bf16-operand MMA (tcgen05 kind::f16), fp32 accumulate; fp32 l1 distances and exp; "
                 "split-TF32 Newton-Schulz (3 tcgen05 kind::tf32 products per step)")
+    if kernel == "k_stream_pass2":
+        return ("fp32 l1 distances and exp; bf16-operand C^T V and C M' on tcgen05 (kind::f16), fp32 accumulate; "
+                "split-TF32 tcgen05 Newton-Schulz")
     return "fp32 SIMT distances and products; split-TF32 tcgen05 Newton-Schulz"
 
 
@@ -321,7 +324,7 @@ def run_backward(args):
         "metric": "tokens/s per forward + backward call", "value": wl.units * wl.N / (step_ms * 1e-3),
         "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": step_ms,
         "forward_ms": fwd_ms / K, "backward_ms": bwd_ms / K, "higher_is_better": True,
-        "dtype": dtype_label(mod.path) + "; backward: fp32 SIMT main pass, split-TF32 tcgen05 reverse products",
+        "dtype": dtype_label(mod.path, mod.dominant_kernel) + "; backward: fp32 SIMT main pass, split-TF32 tcgen05 reverse products",
         "data": "synthetic", "config": workload_config(wl, {"path": mod.path, "inputs": "resident, no L2 flush"}),
     }), flush=True)
 
@@ -397,7 +400,8 @@ def run_seqsplit(args):
             "metric": f"tokens/s per Laplacian-Nyström attention call (N={wl.N},d={wl.d},m={wl.m}), "
                       f"grid rows split over ranks", "value": tokens * K / (ms * 1e-3), "unit": "tokens/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
-            "scaling": "strong", "vs_baseline": None, "dtype": dtype_label("generic"),
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": dtype_label("generic", "k_stream_pass2" if wl.dtype == "bf16" and wl.d == 64 else ""),
             "data": "synthetic",
             "config": workload_config(wl, {"path": "generic (band calls)", "parallelism": f"seqsplit{world}",
                                            "bands": [seqsplit.band_rows(wl.H, world, k) for k in range(world)],
@@ -523,7 +527,7 @@ def main():
             f"tokens/s per Laplacian-Nyström attention call (N={wl.N},d={wl.d},m={wl.m}); % of roofline",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": dtype_label(mod.path), "data": "synthetic",
+            "vs_baseline": None, "dtype": dtype_label(mod.path, mod.dominant_kernel), "data": "synthetic",
             "config": workload_config(wl, {
                 "path": mod.path, "whiten": args.whiten,
                 "parallelism": f"replicas{world}" if world > 1 else "single",

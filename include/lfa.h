@@ -247,8 +247,8 @@ lfa_status lfa_cg_solve(const float* W, const float* B, float* Y, int U, int m, 
  * written as fp32 [N][m] to the device buffer C_out by the per-stage kernels' tile code
  * (fp32 distance and exp2f), after pooling Q's landmarks into the handle's workspace. That
  * pooling replaces the saved forward context: lfa_backward then needs a new lfa_forward
- * (LFA_ERR_STATE until then). For the C that a fused forward itself computes, see
- * lfa_debug_capture_cross. */
+ * (LFA_ERR_STATE until then). For the C that a forward itself multiplies (the fused kernel, or the
+ * tensor-core pass 2 of the per-stage path), see lfa_debug_capture_cross. */
 lfa_status lfa_debug_cross_kernel(lfa_handle h, const void* Q, int unit, float* C_out,
                                   void* stream);
 
@@ -269,8 +269,11 @@ lfa_status lfa_debug_spin_test(lfa_handle h, long long budget_cycles);
  * of C over the first 16 tokens of its rows of the unit (the bias of pass 2 adds c back exactly); C
  * is computed by ex2.approx from the fp32 distance sum. The copy is that bf16 value widened to fp32
  * plus c, and shift_out (NULL, or a device buffer of N*m floats) receives c for every entry. On the
- * per-stage path the forward's tile code computes C again for the copy, in fp32, and shift_out is
- * zeroed. Host-only; LFA_ERR_INVALID_ARG for a bad unit or a NULL C_out. */
+ * per-stage path with bf16 tokens and d = 64, pass 2 multiplies bf16(C - mu) on the tensor cores (mu the
+ * column mean, C again by ex2.approx from the fp32 distance sum) and copies that value widened plus mu,
+ * with mu in shift_out. On the other per-stage shapes (fp32 tokens, d != 64) the forward's CUDA-core tile
+ * code computes C again for the copy, in fp32, and shift_out is zeroed. Host-only; LFA_ERR_INVALID_ARG
+ * for a bad unit or a NULL C_out. */
 lfa_status lfa_debug_capture_cross(lfa_handle h, int unit, float* C_out, float* shift_out);
 
 /* Copy the forward context of one unit (device -> device, fp32): landmarks L [m][d],

@@ -195,6 +195,7 @@ lfa_status ensure_attributes() {
   if (lfa::gemm_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::ns_tc_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (lfa::cg_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
+  if (lfa::stream_set_attributes() != cudaSuccess) return LFA_ERR_CUDA;
   if (dev < 64) g_attr_done |= 1ull << dev;
   return LFA_OK;
 }
@@ -329,10 +330,17 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
     if (lfa::launch_fused_forward(p, h->grid, h->ws + h->lay.fused, epoch, st) != cudaSuccess) return LFA_ERR_CUDA;
     h->epoch = epoch;
   } else {
+    // the tcgen05 pass 2 copies the C it multiplies (bf16(C - mu) widened, mu added back) as it goes;
+    // the CUDA-core passes keep C in registers: their tile code runs once more for the copy
+    const bool in_pass = cap && lfa::stream_eligible(p);
+    if (in_pass) {
+      p.dbgC = cap;
+      p.dbgS = cap_s;
+      p.dbg_unit = h->cap_unit;
+    }
     if (lfa::launch_generic_forward(p, st) != cudaSuccess) return LFA_ERR_CUDA;
-    // the per-stage passes keep C in registers: the same tile code, run once more for the copy
-    if (cap && lfa::launch_cross_kernel(p, h->cap_unit, cap, st) != cudaSuccess) return LFA_ERR_CUDA;
-    if (cap && cap_s &&
+    if (cap && !in_pass && lfa::launch_cross_kernel(p, h->cap_unit, cap, st) != cudaSuccess) return LFA_ERR_CUDA;
+    if (cap && !in_pass && cap_s &&
         cudaMemsetAsync(cap_s, 0, sizeof(float) * (size_t)h->p.N * h->p.m, st) != cudaSuccess)
       return LFA_ERR_CUDA;
   }
@@ -620,7 +628,8 @@ lfa_status lfa_debug_trace(lfa_handle h, unsigned long long* dev_buf) {
 
 const char* lfa_dominant_kernel(lfa_handle h) {
   if (!h) return "invalid";
-  return h->path == 1 ? "k_fused_forward" : "k_pass2";
+  if (h->path == 1) return "k_fused_forward";
+  return lfa::stream_eligible(h->p) ? "k_stream_pass2" : "k_pass2";
 }
 
 int lfa_fused_grid(lfa_handle h) { return h ? h->grid : 0; }

@@ -839,10 +839,21 @@ void pass1_t(const Params& p, cudaStream_t st) {
   else k_pass1<T, 4><<<g1, kThreads, s1, st>>>(p);
 }
 
+// (bf16 tokens with d = 64 take the tcgen05 streaming pass, whose partial records come with their own
+// count per unit)
 template <typename T>
 void pass1_reduce_t(const Params& p, cudaStream_t st) {
-  pass1_t<T>(p, st);
-  k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), p.U), kThreads, 0, st>>>(p);
+  Params q = p;
+  const int P = stream_pass1(p, st);
+  if (P > 0) q.P = P;
+  else pass1_t<T>(p, st);
+  k_combine_reduce<<<dim3(ceil_div(q.part_stride, kThreads), q.U), kThreads, 0, st>>>(q);
+}
+
+// pass 2: the tcgen05 streaming kernel for bf16 tokens with d = 64, else the CUDA-core one
+template <typename T>
+void pass2_t(const Params& p, cudaStream_t st) {
+  if (!stream_pass2(p, st)) k_pass2<T><<<dim3(p.P, p.U), kThreads, generic_smem_pass2(p.m, p.d), st>>>(p);
 }
 
 size_t rb_gram_smem(int m, int d) {
@@ -929,10 +940,9 @@ void context_t(const Params& p, cudaStream_t st) {
 
 template <typename T>
 cudaError_t forward_t(const Params& p, cudaStream_t st) {
-  const int U = p.U, m = p.m, d = p.d;
   context_t<T>(p, st);
   if (p.ev_begin) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_begin), st);
-  k_pass2<T><<<dim3(p.P, U), kThreads, generic_smem_pass2(m, d), st>>>(p);
+  pass2_t<T>(p, st);
   if (p.ev_end) cudaEventRecord(static_cast<cudaEvent_t>(p.ev_end), st);
   return cudaGetLastError();
 }
@@ -1016,10 +1026,8 @@ cudaError_t launch_ns_from_w(const Params& p, cudaStream_t st) {
 // The combine from the fp64 totals in the workspace (mu, s, A, M, M', b), then pass 2.
 cudaError_t launch_generic_finish(const Params& p, cudaStream_t st) {
   k_combine_finish<<<dim3(p.n_chunks, p.U), kThreads, (size_t)(p.m * p.d + 2 * p.m) * sizeof(float), st>>>(p);
-  if (p.dtype == LFA_BF16)
-    k_pass2<__nv_bfloat16><<<dim3(p.P, p.U), kThreads, generic_smem_pass2(p.m, p.d), st>>>(p);
-  else
-    k_pass2<float><<<dim3(p.P, p.U), kThreads, generic_smem_pass2(p.m, p.d), st>>>(p);
+  if (p.dtype == LFA_BF16) pass2_t<__nv_bfloat16>(p, st);
+  else pass2_t<float>(p, st);
   return cudaGetLastError();
 }
 

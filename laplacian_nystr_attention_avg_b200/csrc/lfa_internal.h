@@ -190,6 +190,13 @@ size_t generic_smem_pass1(int m, int d);
 size_t generic_smem_pass2(int m, int d);
 cudaError_t generic_set_attributes();
 int generic_launch_count(const Params& p);
+// tcgen05 streaming passes for bf16 tokens, d = 64, m <= 256 (lfa_stream.cu): pass 1 writes its
+// partial records with its own CTA count per unit, which it returns (0: not launched); pass 2 returns
+// false when it does not apply
+bool stream_eligible(const Params& p);
+cudaError_t stream_set_attributes();
+int stream_pass1(const Params& p, cudaStream_t st);
+bool stream_pass2(const Params& p, cudaStream_t st);
 size_t fused_workspace_bytes(int U);
 int fused_grid(const Params& p);
 cudaError_t launch_fused_forward(const Params& p, int G, unsigned char* fused_ws, unsigned long long epoch,

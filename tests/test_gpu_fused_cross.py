@@ -55,16 +55,44 @@ def test_fused_cross_kernel(name, lam):
         assert r <= 1.0, f"{name} lam={lam} unit {u}: C error {r:.3f} of the bound"
 
 
-def test_capture_on_generic_path_matches_debug_kernel(monkeypatch):
-    # the per-stage path copies C with its own tile code: identical to lfa_debug_cross_kernel
-    monkeypatch.setenv("LFA_FORWARD_PATH", "generic")
-    wl = pu.workload("pvt2")
+# Per-stage path with bf16 tokens and d = 64: pass 2 multiplies bf16(C - mu) on the tensor cores, mu
+# the column mean; the copy is that value widened plus mu, under the same bound (shift mu). Large grids
+# are checked on a row sample (every 7th row and the last rows).
+STREAM_CASES = [("pvt2", 4.0, "generic"), ("pvt2", 32.0, "generic"), ("hr196", 4.0, None), ("long", 4.0, None)]
+
+
+@pytest.mark.parametrize("name,lam,path", STREAM_CASES)
+def test_stream_cross_kernel(name, lam, path, monkeypatch):
+    wl = pu.workload(name, lam=lam)
+    x = pu.inputs_for(wl)
+    if path:
+        monkeypatch.setenv("LFA_FORWARD_PATH", path)
+    mod = pu.gpu_module(wl, True, False)
+    monkeypatch.delenv("LFA_FORWARD_PATH", raising=False)
+    assert mod.path == "generic"
+    Q, V = x.Q_store.cuda(), x.V_store.cuda()
+    rows = np.unique(np.concatenate([np.arange(0, wl.H * wl.W, 7), np.arange(wl.H * wl.W - 70, wl.H * wl.W)]))
+    for u in sorted({0, wl.units - 1}):
+        Cg, Sg = (t.cpu().numpy().astype(np.float64)[rows] for t in mod.capture_cross(Q, V, u))
+        b, h = divmod(u, wl.heads)
+        q = x.Q[b, h].double().numpy()
+        L = O.pool_landmarks(q, wl.H, wl.W, wl.r)
+        mu_ref = O.laplacian_kernel(q, L, wl.lam).mean(axis=0)
+        assert np.allclose(Sg, mu_ref[None, :], rtol=1e-4, atol=0.0), f"{name}: shift is not the column mean"
+        r = fused_c_error(Cg, Sg, q[rows], L, wl.lam)
+        assert r <= 1.0, f"{name} lam={lam} unit {u}: C error {r:.3f} of the bound"
+
+
+def test_capture_on_cuda_core_path_matches_debug_kernel():
+    # fp32 tokens take the CUDA-core passes, which copy C with their own tile code: identical to
+    # lfa_debug_cross_kernel
+    wl = pu.workload("pr1")
     x = pu.inputs_for(wl)
     mod = pu.gpu_module(wl, True, False)
-    monkeypatch.delenv("LFA_FORWARD_PATH")
+    assert mod.path == "generic"
     Q, V = x.Q_store.cuda(), x.V_store.cuda()
-    a, sh = mod.capture_cross(Q, V, 5)
-    b = mod.cross_kernel(Q, 5)
+    a, sh = mod.capture_cross(Q, V, 0)
+    b = mod.cross_kernel(Q, 0)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     assert not sh.any()
