@@ -3,9 +3,17 @@ forward and the oracle.
 
 laplacian_nystr_attention_avg_b200.seqsplit.forward_bands runs the same three exchanges as the
 multi-rank driver (sums of the landmark shares and of the fp64 pass-1 partials, neighbouring V rows
-as the DWC halo) in one process. The assembled O must match the per-stage whole-grid forward to fp32
-rounding (only the order of the sums differs: max |diff| / max |O| <= 1e-5 per unit) and the oracle
-within the forward tolerances (1e-3 max-relative for fp32, 2e-2 normwise for bf16).
+as the DWC halo) in one process. The assembled O must match the per-stage whole-grid forward and the oracle
+within the forward tolerances (1e-3 max-relative for fp32, 2e-2 normwise for bf16). Against the
+whole-grid forward:
+  * fp32 tokens (CUDA-core passes): only the order of the sums differs, max |diff| / max |O| <= 1e-5
+    per unit;
+  * bf16 tokens with d = 64 (tensor-core passes): pass 1 multiplies bf16(C - c), c the column mean of
+    C over each thread block's first tile, so the band split (other blocks, other c) changes the
+    rounding. Unwhitened, that rounding is relative to C - c, far below the mean part of C that
+    dominates O: max |diff| / max |O| <= 2^-8 (one bf16 rounding of the result). Whitened, O keeps
+    only the centred part, of the size of C - c, so each side carries the bf16 unit roundoff 2^-8 of
+    its products: normwise |diff| / |O| <= 2 x 2^-8 = 2^-7 per unit.
 """
 import numpy as np
 import pytest
@@ -52,10 +60,13 @@ def test_bands_match_whole_grid(wl, nb, whiten, monkeypatch):
     torch.cuda.synchronize()
     units = tuple(range(wl.units))
     a, b = pu.unit_rows(O_sp, units), pu.unit_rows(O_full, units)
-    # identical up to the order of the fp64 sums (and one bf16 rounding of each result)
-    ulp = 2.0 ** -8 if wl.dtype == "bf16" else 1e-5
+    bf16 = wl.dtype == "bf16"
     for u in units:
-        assert np.max(np.abs(a[u] - b[u])) <= ulp * np.max(np.abs(b[u])), f"unit {u}"
+        if bf16 and whiten:
+            assert np.linalg.norm(a[u] - b[u]) <= 2.0 ** -7 * np.linalg.norm(b[u]), f"unit {u}"
+        else:
+            ulp = 2.0 ** -8 if bf16 else 1e-5
+            assert np.max(np.abs(a[u] - b[u])) <= ulp * np.max(np.abs(b[u])), f"unit {u}"
     check = (0, wl.units - 1)
     ref = pu.oracle_forward(wl, whiten, False, check)
     want = np.stack([ref.O[divmod(u, wl.heads)] for u in check])
