@@ -499,13 +499,15 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
             [&](cudaStream_t s) {
               if (T_ == 0) return;
               k_init_iterate<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, s>>>(b);
+              const NsChain c{p.Wm, mm, p.Y, mm, b.its, nullptr, its_stride, mm, m, T_ - 1, 1, p.status};
+              if (m > kSmallM && launch_ns_chain(c, U, s)) return;
               for (int k = 0; k + 1 < T_; ++k) {
                 const float* Xk = b.its + k * mm;
                 const MmJob y{p.Wm, mm, Xk, its_stride, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};  // Y = 2I - W X_k
-                launch_mm(&y, 1, m, U, s);
+                launch_mm(&y, 1, m, U, s, p.status);
                 const MmJob xn{Xk, its_stride, p.Y, mm, nullptr, 0, b.its + (k + 1) * mm, its_stride,  // X_{k+1} = X_k Y
                                1.f, 0.f, 0.f, 0, 0};
-                launch_mm(&xn, 1, m, U, s);
+                launch_mm(&xn, 1, m, U, s, p.status);
               }
             });
   if (e != cudaSuccess) return e;
@@ -519,13 +521,13 @@ cudaError_t backward_t(const BwdParams& b, cudaStream_t st) {
         {Xk, its_stride, G, mm, nullptr, 0, b.T1, mm, 1.f, 0.f, 0.f, 1, 0},      // T1 = X_k^T G
         {G, mm, Xk, its_stride, nullptr, 0, b.T2, mm, 1.f, 0.f, 0.f, 0, 1},      // T2 = G X_k^T
         {p.Wm, mm, Xk, its_stride, nullptr, 0, b.T3, mm, 1.f, 0.f, 0.f, 1, 1}};  // T3 = W^T X_k^T
-    launch_mm(s1, 3, m, U, st);
+    launch_mm(s1, 3, m, U, st, p.status);
     const MmJob s2[2] = {
         {b.T1, mm, Xk, its_stride, b.dW, mm, b.dW, mm, -1.f, 1.f, 0.f, 0, 1},    // dW -= T1 X_k^T
         {b.T2, mm, p.Wm, mm, G, mm, Gn, mm, -1.f, 2.f, 0.f, 0, 1}};              // Gn = 2G - T2 W^T
-    launch_mm(s2, 2, m, U, st);
+    launch_mm(s2, 2, m, U, st, p.status);
     const MmJob s3{b.T3, mm, G, mm, Gn, mm, Gn, mm, -1.f, 1.f, 0.f, 0, 0};      // Gn -= T3 G
-    launch_mm(&s3, 1, m, U, st);
+    launch_mm(&s3, 1, m, U, st, p.status);
     float* tmp = G;
     G = Gn;
     Gn = tmp;
@@ -570,9 +572,9 @@ cudaError_t backward_set_attributes() {
 }
 
 int backward_launch_count(const Params& p) {
-  // pass 1 + reduce, combine, iterates (1 + 2 (T - 1)), 3 T reverse launches (6 products per step, batched), gram part of dL,
+  // pass 1 + reduce, combine, iterates (1 + 2 (T - 1), or 1 + 1 as one cluster launch), 3 T reverse launches (6 products per step, batched), gram part of dL,
   // main pass, dL reduction, dQ
-  const int its = p.T > 0 ? 1 + 2 * (p.T - 1) : 0;
+  const int its = p.T > 0 ? 1 + (p.m > kSmallM && ns_chain_fits(p.m) ? (p.T > 1 ? 1 : 0) : 2 * (p.T - 1)) : 0;
   return 2 + 1 + (p.whiten == 2 ? 1 : 0) + its + 3 * p.T + 1 + 1 + 1 + 1;
 }
 

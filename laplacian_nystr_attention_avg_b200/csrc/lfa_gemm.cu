@@ -10,6 +10,14 @@
 // (two 128-byte SW128 K-halves of fp32 per row). The operands of step c + 1 are already in registers
 // while the 24 MMAs of step c run: they are split and stored into the other shared-memory stage, and
 // the global loads of step c + 2 are issued right after, so one L2 latency overlaps each step.
+//
+// The Newton-Schulz chains (the forward's X_{k+1} = X_k (2I - W X_k), k < T, and the backward's
+// iterates X_1 .. X_{T-1}) also run as ONE launch, k_ns_chain: a thread-block cluster per unit whose
+// blocks each own one 128 x 64 output tile of every product and meet at a cluster barrier between
+// products (operands through L2, loads that bypass L1). This removes the per-product launch and the
+// cold instruction fetch that dominated it.
+#include <mutex>
+
 #include "lfa_internal.h"
 #include "lfa_sm100.cuh"
 
@@ -19,15 +27,15 @@ namespace {
 using namespace sm100;
 
 constexpr int kTM = 128, kTN = 64, kKS = 64;
-constexpr int kGT = 256;                          // threads per CTA
+constexpr int kGT = 512;                          // threads per CTA
 constexpr uint32_t kAH = kTM * 128;               // bytes of one K-half of one A split tile
 constexpr uint32_t kBH = kTN * 128;               // bytes of one K-half of one B split tile
 // stage: A hi [2 halves], A lo [2], B hi [2], B lo [2]
 constexpr uint32_t kOffAhi = 0, kOffAlo = 2 * kAH, kOffBhi = 4 * kAH, kOffBlo = 4 * kAH + 2 * kBH;
 constexpr uint32_t kStage = 4 * kAH + 4 * kBH;    // 96 KB
 constexpr uint32_t kGemmSmem = 2 * kStage + 1024 + 64;
-constexpr int kAR = kTM * kKS / 4 / kGT;          // float4 groups of A per thread and step (8)
-constexpr int kBR = kTN * kKS / 4 / kGT;          // of B (4)
+constexpr int kAR = kTM * kKS / 4 / kGT;          // float4 groups of A per thread and step (4)
+constexpr int kBR = kTN * kKS / 4 / kGT;          // of B (2)
 
 // byte offset of (row, fp32 column k < 64) in a K-major split tile made of two SW128 K-halves
 __device__ __forceinline__ uint32_t kofs(int row, int k, uint32_t half_bytes) {
@@ -39,32 +47,21 @@ struct Regs {
   float4 b[kBR];
 };
 
-__global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
-  unsigned char* sm = smem_raw + pad;
-  const uint32_t sbase = smem_u32(sm);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kStage);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + 2 * kStage + 32);
-  __shared__ int status_dummy;
-  const int jz = blockIdx.z / U, u = blockIdx.z % U;
-  const MmJob J = jobs.job[jz];
+// One 128 x 64 output tile (rows i0.., columns j0..) of job J for unit u. The two shared-memory stages
+// and their commit barriers continue across calls: step c of this tile is global step gs + c, staged in
+// buffer (gs + c) & 1 and committed on that buffer's barrier as its ((gs + c) >> 1)-th completion; gs
+// advances by the tile's step count. Every commit is waited before the call returns, so the stages
+// and the TMEM accumulator are free for the next call. Operands are read through L2 (ld.global.cg):
+// in a chain they were written by other thread blocks since the previous product. TA / TB: the job's
+// transposes (J.ta, J.tb), fixed at compile time so that each variant's code holds only its own paths.
+template <int TA, int TB>
+__device__ __noinline__ void mm_tile(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm, uint32_t sbase, uint32_t tmem,
+                        uint64_t* bars, int* status, int& gs) {
   const float* A = J.A + u * J.a_stride;
   const float* B = J.B + u * J.b_stride;
   const float* Cin = J.C ? J.C + u * J.c_stride : nullptr;
   float* Out = J.O + u * J.o_stride;
-  const int i0 = blockIdx.y * kTM, j0 = blockIdx.x * kTN;
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-  if (w == 0) {
-    tmem_alloc(tmem_slot, 64);
-    tmem_relinquish();
-  }
-  if (t == 0) {
-    mbar_init(bars + 0, 1);
-    mbar_init(bars + 1, 1);
-    mbar_init_fence();
-    status_dummy = 0;
-  }
   const bool vec = (m & 3) == 0;   // rows start on 16-byte boundaries
   // Group e of a step covers 4 consecutive elements along the stored matrix's contiguous index:
   //   A untransposed: row i = e / 16, k = 4 (e % 16) .. ;  transposed: row k = e / 32, i = 4 (e % 32) ..
@@ -73,12 +70,12 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (row < nrow) {
       const float* src = base + (size_t)row * m + col;
-      if (vec && col + 3 < ncol) v = *reinterpret_cast<const float4*>(src);
+      if (vec && col + 3 < ncol) v = __ldcg(reinterpret_cast<const float4*>(src));
       else {
-        v.x = col + 0 < ncol ? src[0] : 0.f;
-        v.y = col + 1 < ncol ? src[1] : 0.f;
-        v.z = col + 2 < ncol ? src[2] : 0.f;
-        v.w = col + 3 < ncol ? src[3] : 0.f;
+        v.x = col + 0 < ncol ? __ldcg(src + 0) : 0.f;
+        v.y = col + 1 < ncol ? __ldcg(src + 1) : 0.f;
+        v.z = col + 2 < ncol ? __ldcg(src + 2) : 0.f;
+        v.w = col + 3 < ncol ? __ldcg(src + 3) : 0.f;
       }
     }
     return v;
@@ -88,12 +85,12 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
 #pragma unroll
     for (int x = 0; x < kAR; ++x) {
       const int e = t + kGT * x;
-      r.a[x] = J.ta ? ld4(A, k0 + (e >> 5), i0 + 4 * (e & 31), m, m) : ld4(A, i0 + (e >> 4), k0 + 4 * (e & 15), m, m);
+      r.a[x] = TA ? ld4(A, k0 + (e >> 5), i0 + 4 * (e & 31), m, m) : ld4(A, i0 + (e >> 4), k0 + 4 * (e & 15), m, m);
     }
 #pragma unroll
     for (int x = 0; x < kBR; ++x) {
       const int e = t + kGT * x;
-      r.b[x] = J.tb ? ld4(B, j0 + (e >> 4), k0 + 4 * (e & 15), m, m) : ld4(B, k0 + (e >> 4), j0 + 4 * (e & 15), m, m);
+      r.b[x] = TB ? ld4(B, j0 + (e >> 4), k0 + 4 * (e & 15), m, m) : ld4(B, k0 + (e >> 4), j0 + 4 * (e & 15), m, m);
     }
   };
   auto put = [&](unsigned char* hi, unsigned char* lo, uint32_t off, float v) {
@@ -116,7 +113,7 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
 #pragma unroll
     for (int x = 0; x < kAR; ++x) {
       const int e = t + kGT * x;
-      if (!J.ta) {
+      if constexpr (!TA) {
         put4(st + kOffAhi, st + kOffAlo, kofs(e >> 4, 4 * (e & 15), kAH), r.a[x]);
       } else {
         const int k = e >> 5, i = 4 * (e & 31);
@@ -129,7 +126,7 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
 #pragma unroll
     for (int x = 0; x < kBR; ++x) {
       const int e = t + kGT * x;
-      if (J.tb) {
+      if constexpr (TB) {
         put4(st + kOffBhi, st + kOffBlo, kofs(e >> 4, 4 * (e & 15), kBH), r.b[x]);
       } else {
         const int k = e >> 4, j = 4 * (e & 15);
@@ -143,35 +140,35 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
   const int nk = (m + kKS - 1) / kKS;
   Regs r;
   load(0, r);
-  store(r, 0);
+  store(r, gs & 1);
   if (nk > 1) load(1, r);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
   const uint32_t id = idesc(2, kTM, kTN, 0, 0);
   for (int c = 0; c < nk; ++c) {
-    const int buf = c & 1;
+    const int g = gs + c, buf = g & 1;
     if (t == 0) {
       tc_fence_after();
       const uint32_t sb = sbase + buf * kStage;
 #pragma unroll
-      for (int g = 0; g < 3; ++g) {
-        const uint32_t ab = sb + ((g == 2) ? kOffAlo : kOffAhi);
-        const uint32_t bb = sb + ((g == 1) ? kOffBlo : kOffBhi);
+      for (int pr = 0; pr < 3; ++pr) {
+        const uint32_t ab = sb + ((pr == 2) ? kOffAlo : kOffAhi);
+        const uint32_t bb = sb + ((pr == 1) ? kOffBlo : kOffBhi);
 #pragma unroll
         for (int ks = 0; ks < kKS / 8; ++ks) {
           const uint64_t ad = desc_sw128(ab + (ks >> 2) * kAH, 16, 1024) + (uint64_t)((ks & 3) * 2);
           const uint64_t bd = desc_sw128(bb + (ks >> 2) * kBH, 16, 1024) + (uint64_t)((ks & 3) * 2);
-          mma_tf32(tmem, ad, bd, id, (c > 0 || g > 0 || ks > 0) ? 1u : 0u);
+          mma_tf32(tmem, ad, bd, id, (c > 0 || pr > 0 || ks > 0) ? 1u : 0u);
         }
       }
       mma_commit(bars + buf);
     }
     if (c + 1 < nk) {
-      // buffer buf ^ 1 was read by the products of step c - 1 (the ((c - 1) >> 1)-th commit on it)
-      if (c >= 1) mbar_wait(bars + (buf ^ 1), ((c - 1) >> 1) & 1, &status_dummy, 1);
+      // buffer buf ^ 1 was read by the products of global step g - 1 (its ((g - 1) >> 1)-th commit);
+      // at c = 0 that step belongs to an earlier tile, whose last wait covered it
+      if (c >= 1) mbar_wait(bars + (buf ^ 1), ((g - 1) >> 1) & 1, status, kStatusTimeout);
       store(r, buf ^ 1);
       if (c + 2 < nk) load(c + 2, r);
       fence_async_smem();
@@ -179,48 +176,190 @@ __global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs) {
       __syncthreads();
     }
   }
-  // the last commit covers every product issued before it
-  mbar_wait(bars + ((nk - 1) & 1), ((nk - 1) >> 1) & 1, &status_dummy, 1);
+  // the last commit covers every product issued before it (and completes the earlier commits that
+  // were not waited: the step before it on the other buffer)
+  {
+    const int g = gs + nk - 1;
+    mbar_wait(bars + (g & 1), (g >> 1) & 1, status, kStatusTimeout);
+    if (nk >= 2) mbar_wait(bars + ((g - 1) & 1), ((g - 1) >> 1) & 1, status, kStatusTimeout);
+  }
+  gs += nk;
   tc_fence_after();
-  // epilogue: warp w reads TMEM lanes 32 (w % 4) .., columns 32 (w / 4) ..
+  // epilogue: warp w reads TMEM lanes 32 (w % 4) .., columns 16 (w / 4) .. into a [128][65] fp32
+  // staging tile over stage 0 (every product is complete), then the rows go out coalesced
+  float* stg = reinterpret_cast<float*>(sm);
   {
     const int q = w & 3, h = w >> 2;
-    float v[32];
-    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32 * h, v);
-    const int i = i0 + 32 * q + lane;
-    if (i < m) {
+    float v[16];
+    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + 16 * h, v);
+    const int il = 32 * q + lane;
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int j = j0 + 32 * h + x;
-        if (j < m) {
-          float o = J.scale * v[x] + (i == j ? J.add_diag : 0.f);
-          if (Cin) o = fmaf(J.beta, Cin[(size_t)i * m + j], o);
-          Out[(size_t)i * m + j] = o;
-        }
-      }
+    for (int x = 0; x < 16; ++x) stg[il * 65 + 16 * h + x] = v[x];
+  }
+  __syncthreads();
+  for (int e = t; e < kTM * kTN; e += kGT) {
+    const int il = e >> 6, jl = e & 63, i = i0 + il, j = j0 + jl;
+    if (i < m && j < m) {
+      float o = J.scale * stg[il * 65 + jl] + (i == j ? J.add_diag : 0.f);
+      if (Cin) o = fmaf(J.beta, __ldcg(Cin + (size_t)i * m + j), o);
+      Out[(size_t)i * m + j] = o;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (w == 0) {
+}
+
+// job J (transposes read at run time) by its compile-time variant
+__device__ __forceinline__ void mm_tile_any(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm,
+                                            uint32_t sbase, uint32_t tmem, uint64_t* bars, int* status, int& gs) {
+  if (J.ta) {
+    if (J.tb) mm_tile<1, 1>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+    else mm_tile<1, 0>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+  } else {
+    if (J.tb) mm_tile<0, 1>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+    else mm_tile<0, 0>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+  }
+}
+
+__device__ __forceinline__ uint32_t gemm_setup(unsigned char* sm) {
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kStage);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + 2 * kStage + 32);
+  const int t = threadIdx.x;
+  if ((t >> 5) == 0) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  if (t == 0) {
+    mbar_init(bars + 0, 1);
+    mbar_init(bars + 1, 1);
+    mbar_init_fence();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  return *tmem_slot;
+}
+
+__device__ __forceinline__ void gemm_teardown(uint32_t tmem) {
+  tc_fence_before();
+  __syncthreads();
+  if ((threadIdx.x >> 5) == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 64);
   }
 }
 
+__global__ void __launch_bounds__(kGT) k_mm_tc(int m, int U, MmJobs jobs, int* status) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sm = smem_raw + pad;
+  const uint32_t tmem = gemm_setup(sm);
+  const int jz = blockIdx.z / U, u = blockIdx.z % U;
+  int gs = 0;
+  mm_tile_any(jobs.job[jz], m, u, blockIdx.y * kTM, blockIdx.x * kTN, sm, smem_u32(sm),
+              tmem, reinterpret_cast<uint64_t*>(sm + 2 * kStage), status, gs);
+  gemm_teardown(tmem);
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Newton-Schulz chain of unit blockIdx.y: for k < steps, Y = 2I - W X_k, X_{k+1} = X_k Y. Cluster
+// (gridDim.x blocks, one per 128 x 64 output tile) per unit; the cluster barrier after each product
+// publishes its tiles (release / acquire at cluster scope) before any block reads them. X_k is at
+// xa + (k & 1 ? xb - xa : 0) (ping-pong, seq = 0) or xa + k step (seq = 1).
+__global__ void __launch_bounds__(kGT) k_ns_chain(const NsChain c) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sm = smem_raw + pad;
+  const uint32_t tmem = gemm_setup(sm);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kStage);
+  const int m = c.m, u = blockIdx.y, nj = (m + kTN - 1) / kTN;
+  const int i0 = (blockIdx.x / nj) * kTM, j0 = (blockIdx.x % nj) * kTN;
+  int gs = 0;
+  for (int k = 0; k < c.steps; ++k) {
+    float* xk = c.seq ? c.xa + (size_t)k * c.step : ((k & 1) ? c.xb : c.xa);
+    float* xn = c.seq ? c.xa + (size_t)(k + 1) * c.step : ((k & 1) ? c.xa : c.xb);
+    const MmJob y{c.W, c.w_stride, xk, c.x_stride, nullptr, 0, c.Y, c.y_stride, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X_k
+    mm_tile<0, 0>(y, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    cluster_sync_all();
+    const MmJob x{xk, c.x_stride, c.Y, c.y_stride, nullptr, 0, xn, c.x_stride, 1.f, 0.f, 0.f, 0, 0};      // X_{k+1} = X_k Y
+    mm_tile<0, 0>(x, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    cluster_sync_all();
+  }
+  gemm_teardown(tmem);
+}
+
 }  // namespace
 
 cudaError_t gemm_set_attributes() {
-  return cudaFuncSetAttribute(k_mm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_mm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_ns_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem);
+  return e;
 }
 
-cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st) {
+namespace {
+
+// launch configuration of the chain for m: G blocks per unit, one cluster of G per unit
+int chain_blocks(int m) { return ((m + kTM - 1) / kTM) * ((m + kTN - 1) / kTN); }
+
+void chain_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int G, int U, cudaStream_t st) {
+  cfg = {};
+  cfg.gridDim = dim3(G, U, 1);
+  cfg.blockDim = dim3(kGT, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = G;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+}
+
+}  // namespace
+
+// A cluster of the unit's G tiles (G <= 8, the portable cluster size: m <= 256) must fit on the device
+// (one block per SM at this shared-memory size). Cached per (device, m).
+bool ns_chain_fits(int m) {
+  const int G = chain_blocks(m);
+  if (m < 1 || m > kMaxM || G < 1 || G > 8) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+  static std::mutex mu;
+  static signed char fits[64][kMaxM + 1];   // 0 unknown, 1 yes, -1 no
+  std::lock_guard<std::mutex> lk(mu);
+  if (fits[dev][m] == 0) {
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    chain_config(cfg, attr, G, 1, 0);
+    int n = 0;
+    const bool ok = cudaOccupancyMaxActiveClusters(&n, k_ns_chain, &cfg) == cudaSuccess && n >= 1;
+    if (!ok) cudaGetLastError();
+    fits[dev][m] = ok ? 1 : -1;
+  }
+  return fits[dev][m] > 0;
+}
+
+// One launch for the whole chain when the unit's cluster fits; otherwise (returns false, nothing
+// launched) the caller runs the products one launch each.
+bool launch_ns_chain(const NsChain& c, int U, cudaStream_t st) {
+  if (c.steps <= 0) return true;
+  if (!ns_chain_fits(c.m)) return false;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  chain_config(cfg, attr, chain_blocks(c.m), U, st);
+  return cudaLaunchKernelEx(&cfg, k_ns_chain, c) == cudaSuccess;
+}
+
+cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st, int* status) {
   if (njobs < 1 || njobs > 3) return cudaErrorInvalidValue;
   MmJobs js{};
   for (int i = 0; i < njobs; ++i) js.job[i] = jobs[i];
   js.n = njobs;
   const dim3 g(ceil_div(m, kTN), ceil_div(m, kTM), U * njobs);
-  k_mm_tc<<<g, kGT, kGemmSmem, st>>>(m, U, js);
+  k_mm_tc<<<g, kGT, kGemmSmem, st>>>(m, U, js, status);
   return cudaGetLastError();
 }
 

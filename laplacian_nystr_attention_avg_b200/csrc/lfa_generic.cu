@@ -78,30 +78,28 @@ __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
 // Small-m landmark kernel + alpha + Newton-Schulz, one CTA per unit, all in shared memory.
 // ---------------------------------------------------------------------------------------
 // Sum of v over the block (every thread gets the total; all threads must call it).
-__device__ float block_sum(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x / 32, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) red[w] = v;
-  __syncthreads();
-  float s = 0.f;
-  for (int i = 0; i < (int)(blockDim.x / 32); ++i) s += red[i];
-  return s;
-}
-
 // ---------------------------------------------------------------------------------------
 // Large-m Newton-Schulz (64 < m <= 256): W and X in global memory, one launch per product.
 // ---------------------------------------------------------------------------------------
+// W = exp(-||l_a - l_b||_1 / lambda) + eps I: the unit's landmarks staged in shared memory (row stride
+// d + 1, conflict-free), rows a of this CTA's group of 16, thread = column b (m <= kThreads); the
+// distance is summed over k in order, so W is exactly symmetric.
 __global__ void __launch_bounds__(kThreads) k_gram(Params p) {
-  const int u = blockIdx.y, m = p.m, d = p.d;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= m * m) return;
-  const int a = e / m, b = e % m;
-  const float* La = p.L + ((size_t)u * m + a) * d;
-  const float* Lb = p.L + ((size_t)u * m + b) * d;
-  float acc = 0.f;
-  for (int k = 0; k < d; ++k) acc += fabsf(La[k] - Lb[k]);
-  p.Wm[(size_t)u * m * m + e] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
+  extern __shared__ float4 smem_f4[];
+  float* Ls = reinterpret_cast<float*>(smem_f4);   // [m][d + 1]
+  const int u = blockIdx.y, m = p.m, d = p.d, ds = d + 1, t = threadIdx.x;
+  const float* Lg = p.L + (size_t)u * m * d;
+  for (int e = t; e < m * d; e += blockDim.x) Ls[(e / d) * ds + e % d] = Lg[e];
+  __syncthreads();
+  const int b = t;
+  if (b >= m) return;
+  for (int r = 0; r < 16; ++r) {
+    const int a = blockIdx.x * 16 + r;
+    if (a >= m) break;
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc += fabsf(Ls[a * ds + k] - Ls[b * ds + k]);
+    p.Wm[((size_t)u * m + a) * m + b] = exp2f(acc * p.neg_log2e_over_lam) + (a == b ? p.eps : 0.f);
+  }
 }
 
 // Power iteration for ||W||_2 with 1024 threads; the first alpha_rows(m) rows of W are staged in
@@ -113,7 +111,7 @@ __host__ __device__ inline int alpha_rows(int m) {
 }
 
 __global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
-  __shared__ float v[kMaxM], w[kMaxM], red[32];
+  __shared__ float v[2][kMaxM], w[kMaxM];
   extern __shared__ float4 smem_f4[];
   float* Ws = reinterpret_cast<float*>(smem_f4);   // [alpha_rows(m)][m]
   const int u = blockIdx.x, m = p.m, t = threadIdx.x;
@@ -121,27 +119,37 @@ __global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
   const int warp = t / 32, lane = t & 31, nw = blockDim.x / 32;
   const int rs = alpha_rows(m);
   for (int e = t; e < rs * m; e += blockDim.x) Ws[e] = Wg[e];
-  if (t < m) v[t] = rsqrtf(float(m));
+  if (t < m) v[0][t] = rsqrtf(float(m));
   __syncthreads();
   float rq = 0.f;
   const int iters = 24;
+  int cur = 0;
   for (int it = 0; it <= iters; ++it) {
     // w = W v, one warp per row (coalesced along the row)
     for (int i = warp; i < m; i += nw) {
       const float* row = i < rs ? Ws + (size_t)i * m : Wg + (size_t)i * m;
       float acc = 0.f;
-      for (int j = lane; j < m; j += 32) acc = fmaf(row[j], v[j], acc);
+      for (int j = lane; j < m; j += 32) acc = fmaf(row[j], v[cur][j], acc);
       for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if (lane == 0) w[i] = acc;
     }
     __syncthreads();
-    const float vw = block_sum(t < m ? w[t] * v[t] : 0.f, red);
-    const float nn = block_sum(t < m ? w[t] * w[t] : 0.f, red);
+    // v^T w and ||w||^2, formed by every warp in the same order (so every warp holds the same values):
+    // no further block-wide reduction; the next v goes to the other buffer
+    float vw = 0.f, nn = 0.f;
+    for (int j = lane; j < m; j += 32) {
+      vw = fmaf(w[j], v[cur][j], vw);
+      nn = fmaf(w[j], w[j], nn);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      vw += __shfl_xor_sync(0xffffffffu, vw, o);
+      nn += __shfl_xor_sync(0xffffffffu, nn, o);
+    }
     rq = vw;
     if (it == iters) break;
     const float inv = rsqrtf(nn);
-    __syncthreads();
-    if (t < m) v[t] = w[t] * inv;
+    if (t < m) v[cur ^ 1][t] = w[t] * inv;
+    cur ^= 1;
     __syncthreads();
   }
   const float lmax = rq;
@@ -877,9 +885,9 @@ void reading_b_t(const Params& p, cudaStream_t st) {
   k_combine_reduce<<<dim3(ceil_div(p.part_stride, kThreads), U), kThreads, 0, st>>>(p);
   k_rb_cov<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
   const MmJob sx{p.Y, mm, p.X, mm, nullptr, 0, p.Xb, mm, 1.f, 0.f, 0.f, 0, 0};   // Xb = S X
-  launch_mm(&sx, 1, m, U, st);
+  launch_mm(&sx, 1, m, U, st, p.status);
   const MmJob k{p.X, mm, p.Xb, mm, nullptr, 0, p.Y, mm, 1.f, 0.f, 0.f, 1, 0};     // Y = X^T (S X)
-  launch_mm(&k, 1, m, U, st);
+  launch_mm(&k, 1, m, U, st, p.status);
   k_rb_pass<T><<<dim3(p.P, U), kThreads, rb_pass_smem(m, d), st>>>(p);
   k_rb_reduce<<<dim3(ceil_div(m * d, kThreads), U), kThreads, 0, st>>>(p);
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
@@ -894,11 +902,14 @@ void ns_from_w(const Params& p, cudaStream_t st) {
   float* x = p.X;
   float* xb = p.Xb;
   const size_t mm = (size_t)m * m;
-  for (int k = 0; k < p.T; ++k) {
+  const NsChain c{p.Wm, mm, p.Y, mm, p.X, p.Xb, mm, 0, m, p.T, 0, p.status};
+  if (launch_ns_chain(c, U, st)) {
+    if (p.T & 1) { x = p.Xb; xb = p.X; }
+  } else for (int k = 0; k < p.T; ++k) {
     const MmJob y{p.Wm, mm, x, mm, nullptr, 0, p.Y, mm, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X
-    launch_mm(&y, 1, m, U, st);
+    launch_mm(&y, 1, m, U, st, p.status);
     const MmJob xn{x, mm, p.Y, mm, nullptr, 0, xb, mm, 1.f, 0.f, 0.f, 0, 0};     // X' = X Y
-    launch_mm(&xn, 1, m, U, st);
+    launch_mm(&xn, 1, m, U, st, p.status);
     float* tmp = x; x = xb; xb = tmp;
   }
   if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
@@ -912,7 +923,7 @@ void ns_t(const Params& p, cudaStream_t st) {
   if (m <= kSmallM) {
     launch_ns_tc(p, st);
   } else {
-    k_gram<<<dim3(ceil_div(m * m, kThreads), U), kThreads, 0, st>>>(p);
+    k_gram<<<dim3(ceil_div(m, 16), U), kThreads, sizeof(float) * (size_t)m * (p.d + 1), st>>>(p);
     ns_from_w(p, st);
   }
 }
@@ -971,6 +982,7 @@ cudaError_t generic_set_attributes() {
   LFA_ATTR((k_pass1<__nv_bfloat16, 2>));
   LFA_ATTR((k_pass1<__nv_bfloat16, 4>));
   LFA_ATTR(k_combine_finish);
+  LFA_ATTR(k_gram);
   LFA_ATTR(k_rb_finish);
   LFA_ATTR(k_rb_gram<float>);
   LFA_ATTR(k_rb_gram<__nv_bfloat16>);
@@ -990,8 +1002,9 @@ cudaError_t generic_set_attributes() {
 
 int generic_launch_count(const Params& p) {
   // pool, Newton-Schulz chain, pass 1, two combine kernels (three with batch-pooled statistics),
-  // pass 2
-  const int ns = p.m <= kSmallM ? 1 : 2 + 2 * p.T + 2;
+  // pass 2; the chain for m > 64 is gram, alpha, the steps (one cluster launch, or two per step),
+  // the residual product and its square root
+  const int ns = p.m <= kSmallM ? 1 : 2 + (p.T > 0 ? (ns_chain_fits(p.m) ? 1 : 2 * p.T) : 0) + 2;
   // Reading B: pass 1, C^T C, reduction, covariance, two products, token pass, reduction, finish
   if (p.whiten == 3) return 1 + ns + 9 + 1;
   return 1 + ns + 1 + 2 + (p.whiten == 2 ? 1 : 0) + 1;

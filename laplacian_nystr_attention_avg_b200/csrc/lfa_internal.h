@@ -143,9 +143,31 @@ struct MmJobs {
   int n;
 };
 
+// A Newton-Schulz chain for k < steps: Y = 2I - W X_k, X_{k+1} = X_k Y, per unit (strides in floats
+// between units' matrices). X_k: seq = 0 ping-pongs between xa (k even) and xb (k odd); seq = 1 reads
+// X_k at xa + k step and writes X_{k+1} at xa + (k + 1) step. status: the device status word (timeout
+// bit of the bounded waits).
+struct NsChain {
+  const float* W;
+  size_t w_stride;
+  float* Y;
+  size_t y_stride;
+  float* xa;
+  float* xb;
+  size_t x_stride;
+  size_t step;
+  int m, steps, seq;
+  int* status;
+};
+
 // host helpers implemented in lfa_generic.cu / lfa_fused.cu / lfa_backward.cu / lfa_gemm.cu
-// Up to three independent jobs (none reads another's output) in one launch.
-cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st);
+// Up to three independent jobs (none reads another's output) in one launch; status as above.
+cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t st, int* status);
+// the whole chain in one launch (a thread-block cluster per unit); false: not launched (no cluster of
+// the needed size fits), the caller runs the products with launch_mm
+bool launch_ns_chain(const NsChain& c, int U, cudaStream_t st);
+// whether launch_ns_chain runs for this m on the current device
+bool ns_chain_fits(int m);
 cudaError_t gemm_set_attributes();
 cudaError_t ns_tc_set_attributes();
 cudaError_t launch_ns_tc(const Params& p, cudaStream_t st);
