@@ -47,6 +47,9 @@ struct Regs {
   float4 b[kBR];
 };
 
+__device__ __forceinline__ void tile_epilogue(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm,
+                                              uint32_t tmem);
+
 // One 128 x 64 output tile (rows i0.., columns j0..) of job J for unit u. The two shared-memory stages
 // and their commit barriers continue across calls: step c of this tile is global step gs + c, staged in
 // buffer (gs + c) & 1 and committed on that buffer's barrier as its ((gs + c) >> 1)-th completion; gs
@@ -59,9 +62,7 @@ __device__ __noinline__ void mm_tile(const MmJob& J, int m, int u, int i0, int j
                         uint64_t* bars, int* status, int& gs) {
   const float* A = J.A + u * J.a_stride;
   const float* B = J.B + u * J.b_stride;
-  const float* Cin = J.C ? J.C + u * J.c_stride : nullptr;
-  float* Out = J.O + u * J.o_stride;
-  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int t = threadIdx.x;
   const bool vec = (m & 3) == 0;   // rows start on 16-byte boundaries
   // Group e of a step covers 4 consecutive elements along the stored matrix's contiguous index:
   //   A untransposed: row i = e / 16, k = 4 (e % 16) .. ;  transposed: row k = e / 32, i = 4 (e % 32) ..
@@ -185,8 +186,18 @@ __device__ __noinline__ void mm_tile(const MmJob& J, int m, int u, int i0, int j
   }
   gs += nk;
   tc_fence_after();
-  // epilogue: warp w reads TMEM lanes 32 (w % 4) .., columns 16 (w / 4) .. into a [128][65] fp32
-  // staging tile over stage 0 (every product is complete), then the rows go out coalesced
+  tile_epilogue(J, m, u, i0, j0, sm, tmem);
+}
+
+// Epilogue of a tile whose products are complete: warp w reads TMEM lanes 32 (w % 4) .., columns
+// 16 (w / 4) .. into a [128][65] fp32 staging tile at sm (free), then the rows go out coalesced as
+// Out = scale * acc + beta * Cin + add_diag * I.
+__device__ __forceinline__ void tile_epilogue(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm,
+                                              uint32_t tmem) {
+  const float* Cin = J.C ? J.C + u * J.c_stride : nullptr;
+  float* Out = J.O + u * J.o_stride;
+  const float scale = J.scale, beta = J.beta, add_diag = J.add_diag;
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   float* stg = reinterpret_cast<float*>(sm);
   {
     const int q = w & 3, h = w >> 2;
@@ -197,21 +208,206 @@ __device__ __noinline__ void mm_tile(const MmJob& J, int m, int u, int i0, int j
     for (int x = 0; x < 16; ++x) stg[il * 65 + 16 * h + x] = v[x];
   }
   __syncthreads();
-  for (int e = t; e < kTM * kTN; e += kGT) {
-    const int il = e >> 6, jl = e & 63, i = i0 + il, j = j0 + jl;
-    if (i < m && j < m) {
-      float o = J.scale * stg[il * 65 + jl] + (i == j ? J.add_diag : 0.f);
-      if (Cin) o = fmaf(J.beta, __ldcg(Cin + (size_t)i * m + j), o);
-      Out[(size_t)i * m + j] = o;
+  if ((m & 3) == 0) {
+    // four columns per store (rows start on 16-byte boundaries; j < m covers j + 3 < m)
+    for (int e = t; e < kTM * kTN / 4; e += kGT) {
+      const int il = e >> 4, jl = 4 * (e & 15), i = i0 + il, j = j0 + jl;
+      if (i < m && j < m) {
+        const float* sr = stg + il * 65 + jl;
+        float4 o = make_float4(scale * sr[0] + (i == j ? add_diag : 0.f), scale * sr[1] + (i == j + 1 ? add_diag : 0.f),
+                               scale * sr[2] + (i == j + 2 ? add_diag : 0.f), scale * sr[3] + (i == j + 3 ? add_diag : 0.f));
+        if (Cin) {
+          const float4 c = __ldcg(reinterpret_cast<const float4*>(Cin + (size_t)i * m + j));
+          o.x = fmaf(beta, c.x, o.x);
+          o.y = fmaf(beta, c.y, o.y);
+          o.z = fmaf(beta, c.z, o.z);
+          o.w = fmaf(beta, c.w, o.w);
+        }
+        *reinterpret_cast<float4*>(Out + (size_t)i * m + j) = o;
+      }
+    }
+  } else {
+    for (int e = t; e < kTM * kTN; e += kGT) {
+      const int il = e >> 6, jl = e & 63, i = i0 + il, j = j0 + jl;
+      if (i < m && j < m) {
+        float o = scale * stg[il * 65 + jl] + (i == j ? add_diag : 0.f);
+        if (Cin) o = fmaf(beta, __ldcg(Cin + (size_t)i * m + j), o);
+        Out[(size_t)i * m + j] = o;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
 }
 
-// job J (transposes read at run time) by its compile-time variant
+// ---- asynchronous-copy variant (m % 4 == 0: every matrix row starts on a 16-byte boundary) -------
+// K advances in steps of 32. The raw fp32 operand tiles of a step land by cp.async (16-byte chunks
+// through L2, zero-filled past m) in one of three ring slots, already in the layout the tensor cores
+// read, so no transpose is needed:
+//   A untransposed (rows i, k contiguous): K-major, one SW128 K-half of 128 rows;
+//   A transposed (stored [k][i]): MN-major, four 4 KB blocks of 32 i, one 128-byte line per k;
+//   B untransposed (stored [k][j]): MN-major, two 4 KB blocks of 32 j, one line per k;
+//   B transposed (rows j, k contiguous): K-major, one SW128 K-half of 64 rows.
+// MN-major 32-bit operands use the 128-byte swizzle with 32-byte granules (descriptor layout type
+// 1): the granule g < 4 of line k sits at position g ^ (k % 4); LBO = 4096 (next 32-element block
+// along M / N), SBO = 512 (next group of 4 lines along K); one K = 8 product step is 8 lines, 1024
+// bytes. A step is split in place (hi = tf32(x) over x, lo = x - hi beside it); its products then
+// run while the next step is split, and the copies of step c + 2 go out once the products of step
+// c - 1 have released their slot.
+constexpr int kKS2 = 32;
+constexpr uint32_t kQA = 16384, kQB = 8192;                                  // hi (raw) tiles
+constexpr uint32_t kSlotHiA = 0, kSlotHiB = kQA, kSlotLoA = kQA + kQB, kSlotLoB = 2 * kQA + kQB;
+constexpr uint32_t kSlot = 2 * (kQA + kQB);                                  // 48 KB
+static_assert(3 * kSlot <= 2 * kStage, "ring slots beyond the tile's shared memory");
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const float* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// byte offset of (line, 16-byte chunk c < 8) in an MN-major block of 128-byte lines (32-byte granules
+// swizzled by line % 4)
+__device__ __forceinline__ uint32_t mnofs(int line, int c) {
+  return (uint32_t)(line * 128 + ((((c >> 1) ^ (line & 3)) << 5) | ((c & 1) << 4)));
+}
+
+// descriptor of an MN-major 32-bit operand in that layout, blocks of 32 elements 4096 bytes apart
+__device__ __forceinline__ uint64_t desc_mn32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((4096u >> 4) & 0x3FFF) << 16;       // LBO
+  d |= (uint64_t)((512u >> 4) & 0x3FFF) << 32;        // SBO
+  d |= (uint64_t)1 << 46;                             // descriptor version (sm_100)
+  d |= (uint64_t)1 << 61;                             // 128-byte swizzle, 32-byte atomicity
+  return d;
+}
+
+// Ring slot and barrier of global step g: slot g % 3, committed on bars[g % 3] as that barrier's
+// (g / 3)-th completion; every commit is waited once, in order. Warps 0-14 copy and split; lane 0 of
+// warp 15 issues the products, so a step's split overlaps the products of the step before. Step c's
+// hand-over from the splitters to the issuer is named barrier 2 + (c & 1) (the splitters arrive, the
+// issuer warp waits): before the splitters arrive at step c + 2 they have waited (at step c + 1) for
+// the products of step c, which the issuer issues only after its wait at step c, so an instance of a
+// barrier never collects arrivals of two steps.
+constexpr int kSplitters = kGT - 32;
+template <int TA, int TB>
+__device__ __noinline__ void mm_tile_async(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm,
+                                           uint32_t sbase, uint32_t tmem, uint64_t* bars, int* status, int& gs) {
+  const float* A = J.A + u * J.a_stride;
+  const float* B = J.B + u * J.b_stride;
+  const int t = threadIdx.x;
+  const bool issuer = t >= kSplitters;
+  const int nk = (m + kKS2 - 1) / kKS2;
+  auto issue = [&](int c) {
+    const int k0 = c * kKS2;
+    const uint32_t sa = sbase + ((gs + c) % 3) * kSlot + kSlotHiA, sb = sbase + ((gs + c) % 3) * kSlot + kSlotHiB;
+    for (int e = t; e < 1024; e += kSplitters) {   // A
+      if constexpr (!TA) {
+        const int row = e >> 3, kc = e & 7, i = i0 + row, k = k0 + 4 * kc;
+        const bool ok = i < m && k < m;
+        cp_async16(sa + sw128(row, kc), ok ? A + (size_t)i * m + k : A, ok);
+      } else {
+        const int kl = e >> 5, ic = e & 31, k = k0 + kl, i = i0 + 4 * ic;
+        const bool ok = k < m && i < m;
+        cp_async16(sa + (ic >> 3) * 4096 + mnofs(kl, ic & 7), ok ? A + (size_t)k * m + i : A, ok);
+      }
+    }
+    for (int e = t; e < 512; e += kSplitters) {    // B
+      if constexpr (!TB) {
+        const int kl = e >> 4, jc = e & 15, k = k0 + kl, j = j0 + 4 * jc;
+        const bool ok = k < m && j < m;
+        cp_async16(sb + (jc >> 3) * 4096 + mnofs(kl, jc & 7), ok ? B + (size_t)k * m + j : B, ok);
+      } else {
+        const int jl = e >> 3, kc = e & 7, j = j0 + jl, k = k0 + 4 * kc;
+        const bool ok = j < m && k < m;
+        cp_async16(sb + sw128(jl, kc), ok ? B + (size_t)j * m + k : B, ok);
+      }
+    }
+    cp_async_commit();
+  };
+  auto split4 = [&](uint32_t off_hi, uint32_t off_lo) {
+    float4* ph = reinterpret_cast<float4*>(sm + off_hi);
+    const float4 v = *ph;
+    float4 h, l;
+    h.x = tf32_round(v.x); l.x = v.x - h.x;
+    h.y = tf32_round(v.y); l.y = v.y - h.y;
+    h.z = tf32_round(v.z); l.z = v.z - h.z;
+    h.w = tf32_round(v.w); l.w = v.w - h.w;
+    *ph = h;
+    *reinterpret_cast<float4*>(sm + off_lo) = l;
+  };
+  if (!issuer) {
+    issue(0);
+    if (nk > 1) issue(1);
+    for (int c = 0; c < nk; ++c) {
+      const int g = gs + c;
+      const uint32_t slot = (g % 3) * kSlot;
+      // this thread's copies of step c are in (those of step c + 1 may still be in flight)
+      if (c + 1 < nk) cp_async_wait<1>();
+      else cp_async_wait<0>();
+      named_bar_sync(1, kSplitters);
+      for (int e = t; e < 1536; e += kSplitters) {
+        const uint32_t o = 16u * (e < 1024 ? e : e - 1024);
+        if (e < 1024) split4(slot + kSlotHiA + o, slot + kSlotLoA + o);
+        else split4(slot + kSlotHiB + o, slot + kSlotLoB + o);
+      }
+      fence_async_smem();
+      named_bar_arrive(2 + (c & 1), kGT);
+      // the products of step c - 1 are complete: their slot takes the copies of step c + 2
+      if (c >= 1) mbar_wait(bars + (g - 1) % 3, ((g - 1) / 3) & 1, status, kStatusTimeout);
+      if (c + 2 < nk) issue(c + 2);
+    }
+  } else {
+    const uint32_t id = idesc(2, kTM, kTN, TA, TB ? 0 : 1);
+    for (int c = 0; c < nk; ++c) {
+      const int g = gs + c;
+      named_bar_sync(2 + (c & 1), kGT);
+      if (t == kSplitters) {
+        tc_fence_after();
+        const uint32_t sl = sbase + (g % 3) * kSlot;
+#pragma unroll
+        for (int pr = 0; pr < 3; ++pr) {
+          const uint32_t ab = sl + ((pr == 2) ? kSlotLoA : kSlotHiA);
+          const uint32_t bb = sl + ((pr == 1) ? kSlotLoB : kSlotHiB);
+#pragma unroll
+          for (int ks = 0; ks < kKS2 / 8; ++ks) {
+            const uint64_t ad = TA ? desc_mn32(ab + ks * 1024) : desc_sw128(ab, 16, 1024) + (uint64_t)(ks * 2);
+            const uint64_t bd = TB ? desc_sw128(bb, 16, 1024) + (uint64_t)(ks * 2) : desc_mn32(bb + ks * 1024);
+            mma_tf32(tmem, ad, bd, id, (c > 0 || pr > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bars + g % 3);
+      }
+      __syncwarp();
+    }
+  }
+  {
+    const int g = gs + nk - 1;
+    mbar_wait(bars + g % 3, (g / 3) & 1, status, kStatusTimeout);
+  }
+  gs += nk;
+  tc_fence_after();
+  __syncthreads();
+  tile_epilogue(J, m, u, i0, j0, sm, tmem);
+}
+
+// job J (transposes read at run time) by its compile-time variant; the asynchronous-copy tile when
+// every row is 16-byte aligned
 __device__ __forceinline__ void mm_tile_any(const MmJob& J, int m, int u, int i0, int j0, unsigned char* sm,
                                             uint32_t sbase, uint32_t tmem, uint64_t* bars, int* status, int& gs) {
+  if ((m & 3) == 0) {
+    if (J.ta) {
+      if (J.tb) mm_tile_async<1, 1>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+      else mm_tile_async<1, 0>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+    } else {
+      if (J.tb) mm_tile_async<0, 1>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+      else mm_tile_async<0, 0>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
+    }
+    return;
+  }
   if (J.ta) {
     if (J.tb) mm_tile<1, 1>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
     else mm_tile<1, 0>(J, m, u, i0, j0, sm, sbase, tmem, bars, status, gs);
@@ -232,6 +428,7 @@ __device__ __forceinline__ uint32_t gemm_setup(unsigned char* sm) {
   if (t == 0) {
     mbar_init(bars + 0, 1);
     mbar_init(bars + 1, 1);
+    mbar_init(bars + 2, 1);
     mbar_init_fence();
   }
   tc_fence_before();
@@ -277,15 +474,18 @@ __global__ void __launch_bounds__(kGT) k_ns_chain(const NsChain c) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 2 * kStage);
   const int m = c.m, u = blockIdx.y, nj = (m + kTN - 1) / kTN;
   const int i0 = (blockIdx.x / nj) * kTM, j0 = (blockIdx.x % nj) * kTN;
+  const bool vec = (m & 3) == 0;
   int gs = 0;
   for (int k = 0; k < c.steps; ++k) {
     float* xk = c.seq ? c.xa + (size_t)k * c.step : ((k & 1) ? c.xb : c.xa);
     float* xn = c.seq ? c.xa + (size_t)(k + 1) * c.step : ((k & 1) ? c.xa : c.xb);
     const MmJob y{c.W, c.w_stride, xk, c.x_stride, nullptr, 0, c.Y, c.y_stride, -1.f, 0.f, 2.f, 0, 0};   // Y = 2I - W X_k
-    mm_tile<0, 0>(y, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    if (vec) mm_tile_async<0, 0>(y, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    else mm_tile<0, 0>(y, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
     cluster_sync_all();
     const MmJob x{xk, c.x_stride, c.Y, c.y_stride, nullptr, 0, xn, c.x_stride, 1.f, 0.f, 0.f, 0, 0};      // X_{k+1} = X_k Y
-    mm_tile<0, 0>(x, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    if (vec) mm_tile_async<0, 0>(x, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
+    else mm_tile<0, 0>(x, m, u, i0, j0, sm, smem_u32(sm), tmem, bars, c.status, gs);
     cluster_sync_all();
   }
   gemm_teardown(tmem);
