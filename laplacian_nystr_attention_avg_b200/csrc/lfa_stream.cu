@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kST, 1) k_stream_pass2(const Params p, const S
           const int xx = gx + b - 1;
           if (xx < 0 || xx >= p.W) continue;
           const uint4* src = reinterpret_cast<const uint4*>(vrow + (size_t)xx * 64 + 16 * h);
-          const uint4 r0 = src[0], r1 = src[1];
+          const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
           const uint32_t rv[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
           const float* tp = taps + (a * 3 + b) * 64 + 16 * h;
 #pragma unroll
