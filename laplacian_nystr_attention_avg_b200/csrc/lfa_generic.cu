@@ -81,6 +81,24 @@ __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
 // ---------------------------------------------------------------------------------------
 // Large-m Newton-Schulz (64 < m <= 256): W and X in global memory, one launch per product.
 // ---------------------------------------------------------------------------------------
+// dst[i * ds + c] = src[i * d + c] for i * d + c < n (ds = d for a plain copy), with eight loads in flight
+// per thread
+__device__ __forceinline__ void stage_floats(float* dst, const float* src, int n, int d, int ds) {
+  const int nt = blockDim.x;
+  int e = threadIdx.x;
+  for (; e + 7 * nt < n; e += 8 * nt) {
+    float r[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) r[x] = __ldg(src + e + x * nt);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int f = e + x * nt;
+      dst[(f / d) * ds + f % d] = r[x];
+    }
+  }
+  for (; e < n; e += nt) dst[(e / d) * ds + e % d] = __ldg(src + e);
+}
+
 // W = exp(-||l_a - l_b||_1 / lambda) + eps I: the unit's landmarks staged in shared memory (row stride
 // d + 1, conflict-free), rows a of this CTA's group of 16, thread = column b (m <= kThreads); the
 // distance is summed over k in order, so W is exactly symmetric.
@@ -88,8 +106,7 @@ __global__ void __launch_bounds__(kThreads) k_gram(Params p) {
   extern __shared__ float4 smem_f4[];
   float* Ls = reinterpret_cast<float*>(smem_f4);   // [m][d + 1]
   const int u = blockIdx.y, m = p.m, d = p.d, ds = d + 1, t = threadIdx.x;
-  const float* Lg = p.L + (size_t)u * m * d;
-  for (int e = t; e < m * d; e += blockDim.x) Ls[(e / d) * ds + e % d] = Lg[e];
+  stage_floats(Ls, p.L + (size_t)u * m * d, m * d, d, ds);
   __syncthreads();
   const int b = t;
   if (b >= m) return;
@@ -102,64 +119,84 @@ __global__ void __launch_bounds__(kThreads) k_gram(Params p) {
   }
 }
 
-// Power iteration for ||W||_2 with 1024 threads; the first alpha_rows(m) rows of W are staged in
-// shared memory once (the rest are read from L2 at every step).
-constexpr int kAlphaThreads = 1024;
-__host__ __device__ inline int alpha_rows(int m) {
-  const int cap = (200 * 1024) / (4 * (m > 0 ? m : 1));
-  return m < cap ? m : cap;
+// Power iteration for ||W||_2: one CTA of kAlphaThreads per unit, thread t owns entry t of the iterate
+// (m <= kAlphaThreads). W is symmetric, so thread t forms (W v)_t as column t, sum_j W[j][t] v_j: the
+// threads of a warp read consecutive words of one row (conflict-free in shared memory, coalesced in L2).
+// The first alpha_rows(m) rows of W are staged in shared memory once, the rest (at most 56, for m = 256)
+// in registers, column t of each in thread t. Four partial sums per thread shorten the dependent chain.
+constexpr int kAlphaThreads = 256;
+__host__ __device__ constexpr int alpha_rows(int m) {
+  return m < (200 * 1024) / (4 * (m > 0 ? m : 1)) ? m : (200 * 1024) / (4 * (m > 0 ? m : 1));
+}
+constexpr int kAlphaRegRows = 56;
+static_assert(kMaxM - alpha_rows(kMaxM) <= kAlphaRegRows, "rows of W beyond shared memory and registers");
+static_assert(kMaxM <= kAlphaThreads, "one thread per entry of the power-iteration vector");
+
+__device__ __forceinline__ float block_sum256(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kAlphaThreads / 32; ++i) s += red[i];
+  return s;
 }
 
 __global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
-  __shared__ float v[2][kMaxM], w[kMaxM];
+  __shared__ float v[kMaxM], red[2][kAlphaThreads / 32];
   extern __shared__ float4 smem_f4[];
   float* Ws = reinterpret_cast<float*>(smem_f4);   // [alpha_rows(m)][m]
   const int u = blockIdx.x, m = p.m, t = threadIdx.x;
   const float* Wg = p.Wm + (size_t)u * m * m;
-  const int warp = t / 32, lane = t & 31, nw = blockDim.x / 32;
   const int rs = alpha_rows(m);
-  for (int e = t; e < rs * m; e += blockDim.x) Ws[e] = Wg[e];
-  if (t < m) v[0][t] = rsqrtf(float(m));
+  stage_floats(Ws, Wg, rs * m, m, m);
+  float wr[kAlphaRegRows];
+#pragma unroll
+  for (int q = 0; q < kAlphaRegRows; ++q) wr[q] = (t < m && rs + q < m) ? Wg[(size_t)(rs + q) * m + t] : 0.f;
+  if (t < m) v[t] = rsqrtf(float(m));
   __syncthreads();
   float rq = 0.f;
   const int iters = 24;
-  int cur = 0;
+  const int r4 = rs & ~3;
   for (int it = 0; it <= iters; ++it) {
-    // w = W v, one warp per row (coalesced along the row)
-    for (int i = warp; i < m; i += nw) {
-      const float* row = i < rs ? Ws + (size_t)i * m : Wg + (size_t)i * m;
-      float acc = 0.f;
-      for (int j = lane; j < m; j += 32) acc = fmaf(row[j], v[cur][j], acc);
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) w[i] = acc;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    if (t < m) {
+      for (int j = 0; j < r4; j += 4) {
+        a0 = fmaf(Ws[(size_t)j * m + t], v[j], a0);
+        a1 = fmaf(Ws[(size_t)(j + 1) * m + t], v[j + 1], a1);
+        a2 = fmaf(Ws[(size_t)(j + 2) * m + t], v[j + 2], a2);
+        a3 = fmaf(Ws[(size_t)(j + 3) * m + t], v[j + 3], a3);
+      }
+      for (int j = r4; j < rs; ++j) a0 = fmaf(Ws[(size_t)j * m + t], v[j], a0);
+      if (rs < m) {
+#pragma unroll
+        for (int q = 0; q < kAlphaRegRows; q += 4) {
+          if (rs + q < m) a1 = fmaf(wr[q], v[rs + q], a1);
+          if (rs + q + 1 < m) a2 = fmaf(wr[q + 1], v[rs + q + 1], a2);
+          if (rs + q + 2 < m) a3 = fmaf(wr[q + 2], v[rs + q + 2], a3);
+          if (rs + q + 3 < m) a0 = fmaf(wr[q + 3], v[rs + q + 3], a0);
+        }
+      }
     }
-    __syncthreads();
-    // v^T w and ||w||^2, formed by every warp in the same order (so every warp holds the same values):
-    // no further block-wide reduction; the next v goes to the other buffer
-    float vw = 0.f, nn = 0.f;
-    for (int j = lane; j < m; j += 32) {
-      vw = fmaf(w[j], v[cur][j], vw);
-      nn = fmaf(w[j], w[j], nn);
-    }
-    for (int o = 16; o > 0; o >>= 1) {
-      vw += __shfl_xor_sync(0xffffffffu, vw, o);
-      nn += __shfl_xor_sync(0xffffffffu, nn, o);
-    }
+    const float w = (a0 + a1) + (a2 + a3);
+    // v^T w and ||w||^2 (two reduction buffers: the second sum may start before every thread has
+    // read the first one's result, and v is rewritten only after both)
+    const float vw = block_sum256(t < m ? w * v[t] : 0.f, red[0]);
+    const float nn = block_sum256(t < m ? w * w : 0.f, red[1]);
     rq = vw;
     if (it == iters) break;
-    const float inv = rsqrtf(nn);
-    if (t < m) v[cur ^ 1][t] = w[t] * inv;
-    cur ^= 1;
+    if (t < m) v[t] = w * rsqrtf(nn);
     __syncthreads();
   }
   const float lmax = rq;
   const float alpha_p = 2.f / lmax;
   const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
   const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
+  // X_0 = alpha W^T, the transposed read from the staged rows where they are
   float* Xg = p.X + (size_t)u * m * m;
   for (int e = t; e < m * m; e += blockDim.x) {
     const int a = e / m, b = e % m;
-    Xg[e] = alpha * Wg[(size_t)b * m + a];
+    Xg[e] = alpha * (b < rs ? Ws[(size_t)b * m + a] : Wg[(size_t)b * m + a]);
   }
   if (t == 0) {
     float* inf = p.info + (size_t)u * kInfoStride;

@@ -45,7 +45,7 @@ constexpr int kOffMimg = kOffStage + 3 * kStageBytes;   // pass 2: M'^T, bf16, K
 constexpr int kOffL = kOffMimg + kCbBytes;       // landmarks, fp32 [m][64]
 constexpr int kOffSh = kOffL + kMaxM * 64 * 4;   // column shifts c, fp32 [m]
 constexpr int kOffAux = kOffSh + kMaxM * 4;      // pass 1: sum-V partials; pass 2: bias, DWC taps
-constexpr int kAuxFloats = 768;
+constexpr int kAuxFloats = 64 + 9 * 64 + 8 * 64;   // pass 2: bias, DWC taps, bias partials
 constexpr int kOffBar = kOffAux + kAuxFloats * 4;
 constexpr int kBarFull = 0, kBarMma = 3, kNumBars = 5;
 constexpr int kOffTmem = kOffBar + 64;
@@ -273,7 +273,16 @@ __device__ __forceinline__ uint32_t stream_setup(const Params& p, unsigned char*
   }
   for (int e = t; e < 2 * kCbBytes / 16; e += kST) reinterpret_cast<uint4*>(sm + kOffCb)[e] = make_uint4(0u, 0u, 0u, 0u);
   const float4* Lg = reinterpret_cast<const float4*>(p.L + (size_t)u * p.m * 64);
-  for (int e = t; e < p.m * 16; e += kST) reinterpret_cast<float4*>(sm + kOffL)[e] = Lg[e];
+  float4* Ld = reinterpret_cast<float4*>(sm + kOffL);
+  int e = t;
+  for (; e + 3 * kST < p.m * 16; e += 4 * kST) {   // four loads in flight per thread
+    float4 r[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) r[x] = __ldg(Lg + e + x * kST);
+#pragma unroll
+    for (int x = 0; x < 4; ++x) Ld[e + x * kST] = r[x];
+  }
+  for (; e < p.m * 16; e += kST) Ld[e] = __ldg(Lg + e);
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -429,24 +438,34 @@ __global__ void __launch_bounds__(kST, 1) k_stream_pass2(const Params p, const S
   // m), the DWC taps of this unit's head
   const double* red = p.red + (size_t)u * p.part_stride;
   for (int j = t; j < m; j += kST) shs[j] = (float)(red[j] / (double)p.Ng);
+  __syncthreads();
+  // thread t takes channel k = t % 64 and landmark pairs (t / 64) + 8 i: it also sums mu_j M'[j][k] over
+  // its landmarks for the bias (the eight partial sums of a channel meet in aux below)
   const float* Mp = p.Mp + (size_t)u * m * 64;
+  float bmu = 0.f;
+#pragma unroll 4
   for (int e = t; e < npan * 32 * 64; e += kST) {
     const int k = e & 63, j = 2 * (e >> 6);
-    const float lo = j < m ? Mp[(size_t)j * 64 + k] : 0.f;
-    const float hi = j + 1 < m ? Mp[(size_t)(j + 1) * 64 + k] : 0.f;
+    const float lo = j < m ? __ldg(Mp + (size_t)j * 64 + k) : 0.f;
+    const float hi = j + 1 < m ? __ldg(Mp + (size_t)(j + 1) * 64 + k) : 0.f;
+    if (j < m) bmu = fmaf(shs[j], lo, bmu);
+    if (j + 1 < m) bmu = fmaf(shs[j + 1], hi, bmu);
     *reinterpret_cast<uint32_t*>(sm + kOffMimg + (j >> 6) * kPanel + sw128(k, (j & 63) >> 3) + ((j & 7) << 1)) =
         pack2(lo, hi);
   }
+  float* bpartial = taps + 9 * 64;   // [8][64]
+  bpartial[(t >> 6) * 64 + (t & 63)] = bmu;
   const int hd = u % p.heads;
   for (int e = t; e < 9 * 64; e += kST) {
     const int tap = e >> 6, k = e & 63;
     taps[e] = p.dwc[((size_t)hd * 64 + k) * 9 + tap];
   }
-  const uint32_t tmem = stream_setup(p, sm, 128, u);   // (its barrier also publishes shs, M'^T, taps)
+  const uint32_t tmem = stream_setup(p, sm, 128, u);   // (its barrier also publishes M'^T, taps, partials)
   if (t < 64) {
     float b = 0.f;
-    for (int c = 0; c < p.n_chunks; ++c) b += p.bpart[((size_t)u * p.n_chunks + c) * 64 + t];
-    for (int j = 0; j < m; ++j) b = fmaf(shs[j], Mp[(size_t)j * 64 + t], b);
+    for (int c = 0; c < p.n_chunks; ++c) b += __ldg(p.bpart + ((size_t)u * p.n_chunks + c) * 64 + t);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) b += bpartial[r * 64 + t];
     bias[t] = b;
   }
   auto issue = [&](int i) {
