@@ -223,7 +223,8 @@ lfa_status lfa_sp_pass2(lfa_handle h, const void* Q_local, const void* V_local, 
 size_t lfa_solver_workspace_size(int U, int m);
 
 /* X [U][m][m] = the T-step Newton-Schulz approximation of W^-1 the forward pass computes:
- * alpha = 2 / ||W||_2 (power iteration), or 1 / ||W||_2^2 when the printed condition
+ * alpha = 2 / ||W||_2 (power iteration; W must be symmetric, the iteration forms W v as the
+ * columns' sums), or 1 / ||W||_2^2 when the printed condition
  * ||I - alpha W W^T||_2 < 1 fails; X_0 = alpha W^T; X <- X (2I - W X), each product on tcgen05 in
  * split TF32 (hi*hi + hi*lo + lo*hi, about 2^-21 relative). workspace: lfa_solver_workspace_size
  * bytes, 256-byte aligned, overwritten. host_out (optional, U entries): alpha, lambda_max,
