@@ -47,6 +47,21 @@ __device__ __forceinline__ void store4(__nv_bfloat16* g, float4 v) {
 // sign(t) * x with sign(0) = 0
 __device__ __forceinline__ float sgn_mul(float t, float x) { return t > 0.f ? x : (t < 0.f ? -x : 0.f); }
 
+// acc + sign(t) x with sign(0) = 0: x with t's sign bit folded in (one logic instruction), kept where t != 0
+__device__ __forceinline__ float add_sgn(float acc, float t, float x) {
+  const float r = __int_as_float(__float_as_int(x) ^ (__float_as_int(t) & 0x80000000));
+  return acc + (t != 0.f ? r : 0.f);
+}
+
+// acc - sign(t) x with sign(0) = 0 on the FMA pipe: sat(t 2^126) is 1 for t >= 2^-126 and 0 for t <= 0
+// (and sat(-t 2^126) the other way round), so the two products add exactly -x, +x or nothing; the logic /
+// compare pipe, which the other sign contraction keeps busy, is not used. (A nonzero |t| below 2^-126
+// would give a fraction; t is a difference of a token entry and a landmark average.)
+__device__ __forceinline__ float sub_sgn_fma(float acc, float t, float x) {
+  const float sp = __saturatef(t * 0x1p126f), sn = __saturatef(t * -0x1p126f);
+  return fmaf(x, sn, fmaf(-x, sp, acc));
+}
+
 // X_0 = alpha W^T with the alpha the forward chose (per-unit info slot).
 __global__ void k_init_iterate(BwdParams b) {
   const Params& p = b.p;
@@ -368,7 +383,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_main(BwdParams b) {
             const float dd = Ds[(4 * ib + x) * kCS + lr], cv = Cs[(4 * ib + x) * kCS + lr];
 #pragma unroll
             for (int y = 0; y < 4; ++y) {
-              accQ[x][y] += sgn_mul(qv[x][y] - lv[y], dd);
+              accQ[x][y] = add_sgn(accQ[x][y], qv[x][y] - lv[y], dd);
               accV[x][y] = fmaf(cv, gv[y], accV[x][y]);
             }
           }
@@ -387,7 +402,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd_main(BwdParams b) {
 #pragma unroll
           for (int x = 0; x < 4; ++x)
 #pragma unroll
-            for (int y = 0; y < 4; ++y) accL[c][x][y] -= sgn_mul(qq[y] - lv[x][y], dd[x]);
+            for (int y = 0; y < 4; ++y) accL[c][x][y] = sub_sgn_fma(accL[c][x][y], qq[y] - lv[x][y], dd[x]);
         }
       }
     }
