@@ -125,6 +125,11 @@ EDGE = [
     Workload("m81", B=1, heads=2, H=36, W=36, d=64, r=4, T=24),
     # non-square grid
     Workload("rect", B=1, heads=1, H=24, W=40, d=64, r=8, T=20),
+    # more units than SMs: the per-stage path with one streaming thread block per unit, in two waves
+    Workload("many_units", B=80, heads=2, H=16, W=16, d=64, r=4, T=20),
+    # one landmark on the streaming passes (80 units: past the fused kernel's unit limit), 15 of 16 warps
+    # without a landmark
+    Workload("m1_stream", B=80, heads=1, H=16, W=16, d=64, r=16, T=20),
 ]
 
 

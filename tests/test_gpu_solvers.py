@@ -6,7 +6,9 @@ Newton-Schulz converges stably after a warm-up).
 Inputs: symmetric positive-definite W with a geometric spectrum between 1 and kappa (the same
 construction as the CPU robustness test) and standard normal right-hand sides, in batches of
 several systems, with m = 49 (the PVT landmark count), 196 and 256 and a ragged number of
-right-hand sides (70: two full 32-column blocks and a partial one).
+right-hand sides (70: two full 32-column blocks and a partial one). The Newton-Schulz call also runs at
+m = 64, 81, 100, 130 and 224: its chain launch takes one thread block per 128 x 64 tile of X (clusters
+of 1 to 8 blocks), and an m that is not a multiple of 4 takes the register-staged product tiles.
 
 Tolerances:
   * CG: the device runs the oracle's recursion in fp32 with another summation order. Its distance
@@ -73,7 +75,7 @@ def test_cg_is_deterministic():
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("m", [49, 196, 256])
+@pytest.mark.parametrize("m", [49, 64, 81, 100, 130, 196, 224, 256])
 def test_ns_solve_matches_oracle(m):
     U = 2
     W, _ = _systems(m, 50.0, U, 1, seed=m)
