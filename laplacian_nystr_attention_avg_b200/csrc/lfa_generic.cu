@@ -49,8 +49,25 @@ __device__ __forceinline__ float l1_4(float4 a, float4 b, float acc) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Landmark pooling: one warp per landmark, lanes over channels (coalesced along d).
+// Landmark pooling: one warp per landmark. A token row is C16 = d * sizeof(T) / 16 chunks of 16 bytes
+// (C16 in {4, 8, 16}); lane = (token group tg = lane / C16, chunk c = lane % C16), so one load
+// instruction of the warp covers 32 / C16 window tokens in full rows. The token groups' sums meet by
+// shuffles, in a fixed order. (Other d: one lane per channel.)
 // ---------------------------------------------------------------------------------------
+__device__ __forceinline__ int unpack16(const uint4& raw, float* f, const float*) {
+  f[0] = __uint_as_float(raw.x); f[1] = __uint_as_float(raw.y); f[2] = __uint_as_float(raw.z); f[3] = __uint_as_float(raw.w);
+  return 4;
+}
+__device__ __forceinline__ int unpack16(const uint4& raw, float* f, const __nv_bfloat16*) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+  return 8;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.status = 0;
@@ -62,7 +79,35 @@ __global__ void __launch_bounds__(kThreads) k_pool(Params p) {
   const int Y0 = (l / Wr) * p.r, X0 = (l % Wr) * p.r;
   const T* q = static_cast<const T*>(p.Q) + (size_t)u * p.N * p.d;
   const float inv = 1.0f / float(p.r * p.r);
-  // window rows outside this call's band of grid rows (sequence split) contribute nothing here
+  constexpr int kPer = 16 / (int)sizeof(T);   // values per 16-byte chunk
+  const int C16 = p.d / kPer;
+  if (p.d % kPer == 0 && (C16 == 4 || C16 == 8 || C16 == 16)) {
+    const int TG = 32 / C16, tg = lane / C16, c = lane % C16, rr = p.r * p.r;
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int t = tg; t < rr; t += TG) {
+      // window rows outside this call's band of grid rows (sequence split) contribute nothing here
+      const int yl = Y0 + t / p.r - p.y0;
+      if (yl < 0 || yl >= p.H) continue;
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)yl * p.W + X0 + t % p.r) * p.d) + c);
+      float f[kPer];
+      unpack16(raw, f, q);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += f[i];
+    }
+    for (int o = C16; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (tg == 0) {
+      float* dst = p.L + ((size_t)u * p.m + l) * p.d + c * kPer;
+#pragma unroll
+      for (int i = 0; i < kPer; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(acc[i] * inv, acc[i + 1] * inv, acc[i + 2] * inv, acc[i + 3] * inv);
+    }
+    return;
+  }
   for (int k = lane; k < p.d; k += 32) {
     float acc = 0.f;
     for (int dy = 0; dy < p.r; ++dy) {
