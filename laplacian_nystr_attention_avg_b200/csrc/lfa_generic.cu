@@ -478,11 +478,15 @@ __global__ void __launch_bounds__(kThreads) k_pool_batch_stats(Params p) {
 }
 
 // mu, s, A (all landmarks), then M = X A, M' and bias partials for 16 landmark rows.
+__host__ __device__ inline size_t combine_smem(int m, int d) {
+  return 2 * sizeof(double) * (size_t)m + sizeof(float) * ((size_t)m * d + 2 * m + 16 * (size_t)m + 16 * (size_t)d);
+}
 __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   extern __shared__ float4 smem_f4[];
-  float* sm = reinterpret_cast<float*>(smem_f4);
   const int m = p.m, d = p.d, u = blockIdx.y, c = blockIdx.x, t = threadIdx.x;
-  float* As = sm;               // [m][d]
+  double* mud = reinterpret_cast<double*>(smem_f4);   // [m] fp64 mean and scale, formed once
+  double* sd = mud + m;
+  float* As = reinterpret_cast<float*>(sd + m);       // [m][d]
   float* mus = As + m * d;      // [m]
   float* ss = mus + m;          // [m]
   const double* red = p.red + (size_t)u * p.part_stride;
@@ -492,6 +496,8 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
     double var = red[m + j] * invN - mu * mu;
     if (var < 0.0) var = 0.0;
     const double s = 1.0 / sqrt(var + (double)p.eps);
+    mud[j] = mu;
+    sd[j] = s;
     mus[j] = (float)mu;
     ss[j] = (float)s;
     if (c == 0) {
@@ -499,17 +505,14 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
       p.s[(size_t)u * m + j] = (float)s;
     }
   }
+  __syncthreads();
   const double* P = red + 2 * m;
   const double* SV = red + 2 * m + m * d;
   for (int e = t; e < m * d; e += blockDim.x) {
     const int j = e / d, k = e % d;
     double a;
     if (p.whiten) {
-      const double mu = red[j] * invN;
-      double var = red[m + j] * invN - mu * mu;
-      if (var < 0.0) var = 0.0;
-      const double s = 1.0 / sqrt(var + (double)p.eps);
-      a = s * (P[e] - mu * SV[k]) + SV[k] * invN;
+      a = sd[j] * (P[e] - mud[j] * SV[k]) + SV[k] * invN;
     } else {
       a = P[e];
     }
@@ -517,17 +520,39 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
     if (c == 0) p.A[(size_t)u * m * d + e] = (float)a;
   }
   __syncthreads();
-  // rows [16c, 16c + 16) of M = X A
+  // rows [16c, 16c + 16) of M = X A: the rows of X staged in shared memory, four output entries per
+  // thread with their sums over l interleaved (each one still in l order); 16 d <= 4 kThreads because
+  // the library accepts d = 32 and 64 only
   const float* Xg = p.X + (size_t)u * m * m;
   float* bp = p.bpart + ((size_t)u * p.n_chunks + c) * d;
-  const int j0 = c * 16;
-  for (int e = t; e < 16 * d; e += blockDim.x) {
-    const int jj = e / d, k = e % d, j = j0 + jj;
-    if (j < m) {
-      float acc = 0.f;
-      for (int l = 0; l < m; ++l) acc = fmaf(Xg[(size_t)j * m + l], As[l * d + k], acc);
-      p.M[((size_t)u * m + j) * d + k] = acc;
-      p.Mp[((size_t)u * m + j) * d + k] = p.whiten ? ss[j] * acc : acc;
+  const int j0 = c * 16, nj = min(16, m - j0);
+  float* Xs = ss + m;        // [16][m]
+  float* Ms = Xs + 16 * m;   // [16][d]
+  for (int e = t; e < nj * m; e += blockDim.x) Xs[e] = __ldg(Xg + (size_t)j0 * m + e);
+  __syncthreads();
+  {
+    int jj[4], kk[4];
+    bool ok[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int e = t + kThreads * x;
+      jj[x] = e / d;
+      kk[x] = e % d;
+      ok[x] = e < 16 * d && jj[x] < nj;
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int l = 0; l < m; ++l) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        if (ok[x]) acc[x] = fmaf(Xs[jj[x] * m + l], As[l * d + kk[x]], acc[x]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      if (!ok[x]) continue;
+      const int j = j0 + jj[x];
+      p.M[((size_t)u * m + j) * d + kk[x]] = acc[x];
+      p.Mp[((size_t)u * m + j) * d + kk[x]] = p.whiten ? ss[j] * acc[x] : acc[x];
+      Ms[jj[x] * d + kk[x]] = acc[x];
     }
   }
   __syncthreads();
@@ -535,9 +560,9 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   for (int k = t; k < d; k += blockDim.x) {
     float acc = 0.f;
     if (p.whiten) {
-      for (int jj = 0; jj < 16; ++jj) {
+      for (int jj = 0; jj < nj; ++jj) {
         const int j = j0 + jj;
-        if (j < m) acc += (float)(invN - (double)ss[j] * (double)mus[j]) * p.M[((size_t)u * m + j) * d + k];
+        acc += (float)(invN - (double)ss[j] * (double)mus[j]) * Ms[jj * d + k];
       }
     }
     bp[k] = acc;
@@ -1028,7 +1053,7 @@ void context_t(const Params& p, cudaStream_t st) {
               if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, s>>>(p);
             },
             [&](cudaStream_t s) { ns_t(p, s); });
-  k_combine_finish<<<dim3(p.n_chunks, U), kThreads, (size_t)(m * d + 2 * m) * sizeof(float), st>>>(p);
+  k_combine_finish<<<dim3(p.n_chunks, U), kThreads, combine_smem(m, d), st>>>(p);
 }
 
 template <typename T>
@@ -1120,7 +1145,7 @@ cudaError_t launch_ns_from_w(const Params& p, cudaStream_t st) {
 
 // The combine from the fp64 totals in the workspace (mu, s, A, M, M', b), then pass 2.
 cudaError_t launch_generic_finish(const Params& p, cudaStream_t st) {
-  k_combine_finish<<<dim3(p.n_chunks, p.U), kThreads, (size_t)(p.m * p.d + 2 * p.m) * sizeof(float), st>>>(p);
+  k_combine_finish<<<dim3(p.n_chunks, p.U), kThreads, combine_smem(p.m, p.d), st>>>(p);
   if (p.dtype == LFA_BF16) pass2_t<__nv_bfloat16>(p, st);
   else pass2_t<float>(p, st);
   return cudaGetLastError();
