@@ -508,16 +508,26 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   __syncthreads();
   const double* P = red + 2 * m;
   const double* SV = red + 2 * m + m * d;
-  for (int e = t; e < m * d; e += blockDim.x) {
-    const int j = e / d, k = e % d;
-    double a;
-    if (p.whiten) {
-      a = sd[j] * (P[e] - mud[j] * SV[k]) + SV[k] * invN;
-    } else {
-      a = P[e];
+  // eight entries of A per thread and step, their fp64 loads issued first
+  const int md = m * d, nt = blockDim.x;
+  for (int e0 = t; e0 < md; e0 += 8 * nt) {
+    double pv[8], sv[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int e = e0 + x * nt;
+      pv[x] = e < md ? __ldg(P + e) : 0.0;
+      sv[x] = e < md ? __ldg(SV + e % d) : 0.0;
     }
-    As[e] = (float)a;
-    if (c == 0) p.A[(size_t)u * m * d + e] = (float)a;
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int e = e0 + x * nt;
+      if (e < md) {
+        const int j = e / d;
+        const double a = p.whiten ? sd[j] * (pv[x] - mud[j] * sv[x]) + sv[x] * invN : pv[x];
+        As[e] = (float)a;
+        if (c == 0) p.A[(size_t)u * m * d + e] = (float)a;
+      }
+    }
   }
   __syncthreads();
   // rows [16c, 16c + 16) of M = X A: the rows of X staged in shared memory, four output entries per
@@ -528,7 +538,7 @@ __global__ void __launch_bounds__(kThreads) k_combine_finish(Params p) {
   const int j0 = c * 16, nj = min(16, m - j0);
   float* Xs = ss + m;        // [16][m]
   float* Ms = Xs + 16 * m;   // [16][d]
-  for (int e = t; e < nj * m; e += blockDim.x) Xs[e] = __ldg(Xg + (size_t)j0 * m + e);
+  stage_floats(Xs, Xg + (size_t)j0 * m, nj * m, m, m);
   __syncthreads();
   {
     int jj[4], kk[4];
