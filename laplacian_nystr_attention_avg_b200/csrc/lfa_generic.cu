@@ -177,18 +177,29 @@ constexpr int kAlphaRegRows = 56;
 static_assert(kMaxM - alpha_rows(kMaxM) <= kAlphaRegRows, "rows of W beyond shared memory and registers");
 static_assert(kMaxM <= kAlphaThreads, "one thread per entry of the power-iteration vector");
 
-__device__ __forceinline__ float block_sum256(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+// block sums of a and b (kAlphaThreads threads; red holds 2 x kAlphaThreads / 32 floats): one barrier
+__device__ __forceinline__ void block_sum2_256(float& a, float& b, float* red) {
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[threadIdx.x >> 5] = a;
+    red[kAlphaThreads / 32 + (threadIdx.x >> 5)] = b;
+  }
   __syncthreads();
-  float s = 0.f;
+  float sa = 0.f, sb = 0.f;
 #pragma unroll
-  for (int i = 0; i < kAlphaThreads / 32; ++i) s += red[i];
-  return s;
+  for (int i = 0; i < kAlphaThreads / 32; ++i) {
+    sa += red[i];
+    sb += red[kAlphaThreads / 32 + i];
+  }
+  a = sa;
+  b = sb;
 }
 
 __global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
-  __shared__ float v[kMaxM], red[2][kAlphaThreads / 32];
+  __shared__ float v[kMaxM], red[2][2 * kAlphaThreads / 32];
   extern __shared__ float4 smem_f4[];
   float* Ws = reinterpret_cast<float*>(smem_f4);   // [alpha_rows(m)][m]
   const int u = blockIdx.x, m = p.m, t = threadIdx.x;
@@ -224,10 +235,10 @@ __global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
       }
     }
     const float w = (a0 + a1) + (a2 + a3);
-    // v^T w and ||w||^2 (two reduction buffers: the second sum may start before every thread has
-    // read the first one's result, and v is rewritten only after both)
-    const float vw = block_sum256(t < m ? w * v[t] : 0.f, red[0]);
-    const float nn = block_sum256(t < m ? w * w : 0.f, red[1]);
+    // v^T w and ||w||^2 in one reduction (the buffer alternates between steps: a step's sums may be
+    // written before every thread has read the previous step's; v is rewritten after the barrier)
+    float vw = t < m ? w * v[t] : 0.f, nn = t < m ? w * w : 0.f;
+    block_sum2_256(vw, nn, red[it & 1]);
     rq = vw;
     if (it == iters) break;
     if (t < m) v[t] = w * rsqrtf(nn);
