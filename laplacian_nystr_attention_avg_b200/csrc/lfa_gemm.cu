@@ -4,12 +4,17 @@
 // Reading-B products.
 //
 // Out = scale * op(A) op(B) + beta * Cin + add_diag * I per (job, unit); up to three independent jobs
-// share one launch (grid z = job * U + unit). Each CTA forms a 128 x 64 output tile (M = 128 rows i,
-// N = 64 columns j) in a TMEM accumulator, fp32-accurate by three TF32 products (hi*hi + hi*lo +
-// lo*hi with hi = tf32(x), lo = x - hi: about 2^-21 relative per product). K advances in steps of 64
-// (two 128-byte SW128 K-halves of fp32 per row). The operands of step c + 1 are already in registers
-// while the 24 MMAs of step c run: they are split and stored into the other shared-memory stage, and
-// the global loads of step c + 2 are issued right after, so one L2 latency overlaps each step.
+// share one launch (grid z = job * U + unit). Each CTA (512 threads) forms a 128 x 64 output tile
+// (M = 128 rows i, N = 64 columns j) in a TMEM accumulator, fp32-accurate by three TF32 products
+// (hi*hi + hi*lo + lo*hi with hi = tf32(x), lo = x - hi: about 2^-21 relative per product). Two tile
+// bodies, each compiled per transpose combination:
+//   * m % 4 == 0 (mm_tile_async): K in steps of 32; the operands arrive by cp.async in a three-slot
+//     ring in the layout the tensor cores read (K- or MN-major, no transposing stores), fifteen warps
+//     split each step in place while one lane of the last warp issues the products of the step before;
+//   * other m (mm_tile): K in steps of 64; the operands of step c + 1 wait in registers while the 24
+//     MMAs of step c run, then are split and stored (transposes element by element) into the other of
+//     two stages, and the loads of step c + 2 go out right after.
+// The epilogue stages the tile through shared memory and writes whole rows.
 //
 // The Newton-Schulz chains (the forward's X_{k+1} = X_k (2I - W X_k), k < T, and the backward's
 // iterates X_1 .. X_{T-1}) also run as ONE launch, k_ns_chain: a thread-block cluster per unit whose
