@@ -25,12 +25,12 @@
  *   - Tensors Q, V, O, dO, dQ, dV are contiguous [B][heads][N][d] in the config's
  *     dtype (fp32 or bf16). Device pointers must be 16-byte aligned.
  *     Arithmetic: distances, exponentials, sums and the whitening statistics are fp32 (the
- *     statistics' cross-CTA reductions fp64). The per-stage kernels (every fp32 shape, and
- *     the bf16 shapes the fused kernel does not take) do every product in fp32 on CUDA
- *     cores. The fused bf16 kernel (lfa_forward_path "fused") instead keeps C as bf16 on
- *     chip and runs C^T V and C M' as bf16-operand tensor-core products with fp32
- *     accumulation, and the m x m Newton-Schulz and M = X A products as split-TF32
- *     tensor-core products (hi*hi + hi*lo + lo*hi, fp32 accumulation).
+ *     statistics' cross-CTA reductions fp64). The m x m Newton-Schulz products (and, in the
+ *     fused kernel, M = X A) are split-TF32 tensor-core products (hi*hi + hi*lo + lo*hi, fp32
+ *     accumulation). For bf16 tokens with d = 64 (the fused kernel, lfa_forward_path "fused",
+ *     and the per-stage streaming passes) C^T V and C M' are bf16-operand tensor-core products
+ *     with fp32 accumulation, taken on bf16(C - c) with c a per-column shift; for fp32 tokens and
+ *     d = 32 the per-stage kernels run those two products in fp32 on CUDA cores.
  *   - The DWC weight is fp32 [heads][d][3][3] on the device.
  *   - All device memory is owned by the caller. The handle owns host state only and
  *     keeps the weight and workspace pointers it was created with; the weight is read
