@@ -157,6 +157,15 @@ lfa_status lfa_forward_noalloc(const lfa_config* cfg, const float* dwc_weight, c
 lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
                             void* Q_dev, void* V_dev, void* O_dev, void* stream);
 
+/* lfa_forward_host without the final synchronisation: the two copies in, the forward and the copy out
+ * are only enqueued on `stream`. O_host is ready, and the host and device buffers may be reused or
+ * freed, once the caller has synchronised `stream` (or waited on an event recorded after the call).
+ * With pinned host buffers, calls on two streams (two handles: a handle's workspace serves one call
+ * at a time) overlap one call's copies with the other's forward and copies. Same arguments and argument
+ * errors as lfa_forward_host. */
+lfa_status lfa_forward_host_async(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
+                                  void* Q_dev, void* V_dev, void* O_dev, void* stream);
+
 /* Backward pass for the loss <dO, O>: writes dQ and dV ([B][heads][N][d], cfg.dtype).
  * Reuses the context saved by the most recent lfa_forward on this handle, which
  * must have been called with the same Q and V pointers (else LFA_ERR_STATE).

@@ -181,6 +181,32 @@ void bind_backward(lfa::BwdParams* b, const Params& p, const Layout& L, unsigned
   b->dQd = f(L.b_dQd);
 }
 
+// Fused forwards on one device run one at a time, in the order they were enqueued, whatever their
+// stream: each waits for the previous one's completion event and records its own. (Its thread blocks wait
+// on flags of the same launch, so a launch should not share the SMs with another one; host-buffer calls
+// on two streams still overlap their copies with each other's forwards.)
+std::mutex g_fused_mu;
+cudaEvent_t g_fused_ev[64] = {};
+
+cudaError_t launch_fused_in_order(const Params& p, int grid, unsigned char* ws, unsigned long long epoch,
+                                  cudaStream_t st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_fused_mu);
+  if (!g_fused_ev[dev]) {
+    const cudaError_t e = cudaEventCreateWithFlags(&g_fused_ev[dev], cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  } else if (cudaStreamWaitEvent(st, g_fused_ev[dev], 0) != cudaSuccess) {
+    // an event of an earlier context (the device was reset since): start the order afresh
+    cudaGetLastError();
+    const cudaError_t e = cudaEventCreateWithFlags(&g_fused_ev[dev], cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  const cudaError_t e = lfa::launch_fused_forward(p, grid, ws, epoch, st);
+  if (e != cudaSuccess) return e;
+  return cudaEventRecord(g_fused_ev[dev], st);
+}
+
 // Kernel attributes (dynamic shared memory opt-in) are per device; set them once each.
 std::mutex g_attr_mu;
 unsigned long long g_attr_done = 0;
@@ -327,7 +353,7 @@ lfa_status lfa_forward(lfa_handle h, const void* Q, const void* V, void* O, void
       p.spin_budget = h->spin_test_budget;
       h->spin_test_budget = -1;   // one-shot
     }
-    if (lfa::launch_fused_forward(p, h->grid, h->ws + h->lay.fused, epoch, st) != cudaSuccess) return LFA_ERR_CUDA;
+    if (launch_fused_in_order(p, h->grid, h->ws + h->lay.fused, epoch, st) != cudaSuccess) return LFA_ERR_CUDA;
     h->epoch = epoch;
   } else {
     // the tcgen05 pass 2 copies the C it multiplies (bf16(C - mu) widened, mu added back) as it goes;
@@ -396,8 +422,8 @@ lfa_status lfa_forward_noalloc(const lfa_config* cfg, const float* dwc_weight, c
                                                                                            : LFA_ERR_CUDA;
 }
 
-lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
-                            void* Q_dev, void* V_dev, void* O_dev, void* stream) {
+lfa_status lfa_forward_host_async(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
+                                  void* Q_dev, void* V_dev, void* O_dev, void* stream) {
   if (!h || !Q_host || !V_host || !O_host || !Q_dev || !V_dev || !O_dev) return LFA_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t bytes = (size_t)h->p.U * h->p.N * h->p.d * elem_bytes(h->cfg);
@@ -406,7 +432,14 @@ lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host
   lfa_status s = lfa_forward(h, Q_dev, V_dev, O_dev, stream);
   if (s != LFA_OK) return s;
   if (cudaMemcpyAsync(O_host, O_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return LFA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return LFA_ERR_CUDA;
+  return LFA_OK;
+}
+
+lfa_status lfa_forward_host(lfa_handle h, const void* Q_host, const void* V_host, void* O_host,
+                            void* Q_dev, void* V_dev, void* O_dev, void* stream) {
+  const lfa_status s = lfa_forward_host_async(h, Q_host, V_host, O_host, Q_dev, V_dev, O_dev, stream);
+  if (s != LFA_OK) return s;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return LFA_ERR_CUDA;
   return LFA_OK;
 }
 

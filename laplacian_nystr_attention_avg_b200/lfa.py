@@ -55,6 +55,7 @@ def _declare(lib: ctypes.CDLL) -> None:
         "lfa_create": (ci, [cfgp, vp, vp, sz, ctypes.POINTER(vp)]),
         "lfa_forward": (ci, [vp, vp, vp, vp, vp]),
         "lfa_forward_host": (ci, [vp, vp, vp, vp, vp, vp, vp, vp]),
+        "lfa_forward_host_async": (ci, [vp, vp, vp, vp, vp, vp, vp, vp]),
         "lfa_forward_noalloc": (ci, [cfgp, vp, vp, vp, vp, vp]),
         "lfa_backward": (ci, [vp, vp, vp, vp, vp, vp, vp]),
         "lfa_get_info": (ci, [vp, ctypes.POINTER(UnitInfo), ci, vp]),
@@ -317,6 +318,16 @@ class LaplacianNystromAttention:
             _require(t, name, self.shape, self.dtype, self.device)
         _check(self.lib.lfa_forward_host(self.handle, _ptr(Q_host), _ptr(V_host), _ptr(O_host), _ptr(Q_dev),
                                          _ptr(V_dev), _ptr(O_dev), _stream(stream)), "lfa_forward_host")
+
+    def forward_host_async(self, Q_host, V_host, O_host, Q_dev, V_dev, O_dev, stream=None) -> None:
+        """lfa_forward_host_async: enqueue copies in, the forward and the copy out; O_host is ready once
+        `stream` has been synchronised."""
+        for name, t in (("Q_host", Q_host), ("V_host", V_host), ("O_host", O_host)):
+            _require(t, name, self.shape, self.dtype, host=True)
+        for name, t in (("Q_dev", Q_dev), ("V_dev", V_dev), ("O_dev", O_dev)):
+            _require(t, name, self.shape, self.dtype, self.device)
+        _check(self.lib.lfa_forward_host_async(self.handle, _ptr(Q_host), _ptr(V_host), _ptr(O_host), _ptr(Q_dev),
+                                               _ptr(V_dev), _ptr(O_dev), _stream(stream)), "lfa_forward_host_async")
 
     def backward(self, Q, V, dO, dQ=None, dV=None, stream=None):
         if dQ is None:

@@ -187,6 +187,34 @@ def test_forward_host_buffers():
     assert torch.equal(Oh, ref)
 
 
+@pytest.mark.parametrize("name", ["pvt1", "hr196"])
+def test_forward_host_async_on_two_streams(name):
+    # two handles on two streams, alternate steps with their own pinned buffers: every step's O equals the
+    # one-stream forward's (fused launches are ordered per device; the copies overlap)
+    wl = pu.workload(name)
+    x = pu.inputs_for(wl)
+    mods = [pu.gpu_module(wl, True, False) for _ in range(2)]
+    ref = mods[0].forward(x.Q_store.cuda(), x.V_store.cuda()).cpu()
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    host = [(x.Q_store.pin_memory(), x.V_store.pin_memory(), torch.empty(x.Q_store.shape, dtype=x.Q_store.dtype).pin_memory())
+            for _ in range(2)]
+    dev = [tuple(torch.empty(x.Q_store.shape, dtype=x.Q_store.dtype, device="cuda") for _ in range(3)) for _ in range(2)]
+    outs = []
+    for k in range(6):
+        i = k % 2
+        host[i][2].zero_()
+        mods[i].forward_host_async(*host[i], *dev[i], stream=streams[i])
+        if k >= 1:
+            j = 1 - i
+            streams[j].synchronize()
+            outs.append(host[j][2].clone())
+    streams[1 - (5 % 2)].synchronize()
+    streams[5 % 2].synchronize()
+    outs.append(host[5 % 2][2].clone())
+    for o in outs:
+        assert torch.equal(o, ref)
+
+
 @pytest.mark.parametrize("name", ["pvt1", "pvt2", "hr49"])
 def test_fused_and_generic_paths_agree(name, monkeypatch):
     wl = pu.workload(name)
