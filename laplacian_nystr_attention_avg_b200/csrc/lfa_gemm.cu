@@ -306,43 +306,95 @@ __device__ __noinline__ void mm_tile_async(const MmJob& J, int m, int u, int i0,
   const int t = threadIdx.x;
   const bool issuer = t >= kSplitters;
   const int nk = (m + kKS2 - 1) / kKS2;
+  // This thread's copy items, fixed for the tile: up to three 16-byte chunks of A (1024 per step) and
+  // two of B (512), each with its shared-memory offset inside a slot, its source at k0 = 0, the position
+  // along K that bounds it (k0 + kpos < m) and whether its row / column lies inside the matrix. A step
+  // advances K-major sources by k0 elements and MN-major ones by k0 rows.
+  struct Item {
+    const float* base;
+    uint32_t dst;
+    int kpos;
+    bool in;
+  };
+  Item ia[3], ib[2];
+#pragma unroll
+  for (int x = 0; x < 3; ++x) {
+    const int e = t + kSplitters * x;
+    Item it{A, 0u, 0, false};
+    if (e < 1024) {
+      if constexpr (!TA) {
+        const int row = e >> 3, kc = e & 7;
+        it = Item{A + (size_t)(i0 + row) * m + 4 * kc, kSlotHiA + sw128(row, kc), 4 * kc, i0 + row < m};
+      } else {
+        const int kl = e >> 5, ic = e & 31;
+        it = Item{A + (size_t)kl * m + i0 + 4 * ic, kSlotHiA + (ic >> 3) * 4096 + mnofs(kl, ic & 7), kl, i0 + 4 * ic < m};
+      }
+    }
+    ia[x] = it;
+  }
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int e = t + kSplitters * x;
+    Item it{B, 0u, 0, false};
+    if (e < 512) {
+      if constexpr (!TB) {
+        const int kl = e >> 4, jc = e & 15;
+        it = Item{B + (size_t)kl * m + j0 + 4 * jc, kSlotHiB + (jc >> 3) * 4096 + mnofs(kl, jc & 7), kl, j0 + 4 * jc < m};
+      } else {
+        const int jl = e >> 3, kc = e & 7;
+        it = Item{B + (size_t)(j0 + jl) * m + 4 * kc, kSlotHiB + sw128(jl, kc), 4 * kc, j0 + jl < m};
+      }
+    }
+    ib[x] = it;
+  }
+  const bool has_a[3] = {t < 1024, t + kSplitters < 1024, t + 2 * kSplitters < 1024};
+  const bool has_b[2] = {t < 512, t + kSplitters < 512};
   auto issue = [&](int c) {
     const int k0 = c * kKS2;
-    const uint32_t sa = sbase + ((gs + c) % 3) * kSlot + kSlotHiA, sb = sbase + ((gs + c) % 3) * kSlot + kSlotHiB;
-    for (int e = t; e < 1024; e += kSplitters) {   // A
-      if constexpr (!TA) {
-        const int row = e >> 3, kc = e & 7, i = i0 + row, k = k0 + 4 * kc;
-        const bool ok = i < m && k < m;
-        cp_async16(sa + sw128(row, kc), ok ? A + (size_t)i * m + k : A, ok);
-      } else {
-        const int kl = e >> 5, ic = e & 31, k = k0 + kl, i = i0 + 4 * ic;
-        const bool ok = k < m && i < m;
-        cp_async16(sa + (ic >> 3) * 4096 + mnofs(kl, ic & 7), ok ? A + (size_t)k * m + i : A, ok);
+    const uint32_t sl = sbase + ((gs + c) % 3) * kSlot;
+    const size_t sa = TA ? (size_t)k0 * m : (size_t)k0, sb = TB ? (size_t)k0 : (size_t)k0 * m;
+#pragma unroll
+    for (int x = 0; x < 3; ++x)
+      if (has_a[x]) {
+        const bool ok = ia[x].in && k0 + ia[x].kpos < m;
+        cp_async16(sl + ia[x].dst, ok ? ia[x].base + sa : A, ok);
       }
-    }
-    for (int e = t; e < 512; e += kSplitters) {    // B
-      if constexpr (!TB) {
-        const int kl = e >> 4, jc = e & 15, k = k0 + kl, j = j0 + 4 * jc;
-        const bool ok = k < m && j < m;
-        cp_async16(sb + (jc >> 3) * 4096 + mnofs(kl, jc & 7), ok ? B + (size_t)k * m + j : B, ok);
-      } else {
-        const int jl = e >> 3, kc = e & 7, j = j0 + jl, k = k0 + 4 * kc;
-        const bool ok = j < m && k < m;
-        cp_async16(sb + sw128(jl, kc), ok ? B + (size_t)j * m + k : B, ok);
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+      if (has_b[x]) {
+        const bool ok = ib[x].in && k0 + ib[x].kpos < m;
+        cp_async16(sl + ib[x].dst, ok ? ib[x].base + sb : B, ok);
       }
-    }
     cp_async_commit();
   };
-  auto split4 = [&](uint32_t off_hi, uint32_t off_lo) {
-    float4* ph = reinterpret_cast<float4*>(sm + off_hi);
-    const float4 v = *ph;
-    float4 h, l;
-    h.x = tf32_round(v.x); l.x = v.x - h.x;
-    h.y = tf32_round(v.y); l.y = v.y - h.y;
-    h.z = tf32_round(v.z); l.z = v.z - h.z;
-    h.w = tf32_round(v.w); l.w = v.w - h.w;
-    *ph = h;
-    *reinterpret_cast<float4*>(sm + off_lo) = l;
+  // a step's split: up to four float4 per thread, all loaded before any is converted (in place: hi over
+  // the raw value, lo beside it)
+  uint32_t so_hi[4], so_lo[4];
+  bool so_ok[4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int e = t + kSplitters * x;
+    so_ok[x] = e < 1536;
+    const uint32_t o = 16u * (e < 1024 ? e : e - 1024);
+    so_hi[x] = (e < 1024 ? kSlotHiA : kSlotHiB) + o;
+    so_lo[x] = (e < 1024 ? kSlotLoA : kSlotLoB) + o;
+  }
+  auto split_step = [&](uint32_t slot) {
+    float4 v[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+      if (so_ok[x]) v[x] = *reinterpret_cast<const float4*>(sm + slot + so_hi[x]);
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+      if (so_ok[x]) {
+        float4 h, l;
+        h.x = tf32_round(v[x].x); l.x = v[x].x - h.x;
+        h.y = tf32_round(v[x].y); l.y = v[x].y - h.y;
+        h.z = tf32_round(v[x].z); l.z = v[x].z - h.z;
+        h.w = tf32_round(v[x].w); l.w = v[x].w - h.w;
+        *reinterpret_cast<float4*>(sm + slot + so_hi[x]) = h;
+        *reinterpret_cast<float4*>(sm + slot + so_lo[x]) = l;
+      }
   };
   if (!issuer) {
     issue(0);
@@ -354,11 +406,7 @@ __device__ __noinline__ void mm_tile_async(const MmJob& J, int m, int u, int i0,
       if (c + 1 < nk) cp_async_wait<1>();
       else cp_async_wait<0>();
       named_bar_sync(1, kSplitters);
-      for (int e = t; e < 1536; e += kSplitters) {
-        const uint32_t o = 16u * (e < 1024 ? e : e - 1024);
-        if (e < 1024) split4(slot + kSlotHiA + o, slot + kSlotLoA + o);
-        else split4(slot + kSlotHiB + o, slot + kSlotLoB + o);
-      }
+      split_step(slot);
       fence_async_smem();
       named_bar_arrive(2 + (c & 1), kGT);
       // the products of step c - 1 are complete: their slot takes the copies of step c + 2
