@@ -164,97 +164,109 @@ __global__ void __launch_bounds__(kThreads) k_gram(Params p) {
   }
 }
 
-// Power iteration for ||W||_2: one CTA of kAlphaThreads per unit, thread t owns entry t of the iterate
-// (m <= kAlphaThreads). W is symmetric, so thread t forms (W v)_t as column t, sum_j W[j][t] v_j: the
-// threads of a warp read consecutive words of one row (conflict-free in shared memory, coalesced in L2).
-// The first alpha_rows(m) rows of W are staged in shared memory once, the rest (at most 56, for m = 256)
-// in registers, column t of each in thread t. Four partial sums per thread shorten the dependent chain.
-constexpr int kAlphaThreads = 256;
+// Power iteration for ||W||_2: one CTA of kAlphaThreads per unit, four groups of kAlphaCols threads.
+// Thread t of group g owns column t (m <= kAlphaCols): W is symmetric, so (W v)_t is column t,
+// sum_j W[j][t] v_j, and the threads of a warp read consecutive words of one row (conflict-free in
+// shared memory, coalesced in L2). Group g sums a quarter of the rows j; the four partials meet in
+// shared memory in a fixed order. The first alpha_rows(m) rows of W are staged in shared memory once,
+// the rest (at most 56, for m = 256) in registers, kAlphaRegRows of them per group. The split keeps
+// 32 warps per SM and a short dependent chain: a step's time is the shared-memory reads of W.
+constexpr int kAlphaCols = 256;
+constexpr int kAlphaGroups = 4;
+constexpr int kAlphaThreads = kAlphaCols * kAlphaGroups;
 __host__ __device__ constexpr int alpha_rows(int m) {
   return m < (200 * 1024) / (4 * (m > 0 ? m : 1)) ? m : (200 * 1024) / (4 * (m > 0 ? m : 1));
 }
-constexpr int kAlphaRegRows = 56;
-static_assert(kMaxM - alpha_rows(kMaxM) <= kAlphaRegRows, "rows of W beyond shared memory and registers");
-static_assert(kMaxM <= kAlphaThreads, "one thread per entry of the power-iteration vector");
+constexpr int kAlphaRegRows = 14;
+static_assert(kMaxM - alpha_rows(kMaxM) <= kAlphaGroups * kAlphaRegRows, "rows of W beyond shared memory and registers");
+static_assert(kMaxM <= kAlphaCols, "one thread per entry of the power-iteration vector");
 
-// block sums of a and b (kAlphaThreads threads; red holds 2 x kAlphaThreads / 32 floats): one barrier
-__device__ __forceinline__ void block_sum2_256(float& a, float& b, float* red) {
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-  if ((threadIdx.x & 31) == 0) {
-    red[threadIdx.x >> 5] = a;
-    red[kAlphaThreads / 32 + (threadIdx.x >> 5)] = b;
-  }
-  __syncthreads();
-  float sa = 0.f, sb = 0.f;
-#pragma unroll
-  for (int i = 0; i < kAlphaThreads / 32; ++i) {
-    sa += red[i];
-    sb += red[kAlphaThreads / 32 + i];
-  }
-  a = sa;
-  b = sb;
-}
-
-__global__ void __launch_bounds__(kAlphaThreads) k_alpha(Params p) {
-  __shared__ float v[kMaxM], red[2][2 * kAlphaThreads / 32];
+__global__ void __launch_bounds__(kAlphaThreads, 1) k_alpha(Params p) {
+  __shared__ __align__(16) float v[kMaxM];
+  __shared__ float part[kAlphaGroups][kAlphaCols], red[2 * kAlphaCols / 32];
   extern __shared__ float4 smem_f4[];
   float* Ws = reinterpret_cast<float*>(smem_f4);   // [alpha_rows(m)][m]
-  const int u = blockIdx.x, m = p.m, t = threadIdx.x;
+  const int u = blockIdx.x, m = p.m;
+  const int t = threadIdx.x % kAlphaCols, g = threadIdx.x / kAlphaCols;
   const float* Wg = p.Wm + (size_t)u * m * m;
   const int rs = alpha_rows(m);
   stage_floats(Ws, Wg, rs * m, m, m);
+  // this group's rows: [j0, j1) of the staged ones (j0 a multiple of 4, so v[j0..] reads as float4),
+  // then rows rg + q (q < kAlphaRegRows) from registers
+  const int qrows = ((rs + 4 * kAlphaGroups - 1) / (4 * kAlphaGroups)) * 4;
+  const int j0 = min(rs, g * qrows), j1 = min(rs, j0 + qrows);
+  const int rg = rs + g * kAlphaRegRows;
   float wr[kAlphaRegRows];
 #pragma unroll
-  for (int q = 0; q < kAlphaRegRows; ++q) wr[q] = (t < m && rs + q < m) ? Wg[(size_t)(rs + q) * m + t] : 0.f;
-  if (t < m) v[t] = rsqrtf(float(m));
+  for (int q = 0; q < kAlphaRegRows; ++q) wr[q] = (t < m && rg + q < m) ? Wg[(size_t)(rg + q) * m + t] : 0.f;
+  if (threadIdx.x < m) v[threadIdx.x] = rsqrtf(float(m));
   __syncthreads();
   float rq = 0.f;
   const int iters = 24;
-  const int r4 = rs & ~3;
+  const int j4 = j0 + ((j1 - j0) & ~3);
   for (int it = 0; it <= iters; ++it) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
     if (t < m) {
-      for (int j = 0; j < r4; j += 4) {
-        a0 = fmaf(Ws[(size_t)j * m + t], v[j], a0);
-        a1 = fmaf(Ws[(size_t)(j + 1) * m + t], v[j + 1], a1);
-        a2 = fmaf(Ws[(size_t)(j + 2) * m + t], v[j + 2], a2);
-        a3 = fmaf(Ws[(size_t)(j + 3) * m + t], v[j + 3], a3);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      for (int j = j0; j < j4; j += 4) {
+        const float4 vj = *reinterpret_cast<const float4*>(v + j);
+        a0 = fmaf(Ws[(size_t)j * m + t], vj.x, a0);
+        a1 = fmaf(Ws[(size_t)(j + 1) * m + t], vj.y, a1);
+        a2 = fmaf(Ws[(size_t)(j + 2) * m + t], vj.z, a2);
+        a3 = fmaf(Ws[(size_t)(j + 3) * m + t], vj.w, a3);
       }
-      for (int j = r4; j < rs; ++j) a0 = fmaf(Ws[(size_t)j * m + t], v[j], a0);
-      if (rs < m) {
+      for (int j = j4; j < j1; ++j) a0 = fmaf(Ws[(size_t)j * m + t], v[j], a0);
+      if (rg < m) {
 #pragma unroll
-        for (int q = 0; q < kAlphaRegRows; q += 4) {
-          if (rs + q < m) a1 = fmaf(wr[q], v[rs + q], a1);
-          if (rs + q + 1 < m) a2 = fmaf(wr[q + 1], v[rs + q + 1], a2);
-          if (rs + q + 2 < m) a3 = fmaf(wr[q + 2], v[rs + q + 2], a3);
-          if (rs + q + 3 < m) a0 = fmaf(wr[q + 3], v[rs + q + 3], a0);
+        for (int q = 0; q < kAlphaRegRows; ++q) {
+          if (rg + q >= m) break;
+          if (q % 4 == 0) a1 = fmaf(wr[q], v[rg + q], a1);
+          if (q % 4 == 1) a2 = fmaf(wr[q], v[rg + q], a2);
+          if (q % 4 == 2) a3 = fmaf(wr[q], v[rg + q], a3);
+          if (q % 4 == 3) a0 = fmaf(wr[q], v[rg + q], a0);
         }
       }
+      part[g][t] = (a0 + a1) + (a2 + a3);
     }
-    const float w = (a0 + a1) + (a2 + a3);
-    // v^T w and ||w||^2 in one reduction (the buffer alternates between steps: a step's sums may be
-    // written before every thread has read the previous step's; v is rewritten after the barrier)
-    float vw = t < m ? w * v[t] : 0.f, nn = t < m ? w * w : 0.f;
-    block_sum2_256(vw, nn, red[it & 1]);
+    __syncthreads();
+    // w = W v (the group partials in order), v^T w and ||w||^2 over the first group's warps
+    float w = 0.f;
+    if (g == 0) {
+      float vw = 0.f, nn = 0.f;
+      if (t < m) {
+        w = (part[0][t] + part[1][t]) + (part[2][t] + part[3][t]);
+        vw = w * v[t];
+        nn = w * w;
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        vw += __shfl_xor_sync(0xffffffffu, vw, o);
+        nn += __shfl_xor_sync(0xffffffffu, nn, o);
+      }
+      if ((t & 31) == 0) {
+        red[t >> 5] = vw;
+        red[kAlphaCols / 32 + (t >> 5)] = nn;
+      }
+    }
+    __syncthreads();
+    float vw = 0.f, nn = 0.f;
+#pragma unroll
+    for (int i = 0; i < kAlphaCols / 32; ++i) {
+      vw += red[i];
+      nn += red[kAlphaCols / 32 + i];
+    }
     rq = vw;
     if (it == iters) break;
-    if (t < m) v[t] = w * rsqrtf(nn);
+    if (g == 0 && t < m) v[t] = w * rsqrtf(nn);
     __syncthreads();
   }
   const float lmax = rq;
   const float alpha_p = 2.f / lmax;
   const int fallback = (alpha_p * lmax * lmax < 2.f) ? 0 : 1;
   const float alpha = fallback ? 1.f / (lmax * lmax) : alpha_p;
-  // X_0 = alpha W^T, the transposed read from the staged rows where they are
+  // X_0 = alpha W^T = alpha W (W symmetric), from the staged rows where they are
   float* Xg = p.X + (size_t)u * m * m;
-  for (int e = t; e < m * m; e += blockDim.x) {
-    const int a = e / m, b = e % m;
-    Xg[e] = alpha * (b < rs ? Ws[(size_t)b * m + a] : Wg[(size_t)b * m + a]);
-  }
-  if (t == 0) {
+  const int ns = rs * m;
+  for (int e = threadIdx.x; e < m * m; e += blockDim.x) Xg[e] = alpha * (e < ns ? Ws[e] : Wg[e]);
+  if (threadIdx.x == 0) {
     float* inf = p.info + (size_t)u * kInfoStride;
     inf[kInfoAlpha] = alpha;
     inf[kInfoLambdaMax] = lmax;
