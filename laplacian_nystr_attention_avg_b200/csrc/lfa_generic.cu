@@ -1033,12 +1033,11 @@ void reading_b_t(const Params& p, cudaStream_t st) {
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
 
-// alpha (power iteration and the fallback rule), the T Newton-Schulz steps X <- X (2I - W X) as
-// tcgen05 products, and the closing residual ||I - W X_T||_F, from W in p.Wm (p.Y and p.Xb are scratch).
-void ns_from_w(const Params& p, cudaStream_t st) {
+// alpha (power iteration and the fallback rule) and the T Newton-Schulz steps X <- X (2I - W X) as
+// tcgen05 products, from W in p.Wm (p.Y and p.Xb are scratch); X_T ends in p.X.
+void ns_steps_from_w(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m;
   k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
-  const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
   float* x = p.X;
   float* xb = p.Xb;
   const size_t mm = (size_t)m * m;
@@ -1053,24 +1052,38 @@ void ns_from_w(const Params& p, cudaStream_t st) {
     float* tmp = x; x = xb; xb = tmp;
   }
   if (x != p.X) cudaMemcpyAsync(p.X, x, sizeof(float) * (size_t)U * m * m, cudaMemcpyDeviceToDevice, st);
+}
+
+// the closing residual ||I - W X_T||_F of each unit into its info record (p.Y is scratch)
+void ns_residual(const Params& p, cudaStream_t st) {
+  const int U = p.U, m = p.m;
+  const dim3 g(ceil_div(m, 64), ceil_div(m, 64), U);
   k_ns_gemm<<<g, kThreads, 0, st>>>(p, p.Wm, p.X, p.Y, -1.f, 1.f, 1);  // I - W X, ||.||_F^2
   k_residual_sqrt<<<ceil_div(U, 128), 128, 0, st>>>(p);
 }
 
-// W, alpha and the Newton-Schulz chain from the landmarks in the workspace.
-void ns_t(const Params& p, cudaStream_t st) {
+void ns_from_w(const Params& p, cudaStream_t st) {
+  ns_steps_from_w(p, st);
+  ns_residual(p, st);
+}
+
+// W, alpha and the Newton-Schulz chain from the landmarks in the workspace (X_T in p.X); the closing
+// residual too unless with_residual is false (m > 64 only: the m <= 64 kernel always forms it).
+void ns_t(const Params& p, cudaStream_t st, bool with_residual = true) {
   const int U = p.U, m = p.m;
   if (m <= kSmallM) {
     launch_ns_tc(p, st);
   } else {
     k_gram<<<dim3(ceil_div(m, 16), U), kThreads, sizeof(float) * (size_t)m * (p.d + 1), st>>>(p);
-    ns_from_w(p, st);
+    if (with_residual) ns_from_w(p, st);
+    else ns_steps_from_w(p, st);
   }
 }
 
 // Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b. The
 // Newton-Schulz chain (W, alpha, X) and pass 1 (the column sums, C^T V) share no data: with an
-// auxiliary stream they run concurrently, joined before the combine.
+// auxiliary stream they run concurrently, joined before the combine. The closing residual of the
+// chain (m > 64) only reports: it runs on the auxiliary stream beside the combine, joined after it.
 template <typename T>
 void context_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
@@ -1080,13 +1093,29 @@ void context_t(const Params& p, cudaStream_t st) {
     reading_b_t<T>(p, st);
     return;
   }
-  fork_join(p, st,
-            [&](cudaStream_t s) {
-              pass1_reduce_t<T>(p, s);
-              if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, s>>>(p);
-            },
-            [&](cudaStream_t s) { ns_t(p, s); });
-  k_combine_finish<<<dim3(p.n_chunks, U), kThreads, combine_smem(m, d), st>>>(p);
+  auto pass1 = [&](cudaStream_t s) {
+    pass1_reduce_t<T>(p, s);
+    if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, s>>>(p);
+  };
+  auto combine = [&](cudaStream_t s) {
+    k_combine_finish<<<dim3(p.n_chunks, U), kThreads, combine_smem(m, d), s>>>(p);
+  };
+  if (m > kSmallM && p.aux_stream && p.ev_fork && p.ev_mid && p.ev_join) {
+    cudaStream_t aux = static_cast<cudaStream_t>(p.aux_stream);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), st);
+    cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_fork), 0);
+    ns_t(p, aux, false);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_mid), aux);
+    ns_residual(p, aux);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_join), aux);
+    pass1(st);
+    cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_mid), 0);
+    combine(st);
+    cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_join), 0);
+    return;
+  }
+  fork_join(p, st, pass1, [&](cudaStream_t s) { ns_t(p, s); });
+  combine(st);
 }
 
 template <typename T>

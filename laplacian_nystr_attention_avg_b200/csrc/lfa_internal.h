@@ -76,9 +76,11 @@ struct Params {
   void* ev_begin;
   void* ev_end;
   // optional second stream and fork / join events (cudaStream_t, cudaEvent_t, or null): the
-  // per-stage kernels run the Newton-Schulz chain there, concurrently with pass 1 (they share no data)
+  // per-stage kernels run the Newton-Schulz chain there, concurrently with pass 1 (they share no data);
+  // ev_mid marks X_T ready, so that the closing residual runs beside the combine
   void* aux_stream;
   void* ev_fork;
+  void* ev_mid;
   void* ev_join;
   // optional per-CTA phase timestamps (%globaltimer, ns) of the fused kernel: [grid][16]
   unsigned long long* trace;
