@@ -259,21 +259,24 @@ size_t lfa_workspace_size(const lfa_config* cfg) {
 void free_aux(lfa_ctx* h) {
   if (h->p.ev_fork) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_fork));
   if (h->p.ev_mid) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_mid));
+  if (h->p.ev_x) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_x));
   if (h->p.ev_join) cudaEventDestroy(static_cast<cudaEvent_t>(h->p.ev_join));
   if (h->p.aux_stream) cudaStreamDestroy(static_cast<cudaStream_t>(h->p.aux_stream));
-  h->p.ev_fork = h->p.ev_mid = h->p.ev_join = h->p.aux_stream = nullptr;
+  h->p.ev_fork = h->p.ev_mid = h->p.ev_x = h->p.ev_join = h->p.aux_stream = nullptr;
 }
 bool make_aux(lfa_ctx* h) {
   cudaStream_t s = nullptr;
-  cudaEvent_t a = nullptr, b = nullptr, c = nullptr;
+  cudaEvent_t a = nullptr, b = nullptr, c = nullptr, x = nullptr;
   const bool ok = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess &&
                   cudaEventCreateWithFlags(&a, cudaEventDisableTiming) == cudaSuccess &&
                   cudaEventCreateWithFlags(&b, cudaEventDisableTiming) == cudaSuccess &&
-                  cudaEventCreateWithFlags(&c, cudaEventDisableTiming) == cudaSuccess;
+                  cudaEventCreateWithFlags(&c, cudaEventDisableTiming) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&x, cudaEventDisableTiming) == cudaSuccess;
   h->p.aux_stream = s;
   h->p.ev_fork = a;
   h->p.ev_join = b;
   h->p.ev_mid = c;
+  h->p.ev_x = x;
   if (!ok) {
     free_aux(h);
     cudaGetLastError();

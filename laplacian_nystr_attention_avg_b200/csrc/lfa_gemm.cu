@@ -573,6 +573,8 @@ void chain_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int G, int
 
 }  // namespace
 
+int ns_chain_blocks(int m) { return chain_blocks(m); }
+
 // A cluster of the unit's G tiles (G <= 8, the portable cluster size: m <= 256) must fit on the device
 // (one block per SM at this shared-memory size). Cached per (device, m).
 bool ns_chain_fits(int m) {

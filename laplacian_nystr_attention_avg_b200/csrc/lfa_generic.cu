@@ -13,6 +13,8 @@
 //   k_pass2         O = C M' + 1 b^T + DWC(V)                                  (§关键设计 1)
 #include <math.h>
 
+#include <algorithm>
+
 #include "lfa_internal.h"
 
 namespace lfa {
@@ -1033,11 +1035,15 @@ void reading_b_t(const Params& p, cudaStream_t st) {
   k_rb_finish<<<dim3(p.n_chunks, U), kThreads, sizeof(float) * (size_t)m * d, st>>>(p);
 }
 
-// alpha (power iteration and the fallback rule) and the T Newton-Schulz steps X <- X (2I - W X) as
-// tcgen05 products, from W in p.Wm (p.Y and p.Xb are scratch); X_T ends in p.X.
-void ns_steps_from_w(const Params& p, cudaStream_t st) {
+// alpha (power iteration and the fallback rule) and X_0 = alpha W^T in p.X, from W in p.Wm
+void ns_alpha(const Params& p, cudaStream_t st) {
+  k_alpha<<<p.U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(p.m) * p.m, st>>>(p);
+}
+
+// the T Newton-Schulz steps X <- X (2I - W X) from X_0 in p.X as tcgen05 products (p.Y and p.Xb are
+// scratch); X_T ends in p.X.
+void ns_steps(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m;
-  k_alpha<<<U, kAlphaThreads, sizeof(float) * (size_t)alpha_rows(m) * m, st>>>(p);
   float* x = p.X;
   float* xb = p.Xb;
   const size_t mm = (size_t)m * m;
@@ -1063,7 +1069,8 @@ void ns_residual(const Params& p, cudaStream_t st) {
 }
 
 void ns_from_w(const Params& p, cudaStream_t st) {
-  ns_steps_from_w(p, st);
+  ns_alpha(p, st);
+  ns_steps(p, st);
   ns_residual(p, st);
 }
 
@@ -1075,9 +1082,33 @@ void ns_t(const Params& p, cudaStream_t st, bool with_residual = true) {
     launch_ns_tc(p, st);
   } else {
     k_gram<<<dim3(ceil_div(m, 16), U), kThreads, sizeof(float) * (size_t)m * (p.d + 1), st>>>(p);
-    if (with_residual) ns_from_w(p, st);
-    else ns_steps_from_w(p, st);
+    if (with_residual) {
+      ns_from_w(p, st);
+    } else {
+      ns_alpha(p, st);
+      ns_steps(p, st);
+    }
   }
+}
+
+// Pass-1 blocks per unit for the chain-first schedule of context_t, or 0 for the concurrent one. Pass 1
+// (one block per SM) dispatched first leaves no whole group of SMs for the chain's clusters, so the two
+// run one after the other. Chain first: W and alpha before the fork, then the chain's U clusters of G
+// blocks, and pass 1 on the SMs they leave. That pays when pass 1 on those SMs ends before the chain.
+// Estimates: 2T chain products of about 9.5 us; pass 1's 2 U N m d FP32 instructions at 45 % of the
+// issue rate of its SMs (128 lanes at 1.9 GHz).
+int chain_first_pass1(const Params& p) {
+  if (p.m <= kSmallM || p.T <= 0 || !stream_eligible(p) || !ns_chain_fits(p.m)) return 0;
+  if (!(p.aux_stream && p.ev_fork && p.ev_mid && p.ev_x && p.ev_join)) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const int pc = std::min((sms - p.U * ns_chain_blocks(p.m)) / p.U, p.P);
+  if (pc < 1) return 0;
+  const double t_chain = 2.0 * p.T * 9.5e-6;
+  const double t_pass1 = 2.0 * p.U * (double)p.N * p.m * p.d / ((double)pc * p.U * 128 * 1.9e9 * 0.45);
+  return t_pass1 < t_chain ? pc : 0;
 }
 
 // Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b. The
@@ -1100,6 +1131,30 @@ void context_t(const Params& p, cudaStream_t st) {
   auto combine = [&](cudaStream_t s) {
     k_combine_finish<<<dim3(p.n_chunks, U), kThreads, combine_smem(m, d), s>>>(p);
   };
+  const int pc = chain_first_pass1(p);
+  if (pc > 0) {
+    // main: W, alpha, the chain, then (after pass 1) the combine; auxiliary: pass 1 on pc blocks per
+    // unit once alpha is done, then the residual once X_T is
+    cudaStream_t aux = static_cast<cudaStream_t>(p.aux_stream);
+    Params q = p;
+    q.P = pc;
+    k_gram<<<dim3(ceil_div(m, 16), U), kThreads, sizeof(float) * (size_t)m * (p.d + 1), st>>>(p);
+    ns_alpha(p, st);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), st);
+    ns_steps(p, st);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_x), st);
+    cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_fork), 0);
+    pass1_reduce_t<T>(q, aux);
+    if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, aux>>>(p);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_mid), aux);
+    cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_x), 0);
+    ns_residual(p, aux);
+    cudaEventRecord(static_cast<cudaEvent_t>(p.ev_join), aux);
+    cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_mid), 0);
+    combine(st);
+    cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_join), 0);
+    return;
+  }
   if (m > kSmallM && p.aux_stream && p.ev_fork && p.ev_mid && p.ev_join) {
     cudaStream_t aux = static_cast<cudaStream_t>(p.aux_stream);
     cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), st);

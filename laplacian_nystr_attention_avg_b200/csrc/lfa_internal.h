@@ -77,10 +77,11 @@ struct Params {
   void* ev_end;
   // optional second stream and fork / join events (cudaStream_t, cudaEvent_t, or null): the
   // per-stage kernels run the Newton-Schulz chain there, concurrently with pass 1 (they share no data);
-  // ev_mid marks X_T ready, so that the closing residual runs beside the combine
+  // ev_mid and ev_x mark pass 1 done and X_T ready, so that the closing residual runs beside the combine
   void* aux_stream;
   void* ev_fork;
   void* ev_mid;
+  void* ev_x;
   void* ev_join;
   // optional per-CTA phase timestamps (%globaltimer, ns) of the fused kernel: [grid][16]
   unsigned long long* trace;
@@ -170,6 +171,8 @@ cudaError_t launch_mm(const MmJob* jobs, int njobs, int m, int U, cudaStream_t s
 bool launch_ns_chain(const NsChain& c, int U, cudaStream_t st);
 // whether launch_ns_chain runs for this m on the current device
 bool ns_chain_fits(int m);
+// blocks (one per SM) of one unit's cluster in launch_ns_chain
+int ns_chain_blocks(int m);
 cudaError_t gemm_set_attributes();
 cudaError_t ns_tc_set_attributes();
 cudaError_t launch_ns_tc(const Params& p, cudaStream_t st);
