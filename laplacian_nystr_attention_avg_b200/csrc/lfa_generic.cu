@@ -1091,24 +1091,42 @@ void ns_t(const Params& p, cudaStream_t st, bool with_residual = true) {
   }
 }
 
-// Pass-1 blocks per unit for the chain-first schedule of context_t, or 0 for the concurrent one. Pass 1
-// (one block per SM) dispatched first leaves no whole group of SMs for the chain's clusters, so the two
-// run one after the other. Chain first: W and alpha before the fork, then the chain's U clusters of G
-// blocks, and pass 1 on the SMs they leave. That pays when pass 1 on those SMs ends before the chain.
-// Estimates: 2T chain products of about 9.5 us; pass 1's 2 U N m d FP32 instructions at 45 % of the
-// issue rate of its SMs (128 lanes at 1.9 GHz).
-int chain_first_pass1(const Params& p) {
-  if (p.m <= kSmallM || p.T <= 0 || !stream_eligible(p) || !ns_chain_fits(p.m)) return 0;
-  if (!(p.aux_stream && p.ev_fork && p.ev_mid && p.ev_x && p.ev_join)) return 0;
+// The chain-first schedule of context_t. Pass 1 (one block per SM) dispatched first leaves no whole
+// group of SMs for the chain's clusters, so the two would run one after the other. Chain first: W and
+// alpha before the fork, then the chain's U clusters of G blocks, and pass 1 beside it on the pa blocks
+// per unit that the clusters leave, over the first ta tiles of each unit: as many as those blocks finish
+// in about the chain's time. The other tiles, if any, run after the chain on pb blocks per unit (every
+// SM). pa = 0: the concurrent order instead. Estimates: 2T chain products of about 9.5 us; a 64-token
+// tile about 16 us per block at 256 landmark columns and d = 64, in proportion to both. Worth it when
+// the chain takes longer than W and alpha (about 0.1 ms at m = 256) by a margin.
+struct ChainFirst {
+  int pa, ta, pb;
+};
+
+ChainFirst chain_first_plan(const Params& p, bool check_maps = true) {
+  ChainFirst cf{0, 0, 0};
+  if (p.m <= kSmallM || p.T <= 0 || !stream_eligible(p) || !ns_chain_fits(p.m)) return cf;
+  if (check_maps && !stream_maps_ok(p)) return cf;
+  if (!(p.aux_stream && p.ev_fork && p.ev_mid && p.ev_x && p.ev_join)) return cf;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 0;
-  const int pc = std::min((sms - p.U * ns_chain_blocks(p.m)) / p.U, p.P);
-  if (pc < 1) return 0;
+    return cf;
+  const int pa = std::min((sms - p.U * ns_chain_blocks(p.m)) / p.U, p.P);
   const double t_chain = 2.0 * p.T * 9.5e-6;
-  const double t_pass1 = 2.0 * p.U * (double)p.N * p.m * p.d / ((double)pc * p.U * 128 * 1.9e9 * 0.45);
-  return t_pass1 < t_chain ? pc : 0;
+  if (pa < 1 || t_chain < 150e-6) return cf;
+  const double t_tile = 16e-6 * (double)((p.m + 63) / 64) / 4.0 * ((double)p.d / 64.0);
+  const int n = stream_tiles(p);
+  const int ta = std::min(n, pa * std::max(1, (int)(t_chain / t_tile)));
+  int pb = 0;
+  if (ta < n) {
+    pb = std::min(std::max(sms / p.U, 1), p.P - stream_range_blocks(0, ta, pa));
+    if (pb < 1) return cf;
+  }
+  cf.pa = pa;
+  cf.ta = ta;
+  cf.pb = pb;
+  return cf;
 }
 
 // Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b. The
@@ -1131,26 +1149,35 @@ void context_t(const Params& p, cudaStream_t st) {
   auto combine = [&](cudaStream_t s) {
     k_combine_finish<<<dim3(p.n_chunks, U), kThreads, combine_smem(m, d), s>>>(p);
   };
-  const int pc = chain_first_pass1(p);
-  if (pc > 0) {
-    // main: W, alpha, the chain, then (after pass 1) the combine; auxiliary: pass 1 on pc blocks per
-    // unit once alpha is done, then the residual once X_T is
+  const ChainFirst cf = chain_first_plan(p);
+  if (cf.pa > 0) {
+    // main: W, alpha, the chain, the tiles after ta (if any) on every SM, then the combine; auxiliary:
+    // pass 1 over the first ta tiles on pa blocks per unit once alpha is done, then the residual once X_T
+    // (and the main stream's pass-1 tiles) are. The records are reduced after the last pass-1 launch.
     cudaStream_t aux = static_cast<cudaStream_t>(p.aux_stream);
+    const int n = stream_tiles(p);
+    const int ra = stream_range_blocks(0, cf.ta, cf.pa), rb = stream_range_blocks(cf.ta, n, cf.pb);
     Params q = p;
-    q.P = pc;
+    q.P = ra + rb;   // the records of both launches, per unit
+    auto reduce = [&](cudaStream_t s) {
+      k_combine_reduce<<<dim3(ceil_div(q.part_stride, kThreads), q.U), kThreads, 0, s>>>(q);
+      if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, s>>>(p);
+    };
     k_gram<<<dim3(ceil_div(m, 16), U), kThreads, sizeof(float) * (size_t)m * (p.d + 1), st>>>(p);
     ns_alpha(p, st);
     cudaEventRecord(static_cast<cudaEvent_t>(p.ev_fork), st);
     ns_steps(p, st);
+    if (rb > 0) stream_pass1_range(p, cf.ta, n, cf.pb, ra, q.P, st);
     cudaEventRecord(static_cast<cudaEvent_t>(p.ev_x), st);
     cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_fork), 0);
-    pass1_reduce_t<T>(q, aux);
-    if (p.whiten == 2) k_pool_batch_stats<<<dim3(ceil_div(2 * m, kThreads), p.heads), kThreads, 0, aux>>>(p);
+    stream_pass1_range(p, 0, cf.ta, cf.pa, 0, q.P, aux);
+    if (rb == 0) reduce(aux);
     cudaEventRecord(static_cast<cudaEvent_t>(p.ev_mid), aux);
     cudaStreamWaitEvent(aux, static_cast<cudaEvent_t>(p.ev_x), 0);
     ns_residual(p, aux);
     cudaEventRecord(static_cast<cudaEvent_t>(p.ev_join), aux);
     cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_mid), 0);
+    if (rb > 0) reduce(st);
     combine(st);
     cudaStreamWaitEvent(st, static_cast<cudaEvent_t>(p.ev_join), 0);
     return;
@@ -1225,13 +1252,14 @@ cudaError_t generic_set_attributes() {
 }
 
 int generic_launch_count(const Params& p) {
-  // pool, Newton-Schulz chain, pass 1, two combine kernels (three with batch-pooled statistics),
-  // pass 2; the chain for m > 64 is gram, alpha, the steps (one cluster launch, or two per step),
-  // the residual product and its square root
+  // pool, Newton-Schulz chain, pass 1 (two launches when the chain-first schedule splits it), two
+  // combine kernels (three with batch-pooled statistics), pass 2; the chain for m > 64 is gram, alpha,
+  // the steps (one cluster launch, or two per step), the residual product and its square root
   const int ns = p.m <= kSmallM ? 1 : 2 + (p.T > 0 ? (ns_chain_fits(p.m) ? 1 : 2 * p.T) : 0) + 2;
   // Reading B: pass 1, C^T C, reduction, covariance, two products, token pass, reduction, finish
   if (p.whiten == 3) return 1 + ns + 9 + 1;
-  return 1 + ns + 1 + 2 + (p.whiten == 2 ? 1 : 0) + 1;
+  const int split = chain_first_plan(p, false).pb > 0 ? 1 : 0;
+  return 1 + ns + 1 + split + 2 + (p.whiten == 2 ? 1 : 0) + 1;
 }
 
 cudaError_t launch_generic_forward(const Params& p, cudaStream_t st) {

@@ -223,6 +223,13 @@ int generic_launch_count(const Params& p);
 bool stream_eligible(const Params& p);
 cudaError_t stream_set_attributes();
 int stream_pass1(const Params& p, cudaStream_t st);
+// pass 1 split over launches: tiles (64 tokens) per unit; the CTAs per unit one launch over the tiles
+// [t_begin, t_end) takes with at most P; that launch, its records rec0 .. of rec_n per unit (rec_n <= p.P),
+// false when it does not apply
+int stream_tiles(const Params& p);
+bool stream_maps_ok(const Params& p);
+int stream_range_blocks(int t_begin, int t_end, int P);
+bool stream_pass1_range(const Params& p, int t_begin, int t_end, int P, int rec0, int rec_n, cudaStream_t st);
 bool stream_pass2(const Params& p, cudaStream_t st);
 size_t fused_workspace_bytes(int U);
 int fused_grid(const Params& p);

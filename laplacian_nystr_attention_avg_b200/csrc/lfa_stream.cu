@@ -57,7 +57,10 @@ static_assert(kNumBars * 8 <= 64, "mbarriers overlap the TMEM address slot");
 struct StreamArgs {
   int P;         // CTAs per unit
   int tpc;       // tiles per CTA
-  int n_tiles;   // tiles per unit
+  int n_tiles;   // end (exclusive) of this launch's tiles of a unit
+  int t0;        // pass 1: first tile of this launch (its CTA c takes tiles t0 + c tpc ..)
+  int rec0;      // pass 1: record of this launch's CTA 0 in the unit's records
+  int rec_n;     // pass 1: records per unit in p.part
 };
 
 __device__ __forceinline__ float bflo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -312,10 +315,10 @@ __global__ void __launch_bounds__(kST, 1) k_stream_pass1(const Params p, const S
   float* aux = reinterpret_cast<float*>(sm + kOffAux);
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
   const int u = blockIdx.y, pc = blockIdx.x, m = p.m;
-  const int tile0 = pc * sa.tpc;
+  const int tile0 = sa.t0 + pc * sa.tpc;
   const int tile1 = min(tile0 + sa.tpc, sa.n_tiles);
   const int ntl = tile1 - tile0;
-  float* out = p.part + ((size_t)u * sa.P + pc) * p.part_stride;
+  float* out = p.part + ((size_t)u * sa.rec_n + sa.rec0 + pc) * p.part_stride;
   if (ntl <= 0) {   // (the host's plan gives every CTA a tile)
     for (int e = t; e < p.part_stride; e += kST) out[e] = 0.f;
     return;
@@ -577,6 +580,24 @@ StreamArgs stream_plan(const Params& p) {
   if (P > sa.n_tiles) P = sa.n_tiles;
   sa.tpc = ceil_div(sa.n_tiles, P);
   sa.P = ceil_div(sa.n_tiles, sa.tpc);
+  sa.t0 = 0;
+  sa.rec0 = 0;
+  sa.rec_n = sa.P;
+  return sa;
+}
+
+// pass 1 over the tiles [t_begin, t_end) of every unit with at most P CTAs per unit
+StreamArgs stream_range_plan(int t_begin, int t_end, int P) {
+  StreamArgs sa;
+  const int nt = t_end - t_begin;
+  if (P > nt) P = nt;
+  if (P < 1) P = 1;
+  sa.tpc = ceil_div(nt, P);
+  sa.P = ceil_div(nt, sa.tpc);
+  sa.n_tiles = t_end;
+  sa.t0 = t_begin;
+  sa.rec0 = 0;
+  sa.rec_n = sa.P;
   return sa;
 }
 
@@ -600,6 +621,32 @@ int stream_pass1(const Params& p, cudaStream_t st) {
     return 0;
   k_stream_pass1<<<dim3(sa.P, p.U), kST, kStreamSmem, st>>>(p, sa, tq, tv);
   return sa.P;
+}
+
+int stream_tiles(const Params& p) { return ceil_div(p.N, kSTile); }
+
+bool stream_maps_ok(const Params& p) {
+  CUtensorMap tq, tv;
+  return stream_eligible(p) && make_tmap_rows_bf16(&tq, p.Q, (uint64_t)p.N, (uint64_t)p.U, kSTile) &&
+         make_tmap_rows_bf16(&tv, p.V, (uint64_t)p.N, (uint64_t)p.U, kSTile);
+}
+
+int stream_range_blocks(int t_begin, int t_end, int P) {
+  return t_end > t_begin ? stream_range_plan(t_begin, t_end, P).P : 0;
+}
+
+bool stream_pass1_range(const Params& p, int t_begin, int t_end, int P, int rec0, int rec_n, cudaStream_t st) {
+  if (!stream_eligible(p) || t_begin < 0 || t_end > stream_tiles(p) || t_end <= t_begin) return false;
+  StreamArgs sa = stream_range_plan(t_begin, t_end, P);
+  if (rec0 < 0 || rec0 + sa.P > rec_n || rec_n > p.P) return false;
+  sa.rec0 = rec0;
+  sa.rec_n = rec_n;
+  CUtensorMap tq, tv;
+  if (!make_tmap_rows_bf16(&tq, p.Q, (uint64_t)p.N, (uint64_t)p.U, kSTile) ||
+      !make_tmap_rows_bf16(&tv, p.V, (uint64_t)p.N, (uint64_t)p.U, kSTile))
+    return false;
+  k_stream_pass1<<<dim3(sa.P, p.U), kST, kStreamSmem, st>>>(p, sa, tq, tv);
+  return true;
 }
 
 bool stream_pass2(const Params& p, cudaStream_t st) {
