@@ -1131,8 +1131,9 @@ ChainFirst chain_first_plan(const Params& p, bool check_maps = true) {
 
 // Every forward stage before pass 2: L, W, alpha, X, the column statistics, A, M, M', b. The
 // Newton-Schulz chain (W, alpha, X) and pass 1 (the column sums, C^T V) share no data: with an
-// auxiliary stream they run concurrently, joined before the combine. The closing residual of the
-// chain (m > 64) only reports: it runs on the auxiliary stream beside the combine, joined after it.
+// auxiliary stream they run concurrently, joined before the combine, in the chain-first schedule
+// (chain_first_plan) where it applies. The closing residual of the chain (m > 64) only reports: it
+// runs on the auxiliary stream beside the combine, joined after it.
 template <typename T>
 void context_t(const Params& p, cudaStream_t st) {
   const int U = p.U, m = p.m, d = p.d;
