@@ -84,7 +84,7 @@ def workload_config(wl, extra=None):
                        f"Q~{wl.qdist}",
            "B": wl.B, "heads": wl.heads, "H": wl.H, "W": wl.W, "N": wl.N, "d": wl.d, "r": wl.r,
            "m": wl.m, "lambda": wl.lam, "eps": wl.eps, "T": wl.T, "storage": wl.dtype,
-           "whiten": True}
+           "whiten": "unit"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -249,7 +249,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": workload_config(wl, {"whiten": "unit", "sample": f"{per_step} of {wl.units} units per step"}),
+            "config": workload_config(wl, {"sample": f"{per_step} of {wl.units} units per step"}),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{per_step} (batch, head) unit of {wl.N} tokens per step, "
                                        f"{args.steps} steps"},
