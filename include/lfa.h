@@ -36,7 +36,11 @@
  *     keeps the weight and workspace pointers it was created with; the weight is read
  *     at every call, not copied.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Forward and
- *     backward only enqueue work: they never synchronise the host.
+ *     backward only enqueue work: they never synchronise the host. The per-stage
+ *     kernels also use the handle's own auxiliary stream (the landmark solver beside
+ *     pass 1): that work waits for what `stream` held at the call and `stream` waits
+ *     for it before the call's last kernels, so every call stays ordered on `stream`
+ *     (and captures into a CUDA graph begun on `stream`).
  *   - Errors are returned as lfa_status; nothing is thrown across the ABI and the
  *     library never exits the process. Argument errors are detected on the host
  *     before any launch. Device-side conditions (a bounded wait that expired, a
@@ -110,7 +114,9 @@ size_t lfa_workspace_size(const lfa_config* cfg);
 
 /* Validate cfg and build a handle. dwc_weight: device fp32 [heads][d][3][3].
  * workspace: device, >= lfa_workspace_size(cfg) bytes, 256-byte aligned, caller
- * owned for the handle's lifetime. No launch happens here. */
+ * owned for the handle's lifetime. No launch happens here; the handle creates its
+ * auxiliary stream and four events, which lfa_destroy releases (without them the
+ * per-stage kernels run one after the other on `stream`). */
 lfa_status lfa_create(const lfa_config* cfg, const float* dwc_weight, void* workspace,
                       size_t workspace_bytes, lfa_handle* out);
 
